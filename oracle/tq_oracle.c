@@ -1,0 +1,616 @@
+/*
+ * tq_oracle.c -- plain fp64 CPU oracle for imatrix-weighted group-scale search,
+ * round-to-nearest, low-bit packing and weighted reconstruction error.
+ *
+ * TEST INFRASTRUCTURE.  This file is the checker the CUDA library is compared
+ * against.  Only the test suite, the smoke check and the benchmark's CPU
+ * baseline leg may load it.  It shares no code, header, table or constant
+ * generator with the CUDA path: every table below is computed here from its
+ * definition.
+ *
+ * Sources (web pages; cited by title and section):
+ *  [NeUQI]  "NeUQI Accuracy Validation" (intel/auto-round docs/neuqi_acc.md),
+ *           opening paragraph: asymmetric layers run a joint (scale, integer
+ *           zero-point) search, symmetric layers a two-stage signed-scale search,
+ *           both weighted by the activation imatrix; results bullet 2: the
+ *           "64/32" grid.
+ *  [TT]     "Quantize on TT cards: CUDA-free GPTQ/LDLQ bfp4 pipeline" (tt-stack
+ *           issue #67), pipeline table step 1 (H = sum X^T X) and "Risks to
+ *           measure: Precision" (proxy error tr(E H E^T)/tr(W H W^T)).
+ *  [NVFP4]  "Nemotron-Cascade-2-30B-A3B-NVFP4" model card, Quantization Recipe
+ *           table (NVFP4 group 16, MSE-calibrated static block scales) and the
+ *           Calibration line (weight-MSE calibration).
+ *  [INT3]   "int3-g64 (fmt=5)" (colibri PR #168), Design: Layout bullet
+ *           (24 bytes per 64 weights: 16 B low plane of 2-bit values, 8 B high
+ *           plane of 1-bit values, v in [-4,3] stored as v+4, one f32 scale per
+ *           group) and Tests (outlier-row RMS vs per-row int4).
+ *
+ * Readings where the pages are silent are listed beside each function.  All
+ * code decisions (round-to-nearest of w/s) are taken on the IEEE fp32
+ * quotient, the precision the weights and scales are stored in; losses and
+ * sums are accumulated in fp64 in natural element order.
+ *
+ * Build: gcc -O2 -fPIC -shared -fopenmp -ffp-contract=off (no fast-math).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_API __attribute__((visibility("default")))
+
+/* ------------------------------------------------------------------ */
+/* imatrix                                                             */
+/* ------------------------------------------------------------------ */
+
+/* m_j = (1/T) * sum_t x_{t,j}^2 for one [T, I] activation matrix with row
+ * stride ld.  [NeUQI] opening paragraph ("weighted by the activation
+ * imatrix"); [TT] step 1: H = sum_t x_t^T x_t, whose diagonal is T * m. */
+ORC_API void orc_imatrix(const float* X, int64_t T, int64_t I, int64_t ld, double* m)
+{
+    #pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < I; ++j) {
+        double s = 0.0;
+        for (int64_t t = 0; t < T; ++t) {
+            double x = (double)X[t * ld + j];
+            s += x * x;
+        }
+        m[j] = T > 0 ? s / (double)T : 0.0;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Round-to-nearest helpers                                            */
+/* ------------------------------------------------------------------ */
+
+/* Integer code of w under scale s: round half to even of the fp32 quotient
+ * w/s, clamped to [lo, hi].  A zero scale gives code 0 (the group or block
+ * holds no magnitude to represent). */
+static double rtn_code(float w, float s, double lo, double hi)
+{
+    if (s == 0.0f) return 0.0;
+    float y = w / s;                 /* IEEE single division */
+    double q = nearbyint((double)y); /* current rounding mode: to nearest, ties to even */
+    if (q < lo) q = lo;
+    if (q > hi) q = hi;
+    return q;
+}
+
+/* ------------------------------------------------------------------ */
+/* Symmetric int3-g64 two-stage signed-scale search                    */
+/* ------------------------------------------------------------------ */
+
+/* Stage-1 magnitude ratios r_k = fl32(lo + ((hi - lo) * k) / (n1 - 1)),
+ * k = 0..n1-1, i.e. n1 points of linspace(lo, hi) rounded once to fp32.
+ * Scale of candidate c = 2k + sigma: s = (1 - 2 sigma) * fl32(r_k * M) * 0.25,
+ * with M = max|w| over the group and 0.25 = 1/4 (the int3 grid's positive
+ * reach).  [NeUQI] opening paragraph: "two-stage signed scale search". */
+ORC_API float orc_sym_stage1_ratio(int n1, double lo, double hi, int k)
+{
+    return (float)(lo + ((hi - lo) * (double)k) / (double)(n1 - 1));
+}
+
+/* Stage-2 ratio i around stage-1 magnitude k*: n2 points of linspace over
+ * [r_{k*} - delta, r_{k*} + delta] in fp64, rounded once to fp32, where
+ * delta = (hi - lo)/(n1 - 1) is the stage-1 spacing (reading: "refinements
+ * around the best" span the neighbouring stage-1 points). */
+ORC_API float orc_sym_stage2_ratio(int n1, int n2, double lo, double hi, int kstar, int i)
+{
+    double delta = (hi - lo) / (double)(n1 - 1);
+    double center = lo + ((hi - lo) * (double)kstar) / (double)(n1 - 1);
+    return (float)((center - delta) + (2.0 * delta * (double)i) / (double)(n2 - 1));
+}
+
+static float sym_scale(float r, float M, int negative)
+{
+    float a = (float)((double)r * (double)M); /* exact product, rounded once */
+    a = a * 0.25f;
+    return negative ? -a : a;
+}
+
+/* Weighted squared error of one group under scale s, codes v in [-4, 3]:
+ * L = sum_j m_j (w_j - s v_j)^2 in fp64. */
+ORC_API double orc_sym_loss(const float* w, const float* m, int n, float s, int8_t* v_out)
+{
+    double L = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double v = rtn_code(w[j], s, -4.0, 3.0);
+        double e = (double)w[j] - (double)s * v;
+        L += (double)m[j] * (e * e);
+        if (v_out) v_out[j] = (int8_t)v;
+    }
+    return L;
+}
+
+/* One group of n <= 64 weights.  Returns the candidate index: 2k+sigma for a
+ * stage-1 winner, 2*n1 + i for a stage-2 winner, -1 for an all-zero group.
+ * Ties keep the lower index (a candidate replaces the incumbent only when its
+ * loss is strictly smaller).  Stage 2 keeps the stage-1 sign and replaces the
+ * stage-1 winner only on a strict improvement. */
+ORC_API int orc_search_sym_group(const float* w, const float* m, int n, int n1, int n2,
+                                 double lo, double hi, float* scale_out, double* loss_out,
+                                 int8_t* codes_out)
+{
+    float M = 0.0f;
+    for (int j = 0; j < n; ++j) { float a = fabsf(w[j]); if (a > M) M = a; }
+    if (M == 0.0f) {
+        *scale_out = 0.0f; *loss_out = 0.0;
+        if (codes_out) memset(codes_out, 0, (size_t)n);
+        return -1;
+    }
+    int best = -1; double bestL = INFINITY; float bestS = 0.0f;
+    for (int k = 0; k < n1; ++k) {
+        float r = orc_sym_stage1_ratio(n1, lo, hi, k);
+        for (int sg = 0; sg < 2; ++sg) {
+            float s = sym_scale(r, M, sg);
+            double L = orc_sym_loss(w, m, n, s, NULL);
+            if (L < bestL) { bestL = L; best = 2 * k + sg; bestS = s; }
+        }
+    }
+    int kstar = best / 2, sgstar = best % 2;
+    int best2 = best; double bestL2 = bestL; float bestS2 = bestS;
+    for (int i = 0; i < n2; ++i) {
+        float r = orc_sym_stage2_ratio(n1, n2, lo, hi, kstar, i);
+        float s = sym_scale(r, M, sgstar);
+        double L = orc_sym_loss(w, m, n, s, NULL);
+        if (L < bestL2) { bestL2 = L; best2 = 2 * n1 + i; bestS2 = s; }
+    }
+    *scale_out = bestS2; *loss_out = bestL2;
+    if (codes_out) orc_sym_loss(w, m, n, bestS2, codes_out);
+    return best2;
+}
+
+/* ------------------------------------------------------------------ */
+/* Asymmetric int4-g128 joint (scale, integer zero-point) search       */
+/* ------------------------------------------------------------------ */
+
+/* Scale factor table c_k = fl32(f_k / 15), f_k = lo + ((hi - lo) * k)/(ns - 1):
+ * candidate scale s_k = fl32(c_k * R), R = fl32(wmax - wmin).  Reading: the
+ * pages give the "64/32" grid size but not its range; the range is taken
+ * equal to the symmetric stage-1 window [0.5, 1.2]. */
+ORC_API float orc_asym_scale_factor(int ns, double lo, double hi, int k)
+{
+    double f = lo + ((hi - lo) * (double)k) / (double)(ns - 1);
+    return (float)(f / 15.0);
+}
+
+/* Zero-point i of nz: z_i = rint(15 i / (nz - 1)) (ties to even).  Reading:
+ * "32 integer zero-points in [0,15]" names more points than integers in the
+ * range; the nz points are spread evenly over [0,15] and rounded, so every
+ * integer 0..15 occurs and duplicates never win under the strict-improvement
+ * rule. */
+ORC_API int orc_asym_zero(int nz, int i)
+{
+    return (int)nearbyint((15.0 * (double)i) / (double)(nz - 1));
+}
+
+ORC_API double orc_asym_loss(const float* w, const float* m, int n, float s, int z, uint8_t* q_out)
+{
+    double L = 0.0;
+    for (int j = 0; j < n; ++j) {
+        double q;
+        if (s == 0.0f) q = (double)z;
+        else {
+            float y = w[j] / s;
+            q = nearbyint((double)y) + (double)z;
+            if (q < 0.0) q = 0.0;
+            if (q > 15.0) q = 15.0;
+        }
+        double e = (double)w[j] - (double)s * (q - (double)z);
+        L += (double)m[j] * (e * e);
+        if (q_out) q_out[j] = (uint8_t)q;
+    }
+    return L;
+}
+
+/* One group of n <= 128 weights.  Candidate index ns_idx = nz * k + i.
+ * Degenerate groups: wmax == wmin == 0 gives s = 0, z = 0 and index -1;
+ * wmax == wmin != 0 uses R = |wmax|. */
+ORC_API int orc_search_asym_group(const float* w, const float* m, int n, int ns, int nz,
+                                  double lo, double hi, float* scale_out, uint8_t* zero_out,
+                                  double* loss_out, uint8_t* q_out)
+{
+    float wmin = w[0], wmax = w[0];
+    for (int j = 1; j < n; ++j) { if (w[j] < wmin) wmin = w[j]; if (w[j] > wmax) wmax = w[j]; }
+    float R = (float)((double)wmax - (double)wmin);
+    if (R == 0.0f) {
+        if (wmax == 0.0f) {
+            *scale_out = 0.0f; *zero_out = 0; *loss_out = 0.0;
+            if (q_out) memset(q_out, 0, (size_t)n);
+            return -1;
+        }
+        R = fabsf(wmax);
+    }
+    int best = -1; double bestL = INFINITY; float bestS = 0.0f; int bestZ = 0;
+    for (int k = 0; k < ns; ++k) {
+        float c = orc_asym_scale_factor(ns, lo, hi, k);
+        float s = (float)((double)c * (double)R);
+        for (int i = 0; i < nz; ++i) {
+            int z = orc_asym_zero(nz, i);
+            double L = orc_asym_loss(w, m, n, s, z, NULL);
+            if (L < bestL) { bestL = L; best = nz * k + i; bestS = s; bestZ = z; }
+        }
+    }
+    *scale_out = bestS; *zero_out = (uint8_t)bestZ; *loss_out = bestL;
+    if (q_out) orc_asym_loss(w, m, n, bestS, bestZ, q_out);
+    return best;
+}
+
+/* ------------------------------------------------------------------ */
+/* NVFP4-g16: E2M1 elements, E4M3 block scales, fp32 global scale      */
+/* ------------------------------------------------------------------ */
+
+/* E4M3 (e4m3fn) decode: s eeee mmm, bias 7; exponent 0 is subnormal
+ * (m * 2^-9); 0x7F / 0xFF are NaN; 0x7E = 448 is the largest finite value. */
+ORC_API double orc_e4m3_decode(int code)
+{
+    int s = (code >> 7) & 1, e = (code >> 3) & 15, mt = code & 7;
+    if (e == 15 && mt == 7) return NAN;
+    double v = (e == 0) ? ldexp((double)mt, -9) : ldexp(1.0 + (double)mt / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+static const double E2M1_MAG[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+/* Magnitude code (0..7) of y >= 0 under E2M1 round-to-nearest-even with
+ * saturation: the nearest of {0,.5,1,1.5,2,3,4,6}; a tie goes to the even
+ * code; values above 6 (and +inf) give 6; NaN gives 0. */
+ORC_API int orc_e2m1_rne_mag(float y)
+{
+    if (isnan(y)) return 0;
+    if (y > 6.0f) return 7;   /* saturate: also keeps huge y from tying 4 and 6 */
+    double best_d = INFINITY; int best = 0;
+    for (int i = 0; i < 8; ++i) {
+        double d = fabs((double)y - E2M1_MAG[i]);
+        if (d < best_d || (d == best_d && (i % 2) == 0)) { best_d = d; best = i; }
+    }
+    return best;
+}
+
+/* Per-tensor global scale g = fl32(amax / (6 * 448)). */
+ORC_API float orc_nvfp4_global(const float* W, int64_t n)
+{
+    float amax = 0.0f;
+    for (int64_t i = 0; i < n; ++i) { float a = fabsf(W[i]); if (a > amax) amax = a; }
+    return (float)((double)amax / 2688.0);
+}
+
+/* The `window` positive finite E4M3 codes (1..126) whose values lie nearest
+ * t, ties to the lower code, listed in ascending code order.  Done as the
+ * plain definition: rank all 126 codes by (|dec(c) - t|, c) and keep the
+ * first `window`.  Reading of "the 16 E4M3 codes nearest amax/6": t is the
+ * block amax over 6 in units of the global scale. */
+ORC_API void orc_nvfp4_window(double t, int window, int* codes_out)
+{
+    int chosen[127]; memset(chosen, 0, sizeof chosen);
+    for (int r = 0; r < window; ++r) {
+        int best = -1; double bd = INFINITY;
+        for (int c = 1; c <= 126; ++c) {
+            if (chosen[c]) continue;
+            double d = fabs(orc_e4m3_decode(c) - t);
+            if (d < bd) { bd = d; best = c; }   /* strict: ties keep the lower code */
+        }
+        chosen[best] = 1;
+    }
+    int k = 0;
+    for (int c = 1; c <= 126; ++c) if (chosen[c]) codes_out[k++] = c;
+}
+
+ORC_API double orc_nvfp4_loss(const float* w, const float* m, int n, float S, uint8_t* c_out)
+{
+    double L = 0.0;
+    for (int j = 0; j < n; ++j) {
+        int mag;
+        if (S == 0.0f) mag = 0;
+        else mag = orc_e2m1_rne_mag(fabsf(w[j]) / S);
+        double e = fabs((double)w[j]) - (double)S * E2M1_MAG[mag];
+        L += (double)m[j] * (e * e);
+        if (c_out) c_out[j] = (uint8_t)((mag != 0 && w[j] < 0.0f) ? (mag | 8) : mag);
+    }
+    return L;
+}
+
+/* One block of n <= 16 weights under global scale g.  Returns the chosen
+ * E4M3 scale code (1..126), or -1 (scale byte 0, codes 0) for an all-zero
+ * block or g == 0.  Candidates are the window codes in ascending order with
+ * block scale S = fl32(g * dec(e)); ties keep the lower code. */
+ORC_API int orc_search_nvfp4_block(const float* w, const float* m, int n, float g, int window,
+                                   double* loss_out, uint8_t* c_out)
+{
+    float a = 0.0f;
+    for (int j = 0; j < n; ++j) { float v = fabsf(w[j]); if (v > a) a = v; }
+    if (a == 0.0f || g == 0.0f) {
+        double L = 0.0;
+        for (int j = 0; j < n; ++j) L += (double)m[j] * ((double)w[j] * (double)w[j]);
+        *loss_out = L;
+        if (c_out) memset(c_out, 0, (size_t)n);
+        return -1;
+    }
+    double t = (double)a / (6.0 * (double)g);
+    int codes[126];
+    orc_nvfp4_window(t, window, codes);
+    int best = -1; double bestL = INFINITY;
+    for (int r = 0; r < window; ++r) {
+        float S = (float)((double)g * orc_e4m3_decode(codes[r]));
+        double L = orc_nvfp4_loss(w, m, n, S, NULL);
+        if (L < bestL) { bestL = L; best = codes[r]; }
+    }
+    *loss_out = bestL;
+    if (c_out) orc_nvfp4_loss(w, m, n, (float)((double)g * orc_e4m3_decode(best)), c_out);
+    return best;
+}
+
+/* ------------------------------------------------------------------ */
+/* Batched searches over [n_mat, O, I] (OpenMP over independent groups) */
+/* ------------------------------------------------------------------ */
+
+/* W: n_mat matrices, row stride ld, matrix stride ms.  m: imatrix of matrix e
+ * at m + e * m_stride (m_stride 0 = shared).  Outputs per group [n_mat, O, G]
+ * and codes [n_mat, O, I] (int8 v for int3; uint8 q for int4; uint8 E2M1 code
+ * for NVFP4).  Any output pointer may be NULL. */
+ORC_API void orc_search_sym_int3(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                                 int64_t ms, const float* m, int64_t m_stride, int n1, int n2,
+                                 double lo, double hi, float* scales, int32_t* idx, double* loss,
+                                 int8_t* codes)
+{
+    const int64_t G = (I + 63) / 64;
+    #pragma omp parallel for schedule(dynamic, 64)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 64; int n = (int)((I - j0) < 64 ? (I - j0) : 64);
+        const float* w = W + e * ms + o * ld + j0;
+        const float* mm = m + e * m_stride + j0;
+        float s; double L;
+        int c = orc_search_sym_group(w, mm, n, n1, n2, lo, hi, &s, &L,
+                                     codes ? codes + (e * O + o) * I + j0 : NULL);
+        if (scales) scales[gi] = s;
+        if (idx) idx[gi] = c;
+        if (loss) loss[gi] = L;
+    }
+}
+
+ORC_API void orc_search_asym_int4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                                  int64_t ms, const float* m, int64_t m_stride, int ns, int nz,
+                                  double lo, double hi, float* scales, uint8_t* zeros, int32_t* idx,
+                                  double* loss, uint8_t* codes)
+{
+    const int64_t G = (I + 127) / 128;
+    #pragma omp parallel for schedule(dynamic, 16)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 128; int n = (int)((I - j0) < 128 ? (I - j0) : 128);
+        const float* w = W + e * ms + o * ld + j0;
+        const float* mm = m + e * m_stride + j0;
+        float s; uint8_t z; double L;
+        int c = orc_search_asym_group(w, mm, n, ns, nz, lo, hi, &s, &z, &L,
+                                      codes ? codes + (e * O + o) * I + j0 : NULL);
+        if (scales) scales[gi] = s;
+        if (zeros) zeros[gi] = z;
+        if (idx) idx[gi] = c;
+        if (loss) loss[gi] = L;
+    }
+}
+
+/* gscale: per-matrix global scale g (computed by the caller with
+ * orc_nvfp4_global, or any given value).  scale_codes: E4M3 byte per block. */
+ORC_API void orc_search_nvfp4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                              int64_t ms, const float* m, int64_t m_stride, const float* gscale,
+                              int window, uint8_t* scale_codes, int32_t* idx, double* loss,
+                              uint8_t* codes)
+{
+    const int64_t G = (I + 15) / 16;
+    #pragma omp parallel for schedule(dynamic, 256)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 16; int n = (int)((I - j0) < 16 ? (I - j0) : 16);
+        const float* w = W + e * ms + o * ld + j0;
+        const float* mm = m + e * m_stride + j0;
+        double L;
+        int c = orc_search_nvfp4_block(w, mm, n, gscale[e], window, &L,
+                                       codes ? codes + (e * O + o) * I + j0 : NULL);
+        if (scale_codes) scale_codes[gi] = (uint8_t)(c < 0 ? 0 : c);
+        if (idx) idx[gi] = c;
+        if (loss) loss[gi] = L;
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Round-to-nearest with given scales (pack path)                      */
+/* ------------------------------------------------------------------ */
+
+/* rows = n_mat * O contiguous rows of I weights (row stride I). */
+ORC_API void orc_rtn_int3(const float* W, int64_t rows, int64_t I, const float* scales, int8_t* v)
+{
+    const int64_t G = (I + 63) / 64;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j)
+            v[r * I + j] = (int8_t)rtn_code(W[r * I + j], scales[r * G + j / 64], -4.0, 3.0);
+}
+
+ORC_API void orc_rtn_int4(const float* W, int64_t rows, int64_t I, const float* scales,
+                          const uint8_t* zeros, uint8_t* q)
+{
+    const int64_t G = (I + 127) / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            float s = scales[r * G + j / 128]; int z = zeros[r * G + j / 128];
+            double qq;
+            if (s == 0.0f) qq = (double)z;
+            else {
+                qq = nearbyint((double)(W[r * I + j] / s)) + (double)z;
+                if (qq < 0.0) qq = 0.0;
+                if (qq > 15.0) qq = 15.0;
+            }
+            q[r * I + j] = (uint8_t)qq;
+        }
+}
+
+/* rows of one matrix share g; mat_rows = O (rows per matrix). */
+ORC_API void orc_rtn_nvfp4(const float* W, int64_t rows, int64_t mat_rows, int64_t I,
+                           const uint8_t* scale_codes, const float* gscale, uint8_t* c)
+{
+    const int64_t G = (I + 15) / 16;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        float g = gscale[r / mat_rows];
+        for (int64_t j = 0; j < I; ++j) {
+            int sc = scale_codes[r * G + j / 16];
+            float S = (float)((double)g * orc_e4m3_decode(sc));
+            float w = W[r * I + j];
+            int mag = (S == 0.0f) ? 0 : orc_e2m1_rne_mag(fabsf(w) / S);
+            c[r * I + j] = (uint8_t)((mag != 0 && w < 0.0f) ? (mag | 8) : mag);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* Packing ([INT3] Design: Layout; nibble order for int4 / NVFP4)      */
+/* ------------------------------------------------------------------ */
+
+/* int3-g64: per group a 24-byte record.  u_i = v_i + 4.  Bytes 0..15: low
+ * plane, element i in byte i/4 at bits 2(i%4).  Bytes 16..23: high plane,
+ * element i at bit i%8 of byte 16 + i/8.  Records in [row][group] order; tail
+ * positions past I hold v = 0 (u = 4). */
+ORC_API void orc_pack_int3(const int8_t* v, int64_t rows, int64_t I, uint8_t* out)
+{
+    const int64_t G = (I + 63) / 64;
+    memset(out, 0, (size_t)(rows * G * 24));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < G; ++k) {
+            uint8_t* rec = out + (r * G + k) * 24;
+            for (int i = 0; i < 64; ++i) {
+                int64_t j = k * 64 + i;
+                int u = (j < I ? v[r * I + j] : 0) + 4;
+                rec[i / 4] |= (uint8_t)((u & 3) << (2 * (i % 4)));
+                rec[16 + i / 8] |= (uint8_t)(((u >> 2) & 1) << (i % 8));
+            }
+        }
+}
+
+ORC_API void orc_unpack_int3(const uint8_t* in, int64_t rows, int64_t I, int8_t* v)
+{
+    const int64_t G = (I + 63) / 64;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            const uint8_t* rec = in + (r * G + j / 64) * 24;
+            int i = (int)(j % 64);
+            int lo = (rec[i / 4] >> (2 * (i % 4))) & 3;
+            int hi = (rec[16 + i / 8] >> (i % 8)) & 1;
+            v[r * I + j] = (int8_t)((lo | (hi << 2)) - 4);
+        }
+}
+
+/* Nibble pack: group of `g` codes in g/2 bytes, element 2k in the low
+ * nibble of byte k, element 2k+1 in the high nibble.  Tail positions hold
+ * `pad` (per group: the zero-point for int4 so they dequantize to 0; 0 for
+ * NVFP4). */
+ORC_API void orc_pack_nibbles(const uint8_t* c, int64_t rows, int64_t I, int g,
+                              const uint8_t* pad_per_group, uint8_t* out)
+{
+    const int64_t G = (I + g - 1) / g;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < G; ++k) {
+            uint8_t pad = pad_per_group ? pad_per_group[r * G + k] : 0;
+            uint8_t* rec = out + (r * G + k) * (g / 2);
+            for (int i = 0; i < g / 2; ++i) {
+                int64_t j0 = k * g + 2 * i, j1 = j0 + 1;
+                int lo = (j0 < I ? c[r * I + j0] : pad) & 15;
+                int hi = (j1 < I ? c[r * I + j1] : pad) & 15;
+                rec[i] = (uint8_t)(lo | (hi << 4));
+            }
+        }
+}
+
+ORC_API void orc_unpack_nibbles(const uint8_t* in, int64_t rows, int64_t I, int g, uint8_t* c)
+{
+    const int64_t G = (I + g - 1) / g;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            uint8_t b = in[(r * G + j / g) * (g / 2) + (j % g) / 2];
+            c[r * I + j] = (uint8_t)((j % 2) ? (b >> 4) : (b & 15));
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Dequantization (fp32 semantics, rounded once)                       */
+/* ------------------------------------------------------------------ */
+
+ORC_API void orc_dequant_int3(const int8_t* v, int64_t rows, int64_t I, const float* scales, float* out)
+{
+    const int64_t G = (I + 63) / 64;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j)
+            out[r * I + j] = (float)((double)scales[r * G + j / 64] * (double)v[r * I + j]);
+}
+
+ORC_API void orc_dequant_int4(const uint8_t* q, int64_t rows, int64_t I, const float* scales,
+                              const uint8_t* zeros, float* out)
+{
+    const int64_t G = (I + 127) / 128;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            int64_t gi = r * G + j / 128;
+            out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));
+        }
+}
+
+ORC_API void orc_dequant_nvfp4(const uint8_t* c, int64_t rows, int64_t mat_rows, int64_t I,
+                               const uint8_t* scale_codes, const float* gscale, float* out)
+{
+    const int64_t G = (I + 15) / 16;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            float S = (float)((double)gscale[r / mat_rows] * orc_e4m3_decode(scale_codes[r * G + j / 16]));
+            int code = c[r * I + j];
+            double v = E2M1_MAG[code & 7] * ((code & 8) ? -1.0 : 1.0);
+            out[r * I + j] = (float)((double)S * v);
+        }
+}
+
+/* ------------------------------------------------------------------ */
+/* Weighted reconstruction error ([TT] Risks to measure: Precision)    */
+/* ------------------------------------------------------------------ */
+
+/* num = sum_{o,j} m_j (W - What)^2 = tr(E H E^T), den = sum m_j W^2 =
+ * tr(W H W^T) with H = diag(m), over one O x I matrix (row stride I). */
+ORC_API void orc_proxy_error(const float* W, const float* What, int64_t O, int64_t I,
+                             const float* m, double* num, double* den)
+{
+    double a = 0.0, b = 0.0;
+    for (int64_t o = 0; o < O; ++o)
+        for (int64_t j = 0; j < I; ++j) {
+            double w = (double)W[o * I + j];
+            double e = w - (double)What[o * I + j];
+            a += (double)m[j] * (e * e);
+            b += (double)m[j] * (w * w);
+        }
+    *num = a; *den = b;
+}
+
+/* Per-row int4 absmax baseline of [INT3] Tests (the shipped per-row format
+ * the outlier-row RMS test compares against): s = max|w_row| / 7,
+ * q = clamp(rint(w/s), -8, 7), What = fl32(s q). */
+ORC_API void orc_rowwise_int4(const float* W, int64_t rows, int64_t I, float* What)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        float M = 0.0f;
+        for (int64_t j = 0; j < I; ++j) { float a = fabsf(W[r * I + j]); if (a > M) M = a; }
+        float s = (float)((double)M / 7.0);
+        for (int64_t j = 0; j < I; ++j) {
+            double q = rtn_code(W[r * I + j], s, -8.0, 7.0);
+            What[r * I + j] = (float)((double)s * q);
+        }
+    }
+}
+
+ORC_API int orc_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
