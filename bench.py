@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Throughput benchmark: weights quantized per second through the whole hot
+path on B200 -- imatrix -> group-scale search with fused RTN + pack ->
+dequant -> imatrix-weighted proxy error -- one JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl tq|reference]
+
+A step is one pass of every row of the path over one batch of synthetic input
+(the workload named by --config; default: the dense int4-g128 4096 x 4096
+workload).  `value` is device-timed with inputs resident in HBM (CUDA events,
+barrier + synchronize on both sides, max over ranks); `e2e` repeats the step
+through the public API starting from pinned host buffers, with the host->device
+copies of the inputs and the device->host read of the results inside the
+timed region.  `roofline` reports the dominant kernel (the search) against the
+FP32 CUDA-core issue peak.  Under torchrun every rank quantizes its own
+independent copy of the workload (weak scaling; no collective on the data
+path).  --impl reference times the CPU oracle on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "weights quantized/sec (search+pack) on 1 B200; % of FP32 / HBM roofline"
+L2_BYTES = 126 * 2 ** 20
+# FP32 lane-instructions per weight of the search (the dominant kernel):
+# candidate-element evaluations per weight x instructions per evaluation
+# (sym int3: 96 x 7; asym int4: 1024 x 5; NVFP4: 16 x 10).
+SEARCH_INSTR_PER_W = {"int3_g64_sym": 96 * 7, "int4_g128_asym": 1024 * 5, "nvfp4_g16": 16 * 10}
+SEARCH_CEE_PER_W = {"int3_g64_sym": 96, "int4_g128_asym": 1024, "nvfp4_g16": 16}
+# our kernels per call: imatrix 2 (partial + final), search 1 (NVFP4: amax +
+# global + search = 3), dequant 1, proxy 1
+KERNELS = {"imatrix": 2, "search": {"int3_g64_sym": 1, "int4_g128_asym": 1, "nvfp4_g16": 3},
+           "dequant": 1, "proxy": 1}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def peaks():
+    p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+    f = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(f):
+        d = json.load(open(f))
+        p = {"hbm_gbs": d.get("hbm_gbs", 6650.0), "sm_max_mhz": d.get("sm_max_mhz", 1965.0),
+             "source": "measured"}
+    return p
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: torch.device):
+        self.rows = []
+        self.proc = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not self.uuid.startswith("GPU-"):
+                self.uuid = "GPU-" + self.uuid
+        except Exception:
+            self.uuid = None
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.uuid:
+            cmd[1:1] = ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append([x.strip() for x in line.split(",")])
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm = [float(r[0]) for r in self.rows if len(r) >= 7 and r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if len(r) >= 7 and r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows if len(r) >= 7 for i in range(4)
+                          if r[3 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ the step
+
+class Step:
+    """One pass of the whole path over one input set, on the current stream."""
+
+    def __init__(self, tq, wl, sets):
+        self.tq = tq
+        self.wl = wl
+        self.sets = sets            # list of (sites dict name->X, units list of W)
+        self.fmts = [tq.FORMATS[u.fmt] for u in wl.units if u.timed]
+        self.units = [u for u in wl.units if u.timed]
+        dev = self.units[0].W.device
+        # preallocated outputs and workspaces (the timed region allocates nothing)
+        self.m = {}
+        self.ws_im = {}
+        for name, site in wl.sites.items():
+            if not any(u.site == name for u in self.units):
+                continue
+            X = site.X
+            self.m[name] = torch.zeros((X.shape[0], X.shape[2]), dtype=torch.float32, device=dev)
+            self.ws_im[name] = torch.empty(max(16, tq.imatrix_workspace_bytes(X)), dtype=torch.uint8, device=dev)
+        self.res, self.dq, self.px, self.ws_px = [], [], [], []
+        for u, fmt in zip(self.units, self.fmts):
+            E, O, I = u.W.shape
+            m = self._m_for(u)
+            self.res.append(tq.tq_search_groups(u.W, m, fmt))
+            self.dq.append(torch.empty((E, O, I), dtype=torch.bfloat16, device=dev))
+            self.px.append((torch.empty(E, dtype=torch.float64, device=dev),
+                            torch.empty(E, dtype=torch.float64, device=dev)))
+            self.ws_px.append(torch.empty(max(16, tq.proxy_workspace_bytes(u.W, fmt)), dtype=torch.uint8,
+                                          device=dev))
+        self.search_events = []
+
+    def _m_for(self, u):
+        m = self.m[u.site]
+        return m if u.W.shape[0] > 1 else m[0]
+
+    def kernels_per_step(self):
+        n = KERNELS["imatrix"] * len(self.m)
+        for u in self.units:
+            n += KERNELS["search"][u.fmt] + KERNELS["dequant"] + KERNELS["proxy"]
+        return n
+
+    def __call__(self, k: int, time_search: bool = False):
+        tq = self.tq
+        sites, Ws = self.sets[k % len(self.sets)]
+        for name in self.m:
+            X = sites[name]
+            tq.tq_imatrix(X, m=self.m[name], alpha=1.0 / X.shape[1], workspace=self.ws_im[name])
+        for i, (u, fmt) in enumerate(zip(self.units, self.fmts)):
+            W = Ws[i]
+            m = self._m_for(u)
+            E, O, I = W.shape
+            if time_search:
+                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                a.record()
+            r = tq.tq_search_groups(W, m, fmt, out=self.res[i])
+            if time_search:
+                b.record()
+                self.search_events.append((u.fmt, W.numel(), a, b))
+            tq.tq_dequant(r.packed, fmt, r.scales, r.zeros, r.global_scale, E, O, I, out=self.dq[i])
+            tq.tq_proxy_error(W, r.packed, fmt, r.scales, r.zeros, r.global_scale, m, out=self.px[i],
+                              workspace=self.ws_px[i])
+
+
+def make_sets(wl, n_sets):
+    """Input sets rotated through HBM so that no step finds its inputs in L2
+    (set 0 is the workload itself, the others are copies)."""
+    units = [u for u in wl.units if u.timed]
+    sets = [({k: v.X for k, v in wl.sites.items()}, [u.W for u in units])]
+    for _ in range(1, n_sets):
+        sets.append(({k: v.X.clone() for k, v in wl.sites.items()}, [u.W.clone() for u in units]))
+    return sets
+
+
+def input_bytes(wl):
+    b = sum(u.W.numel() * u.W.element_size() for u in wl.units if u.timed)
+    b += sum(s.X.numel() * s.X.element_size() for s in wl.sites.values())
+    return b
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+
+def oracle_sample(wl, budget_s: float = 12.0):
+    """Times the oracle (as it stands) on a bounded sample of the workload:
+    for each unit, the imatrix of its site (first matrix) and search + pack +
+    dequant + proxy error over the first rows of its first matrix, the row
+    count sized to about `budget_s` seconds.  Returns (weights/s, cores,
+    description, seconds)."""
+    import oracle
+    oracle.build()
+    units = [u for u in wl.units if u.timed]
+    # size the sample: rows per unit so that the search takes ~budget_s in total
+    probe_rows = 8
+    t0 = time.perf_counter()
+    for u in units[:1]:
+        _oracle_unit(oracle, wl, u, probe_rows)
+    per_row = (time.perf_counter() - t0) / probe_rows
+    rows = max(8, min(units[0].W.shape[1], int(budget_s / max(per_row, 1e-6))))
+    t0 = time.perf_counter()
+    n = 0
+    for u in units:
+        r = min(rows, u.W.shape[1])
+        _oracle_unit(oracle, wl, u, r)
+        n += r * u.W.shape[2]
+    dt = time.perf_counter() - t0
+    desc = (f"oracle (C, fp64, OpenMP) on {rows} rows of the first matrix of each of {len(units)} unit(s) "
+            f"= {n} weights: imatrix of the site's columns over all tokens, search+pack, dequant, proxy")
+    return n / dt, oracle.num_threads(), desc, dt
+
+
+def _oracle_unit(oracle, wl, u, rows):
+    X = wl.sites[u.site].X[0].float().cpu().numpy()
+    m = oracle.imatrix(X).astype(np.float32)
+    W = u.W[0, :rows].float().cpu().numpy()[None]
+    if u.fmt == "int3_g64_sym":
+        s, i, L, v = oracle.search_sym_int3(W, m)
+        oracle.pack_int3(v[0])
+        What = oracle.dequant_int3(v[0], s[0])
+    elif u.fmt == "int4_g128_asym":
+        s, z, i, L, q = oracle.search_asym_int4(W, m)
+        oracle.pack_nibbles(q[0], 128, z[0])
+        What = oracle.dequant_int4(q[0], s[0], z[0])
+    else:
+        g = oracle.nvfp4_global(u.W[0].float().cpu().numpy())
+        g, sc, i, L, c = oracle.search_nvfp4(W, m, gscale=g)
+        oracle.pack_nibbles(c[0], 16)
+        What = oracle.dequant_nvfp4(c, sc, g)[0]
+    oracle.proxy_error(W[0], What, m)
+
+
+# ------------------------------------------------------------------ main
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"),
+                    help="ncu DRAM bytes per launch of the dominant kernel, keyed by workload")
+    return ap.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return 0
+    wl = synth.make(args.config, "cpu", seed=0)
+    nw = wl.n_weights
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(wl, budget_s=2.0)
+    desc = cores = None
+    for _ in range(args.steps):
+        v, cores, desc, dt = oracle_sample(wl, budget_s=4.0)
+        vals.append(v)
+    v = statistics.median(vals)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": nw / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}", "weights": nw},
+            "cpu_baseline": {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    args = parse()
+    assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return reference_arm(args, world, rank)
+
+    import group_scale_search_b200 as tq
+    tq.lib()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wl = synth.make(args.config, dev, seed=rank)
+    nbytes = input_bytes(wl)
+    n_sets = max(1, min(64, math.ceil(2 * L2_BYTES / nbytes)))
+    sets = make_sets(wl, n_sets)
+    step = Step(tq, wl, sets)
+    nw = sum(u.W.numel() for u in step.units)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    for k in range(args.warmup):
+        step(k)
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev) as clk:
+        ev0.record(stream)
+        for k in range(args.steps):
+            step(k, time_search=True)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    ms_step = ms / args.steps
+    value = world * nw / (ms_step * 1e-3)
+
+    # dominant kernel: the search (CUDA events on the launching stream)
+    by_fmt = {}
+    for fmt, n, a, b in step.search_events:
+        d = by_fmt.setdefault(fmt, [0.0, 0])
+        d[0] += a.elapsed_time(b)
+        d[1] += n
+    fmt_main = max(by_fmt, key=lambda f: by_fmt[f][0])
+    search_ms = by_fmt[fmt_main][0] / args.steps
+    w_per_launch = by_fmt[fmt_main][1] / args.steps
+    pk = peaks()
+    props = torch.cuda.get_device_properties(dev)
+    sms = props.multi_processor_count
+    peak_tinst = sms * 128 * pk["sm_max_mhz"] * 1e6 / 1e12
+    achieved = SEARCH_INSTR_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3) / 1e12
+    traffic = None
+    try:
+        tj = json.load(open(args.traffic_json))
+        traffic = tj.get(args.config)
+    except Exception:
+        pass
+    clocks = clk.summary()
+    roofline = {"bound": "alu", "achieved": achieved, "peak": peak_tinst, "unit": "Tinst/s",
+                "frac": achieved / peak_tinst, "traffic": traffic,
+                "kernel": f"search {fmt_main}", "kernel_ms": search_ms,
+                "per_unit": f"{SEARCH_INSTR_PER_W[fmt_main]} FP32 lane-instr/weight "
+                            f"({SEARCH_CEE_PER_W[fmt_main]} candidate-element evaluations)",
+                "peak_basis": f"{sms} SMs x 128 FP32 lanes x {pk['sm_max_mhz']:.0f} MHz ({pk['source']} max clock)",
+                "frac_at_observed_clock": (achieved / (sms * 128 * clocks["sm_mhz"] * 1e6 / 1e12))
+                if clocks.get("sm_mhz") else None,
+                "cee_per_s": SEARCH_CEE_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3)}
+
+    # end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(tq, wl, step, args, world, barrier, dev)
+
+    line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}",
+                       "weights_per_gpu": nw,
+                       "groups_per_gpu": sum(tq.tq_num_groups(tq.FORMATS[u.fmt], u.W.shape[0] * u.W.shape[1],
+                                                              u.W.shape[2]) for u in step.units),
+                       "step": "imatrix + search with fused RTN/pack + dequant(bf16) + proxy error",
+                       "l2": (f"{n_sets} rotating input sets, {n_sets * nbytes / 2**20:.0f} MiB > 126 MiB L2"
+                              if n_sets * nbytes > L2_BYTES else
+                              f"{n_sets} input sets ({n_sets * nbytes / 2**20:.1f} MiB) fit in L2"),
+                       "parallelism": f"weak x{world}: independent workload per GPU"},
+            "groups_per_s": value / tq.tq_group_size(tq.FORMATS[fmt_main]),
+            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "gpu_launches": step.kernels_per_step() * args.steps}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc, dt = oracle_sample(wl)
+        line["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": dt}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_e2e(tq, wl, step, args, world, barrier, dev):
+    """Same step from pinned host inputs: H2D copies, the path, D2H of the
+    quantized weights (packed codes + scales + zeros/global scales) and of the
+    proxy-error sums, all inside the timed region."""
+    host_sites = {k: v.X.cpu().pin_memory() for k, v in wl.sites.items() if k in step.m}
+    host_W = [u.W.cpu().pin_memory() for u in step.units]
+    dev_sites = {k: torch.empty_like(v.X) for k, v in wl.sites.items() if k in step.m}
+    dev_W = [torch.empty_like(u.W) for u in step.units]
+    outs = []
+    for r, (a, b) in zip(step.res, step.px):
+        ts = [r.packed, r.scales] + ([r.zeros] if r.zeros is not None else []) + \
+             ([r.global_scale] if r.global_scale is not None else []) + [a, b]
+        outs.append([(t, torch.empty(t.shape, dtype=t.dtype, pin_memory=True)) for t in ts])
+    h2d = sum(t.numel() * t.element_size() for t in list(host_sites.values()) + host_W)
+    d2h = sum(h.numel() * h.element_size() for o in outs for _, h in o)
+    e2e_step = Step.__new__(Step)
+    e2e_step.__dict__.update(step.__dict__)
+    e2e_step.sets = [(dev_sites, dev_W)]
+
+    def one():
+        for k, v in host_sites.items():
+            dev_sites[k].copy_(v, non_blocking=True)
+        for d, h in zip(dev_W, host_W):
+            d.copy_(h, non_blocking=True)
+        e2e_step(0)
+        for o in outs:
+            for d, h in o:
+                h.copy_(d, non_blocking=True)
+
+    for _ in range(max(3, args.warmup // 2)):
+        one()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    steps = max(3, args.steps // 2)
+    a.record()
+    for _ in range(steps):
+        one()
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms = a.elapsed_time(b)
+    if world > 1:
+        import torch.distributed as dist
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    nw = sum(u.W.numel() for u in step.units)
+    return {"value": world * nw / (ms / steps * 1e-3), "unit": "weights/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps}
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,351 @@
+"""Python binding of the tq C ABI (include/tq.h): group-scale search, RTN,
+low-bit packing, dequantization and imatrix-weighted reconstruction error on
+NVIDIA B200 (sm_100a).
+
+This module only marshals arguments: torch tensors supply device memory and
+the current CUDA stream; every step runs in the CUDA kernels of libtq.so.
+There is no CPU fallback -- importing works without a GPU (so the library's
+exports can be inspected), but every call needs CUDA tensors and the built
+library, and raises otherwise.
+
+Function names match the C entry points:
+
+    tq_imatrix(X)                      -> m            (per-column mean of x^2)
+    tq_amax(W)                         -> amax per matrix
+    tq_search_groups(W, m, fmt)        -> SearchResult (scales, zeros, global scale,
+                                                        candidate index, loss, packed)
+    tq_pack(W, fmt, scales, ...)       -> packed bytes
+    tq_pack_codes / tq_unpack_codes    -> packed bytes / codes
+    tq_dequant(packed, fmt, ...)       -> What
+    tq_proxy_error(W, packed, fmt, ..) -> (num, den) per matrix
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "INT3_G64_SYM", "INT4_G128_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
+    "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
+    "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
+    "tq_dequant", "tq_proxy_error", "tq_sync", "FORMATS", "EXPORTS",
+]
+
+INT4_G128_ASYM = 4
+INT3_G64_SYM = 5
+NVFP4_G16 = 16
+FORMATS = {"int3_g64_sym": INT3_G64_SYM, "int4_g128_asym": INT4_G128_ASYM, "nvfp4_g16": NVFP4_G16}
+_GROUP = {INT3_G64_SYM: 64, INT4_G128_ASYM: 128, NVFP4_G16: 16}
+_F32, _BF16 = 0, 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libtq.so")
+_lib = None
+
+# every symbol include/tq.h declares
+EXPORTS = [
+    "tq_default_params", "tq_last_error_string", "tq_version", "tq_group_size", "tq_num_groups",
+    "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
+    "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
+    "tq_proxy_error", "tq_sync",
+]
+
+
+class TQError(RuntimeError):
+    """A tq_* call returned a non-zero status."""
+
+
+class _Mat(ctypes.Structure):
+    _fields_ = [("ptr", ctypes.c_void_p), ("dtype", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("n_mat", ctypes.c_int64), ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("ld", ctypes.c_int64), ("mat_stride", ctypes.c_int64)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("sym_n1", ctypes.c_int32), ("sym_n2", ctypes.c_int32), ("sym_lo", ctypes.c_double),
+                ("sym_hi", ctypes.c_double), ("asym_n_scale", ctypes.c_int32),
+                ("asym_n_zero", ctypes.c_int32), ("asym_lo", ctypes.c_double),
+                ("asym_hi", ctypes.c_double), ("fp4_window", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
+
+
+@dataclasses.dataclass
+class SearchParams:
+    """Candidate grids (defaults: the workloads' 32+32 symmetric, 64x32
+    asymmetric and 16-code NVFP4 grids)."""
+    sym_n1: int = 32
+    sym_n2: int = 32
+    sym_lo: float = 0.5
+    sym_hi: float = 1.2
+    asym_n_scale: int = 64
+    asym_n_zero: int = 32
+    asym_lo: float = 0.5
+    asym_hi: float = 1.2
+    fp4_window: int = 16
+
+    def _c(self) -> _Params:
+        return _Params(self.sym_n1, self.sym_n2, self.sym_lo, self.sym_hi, self.asym_n_scale,
+                       self.asym_n_zero, self.asym_lo, self.asym_hi, self.fp4_window, 0)
+
+
+@dataclasses.dataclass
+class SearchResult:
+    fmt: int
+    scales: torch.Tensor                  # f32 [n_mat, O, G] (int3/int4) or u8 E4M3 codes (NVFP4)
+    zeros: Optional[torch.Tensor]         # u8 [n_mat, O, G] (int4)
+    global_scale: Optional[torch.Tensor]  # f32 [n_mat] (NVFP4)
+    cand_idx: Optional[torch.Tensor]      # int32 [n_mat, O, G]
+    loss: Optional[torch.Tensor]          # f32 [n_mat, O, G]
+    packed: Optional[torch.Tensor]        # u8 [n_mat * O * G * record bytes]
+
+
+def lib_path() -> str:
+    return _LIB_PATH
+
+
+def lib():
+    """The loaded libtq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                              "`python -m group_scale_search_b200.build` (nvcc, sm_100a)")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        Mp = ctypes.POINTER(_Mat)
+        sig = {
+            "tq_default_params": (None, [ctypes.POINTER(_Params)]),
+            "tq_last_error_string": (ctypes.c_char_p, []),
+            "tq_version": (ctypes.c_char_p, []),
+            "tq_group_size": (i64, [i32]),
+            "tq_num_groups": (i64, [i32, i64, i64]),
+            "tq_packed_bytes": (sz, [i32, i64, i64]),
+            "tq_imatrix_workspace_bytes": (sz, [Mp]),
+            "tq_imatrix": (i32, [Mp, P, i64, ctypes.c_float, i32, P, sz, P]),
+            "tq_amax": (i32, [Mp, P, P]),
+            "tq_search_groups": (i32, [Mp, P, i64, i32, ctypes.POINTER(_Params), P, P, P, P, P, P, P]),
+            "tq_pack": (i32, [Mp, i32, P, P, P, P, P]),
+            "tq_pack_codes": (i32, [P, i32, i64, i64, P, P, P]),
+            "tq_unpack_codes": (i32, [P, i32, i64, i64, P, P]),
+            "tq_dequant": (i32, [P, i32, P, P, P, i64, i64, i64, P, i32, P]),
+            "tq_proxy_workspace_bytes": (sz, [Mp, i32]),
+            "tq_proxy_error": (i32, [Mp, P, i32, P, P, P, P, i64, P, P, P, sz, P]),
+            "tq_sync": (i32, [P]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+# ---------------------------------------------------------------- marshalling
+
+def _check(status: int, what: str) -> None:
+    if status != 0:
+        msg = lib().tq_last_error_string().decode(errors="replace")
+        raise TQError(f"{what} failed (status {status}): {msg}")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TQError(f"{name} must be a CUDA tensor (the library has no CPU path)")
+    return t
+
+
+def _mat(t: torch.Tensor, name: str) -> _Mat:
+    _cuda(t, name)
+    if t.dtype == torch.bfloat16:
+        dt = _BF16
+    elif t.dtype == torch.float32:
+        dt = _F32
+    else:
+        raise TQError(f"{name}: dtype {t.dtype} not supported (bf16 or fp32)")
+    if t.dim() == 2:
+        t3 = t.unsqueeze(0)
+    elif t.dim() == 3:
+        t3 = t
+    else:
+        raise TQError(f"{name}: expected [O, I] or [n_mat, O, I]")
+    if t3.stride(2) != 1:
+        raise TQError(f"{name}: the last dimension must be contiguous")
+    E, O, I = t3.shape
+    return _Mat(t3.data_ptr(), dt, 0, E, O, I, t3.stride(1), t3.stride(0) if E > 1 else 0)
+
+
+def _m_stride(m: torch.Tensor) -> int:
+    return m.stride(0) if m.dim() == 2 and m.shape[0] > 1 else 0
+
+
+def _groups(W: torch.Tensor, fmt: int):
+    E, O, I = (W.unsqueeze(0) if W.dim() == 2 else W).shape
+    g = _GROUP[fmt]
+    return E, O, I, (I + g - 1) // g
+
+
+# ---------------------------------------------------------------- API
+
+def tq_version() -> str:
+    return lib().tq_version().decode()
+
+
+def tq_group_size(fmt: int) -> int:
+    return int(lib().tq_group_size(fmt))
+
+
+def tq_num_groups(fmt: int, rows: int, cols: int) -> int:
+    return int(lib().tq_num_groups(fmt, rows, cols))
+
+
+def tq_packed_bytes(fmt: int, rows: int, cols: int) -> int:
+    return int(lib().tq_packed_bytes(fmt, rows, cols))
+
+
+def tq_sync(stream=None) -> None:
+    _check(lib().tq_sync(_stream(stream)), "tq_sync")
+
+
+def tq_imatrix(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optional[float] = None,
+               accumulate: bool = False, workspace: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    """m[e, j] = alpha * sum_t X[e, t, j]^2 (alpha defaults to 1/T): the
+    activation imatrix.  X: [T, I] or [n_mat, T, I] bf16/fp32 on the GPU."""
+    d = _mat(X, "X")
+    if alpha is None:
+        alpha = 1.0 / d.rows
+    if m is None:
+        m = torch.zeros((d.n_mat, d.cols), dtype=torch.float32, device=X.device)
+    _cuda(m, "m")
+    ws_bytes = int(lib().tq_imatrix_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=X.device)
+    _check(lib().tq_imatrix(ctypes.byref(d), _ptr(m), _m_stride(m) if m.dim() == 2 else 0,
+                            ctypes.c_float(alpha), int(accumulate), _ptr(workspace),
+                            workspace.numel(), _stream(stream)), "tq_imatrix")
+    return m
+
+
+def tq_amax(W: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    d = _mat(W, "W")
+    if out is None:
+        out = torch.empty(d.n_mat, dtype=torch.float32, device=W.device)
+    _check(lib().tq_amax(ctypes.byref(d), _ptr(out), _stream(stream)), "tq_amax")
+    return out
+
+
+def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optional[SearchParams] = None,
+                     pack: bool = True, want_idx: bool = True, want_loss: bool = True,
+                     out: Optional[SearchResult] = None, stream=None) -> SearchResult:
+    """imatrix-weighted per-group scale (and zero-point) search; with
+    pack=True the chosen codes are rounded and packed in the same kernel.
+    m: [I] (shared) or [n_mat, I] fp32 imatrix."""
+    d = _mat(W, "W")
+    _cuda(m, "m")
+    E, O, I, G = _groups(W, fmt)
+    dev = W.device
+    if out is None:
+        sdt = torch.uint8 if fmt == NVFP4_G16 else torch.float32
+        out = SearchResult(
+            fmt=fmt,
+            scales=torch.empty((E, O, G), dtype=sdt, device=dev),
+            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt == INT4_G128_ASYM else None,
+            global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
+            cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
+            loss=torch.empty((E, O, G), dtype=torch.float32, device=dev) if want_loss else None,
+            packed=torch.empty(tq_packed_bytes(fmt, E * O, I), dtype=torch.uint8, device=dev) if pack else None,
+        )
+    p = (params or SearchParams())._c()
+    _check(lib().tq_search_groups(ctypes.byref(d), _ptr(m), _m_stride(m), fmt, ctypes.byref(p),
+                                  _ptr(out.scales), _ptr(out.zeros), _ptr(out.global_scale),
+                                  _ptr(out.cand_idx), _ptr(out.loss), _ptr(out.packed),
+                                  _stream(stream)), "tq_search_groups")
+    return out
+
+
+def tq_pack(W: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Optional[torch.Tensor] = None,
+            global_scale: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
+    d = _mat(W, "W")
+    E, O, I, G = _groups(W, fmt)
+    if out is None:
+        out = torch.empty(tq_packed_bytes(fmt, E * O, I), dtype=torch.uint8, device=W.device)
+    _check(lib().tq_pack(ctypes.byref(d), fmt, _ptr(scales), _ptr(zeros), _ptr(global_scale), _ptr(out),
+                         _stream(stream)), "tq_pack")
+    return out
+
+
+def tq_pack_codes(codes: torch.Tensor, fmt: int, zeros: Optional[torch.Tensor] = None,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """codes: [rows, cols] (any leading dims are flattened into rows) int8/uint8."""
+    _cuda(codes, "codes")
+    c = codes.reshape(-1, codes.shape[-1]).contiguous()
+    if c.dtype == torch.int8:
+        c = c.view(torch.uint8)
+    rows, cols = c.shape
+    if out is None:
+        out = torch.empty(tq_packed_bytes(fmt, rows, cols), dtype=torch.uint8, device=codes.device)
+    _check(lib().tq_pack_codes(_ptr(c), fmt, rows, cols, _ptr(zeros), _ptr(out), _stream(stream)),
+           "tq_pack_codes")
+    return out
+
+
+def tq_unpack_codes(packed: torch.Tensor, fmt: int, rows: int, cols: int, stream=None) -> torch.Tensor:
+    _cuda(packed, "packed")
+    out = torch.empty((rows, cols), dtype=torch.uint8, device=packed.device)
+    _check(lib().tq_unpack_codes(_ptr(packed), fmt, rows, cols, _ptr(out), _stream(stream)),
+           "tq_unpack_codes")
+    return out.view(torch.int8) if fmt == INT3_G64_SYM else out
+
+
+def tq_dequant(packed: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Optional[torch.Tensor],
+               global_scale: Optional[torch.Tensor], n_mat: int, O: int, I: int,
+               out_dtype=torch.float32, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _cuda(packed, "packed")
+    if out is None:
+        out = torch.empty((n_mat, O, I), dtype=out_dtype, device=packed.device)
+    odt = _BF16 if out.dtype == torch.bfloat16 else _F32
+    _check(lib().tq_dequant(_ptr(packed), fmt, _ptr(scales), _ptr(zeros), _ptr(global_scale), n_mat, O, I,
+                            _ptr(out), odt, _stream(stream)), "tq_dequant")
+    return out
+
+
+def tq_proxy_error(W: torch.Tensor, packed: torch.Tensor, fmt: int, scales: torch.Tensor,
+                   zeros: Optional[torch.Tensor], global_scale: Optional[torch.Tensor], m: torch.Tensor,
+                   out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                   workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(num, den) fp64 per matrix: tr(E H E^T), tr(W H W^T) with H = diag(m)."""
+    d = _mat(W, "W")
+    if out is None:
+        out = (torch.empty(d.n_mat, dtype=torch.float64, device=W.device),
+               torch.empty(d.n_mat, dtype=torch.float64, device=W.device))
+    ws = int(lib().tq_proxy_workspace_bytes(ctypes.byref(d), fmt))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=W.device)
+    _check(lib().tq_proxy_error(ctypes.byref(d), _ptr(packed), fmt, _ptr(scales), _ptr(zeros),
+                                _ptr(global_scale), _ptr(m), _m_stride(m), _ptr(out[0]), _ptr(out[1]),
+                                _ptr(workspace), workspace.numel(), _stream(stream)), "tq_proxy_error")
+    return out
+
+
+def imatrix_workspace_bytes(X: torch.Tensor) -> int:
+    d = _mat(X, "X")
+    return int(lib().tq_imatrix_workspace_bytes(ctypes.byref(d)))
+
+
+def proxy_workspace_bytes(W: torch.Tensor, fmt: int) -> int:
+    d = _mat(W, "W")
+    return int(lib().tq_proxy_workspace_bytes(ctypes.byref(d), fmt))

@@ -1,0 +1,234 @@
+// Activation imatrix m_j = alpha * sum_t x_{t,j}^2 ("NeUQI Accuracy
+// Validation", opening paragraph: the search is weighted by the activation
+// imatrix; tt-stack issue #67, pipeline step 1: H = sum X^T X, whose diagonal
+// over T is this) and the per-matrix amax for the NVFP4 global scale.
+//
+// B200 mapping (HBM-bound column reduction): a block covers 32 x VEC
+// consecutive columns (16-byte loads, VEC = 8 bf16 / 4 fp32 per lane) and a
+// slice of tokens; its 8 warps walk interleaved tokens with 4 loads in
+// flight each.  Squares are summed in fp32 over runs of 32 tokens and folded
+// into fp64; the 8 warps are combined in shared memory and each (slice,
+// column) partial is written to the caller's workspace.  A second kernel adds
+// the slices in a fixed order, so results do not depend on scheduling.
+#include "tq_internal.cuh"
+
+namespace tq {
+
+constexpr int IM_THREADS = 256;
+constexpr int IM_WARPS = IM_THREADS / 32;
+constexpr int64_t IM_TARGET_BLOCKS = 1184;   // ~8 blocks per SM on a 148-SM B200
+
+template <typename T> struct VecOf { static constexpr int n = 16 / sizeof(T); };
+
+template <typename T>
+__device__ __forceinline__ void load_vec(const T* p, float* out);
+template <>
+__device__ __forceinline__ void load_vec<uint16_t>(const uint16_t* p, float* out) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+    const unsigned u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(u[i] << 16);
+        out[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+template <>
+__device__ __forceinline__ void load_vec<float>(const float* p, float* out) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+    out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+}
+
+struct ImGeom {
+    int64_t col_tiles, slices, tokens_per_slice;
+};
+
+inline ImGeom im_geometry(const tq_mat* X) {
+    const int vec = X->dtype == TQ_BF16 ? 8 : 4;
+    ImGeom g;
+    g.col_tiles = (X->cols + 32 * vec - 1) / (32 * vec);
+    const int64_t base = g.col_tiles * X->n_mat;
+    int64_t s = (IM_TARGET_BLOCKS + base - 1) / base;
+    const int64_t max_s = (X->rows + 255) / 256;   // at least 256 tokens per slice
+    if (s > max_s) s = max_s;
+    if (s < 1) s = 1;
+    g.tokens_per_slice = (X->rows + s - 1) / s;
+    g.slices = (X->rows + g.tokens_per_slice - 1) / g.tokens_per_slice;
+    return g;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(IM_THREADS)
+k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, int64_t ms,
+                  int64_t tps, double* __restrict__ partial, int64_t n_mat) {
+    constexpr int VEC = VecOf<T>::n;
+    __shared__ double red[IM_WARPS][32 * VEC];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t tile = blockIdx.x, slice = blockIdx.y, e = blockIdx.z;
+    const int64_t col = tile * 32 * VEC + lane * VEC;
+    const int64_t t0 = slice * tps, t1 = min(Tn, t0 + tps);
+    const T* base = X + e * ms + col;
+    const bool full = col + VEC <= I;
+
+    double accd[VEC];
+    float acc[VEC];
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) { accd[i] = 0.0; acc[i] = 0.f; }
+    int run = 0;
+    int64_t t = t0 + wid;
+    if (full) {
+        for (; t + 3 * IM_WARPS < t1; t += 4 * IM_WARPS) {
+            float x[4][VEC];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) load_vec<T>(base + (t + u * IM_WARPS) * ld, x[u]);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(x[u][i], x[u][i], acc[i]);
+            run += 4;
+            if (run >= 32) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
+                run = 0;
+            }
+        }
+        for (; t < t1; t += IM_WARPS) {
+            float x[VEC];
+            load_vec<T>(base + t * ld, x);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(x[i], x[i], acc[i]);
+        }
+    } else {
+        for (; t < t1; t += IM_WARPS) {
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) {
+                if (col + i < I) {
+                    const float v = Elem<T>::load(base + t * ld + i);
+                    acc[i] = __fmaf_rn(v, v, acc[i]);
+                }
+            }
+            if (++run >= 32) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
+                run = 0;
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < VEC; ++i) red[wid][lane * VEC + i] = accd[i] + static_cast<double>(acc[i]);
+    __syncthreads();
+    for (int c = threadIdx.x; c < 32 * VEC; c += IM_THREADS) {
+        double s = 0.0;
+#pragma unroll
+        for (int w = 0; w < IM_WARPS; ++w) s += red[w][c];
+        const int64_t j = tile * 32 * VEC + c;
+        if (j < I) partial[(slice * n_mat + e) * I + j] = s;
+    }
+}
+
+__global__ void k_imatrix_final(const double* __restrict__ partial, int64_t slices, int64_t n_mat,
+                                int64_t I, float* __restrict__ m, int64_t m_stride, double alpha,
+                                int accumulate) {
+    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (idx >= n_mat * I) return;
+    const int64_t e = idx / I, j = idx - e * I;
+    double s = 0.0;
+    for (int64_t k = 0; k < slices; ++k) s += partial[(k * n_mat + e) * I + j];
+    float v = static_cast<float>(alpha * s);
+    float* dst = m + e * m_stride + j;
+    if (accumulate) v = __fadd_rn(*dst, v);
+    *dst = v;
+}
+
+// ------------------------------------------------------------------ amax
+
+template <typename T>
+__global__ void k_amax(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms,
+                       unsigned* __restrict__ amax) {
+    constexpr int VEC = VecOf<T>::n;
+    const int64_t e = blockIdx.y;
+    const T* base = W + e * ms;
+    float mx = 0.f;
+    for (int64_t r = blockIdx.x; r < O; r += gridDim.x) {
+        const T* row = base + r * ld;
+        for (int64_t c = static_cast<int64_t>(threadIdx.x) * VEC; c < I; c += static_cast<int64_t>(blockDim.x) * VEC) {
+            if (c + VEC <= I) {
+                float x[VEC];
+                load_vec<T>(row + c, x);
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(x[i]));
+            } else {
+                for (int64_t i = c; i < I; ++i) mx = fmaxf(mx, fabsf(Elem<T>::load(row + i)));
+            }
+        }
+    }
+    unsigned u = __reduce_max_sync(FULL, __float_as_uint(mx));
+    __shared__ unsigned wmax[32];
+    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = u;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        unsigned v = threadIdx.x < (blockDim.x >> 5) ? wmax[threadIdx.x] : 0u;
+        v = __reduce_max_sync(FULL, v);
+        if (threadIdx.x == 0) atomicMax(amax + e, v);   // non-negative floats order like their bits
+    }
+}
+
+tq_status launch_amax(const tq_mat* W, float* amax, cudaStream_t st) {
+    cudaError_t ce = cudaMemsetAsync(amax, 0, static_cast<size_t>(W->n_mat) * sizeof(float), st);
+    if (ce != cudaSuccess) return set_error(TQ_ERR_CUDA, "amax: %s", cudaGetErrorString(ce));
+    const int64_t per = max(static_cast<int64_t>(1), static_cast<int64_t>(num_sms()) * 4 / W->n_mat);
+    const dim3 grid(static_cast<unsigned>(min(per, W->rows)), static_cast<unsigned>(W->n_mat));
+    const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
+    if (W->dtype == TQ_BF16)
+        k_amax<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->rows, W->cols, W->ld, ms,
+                                              reinterpret_cast<unsigned*>(amax));
+    else
+        k_amax<float><<<grid, 256, 0, st>>>(static_cast<const float*>(W->ptr), W->rows, W->cols, W->ld, ms,
+                                           reinterpret_cast<unsigned*>(amax));
+    return check_launch("amax");
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+TQ_API size_t tq_imatrix_workspace_bytes(const tq_mat* X) {
+    if (!X || X->n_mat < 1 || X->rows < 1 || X->cols < 1 || elem_bytes(X->dtype) == 0) return 0;
+    const ImGeom g = im_geometry(X);
+    return static_cast<size_t>(g.slices * X->n_mat * X->cols) * sizeof(double);
+}
+
+TQ_API tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
+                            void* workspace, size_t workspace_bytes, tq_stream_t stream) {
+    clear_error();
+    tq_status s = check_mat(X, "tq_imatrix X");
+    if (s != TQ_OK) return s;
+    TQ_REQUIRE(m != nullptr, "tq_imatrix: null m");
+    TQ_REQUIRE(m_stride >= X->cols || X->n_mat == 1, "tq_imatrix: m_stride < cols");
+    TQ_REQUIRE(workspace != nullptr && aligned16(workspace), "tq_imatrix: workspace null or not 16-byte aligned");
+    const size_t need = tq_imatrix_workspace_bytes(X);
+    TQ_REQUIRE(workspace_bytes >= need, "tq_imatrix: workspace too small (%zu < %zu bytes)", workspace_bytes, need);
+    const ImGeom g = im_geometry(X);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    double* partial = static_cast<double*>(workspace);
+    const dim3 grid(static_cast<unsigned>(g.col_tiles), static_cast<unsigned>(g.slices), static_cast<unsigned>(X->n_mat));
+    const int64_t ms = X->n_mat > 1 ? X->mat_stride : 0;
+    if (X->dtype == TQ_BF16)
+        k_imatrix_partial<uint16_t><<<grid, IM_THREADS, 0, st>>>(static_cast<const uint16_t*>(X->ptr), X->rows, X->cols,
+                                                                 X->ld, ms, g.tokens_per_slice, partial, X->n_mat);
+    else
+        k_imatrix_partial<float><<<grid, IM_THREADS, 0, st>>>(static_cast<const float*>(X->ptr), X->rows, X->cols,
+                                                              X->ld, ms, g.tokens_per_slice, partial, X->n_mat);
+    if ((s = check_launch("imatrix partial")) != TQ_OK) return s;
+    const int64_t n = X->n_mat * X->cols;
+    k_imatrix_final<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
+        partial, g.slices, X->n_mat, X->cols, m, X->n_mat > 1 ? m_stride : 0, static_cast<double>(alpha), accumulate);
+    return check_launch("imatrix final");
+}
+
+TQ_API tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream) {
+    clear_error();
+    tq_status s = check_mat(W, "tq_amax W");
+    if (s != TQ_OK) return s;
+    TQ_REQUIRE(amax != nullptr, "tq_amax: null output");
+    return launch_amax(W, amax, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -1,0 +1,322 @@
+// Symmetric int3-g64 two-stage signed-scale search with fused RTN + pack.
+//
+// Method ("NeUQI Accuracy Validation", opening paragraph: symmetric layers run
+// a two-stage signed scale search weighted by the activation imatrix):
+//   stage 1: candidates s = +-fl32(r_k M)/4, r_k on an n1-point grid of
+//            [lo, hi], M = max|w| of the group;
+//   stage 2: n2 ratios spread over [r_k* - d, r_k* + d] with the stage-1 sign;
+//   codes v = clamp(rint(w/s), -4, 3); loss L = sum_j m_j (w_j - s v_j)^2;
+//   ties keep the lowest candidate index.
+// Layout of the packed record: "int3-g64 (fmt=5)", Design: Layout.
+//
+// B200 mapping: one warp per 64-weight group, lane k = stage-1 magnitude k
+// (both signs) and then stage-2 ratio k.  The group's (w, m) pairs sit in
+// shared memory and are read with broadcast 16-byte loads, so every candidate
+// reuses one HBM read of the group.  Elements are split once per group into
+// "small" ones (|w| < 3.49 s_min: no candidate can clamp them) and the rest:
+// for small elements the +s and -s candidates have identical errors (round
+// half to even is odd-symmetric), so stage 1 evaluates them once per
+// magnitude and only the few large elements per sign.  Candidates are ranked
+// in fp32 with the multiply-by-reciprocal rounding; all candidates within a
+// relative 2^-15 of the best are re-evaluated in fp64 with codes from the IEEE
+// quotient, which decides the winner exactly as the definition does.
+#include "group_pack.cuh"
+
+#include <climits>
+
+namespace tq {
+
+constexpr int SYM_WARPS = 8;
+constexpr float WIN = 3.0517578125e-05f;   // 2^-15: bound on fp32 ranking error x 2 (with margin)
+
+struct SymArgs {
+    const void* W;
+    int64_t n_mat, O, I, ld, ms;
+    const float* m;
+    int64_t m_stride;
+    float* scales;
+    int32_t* idx;
+    float* loss;
+    uint8_t* packed;
+    int n1, n2;
+    float r_lo;          // smallest ratio of either stage
+    float r1[32];
+    float r2[32 * 32];   // [k*][i]
+};
+
+__device__ __forceinline__ float err_free(float w, float m, float s, float inv, float acc) {
+    const float t = __fmaf_rn(w, inv, MAGIC);
+    const float q = __fsub_rn(t, MAGIC);
+    const float e = __fmaf_rn(-s, q, w);
+    return __fmaf_rn(__fmul_rn(m, e), e, acc);
+}
+
+// One element under +s and -s (magnitude s): the rounded quotient is shared,
+// only the clamp differs ([-4, 3] for +s, which is [-3, 4] in units of -s).
+__device__ __forceinline__ void err_both(float w, float m, float s, float inv, float& accP, float& accN) {
+    const float t = __fmaf_rn(w, inv, MAGIC);
+    const float qp = __fsub_rn(fminf(fmaxf(t, MAGIC - 4.f), MAGIC + 3.f), MAGIC);
+    const float qn = __fsub_rn(fminf(fmaxf(t, MAGIC - 3.f), MAGIC + 4.f), MAGIC);
+    const float ep = __fmaf_rn(-s, qp, w);
+    const float en = __fmaf_rn(-s, qn, w);
+    accP = __fmaf_rn(__fmul_rn(m, ep), ep, accP);
+    accN = __fmaf_rn(__fmul_rn(m, en), en, accN);
+}
+
+__device__ __forceinline__ float err_clamped(float w, float m, float s, float inv, float lo, float hi, float acc) {
+    const float t = fminf(fmaxf(__fmaf_rn(w, inv, MAGIC), lo), hi);
+    const float q = __fsub_rn(t, MAGIC);
+    const float e = __fmaf_rn(-s, q, w);
+    return __fmaf_rn(__fmul_rn(m, e), e, acc);
+}
+
+// fp64 loss of signed scale s over the warp's 64 elements (lane: l, l + 32),
+// codes from the IEEE quotient.  Identical in every lane.
+__device__ __forceinline__ double loss64_int3(float w0, float m0, float w1, float m1, float s) {
+    const double v0 = rtn_exact(w0, s, -4.f, 3.f), v1 = rtn_exact(w1, s, -4.f, 3.f);
+    const double e0 = __dsub_rn(static_cast<double>(w0), __dmul_rn(static_cast<double>(s), v0));
+    const double e1 = __dsub_rn(static_cast<double>(w1), __dmul_rn(static_cast<double>(s), v1));
+    const double t = __dadd_rn(__dmul_rn(static_cast<double>(m0), __dmul_rn(e0, e0)),
+                               __dmul_rn(static_cast<double>(m1), __dmul_rn(e1, e1)));
+    return group_sum_d(t, FULL, 32);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(SYM_WARPS * 32)
+k_search_int3(const __grid_constant__ SymArgs a) {
+    __shared__ float r2s[32 * 32];
+    __shared__ __align__(16) float2 lists[SYM_WARPS][2][64];
+
+    for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) r2s[i] = a.r2[i];
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t G = (a.I + 63) >> 6;
+    const int64_t OG = a.O * G;
+    const int64_t total = a.n_mat * OG;
+    const bool act1 = lane < a.n1, act2 = lane < a.n2;
+    const float r1v = a.r1[act1 ? lane : 0];
+    float2* small = lists[wid][0];
+    float2* large = lists[wid][1];
+    const T* W = static_cast<const T*>(a.W);
+    const unsigned lt = (1u << lane) - 1u;
+
+    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total;
+         gid += static_cast<int64_t>(gridDim.x) * SYM_WARPS) {
+        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
+        const int64_t j0 = k << 6;
+        const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
+        const T* wp = W + e * a.ms + o * a.ld + j0;
+        const float* mp = a.m + e * a.m_stride + j0;
+        const bool v0 = lane < n, v1 = lane + 32 < n;
+        const float w0 = v0 ? Elem<T>::load(wp + lane) : 0.f;
+        const float w1 = v1 ? Elem<T>::load(wp + lane + 32) : 0.f;
+        const float m0 = v0 ? __ldg(mp + lane) : 0.f;
+        const float m1 = v1 ? __ldg(mp + lane + 32) : 0.f;
+        const float M = warp_max_abs(w0, w1);
+        uint8_t* rec = a.packed ? a.packed + gid * 24 : nullptr;
+
+        if (M == 0.f) {   // nothing to fit: scale 0, codes 0
+            if (lane == 0) {
+                a.scales[gid] = 0.f;
+                if (a.idx) a.idx[gid] = -1;
+                if (a.loss) a.loss[gid] = 0.f;
+            }
+            if (rec) pack_int3_record(4u, 4u, lane, rec);
+            continue;
+        }
+
+        // ---- split elements: small ones cannot be clamped by any candidate
+        const float s_lo = __fmul_rn(__fmul_rn(a.r_lo, M), 0.25f);
+        const float thr = __fmul_rn(3.49f, s_lo);
+        const bool sm0 = v0 && fabsf(w0) < thr, sm1 = v1 && fabsf(w1) < thr;
+        const bool lg0 = v0 && !sm0, lg1 = v1 && !sm1;
+        const unsigned bs0 = __ballot_sync(FULL, sm0), bs1 = __ballot_sync(FULL, sm1);
+        const unsigned bl0 = __ballot_sync(FULL, lg0), bl1 = __ballot_sync(FULL, lg1);
+        const int ns0 = __popc(bs0), ns = ns0 + __popc(bs1);
+        const int nl0 = __popc(bl0), nl = nl0 + __popc(bl1);
+        const int ns_pad = (ns + 3) & ~3, nl_pad = (nl + 1) & ~1;
+        __syncwarp();   // previous group's readers are done with the lists
+        if (sm0) small[__popc(bs0 & lt)] = make_float2(w0, m0);
+        if (sm1) small[ns0 + __popc(bs1 & lt)] = make_float2(w1, m1);
+        if (lg0) large[__popc(bl0 & lt)] = make_float2(w0, m0);
+        if (lg1) large[nl0 + __popc(bl1 & lt)] = make_float2(w1, m1);
+        if (lane < ns_pad - ns) small[ns + lane] = make_float2(0.f, 0.f);   // zero pairs add exactly 0
+        if (lane < nl_pad - nl) large[nl + lane] = make_float2(0.f, 0.f);
+        __syncwarp();
+        const float4* sp = reinterpret_cast<const float4*>(small);
+        const float4* lp = reinterpret_cast<const float4*>(large);
+
+        // ---- stage 1: lane = magnitude, both signs
+        const float s1 = __fmul_rn(__fmul_rn(r1v, M), 0.25f);
+        const float i1 = __frcp_rn(s1);
+        float accC = 0.f, accP = 0.f, accN = 0.f;
+        for (int j = 0; j < ns_pad; j += 4) {
+            const float4 p = sp[j >> 1], q = sp[(j >> 1) + 1];
+            accC = err_free(p.x, p.y, s1, i1, accC);
+            accC = err_free(p.z, p.w, s1, i1, accC);
+            accC = err_free(q.x, q.y, s1, i1, accC);
+            accC = err_free(q.z, q.w, s1, i1, accC);
+        }
+        for (int j = 0; j < nl_pad; j += 2) {
+            const float4 p = lp[j >> 1];
+            err_both(p.x, p.y, s1, i1, accP, accN);
+            err_both(p.z, p.w, s1, i1, accP, accN);
+        }
+        const float LP = __fadd_rn(accC, accP), LN = __fadd_rn(accC, accN);
+
+        float L = __int_as_float(0x7f800000);
+        int bi = INT_MAX;
+        if (act1) {
+            if (LN < LP) { L = LN; bi = 2 * lane + 1; } else { L = LP; bi = 2 * lane; }
+        }
+        warp_argmin(L, bi);
+        int b1 = bi;
+        bool have64 = false;
+        double L1d = 0.0;
+        {
+            const float thr1 = __fmaf_rn(L, WIN, L);
+            unsigned mpos = __ballot_sync(FULL, act1 && LP <= thr1);
+            unsigned mneg = __ballot_sync(FULL, act1 && LN <= thr1);
+            if (__popc(mpos) + __popc(mneg) > 1) {   // near tie: decide in fp64
+                double best = __longlong_as_double(0x7ff0000000000000ll);
+                int bidx = bi;
+                while (mpos | mneg) {
+                    const int kp = mpos ? __ffs(mpos) - 1 : 64, kn = mneg ? __ffs(mneg) - 1 : 64;
+                    int kk, sg;
+                    if (kp <= kn) { kk = kp; sg = 0; mpos &= mpos - 1; } else { kk = kn; sg = 1; mneg &= mneg - 1; }
+                    const float sk = __shfl_sync(FULL, s1, kk);
+                    const double Ld = loss64_int3(w0, m0, w1, m1, sg ? -sk : sk);
+                    if (Ld < best) { best = Ld; bidx = 2 * kk + sg; }
+                }
+                b1 = bidx; have64 = true; L1d = best;
+            }
+        }
+
+        // ---- stage 2: lane = refinement i around magnitude k*, sign of the winner
+        const int ks = b1 >> 1, sg = b1 & 1;
+        const float r2v = r2s[ks * 32 + (act2 ? lane : 0)];
+        const float s2 = __fmul_rn(__fmul_rn(r2v, M), 0.25f);
+        const float i2 = __frcp_rn(s2);
+        const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
+        float acc2 = 0.f;
+        for (int j = 0; j < ns_pad; j += 4) {
+            const float4 p = sp[j >> 1], q = sp[(j >> 1) + 1];
+            acc2 = err_free(p.x, p.y, s2, i2, acc2);
+            acc2 = err_free(p.z, p.w, s2, i2, acc2);
+            acc2 = err_free(q.x, q.y, s2, i2, acc2);
+            acc2 = err_free(q.z, q.w, s2, i2, acc2);
+        }
+        for (int j = 0; j < nl_pad; j += 2) {
+            const float4 p = lp[j >> 1];
+            acc2 = err_clamped(p.x, p.y, s2, i2, clo, chi, acc2);
+            acc2 = err_clamped(p.z, p.w, s2, i2, clo, chi, acc2);
+        }
+        const float L1f = __shfl_sync(FULL, sg ? LN : LP, ks);   // incumbent's fp32 loss
+        const float L2 = act2 ? acc2 : __int_as_float(0x7f800000);
+        float L2m = L2;
+        int b2 = act2 ? 2 * a.n1 + lane : INT_MAX;
+        warp_argmin(L2m, b2);
+
+        const float Lmin = fminf(L1f, L2m);
+        const float thr2 = __fmaf_rn(Lmin, WIN, Lmin);
+        const bool inc_in = L1f <= thr2;
+        unsigned c2 = __ballot_sync(FULL, act2 && L2 <= thr2);
+        int bf;
+        float lossf;
+        if (static_cast<int>(inc_in) + __popc(c2) > 1) {   // near tie: decide in fp64
+            double best = __longlong_as_double(0x7ff0000000000000ll);
+            int bidx = b2;
+            if (inc_in) {
+                if (!have64) {
+                    const float sk = __shfl_sync(FULL, s1, ks);
+                    L1d = loss64_int3(w0, m0, w1, m1, sg ? -sk : sk);
+                }
+                best = L1d; bidx = b1;
+            }
+            while (c2) {
+                const int i = __ffs(c2) - 1;
+                c2 &= c2 - 1;
+                const float si = __shfl_sync(FULL, s2, i);
+                const double Ld = loss64_int3(w0, m0, w1, m1, sg ? -si : si);
+                if (Ld < best) { best = Ld; bidx = 2 * a.n1 + i; }
+            }
+            bf = bidx;
+            lossf = static_cast<float>(best);
+        } else if (L2m < L1f) {
+            bf = b2; lossf = L2m;
+        } else {
+            bf = b1; lossf = have64 ? static_cast<float>(L1d) : L1f;
+        }
+
+        float sfin;
+        if (bf < 2 * a.n1) {
+            const float sk = __shfl_sync(FULL, s1, bf >> 1);
+            sfin = (bf & 1) ? -sk : sk;
+        } else {
+            const float si = __shfl_sync(FULL, s2, bf - 2 * a.n1);
+            sfin = sg ? -si : si;
+        }
+        if (lane == 0) {
+            a.scales[gid] = sfin;
+            if (a.idx) a.idx[gid] = bf;
+            if (a.loss) a.loss[gid] = lossf;
+        }
+        if (rec) {
+            const unsigned u0 = static_cast<unsigned>(static_cast<int>(rtn_exact(w0, sfin, -4.f, 3.f)) + 4);
+            const unsigned u1 = static_cast<unsigned>(static_cast<int>(rtn_exact(w1, sfin, -4.f, 3.f)) + 4);
+            pack_int3_record(u0, u1, lane, rec);
+        }
+    }
+}
+
+// Host side: candidate ratio tables from their definitions (fp64, rounded
+// once to fp32), then one persistent launch.
+tq_status launch_search_int3(const tq_mat* W, const float* m, int64_t m_stride,
+                             const tq_search_params* p, float* scales, int32_t* idx, float* loss,
+                             uint8_t* packed, cudaStream_t st) {
+    if (p->sym_n1 < 2 || p->sym_n1 > 32 || p->sym_n2 < 2 || p->sym_n2 > 32)
+        return set_error(TQ_ERR_UNSUPPORTED, "int3 search: sym_n1 and sym_n2 must be in [2, 32]");
+    if (!(p->sym_lo > 0.0) || !(p->sym_hi >= p->sym_lo))
+        return set_error(TQ_ERR_INVALID_ARG, "int3 search: need 0 < sym_lo <= sym_hi");
+    static thread_local SymArgs a;
+    a.W = W->ptr; a.n_mat = W->n_mat; a.O = W->rows; a.I = W->cols; a.ld = W->ld;
+    a.ms = W->n_mat > 1 ? W->mat_stride : 0;
+    a.m = m; a.m_stride = m_stride;
+    a.scales = scales; a.idx = idx; a.loss = loss; a.packed = packed;
+    a.n1 = p->sym_n1; a.n2 = p->sym_n2;
+    const double lo = p->sym_lo, hi = p->sym_hi;
+    const double delta = (hi - lo) / static_cast<double>(a.n1 - 1);
+    float rmin = 1e30f;
+    for (int k = 0; k < 32; ++k) {
+        a.r1[k] = k < a.n1 ? static_cast<float>(lo + ((hi - lo) * static_cast<double>(k)) / static_cast<double>(a.n1 - 1)) : 1.0f;
+        if (k < a.n1) rmin = fminf(rmin, a.r1[k]);
+    }
+    for (int k = 0; k < 32; ++k) {
+        const double center = lo + ((hi - lo) * static_cast<double>(k)) / static_cast<double>(a.n1 - 1);
+        for (int i = 0; i < 32; ++i) {
+            float r = 1.0f;
+            if (k < a.n1 && i < a.n2)
+                r = static_cast<float>((center - delta) + (2.0 * delta * static_cast<double>(i)) / static_cast<double>(a.n2 - 1));
+            a.r2[k * 32 + i] = r;
+            if (k < a.n1 && i < a.n2) rmin = fminf(rmin, r);
+        }
+    }
+    if (!(rmin > 0.0f)) return set_error(TQ_ERR_INVALID_ARG, "int3 search: candidate ratios must be positive");
+    a.r_lo = rmin;
+
+    const int64_t G = (W->cols + 63) / 64;
+    const int64_t total = W->n_mat * W->rows * G;
+    int bpsm = 0;
+    const bool bf16 = W->dtype == TQ_BF16;
+    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int3<uint16_t>, SYM_WARPS * 32, 0);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int3<float>, SYM_WARPS * 32, 0);
+    if (bpsm < 1) bpsm = 1;
+    const int64_t need = (total + SYM_WARPS - 1) / SYM_WARPS;
+    const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
+    if (bf16) k_search_int3<uint16_t><<<grid, SYM_WARPS * 32, 0, st>>>(a);
+    else k_search_int3<float><<<grid, SYM_WARPS * 32, 0, st>>>(a);
+    return check_launch("int3 search");
+}
+
+}  // namespace tq

@@ -1,0 +1,292 @@
+// Asymmetric int4-g128 joint (scale, integer zero-point) search with fused
+// RTN + nibble pack.
+//
+// Method ("NeUQI Accuracy Validation", opening paragraph and results bullet 2:
+// asymmetric layers run a joint (scale, integer zero-point) search weighted by
+// the activation imatrix, on a "64/32" grid):
+//   s_k = fl32(c_k R), c_k = fl32(f_k / 15), f_k evenly over [lo, hi], R = wmax - wmin;
+//   z_i = rint(15 i / (nz - 1)); q = clamp(rint(w/s) + z, 0, 15);
+//   L = sum_j m_j (w_j - s (q_j - z))^2; ties keep the lowest index nz k + i.
+//
+// B200 mapping: one warp per 128-weight group; lane l owns scales l and l+32
+// and all 16 distinct zero-points (32 fp32 accumulators).  The group's (w, m)
+// pairs are staged in shared memory and broadcast to all lanes, so the 1024
+// candidates reuse one HBM read.  Per element and scale, rint(w/s) is formed
+// once (an FMA against 1.5*2^23 and a subtract); each zero-point then costs a
+// clamp to [-z, 15-z] (two min/max), the residual FMA and the weighted-square
+// FMA pair.  Zero-points repeated in the 32-point list never win under the
+// lowest-index rule, so only the first occurrence of each is evaluated.
+// Near ties (relative 2^-15) are re-ranked in fp64 with codes from the IEEE
+// quotient, exactly as the definition ranks them.
+#include "group_pack.cuh"
+
+#include <climits>
+
+namespace tq {
+
+constexpr int ASYM_WARPS = 4;
+constexpr float AWIN = 3.0517578125e-05f;   // 2^-15
+
+struct AsymArgs {
+    const void* W;
+    int64_t n_mat, O, I, ld, ms;
+    const float* m;
+    int64_t m_stride;
+    float* scales;
+    uint8_t* zeros;
+    int32_t* idx;
+    float* loss;
+    uint8_t* packed;
+    int ns, nz;
+    int zfirst[16];      // lowest i with z_i = z
+    int8_t zval[64];     // z_i for i < nz (nz <= 64)
+    float c[64];         // fl32(f_k / 15)
+};
+
+// Lane l holds elements 4l..4l+3 of the group.
+template <typename T> struct Load4;
+template <> struct Load4<uint16_t> {
+    static __device__ __forceinline__ void go(const uint16_t* p, float w[4]) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
+        w[0] = __uint_as_float(v.x << 16); w[1] = __uint_as_float(v.x & 0xffff0000u);
+        w[2] = __uint_as_float(v.y << 16); w[3] = __uint_as_float(v.y & 0xffff0000u);
+    }
+};
+template <> struct Load4<float> {
+    static __device__ __forceinline__ void go(const float* p, float w[4]) {
+        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    }
+};
+
+__device__ __forceinline__ unsigned ord_key(float x) {   // order-preserving float -> uint
+    const unsigned b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord_val(unsigned k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ double loss64_int4(const float w[4], const float m[4], float s, int z) {
+    double t = 0.0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float q = (s == 0.f) ? static_cast<float>(z)
+                                   : fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), static_cast<float>(z)), 0.f), 15.f);
+        const double e = __dsub_rn(static_cast<double>(w[i]),
+                                   __dmul_rn(static_cast<double>(s), static_cast<double>(q) - static_cast<double>(z)));
+        t = __dadd_rn(t, __dmul_rn(static_cast<double>(m[i]), __dmul_rn(e, e)));
+    }
+    return group_sum_d(t, FULL, 32);
+}
+
+// The 16 zero-points of one scale for one element: r = rint(w/s) is shared,
+// code - z = clamp(r, -z, 15 - z).
+#define TQ_Z16(ACC, R, S, W, Mv)                                                   \
+    _Pragma("unroll") for (int z = 0; z < 16; ++z) {                               \
+        const float c_ = fminf(fmaxf(R, static_cast<float>(-z)), static_cast<float>(15 - z)); \
+        const float e_ = __fmaf_rn(-(S), c_, W);                                   \
+        ACC[z] = __fmaf_rn(__fmul_rn(Mv, e_), e_, ACC[z]);                         \
+    }
+
+template <typename T>
+__global__ void __launch_bounds__(ASYM_WARPS * 32)
+k_search_int4(const __grid_constant__ AsymArgs a) {
+    __shared__ __align__(16) float2 lists[ASYM_WARPS][128];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int64_t G = (a.I + 127) >> 7;
+    const int64_t OG = a.O * G;
+    const int64_t total = a.n_mat * OG;
+    const bool actA = lane < a.ns, actB = lane + 32 < a.ns;
+    const float cA = a.c[actA ? lane : 0], cB = a.c[actB ? lane + 32 : 0];
+    const T* W = static_cast<const T*>(a.W);
+    float2* list = lists[wid];
+    const float4* list4 = reinterpret_cast<const float4*>(list);
+
+    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * ASYM_WARPS + wid; gid < total;
+         gid += static_cast<int64_t>(gridDim.x) * ASYM_WARPS) {
+        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
+        const int64_t j0 = k << 7;
+        const int n = static_cast<int>(min(static_cast<int64_t>(128), a.I - j0));
+        const T* wp = W + e * a.ms + o * a.ld + j0;
+        const float* mp = a.m + e * a.m_stride + j0;
+        float w[4], mv[4];
+        bool val[4];
+        if (n == 128) {
+            Load4<T>::go(wp + 4 * lane, w);
+            const float4 mm = __ldg(reinterpret_cast<const float4*>(mp + 4 * lane));
+            mv[0] = mm.x; mv[1] = mm.y; mv[2] = mm.z; mv[3] = mm.w;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) val[i] = true;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int j = 4 * lane + i;
+                val[i] = j < n;
+                w[i] = val[i] ? Elem<T>::load(wp + j) : 0.f;
+                mv[i] = val[i] ? __ldg(mp + j) : 0.f;
+            }
+        }
+        unsigned kmin = 0xffffffffu, kmax = 0u;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (val[i]) { kmin = min(kmin, ord_key(w[i])); kmax = max(kmax, ord_key(w[i])); }
+        const float wmin = ord_val(__reduce_min_sync(FULL, kmin));
+        const float wmax = ord_val(__reduce_max_sync(FULL, kmax));
+        float R = __fsub_rn(wmax, wmin);
+        uint8_t* rec = a.packed ? a.packed + gid * 64 : nullptr;
+        if (R == 0.f) {
+            if (wmax == 0.f) {   // all-zero group: s = 0, z = 0, q = 0
+                if (lane == 0) {
+                    a.scales[gid] = 0.f; a.zeros[gid] = 0;
+                    if (a.idx) a.idx[gid] = -1;
+                    if (a.loss) a.loss[gid] = 0.f;
+                }
+                if (rec) { const unsigned q0[4] = {0u, 0u, 0u, 0u}; pack_int4_lane(q0, lane, rec); }
+                continue;
+            }
+            R = fabsf(wmax);
+        }
+
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) list[4 * lane + i] = make_float2(w[i], mv[i]);   // tail: (0, 0)
+        __syncwarp();
+
+        const float sA = __fmul_rn(cA, R), sB = __fmul_rn(cB, R);
+        const float iA = __frcp_rn(sA), iB = __frcp_rn(sB);
+        float accA[16], accB[16];
+#pragma unroll
+        for (int z = 0; z < 16; ++z) { accA[z] = 0.f; accB[z] = 0.f; }
+        const int npair = (n + 1) >> 1;
+        for (int j = 0; j < npair; ++j) {
+            const float4 p = list4[j];
+            {
+                const float rA = __fsub_rn(__fmaf_rn(p.x, iA, MAGIC), MAGIC);
+                TQ_Z16(accA, rA, sA, p.x, p.y)
+                const float rB = __fsub_rn(__fmaf_rn(p.x, iB, MAGIC), MAGIC);
+                TQ_Z16(accB, rB, sB, p.x, p.y)
+            }
+            {
+                const float rA = __fsub_rn(__fmaf_rn(p.z, iA, MAGIC), MAGIC);
+                TQ_Z16(accA, rA, sA, p.z, p.w)
+                const float rB = __fsub_rn(__fmaf_rn(p.z, iB, MAGIC), MAGIC);
+                TQ_Z16(accB, rB, sB, p.z, p.w)
+            }
+        }
+
+        // lane-local argmin in index order (all of scale A precede scale B)
+        float L = __int_as_float(0x7f800000);
+        int bi = INT_MAX;
+        if (actA) {
+#pragma unroll
+            for (int z = 0; z < 16; ++z)
+                if (accA[z] < L) { L = accA[z]; bi = a.nz * lane + a.zfirst[z]; }
+        }
+        if (actB) {
+#pragma unroll
+            for (int z = 0; z < 16; ++z)
+                if (accB[z] < L) { L = accB[z]; bi = a.nz * (lane + 32) + a.zfirst[z]; }
+        }
+        warp_argmin(L, bi);
+        const float thr = __fmaf_rn(L, AWIN, L);
+        unsigned wm = 0u;
+#pragma unroll
+        for (int z = 0; z < 16; ++z) {
+            if (actA && accA[z] <= thr) wm |= 1u << z;
+            if (actB && accB[z] <= thr) wm |= 1u << (16 + z);
+        }
+        const int cnt = static_cast<int>(__reduce_add_sync(FULL, static_cast<unsigned>(__popc(wm))));
+        float lossf = L;
+        if (cnt > 1) {   // near tie: decide in fp64, candidates in index order
+            double best = __longlong_as_double(0x7ff0000000000000ll);
+            int bidx = bi;
+            for (int part = 0; part < 2; ++part) {
+                unsigned ls = __ballot_sync(FULL, part ? (wm >> 16) != 0u : (wm & 0xffffu) != 0u);
+                while (ls) {
+                    const int l2 = __ffs(ls) - 1;
+                    ls &= ls - 1;
+                    unsigned zm = __shfl_sync(FULL, wm, l2);
+                    zm = part ? (zm >> 16) : (zm & 0xffffu);
+                    const float sc = __shfl_sync(FULL, part ? sB : sA, l2);
+                    while (zm) {
+                        const int z = __ffs(zm) - 1;
+                        zm &= zm - 1;
+                        const double Ld = loss64_int4(w, mv, sc, z);
+                        if (Ld < best) { best = Ld; bidx = a.nz * (l2 + 32 * part) + a.zfirst[z]; }
+                    }
+                }
+            }
+            bi = bidx;
+            lossf = static_cast<float>(best);
+        }
+
+        const int kb = bi / a.nz;
+        const int zb = a.zval[bi - kb * a.nz];
+        const float sfin = __fmul_rn(a.c[kb], R);
+        if (lane == 0) {
+            a.scales[gid] = sfin;
+            a.zeros[gid] = static_cast<uint8_t>(zb);
+            if (a.idx) a.idx[gid] = bi;
+            if (a.loss) a.loss[gid] = lossf;
+        }
+        if (rec) {
+            unsigned q[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float qq = (sfin == 0.f || !val[i]) ? static_cast<float>(zb)
+                    : fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], sfin)), static_cast<float>(zb)), 0.f), 15.f);
+                q[i] = static_cast<unsigned>(qq);
+            }
+            pack_int4_lane(q, lane, rec);
+        }
+    }
+}
+
+tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
+                             const tq_search_params* p, float* scales, uint8_t* zeros, int32_t* idx,
+                             float* loss, uint8_t* packed, cudaStream_t st) {
+    if (p->asym_n_scale < 2 || p->asym_n_scale > 64)
+        return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_scale must be in [2, 64]");
+    if (p->asym_n_zero < 16 || p->asym_n_zero > 64)
+        return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_zero must be in [16, 64]");
+    if (!(p->asym_lo > 0.0) || !(p->asym_hi >= p->asym_lo))
+        return set_error(TQ_ERR_INVALID_ARG, "int4 search: need 0 < asym_lo <= asym_hi");
+    AsymArgs a;
+    a.W = W->ptr; a.n_mat = W->n_mat; a.O = W->rows; a.I = W->cols; a.ld = W->ld;
+    a.ms = W->n_mat > 1 ? W->mat_stride : 0;
+    a.m = m; a.m_stride = m_stride;
+    a.scales = scales; a.zeros = zeros; a.idx = idx; a.loss = loss; a.packed = packed;
+    a.ns = p->asym_n_scale; a.nz = p->asym_n_zero;
+    const double lo = p->asym_lo, hi = p->asym_hi;
+    for (int k = 0; k < 64; ++k) {
+        const double f = lo + ((hi - lo) * static_cast<double>(k)) / static_cast<double>(a.ns - 1);
+        a.c[k] = k < a.ns ? static_cast<float>(f / 15.0) : 1.0f;
+    }
+    for (int z = 0; z < 16; ++z) a.zfirst[z] = -1;
+    for (int i = 0; i < 64; ++i) {
+        int z = 0;
+        if (i < a.nz) {
+            z = static_cast<int>(nearbyint((15.0 * static_cast<double>(i)) / static_cast<double>(a.nz - 1)));
+            if (a.zfirst[z] < 0) a.zfirst[z] = i;
+        }
+        a.zval[i] = static_cast<int8_t>(z);
+    }
+    for (int z = 0; z < 16; ++z)
+        if (a.zfirst[z] < 0) return set_error(TQ_ERR_UNSUPPORTED, "int4 search: zero-point %d not on the grid", z);
+
+    const int64_t G = (W->cols + 127) / 128;
+    const int64_t total = W->n_mat * W->rows * G;
+    int bpsm = 0;
+    const bool bf16 = W->dtype == TQ_BF16;
+    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t>, ASYM_WARPS * 32, 0);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<float>, ASYM_WARPS * 32, 0);
+    if (bpsm < 1) bpsm = 1;
+    const int64_t need = (total + ASYM_WARPS - 1) / ASYM_WARPS;
+    const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
+    if (bf16) k_search_int4<uint16_t><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    else k_search_int4<float><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    return check_launch("int4 search");
+}
+
+}  // namespace tq

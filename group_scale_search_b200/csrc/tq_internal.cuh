@@ -1,0 +1,132 @@
+// Private helpers of the tq CUDA library (host validation + device building
+// blocks).  Not part of the C ABI; see include/tq.h for the interface.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <stdarg.h>
+
+#include "../../include/tq.h"
+
+#define TQ_API extern "C" __attribute__((visibility("default")))
+
+namespace tq {
+
+// ------------------------------------------------------------------ host: errors
+
+tq_status set_error(tq_status st, const char* fmt, ...);
+void clear_error();
+tq_status check_launch(const char* what);
+
+#define TQ_REQUIRE(cond, ...)                                          \
+    do {                                                               \
+        if (!(cond)) return ::tq::set_error(TQ_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline int elem_bytes(int32_t dt) { return dt == TQ_BF16 ? 2 : (dt == TQ_F32 ? 4 : 0); }
+
+inline int64_t group_of(int32_t fmt) {
+    return fmt == TQ_INT3_G64_SYM ? 64 : fmt == TQ_INT4_G128_ASYM ? 128 : fmt == TQ_NVFP4_G16 ? 16 : 0;
+}
+inline int64_t record_bytes(int32_t fmt) {
+    return fmt == TQ_INT3_G64_SYM ? 24 : fmt == TQ_INT4_G128_ASYM ? 64 : fmt == TQ_NVFP4_G16 ? 8 : 0;
+}
+
+// Validates a matrix batch descriptor; returns TQ_OK or an error (set).
+tq_status check_mat(const tq_mat* X, const char* name);
+
+int num_sms();
+
+// ------------------------------------------------------------------ device helpers
+
+constexpr unsigned FULL = 0xffffffffu;
+// Adding then subtracting 1.5 * 2^23 rounds an fp32 value of magnitude below
+// 2^22 to an integer, half to even (the sum's ulp is 1 under round-to-nearest).
+constexpr float MAGIC = 12582912.0f;
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float* p) { return __ldg(p); }
+};
+template <> struct Elem<uint16_t> {   // bf16 stored as raw bits
+    static __device__ __forceinline__ float load(const uint16_t* p) { return bf16_bits_to_f32(__ldg(p)); }
+};
+
+// Warp-wide lexicographic (loss, index) minimum; every lane ends with it.
+__device__ __forceinline__ void warp_argmin(float& L, int& idx) {
+#pragma unroll
+    for (int off = 16; off; off >>= 1) {
+        float Lo = __shfl_xor_sync(FULL, L, off);
+        int io = __shfl_xor_sync(FULL, idx, off);
+        if (Lo < L || (Lo == L && io < idx)) { L = Lo; idx = io; }
+    }
+}
+
+// Same over aligned groups of `width` lanes (width a power of two <= 32).
+__device__ __forceinline__ void group_argmin(float& L, int& idx, unsigned mask, int width) {
+    for (int off = width >> 1; off; off >>= 1) {
+        float Lo = __shfl_xor_sync(mask, L, off);
+        int io = __shfl_xor_sync(mask, idx, off);
+        if (Lo < L || (Lo == L && io < idx)) { L = Lo; idx = io; }
+    }
+}
+
+// Butterfly sum: every lane of the group ends with the bit-identical total
+// (each step adds the same pair of operands on both partner lanes).
+__device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width) {
+    for (int off = width >> 1; off; off >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, off));
+    return v;
+}
+
+__device__ __forceinline__ float warp_max_abs(float a, float b) {
+    unsigned u = max(__float_as_uint(fabsf(a)), __float_as_uint(fabsf(b)));
+    return __uint_as_float(__reduce_max_sync(FULL, u));
+}
+
+// Integer code of w under scale s: round half to even of the IEEE fp32
+// quotient w/s, clamped to [lo, hi]; scale 0 gives code 0.
+__device__ __forceinline__ float rtn_exact(float w, float s, float lo, float hi) {
+    if (s == 0.0f) return 0.0f;
+    float y = rintf(__fdiv_rn(w, s));
+    return fminf(fmaxf(y, lo), hi);
+}
+
+// E2M1 round-to-nearest-even with saturation of y >= 0, returned as its value
+// in {0, .5, 1, 1.5, 2, 3, 4, 6}.  The spacing of E2M1 values at y is half
+// the power of two at or below max(y, 1); adding and subtracting 1.5 * 2^22
+// times that power of two rounds y to a multiple of the spacing, half to even
+// (even multiples are exactly the even E2M1 codes), and min(., 6) saturates.
+__device__ __forceinline__ float e2m1_round(float y) {
+    unsigned e = __float_as_uint(y) & 0x7f800000u;
+    e = max(e, 0x3f800000u);
+    float C = __uint_as_float(e + 0x0b400000u);
+    float r = __fsub_rn(__fadd_rn(y, C), C);
+    return fminf(r, 6.0f);
+}
+
+// E2M1 magnitude code (0..7) of a value produced by e2m1_round.
+__device__ __forceinline__ int e2m1_mag_code(float v) {
+    return v < 2.0f ? static_cast<int>(v * 2.0f) : (v < 4.0f ? static_cast<int>(v) + 2 : (v < 5.0f ? 6 : 7));
+}
+
+// E2M1 magnitude of code 0..7: {0, .5, 1, 1.5, 2, 3, 4, 6}.
+__device__ __forceinline__ float e2m1_value(unsigned c) {
+    return c < 4u ? 0.5f * static_cast<float>(c) : (c < 6u ? static_cast<float>(c - 2u) : (c == 6u ? 4.0f : 6.0f));
+}
+
+// E4M3 (e4m3fn) value of a positive code 1..126 (0 for code 0).
+__host__ __device__ __forceinline__ float e4m3_value(int c) {
+    int e = (c >> 3) & 15, m = c & 7;
+    float v = (e == 0) ? ldexpf(static_cast<float>(m), -9) : ldexpf(1.0f + m * 0.125f, e - 7);
+    return v;
+}
+
+}  // namespace tq

@@ -1,0 +1,232 @@
+/*
+ * tq.h -- C ABI of the group-scale search library: imatrix-weighted search of
+ * per-group quantization scales (and integer zero-points), round-to-nearest,
+ * packing into int3-g64 / int4-g128 / NVFP4-g16, dequantization and the
+ * imatrix-weighted reconstruction error.  Every call runs hand-written CUDA
+ * kernels for NVIDIA B200 (sm_100a).
+ *
+ * Sources (web pages, cited by title and section):
+ *  [NeUQI]  "NeUQI Accuracy Validation" (intel/auto-round docs/neuqi_acc.md):
+ *           opening paragraph (asymmetric layers: joint (scale, integer
+ *           zero-point) search; symmetric layers: two-stage signed-scale search;
+ *           both weighted by the activation imatrix) and results bullet 2
+ *           ("64/32" grid).
+ *  [TT]     "Quantize on TT cards: CUDA-free GPTQ/LDLQ bfp4 pipeline" (tt-stack
+ *           issue #67): pipeline table step 1 (H = sum X^T X) and "Risks to
+ *           measure: Precision" (proxy error tr(E H E^T) / tr(W H W^T)).
+ *  [NVFP4]  "Nemotron-Cascade-2-30B-A3B-NVFP4" model card: Quantization Recipe
+ *           table (NVFP4, group size 16, MSE-calibrated static block scales).
+ *  [INT3]   "int3-g64 (fmt=5)" (colibri PR #168): Design, Layout bullet.
+ *
+ * Conventions shared by every call
+ *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller.
+ *    The library never allocates device memory; calls that need scratch take
+ *    a caller-provided workspace sized by the matching *_workspace_bytes().
+ *  - Streams: every call enqueues work on `stream` (NULL = legacy default
+ *    stream) and returns without synchronising.  Errors raised by kernels
+ *    after launch surface at the caller's next synchronisation.
+ *  - Errors: arguments are validated on the host before anything is
+ *    enqueued; a call that returns an error has enqueued nothing (except
+ *    TQ_ERR_CUDA, raised when a launch itself fails).  tq_last_error_string()
+ *    describes the last error of the calling thread.
+ *  - Layout: weights W are batches of n_mat row-major O x I matrices; groups
+ *    run along I (the input dimension), G = ceil(I / g) groups per row.  A
+ *    last group shorter than g is a tail group: only its real elements enter
+ *    maxima and losses, and its packed record is padded (see tq_pack_codes).
+ *    Per-group outputs (scales, zero-points, indices, losses) are dense
+ *    [n_mat][O][G]; packed records are dense in the same order.
+ *  - Alignment: tensor base pointers must be 16-byte aligned and row strides
+ *    (ld * element size) multiples of 16 bytes.
+ */
+#ifndef TQ_H
+#define TQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* tq_stream_t;
+
+typedef enum {
+    TQ_OK = 0,
+    TQ_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad sizes or strides */
+    TQ_ERR_UNSUPPORTED = 2,  /* a dtype/format/grid this build does not run   */
+    TQ_ERR_CUDA = 3          /* a kernel launch or CUDA runtime call failed   */
+} tq_status;
+
+typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
+
+typedef enum {
+    TQ_INT4_G128_ASYM = 4,   /* nibble codes q in [0,15], f32 scale, u8 zero per 128 weights */
+    TQ_INT3_G64_SYM = 5,     /* two bit-planes, v in [-4,3] as v+4, f32 scale per 64 weights  */
+    TQ_NVFP4_G16 = 16        /* E2M1 codes, E4M3 scale byte per 16 weights, f32 global scale   */
+} tq_format;
+
+/* A batch of n_mat matrices of rows x cols elements of `dtype`.
+ * Element (e, o, j) lives at ptr + (e * mat_stride + o * ld + j) elements. */
+typedef struct tq_mat {
+    const void* ptr;
+    int32_t dtype;       /* tq_dtype */
+    int32_t reserved;
+    int64_t n_mat;
+    int64_t rows;        /* O (or T tokens for activations) */
+    int64_t cols;        /* I */
+    int64_t ld;          /* >= cols */
+    int64_t mat_stride;  /* >= rows * ld, or 0 when n_mat == 1 */
+} tq_mat;
+
+/* Candidate grids ([NeUQI]; readings of the unspecified parts in brackets).
+ *  Symmetric int3: stage 1 = sym_n1 magnitude ratios r_k = fl32(lo + ((hi-lo)k)/(n1-1))
+ *    of max|w|/4, each with both signs: candidate 2k+sigma has scale
+ *    (1-2 sigma) fl32(r_k max|w|) / 4.  Stage 2 = sym_n2 ratios spread evenly over
+ *    [r_k* - d, r_k* + d], d = (hi-lo)/(n1-1), with the stage-1 winner's sign,
+ *    candidate index 2 n1 + i [reading: "refinements around the best"].
+ *  Asymmetric int4: scale s_k = fl32(fl32(f_k / 15) (wmax - wmin)),
+ *    f_k = lo + ((hi-lo)k)/(ns-1) [reading: range equal to the symmetric window];
+ *    zero-point z_i = rint(15 i / (nz - 1)) [reading of "32 integer zero-points
+ *    in [0,15]"]; candidate index nz k + i.
+ *  NVFP4: the fp4_window E4M3 codes nearest a/(6 g) (a = block max|w|,
+ *    g = global scale); candidate index = the E4M3 code. */
+typedef struct tq_search_params {
+    int32_t sym_n1;        /* 32 */
+    int32_t sym_n2;        /* 32 */
+    double  sym_lo;        /* 0.5 */
+    double  sym_hi;        /* 1.2 */
+    int32_t asym_n_scale;  /* 64 */
+    int32_t asym_n_zero;   /* 32 */
+    double  asym_lo;       /* 0.5 */
+    double  asym_hi;       /* 1.2 */
+    int32_t fp4_window;    /* 16 */
+    int32_t reserved;
+} tq_search_params;
+
+/* Fills the defaults above. */
+void tq_default_params(tq_search_params* p);
+
+/* Message of the calling thread's last error ("" if none). Never NULL. */
+const char* tq_last_error_string(void);
+
+/* Library version string, e.g. "tq 1.0 sm_100a". */
+const char* tq_version(void);
+
+/* Weights per group: 64, 128 or 16; 0 for an unknown format. */
+int64_t tq_group_size(int32_t fmt);
+
+/* Groups (= scales) of `rows` rows of `cols` weights: rows * ceil(cols / g). */
+int64_t tq_num_groups(int32_t fmt, int64_t rows, int64_t cols);
+
+/* Packed code bytes of `rows` rows of `cols` weights: int3 rows*G*24 ([INT3]
+ * Layout: 3.5 bits/weight with the f32 scale), int4 rows*G*64, NVFP4 rows*G*8.
+ * 0 for an unknown format. */
+size_t tq_packed_bytes(int32_t fmt, int64_t rows, int64_t cols);
+
+/* ------------------------------------------------------------------ imatrix
+ * m[e*m_stride + j] = alpha * sum_t X[e, t, j]^2 (+ m[...] if accumulate).
+ * With alpha = 1/T this is the activation imatrix of [NeUQI], the diagonal of
+ * H = sum X^T X over T ([TT] step 1).  X: bf16 or f32, [n_mat, T, I].
+ * m: f32 device array, m_stride >= I.  Sums are fp32 over short token runs
+ * folded into fp64, reduced across blocks in a fixed order (deterministic).
+ * workspace: device scratch of at least tq_imatrix_workspace_bytes() bytes
+ * (no alignment beyond 16 bytes; contents need no initialisation).
+ * accumulate != 0 adds to the existing m (token-sharded calibration). */
+size_t tq_imatrix_workspace_bytes(const tq_mat* X);
+tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
+                     void* workspace, size_t workspace_bytes, tq_stream_t stream);
+
+/* ------------------------------------------------------------------ amax
+ * amax[e] = max |W[e]| over matrix e (f32).  Used for the NVFP4 per-tensor
+ * global scale g = fl32(amax / (6 * 448)). */
+tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream);
+
+/* ------------------------------------------------------------------ search
+ * For every group (block) of every row of every matrix: pick the candidate of
+ * the format's grid (tq_search_params) with the smallest imatrix-weighted
+ * squared error L = sum_j m_j (w_j - what_j)^2, where the codes of each
+ * candidate are round-to-nearest (half to even) of the fp32 quotient w/s,
+ * clamped to the format's range ([NeUQI] opening paragraph; [NVFP4] recipe
+ * table for the E2M1 / E4M3 search).  Ties keep the lowest candidate index.
+ * Candidates are ranked in fp32; candidates within a relative 2^-15 of the
+ * best are re-ranked in fp64.
+ *
+ *  W:      bf16/f32 weights.  m: f32 imatrix of matrix e at m + e * m_stride
+ *          (m_stride = 0: one imatrix for every matrix), >= cols entries.
+ *  fmt:    tq_format.  params: NULL = tq_default_params.
+ *  scales: int3/int4: f32 [n_mat][O][G] (int3 scales carry the sign);
+ *          NVFP4: u8 E4M3 codes [n_mat][O][G].  Required.
+ *  zeros:  int4: u8 [n_mat][O][G], required; others must be NULL.
+ *  global_scale: NVFP4: f32 [n_mat], written with g = fl32(amax / 2688)
+ *          (computed by this call); others must be NULL.
+ *  cand_idx: optional int32 [n_mat][O][G]: chosen candidate index (int3:
+ *          2k+sigma or 2 n1 + i; int4: nz k + i; NVFP4: the E4M3 code), -1 for
+ *          a group with nothing to fit (all zero).
+ *  loss:   optional f32 [n_mat][O][G]: the chosen candidate's loss.
+ *  packed: optional u8 [n_mat * O * G * record bytes]: the chosen codes packed
+ *          as tq_pack would (round-to-nearest and packing fused into the
+ *          search).
+ * Grid limits of this build: sym_n1, sym_n2 in [2, 32]; asym_n_scale in
+ * [2, 64], asym_n_zero >= 16 (every integer zero-point 0..15 occurs);
+ * fp4_window in [1, 16].  Others return TQ_ERR_UNSUPPORTED. */
+tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_stride, int32_t fmt,
+                           const tq_search_params* params, void* scales, uint8_t* zeros,
+                           float* global_scale, int32_t* cand_idx, float* loss, uint8_t* packed,
+                           tq_stream_t stream);
+
+/* ------------------------------------------------------------------ pack
+ * Round-to-nearest of W with the given scales (and zero-points / global
+ * scale) and pack: bit-identical to the packed output of tq_search_groups for
+ * the same scales.  Arguments as tq_search_groups; global_scale is an INPUT
+ * here (f32 [n_mat]). */
+tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const uint8_t* zeros,
+                  const float* global_scale, uint8_t* packed, tq_stream_t stream);
+
+/* Pack integer codes: `codes` is dense [rows][cols] bytes (int3: int8 v in
+ * [-4,3]; int4: q in [0,15]; NVFP4: 4-bit E2M1 code, sign in bit 3).
+ * Records ([INT3] Layout): int3 = 24 bytes per 64 weights, u = v + 4, low
+ * plane bytes 0..15 with element i at byte i/4 bits 2(i%4), high plane bytes
+ * 16..23 with element i at bit i%8 of byte 16 + i/8.  int4 / NVFP4 = one byte
+ * per two weights, element 2k in the low nibble of byte k.  Tail positions:
+ * int3 v = 0, int4 q = zeros[group] (dequantizes to 0; zeros may be NULL for
+ * q = 0), NVFP4 code 0.  Codes outside the format's range are masked to its
+ * bit width. */
+tq_status tq_pack_codes(const uint8_t* codes, int32_t fmt, int64_t rows, int64_t cols,
+                        const uint8_t* zeros, uint8_t* packed, tq_stream_t stream);
+
+/* Inverse of tq_pack_codes for the real (non-tail) positions. */
+tq_status tq_unpack_codes(const uint8_t* packed, int32_t fmt, int64_t rows, int64_t cols,
+                          uint8_t* codes, tq_stream_t stream);
+
+/* ------------------------------------------------------------------ dequant
+ * What = s v (int3), s (q - z) (int4), fl32(fl32(g dec(e)) dec(c)) (NVFP4),
+ * each rounded once to fp32 (then to bf16, round-to-nearest-even, when
+ * out_dtype is TQ_BF16).  out: dense [n_mat][O][I] of out_dtype. */
+tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scales, const uint8_t* zeros,
+                     const float* global_scale, int64_t n_mat, int64_t O, int64_t I, void* out,
+                     int32_t out_dtype, tq_stream_t stream);
+
+/* ------------------------------------------------------------------ proxy error
+ * Per matrix e ([TT] "Risks to measure: Precision", H = diag(m)):
+ *   num[e] = sum_{o,j} m_j (W - What)^2 = tr(E H E^T),
+ *   den[e] = sum_{o,j} m_j W^2          = tr(W H W^T),
+ * with What the fp32 dequantized weights of `packed`.  fp64 outputs, fixed
+ * reduction order.  workspace: >= tq_proxy_workspace_bytes(); its contents
+ * need no initialisation. */
+size_t tq_proxy_workspace_bytes(const tq_mat* W, int32_t fmt);
+tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, const void* scales,
+                         const uint8_t* zeros, const float* global_scale, const float* m,
+                         int64_t m_stride, double* num, double* den, void* workspace,
+                         size_t workspace_bytes, tq_stream_t stream);
+
+/* ------------------------------------------------------------------ testing aid
+ * Synchronises `stream` and returns TQ_ERR_CUDA if it or an earlier kernel
+ * failed. */
+tq_status tq_sync(tq_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ_H */

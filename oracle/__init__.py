@@ -57,7 +57,7 @@ def lib():
             "orc_e4m3_decode": (f64, [i32]),
             "orc_e2m1_rne_mag": (i32, [f32]),
             "orc_nvfp4_global": (f32, [P, i64]),
-            "orc_nvfp4_window": (None, [f64, i32, P]),
+            "orc_nvfp4_window": (None, [f32, f32, i32, P]),
             "orc_nvfp4_loss": (f64, [P, P, i32, f32, P]),
             "orc_search_nvfp4_block": (i32, [P, P, i32, f32, i32, P, P]),
             "orc_search_sym_int3": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, i32, f64, f64,
@@ -78,6 +78,9 @@ def lib():
             "orc_proxy_error": (None, [P, P, i64, i64, P, P, P]),
             "orc_rowwise_int4": (None, [P, i64, i64, P]),
             "orc_num_threads": (i32, []),
+            "orc_loss_given_int3": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P]),
+            "orc_loss_given_int4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P, P]),
+            "orc_loss_given_nvfp4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -260,9 +263,10 @@ def e2m1_rne_mag(y: float) -> int:
     return lib().orc_e2m1_rne_mag(float(np.float32(y)))
 
 
-def nvfp4_window(t: float, window=16):
+def nvfp4_window(a: float, g: float, window=16):
+    """Window codes for block amax a under global scale g."""
     out = np.empty(window, np.int32)
-    lib().orc_nvfp4_window(float(t), window, _p(out))
+    lib().orc_nvfp4_window(float(np.float32(a)), float(np.float32(g)), window, _p(out))
     return out
 
 
@@ -362,6 +366,39 @@ def rowwise_int4(W) -> np.ndarray:
     W = _f32(W); I = W.shape[-1]; rows = W.size // I
     out = np.empty(W.shape, np.float32)
     lib().orc_rowwise_int4(_p(W), rows, I, _p(out))
+    return out
+
+
+def _batch(W, m):
+    W = _f32(W)
+    if W.ndim == 2:
+        W = W[None]
+    m = _f32(m)
+    E, O, I = W.shape
+    return W, m, E, O, I, (I if m.ndim == 2 else 0)
+
+
+def loss_given_int3(W, m, scales) -> np.ndarray:
+    """fp64 loss of given int3 scales for every group of W [n_mat, O, I]."""
+    W, m, E, O, I, ms = _batch(W, m)
+    out = np.empty((E, O, (I + 63) // 64), np.float64)
+    lib().orc_loss_given_int3(_p(W), E, O, I, I, O * I, _p(m), ms, _p(_f32(scales)), _p(out))
+    return out
+
+
+def loss_given_int4(W, m, scales, zeros) -> np.ndarray:
+    W, m, E, O, I, ms = _batch(W, m)
+    out = np.empty((E, O, (I + 127) // 128), np.float64)
+    lib().orc_loss_given_int4(_p(W), E, O, I, I, O * I, _p(m), ms, _p(_f32(scales)),
+                              _p(np.ascontiguousarray(zeros, np.uint8)), _p(out))
+    return out
+
+
+def loss_given_nvfp4(W, m, scale_codes, gscale) -> np.ndarray:
+    W, m, E, O, I, ms = _batch(W, m)
+    out = np.empty((E, O, (I + 15) // 16), np.float64)
+    lib().orc_loss_given_nvfp4(_p(W), E, O, I, I, O * I, _p(m), ms,
+                               _p(np.ascontiguousarray(scale_codes, np.uint8)), _p(_f32(gscale)), _p(out))
     return out
 
 

@@ -276,18 +276,23 @@ ORC_API float orc_nvfp4_global(const float* W, int64_t n)
 }
 
 /* The `window` positive finite E4M3 codes (1..126) whose values lie nearest
- * t, ties to the lower code, listed in ascending code order.  Done as the
- * plain definition: rank all 126 codes by (|dec(c) - t|, c) and keep the
- * first `window`.  Reading of "the 16 E4M3 codes nearest amax/6": t is the
- * block amax over 6 in units of the global scale. */
-ORC_API void orc_nvfp4_window(double t, int window, int* codes_out)
+ * t = a / (6 g), ties to the lower code, listed in ascending code order.
+ * Reading of "the 16 E4M3 codes nearest amax/6": t is the block amax over 6
+ * in units of the global scale.  Distances are compared as
+ * |6 g dec(c) - a| (the distance to t scaled by 6g > 0, which orders codes
+ * the same way); every term is exact in fp64 (6 g dec(c) has at most 31
+ * significant bits), so no rounding can reorder two codes.  Done as the plain
+ * definition: rank all 126 codes by (distance, code), keep the first
+ * `window`. */
+ORC_API void orc_nvfp4_window(float a, float g, int window, int* codes_out)
 {
     int chosen[127]; memset(chosen, 0, sizeof chosen);
+    double g6 = 6.0 * (double)g;
     for (int r = 0; r < window; ++r) {
         int best = -1; double bd = INFINITY;
         for (int c = 1; c <= 126; ++c) {
             if (chosen[c]) continue;
-            double d = fabs(orc_e4m3_decode(c) - t);
+            double d = fabs(g6 * orc_e4m3_decode(c) - (double)a);
             if (d < bd) { bd = d; best = c; }   /* strict: ties keep the lower code */
         }
         chosen[best] = 1;
@@ -326,9 +331,8 @@ ORC_API int orc_search_nvfp4_block(const float* w, const float* m, int n, float 
         if (c_out) memset(c_out, 0, (size_t)n);
         return -1;
     }
-    double t = (double)a / (6.0 * (double)g);
     int codes[126];
-    orc_nvfp4_window(t, window, codes);
+    orc_nvfp4_window(a, g, window, codes);
     int best = -1; double bestL = INFINITY;
     for (int r = 0; r < window; ++r) {
         float S = (float)((double)g * orc_e4m3_decode(codes[r]));
@@ -411,6 +415,50 @@ ORC_API void orc_search_nvfp4(const float* W, int64_t n_mat, int64_t O, int64_t 
         if (scale_codes) scale_codes[gi] = (uint8_t)(c < 0 ? 0 : c);
         if (idx) idx[gi] = c;
         if (loss) loss[gi] = L;
+    }
+}
+
+/* Loss of GIVEN per-group parameters (for re-evaluating another
+ * implementation's choices): the same per-group losses as above, over every
+ * group of [n_mat, O, I]. */
+ORC_API void orc_loss_given_int3(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                                 int64_t ms, const float* m, int64_t m_stride, const float* scales,
+                                 double* loss)
+{
+    const int64_t G = (I + 63) / 64;
+    #pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 64; int n = (int)((I - j0) < 64 ? (I - j0) : 64);
+        loss[gi] = orc_sym_loss(W + e * ms + o * ld + j0, m + e * m_stride + j0, n, scales[gi], NULL);
+    }
+}
+
+ORC_API void orc_loss_given_int4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                                 int64_t ms, const float* m, int64_t m_stride, const float* scales,
+                                 const uint8_t* zeros, double* loss)
+{
+    const int64_t G = (I + 127) / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 128; int n = (int)((I - j0) < 128 ? (I - j0) : 128);
+        loss[gi] = orc_asym_loss(W + e * ms + o * ld + j0, m + e * m_stride + j0, n, scales[gi],
+                                 zeros[gi], NULL);
+    }
+}
+
+ORC_API void orc_loss_given_nvfp4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
+                                  int64_t ms, const float* m, int64_t m_stride,
+                                  const uint8_t* scale_codes, const float* gscale, double* loss)
+{
+    const int64_t G = (I + 15) / 16;
+    #pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
+        int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
+        int64_t j0 = k * 16; int n = (int)((I - j0) < 16 ? (I - j0) : 16);
+        float S = (float)((double)gscale[e] * orc_e4m3_decode(scale_codes[gi]));
+        loss[gi] = orc_nvfp4_loss(W + e * ms + o * ld + j0, m + e * m_stride + j0, n, S, NULL);
     }
 }
 

@@ -1,0 +1,101 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol
+include/tq.h declares, and its host-side size/validation logic answers."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "tq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from group_scale_search_b200 import build
+    build.build()
+    import group_scale_search_b200 as g
+    g.lib()
+    return g
+
+
+def test_exports_every_declared_symbol(tq):
+    declared = _declared()
+    assert len(declared) >= 15
+    L = ctypes.CDLL(tq.lib_path())
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(tq.EXPORTS) == declared
+
+
+def test_library_targets_sm100a(tq):
+    assert "sm_100a" in tq.tq_version()
+
+
+def test_sizes(tq):
+    assert tq.tq_group_size(tq.INT3_G64_SYM) == 64
+    assert tq.tq_group_size(tq.INT4_G128_ASYM) == 128
+    assert tq.tq_group_size(tq.NVFP4_G16) == 16
+    assert tq.tq_group_size(99) == 0
+    # int3-g64: 24 bytes per 64 weights + f32 scale = 3.5 bits/weight
+    assert tq.tq_packed_bytes(tq.INT3_G64_SYM, 2048, 7168) == 2048 * 112 * 24
+    assert tq.tq_packed_bytes(tq.INT3_G64_SYM, 2048, 7208) == 2048 * 113 * 24
+    assert tq.tq_packed_bytes(tq.INT4_G128_ASYM, 4096, 4096) == 4096 * 32 * 64
+    assert tq.tq_packed_bytes(tq.NVFP4_G16, 1856, 2688) == 1856 * 168 * 8
+    assert tq.tq_num_groups(tq.NVFP4_G16, 3, 17) == 6
+
+
+def test_default_params(tq):
+    p = tq._Params()
+    tq.lib().tq_default_params(ctypes.byref(p))
+    assert (p.sym_n1, p.sym_n2, p.sym_lo, p.sym_hi) == (32, 32, 0.5, 1.2)
+    assert (p.asym_n_scale, p.asym_n_zero, p.asym_lo, p.asym_hi, p.fp4_window) == (64, 32, 0.5, 1.2, 16)
+
+
+def test_invalid_arguments_are_rejected_before_any_launch(tq):
+    L = tq.lib()
+    m = tq._Mat(None, 1, 0, 1, 4, 64, 64, 0)
+    p = tq._Params()
+    L.tq_default_params(ctypes.byref(p))
+    st = L.tq_search_groups(ctypes.byref(m), None, 0, tq.INT3_G64_SYM, ctypes.byref(p),
+                            None, None, None, None, None, None, None)
+    assert st == 1 and b"null" in L.tq_last_error_string()
+    fake = ctypes.c_void_p(0x1000)   # never dereferenced: validation fails first
+    m = tq._Mat(fake, 1, 0, 1, 4, 64, 32, 0)    # ld < cols
+    st = L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, None, fake, None, None,
+                            None, None, None, None)
+    assert st == 1 and b"ld" in L.tq_last_error_string()
+    m = tq._Mat(ctypes.c_void_p(0x1008), 1, 0, 1, 4, 64, 64, 0)    # misaligned
+    st = L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, None, fake, None, None,
+                            None, None, None, None)
+    assert st == 1 and b"aligned" in L.tq_last_error_string()
+    m = tq._Mat(fake, 7, 0, 1, 4, 64, 64, 0)    # unknown dtype
+    assert L.tq_amax(ctypes.byref(m), fake, None) == 2
+    m = tq._Mat(fake, 1, 0, 1, 4, 64, 64, 0)
+    assert L.tq_search_groups(ctypes.byref(m), fake, 0, 99, None, fake, None, None,
+                              None, None, None, None) == 2
+    # int4 needs zeros; others must not get them
+    assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT4_G128_ASYM, None, fake, None, None,
+                              None, None, None, None) == 1
+    assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, None, fake, fake, None,
+                              None, None, None, None) == 1
+    # unsupported grid sizes
+    p.sym_n1 = 40
+    assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, ctypes.byref(p), fake, None,
+                              None, None, None, None, None) == 2
+    # workspace too small
+    x = tq._Mat(fake, 0, 0, 1, 1024, 512, 512, 0)
+    need = L.tq_imatrix_workspace_bytes(ctypes.byref(x))
+    assert need > 0
+    assert L.tq_imatrix(ctypes.byref(x), fake, 512, ctypes.c_float(1.0), 0, fake, need - 8, None) == 1
+
+
+def test_binding_refuses_cpu_tensors(tq):
+    import torch
+    with pytest.raises(tq.TQError):
+        tq.tq_imatrix(torch.zeros(8, 64))

@@ -315,15 +315,25 @@ def test_asym_search_vs_brute_force(orc):
 
 
 def test_nvfp4_window_is_sixteen_nearest(orc):
-    vals = np.array([orc.e4m3_decode(cd) for cd in range(1, 127)])
-    codes = np.arange(1, 127)
+    """The window = the 16 codes nearest a/(6g) by exact rational distance,
+    ties to the lower code (brute force with fractions.Fraction)."""
+    from fractions import Fraction
+    vals = [Fraction(orc.e4m3_decode(cd)) for cd in range(1, 127)]
     rng = _rng(13)
-    ts = np.concatenate([rng.uniform(0, 460, 500), np.exp(rng.uniform(-9, 6.2, 500)),
-                         vals[:40], (vals[:-1] + vals[1:]) / 2])
-    for t in ts:
-        order = np.lexsort((codes, np.abs(vals - t)))  # by distance, then by code
-        expect = np.sort(codes[order[:16]])
-        assert np.array_equal(orc.nvfp4_window(t), expect), t
+    cases = []
+    for _ in range(300):
+        g = np.float32(rng.uniform(1e-5, 1e-3))
+        cases.append((np.float32(np.float64(g) * 6 * rng.uniform(0, 460)), g))
+        cases.append((np.float32(np.float64(g) * 6 * np.exp(rng.uniform(-9, 6.2))), g))
+    g = np.float32(2.0 ** -10)
+    for i in range(40):   # values and exact midpoints of codes (in units of 6g)
+        cases.append((np.float32(6 * 2.0 ** -10 * float(vals[i])), g))
+        cases.append((np.float32(6 * 2.0 ** -10 * float((vals[i] + vals[i + 1]) / 2)), g))
+    for a, g in cases:
+        t = Fraction(float(a)) / (6 * Fraction(float(g)))
+        order = sorted(range(126), key=lambda i: (abs(vals[i] - t), i))
+        expect = sorted(i + 1 for i in order[:16])
+        assert orc.nvfp4_window(a, g).tolist() == expect, (a, g)
 
 
 def test_nvfp4_search_vs_brute_force(orc):
@@ -335,8 +345,7 @@ def test_nvfp4_search_vs_brute_force(orc):
         g = np.float32(np.float32(np.abs(w).max() * rng.uniform(1, 3)) / np.float32(2688))
         e, L, c = orc.nvfp4_block(w, m, g)
         a = np.abs(w).max()
-        t = np.float64(a) / (6.0 * np.float64(g))
-        win = orc.nvfp4_window(t)
+        win = orc.nvfp4_window(a, g)
         bestL, beste = np.inf, None
         for cd in win:
             S = np.float32(np.float64(g) * orc.e4m3_decode(cd))
