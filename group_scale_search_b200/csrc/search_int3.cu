@@ -171,6 +171,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             if (LN < LP) { L = LN; bi = 2 * lane + 1; } else { L = LP; bi = 2 * lane; }
         }
         warp_argmin(L, bi);
+        if (bi < 0 || bi >= 2 * a.n1) bi = 0;   // every loss non-finite: keep index 0
         int b1 = bi;
         bool have64 = false;
         double L1d = 0.0;
@@ -249,6 +250,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             bf = b1; lossf = have64 ? static_cast<float>(L1d) : L1f;
         }
 
+        if (bf < 0 || bf >= 2 * a.n1 + a.n2) bf = b1;
         float sfin;
         if (bf < 2 * a.n1) {
             const float sk = __shfl_sync(FULL, s1, bf >> 1);

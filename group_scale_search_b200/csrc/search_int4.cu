@@ -221,6 +221,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             lossf = static_cast<float>(best);
         }
 
+        if (bi < 0 || bi >= a.nz * a.ns) bi = a.zfirst[0];   // every loss non-finite
         const int kb = bi / a.nz;
         const int zb = a.zval[bi - kb * a.nz];
         const float sfin = __fmul_rn(a.c[kb], R);

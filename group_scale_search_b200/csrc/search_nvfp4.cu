@@ -160,6 +160,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             }
         }
         if (need) { ci = bcode; lossf = static_cast<float>(best); }
+        if (!degen && (ci < lo || ci >= lo + Wn)) ci = lo;   // every loss non-finite
 
         // ---- outputs and exact RTN + pack
         const int src = (half << 4) + (degen ? 0 : (ci - lo));

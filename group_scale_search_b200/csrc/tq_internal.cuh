@@ -61,7 +61,9 @@ template <> struct Elem<uint16_t> {   // bf16 stored as raw bits
 };
 
 // Warp-wide lexicographic (loss, index) minimum; every lane ends with it.
+// NaN losses rank as +inf so every lane agrees on the result.
 __device__ __forceinline__ void warp_argmin(float& L, int& idx) {
+    if (L != L) L = __int_as_float(0x7f800000);
 #pragma unroll
     for (int off = 16; off; off >>= 1) {
         float Lo = __shfl_xor_sync(FULL, L, off);
@@ -72,6 +74,7 @@ __device__ __forceinline__ void warp_argmin(float& L, int& idx) {
 
 // Same over aligned groups of `width` lanes (width a power of two <= 32).
 __device__ __forceinline__ void group_argmin(float& L, int& idx, unsigned mask, int width) {
+    if (L != L) L = __int_as_float(0x7f800000);
     for (int off = width >> 1; off; off >>= 1) {
         float Lo = __shfl_xor_sync(mask, L, off);
         int io = __shfl_xor_sync(mask, idx, off);
