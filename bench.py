@@ -252,8 +252,8 @@ def _oracle_unit(oracle, wl, u, rows):
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="c1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")

@@ -99,7 +99,7 @@ class SearchResult:
     zeros: Optional[torch.Tensor]         # u8 [n_mat, O, G] (int4)
     global_scale: Optional[torch.Tensor]  # f32 [n_mat] (NVFP4)
     cand_idx: Optional[torch.Tensor]      # int32 [n_mat, O, G]
-    loss: Optional[torch.Tensor]          # f32 [n_mat, O, G]
+    loss: Optional[torch.Tensor]          # f64 [n_mat, O, G]
     packed: Optional[torch.Tensor]        # u8 [n_mat * O * G * record bytes]
 
 
@@ -265,7 +265,7 @@ def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optiona
             zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt == INT4_G128_ASYM else None,
             global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
             cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
-            loss=torch.empty((E, O, G), dtype=torch.float32, device=dev) if want_loss else None,
+            loss=torch.empty((E, O, G), dtype=torch.float64, device=dev) if want_loss else None,
             packed=torch.empty(tq_packed_bytes(fmt, E * O, I), dtype=torch.uint8, device=dev) if pack else None,
         )
     p = (params or SearchParams())._c()

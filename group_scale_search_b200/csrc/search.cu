@@ -4,12 +4,12 @@
 
 namespace tq {
 tq_status launch_search_int3(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
-                             float* scales, int32_t* idx, float* loss, uint8_t* packed, cudaStream_t st);
+                             float* scales, int32_t* idx, double* loss, uint8_t* packed, cudaStream_t st);
 tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
-                             float* scales, uint8_t* zeros, int32_t* idx, float* loss, uint8_t* packed,
+                             float* scales, uint8_t* zeros, int32_t* idx, double* loss, uint8_t* packed,
                              cudaStream_t st);
 tq_status launch_search_nvfp4(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
-                              uint8_t* scales, float* gscale, int32_t* idx, float* loss, uint8_t* packed,
+                              uint8_t* scales, float* gscale, int32_t* idx, double* loss, uint8_t* packed,
                               cudaStream_t st);
 }  // namespace tq
 
@@ -17,7 +17,7 @@ using namespace tq;
 
 TQ_API tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_stride, int32_t fmt,
                                   const tq_search_params* params, void* scales, uint8_t* zeros,
-                                  float* global_scale, int32_t* cand_idx, float* loss, uint8_t* packed,
+                                  float* global_scale, int32_t* cand_idx, double* loss, uint8_t* packed,
                                   tq_stream_t stream) {
     clear_error();
     tq_status s = check_mat(W, "tq_search_groups W");

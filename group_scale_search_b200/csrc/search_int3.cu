@@ -36,7 +36,7 @@ struct SymArgs {
     int64_t m_stride;
     float* scales;
     int32_t* idx;
-    float* loss;
+    double* loss;
     uint8_t* packed;
     int n1, n2;
     float r_lo;          // smallest ratio of either stage
@@ -120,16 +120,25 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             if (lane == 0) {
                 a.scales[gid] = 0.f;
                 if (a.idx) a.idx[gid] = -1;
-                if (a.loss) a.loss[gid] = 0.f;
+                if (a.loss) a.loss[gid] = 0.0;
             }
             if (rec) pack_int3_record(4u, 4u, lane, rec);
             continue;
         }
 
+        // ---- fp32 ranking works on w, m scaled by exact powers of two
+        const float pw = pow2_inv_binade(M);
+        const float mmax = warp_max_abs(m0, m1);
+        const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
+        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
+        const float Ms = __fmul_rn(M, pw);
+        const float x0 = __fmul_rn(w0, pw), x1 = __fmul_rn(w1, pw);
+        const float n0 = __fmul_rn(m0, pm), n1v = __fmul_rn(m1, pm);
+
         // ---- split elements: small ones cannot be clamped by any candidate
-        const float s_lo = __fmul_rn(__fmul_rn(a.r_lo, M), 0.25f);
+        const float s_lo = __fmul_rn(__fmul_rn(a.r_lo, Ms), 0.25f);
         const float thr = __fmul_rn(3.49f, s_lo);
-        const bool sm0 = v0 && fabsf(w0) < thr, sm1 = v1 && fabsf(w1) < thr;
+        const bool sm0 = v0 && fabsf(x0) < thr, sm1 = v1 && fabsf(x1) < thr;
         const bool lg0 = v0 && !sm0, lg1 = v1 && !sm1;
         const unsigned bs0 = __ballot_sync(FULL, sm0), bs1 = __ballot_sync(FULL, sm1);
         const unsigned bl0 = __ballot_sync(FULL, lg0), bl1 = __ballot_sync(FULL, lg1);
@@ -137,10 +146,10 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const int nl0 = __popc(bl0), nl = nl0 + __popc(bl1);
         const int ns_pad = (ns + 3) & ~3, nl_pad = (nl + 1) & ~1;
         __syncwarp();   // previous group's readers are done with the lists
-        if (sm0) small[__popc(bs0 & lt)] = make_float2(w0, m0);
-        if (sm1) small[ns0 + __popc(bs1 & lt)] = make_float2(w1, m1);
-        if (lg0) large[__popc(bl0 & lt)] = make_float2(w0, m0);
-        if (lg1) large[nl0 + __popc(bl1 & lt)] = make_float2(w1, m1);
+        if (sm0) small[__popc(bs0 & lt)] = make_float2(x0, n0);
+        if (sm1) small[ns0 + __popc(bs1 & lt)] = make_float2(x1, n1v);
+        if (lg0) large[__popc(bl0 & lt)] = make_float2(x0, n0);
+        if (lg1) large[nl0 + __popc(bl1 & lt)] = make_float2(x1, n1v);
         if (lane < ns_pad - ns) small[ns + lane] = make_float2(0.f, 0.f);   // zero pairs add exactly 0
         if (lane < nl_pad - nl) large[nl + lane] = make_float2(0.f, 0.f);
         __syncwarp();
@@ -148,7 +157,8 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float4* lp = reinterpret_cast<const float4*>(large);
 
         // ---- stage 1: lane = magnitude, both signs
-        const float s1 = __fmul_rn(__fmul_rn(r1v, M), 0.25f);
+        const float s1 = __fmul_rn(__fmul_rn(r1v, Ms), 0.25f);    // scaled candidate
+        const float s1o = __fmul_rn(__fmul_rn(r1v, M), 0.25f);    // the candidate itself
         const float i1 = __frcp_rn(s1);
         float accC = 0.f, accP = 0.f, accN = 0.f;
         for (int j = 0; j < ns_pad; j += 4) {
@@ -186,7 +196,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
                     const int kp = mpos ? __ffs(mpos) - 1 : 64, kn = mneg ? __ffs(mneg) - 1 : 64;
                     int kk, sg;
                     if (kp <= kn) { kk = kp; sg = 0; mpos &= mpos - 1; } else { kk = kn; sg = 1; mneg &= mneg - 1; }
-                    const float sk = __shfl_sync(FULL, s1, kk);
+                    const float sk = __shfl_sync(FULL, s1o, kk);
                     const double Ld = loss64_int3(w0, m0, w1, m1, sg ? -sk : sk);
                     if (Ld < best) { best = Ld; bidx = 2 * kk + sg; }
                 }
@@ -197,7 +207,8 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         // ---- stage 2: lane = refinement i around magnitude k*, sign of the winner
         const int ks = b1 >> 1, sg = b1 & 1;
         const float r2v = r2s[ks * 32 + (act2 ? lane : 0)];
-        const float s2 = __fmul_rn(__fmul_rn(r2v, M), 0.25f);
+        const float s2 = __fmul_rn(__fmul_rn(r2v, Ms), 0.25f);
+        const float s2o = __fmul_rn(__fmul_rn(r2v, M), 0.25f);
         const float i2 = __frcp_rn(s2);
         const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
         float acc2 = 0.f;
@@ -224,13 +235,13 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const bool inc_in = L1f <= thr2;
         unsigned c2 = __ballot_sync(FULL, act2 && L2 <= thr2);
         int bf;
-        float lossf;
+        double lossd;
         if (static_cast<int>(inc_in) + __popc(c2) > 1) {   // near tie: decide in fp64
             double best = __longlong_as_double(0x7ff0000000000000ll);
             int bidx = b2;
             if (inc_in) {
                 if (!have64) {
-                    const float sk = __shfl_sync(FULL, s1, ks);
+                    const float sk = __shfl_sync(FULL, s1o, ks);
                     L1d = loss64_int3(w0, m0, w1, m1, sg ? -sk : sk);
                 }
                 best = L1d; bidx = b1;
@@ -238,31 +249,31 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             while (c2) {
                 const int i = __ffs(c2) - 1;
                 c2 &= c2 - 1;
-                const float si = __shfl_sync(FULL, s2, i);
+                const float si = __shfl_sync(FULL, s2o, i);
                 const double Ld = loss64_int3(w0, m0, w1, m1, sg ? -si : si);
                 if (Ld < best) { best = Ld; bidx = 2 * a.n1 + i; }
             }
             bf = bidx;
-            lossf = static_cast<float>(best);
+            lossd = best;
         } else if (L2m < L1f) {
-            bf = b2; lossf = L2m;
+            bf = b2; lossd = static_cast<double>(L2m) * back;
         } else {
-            bf = b1; lossf = have64 ? static_cast<float>(L1d) : L1f;
+            bf = b1; lossd = have64 ? L1d : static_cast<double>(L1f) * back;
         }
 
         if (bf < 0 || bf >= 2 * a.n1 + a.n2) bf = b1;
         float sfin;
         if (bf < 2 * a.n1) {
-            const float sk = __shfl_sync(FULL, s1, bf >> 1);
+            const float sk = __shfl_sync(FULL, s1o, bf >> 1);
             sfin = (bf & 1) ? -sk : sk;
         } else {
-            const float si = __shfl_sync(FULL, s2, bf - 2 * a.n1);
+            const float si = __shfl_sync(FULL, s2o, bf - 2 * a.n1);
             sfin = sg ? -si : si;
         }
         if (lane == 0) {
             a.scales[gid] = sfin;
             if (a.idx) a.idx[gid] = bf;
-            if (a.loss) a.loss[gid] = lossf;
+            if (a.loss) a.loss[gid] = lossd;
         }
         if (rec) {
             const unsigned u0 = static_cast<unsigned>(static_cast<int>(rtn_exact(w0, sfin, -4.f, 3.f)) + 4);
@@ -275,7 +286,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
 // Host side: candidate ratio tables from their definitions (fp64, rounded
 // once to fp32), then one persistent launch.
 tq_status launch_search_int3(const tq_mat* W, const float* m, int64_t m_stride,
-                             const tq_search_params* p, float* scales, int32_t* idx, float* loss,
+                             const tq_search_params* p, float* scales, int32_t* idx, double* loss,
                              uint8_t* packed, cudaStream_t st) {
     if (p->sym_n1 < 2 || p->sym_n1 > 32 || p->sym_n2 < 2 || p->sym_n2 > 32)
         return set_error(TQ_ERR_UNSUPPORTED, "int3 search: sym_n1 and sym_n2 must be in [2, 32]");

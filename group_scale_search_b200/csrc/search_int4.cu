@@ -35,7 +35,7 @@ struct AsymArgs {
     float* scales;
     uint8_t* zeros;
     int32_t* idx;
-    float* loss;
+    double* loss;
     uint8_t* packed;
     int ns, nz;
     int zfirst[16];      // lowest i with z_i = z
@@ -140,7 +140,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                 if (lane == 0) {
                     a.scales[gid] = 0.f; a.zeros[gid] = 0;
                     if (a.idx) a.idx[gid] = -1;
-                    if (a.loss) a.loss[gid] = 0.f;
+                    if (a.loss) a.loss[gid] = 0.0;
                 }
                 if (rec) { const unsigned q0[4] = {0u, 0u, 0u, 0u}; pack_int4_lane(q0, lane, rec); }
                 continue;
@@ -148,12 +148,23 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             R = fabsf(wmax);
         }
 
+        // fp32 ranking works on w, m scaled by exact powers of two
+        const float pw = pow2_inv_binade(fmaxf(fabsf(wmin), fabsf(wmax)));
+        float mloc = 0.f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) mloc = fmaxf(mloc, fabsf(mv[i]));
+        const float mmax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(mloc)));
+        const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
+        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
+        const float Rs = __fmul_rn(R, pw);
         __syncwarp();
 #pragma unroll
-        for (int i = 0; i < 4; ++i) list[4 * lane + i] = make_float2(w[i], mv[i]);   // tail: (0, 0)
+        for (int i = 0; i < 4; ++i)   // tail: (0, 0)
+            list[4 * lane + i] = make_float2(__fmul_rn(w[i], pw), __fmul_rn(mv[i], pm));
         __syncwarp();
 
-        const float sA = __fmul_rn(cA, R), sB = __fmul_rn(cB, R);
+        const float sA = __fmul_rn(cA, Rs), sB = __fmul_rn(cB, Rs);
+        const float sAo = __fmul_rn(cA, R), sBo = __fmul_rn(cB, R);
         const float iA = __frcp_rn(sA), iB = __frcp_rn(sB);
         float accA[16], accB[16];
 #pragma unroll
@@ -197,7 +208,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             if (actB && accB[z] <= thr) wm |= 1u << (16 + z);
         }
         const int cnt = static_cast<int>(__reduce_add_sync(FULL, static_cast<unsigned>(__popc(wm))));
-        float lossf = L;
+        double lossd = static_cast<double>(L) * back;
         if (cnt > 1) {   // near tie: decide in fp64, candidates in index order
             double best = __longlong_as_double(0x7ff0000000000000ll);
             int bidx = bi;
@@ -208,7 +219,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                     ls &= ls - 1;
                     unsigned zm = __shfl_sync(FULL, wm, l2);
                     zm = part ? (zm >> 16) : (zm & 0xffffu);
-                    const float sc = __shfl_sync(FULL, part ? sB : sA, l2);
+                    const float sc = __shfl_sync(FULL, part ? sBo : sAo, l2);
                     while (zm) {
                         const int z = __ffs(zm) - 1;
                         zm &= zm - 1;
@@ -218,7 +229,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                 }
             }
             bi = bidx;
-            lossf = static_cast<float>(best);
+            lossd = best;
         }
 
         if (bi < 0 || bi >= a.nz * a.ns) bi = a.zfirst[0];   // every loss non-finite
@@ -229,7 +240,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             a.scales[gid] = sfin;
             a.zeros[gid] = static_cast<uint8_t>(zb);
             if (a.idx) a.idx[gid] = bi;
-            if (a.loss) a.loss[gid] = lossf;
+            if (a.loss) a.loss[gid] = lossd;
         }
         if (rec) {
             unsigned q[4];
@@ -246,7 +257,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
 
 tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
                              const tq_search_params* p, float* scales, uint8_t* zeros, int32_t* idx,
-                             float* loss, uint8_t* packed, cudaStream_t st) {
+                             double* loss, uint8_t* packed, cudaStream_t st) {
     if (p->asym_n_scale < 2 || p->asym_n_scale > 64)
         return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_scale must be in [2, 64]");
     if (p->asym_n_zero < 16 || p->asym_n_zero > 64)

@@ -32,7 +32,7 @@ struct Fp4Args {
     const float* g;        // per-matrix global scale
     uint8_t* scales;
     int32_t* idx;
-    float* loss;
+    double* loss;
     uint8_t* packed;
     int window;
 };
@@ -99,8 +99,15 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
         const float g = vb ? __ldg(a.g + e) : 0.f;
         const bool degen = (amax == 0.f) || (g == 0.f);
 
+        // fp32 ranking works on |w|, m scaled by exact powers of two
+        const float pw = amax > 0.f ? pow2_inv_binade(amax) : 1.f;
+        float mmax = fabsf(mv);
+#pragma unroll
+        for (int off = 8; off; off >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(FULL, mmax, off));
+        const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
+        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
         __syncwarp();
-        blk[wid][half][hl] = make_float2(aw, mv);
+        blk[wid][half][hl] = make_float2(__fmul_rn(aw, pw), __fmul_rn(mv, pm));
         __syncwarp();
 
         // ---- window: first lo with d(lo) <= d(lo + Wn), d(c) = |6 g dec(c) - a| (exact in fp64)
@@ -120,20 +127,21 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
         // ---- candidate loop: lane hl = code lo + hl
         const bool act = hl < Wn;
         const int code = lo + (act ? hl : 0);
-        const float S = __fmul_rn(g, dec[code]);
-        const float invS = __frcp_rn(S);
+        const float S = __fmul_rn(g, dec[code]);       // the candidate block scale
+        const float Ss = __fmul_rn(S, pw);               // scaled like the block
+        const float invS = __frcp_rn(Ss);
         float acc = 0.f;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 p = mine4[j];
             {
                 const float y = e2m1_round(__fmul_rn(p.x, invS));
-                const float er = __fmaf_rn(-S, y, p.x);
+                const float er = __fmaf_rn(-Ss, y, p.x);
                 acc = __fmaf_rn(__fmul_rn(p.y, er), er, acc);
             }
             {
                 const float y = e2m1_round(__fmul_rn(p.z, invS));
-                const float er = __fmaf_rn(-S, y, p.z);
+                const float er = __fmaf_rn(-Ss, y, p.z);
                 acc = __fmaf_rn(__fmul_rn(p.w, er), er, acc);
             }
         }
@@ -143,7 +151,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
         group_argmin(L, ci, FULL, 16);
         const float thr = __fmaf_rn(L, FWIN, L);
         unsigned win = (__ballot_sync(FULL, act && !degen && Lmine <= thr) & hbits) >> (16 * half);
-        float lossf = L;
+        double lossd = static_cast<double>(L) * back;
         // near ties: both halves walk their in-window candidates in code order
         int nwin = __popc(win);
         const bool need = nwin > 1;
@@ -159,7 +167,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
                 todo &= todo - 1;
             }
         }
-        if (need) { ci = bcode; lossf = static_cast<float>(best); }
+        if (need) { ci = bcode; lossd = best; }
         if (!degen && (ci < lo || ci >= lo + Wn)) ci = lo;   // every loss non-finite
 
         // ---- outputs and exact RTN + pack
@@ -178,7 +186,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
         if (vb && hl == 0) {
             a.scales[bid] = degen ? 0 : static_cast<uint8_t>(ci);
             if (a.idx) a.idx[bid] = degen ? -1 : ci;
-            if (a.loss) a.loss[bid] = degen ? static_cast<float>(dl) : lossf;
+            if (a.loss) a.loss[bid] = degen ? dl : lossd;
         }
         if (a.packed) {
             unsigned v = (c4 & 15u) << (4u * static_cast<unsigned>(hl & 7));
@@ -200,7 +208,7 @@ tq_status launch_amax(const tq_mat* W, float* amax, cudaStream_t st);   // imatr
 
 tq_status launch_search_nvfp4(const tq_mat* W, const float* m, int64_t m_stride,
                               const tq_search_params* p, uint8_t* scales, float* gscale, int32_t* idx,
-                              float* loss, uint8_t* packed, cudaStream_t st) {
+                              double* loss, uint8_t* packed, cudaStream_t st) {
     if (p->fp4_window < 1 || p->fp4_window > 16)
         return set_error(TQ_ERR_UNSUPPORTED, "nvfp4 search: fp4_window must be in [1, 16]");
     tq_status s = launch_amax(W, gscale, st);

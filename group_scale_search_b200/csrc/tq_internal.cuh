@@ -89,6 +89,17 @@ __device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width
     return v;
 }
 
+// 2^-e for the binade e of x > 0 (x * pow2_inv_binade(x) lies in [1, 2) for
+// normal x; subnormal x are scaled by 2^126).  Multiplying by it is exact for
+// normal results, so codes and candidate scales are unchanged and losses
+// scale by exact powers of two: the fp32 ranking works on values of order one
+// whatever the group's magnitude (it cannot underflow or overflow).
+__device__ __forceinline__ float pow2_inv_binade(float x) {
+    int E = static_cast<int>((__float_as_uint(x) >> 23) & 255u);
+    E = min(max(E, 1), 253);
+    return __uint_as_float(static_cast<unsigned>(254 - E) << 23);
+}
+
 __device__ __forceinline__ float warp_max_abs(float a, float b) {
     unsigned u = max(__float_as_uint(fabsf(a)), __float_as_uint(fabsf(b)));
     return __uint_as_float(__reduce_max_sync(FULL, u));

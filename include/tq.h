@@ -149,8 +149,10 @@ tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream);
  * candidate are round-to-nearest (half to even) of the fp32 quotient w/s,
  * clamped to the format's range ([NeUQI] opening paragraph; [NVFP4] recipe
  * table for the E2M1 / E4M3 search).  Ties keep the lowest candidate index.
- * Candidates are ranked in fp32; candidates within a relative 2^-15 of the
- * best are re-ranked in fp64.
+ * Candidates are ranked in fp32 on the group's weights and imatrix scaled by
+ * exact powers of two (so magnitudes never under- or overflow); candidates
+ * within a relative 2^-15 of the best are re-ranked in fp64 with codes from
+ * the IEEE quotient, which reproduces the definition's choice.
  *
  *  W:      bf16/f32 weights.  m: f32 imatrix of matrix e at m + e * m_stride
  *          (m_stride = 0: one imatrix for every matrix), >= cols entries.
@@ -163,7 +165,8 @@ tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream);
  *  cand_idx: optional int32 [n_mat][O][G]: chosen candidate index (int3:
  *          2k+sigma or 2 n1 + i; int4: nz k + i; NVFP4: the E4M3 code), -1 for
  *          a group with nothing to fit (all zero).
- *  loss:   optional f32 [n_mat][O][G]: the chosen candidate's loss.
+ *  loss:   optional f64 [n_mat][O][G]: the chosen candidate's loss (from the
+ *          fp32 ranking, or its fp64 value when a near tie was re-ranked).
  *  packed: optional u8 [n_mat * O * G * record bytes]: the chosen codes packed
  *          as tq_pack would (round-to-nearest and packing fused into the
  *          search).
@@ -172,7 +175,7 @@ tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream);
  * fp4_window in [1, 16].  Others return TQ_ERR_UNSUPPORTED. */
 tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_stride, int32_t fmt,
                            const tq_search_params* params, void* scales, uint8_t* zeros,
-                           float* global_scale, int32_t* cand_idx, float* loss, uint8_t* packed,
+                           float* global_scale, int32_t* cand_idx, double* loss, uint8_t* packed,
                            tq_stream_t stream);
 
 /* ------------------------------------------------------------------ pack
