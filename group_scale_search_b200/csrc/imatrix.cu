@@ -48,7 +48,7 @@ inline ImGeom im_geometry(const tq_mat* X) {
     g.col_tiles = (X->cols + 32 * vec - 1) / (32 * vec);
     const int64_t base = g.col_tiles * X->n_mat;
     int64_t s = (IM_TARGET_BLOCKS + base - 1) / base;
-    const int64_t max_s = (X->rows + 255) / 256;   // at least 256 tokens per slice
+    const int64_t max_s = (X->rows + 63) / 64;   // at least 64 tokens per slice
     if (s > max_s) s = max_s;
     if (s < 1) s = 1;
     g.tokens_per_slice = (X->rows + s - 1) / s;

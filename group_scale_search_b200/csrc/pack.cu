@@ -190,25 +190,31 @@ __device__ __forceinline__ void store16(O* dst, const float v[16], bool vec_ok, 
     }
 }
 
+// Grid: x = 256-chunk column tiles of a row (a chunk = 16 weights of one
+// group), y = row slices, z = matrices; each thread keeps its chunk column and
+// walks the rows of its slice (no integer division in the loop).
 template <typename O>
-__global__ void k_dequant(const uint8_t* __restrict__ packed, int fmt, const void* scales,
-                          const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
-                          int64_t n_mat, int64_t Orows, int64_t I, O* __restrict__ out) {
-    const int g = fmt == TQ_INT3_G64_SYM ? 64 : (fmt == TQ_INT4_G128_ASYM ? 128 : 16);
-    const int parts = g / 16;
-    const int64_t G = (I + g - 1) / g;
-    const int64_t units = n_mat * Orows * G * parts;
+__global__ void __launch_bounds__(256)
+k_dequant(const uint8_t* __restrict__ packed, int fmt, const void* scales, const uint8_t* __restrict__ zeros,
+          const float* __restrict__ gs, int64_t Orows, int64_t I, int64_t rows_per_slice, O* __restrict__ out) {
+    const int lg = fmt == TQ_INT3_G64_SYM ? 2 : (fmt == TQ_INT4_G128_ASYM ? 3 : 0);   // log2(chunks per group)
+    const int64_t G = (I + (16 << lg) - 1) >> (4 + lg);
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+    const int64_t C = (I + 15) >> 4;
+    if (c >= C) return;
+    const int64_t k = c >> lg;
+    const int part = static_cast<int>(c & ((1 << lg) - 1));
+    const int64_t e = blockIdx.z;
+    const int64_t j = c << 4;
+    const int nvalid = static_cast<int>(min(static_cast<int64_t>(16), I - j));
     const bool vec_ok = ((I * static_cast<int64_t>(sizeof(O))) % 16) == 0;
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < units;
-         u += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t gid = u / parts;
-        const int part = static_cast<int>(u - gid * parts);
-        const int64_t row = gid / G, k = gid - row * G;
-        const int64_t j = k * g + part * 16;
-        if (j >= I) continue;
+    const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rows_per_slice;
+    const int64_t o1 = min(Orows, o0 + rows_per_slice);
+    for (int64_t o = o0; o < o1; ++o) {
+        const int64_t row = e * Orows + o;
         float v[16];
-        dq_unit(fmt, packed, scales, zeros, gs, Orows * G, gid, part, v);
-        store16<O>(out + row * I + j, v, vec_ok, static_cast<int>(min(static_cast<int64_t>(16), I - j)));
+        dq_unit(fmt, packed, scales, zeros, gs, Orows * G, row * G + k, part, v);
+        store16<O>(out + row * I + j, v, vec_ok, nvalid);
     }
 }
 
@@ -290,15 +296,19 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_dequant: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant: NVFP4 needs global_scale");
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant: out dtype %d", out_dtype);
-    const int64_t g = group_of(fmt);
-    const int64_t units = n_mat * O * ((I + g - 1) / g) * (g / 16);
-    const int grid = static_cast<int>(min((units + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
+    const int64_t C = (I + 15) / 16;
+    const int64_t cblocks = (C + 255) / 256;
+    int64_t slices = (4 * static_cast<int64_t>(num_sms()) + cblocks * n_mat - 1) / (cblocks * n_mat);
+    slices = max(static_cast<int64_t>(1), min(slices, O));
+    const int64_t rps = (O + slices - 1) / slices;
+    slices = (O + rps - 1) / rps;
+    const dim3 grid(static_cast<unsigned>(cblocks), static_cast<unsigned>(slices), static_cast<unsigned>(n_mat));
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (out_dtype == TQ_BF16)
-        k_dequant<__nv_bfloat16><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, n_mat, O, I,
+        k_dequant<__nv_bfloat16><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, O, I, rps,
                                                        static_cast<__nv_bfloat16*>(out));
     else
-        k_dequant<float><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, n_mat, O, I,
+        k_dequant<float><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, O, I, rps,
                                                static_cast<float*>(out));
     return check_launch("tq_dequant");
 }

@@ -16,12 +16,20 @@ namespace tq {
 
 constexpr int PX_THREADS = 256;
 
-inline int64_t px_blocks(int64_t n_mat, int64_t units) {
-    int64_t cap = (8 * 148) / n_mat;
-    if (cap < 1) cap = 1;
-    int64_t need = (units + PX_THREADS - 1) / PX_THREADS;
-    if (need < 1) need = 1;
-    return need < cap ? need : cap;
+// Grid: x = 256-chunk column tiles (a chunk = 16 weights of one group),
+// y = row slices, z = matrices.  Each thread loads its chunk's 16 imatrix
+// weights once and walks the rows of its slice.
+struct PxGeom { int64_t cblocks, slices, rps; };
+
+inline PxGeom px_geometry(int64_t n_mat, int64_t O, int64_t I) {
+    PxGeom g;
+    const int64_t C = (I + 15) / 16;
+    g.cblocks = (C + PX_THREADS - 1) / PX_THREADS;
+    int64_t s = (4 * 148 + g.cblocks * n_mat - 1) / (g.cblocks * n_mat);
+    s = s < 1 ? 1 : (s > O ? O : s);
+    g.rps = (O + s - 1) / s;
+    g.slices = (O + g.rps - 1) / g.rps;
+    return g;
 }
 
 template <typename T>
@@ -60,47 +68,50 @@ template <typename T>
 __global__ void __launch_bounds__(PX_THREADS)
 k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, const uint8_t* __restrict__ packed,
         int fmt, const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
-        const float* __restrict__ m, int64_t m_stride, double* __restrict__ part_out,
+        const float* __restrict__ m, int64_t m_stride, int64_t rps, double* __restrict__ part_out,
         unsigned* __restrict__ tickets, double* __restrict__ num, double* __restrict__ den) {
-    const int g = fmt == TQ_INT3_G64_SYM ? 64 : (fmt == TQ_INT4_G128_ASYM ? 128 : 16);
-    const int parts = g / 16;
-    const int64_t G = (I + g - 1) / g;
-    const int64_t units = O * G * parts;
-    const int64_t e = blockIdx.y;
-    const int64_t nblk = gridDim.x;
+    const int lg = fmt == TQ_INT3_G64_SYM ? 2 : (fmt == TQ_INT4_G128_ASYM ? 3 : 0);   // log2(chunks per group)
+    const int64_t G = (I + (16 << lg) - 1) >> (4 + lg);
+    const int64_t C = (I + 15) >> 4;
+    const int64_t e = blockIdx.z;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * PX_THREADS + threadIdx.x;
+    const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
+    const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     double an = 0.0, ad = 0.0;
-    for (int64_t u = static_cast<int64_t>(blockIdx.x) * PX_THREADS + threadIdx.x; u < units;
-         u += nblk * PX_THREADS) {
-        const int64_t gl = u / parts;             // group within matrix
-        const int part = static_cast<int>(u - gl * parts);
-        const int64_t o = gl / G, k = gl - o * G;
-        const int64_t j = k * g + part * 16;
-        if (j >= I) continue;
+    if (c < C) {
+        const int64_t k = c >> lg;
+        const int part = static_cast<int>(c & ((1 << lg) - 1));
+        const int64_t j = c << 4;
         const int n = static_cast<int>(min(static_cast<int64_t>(16), I - j));
         const bool full = n == 16;
-        float v[16], w[16], mm[16];
-        dq_unit(fmt, packed, scales, zeros, gs, O * G, e * O * G + gl, part, v);
-        load16<T>(W + e * ms + o * ld + j, full, n, w);
+        float mm[16];
         const float* mp = m + e * m_stride + j;
         if (full) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                const float4 a = __ldg(reinterpret_cast<const float4*>(mp) + i);
-                mm[4 * i] = a.x; mm[4 * i + 1] = a.y; mm[4 * i + 2] = a.z; mm[4 * i + 3] = a.w;
+                const float4 a4 = __ldg(reinterpret_cast<const float4*>(mp) + i);
+                mm[4 * i] = a4.x; mm[4 * i + 1] = a4.y; mm[4 * i + 2] = a4.z; mm[4 * i + 3] = a4.w;
             }
         } else {
 #pragma unroll
             for (int i = 0; i < 16; ++i) mm[i] = i < n ? __ldg(mp + i) : 0.f;
         }
-        float sn = 0.f, sd = 0.f;
+        const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rps;
+        const int64_t o1 = min(O, o0 + rps);
+        for (int64_t o = o0; o < o1; ++o) {
+            float v[16], w[16];
+            dq_unit(fmt, packed, scales, zeros, gs, O * G, (e * O + o) * G + k, part, v);
+            load16<T>(W + e * ms + o * ld + j, full, n, w);
+            float sn = 0.f, sd = 0.f;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const float d = __fsub_rn(w[i], v[i]);
-            sn = __fmaf_rn(__fmul_rn(mm[i], d), d, sn);
-            sd = __fmaf_rn(__fmul_rn(mm[i], w[i]), w[i], sd);
+            for (int i = 0; i < 16; ++i) {
+                const float d = __fsub_rn(w[i], v[i]);
+                sn = __fmaf_rn(__fmul_rn(mm[i], d), d, sn);
+                sd = __fmaf_rn(__fmul_rn(mm[i], w[i]), w[i], sd);
+            }
+            an += static_cast<double>(sn);
+            ad += static_cast<double>(sd);
         }
-        an += static_cast<double>(sn);
-        ad += static_cast<double>(sd);
     }
     // block reduction in fp64, fixed order
 #pragma unroll
@@ -116,8 +127,8 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
     if (threadIdx.x == 0) {
         double bn = 0.0, bd = 0.0;
         for (int i = 0; i < PX_THREADS / 32; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
-        part_out[(e * nblk + blockIdx.x) * 2] = bn;
-        part_out[(e * nblk + blockIdx.x) * 2 + 1] = bd;
+        part_out[(e * nblk + bid) * 2] = bn;
+        part_out[(e * nblk + bid) * 2 + 1] = bd;
         __threadfence();
         last = atomicAdd(tickets + e, 1u) == static_cast<unsigned>(nblk - 1);
     }
@@ -141,10 +152,9 @@ using namespace tq;
 TQ_API size_t tq_proxy_workspace_bytes(const tq_mat* W, int32_t fmt) {
     const int64_t g = group_of(fmt);
     if (!W || g == 0 || W->n_mat < 1 || W->rows < 1 || W->cols < 1) return 0;
-    const int64_t units = W->rows * ((W->cols + g - 1) / g) * (g / 16);
-    const int64_t nblk = px_blocks(W->n_mat, units);
+    const PxGeom pg = px_geometry(W->n_mat, W->rows, W->cols);
     const int64_t tick = ((W->n_mat * 4 + 15) / 16) * 16;
-    return static_cast<size_t>(tick + W->n_mat * nblk * 16);
+    return static_cast<size_t>(tick + W->n_mat * pg.cblocks * pg.slices * 16);
 }
 
 TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, const void* scales,
@@ -166,23 +176,22 @@ TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t 
     const size_t need = tq_proxy_workspace_bytes(W, fmt);
     TQ_REQUIRE(workspace_bytes >= need, "tq_proxy_error: workspace too small (%zu < %zu)", workspace_bytes, need);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t units = W->rows * ((W->cols + g - 1) / g) * (g / 16);
-    const int64_t nblk = px_blocks(W->n_mat, units);
+    const PxGeom pg = px_geometry(W->n_mat, W->rows, W->cols);
     const int64_t tick = ((W->n_mat * 4 + 15) / 16) * 16;
     unsigned* tickets = static_cast<unsigned*>(workspace);
     double* parts = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + tick);
     cudaError_t ce = cudaMemsetAsync(tickets, 0, static_cast<size_t>(W->n_mat) * 4, st);
     if (ce != cudaSuccess) return set_error(TQ_ERR_CUDA, "tq_proxy_error: %s", cudaGetErrorString(ce));
-    const dim3 grid(static_cast<unsigned>(nblk), static_cast<unsigned>(W->n_mat));
+    const dim3 grid(static_cast<unsigned>(pg.cblocks), static_cast<unsigned>(pg.slices), static_cast<unsigned>(W->n_mat));
     const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
     const int64_t mst = W->n_mat > 1 ? m_stride : 0;
     if (W->dtype == TQ_BF16)
         k_proxy<uint16_t><<<grid, PX_THREADS, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->rows, W->cols, W->ld, ms,
-                                                      packed, fmt, scales, zeros, global_scale, m, mst, parts,
+                                                      packed, fmt, scales, zeros, global_scale, m, mst, pg.rps, parts,
                                                       tickets, num, den);
     else
         k_proxy<float><<<grid, PX_THREADS, 0, st>>>(static_cast<const float*>(W->ptr), W->rows, W->cols, W->ld, ms,
-                                                   packed, fmt, scales, zeros, global_scale, m, mst, parts,
+                                                   packed, fmt, scales, zeros, global_scale, m, mst, pg.rps, parts,
                                                    tickets, num, den);
     return check_launch("tq_proxy_error");
 }

@@ -9,15 +9,25 @@
 //   L = sum_j m_j (w_j - s (q_j - z))^2; ties keep the lowest index nz k + i.
 //
 // B200 mapping: one warp per 128-weight group; lane l owns scales l and l+32
-// and all 16 distinct zero-points (32 fp32 accumulators).  The group's (w, m)
-// pairs are staged in shared memory and broadcast to all lanes, so the 1024
-// candidates reuse one HBM read.  Per element and scale, rint(w/s) is formed
-// once (an FMA against 1.5*2^23 and a subtract); each zero-point then costs a
-// clamp to [-z, 15-z] (two min/max), the residual FMA and the weighted-square
-// FMA pair.  Zero-points repeated in the 32-point list never win under the
-// lowest-index rule, so only the first occurrence of each is evaluated.
-// Near ties (relative 2^-15) are re-ranked in fp64 with codes from the IEEE
-// quotient, exactly as the definition ranks them.
+// and all 16 distinct zero-points.  The group's weights (and sqrt of their
+// imatrix weights) are staged in shared memory and broadcast to all lanes, so
+// the 1024 candidates reuse one HBM read.  Zero-points repeated in the
+// 32-point list never win under the lowest-index rule, so only the first
+// occurrence of each is evaluated.
+//
+// Per candidate-element the error is one min or max: with s > 0 the code
+// r = rint(w/s) has the sign of w, so a negative weight can only be clamped
+// at the low end (code -z, error w + s z) and a non-negative one only at the
+// high end (code 15 - z, error w - s (15 - z)); clamping only ever moves the
+// error further from zero, hence
+//   e(z) = min(u, w + s z)          for w < 0,
+//   e(z) = max(u, w - s (15 - z))   for w >= 0,     u = w - s r (unclamped).
+// Elements are split by sign once per group (uniform branches), all errors
+// carry a factor sqrt(m) so the weighted square is one FMA, and Blackwell's
+// packed fp32x2 FMA evaluates two zero-points per instruction: per pair of
+// candidate-elements two FFMA2 (bound, accumulate) and two FMNMX.  Near ties
+// (relative 2^-14) are re-ranked in fp64 with codes from the IEEE quotient,
+// exactly as the definition ranks them.
 #include "group_pack.cuh"
 
 #include <climits>
@@ -25,7 +35,7 @@
 namespace tq {
 
 constexpr int ASYM_WARPS = 4;
-constexpr float AWIN = 3.0517578125e-05f;   // 2^-15
+constexpr float AWIN = 6.103515625e-05f;   // 2^-14: bound on fp32 ranking error x 2 (with margin)
 
 struct AsymArgs {
     const void* W;
@@ -80,19 +90,29 @@ __device__ __forceinline__ double loss64_int4(const float w[4], const float m[4]
     return group_sum_d(t, FULL, 32);
 }
 
-// The 16 zero-points of one scale for one element: r = rint(w/s) is shared,
-// code - z = clamp(r, -z, 15 - z).
-#define TQ_Z16(ACC, R, S, W, Mv)                                                   \
-    _Pragma("unroll") for (int z = 0; z < 16; ++z) {                               \
-        const float c_ = fminf(fmaxf(R, static_cast<float>(-z)), static_cast<float>(15 - z)); \
-        const float e_ = __fmaf_rn(-(S), c_, W);                                   \
-        ACC[z] = __fmaf_rn(__fmul_rn(Mv, e_), e_, ACC[z]);                         \
+// Accumulates sum over elements of e(z)^2 for the 16 zero-points of one scale
+// (pairs z = 2p, 2p + 1 packed in float2).  wm = sqrt(m) w, sm = sqrt(m).
+template <bool POS>
+__device__ __forceinline__ void acc_scale(float w, float wm, float sm, float s, float inv, float2 (&acc)[8]) {
+    const float q = __fmul_rn(sm, s);                                   // sqrt(m) s
+    const float r = __fsub_rn(__fmaf_rn(w, inv, MAGIC), MAGIC);         // rint(w/s)
+    const float u = __fmaf_rn(-q, r, wm);                               // sqrt(m) (w - s r)
+    const float base = POS ? __fmaf_rn(-15.f, q, wm) : wm;              // bound(z) = base + q z
+    const float2 qq = make_float2(q, q), bb = make_float2(base, base);
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+        const float2 bnd = __ffma2_rn(qq, make_float2(static_cast<float>(2 * p), static_cast<float>(2 * p + 1)), bb);
+        float2 e;
+        if (POS) { e.x = fmaxf(u, bnd.x); e.y = fmaxf(u, bnd.y); }
+        else     { e.x = fminf(u, bnd.x); e.y = fminf(u, bnd.y); }
+        acc[p] = __ffma2_rn(e, e, acc[p]);
     }
+}
 
 template <typename T>
 __global__ void __launch_bounds__(ASYM_WARPS * 32)
 k_search_int4(const __grid_constant__ AsymArgs a) {
-    __shared__ __align__(16) float2 lists[ASYM_WARPS][128];
+    __shared__ __align__(16) float2 lists[ASYM_WARPS][132];   // two sign lists, each padded to even length
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t G = (a.I + 127) >> 7;
     const int64_t OG = a.O * G;
@@ -157,33 +177,66 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
         const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
         const float Rs = __fmul_rn(R, pw);
-        __syncwarp();
+        // split by sign: negative weights first, non-negative after (tail: (0, 0))
+        float x[4], sq[4];
+        bool neg[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)   // tail: (0, 0)
-            list[4 * lane + i] = make_float2(__fmul_rn(w[i], pw), __fmul_rn(mv[i], pm));
+        for (int i = 0; i < 4; ++i) {
+            x[i] = __fmul_rn(w[i], pw);
+            sq[i] = sqrtf(__fmul_rn(mv[i], pm));
+            neg[i] = val[i] && x[i] < 0.f;
+        }
+        unsigned bn[4];
+        int nneg = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) { bn[i] = __ballot_sync(FULL, neg[i]); nneg += __popc(bn[i]); }
+        const int npos_real = n - nneg;
+        const int nneg_pad = (nneg + 1) & ~1;
+        const int npos_pad = (npos_real + 1) & ~1;
+        __syncwarp();
+        {
+            int before_n = 0, before_p = 0;
+            const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const unsigned bp = __ballot_sync(FULL, val[i] && !neg[i]);
+                if (neg[i]) list[before_n + __popc(bn[i] & lt)] = make_float2(x[i], sq[i]);
+                else if (val[i]) list[nneg_pad + before_p + __popc(bp & lt)] = make_float2(x[i], sq[i]);
+                before_n += __popc(bn[i]);
+                before_p += __popc(bp);
+            }
+            if (lane == 0 && nneg_pad > nneg) list[nneg] = make_float2(0.f, 0.f);
+            if (lane == 0 && npos_pad > npos_real) list[nneg_pad + npos_real] = make_float2(0.f, 0.f);
+        }
         __syncwarp();
 
         const float sA = __fmul_rn(cA, Rs), sB = __fmul_rn(cB, Rs);
         const float sAo = __fmul_rn(cA, R), sBo = __fmul_rn(cB, R);
         const float iA = __frcp_rn(sA), iB = __frcp_rn(sB);
+        float2 a2[8], b2[8];
+#pragma unroll
+        for (int p = 0; p < 8; ++p) { a2[p] = make_float2(0.f, 0.f); b2[p] = make_float2(0.f, 0.f); }
+        for (int j = 0; j < (nneg_pad >> 1); ++j) {
+            const float4 p = list4[j];
+            const float wm0 = __fmul_rn(p.x, p.y), wm1 = __fmul_rn(p.z, p.w);
+            acc_scale<false>(p.x, wm0, p.y, sA, iA, a2);
+            acc_scale<false>(p.x, wm0, p.y, sB, iB, b2);
+            acc_scale<false>(p.z, wm1, p.w, sA, iA, a2);
+            acc_scale<false>(p.z, wm1, p.w, sB, iB, b2);
+        }
+        for (int j = nneg_pad >> 1; j < ((nneg_pad + npos_pad) >> 1); ++j) {
+            const float4 p = list4[j];
+            const float wm0 = __fmul_rn(p.x, p.y), wm1 = __fmul_rn(p.z, p.w);
+            acc_scale<true>(p.x, wm0, p.y, sA, iA, a2);
+            acc_scale<true>(p.x, wm0, p.y, sB, iB, b2);
+            acc_scale<true>(p.z, wm1, p.w, sA, iA, a2);
+            acc_scale<true>(p.z, wm1, p.w, sB, iB, b2);
+        }
         float accA[16], accB[16];
 #pragma unroll
-        for (int z = 0; z < 16; ++z) { accA[z] = 0.f; accB[z] = 0.f; }
-        const int npair = (n + 1) >> 1;
-        for (int j = 0; j < npair; ++j) {
-            const float4 p = list4[j];
-            {
-                const float rA = __fsub_rn(__fmaf_rn(p.x, iA, MAGIC), MAGIC);
-                TQ_Z16(accA, rA, sA, p.x, p.y)
-                const float rB = __fsub_rn(__fmaf_rn(p.x, iB, MAGIC), MAGIC);
-                TQ_Z16(accB, rB, sB, p.x, p.y)
-            }
-            {
-                const float rA = __fsub_rn(__fmaf_rn(p.z, iA, MAGIC), MAGIC);
-                TQ_Z16(accA, rA, sA, p.z, p.w)
-                const float rB = __fsub_rn(__fmaf_rn(p.z, iB, MAGIC), MAGIC);
-                TQ_Z16(accB, rB, sB, p.z, p.w)
-            }
+        for (int p = 0; p < 8; ++p) {
+            accA[2 * p] = a2[p].x; accA[2 * p + 1] = a2[p].y;
+            accB[2 * p] = b2[p].x; accB[2 * p + 1] = b2[p].y;
         }
 
         // lane-local argmin in index order (all of scale A precede scale B)
