@@ -15,19 +15,19 @@
 // 32-point list never win under the lowest-index rule, so only the first
 // occurrence of each is evaluated.
 //
-// Per candidate-element the error is one min or max: with s > 0 the code
+// Per candidate-element the clamp is one min or max: with s > 0 the code
 // r = rint(w/s) has the sign of w, so a negative weight can only be clamped
-// at the low end (code -z, error w + s z) and a non-negative one only at the
-// high end (code 15 - z, error w - s (15 - z)); clamping only ever moves the
-// error further from zero, hence
-//   e(z) = min(u, w + s z)          for w < 0,
-//   e(z) = max(u, w - s (15 - z))   for w >= 0,     u = w - s r (unclamped).
-// Elements are split by sign once per group (uniform branches), all errors
-// carry a factor sqrt(m) so the weighted square is one FMA, and Blackwell's
-// packed fp32x2 FMA evaluates two zero-points per instruction: per pair of
-// candidate-elements two FFMA2 (bound, accumulate) and two FMNMX.  Near ties
-// (relative 2^-14) are re-ranked in fp64 with codes from the IEEE quotient,
-// exactly as the definition ranks them.
+// at the low end (code -z) and a non-negative one only at the high end (code
+// 15 - z).  With u = w - s r the unclamped error the clamped error is
+// u + s d(z), d(z) = min(r + z, 0) for w < 0 and max(r - 15 + z, 0) for
+// w >= 0.  Elements are split by sign once per group (uniform branches), every
+// error carries a factor sqrt(m) so the weighted square is one FMA, and
+// Blackwell's packed fp32x2 add/FMA evaluate two zero-points per instruction:
+// per pair of candidate-elements FADD2 (excess), two FMNMX, FFMA2 (error),
+// FFMA2 (accumulate).  Each error is formed by one FMA from exact products,
+// so every term keeps a few ulp of relative accuracy.  Near ties (relative
+// 2^-15) are re-ranked in fp64 with codes from the IEEE quotient, exactly as
+// the definition ranks them.
 #include "group_pack.cuh"
 
 #include <climits>
@@ -35,7 +35,7 @@
 namespace tq {
 
 constexpr int ASYM_WARPS = 4;
-constexpr float AWIN = 6.103515625e-05f;   // 2^-14: bound on fp32 ranking error x 2 (with margin)
+constexpr float AWIN = 3.0517578125e-05f;   // 2^-15: bound on fp32 ranking error x 2 (with margin)
 
 struct AsymArgs {
     const void* W;
@@ -90,21 +90,26 @@ __device__ __forceinline__ double loss64_int4(const float w[4], const float m[4]
     return group_sum_d(t, FULL, 32);
 }
 
-// Accumulates sum over elements of e(z)^2 for the 16 zero-points of one scale
-// (pairs z = 2p, 2p + 1 packed in float2).  wm = sqrt(m) w, sm = sqrt(m).
+// Accumulates, for the 16 zero-points of one scale, m e(z)^2 of one element
+// (pairs z = 2p, 2p + 1 packed in float2).  With u = w - s r the unclamped
+// error and d(z) the integer clamp excess -- max(r - 15 + z, 0) for w >= 0,
+// min(r + z, 0) for w < 0 -- the error is e = u + s d.  Every quantity carries
+// sqrt(m): u' = sqrt(m) u, q = sqrt(m) s, e' = fma(q, d, u') (exact product,
+// one rounding, no cancellation), and the weighted square is fma(e', e', acc).
 template <bool POS>
-__device__ __forceinline__ void acc_scale(float w, float wm, float sm, float s, float inv, float2 (&acc)[8]) {
-    const float q = __fmul_rn(sm, s);                                   // sqrt(m) s
+__device__ __forceinline__ void acc_scale(float w, float sm, float s, float inv, float2 (&acc)[8]) {
     const float r = __fsub_rn(__fmaf_rn(w, inv, MAGIC), MAGIC);         // rint(w/s)
-    const float u = __fmaf_rn(-q, r, wm);                               // sqrt(m) (w - s r)
-    const float base = POS ? __fmaf_rn(-15.f, q, wm) : wm;              // bound(z) = base + q z
-    const float2 qq = make_float2(q, q), bb = make_float2(base, base);
+    const float u = __fmul_rn(sm, __fmaf_rn(-s, r, w));                  // sqrt(m) (w - s r)
+    const float q = __fmul_rn(sm, s);                                   // sqrt(m) s
+    const float rb = POS ? __fsub_rn(r, 15.f) : r;                      // d(z) = clamp excess of rb + z
+    const float2 qq = make_float2(q, q), uu = make_float2(u, u), rr = make_float2(rb, rb);
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
-        const float2 bnd = __ffma2_rn(qq, make_float2(static_cast<float>(2 * p), static_cast<float>(2 * p + 1)), bb);
-        float2 e;
-        if (POS) { e.x = fmaxf(u, bnd.x); e.y = fmaxf(u, bnd.y); }
-        else     { e.x = fminf(u, bnd.x); e.y = fminf(u, bnd.y); }
+        const float2 t = __fadd2_rn(rr, make_float2(static_cast<float>(2 * p), static_cast<float>(2 * p + 1)));
+        float2 d;
+        if (POS) { d.x = fmaxf(t.x, 0.f); d.y = fmaxf(t.y, 0.f); }
+        else     { d.x = fminf(t.x, 0.f); d.y = fminf(t.y, 0.f); }
+        const float2 e = __ffma2_rn(qq, d, uu);
         acc[p] = __ffma2_rn(e, e, acc[p]);
     }
 }
@@ -218,19 +223,17 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         for (int p = 0; p < 8; ++p) { a2[p] = make_float2(0.f, 0.f); b2[p] = make_float2(0.f, 0.f); }
         for (int j = 0; j < (nneg_pad >> 1); ++j) {
             const float4 p = list4[j];
-            const float wm0 = __fmul_rn(p.x, p.y), wm1 = __fmul_rn(p.z, p.w);
-            acc_scale<false>(p.x, wm0, p.y, sA, iA, a2);
-            acc_scale<false>(p.x, wm0, p.y, sB, iB, b2);
-            acc_scale<false>(p.z, wm1, p.w, sA, iA, a2);
-            acc_scale<false>(p.z, wm1, p.w, sB, iB, b2);
+            acc_scale<false>(p.x, p.y, sA, iA, a2);
+            acc_scale<false>(p.x, p.y, sB, iB, b2);
+            acc_scale<false>(p.z, p.w, sA, iA, a2);
+            acc_scale<false>(p.z, p.w, sB, iB, b2);
         }
         for (int j = nneg_pad >> 1; j < ((nneg_pad + npos_pad) >> 1); ++j) {
             const float4 p = list4[j];
-            const float wm0 = __fmul_rn(p.x, p.y), wm1 = __fmul_rn(p.z, p.w);
-            acc_scale<true>(p.x, wm0, p.y, sA, iA, a2);
-            acc_scale<true>(p.x, wm0, p.y, sB, iB, b2);
-            acc_scale<true>(p.z, wm1, p.w, sA, iA, a2);
-            acc_scale<true>(p.z, wm1, p.w, sB, iB, b2);
+            acc_scale<true>(p.x, p.y, sA, iA, a2);
+            acc_scale<true>(p.x, p.y, sB, iB, b2);
+            acc_scale<true>(p.z, p.w, sA, iA, a2);
+            acc_scale<true>(p.z, p.w, sB, iB, b2);
         }
         float accA[16], accB[16];
 #pragma unroll
