@@ -247,6 +247,18 @@ def _oracle_unit(oracle, wl, u, rows):
     oracle.proxy_error(W[0], What, m)
 
 
+def read_traffic(path, workload):
+    """DRAM bytes per launch of the dominant kernel from the profiles table."""
+    try:
+        for line in open(path):
+            cells = [c.strip() for c in line.strip().strip("|").split("|")]
+            if len(cells) >= 3 and cells[0] == workload and cells[2].isdigit():
+                return int(cells[2])
+    except OSError:
+        pass
+    return None
+
+
 # ------------------------------------------------------------------ main
 
 def parse():
@@ -258,8 +270,8 @@ def parse():
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic-json", default=os.path.join(ROOT, "profiles", "traffic.json"),
-                    help="ncu DRAM bytes per launch of the dominant kernel, keyed by workload")
+    ap.add_argument("--traffic-table", default=os.path.join(ROOT, "profiles", "traffic.md"),
+                    help="ncu DRAM bytes per launch of the dominant kernel, by workload")
     return ap.parse_args()
 
 
@@ -363,12 +375,7 @@ def main():
     sms = props.multi_processor_count
     peak_tinst = sms * 128 * pk["sm_max_mhz"] * 1e6 / 1e12
     achieved = SEARCH_INSTR_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3) / 1e12
-    traffic = None
-    try:
-        tj = json.load(open(args.traffic_json))
-        traffic = tj.get(args.config)
-    except Exception:
-        pass
+    traffic = read_traffic(args.traffic_table, args.config)
     clocks = clk.summary()
     roofline = {"bound": "alu", "achieved": achieved, "peak": peak_tinst, "unit": "Tinst/s",
                 "frac": achieved / peak_tinst, "traffic": traffic,
