@@ -51,7 +51,7 @@ EXPORTS = [
     "tq_default_params", "tq_last_error_string", "tq_version", "tq_group_size", "tq_num_groups",
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
-    "tq_proxy_error", "tq_sync",
+    "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static",
 ]
 
 
@@ -135,6 +135,8 @@ def lib():
             "tq_proxy_workspace_bytes": (sz, [Mp, i32]),
             "tq_proxy_error": (i32, [Mp, P, i32, P, P, P, P, i64, P, P, P, sz, P]),
             "tq_sync": (i32, [P]),
+            "tq_imatrix_static_capacity": (sz, []),
+            "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -237,6 +239,26 @@ def tq_imatrix(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optiona
                             ctypes.c_float(alpha), int(accumulate), _ptr(workspace),
                             workspace.numel(), _stream(stream)), "tq_imatrix")
     return m
+
+
+def tq_imatrix_static(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optional[float] = None,
+                      accumulate: bool = False, stream=None) -> torch.Tensor:
+    """tq_imatrix without a caller workspace: the library's fixed device
+    scratch is used instead (see include/tq.h for its limits and the rule
+    that calls must not overlap on the GPU)."""
+    d = _mat(X, "X")
+    if alpha is None:
+        alpha = 1.0 / d.rows
+    if m is None:
+        m = torch.zeros((d.n_mat, d.cols), dtype=torch.float32, device=X.device)
+    _cuda(m, "m")
+    _check(lib().tq_imatrix_static(ctypes.byref(d), _ptr(m), _m_stride(m) if m.dim() == 2 else 0,
+                                   ctypes.c_float(alpha), int(accumulate), _stream(stream)), "tq_imatrix_static")
+    return m
+
+
+def tq_imatrix_static_capacity() -> int:
+    return int(lib().tq_imatrix_static_capacity())
 
 
 def tq_amax(W: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -12,6 +12,8 @@
 // the slices in a fixed order, so results do not depend on scheduling.
 #include "tq_internal.cuh"
 
+#include <mutex>
+
 namespace tq {
 
 constexpr int IM_THREADS = 256;
@@ -223,6 +225,54 @@ TQ_API tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float a
     k_imatrix_final<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
         partial, g.slices, X->n_mat, X->cols, m, X->n_mat > 1 ? m_stride : 0, static_cast<double>(alpha), accumulate);
     return check_launch("imatrix final");
+}
+
+// ------------------------------------------------------------------ allocation-free variant
+//
+// Scratch for tq_imatrix_static: a fixed 4 MiB of device memory that every
+// GPU loading this library keeps until the process exits.  In host code the
+// symbol only names a host-side shadow, so its device address is looked up
+// once per device (with that device current) and cached.
+
+constexpr size_t IM_STATIC_BYTES = size_t(4) << 20;
+static __device__ __align__(256) double g_im_scratch[IM_STATIC_BYTES / sizeof(double)];
+
+static std::mutex g_im_mu;
+static void* g_im_ptr[64];
+
+static tq_status im_static_ptr(void** out) {
+    int dev = 0;
+    cudaError_t ce = cudaGetDevice(&dev);
+    if (ce != cudaSuccess) return set_error(TQ_ERR_CUDA, "tq_imatrix_static: %s", cudaGetErrorString(ce));
+    if (dev < 0 || dev >= 64) return set_error(TQ_ERR_UNSUPPORTED, "tq_imatrix_static: device %d", dev);
+    std::lock_guard<std::mutex> lk(g_im_mu);
+    if (!g_im_ptr[dev]) {
+        void* p = nullptr;
+        ce = cudaGetSymbolAddress(&p, g_im_scratch);
+        if (ce != cudaSuccess || !p)
+            return set_error(TQ_ERR_CUDA, "tq_imatrix_static: scratch lookup: %s", cudaGetErrorString(ce));
+        g_im_ptr[dev] = p;
+    }
+    *out = g_im_ptr[dev];
+    return TQ_OK;
+}
+
+TQ_API size_t tq_imatrix_static_capacity(void) { return IM_STATIC_BYTES; }
+
+TQ_API tq_status tq_imatrix_static(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
+                                   tq_stream_t stream) {
+    clear_error();
+    tq_status s = check_mat(X, "tq_imatrix_static X");
+    if (s != TQ_OK) return s;
+    const size_t need = tq_imatrix_workspace_bytes(X);
+    if (need > IM_STATIC_BYTES)
+        return set_error(TQ_ERR_INVALID_ARG,
+                         "tq_imatrix_static: this shape needs %zu bytes of scratch, above the fixed %zu; "
+                         "use tq_imatrix with a caller-provided workspace",
+                         need, IM_STATIC_BYTES);
+    void* ws = nullptr;
+    if ((s = im_static_ptr(&ws)) != TQ_OK) return s;
+    return tq_imatrix(X, m, m_stride, alpha, accumulate, ws, IM_STATIC_BYTES, stream);
 }
 
 TQ_API tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream) {

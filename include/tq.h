@@ -137,6 +137,29 @@ size_t tq_imatrix_workspace_bytes(const tq_mat* X);
 tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
                      void* workspace, size_t workspace_bytes, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ imatrix without allocation
+ * No counterpart in the source pages: this is a packaging variant of
+ * tq_imatrix for callers that cannot allocate device memory on the path that
+ * calls it -- for example code running inside another engine's enqueue hook
+ * that is handed only its input and output buffers, or a process whose
+ * device memory is fully pre-planned by an arena that does not grant
+ * scratch.  Same arguments and results as tq_imatrix, but the scratch is a
+ * fixed tq_imatrix_static_capacity() bytes (4 MiB) of device memory inside
+ * the library, held by every GPU that loads it until the process exits.
+ *  - Shapes whose tq_imatrix_workspace_bytes() exceed the capacity are
+ *    rejected with TQ_ERR_INVALID_ARG (use tq_imatrix with a workspace).
+ *  - The first call on each device looks up the scratch address on that
+ *    device (it must be the current device); make that first call before
+ *    any stream capture.
+ *  - All calls share the one scratch array: calls whose kernels may overlap
+ *    on the GPU (other streams, other host threads) race and give wrong
+ *    results; serialise them.  Nothing in the scratch needs to start at
+ *    zero, so the previous call's leftovers are harmless.
+ *  - Calls no allocating routine (no cudaMalloc/cudaFree). */
+size_t tq_imatrix_static_capacity(void);
+tq_status tq_imatrix_static(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
+                            tq_stream_t stream);
+
 /* ------------------------------------------------------------------ amax
  * amax[e] = max |W[e]| over matrix e (f32).  Used for the NVFP4 per-tensor
  * global scale g = fl32(amax / (6 * 448)). */
