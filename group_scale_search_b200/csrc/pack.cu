@@ -298,7 +298,7 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant: out dtype %d", out_dtype);
     const int64_t C = (I + 15) / 16;
     const int64_t cblocks = (C + 255) / 256;
-    int64_t slices = (4 * static_cast<int64_t>(num_sms()) + cblocks * n_mat - 1) / (cblocks * n_mat);
+    int64_t slices = (16 * static_cast<int64_t>(num_sms()) + cblocks * n_mat - 1) / (cblocks * n_mat);
     slices = max(static_cast<int64_t>(1), min(slices, O));
     const int64_t rps = (O + slices - 1) / slices;
     slices = (O + rps - 1) / rps;

@@ -25,7 +25,7 @@ inline PxGeom px_geometry(int64_t n_mat, int64_t O, int64_t I) {
     PxGeom g;
     const int64_t C = (I + 15) / 16;
     g.cblocks = (C + PX_THREADS - 1) / PX_THREADS;
-    int64_t s = (4 * 148 + g.cblocks * n_mat - 1) / (g.cblocks * n_mat);
+    int64_t s = (16 * 148 + g.cblocks * n_mat - 1) / (g.cblocks * n_mat);
     s = s < 1 ? 1 : (s > O ? O : s);
     g.rps = (O + s - 1) / s;
     g.slices = (O + g.rps - 1) / g.rps;
@@ -133,15 +133,27 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
         last = atomicAdd(tickets + e, 1u) == static_cast<unsigned>(nblk - 1);
     }
     __syncthreads();
-    if (last && threadIdx.x == 0) {
+    if (last) {   // the matrix's last block adds the partials: fixed strides, fixed tree
         __threadfence();
         double tn = 0.0, td = 0.0;
-        for (int64_t b = 0; b < nblk; ++b) {
+        for (int64_t b = threadIdx.x; b < nblk; b += PX_THREADS) {
             tn += __ldcg(part_out + (e * nblk + b) * 2);
             td += __ldcg(part_out + (e * nblk + b) * 2 + 1);
         }
-        num[e] = tn;
-        den[e] = td;
+#pragma unroll
+        for (int off = 16; off; off >>= 1) {
+            tn += __shfl_xor_sync(FULL, tn, off);
+            td += __shfl_xor_sync(FULL, td, off);
+        }
+        __syncthreads();
+        if (lane == 0) { sw[0][wid] = tn; sw[1][wid] = td; }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            double bn = 0.0, bd = 0.0;
+            for (int i = 0; i < PX_THREADS / 32; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
+            num[e] = bn;
+            den[e] = bd;
+        }
     }
 }
 

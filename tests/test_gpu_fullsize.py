@@ -1,0 +1,146 @@
+"""Full-size parity: each workload at its full size, run exactly as bench.py
+runs it (one call per unit over all matrices), checked against the oracle on
+outputs it can compute one by one -- whole sampled rows of every unit
+(search choice and loss, scales, packed records, dequantized weights),
+sampled imatrix columns, and the proxy error of one whole matrix per unit."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_checks import LOSS_RTOL, MATCH_MIN, SUM_RTOL, host32, oracle_dequant, oracle_packed, rel_close
+
+pytestmark = pytest.mark.gpu
+
+tq = pytest.importorskip("group_scale_search_b200")
+import oracle  # noqa: E402
+
+DEV = "cuda"
+RECORD = {tq.INT3_G64_SYM: 24, tq.INT4_G128_ASYM: 64, tq.NVFP4_G16: 8}
+GROUP = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.NVFP4_G16: 16}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    oracle.build()
+    tq.lib()
+
+
+def _sample_rows(E, O, n, seed):
+    rng = np.random.default_rng(seed)
+    rows = {(0, 0), (E - 1, O - 1), (E // 2, O // 2)}
+    while len(rows) < n:
+        rows.add((int(rng.integers(E)), int(rng.integers(O))))
+    return sorted(rows)
+
+
+def _check_unit(u, m_full, res, n_rows, seed, gscale_oracle=None):
+    fmt = tq.FORMATS[u.fmt]
+    E, O, I = u.W.shape
+    g = GROUP[fmt]
+    G = (I + g - 1) // g
+    rows = _sample_rows(E, O, n_rows, seed)
+    idx = torch.tensor([e * O + o for e, o in rows], device=DEV)
+    Wh = host32(u.W.reshape(E * O, I)[idx]).reshape(len(rows), 1, I)
+    mh = m_full.reshape(-1, I).cpu().numpy()
+    mrows = np.stack([mh[e if mh.shape[0] > 1 else 0] for e, _ in rows])     # one imatrix per sampled row
+    gi = res.cand_idx.reshape(E * O, G)[idx].cpu().numpy()
+    gs = res.scales.reshape(E * O, G)[idx].cpu().numpy()
+    gz = res.zeros.reshape(E * O, G)[idx].cpu().numpy() if res.zeros is not None else None
+    if fmt == tq.INT3_G64_SYM:
+        s, oi, L, v = oracle.search_sym_int3(Wh, mrows)
+        Lg = oracle.loss_given_int3(Wh, mrows, gs.reshape(len(rows), 1, G))
+    elif fmt == tq.INT4_G128_ASYM:
+        s, z, oi, L, q = oracle.search_asym_int4(Wh, mrows)
+        Lg = oracle.loss_given_int4(Wh, mrows, gs.reshape(len(rows), 1, G), gz.reshape(len(rows), 1, G))
+    else:
+        grow = np.array([gscale_oracle[e] for e, _ in rows], np.float32)
+        assert np.array_equal(res.global_scale.cpu().numpy(), gscale_oracle), "global scale"
+        _, s, oi, L, c = oracle.search_nvfp4(Wh, mrows, gscale=grow)
+        Lg = oracle.loss_given_nvfp4(Wh, mrows, gs.reshape(len(rows), 1, G), grow)
+    oi = oi.reshape(len(rows), G)
+    L = L.reshape(len(rows), G)
+    Lg = Lg.reshape(len(rows), G)
+    match = float((gi == oi).mean())
+    assert match >= MATCH_MIN, f"{u.name}: match {match}"
+    assert np.all(Lg <= L * (1 + LOSS_RTOL) + 1e-30), f"{u.name}: loss above the oracle minimum"
+    same = gi == oi
+    assert np.array_equal(gs[same], s.reshape(len(rows), G)[same])
+    lo = res.loss.reshape(E * O, G)[idx].cpu().numpy()
+    nz = Lg > 0
+    assert np.max(np.abs(lo[nz] - Lg[nz]) / Lg[nz]) <= LOSS_RTOL
+    # packed records and dequantized weights of the sampled rows, bit-exact
+    rec = RECORD[fmt]
+    packed = res.packed.reshape(E * O, G * rec)[idx].cpu().numpy()
+    if fmt == tq.NVFP4_G16:
+        ref_packed, codes = oracle_packed(fmt, Wh, gs.reshape(len(rows), 1, G), gscale=grow)
+    else:
+        ref_packed, codes = oracle_packed(fmt, Wh, gs.reshape(len(rows), 1, G),
+                                          None if gz is None else gz.reshape(len(rows), 1, G))
+    assert np.array_equal(packed.reshape(-1), ref_packed), f"{u.name}: packed records"
+    return rows, idx, codes, gs, gz, (grow if fmt == tq.NVFP4_G16 else None), match
+
+
+def _run_workload(name, n_rows=24, seed=0):
+    wl = synth.make(name, DEV)
+    ms = {}
+    for sname, site in wl.sites.items():
+        m = tq.tq_imatrix(site.X)
+        torch.cuda.synchronize()
+        # sampled columns of every site's imatrix
+        I = site.X.shape[2]
+        cols = torch.tensor(sorted(set(np.random.default_rng(seed).integers(0, I, 96).tolist()) | {0, I - 1}),
+                            device=DEV)
+        for e in {0, site.X.shape[0] - 1}:
+            Xs = host32(site.X[e][:, cols])
+            ref = oracle.imatrix(Xs)
+            assert rel_close(m[e][cols].cpu().numpy(), ref, SUM_RTOL) <= SUM_RTOL, f"{name}/{sname} imatrix"
+        ms[sname] = m
+    out = []
+    for k, u in enumerate(wl.units):
+        fmt = tq.FORMATS[u.fmt]
+        m = ms[u.site]
+        m = m if u.W.shape[0] > 1 else m[0]
+        res = tq.tq_search_groups(u.W, m, fmt)
+        E, O, I = u.W.shape
+        dq = tq.tq_dequant(res.packed, fmt, res.scales, res.zeros, res.global_scale, E, O, I)
+        num, den = tq.tq_proxy_error(u.W, res.packed, fmt, res.scales, res.zeros, res.global_scale, m)
+        torch.cuda.synchronize()
+        gso = None
+        if fmt == tq.NVFP4_G16:   # per-tensor global scales, one expert at a time
+            gso = np.concatenate([oracle.nvfp4_global(host32(u.W[e:e + 1])) for e in range(E)])
+        rows, idx, codes, gs, gz, grow, match = _check_unit(u, m, res, n_rows, seed + k, gso)
+        # dequantized weights of the sampled rows, bit-exact
+        ref = oracle_dequant(fmt, codes, gs.reshape(len(rows), 1, -1),
+                             None if gz is None else gz.reshape(len(rows), 1, -1), grow)
+        assert np.array_equal(dq.reshape(E * O, I)[idx].cpu().numpy(), ref.reshape(len(rows), I)), \
+            f"{name}/{u.name}: dequant"
+        # proxy error of one whole matrix against the oracle
+        e = E - 1
+        We = host32(u.W[e])
+        G = res.scales.shape[-1]
+        se = res.scales[e].cpu().numpy()
+        if fmt == tq.INT3_G64_SYM:
+            What = oracle.dequant_int3(oracle.rtn_int3(We, se), se)
+        elif fmt == tq.INT4_G128_ASYM:
+            ze = res.zeros[e].cpu().numpy()
+            What = oracle.dequant_int4(oracle.rtn_int4(We, se, ze), se, ze)
+        else:
+            ce = oracle.rtn_nvfp4(We[None], se[None], gso[e:e + 1])
+            What = oracle.dequant_nvfp4(ce, se[None], gso[e:e + 1])[0]
+        me = (m[e] if m.dim() == 2 else m).cpu().numpy()
+        rn, rd = oracle.proxy_error(We, What, me)
+        assert rel_close(num[e].item(), rn, SUM_RTOL) <= SUM_RTOL, f"{name}/{u.name}: proxy num"
+        assert rel_close(den[e].item(), rd, SUM_RTOL) <= SUM_RTOL, f"{name}/{u.name}: proxy den"
+        assert 0.0 < num[e].item() < den[e].item()
+        out.append((u.name, match))
+        del res, dq
+    return out
+
+
+@pytest.mark.parametrize("name", ["c0", "c1", "c2", "c3", "c4"])
+def test_full_size_workload(name):
+    results = _run_workload(name)
+    assert results
