@@ -268,6 +268,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="c1", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
+    ap.add_argument("--scale", type=float, default=1.0,
+                    help="shrink the workload (profiling and tests only; the reported line is for scale 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-table", default=os.path.join(ROOT, "profiles", "traffic.md"),
@@ -324,7 +326,7 @@ def main():
     import group_scale_search_b200 as tq
     tq.lib()
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = synth.make(args.config, dev, seed=rank)
+    wl = synth.make(args.config, dev, seed=rank, scale=args.scale)
     nbytes = input_bytes(wl)
     n_sets = max(1, min(64, math.ceil(2 * L2_BYTES / nbytes)))
     sets = make_sets(wl, n_sets)
@@ -395,7 +397,8 @@ def main():
     line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}",
+            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}"
+                                   + ("" if args.scale == 1.0 else f" (scaled x{args.scale})"),
                        "weights_per_gpu": nw,
                        "groups_per_gpu": sum(tq.tq_num_groups(tq.FORMATS[u.fmt], u.W.shape[0] * u.W.shape[1],
                                                               u.W.shape[2]) for u in step.units),

@@ -38,6 +38,7 @@ struct SymArgs {
     int32_t* idx;
     double* loss;
     uint8_t* packed;
+    GroupIndex gi;
     int n1, n2;
     float r_lo;          // smallest ratio of either stage
     float r1[32];
@@ -103,7 +104,9 @@ k_search_int3(const __grid_constant__ SymArgs a) {
 
     for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total;
          gid += static_cast<int64_t>(gridDim.x) * SYM_WARPS) {
-        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
+        uint32_t e32, o32, k32;
+        a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
+        const int64_t e = e32, o = o32, k = k32;
         const int64_t j0 = k << 6;
         const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
         const T* wp = W + e * a.ms + o * a.ld + j0;
@@ -320,6 +323,8 @@ tq_status launch_search_int3(const tq_mat* W, const float* m, int64_t m_stride,
 
     const int64_t G = (W->cols + 63) / 64;
     const int64_t total = W->n_mat * W->rows * G;
+    if (total >= (int64_t(1) << 32)) return set_error(TQ_ERR_UNSUPPORTED, "int3 search: more than 2^32 groups");
+    a.gi = GroupIndex(W->rows, G);
     int bpsm = 0;
     const bool bf16 = W->dtype == TQ_BF16;
     if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int3<uint16_t>, SYM_WARPS * 32, 0);

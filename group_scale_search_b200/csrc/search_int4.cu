@@ -47,6 +47,7 @@ struct AsymArgs {
     int32_t* idx;
     double* loss;
     uint8_t* packed;
+    GroupIndex gi;
     int ns, nz;
     int zfirst[16];      // lowest i with z_i = z
     int8_t zval[64];     // z_i for i < nz (nz <= 64)
@@ -130,7 +131,9 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
 
     for (int64_t gid = static_cast<int64_t>(blockIdx.x) * ASYM_WARPS + wid; gid < total;
          gid += static_cast<int64_t>(gridDim.x) * ASYM_WARPS) {
-        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
+        uint32_t e32, o32, k32;
+        a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
+        const int64_t e = e32, o = o32, k = k32;
         const int64_t j0 = k << 7;
         const int n = static_cast<int>(min(static_cast<int64_t>(128), a.I - j0));
         const T* wp = W + e * a.ms + o * a.ld + j0;
@@ -345,6 +348,8 @@ tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
 
     const int64_t G = (W->cols + 127) / 128;
     const int64_t total = W->n_mat * W->rows * G;
+    if (total >= (int64_t(1) << 32)) return set_error(TQ_ERR_UNSUPPORTED, "int4 search: more than 2^32 groups");
+    a.gi = GroupIndex(W->rows, G);
     int bpsm = 0;
     const bool bf16 = W->dtype == TQ_BF16;
     if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t>, ASYM_WARPS * 32, 0);

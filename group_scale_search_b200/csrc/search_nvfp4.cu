@@ -11,17 +11,26 @@
 //   codes c = E2M1 round-to-nearest-even (saturating) of |w| / S, sign apart;
 //   L = sum_j m_j (|w_j| - S dec(c_j))^2; ties keep the lower code.
 //
-// B200 mapping: a half-warp per block, lane = one window code; each warp
-// works on two blocks at a time.  E2M1 rounding is done in the FMA pipe by
-// adding and subtracting a binade-dependent power of two.  Near ties are
-// re-ranked in fp64 with codes from the IEEE quotient.
+// B200 mapping: one lane per 16-weight block.  A lane loads its block's
+// weights (two 16-byte loads) and imatrix (four) into registers, finds the
+// window start by a binary search of exact fp64 predicates, and loops over the
+// window codes with the block in registers: per candidate-element one packed
+// fp32x2 multiply, an AND and an add-then-max (DPX) to form the E2M1 rounding
+// constant, a packed add and FMA that round, a min that saturates, and packed
+// FMA/multiply/FMA for the weighted square -- two elements per packed
+// instruction.  Candidates whose fp32 loss is within a relative 2^-15 of the
+// lane's best are queued; half-warps then re-rank each queued block in fp64
+// with codes from the IEEE quotient (one lane per element), which decides the
+// winner exactly as the definition does.  The winner's codes are rounded
+// from the IEEE quotient and packed into the block's 8 bytes by the lane.
 #include "group_pack.cuh"
 
 #include <climits>
 
 namespace tq {
 
-constexpr int FP4_WARPS = 8;
+constexpr int FP4_THREADS = 128;
+constexpr int FP4_WARPS = FP4_THREADS / 32;
 constexpr float FWIN = 3.0517578125e-05f;   // 2^-15
 
 struct Fp4Args {
@@ -34,11 +43,12 @@ struct Fp4Args {
     int32_t* idx;
     double* loss;
     uint8_t* packed;
+    GroupIndex gi;
     int window;
 };
 
 // Largest E4M3 code whose value does not exceed t (clamped to [1, 126]); only
-// an estimate is needed (the window search tests 32 positions around it).
+// an estimate is needed (the exact window search brackets it).
 __device__ __forceinline__ int e4m3_floor_code(float t) {
     if (!(t > 0.f)) return 1;
     if (t < 0.015625f) return max(1, static_cast<int>(t * 512.f));
@@ -54,146 +64,231 @@ __device__ __forceinline__ double half_sum_d(double v) {
     return v;
 }
 
-// fp64 loss of block scale S for this lane's element (|w| = aw), summed over
-// the half-warp; codes from the IEEE quotient.
-__device__ __forceinline__ double loss64_fp4(float aw, float mv, float S) {
-    const float y = (S == 0.f) ? 0.f : e2m1_round(__fdiv_rn(aw, S));
-    const double e = __dsub_rn(static_cast<double>(aw), __dmul_rn(static_cast<double>(S), static_cast<double>(y)));
-    return half_sum_d(__dmul_rn(static_cast<double>(mv), __dmul_rn(e, e)));
+// E2M1 rounding of a pair (see e2m1_round): binade constant with an AND and
+// an add-then-max, then a packed add/subtract and a saturating min.
+__device__ __forceinline__ float2 e2m1_round2(float2 x) {
+    const unsigned c0 = __viaddmax_u32(__float_as_uint(x.x) & 0x7f800000u, 0x0b400000u, 0x4ac00000u);
+    const unsigned c1 = __viaddmax_u32(__float_as_uint(x.y) & 0x7f800000u, 0x0b400000u, 0x4ac00000u);
+    const float2 C = make_float2(__uint_as_float(c0), __uint_as_float(c1));
+    const float2 t = __fadd2_rn(x, C);
+    float2 y = __ffma2_rn(C, make_float2(-1.f, -1.f), t);
+    y.x = fminf(y.x, 6.0f);
+    y.y = fminf(y.y, 6.0f);
+    return y;
 }
 
+template <typename T> struct Load16;
+template <> struct Load16<uint16_t> {
+    static __device__ __forceinline__ void go(const uint16_t* p, int n, float w[16]) {
+        if (n == 16) {
+            const uint4 a = __ldg(reinterpret_cast<const uint4*>(p));
+            const uint4 b = __ldg(reinterpret_cast<const uint4*>(p) + 1);
+            const unsigned u[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                w[2 * i] = __uint_as_float(u[i] << 16);
+                w[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = i < n ? bf16_bits_to_f32(__ldg(p + i)) : 0.f;
+        }
+    }
+};
+template <> struct Load16<float> {
+    static __device__ __forceinline__ void go(const float* p, int n, float w[16]) {
+        if (n == 16) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const float4 a = __ldg(reinterpret_cast<const float4*>(p) + i);
+                w[4 * i] = a.x; w[4 * i + 1] = a.y; w[4 * i + 2] = a.z; w[4 * i + 3] = a.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = i < n ? __ldg(p + i) : 0.f;
+        }
+    }
+};
+
 template <typename T>
-__global__ void __launch_bounds__(FP4_WARPS * 32)
+__global__ void __launch_bounds__(FP4_THREADS)
 k_search_nvfp4(const __grid_constant__ Fp4Args a) {
     __shared__ float dec[128];
-    __shared__ __align__(16) float2 blk[FP4_WARPS][2][16];
+    __shared__ float2 qdat[FP4_WARPS][32][17];     // each lane's block (w, m), padded against bank conflicts
+    __shared__ int qres_c[FP4_WARPS][32];
+    __shared__ double qres_l[FP4_WARPS][32];
     for (int i = threadIdx.x; i < 128; i += blockDim.x) dec[i] = e4m3_value(i);
     __syncthreads();
 
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int half = lane >> 4, hl = lane & 15;
-    const unsigned hbits = half ? 0xffff0000u : 0x0000ffffu;
     const int64_t G = (a.I + 15) >> 4;
-    const int64_t OG = a.O * G;
-    const int64_t total = a.n_mat * OG;
+    const int64_t total = a.n_mat * a.O * G;
     const int Wn = a.window;
     const int lo_max = 127 - Wn;   // window [lo, lo + Wn - 1] inside codes 1..126
     const T* W = static_cast<const T*>(a.W);
-    const float4* mine4 = reinterpret_cast<const float4*>(blk[wid][half]);
 
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * FP4_WARPS + wid) * 2; base < total;
-         base += static_cast<int64_t>(gridDim.x) * FP4_WARPS * 2) {
-        const int64_t bid = base + half;
+    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * FP4_WARPS + wid) * 32; base < total;
+         base += static_cast<int64_t>(gridDim.x) * FP4_THREADS) {
+        const int64_t bid = base + lane;
         const bool vb = bid < total;
-        int64_t e = 0, o = 0, kb = 0;
-        if (vb) { e = bid / OG; const int64_t rem = bid - e * OG; o = rem / G; kb = rem - o * G; }
-        const int64_t j0 = kb << 4;
-        const int n = vb ? static_cast<int>(min(static_cast<int64_t>(16), a.I - j0)) : 0;
-        const bool ve = hl < n;
-        const float w = ve ? Elem<T>::load(W + e * a.ms + o * a.ld + j0 + hl) : 0.f;
-        const float mv = ve ? __ldg(a.m + e * a.m_stride + j0 + hl) : 0.f;
-        const float aw = fabsf(w);
-        float amax = aw;
+        int64_t e = 0, j0 = 0;
+        int n = 0;
+        float w[16], mv[16];
+        if (vb) {
+            uint32_t e32, o32, k32;
+            a.gi.split(static_cast<uint32_t>(bid), e32, o32, k32);
+            e = e32;
+            j0 = static_cast<int64_t>(k32) << 4;
+            n = static_cast<int>(min(static_cast<int64_t>(16), a.I - j0));
+            Load16<T>::go(W + e * a.ms + static_cast<int64_t>(o32) * a.ld + j0, n, w);
+            const float* mp = a.m + e * a.m_stride + j0;
+            if (n == 16) {
 #pragma unroll
-        for (int off = 8; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, off));
+                for (int i = 0; i < 4; ++i) {
+                    const float4 q = __ldg(reinterpret_cast<const float4*>(mp) + i);
+                    mv[4 * i] = q.x; mv[4 * i + 1] = q.y; mv[4 * i + 2] = q.z; mv[4 * i + 3] = q.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) mv[i] = i < n ? __ldg(mp + i) : 0.f;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) { w[i] = 0.f; mv[i] = 0.f; }
+        }
+        float amax = 0.f, mmax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) { amax = fmaxf(amax, fabsf(w[i])); mmax = fmaxf(mmax, fabsf(mv[i])); }
         const float g = vb ? __ldg(a.g + e) : 0.f;
         const bool degen = (amax == 0.f) || (g == 0.f);
-
-        // fp32 ranking works on |w|, m scaled by exact powers of two
-        const float pw = amax > 0.f ? pow2_inv_binade(amax) : 1.f;
-        float mmax = fabsf(mv);
+        __syncwarp();   // the previous iteration's readers are done with qdat
 #pragma unroll
-        for (int off = 8; off; off >>= 1) mmax = fmaxf(mmax, __shfl_xor_sync(FULL, mmax, off));
-        const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
-        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
-        __syncwarp();
-        blk[wid][half][hl] = make_float2(__fmul_rn(aw, pw), __fmul_rn(mv, pm));
-        __syncwarp();
+        for (int i = 0; i < 16; ++i) qdat[wid][lane][i] = make_float2(w[i], mv[i]);
 
-        // ---- window: first lo with d(lo) <= d(lo + Wn), d(c) = |6 g dec(c) - a| (exact in fp64)
-        const double g6 = 6.0 * static_cast<double>(g), ad = static_cast<double>(amax);
-        const int cdn = e4m3_floor_code(amax / fmaxf(6.f * g, 1e-30f));
-        const int la = min(max(cdn - 16 + hl, 1), lo_max - 1);
-        const int lb = min(max(cdn + hl, 1), lo_max - 1);
-        const bool pa = fabs(__dsub_rn(__dmul_rn(g6, dec[la]), ad)) > fabs(__dsub_rn(__dmul_rn(g6, dec[la + Wn]), ad));
-        const bool pb = fabs(__dsub_rn(__dmul_rn(g6, dec[lb]), ad)) > fabs(__dsub_rn(__dmul_rn(g6, dec[lb + Wn]), ad));
-        const unsigned ba = (__ballot_sync(FULL, pa) & hbits) >> (16 * half);
-        const unsigned bb = (__ballot_sync(FULL, pb) & hbits) >> (16 * half);
-        int lo;
-        if (ba != 0xffffu) lo = min(max(cdn - 16 + (__ffs(~ba) - 1), 1), lo_max - 1);
-        else if (bb != 0xffffu) lo = min(max(cdn + (__ffs(~bb) - 1), 1), lo_max - 1);
-        else lo = min(max(cdn + 16, 1), lo_max);   // every tested start moves right
-
-        // ---- candidate loop: lane hl = code lo + hl
-        const bool act = hl < Wn;
-        const int code = lo + (act ? hl : 0);
-        const float S = __fmul_rn(g, dec[code]);       // the candidate block scale
-        const float Ss = __fmul_rn(S, pw);               // scaled like the block
-        const float invS = __frcp_rn(Ss);
-        float acc = 0.f;
+        int lo = 1, cbest = 0;
+        unsigned winmask = 0u;
+        float Lbest = 0.f;
+        double back = 1.0;
+        if (!degen) {
+            // ---- window start: first lo with d(lo) <= d(lo + Wn), d(c) = |6 g dec(c) - a| (exact in fp64)
+            const double g6 = 6.0 * static_cast<double>(g), ad = static_cast<double>(amax);
+            const int cdn = e4m3_floor_code(amax / fmaxf(6.f * g, 1e-30f));
+            int lo_a = max(1, cdn - 17), hi_a = min(lo_max, cdn + 2);
+            while (lo_a < hi_a) {
+                const int mid = (lo_a + hi_a) >> 1;
+                const bool p = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(dec[mid])), ad)) >
+                               fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(dec[mid + Wn])), ad));
+                if (p) lo_a = mid + 1; else hi_a = mid;
+            }
+            lo = lo_a;
+            // ---- fp32 ranking on |w|, m scaled by exact powers of two
+            const float pw = pow2_inv_binade(amax);
+            const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
+            back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
+            float2 aw2[8], mm2[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 p = mine4[j];
-            {
-                const float y = e2m1_round(__fmul_rn(p.x, invS));
-                const float er = __fmaf_rn(-Ss, y, p.x);
-                acc = __fmaf_rn(__fmul_rn(p.y, er), er, acc);
+            for (int i = 0; i < 8; ++i) {
+                aw2[i] = make_float2(__fmul_rn(fabsf(w[2 * i]), pw), __fmul_rn(fabsf(w[2 * i + 1]), pw));
+                mm2[i] = make_float2(__fmul_rn(mv[2 * i], pm), __fmul_rn(mv[2 * i + 1], pm));
             }
-            {
-                const float y = e2m1_round(__fmul_rn(p.z, invS));
-                const float er = __fmaf_rn(-Ss, y, p.z);
-                acc = __fmaf_rn(__fmul_rn(p.w, er), er, acc);
+            float L[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+                const int code = lo + (c < Wn ? c : 0);
+                const float S = __fmul_rn(__fmul_rn(g, dec[code]), pw);
+                const float inv = __frcp_rn(S);
+                const float2 S2 = make_float2(-S, -S), inv2 = make_float2(inv, inv);
+                float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float2 y = e2m1_round2(__fmul2_rn(aw2[i], inv2));
+                    const float2 er = __ffma2_rn(S2, y, aw2[i]);
+                    acc = __ffma2_rn(__fmul2_rn(mm2[i], er), er, acc);
+                }
+                L[c] = c < Wn ? __fadd_rn(acc.x, acc.y) : __int_as_float(0x7f800000);
             }
+            Lbest = L[0];
+#pragma unroll
+            for (int c = 1; c < 16; ++c)
+                if (L[c] < Lbest) { Lbest = L[c]; cbest = c; }
+            const float thr = __fmaf_rn(Lbest, FWIN, Lbest);
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                if (L[c] <= thr) winmask |= 1u << c;
         }
-        float L = (act && !degen) ? acc : __int_as_float(0x7f800000);
-        int ci = (act && !degen) ? code : INT_MAX;
-        const float Lmine = L;
-        group_argmin(L, ci, FULL, 16);
-        const float thr = __fmaf_rn(L, FWIN, L);
-        unsigned win = (__ballot_sync(FULL, act && !degen && Lmine <= thr) & hbits) >> (16 * half);
-        double lossd = static_cast<double>(L) * back;
-        // near ties: both halves walk their in-window candidates in code order
-        int nwin = __popc(win);
-        const bool need = nwin > 1;
-        double best = __longlong_as_double(0x7ff0000000000000ll);
-        int bcode = ci;
-        unsigned todo = need ? win : 0u;
-        while (__any_sync(FULL, todo != 0u)) {
-            const int pos = todo ? __ffs(todo) - 1 : 0;
-            const float Sc = __shfl_sync(FULL, S, (half << 4) + pos);
-            const double Ld = loss64_fp4(aw, mv, Sc);
-            if (todo) {
-                if (Ld < best) { best = Ld; bcode = lo + pos; }
-                todo &= todo - 1;
-            }
-        }
-        if (need) { ci = bcode; lossd = best; }
-        if (!degen && (ci < lo || ci >= lo + Wn)) ci = lo;   // every loss non-finite
 
-        // ---- outputs and exact RTN + pack
-        const int src = (half << 4) + (degen ? 0 : (ci - lo));
-        const float Sf = __shfl_sync(FULL, S, src);
-        double dl = 0.0;
-        if (__any_sync(FULL, degen)) {
-            const double wd = static_cast<double>(w);
-            dl = half_sum_d(__dmul_rn(static_cast<double>(mv), __dmul_rn(wd, wd)));
+        // ---- near ties: half-warps re-rank queued blocks in fp64, candidates in code order
+        const bool need = __popc(winmask) > 1;
+        unsigned queue = __ballot_sync(FULL, need);
+        if (queue) {
+            __syncwarp();
+            while (queue) {
+                const int own0 = __ffs(queue) - 1;
+                queue &= queue - 1;
+                const int own1 = queue ? __ffs(queue) - 1 : -1;
+                if (own1 >= 0) queue &= queue - 1;
+                const int own = half ? own1 : own0;
+                const int src = own >= 0 ? own : own0;
+                const unsigned omask = __shfl_sync(FULL, winmask, src);
+                const int olo = __shfl_sync(FULL, lo, src);
+                const float og = __shfl_sync(FULL, g, src);
+                float2 d = qdat[wid][src][hl];
+                d.x = fabsf(d.x);
+                unsigned todo = own >= 0 ? omask : 0u;
+                double best = __longlong_as_double(0x7ff0000000000000ll);
+                int bc = 0;
+                while (__any_sync(FULL, todo != 0u)) {
+                    const int c = todo ? __ffs(todo) - 1 : 0;
+                    const float Sc = __fmul_rn(og, dec[olo + c]);
+                    const float y = e2m1_round(__fdiv_rn(d.x, Sc));
+                    const double er = __dsub_rn(static_cast<double>(d.x),
+                                                __dmul_rn(static_cast<double>(Sc), static_cast<double>(y)));
+                    const double Ld = half_sum_d(__dmul_rn(static_cast<double>(d.y), __dmul_rn(er, er)));
+                    if (todo) {
+                        if (Ld < best) { best = Ld; bc = c; }
+                        todo &= todo - 1;
+                    }
+                }
+                if (own >= 0 && hl == 0) { qres_c[wid][own] = bc; qres_l[wid][own] = best; }
+            }
+            __syncwarp();
         }
-        unsigned c4 = 0u;
-        if (!degen && aw != 0.f) {
-            const int mag = e2m1_mag_code(e2m1_round(__fdiv_rn(aw, Sf)));
-            c4 = static_cast<unsigned>(mag) | ((mag != 0 && w < 0.f) ? 8u : 0u);
-        }
-        if (vb && hl == 0) {
-            a.scales[bid] = degen ? 0 : static_cast<uint8_t>(ci);
-            if (a.idx) a.idx[bid] = degen ? -1 : ci;
-            if (a.loss) a.loss[bid] = degen ? dl : lossd;
-        }
-        if (a.packed) {
-            unsigned v = (c4 & 15u) << (4u * static_cast<unsigned>(hl & 7));
-            v |= __shfl_xor_sync(FULL, v, 1);
-            v |= __shfl_xor_sync(FULL, v, 2);
-            v |= __shfl_xor_sync(FULL, v, 4);
-            if (vb && (hl & 7) == 0) reinterpret_cast<uint32_t*>(a.packed + bid * 8)[hl >> 3] = v;
+
+        double lossd;
+        if (need) { cbest = qres_c[wid][lane]; lossd = qres_l[wid][lane]; }
+        else lossd = static_cast<double>(Lbest) * back;
+
+        // ---- outputs and exact RTN + pack of the lane's block
+        if (vb) {
+            const int code = lo + cbest;
+            uint32_t wd0 = 0u, wd1 = 0u;
+            if (!degen) {
+                const float Sf = __fmul_rn(g, dec[code]);
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float wi = qdat[wid][lane][i].x;
+                    const float aw = fabsf(wi);
+                    unsigned c4 = 0u;
+                    if (aw != 0.f) {
+                        const int mag = e2m1_mag_code(e2m1_round(__fdiv_rn(aw, Sf)));
+                        c4 = static_cast<unsigned>(mag) | ((mag != 0 && wi < 0.f) ? 8u : 0u);
+                    }
+                    if (i < 8) wd0 |= c4 << (4 * i); else wd1 |= c4 << (4 * (i - 8));
+                }
+            } else {
+                lossd = 0.0;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float2 d = qdat[wid][lane][i];
+                    const double wdv = static_cast<double>(d.x);
+                    lossd = __dadd_rn(lossd, __dmul_rn(static_cast<double>(d.y), __dmul_rn(wdv, wdv)));
+                }
+            }
+            a.scales[bid] = degen ? 0 : static_cast<uint8_t>(code);
+            if (a.idx) a.idx[bid] = degen ? -1 : code;
+            if (a.loss) a.loss[bid] = lossd;
+            if (a.packed) *reinterpret_cast<uint2*>(a.packed + bid * 8) = make_uint2(wd0, wd1);
         }
     }
 }
@@ -224,15 +319,17 @@ tq_status launch_search_nvfp4(const tq_mat* W, const float* m, int64_t m_stride,
     a.window = p->fp4_window;
     const int64_t G = (W->cols + 15) / 16;
     const int64_t total = W->n_mat * W->rows * G;
+    if (total >= (int64_t(1) << 32)) return set_error(TQ_ERR_UNSUPPORTED, "nvfp4 search: more than 2^32 blocks");
+    a.gi = GroupIndex(W->rows, G);
     int bpsm = 0;
     const bool bf16 = W->dtype == TQ_BF16;
-    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_nvfp4<uint16_t>, FP4_WARPS * 32, 0);
-    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_nvfp4<float>, FP4_WARPS * 32, 0);
+    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_nvfp4<uint16_t>, FP4_THREADS, 0);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_nvfp4<float>, FP4_THREADS, 0);
     if (bpsm < 1) bpsm = 1;
-    const int64_t need = (total + 2 * FP4_WARPS - 1) / (2 * FP4_WARPS);
+    const int64_t need = (total + FP4_THREADS - 1) / FP4_THREADS;
     const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
-    if (bf16) k_search_nvfp4<uint16_t><<<grid, FP4_WARPS * 32, 0, st>>>(a);
-    else k_search_nvfp4<float><<<grid, FP4_WARPS * 32, 0, st>>>(a);
+    if (bf16) k_search_nvfp4<uint16_t><<<grid, FP4_THREADS, 0, st>>>(a);
+    else k_search_nvfp4<float><<<grid, FP4_THREADS, 0, st>>>(a);
     return check_launch("nvfp4 search");
 }
 

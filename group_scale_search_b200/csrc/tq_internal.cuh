@@ -41,6 +41,41 @@ tq_status check_mat(const tq_mat* X, const char* name);
 
 int num_sms();
 
+// ------------------------------------------------------------------ index arithmetic
+
+// Division of 32-bit unsigned integers by a fixed divisor d >= 1 with a
+// multiply-high and a shift (the round-up method of Granlund and Montgomery,
+// "Division by invariant integers using multiplication", 1994): with
+// s = ceil(log2 d) and m = floor(2^32 (2^s - d) / d) + 1,
+// n / d = (umulhi(n, m) + n) >> s for every 32-bit n.
+struct FastDiv {
+    uint32_t d, m;
+    int s;
+    FastDiv() : d(1), m(1), s(0) {}
+    explicit FastDiv(uint32_t dv) : d(dv ? dv : 1), s(0) {
+        while ((uint64_t(1) << s) < d) ++s;
+        m = static_cast<uint32_t>(((uint64_t(1) << 32) * ((uint64_t(1) << s) - d)) / d + 1);
+    }
+    __device__ __forceinline__ uint32_t div(uint32_t n) const {
+        return static_cast<uint32_t>((static_cast<uint64_t>(__umulhi(n, m)) + n) >> s);
+    }
+};
+
+// Group gid of [n_mat][O][G] -> (matrix, row, group) with 32-bit arithmetic.
+struct GroupIndex {
+    FastDiv og, g;
+    uint32_t OG, G;
+    GroupIndex() : OG(1), G(1) {}
+    GroupIndex(int64_t O, int64_t Gn) : og(static_cast<uint32_t>(O * Gn)), g(static_cast<uint32_t>(Gn)),
+                                         OG(static_cast<uint32_t>(O * Gn)), G(static_cast<uint32_t>(Gn)) {}
+    __device__ __forceinline__ void split(uint32_t gid, uint32_t& e, uint32_t& o, uint32_t& k) const {
+        e = og.div(gid);
+        const uint32_t rem = gid - e * OG;
+        o = g.div(rem);
+        k = rem - o * G;
+    }
+};
+
 // ------------------------------------------------------------------ device helpers
 
 constexpr unsigned FULL = 0xffffffffu;
