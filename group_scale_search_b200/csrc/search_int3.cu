@@ -45,30 +45,39 @@ struct SymArgs {
     float r2[32 * 32];   // [k*][i]
 };
 
-__device__ __forceinline__ float err_free(float w, float m, float s, float inv, float acc) {
-    const float t = __fmaf_rn(w, inv, MAGIC);
-    const float q = __fsub_rn(t, MAGIC);
-    const float e = __fmaf_rn(-s, q, w);
-    return __fmaf_rn(__fmul_rn(m, e), e, acc);
+// Two elements (w2, m2) under magnitude s, no clamp possible: the rounded
+// quotient, the residual and the weighted square as packed fp32x2 ops.
+__device__ __forceinline__ float2 err_free2(float2 w2, float2 m2, float2 ns2, float2 inv2, float2 acc) {
+    const float2 t = __ffma2_rn(w2, inv2, make_float2(MAGIC, MAGIC));
+    const float2 q = __fadd2_rn(t, make_float2(-MAGIC, -MAGIC));
+    const float2 e = __ffma2_rn(ns2, q, w2);
+    return __ffma2_rn(__fmul2_rn(m2, e), e, acc);
 }
 
-// One element under +s and -s (magnitude s): the rounded quotient is shared,
-// only the clamp differs ([-4, 3] for +s, which is [-3, 4] in units of -s).
-__device__ __forceinline__ void err_both(float w, float m, float s, float inv, float& accP, float& accN) {
-    const float t = __fmaf_rn(w, inv, MAGIC);
-    const float qp = __fsub_rn(fminf(fmaxf(t, MAGIC - 4.f), MAGIC + 3.f), MAGIC);
-    const float qn = __fsub_rn(fminf(fmaxf(t, MAGIC - 3.f), MAGIC + 4.f), MAGIC);
-    const float ep = __fmaf_rn(-s, qp, w);
-    const float en = __fmaf_rn(-s, qn, w);
-    accP = __fmaf_rn(__fmul_rn(m, ep), ep, accP);
-    accN = __fmaf_rn(__fmul_rn(m, en), en, accN);
+// Two elements under +s and -s: the rounded quotient is shared, only the
+// clamp differs ([-4, 3] for +s, which is [-3, 4] in units of -s).
+__device__ __forceinline__ void err_both2(float2 w2, float2 m2, float2 ns2, float2 inv2, float2& accP, float2& accN) {
+    const float2 t = __ffma2_rn(w2, inv2, make_float2(MAGIC, MAGIC));
+    float2 tp, tn;
+    tp.x = fminf(fmaxf(t.x, MAGIC - 4.f), MAGIC + 3.f);
+    tp.y = fminf(fmaxf(t.y, MAGIC - 4.f), MAGIC + 3.f);
+    tn.x = fminf(fmaxf(t.x, MAGIC - 3.f), MAGIC + 4.f);
+    tn.y = fminf(fmaxf(t.y, MAGIC - 3.f), MAGIC + 4.f);
+    const float2 qp = __fadd2_rn(tp, make_float2(-MAGIC, -MAGIC));
+    const float2 qn = __fadd2_rn(tn, make_float2(-MAGIC, -MAGIC));
+    const float2 ep = __ffma2_rn(ns2, qp, w2);
+    const float2 en = __ffma2_rn(ns2, qn, w2);
+    accP = __ffma2_rn(__fmul2_rn(m2, ep), ep, accP);
+    accN = __ffma2_rn(__fmul2_rn(m2, en), en, accN);
 }
 
-__device__ __forceinline__ float err_clamped(float w, float m, float s, float inv, float lo, float hi, float acc) {
-    const float t = fminf(fmaxf(__fmaf_rn(w, inv, MAGIC), lo), hi);
-    const float q = __fsub_rn(t, MAGIC);
-    const float e = __fmaf_rn(-s, q, w);
-    return __fmaf_rn(__fmul_rn(m, e), e, acc);
+__device__ __forceinline__ float2 err_clamped2(float2 w2, float2 m2, float2 ns2, float2 inv2, float lo, float hi, float2 acc) {
+    float2 t = __ffma2_rn(w2, inv2, make_float2(MAGIC, MAGIC));
+    t.x = fminf(fmaxf(t.x, lo), hi);
+    t.y = fminf(fmaxf(t.y, lo), hi);
+    const float2 q = __fadd2_rn(t, make_float2(-MAGIC, -MAGIC));
+    const float2 e = __ffma2_rn(ns2, q, w2);
+    return __ffma2_rn(__fmul2_rn(m2, e), e, acc);
 }
 
 // fp64 loss of signed scale s over the warp's 64 elements (lane: l, l + 32),
@@ -86,7 +95,7 @@ template <typename T>
 __global__ void __launch_bounds__(SYM_WARPS * 32)
 k_search_int3(const __grid_constant__ SymArgs a) {
     __shared__ float r2s[32 * 32];
-    __shared__ __align__(16) float2 lists[SYM_WARPS][2][64];
+    __shared__ __align__(16) float lists[SYM_WARPS][2][2][64];   // [warp][small|large][w|m][element]
 
     for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x) r2s[i] = a.r2[i];
     __syncthreads();
@@ -97,8 +106,10 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const int64_t total = a.n_mat * OG;
     const bool act1 = lane < a.n1, act2 = lane < a.n2;
     const float r1v = a.r1[act1 ? lane : 0];
-    float2* small = lists[wid][0];
-    float2* large = lists[wid][1];
+    float* smw = lists[wid][0][0];
+    float* smm = lists[wid][0][1];
+    float* lgw = lists[wid][1][0];
+    float* lgm = lists[wid][1][1];
     const T* W = static_cast<const T*>(a.W);
     const unsigned lt = (1u << lane) - 1u;
 
@@ -133,7 +144,6 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float pw = pow2_inv_binade(M);
         const float mmax = warp_max_abs(m0, m1);
         const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
-        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
         const float Ms = __fmul_rn(M, pw);
         const float x0 = __fmul_rn(w0, pw), x1 = __fmul_rn(w1, pw);
         const float n0 = __fmul_rn(m0, pm), n1v = __fmul_rn(m1, pm);
@@ -149,34 +159,33 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const int nl0 = __popc(bl0), nl = nl0 + __popc(bl1);
         const int ns_pad = (ns + 3) & ~3, nl_pad = (nl + 1) & ~1;
         __syncwarp();   // previous group's readers are done with the lists
-        if (sm0) small[__popc(bs0 & lt)] = make_float2(x0, n0);
-        if (sm1) small[ns0 + __popc(bs1 & lt)] = make_float2(x1, n1v);
-        if (lg0) large[__popc(bl0 & lt)] = make_float2(x0, n0);
-        if (lg1) large[nl0 + __popc(bl1 & lt)] = make_float2(x1, n1v);
-        if (lane < ns_pad - ns) small[ns + lane] = make_float2(0.f, 0.f);   // zero pairs add exactly 0
-        if (lane < nl_pad - nl) large[nl + lane] = make_float2(0.f, 0.f);
+        if (sm0) { const int p = __popc(bs0 & lt); smw[p] = x0; smm[p] = n0; }
+        if (sm1) { const int p = ns0 + __popc(bs1 & lt); smw[p] = x1; smm[p] = n1v; }
+        if (lg0) { const int p = __popc(bl0 & lt); lgw[p] = x0; lgm[p] = n0; }
+        if (lg1) { const int p = nl0 + __popc(bl1 & lt); lgw[p] = x1; lgm[p] = n1v; }
+        if (lane < ns_pad - ns) { smw[ns + lane] = 0.f; smm[ns + lane] = 0.f; }   // zero pairs add exactly 0
+        if (lane < nl_pad - nl) { lgw[nl + lane] = 0.f; lgm[nl + lane] = 0.f; }
         __syncwarp();
-        const float4* sp = reinterpret_cast<const float4*>(small);
-        const float4* lp = reinterpret_cast<const float4*>(large);
+        const float4* spw = reinterpret_cast<const float4*>(smw);
+        const float4* spm = reinterpret_cast<const float4*>(smm);
 
         // ---- stage 1: lane = magnitude, both signs
         const float s1 = __fmul_rn(__fmul_rn(r1v, Ms), 0.25f);    // scaled candidate
         const float s1o = __fmul_rn(__fmul_rn(r1v, M), 0.25f);    // the candidate itself
-        const float i1 = __frcp_rn(s1);
-        float accC = 0.f, accP = 0.f, accN = 0.f;
-        for (int j = 0; j < ns_pad; j += 4) {
-            const float4 p = sp[j >> 1], q = sp[(j >> 1) + 1];
-            accC = err_free(p.x, p.y, s1, i1, accC);
-            accC = err_free(p.z, p.w, s1, i1, accC);
-            accC = err_free(q.x, q.y, s1, i1, accC);
-            accC = err_free(q.z, q.w, s1, i1, accC);
+        const float i1 = rcp_approx(s1);
+        const float2 ns1 = make_float2(-s1, -s1), inv1 = make_float2(i1, i1);
+        float2 accC = make_float2(0.f, 0.f), accP = make_float2(0.f, 0.f), accN = make_float2(0.f, 0.f);
+        for (int j = 0; j < (ns_pad >> 2); ++j) {
+            const float4 w4 = spw[j], m4 = spm[j];
+            accC = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns1, inv1, accC);
+            accC = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns1, inv1, accC);
         }
-        for (int j = 0; j < nl_pad; j += 2) {
-            const float4 p = lp[j >> 1];
-            err_both(p.x, p.y, s1, i1, accP, accN);
-            err_both(p.z, p.w, s1, i1, accP, accN);
+        for (int j = 0; j < (nl_pad >> 1); ++j) {
+            const float2 w2 = reinterpret_cast<const float2*>(lgw)[j], m2 = reinterpret_cast<const float2*>(lgm)[j];
+            err_both2(w2, m2, ns1, inv1, accP, accN);
         }
-        const float LP = __fadd_rn(accC, accP), LN = __fadd_rn(accC, accN);
+        const float cC = __fadd_rn(accC.x, accC.y);
+        const float LP = __fadd_rn(cC, __fadd_rn(accP.x, accP.y)), LN = __fadd_rn(cC, __fadd_rn(accN.x, accN.y));
 
         float L = __int_as_float(0x7f800000);
         int bi = INT_MAX;
@@ -212,21 +221,20 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float r2v = r2s[ks * 32 + (act2 ? lane : 0)];
         const float s2 = __fmul_rn(__fmul_rn(r2v, Ms), 0.25f);
         const float s2o = __fmul_rn(__fmul_rn(r2v, M), 0.25f);
-        const float i2 = __frcp_rn(s2);
+        const float i2 = rcp_approx(s2);
         const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
-        float acc2 = 0.f;
-        for (int j = 0; j < ns_pad; j += 4) {
-            const float4 p = sp[j >> 1], q = sp[(j >> 1) + 1];
-            acc2 = err_free(p.x, p.y, s2, i2, acc2);
-            acc2 = err_free(p.z, p.w, s2, i2, acc2);
-            acc2 = err_free(q.x, q.y, s2, i2, acc2);
-            acc2 = err_free(q.z, q.w, s2, i2, acc2);
+        const float2 ns2 = make_float2(-s2, -s2), inv2 = make_float2(i2, i2);
+        float2 a2 = make_float2(0.f, 0.f);
+        for (int j = 0; j < (ns_pad >> 2); ++j) {
+            const float4 w4 = spw[j], m4 = spm[j];
+            a2 = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns2, inv2, a2);
+            a2 = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns2, inv2, a2);
         }
-        for (int j = 0; j < nl_pad; j += 2) {
-            const float4 p = lp[j >> 1];
-            acc2 = err_clamped(p.x, p.y, s2, i2, clo, chi, acc2);
-            acc2 = err_clamped(p.z, p.w, s2, i2, clo, chi, acc2);
+        for (int j = 0; j < (nl_pad >> 1); ++j) {
+            const float2 w2 = reinterpret_cast<const float2*>(lgw)[j], m2 = reinterpret_cast<const float2*>(lgm)[j];
+            a2 = err_clamped2(w2, m2, ns2, inv2, clo, chi, a2);
         }
+        const float acc2 = __fadd_rn(a2.x, a2.y);
         const float L1f = __shfl_sync(FULL, sg ? LN : LP, ks);   // incumbent's fp32 loss
         const float L2 = act2 ? acc2 : __int_as_float(0x7f800000);
         float L2m = L2;
@@ -259,9 +267,9 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             bf = bidx;
             lossd = best;
         } else if (L2m < L1f) {
-            bf = b2; lossd = static_cast<double>(L2m) * back;
+            bf = b2; lossd = static_cast<double>(L2m) * inv_pow2_sq(pw, pm);
         } else {
-            bf = b1; lossd = have64 ? L1d : static_cast<double>(L1f) * back;
+            bf = b1; lossd = have64 ? L1d : static_cast<double>(L1f) * inv_pow2_sq(pw, pm);
         }
 
         if (bf < 0 || bf >= 2 * a.n1 + a.n2) bf = b1;

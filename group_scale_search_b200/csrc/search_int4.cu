@@ -183,7 +183,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         for (int i = 0; i < 4; ++i) mloc = fmaxf(mloc, fabsf(mv[i]));
         const float mmax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(mloc)));
         const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
-        const double back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
+        const double back = inv_pow2_sq(pw, pm);
         const float Rs = __fmul_rn(R, pw);
         // split by sign: negative weights first, non-negative after (tail: (0, 0))
         float x[4], sq[4];
@@ -220,7 +220,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
 
         const float sA = __fmul_rn(cA, Rs), sB = __fmul_rn(cB, Rs);
         const float sAo = __fmul_rn(cA, R), sBo = __fmul_rn(cB, R);
-        const float iA = __frcp_rn(sA), iB = __frcp_rn(sB);
+        const float iA = rcp_approx(sA), iB = rcp_approx(sB);
         float2 a2[8], b2[8];
 #pragma unroll
         for (int p = 0; p < 8; ++p) { a2[p] = make_float2(0.f, 0.f); b2[p] = make_float2(0.f, 0.f); }

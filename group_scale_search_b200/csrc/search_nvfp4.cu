@@ -185,7 +185,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             // ---- fp32 ranking on |w|, m scaled by exact powers of two
             const float pw = pow2_inv_binade(amax);
             const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
-            back = 1.0 / (static_cast<double>(pw) * static_cast<double>(pw) * static_cast<double>(pm));
+            back = inv_pow2_sq(pw, pm);
             float2 aw2[8], mm2[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
@@ -197,7 +197,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             for (int c = 0; c < 16; ++c) {
                 const int code = lo + (c < Wn ? c : 0);
                 const float S = __fmul_rn(__fmul_rn(g, dec[code]), pw);
-                const float inv = __frcp_rn(S);
+                const float inv = rcp_approx(S);
                 const float2 S2 = make_float2(-S, -S), inv2 = make_float2(inv, inv);
                 float2 acc = make_float2(0.f, 0.f);
 #pragma unroll

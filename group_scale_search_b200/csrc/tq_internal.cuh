@@ -140,6 +140,21 @@ __device__ __forceinline__ float warp_max_abs(float a, float b) {
     return __uint_as_float(__reduce_max_sync(FULL, u));
 }
 
+// Approximate reciprocal (hardware, within 1 ulp).  Used only where a value
+// ranks candidates in fp32; every decision it could flip is re-taken in fp64.
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// 1 / (pw^2 pm) for powers of two pw, pm (exact in fp64, no division).
+__device__ __forceinline__ double inv_pow2_sq(float pw, float pm) {
+    const int ew = static_cast<int>((__float_as_uint(pw) >> 23) & 255u) - 127;
+    const int em = static_cast<int>((__float_as_uint(pm) >> 23) & 255u) - 127;
+    return __longlong_as_double(static_cast<long long>(1023 - 2 * ew - em) << 52);
+}
+
 // Integer code of w under scale s: round half to even of the IEEE fp32
 // quotient w/s, clamped to [lo, hi]; scale 0 gives code 0.
 __device__ __forceinline__ float rtn_exact(float w, float s, float lo, float hi) {
