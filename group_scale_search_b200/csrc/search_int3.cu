@@ -113,20 +113,32 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const T* W = static_cast<const T*>(a.W);
     const unsigned lt = (1u << lane) - 1u;
 
-    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total;
-         gid += static_cast<int64_t>(gridDim.x) * SYM_WARPS) {
+    // the next group's weights and imatrix are loaded while this one is searched
+    const int64_t gstride = static_cast<int64_t>(gridDim.x) * SYM_WARPS;
+    float pw0 = 0.f, pw1 = 0.f, pm0 = 0.f, pm1 = 0.f;
+    auto fetch = [&](int64_t g, float& a0, float& a1, float& b0, float& b1) {
+        uint32_t e32, o32, k32;
+        a.gi.split(static_cast<uint32_t>(g), e32, o32, k32);
+        const int64_t j0 = static_cast<int64_t>(k32) << 6;
+        const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
+        const T* wp = W + static_cast<int64_t>(e32) * a.ms + static_cast<int64_t>(o32) * a.ld + j0;
+        const float* mp = a.m + static_cast<int64_t>(e32) * a.m_stride + j0;
+        a0 = lane < n ? Elem<T>::load(wp + lane) : 0.f;
+        a1 = lane + 32 < n ? Elem<T>::load(wp + lane + 32) : 0.f;
+        b0 = lane < n ? __ldg(mp + lane) : 0.f;
+        b1 = lane + 32 < n ? __ldg(mp + lane + 32) : 0.f;
+    };
+    int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid;
+    if (gid < total) fetch(gid, pw0, pw1, pm0, pm1);
+    for (; gid < total; gid += gstride) {
+        const float w0 = pw0, w1 = pw1, m0 = pm0, m1 = pm1;
+        if (gid + gstride < total) fetch(gid + gstride, pw0, pw1, pm0, pm1);
         uint32_t e32, o32, k32;
         a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
-        const int64_t e = e32, o = o32, k = k32;
+        const int64_t k = k32;
         const int64_t j0 = k << 6;
         const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
-        const T* wp = W + e * a.ms + o * a.ld + j0;
-        const float* mp = a.m + e * a.m_stride + j0;
         const bool v0 = lane < n, v1 = lane + 32 < n;
-        const float w0 = v0 ? Elem<T>::load(wp + lane) : 0.f;
-        const float w1 = v1 ? Elem<T>::load(wp + lane + 32) : 0.f;
-        const float m0 = v0 ? __ldg(mp + lane) : 0.f;
-        const float m1 = v1 ? __ldg(mp + lane + 32) : 0.f;
         const float M = warp_max_abs(w0, w1);
         uint8_t* rec = a.packed ? a.packed + gid * 24 : nullptr;
 
@@ -287,8 +299,9 @@ k_search_int3(const __grid_constant__ SymArgs a) {
             if (a.loss) a.loss[gid] = lossd;
         }
         if (rec) {
-            const unsigned u0 = static_cast<unsigned>(static_cast<int>(rtn_exact(w0, sfin, -4.f, 3.f)) + 4);
-            const unsigned u1 = static_cast<unsigned>(static_cast<int>(rtn_exact(w1, sfin, -4.f, 3.f)) + 4);
+            const float invf = rcp_approx(sfin);
+            const unsigned u0 = static_cast<unsigned>(static_cast<int>(rtn_fast(w0, sfin, invf, -4.f, 3.f)) + 4);
+            const unsigned u1 = static_cast<unsigned>(static_cast<int>(rtn_fast(w1, sfin, invf, -4.f, 3.f)) + 4);
             pack_int3_record(u0, u1, lane, rec);
         }
     }

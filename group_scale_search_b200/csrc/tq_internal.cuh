@@ -163,6 +163,18 @@ __device__ __forceinline__ float rtn_exact(float w, float s, float lo, float hi)
     return fminf(fmaxf(y, lo), hi);
 }
 
+// Same code as rtn_exact(w, s, lo, hi) given inv = rcp_approx(s): the
+// approximate quotient w * inv lies within 2^-21 |q| of the IEEE quotient q,
+// so their rounded codes agree unless it is within 2^-20 |q| of a
+// half-integer; only then is the IEEE quotient formed.
+__device__ __forceinline__ float rtn_fast(float w, float s, float inv, float lo, float hi) {
+    if (s == 0.0f) return 0.0f;
+    const float y = __fmul_rn(w, inv);
+    float r = rintf(y);
+    if (fabsf(__fsub_rn(y, r)) >= 0.5f - fabsf(y) * 9.5367431640625e-07f) r = rintf(__fdiv_rn(w, s));
+    return fminf(fmaxf(r, lo), hi);
+}
+
 // E2M1 round-to-nearest-even with saturation of y >= 0, returned as its value
 // in {0, .5, 1, 1.5, 2, 3, 4, 6}.  The spacing of E2M1 values at y is half
 // the power of two at or below max(y, 1); adding and subtracting 1.5 * 2^22
