@@ -113,9 +113,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const T* W = static_cast<const T*>(a.W);
     const unsigned lt = (1u << lane) - 1u;
 
-    // the next group's weights and imatrix are loaded while this one is searched
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * SYM_WARPS;
-    float pw0 = 0.f, pw1 = 0.f, pm0 = 0.f, pm1 = 0.f;
     auto fetch = [&](int64_t g, float& a0, float& a1, float& b0, float& b1) {
         uint32_t e32, o32, k32;
         a.gi.split(static_cast<uint32_t>(g), e32, o32, k32);
@@ -128,11 +126,9 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         b0 = lane < n ? __ldg(mp + lane) : 0.f;
         b1 = lane + 32 < n ? __ldg(mp + lane + 32) : 0.f;
     };
-    int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid;
-    if (gid < total) fetch(gid, pw0, pw1, pm0, pm1);
-    for (; gid < total; gid += gstride) {
-        const float w0 = pw0, w1 = pw1, m0 = pm0, m1 = pm1;
-        if (gid + gstride < total) fetch(gid + gstride, pw0, pw1, pm0, pm1);
+    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total; gid += gstride) {
+        float w0, w1, m0, m1;
+        fetch(gid, w0, w1, m0, m1);
         uint32_t e32, o32, k32;
         a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
         const int64_t k = k32;

@@ -265,30 +265,13 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             uint32_t wd0 = 0u, wd1 = 0u;
             if (!degen) {
                 const float Sf = __fmul_rn(g, dec[code]);
-                const float invf = rcp_approx(Sf);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const float wi = qdat[wid][lane][i].x;
                     const float aw = fabsf(wi);
                     unsigned c4 = 0u;
                     if (aw != 0.f) {
-                        // E2M1 code of the IEEE quotient aw / Sf, taken from the
-                        // approximate quotient x (within 2^-21 x of it) unless x lies
-                        // within 2^-20 x of a rounding midpoint; quotients above 6
-                        // saturate either way.
-                        const float x = __fmul_rn(aw, invf);
-                        float y;
-                        if (x > 6.0f) {
-                            y = 6.0f;
-                        } else {
-                            const unsigned cb = __viaddmax_u32(__float_as_uint(x) & 0x7f800000u, 0x0b400000u, 0x4ac00000u);
-                            const float C = __uint_as_float(cb);
-                            y = fminf(__fsub_rn(__fadd_rn(x, C), C), 6.0f);
-                            const float h = __uint_as_float(cb - 0x0c400000u);   // half the E2M1 spacing at x
-                            if (__fsub_rn(h, fabsf(__fsub_rn(x, y))) <= x * 9.5367431640625e-07f)
-                                y = e2m1_round(__fdiv_rn(aw, Sf));
-                        }
-                        const int mag = e2m1_mag_code(y);
+                        const int mag = e2m1_mag_code(e2m1_round(__fdiv_rn(aw, Sf)));
                         c4 = static_cast<unsigned>(mag) | ((mag != 0 && wi < 0.f) ? 8u : 0u);
                     }
                     if (i < 8) wd0 |= c4 << (4 * i); else wd1 |= c4 << (4 * (i - 8));
