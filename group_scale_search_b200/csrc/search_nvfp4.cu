@@ -14,16 +14,16 @@
 // B200 mapping: one lane per 16-weight block.  A lane loads its block's
 // weights (two 16-byte loads) and imatrix (four) into registers, finds the
 // window start by a binary search of exact fp64 predicates, and loops over the
-// window codes with the block in registers: per candidate-element one packed
-// fp32x2 multiply, an AND and an add-then-max (DPX) to form the E2M1 rounding
-// constant, a packed add and FMA that round, a min that saturates, and packed
-// FMA/multiply/FMA for the weighted square -- two elements per packed
-// instruction.  Candidates whose fp32 loss is within a relative 2^-15 of the
+// window codes with the block in registers: per pair of candidate-elements one
+// packed fp32x2 multiply, the hardware E2M1 conversion (round to nearest even,
+// saturating) and back, and packed FMA/multiply/FMA for the weighted square.  Candidates whose fp32 loss is within a relative 2^-15 of the
 // lane's best are queued; half-warps then re-rank each queued block in fp64
 // with codes from the IEEE quotient (one lane per element), which decides the
 // winner exactly as the definition does.  The winner's codes are rounded
 // from the IEEE quotient and packed into the block's 8 bytes by the lane.
 #include "group_pack.cuh"
+
+#include <cuda_fp16.h>
 
 #include <climits>
 
@@ -64,17 +64,14 @@ __device__ __forceinline__ double half_sum_d(double v) {
     return v;
 }
 
-// E2M1 rounding of a pair (see e2m1_round): binade constant with an AND and
-// an add-then-max, then a packed add/subtract and a saturating min.
-__device__ __forceinline__ float2 e2m1_round2(float2 x) {
-    const unsigned c0 = __viaddmax_u32(__float_as_uint(x.x) & 0x7f800000u, 0x0b400000u, 0x4ac00000u);
-    const unsigned c1 = __viaddmax_u32(__float_as_uint(x.y) & 0x7f800000u, 0x0b400000u, 0x4ac00000u);
-    const float2 C = make_float2(__uint_as_float(c0), __uint_as_float(c1));
-    const float2 t = __fadd2_rn(x, C);
-    float2 y = __ffma2_rn(C, make_float2(-1.f, -1.f), t);
-    y.x = fminf(y.x, 6.0f);
-    y.y = fminf(y.y, 6.0f);
-    return y;
+// E2M1 rounding of a pair with the hardware conversions (round to nearest
+// even, saturating at 6): fp32x2 -> packed e2m1x2 -> f16x2 (exact) -> fp32x2.
+// Ranking only; the exact codes come from e2m1_round on the IEEE quotient.
+__device__ __forceinline__ float2 e2m1_round2_hw(float2 x) {
+    unsigned h2;
+    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %2, %1; cvt.rn.f16x2.e2m1x2 %0, t; }"
+        : "=r"(h2) : "f"(x.x), "f"(x.y));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 
 template <typename T> struct Load16;
@@ -202,7 +199,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
                 float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    const float2 y = e2m1_round2(__fmul2_rn(aw2[i], inv2));
+                    const float2 y = e2m1_round2_hw(__fmul2_rn(aw2[i], inv2));
                     const float2 er = __ffma2_rn(S2, y, aw2[i]);
                     acc = __ffma2_rn(__fmul2_rn(mm2[i], er), er, acc);
                 }
