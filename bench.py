@@ -148,6 +148,7 @@ class Step:
             self.ws_px.append(torch.empty(max(16, tq.proxy_workspace_bytes(u.W, fmt)), dtype=torch.uint8,
                                           device=dev))
         self.search_events = []
+        self.row_events = []
 
     def _m_for(self, u):
         m = self.m[u.site]
@@ -162,23 +163,41 @@ class Step:
     def __call__(self, k: int, time_search: bool = False):
         tq = self.tq
         sites, Ws = self.sets[k % len(self.sets)]
+
+        def mark():
+            if not time_search:
+                return None
+            ev = torch.cuda.Event(enable_timing=True)
+            ev.record()
+            return ev
+
         for name in self.m:
             X = sites[name]
+            a = mark()
             tq.tq_imatrix(X, m=self.m[name], alpha=1.0 / X.shape[1], workspace=self.ws_im[name])
+            if time_search:
+                self.row_events.append(("imatrix", X.numel() * X.element_size(), a, mark()))
         for i, (u, fmt) in enumerate(zip(self.units, self.fmts)):
             W = Ws[i]
             m = self._m_for(u)
             E, O, I = W.shape
-            if time_search:
-                a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                a.record()
+            a = mark()
             r = tq.tq_search_groups(W, m, fmt, out=self.res[i])
             if time_search:
-                b.record()
+                b = mark()
                 self.search_events.append((u.fmt, W.numel(), a, b))
             tq.tq_dequant(r.packed, fmt, r.scales, r.zeros, r.global_scale, E, O, I, out=self.dq[i])
+            if time_search:
+                c = mark()
+                self.row_events.append(("dequant", r.packed.numel() + self.dq[i].numel() * 2
+                                        + r.scales.numel() * r.scales.element_size()
+                                        + (0 if r.zeros is None else r.zeros.numel()), b, c))
             tq.tq_proxy_error(W, r.packed, fmt, r.scales, r.zeros, r.global_scale, m, out=self.px[i],
                               workspace=self.ws_px[i])
+            if time_search:
+                self.row_events.append(("proxy", W.numel() * W.element_size() + r.packed.numel()
+                                        + r.scales.numel() * r.scales.element_size()
+                                        + (0 if r.zeros is None else r.zeros.numel()), c, mark()))
 
 
 def make_sets(wl, n_sets):
@@ -277,20 +296,6 @@ def parse():
     return ap.parse_args()
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return world, rank, local
-
-
 def reference_arm(args, world, rank):
     if rank != 0:
         return 0
@@ -319,11 +324,14 @@ def reference_arm(args, world, rank):
 def main():
     args = parse()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
-    world, rank, local = dist_setup(args)
-    if args.impl == "reference":
-        return reference_arm(args, world, rank)
+    if args.impl == "reference":   # rank 0 alone times the oracle; no process group
+        return reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
 
     import group_scale_search_b200 as tq
+    from group_scale_search_b200.dist import init_from_env, max_over_ranks
+    world, rank, local = init_from_env("nccl", timeout_s=120.0)
+    if world == 1:
+        torch.cuda.set_device(0)
     tq.lib()
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = synth.make(args.config, dev, seed=rank, scale=args.scale)
@@ -354,12 +362,7 @@ def main():
         torch.cuda.synchronize()
     barrier()
     torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms / args.steps
     value = world * nw / (ms_step * 1e-3)
 
@@ -389,6 +392,19 @@ def main():
                 if clocks.get("sm_mhz") else None,
                 "cee_per_s": SEARCH_CEE_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3)}
 
+    # every HBM-bound row of the step: algorithmic bytes / CUDA-event time vs the HBM peak
+    rows = {}
+    for name, nbytes, a, b in step.row_events:
+        d = rows.setdefault(name, [0.0, 0])
+        d[0] += a.elapsed_time(b)
+        d[1] += nbytes
+    hbm_rows = {}
+    for name, (t_ms, nbytes) in rows.items():
+        gbs = nbytes / (t_ms * 1e-3) / 1e9
+        hbm_rows[name] = {"ms": t_ms / args.steps, "bytes": nbytes // args.steps, "GB/s": gbs,
+                          "frac": gbs / pk["hbm_gbs"]}
+    hbm_rows["pack"] = time_pack(tq, step, pk)
+
     # end to end through the public API from pinned host buffers
     e2e = None
     if not args.no_e2e:
@@ -408,7 +424,7 @@ def main():
                               f"{n_sets} input sets ({n_sets * nbytes / 2**20:.1f} MiB) fit in L2"),
                        "parallelism": f"weak x{world}: independent workload per GPU"},
             "groups_per_s": value / tq.tq_group_size(tq.FORMATS[fmt_main]),
-            "roofline": roofline, "clocks": clocks, "e2e": e2e,
+            "roofline": roofline, "hbm_rows": hbm_rows, "clocks": clocks, "e2e": e2e,
             "gpu_launches": step.kernels_per_step() * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc, dt = oracle_sample(wl)
@@ -421,6 +437,29 @@ def main():
         dist.barrier()
         dist.destroy_process_group()
     return 0
+
+
+def time_pack(tq, step, pk, reps=10):
+    """tq_pack (RTN + pack with given scales, the stand-alone form of the fused
+    pack) on the first unit, outside the step: bytes = weights read + packed
+    records written + scales (+ zeros) read."""
+    u, r = step.units[0], step.res[0]
+    fmt = tq.FORMATS[u.fmt]
+    out = torch.empty_like(r.packed)
+    nbytes = (u.W.numel() * u.W.element_size() + out.numel() + r.scales.numel() * r.scales.element_size()
+              + (0 if r.zeros is None else r.zeros.numel()))
+    for _ in range(3):
+        tq.tq_pack(u.W, fmt, r.scales, r.zeros, r.global_scale, out=out)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        tq.tq_pack(u.W, fmt, r.scales, r.zeros, r.global_scale, out=out)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
+            "note": "first unit, back-to-back launches (inputs may be L2-resident when smaller than L2)"}
 
 
 def _empty_like_result(tq, r):
@@ -508,12 +547,8 @@ def run_e2e(tq, wl, step, args, world, barrier, dev):
     a, b = run(steps)
     torch.cuda.synchronize()
     barrier()
-    ms = a.elapsed_time(b)
-    if world > 1:
-        import torch.distributed as dist
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    from group_scale_search_b200.dist import max_over_ranks
+    ms = max_over_ranks(a.elapsed_time(b), dev)
     nw = sum(u.W.numel() for u in step.units)
     return {"value": world * nw / (ms / steps * 1e-3), "unit": "weights/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,

@@ -1,0 +1,49 @@
+"""Process bodies for the two-rank gloo tests (spawned; not collected)."""
+import datetime
+import os
+import sys
+
+import numpy as np
+import torch
+import torch.distributed as dist
+
+
+def _init(rank, world, port, timeout_s=20.0):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=timeout_s))
+
+
+def imatrix_shards(rank, world, port, root, out_dir):
+    sys.path.insert(0, root)
+    import oracle
+    import synth
+    from group_scale_search_b200.dist import allreduce_imatrix, max_over_ranks, shard_range
+    _init(rank, world, port)
+    X = synth.make("c1", "cpu", scale=0.0625).sites["x"].X[0].float().numpy()   # same on every rank
+    T = X.shape[0]
+    t0, t1 = shard_range(T, rank, world)
+    local = oracle.imatrix(X[t0:t1]) * (t1 - t0)          # this rank's raw sums of x^2
+    m = allreduce_imatrix(torch.from_numpy(local.astype(np.float32)), T)
+    slowest = max_over_ranks(float(rank + 1))
+    np.save(os.path.join(out_dir, f"m{rank}.npy"), m.numpy())
+    np.save(os.path.join(out_dir, f"t{rank}.npy"), np.array([slowest]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def peer_dies(rank, world, port, out_dir):
+    """Rank 1 leaves before the collective; rank 0 must get an error, not hang."""
+    _init(rank, world, port, timeout_s=8.0)
+    if rank == 1:
+        os._exit(0)
+    t = torch.ones(4)
+    try:
+        dist.all_reduce(t)
+        status = "completed"
+    except Exception as e:   # noqa: BLE001 -- any error is the expected outcome
+        status = "error: " + type(e).__name__
+    with open(os.path.join(out_dir, "status.txt"), "w") as f:
+        f.write(status)
+    os._exit(0)
