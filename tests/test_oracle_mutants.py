@@ -1,0 +1,87 @@
+"""Mutation check of the oracle's pins: a copy of the oracle with one
+plausible mistake planted (a dropped weight, a wrong rounding or tie rule, an
+off-by-one in a grid, a wrong bit order, ...) must fail at least one pin.
+Mistakes are planted only in temporary copies of the oracle, on the CPU."""
+import importlib.util
+import inspect
+import os
+import subprocess
+
+import pytest
+
+import test_oracle_pins as pins
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "tq_oracle.c")
+
+MUTANTS = {
+    "imatrix_weight_dropped": ("L += (double)m[j] * (e * e);\n        if (v_out) v_out[j] = (int8_t)v;",
+                               "L += (e * e);\n        if (v_out) v_out[j] = (int8_t)v;"),
+    "round_half_away": ("double q = nearbyint((double)y); /* current rounding mode", "double q = round((double)y); /* current rounding mode"),
+    "stage2_narrow": ("return (float)((center - delta) + (2.0 * delta", "return (float)((center - 0.5 * delta) + (1.0 * delta"),
+    "int3_offset": ("int u = (j < I ? v[r * I + j] : 0) + 4;", "int u = (j < I ? v[r * I + j] : 0) + 3;"),
+    "int3_high_bit_order": ("rec[16 + i / 8] |= (uint8_t)(((u >> 2) & 1) << (i % 8));", "rec[16 + i / 8] |= (uint8_t)(((u >> 2) & 1) << (7 - i % 8));"),
+    "zero_grid_16": ("return (int)nearbyint((15.0 * (double)i) / (double)(nz - 1));", "return (int)nearbyint((16.0 * (double)i) / (double)(nz - 1));"),
+    "asym_clamp_14": ("if (q > 15.0) q = 15.0;\n        }\n        double e = (double)w[j] - (double)s * (q - (double)z);",
+                      "if (q > 14.0) q = 14.0;\n        }\n        double e = (double)w[j] - (double)s * (q - (double)z);"),
+    "no_sign_flip": ("return negative ? -a : a;", "return a;"),
+    "window_ties_high": ("if (d < bd) { bd = d; best = c; }   /* strict: ties keep the lower code */",
+                         "if (d <= bd) { bd = d; best = c; }   /* strict: ties keep the lower code */"),
+    "e2m1_ties_odd": ("if (d < best_d || (d == best_d && (i % 2) == 0))", "if (d < best_d || (d == best_d && (i % 2) == 1))"),
+    "imatrix_bessel": ("m[j] = T > 0 ? s / (double)T : 0.0;", "m[j] = T > 1 ? s / (double)(T - 1) : 0.0;"),
+    "proxy_den_error": ("b += (double)m[j] * (w * w);", "b += (double)m[j] * (e * e) + (double)m[j] * (w * w) * 0.0 + (double)m[j] * (w * w);"),
+    "argmin_last_tie": ("if (L < bestL) { bestL = L; best = 2 * k + sg; bestS = s; }", "if (L <= bestL) { bestL = L; best = 2 * k + sg; bestS = s; }"),
+    "nvfp4_global_448": ("return (float)((double)amax / 2688.0);", "return (float)((double)amax / 448.0);"),
+    "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
+                             "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
+}
+
+
+def _mutant_module(tmp_path, name, a, b):
+    src = open(SRC).read()
+    assert a in src, f"mutation site of {name} not found"
+    d = tmp_path / name
+    d.mkdir()
+    (d / "tq_oracle.c").write_text(src.replace(a, b, 1))
+    so = d / "liboracle.so"
+    subprocess.run(["gcc", "-O1", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off", "-o", str(so),
+                    str(d / "tq_oracle.c"), "-lm"], check=True)
+    spec = importlib.util.spec_from_file_location(f"oracle_mut_{name}", os.path.join(ROOT, "oracle", "__init__.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod._LIB_PATH = str(so)
+    mod.build = lambda force=False: str(so)
+    return mod
+
+
+def _pin_calls():
+    """Every pin of test_oracle_pins, with its parametrisations, as callables of orc."""
+    calls = []
+    for name, fn in inspect.getmembers(pins, inspect.isfunction):
+        if not name.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if not params:
+            calls.append((name, lambda orc, fn=fn: fn(orc)))
+            continue
+        argnames, values = params[0].args
+        argnames = [s.strip() for s in argnames.split(",")] if isinstance(argnames, str) else list(argnames)
+        for v in values:
+            v = v if isinstance(v, (tuple, list)) and len(argnames) > 1 else (v,)
+            calls.append((f"{name}{v}", lambda orc, fn=fn, v=v: fn(orc, *v)))
+    return calls
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_every_planted_mistake_fails_a_pin(tmp_path, name):
+    a, b = MUTANTS[name]
+    orc = _mutant_module(tmp_path, name, a, b)
+    caught = []
+    for pin, call in _pin_calls():
+        try:
+            call(orc)
+        except (AssertionError, ValueError, IndexError):
+            caught.append(pin)
+            break
+    assert caught, f"no pin catches the planted mistake {name}"

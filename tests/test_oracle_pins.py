@@ -457,6 +457,32 @@ def test_exactly_representable_group_has_zero_loss(orc):
     assert np.array_equal(qq, q.astype(np.uint8))
 
 
+def test_exact_ties_keep_the_lowest_index(orc):
+    """w = [M, -M, 0, ...]: at the largest stage-1 ratio 1.2 no element is
+    clamped for either sign (|w/s| = 3.33 < 3.5), so +s and -s tie exactly and
+    the lower index (+s) must win stage 1; stage 2 then keeps the + sign."""
+    w = np.zeros(64, np.float32)
+    w[0], w[1] = 1.0, -1.0
+    m = np.ones(64, np.float32)
+    r31 = np.float32(np.linspace(0.5, 1.2, 32)[31])
+    s31 = np.float32(np.float32(r31 * np.float32(1.0)) * np.float32(0.25))
+    assert orc.sym_loss(w, m, s31) == orc.sym_loss(w, m, -s31)     # an exact tie
+    # stage 1's best magnitude is the last one (brute force over the grid)
+    r1 = np.linspace(0.5, 1.2, 32).astype(np.float32)
+    L1 = [min(orc.sym_loss(w, m, np.float32(r * np.float32(0.25))), orc.sym_loss(w, m, -np.float32(r * np.float32(0.25))))
+          for r in r1]
+    assert int(np.argmin(L1)) == 31
+    c, s, L, v = orc.sym_group(w, m)
+    assert s > 0 and (c == 62 or c >= 64)
+    # asymmetric plateau: zero-points that clamp nothing tie exactly; the first wins
+    wa = (np.arange(128, dtype=np.float32) % 4) * np.float32(0.01)     # r in [0, 3] for the grid's scales
+    ca, sa, za, La, qa = orc.asym_group(wa, np.ones(128, np.float32))
+    for z in range(16):
+        if z < za:
+            assert orc.asym_loss(wa, np.ones(128, np.float32), sa, z) > La
+    assert ca % 2 == 0
+
+
 # ----------------------------------------------------------------- imatrix / proxy / dequant
 
 def test_imatrix_closed_form_and_numpy(orc):
