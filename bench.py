@@ -439,27 +439,28 @@ def main():
     return 0
 
 
-def time_pack(tq, step, pk, reps=10):
+def time_pack(tq, step, pk, reps=12):
     """tq_pack (RTN + pack with given scales, the stand-alone form of the fused
-    pack) on the first unit, outside the step: bytes = weights read + packed
-    records written + scales (+ zeros) read."""
+    pack) on the first unit, outside the step, rotating through the input
+    sets: bytes = weights read + packed records written + scales (+ zeros) read."""
     u, r = step.units[0], step.res[0]
     fmt = tq.FORMATS[u.fmt]
     out = torch.empty_like(r.packed)
+    Ws = [s[1][0] for s in step.sets]
     nbytes = (u.W.numel() * u.W.element_size() + out.numel() + r.scales.numel() * r.scales.element_size()
               + (0 if r.zeros is None else r.zeros.numel()))
-    for _ in range(3):
-        tq.tq_pack(u.W, fmt, r.scales, r.zeros, r.global_scale, out=out)
+    for k in range(3):
+        tq.tq_pack(Ws[k % len(Ws)], fmt, r.scales, r.zeros, r.global_scale, out=out)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
-    for _ in range(reps):
-        tq.tq_pack(u.W, fmt, r.scales, r.zeros, r.global_scale, out=out)
+    for k in range(reps):
+        tq.tq_pack(Ws[k % len(Ws)], fmt, r.scales, r.zeros, r.global_scale, out=out)
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
-            "note": "first unit, back-to-back launches (inputs may be L2-resident when smaller than L2)"}
+            "note": f"first unit, back-to-back launches over {len(Ws)} rotating weight copies"}
 
 
 def _empty_like_result(tq, r):

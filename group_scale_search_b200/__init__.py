@@ -32,7 +32,7 @@ __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_proxy_error", "tq_sync", "FORMATS", "EXPORTS",
+    "tq_dequant", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -51,7 +51,7 @@ EXPORTS = [
     "tq_default_params", "tq_last_error_string", "tq_version", "tq_group_size", "tq_num_groups",
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
-    "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static",
+    "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
 ]
 
 
@@ -137,6 +137,7 @@ def lib():
             "tq_sync": (i32, [P]),
             "tq_imatrix_static_capacity": (sz, []),
             "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
+            "tq_selftest_e2m1": (i32, [P, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -219,6 +220,16 @@ def tq_packed_bytes(fmt: int, rows: int, cols: int) -> int:
 
 def tq_sync(stream=None) -> None:
     _check(lib().tq_sync(_stream(stream)), "tq_sync")
+
+
+def tq_selftest_e2m1(stream=None) -> Tuple[int, int]:
+    """(mismatches, first failing pattern) of the GPU's E2M1 conversion
+    instructions against the E2M1 round-half-to-even definition; (0,
+    0xffffffff) on a conforming GPU.  Synchronises the stream."""
+    n = ctypes.c_uint64(0)
+    first = ctypes.c_uint32(0)
+    _check(lib().tq_selftest_e2m1(ctypes.byref(n), ctypes.byref(first), _stream(stream)), "tq_selftest_e2m1")
+    return int(n.value), int(first.value)
 
 
 def tq_imatrix(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optional[float] = None,

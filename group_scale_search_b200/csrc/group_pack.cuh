@@ -47,43 +47,61 @@ __device__ __forceinline__ void pack_nvfp4_half(unsigned code, int hl, unsigned 
     if ((hl & 7) == 0) reinterpret_cast<uint32_t*>(rec)[hl >> 3] = v;
 }
 
-// Dequantizes the 16 weights of unit (group gid, part) into v[], rounding
-// once to fp32: int3 s v, int4 s (q - z), NVFP4 fl32(fl32(g dec(e)) dec(c)).
-// blocks_per_mat (O * G) maps an NVFP4 block to its matrix's global scale.
-__device__ __forceinline__ void dq_unit(int fmt, const uint8_t* __restrict__ packed, const void* scales,
-                                        const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
-                                        int64_t blocks_per_mat, int64_t gid, int part, float v[16]) {
-    if (fmt == TQ_INT3_G64_SYM) {
-        const uint8_t* rec = packed + gid * 24;
-        const uint32_t lo = __ldg(reinterpret_cast<const uint32_t*>(rec) + part);
-        const uint32_t hi = __ldg(reinterpret_cast<const uint16_t*>(rec + 16) + part);
-        const float s = __ldg(static_cast<const float*>(scales) + gid);
+// NVFP4 codes of N (8 or 16) weights under block scale S = fl32(g dec(e)):
+// magnitude = E2M1 round-half-to-even, saturating at 6, of the IEEE fp32
+// quotient |w| / S; sign in bit 3 when w < 0 and the magnitude is not 0
+// (every zero is +0); code 0 when S == 0.  Written as N/8 words of 8
+// nibbles, element i of a word in bits 4i..4i+3.
+//
+// Fast path (S positive, normal and not extreme, every |w| finite): with
+// inv = rcp(S), |w| inv approximates the IEEE quotient within 2^-21 relative,
+// so the products |w| inv (1 -+ 2^-20) bracket it; E2M1 rounding is monotone,
+// so when both ends round to the same code (hardware conversion, checked
+// against the definition by tq_selftest_e2m1) that is the quotient's code.
+// Otherwise -- a quotient within about 2^-20 of a rounding midpoint -- the
+// codes are redone with IEEE divisions.
+template <int N>
+__device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[N / 8]) {
+    unsigned mx = 0u;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int u = static_cast<int>(((lo >> (2 * i)) & 3u) | (((hi >> i) & 1u) << 2));
-            v[i] = __fmul_rn(s, static_cast<float>(u - 4));
-        }
-    } else if (fmt == TQ_INT4_G128_ASYM) {
-        const uint2 b = __ldg(reinterpret_cast<const uint2*>(packed + gid * 64) + part);
-        const float s = __ldg(static_cast<const float*>(scales) + gid);
-        const int z = __ldg(zeros + gid);
+    for (int i = 0; i < N; ++i) mx = max(mx, __float_as_uint(w[i]) & 0x7fffffffu);
+    const unsigned se = __float_as_uint(S) >> 23;   // sign bit included: positive S gives se < 256
+    bool exact = !(S > 0.f) || se < 3u || se > 251u || mx >= 0x7f800000u;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t wd = i < 8 ? b.x : b.y;
-            const int q = static_cast<int>((wd >> (4 * (i & 7))) & 15u);
-            v[i] = __fmul_rn(s, static_cast<float>(q - z));
-        }
-    } else {
-        const uint2 b = __ldg(reinterpret_cast<const uint2*>(packed + gid * 8));
-        const int64_t e = gid / blocks_per_mat;
-        const float S = __fmul_rn(__ldg(gs + e), e4m3_value(__ldg(static_cast<const uint8_t*>(scales) + gid)));
+    for (int h = 0; h < N / 8; ++h) m[h] = 0u;
+    if (!exact) {
+        const float inv = rcp_approx(S);
+        const float ilo = __fmul_rn(inv, 0.99999904632568359375f);   // 1 - 2^-20
+        const float ihi = __fmul_rn(inv, 1.00000095367431640625f);   // 1 + 2^-20
+        unsigned diff = 0u;
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const uint32_t wd = i < 8 ? b.x : b.y;
-            const unsigned c = (wd >> (4 * (i & 7))) & 15u;
-            const float mg = e2m1_value(c & 7u);
-            v[i] = __fmul_rn(S, (c & 8u) ? -mg : mg);
+        for (int p = 0; p < N / 2; ++p) {
+            const float a0 = fabsf(w[2 * p]), a1 = fabsf(w[2 * p + 1]);
+            const unsigned blo = e2m1x2_from_f32(__fmul_rn(a0, ilo), __fmul_rn(a1, ilo));
+            const unsigned bhi = e2m1x2_from_f32(__fmul_rn(a0, ihi), __fmul_rn(a1, ihi));
+            diff |= blo ^ bhi;
+            m[p >> 2] |= blo << (8 * (p & 3));
         }
+        exact = diff != 0u;
+    }
+    if (exact) {
+#pragma unroll
+        for (int h = 0; h < N / 8; ++h) m[h] = 0u;
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const float aw = fabsf(w[i]);
+            unsigned mag = 0u;
+            if (S != 0.f && aw != 0.f) mag = static_cast<unsigned>(e2m1_mag_code(e2m1_round(__fdiv_rn(aw, S)))) & 7u;
+            m[i >> 3] |= mag << (4 * (i & 7));
+        }
+    }
+#pragma unroll
+    for (int h = 0; h < N / 8; ++h) {
+        uint32_t sg = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sg |= (w[8 * h + i] < 0.f ? 8u : 0u) << (4 * i);
+        const uint32_t nz = (m[h] | (m[h] >> 1) | (m[h] >> 2)) & 0x11111111u;
+        m[h] |= sg & (nz << 3);
     }
 }
 

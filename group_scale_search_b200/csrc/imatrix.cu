@@ -18,7 +18,6 @@ namespace tq {
 
 constexpr int IM_THREADS = 256;
 constexpr int IM_WARPS = IM_THREADS / 32;
-constexpr int64_t IM_TARGET_BLOCKS = 1184;   // ~8 blocks per SM on a 148-SM B200
 
 template <typename T> struct VecOf { static constexpr int n = 16 / sizeof(T); };
 
@@ -44,16 +43,30 @@ struct ImGeom {
     int64_t col_tiles, slices, tokens_per_slice;
 };
 
+// Token slices per (column tile, matrix): the count that minimises the
+// modelled time, waves x (tokens per slice + IM_BLOCK_COST), where a wave is
+// IM_RESIDENT blocks per SM (what this kernel's registers allow on sm_100a)
+// and a slice holds at least 64 tokens.  Whole waves matter: a last wave
+// with few blocks costs as much as a full one.
+constexpr int64_t IM_RESIDENT = 4;
+constexpr int64_t IM_BLOCK_COST = 16;
+
 inline ImGeom im_geometry(const tq_mat* X) {
     const int vec = X->dtype == TQ_BF16 ? 8 : 4;
     ImGeom g;
     g.col_tiles = (X->cols + 32 * vec - 1) / (32 * vec);
     const int64_t base = g.col_tiles * X->n_mat;
-    int64_t s = (IM_TARGET_BLOCKS + base - 1) / base;
-    const int64_t max_s = (X->rows + 63) / 64;   // at least 64 tokens per slice
-    if (s > max_s) s = max_s;
-    if (s < 1) s = 1;
-    g.tokens_per_slice = (X->rows + s - 1) / s;
+    const int64_t resident = IM_RESIDENT * num_sms();
+    const int64_t max_s = max(static_cast<int64_t>(1), (X->rows + 63) / 64);
+    int64_t best_s = 1, best_cost = -1;
+    for (int64_t s = 1; s <= min(max_s, static_cast<int64_t>(4096)); ++s) {
+        const int64_t tps = (X->rows + s - 1) / s;
+        const int64_t slices = (X->rows + tps - 1) / tps;
+        const int64_t waves = (base * slices + resident - 1) / resident;
+        const int64_t cost = waves * (tps + IM_BLOCK_COST);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_s = s; }
+    }
+    g.tokens_per_slice = (X->rows + best_s - 1) / best_s;
     g.slices = (X->rows + g.tokens_per_slice - 1) / g.tokens_per_slice;
     return g;
 }

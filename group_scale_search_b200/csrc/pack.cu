@@ -5,96 +5,77 @@
 // records of a 2-bit low plane and a 1-bit high plane, v + 4); int4 and NVFP4
 // records hold one code per nibble, element 2k in the low nibble of byte k.
 // Dequantization rounds once to fp32: s v, s (q - z), fl32(fl32(g dec(e)) dec(c)).
-#include "group_pack.cuh"
+#include "walk.cuh"
 
 namespace tq {
 
-constexpr int PK_WARPS = 8;
-
-inline int pk_grid(int64_t units, int per_block) {
-    const int64_t need = (units + per_block - 1) / per_block;
-    return static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * 16));
+// Blocks of `kernel` (at `threads` per block) resident on one SM.
+template <typename K>
+int64_t resident_blocks(K kernel, int threads) {
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, threads, 0) != cudaSuccess || n < 1) n = 1;
+    return n;
 }
 
 // ------------------------------------------------------------------ RTN + pack with given scales
+// One thread per octet column (8 weights of one group, the last group's
+// padding included); it writes its share of the record: int3 = 2 low-plane
+// bytes + 1 high-plane byte, int4 = 4 bytes, NVFP4 = half the record.
 
-template <typename T>
-__global__ void __launch_bounds__(PK_WARPS * 32)
-k_pack_int3(const T* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
-            const float* __restrict__ scales, uint8_t* __restrict__ packed) {
-    const int lane = threadIdx.x & 31;
-    const int64_t G = (I + 63) >> 6, OG = O * G, total = n_mat * OG;
-    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * PK_WARPS + (threadIdx.x >> 5); gid < total;
-         gid += static_cast<int64_t>(gridDim.x) * PK_WARPS) {
-        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
-        const int64_t j0 = k << 6;
-        const int n = static_cast<int>(min(static_cast<int64_t>(64), I - j0));
-        const T* wp = W + e * ms + o * ld + j0;
-        const float s = __ldg(scales + gid);
-        const float w0 = lane < n ? Elem<T>::load(wp + lane) : 0.f;
-        const float w1 = lane + 32 < n ? Elem<T>::load(wp + lane + 32) : 0.f;
-        const unsigned u0 = static_cast<unsigned>(static_cast<int>(rtn_exact(w0, s, -4.f, 3.f)) + 4);
-        const unsigned u1 = static_cast<unsigned>(static_cast<int>(rtn_exact(w1, s, -4.f, 3.f)) + 4);
-        pack_int3_record(u0, u1, lane, packed + gid * 24);
+template <int FMT, typename T>
+__device__ __forceinline__ void pack_oct(const float w[8], int n, const void* scales, const uint8_t* __restrict__ zeros,
+                                         float g, int64_t gid, int oct, uint8_t* __restrict__ packed) {
+    if constexpr (FMT == TQ_NVFP4_G16) {   // padding has w = 0: code 0
+        const float S = __fmul_rn(g, e4m3_value(__ldg(static_cast<const uint8_t*>(scales) + gid)));
+        uint32_t c;
+        nvfp4_rtn<8>(w, S, &c);
+        reinterpret_cast<uint32_t*>(packed + gid * 8)[oct & 1] = c;
+    } else {
+        unsigned code[8];
+        const float sc = __ldg(static_cast<const float*>(scales) + gid);
+        if constexpr (FMT == TQ_INT3_G64_SYM) rtn_int_oct(w, n, sc, 4, 7.f, code);
+        else rtn_int_oct(w, n, sc, __ldg(zeros + gid), 15.f, code);
+        store_oct<FMT>(packed, gid, oct, code);
     }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(PK_WARPS * 32)
-k_pack_int4(const T* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
-            const float* __restrict__ scales, const uint8_t* __restrict__ zeros, uint8_t* __restrict__ packed) {
-    const int lane = threadIdx.x & 31;
-    const int64_t G = (I + 127) >> 7, OG = O * G, total = n_mat * OG;
-    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * PK_WARPS + (threadIdx.x >> 5); gid < total;
-         gid += static_cast<int64_t>(gridDim.x) * PK_WARPS) {
-        const int64_t e = gid / OG, rem = gid - e * OG, o = rem / G, k = rem - o * G;
-        const int64_t j0 = k << 7;
-        const int n = static_cast<int>(min(static_cast<int64_t>(128), I - j0));
-        const T* wp = W + e * ms + o * ld + j0;
-        const float s = __ldg(scales + gid);
-        const float z = static_cast<float>(__ldg(zeros + gid));
-        unsigned q[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int j = 4 * lane + i;
-            float qq = z;
-            if (j < n && s != 0.f)
-                qq = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(Elem<T>::load(wp + j), s)), z), 0.f), 15.f);
-            q[i] = static_cast<unsigned>(qq);
+// Grid: x = octet-column tiles, y = blocks of consecutive rows of the whole
+// batch (rows of all matrices in order, so every block gets the same number
+// of rows whatever the matrix count).
+template <int FMT, typename T>
+__global__ void __launch_bounds__(256)
+k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, int64_t n_rows, int64_t rpb,
+       const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
+       uint8_t* __restrict__ packed) {
+    using F = FmtTraits<FMT>;
+    const int64_t G = (I + F::group - 1) / F::group;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= (G << F::lg)) return;
+    const int64_t k = c >> F::lg;
+    const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
+    const int64_t j = c << 3;
+    const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j)));
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rpb, r1 = min(n_rows, r0 + rpb);
+    RowCursor<T> cur(W, O, ld, ms, j, r0);
+    for (int64_t r = r0; r < r1; r += 2) {
+        const bool two = r + 1 < r1;
+        const T* wa = cur.ptr;
+        const int64_t ea = cur.e;
+        cur.next();
+        const T* wb = cur.ptr;
+        const int64_t eb = cur.e;
+        cur.next();
+        Oct<T> ra, rb;
+        ra.load(wa, n);
+        if (two) rb.load(wb, n);
+        float w[8];
+        ra.get(w);
+        pack_oct<FMT, T>(w, n, scales, zeros, FMT == TQ_NVFP4_G16 ? __ldg(gs + ea) : 0.f, r * G + k, oct, packed);
+        if (two) {
+            rb.get(w);
+            pack_oct<FMT, T>(w, n, scales, zeros, FMT == TQ_NVFP4_G16 ? __ldg(gs + eb) : 0.f, (r + 1) * G + k, oct,
+                             packed);
         }
-        pack_int4_lane(q, lane, packed + gid * 64);
-    }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(PK_WARPS * 32)
-k_pack_nvfp4(const T* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
-             const uint8_t* __restrict__ scales, const float* __restrict__ gs, uint8_t* __restrict__ packed) {
-    const int lane = threadIdx.x & 31, half = lane >> 4, hl = lane & 15;
-    const int64_t G = (I + 15) >> 4, OG = O * G, total = n_mat * OG;
-    for (int64_t base = (static_cast<int64_t>(blockIdx.x) * PK_WARPS + (threadIdx.x >> 5)) * 2; base < total;
-         base += static_cast<int64_t>(gridDim.x) * PK_WARPS * 2) {
-        const int64_t bid = base + half;
-        const bool vb = bid < total;
-        unsigned c4 = 0u;
-        if (vb) {
-            const int64_t e = bid / OG, rem = bid - e * OG, o = rem / G, kb = rem - o * G;
-            const int64_t j = (kb << 4) + hl;
-            if (j < I) {
-                const float w = Elem<T>::load(W + e * ms + o * ld + j);
-                const float S = __fmul_rn(__ldg(gs + e), e4m3_value(__ldg(scales + bid)));
-                const float aw = fabsf(w);
-                if (S != 0.f && aw != 0.f) {
-                    const int mag = e2m1_mag_code(e2m1_round(__fdiv_rn(aw, S)));
-                    c4 = static_cast<unsigned>(mag) | ((mag != 0 && w < 0.f) ? 8u : 0u);
-                }
-            }
-        }
-        unsigned v = (c4 & 15u) << (4u * static_cast<unsigned>(hl & 7));
-        v |= __shfl_xor_sync(FULL, v, 1);
-        v |= __shfl_xor_sync(FULL, v, 2);
-        v |= __shfl_xor_sync(FULL, v, 4);
-        if (vb && (hl & 7) == 0) reinterpret_cast<uint32_t*>(packed + bid * 8)[hl >> 3] = v;
     }
 }
 
@@ -155,67 +136,121 @@ __global__ void k_unpack_codes(const uint8_t* __restrict__ packed, int fmt, int6
 }
 
 // ------------------------------------------------------------------ dequant
-// One thread per 16 consecutive outputs of one group: int3 = a quarter
-// record (4 low-plane bytes + 2 high-plane bytes), int4 = an eighth (8 bytes),
-// NVFP4 = a whole block (8 bytes).
-
-template <typename O> __device__ __forceinline__ O to_out(float v);
-template <> __device__ __forceinline__ float to_out<float>(float v) { return v; }
-template <> __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+// One thread per octet column (8 consecutive outputs of one group).
 
 template <typename O>
-__device__ __forceinline__ void store16(O* dst, const float v[16], bool vec_ok, int nvalid) {
-    if (vec_ok && nvalid == 16) {
+__device__ __forceinline__ void store8(O* dst, const float v[8], bool vec_ok, int nvalid) {
+    if (vec_ok && nvalid == 8) {
         if constexpr (sizeof(O) == 4) {
             float4* d = reinterpret_cast<float4*>(dst);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            d[0] = make_float4(v[0], v[1], v[2], v[3]);
+            d[1] = make_float4(v[4], v[5], v[6], v[7]);
         } else {
-            uint4* d = reinterpret_cast<uint4*>(dst);
+            uint32_t u[4];
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                uint32_t u[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const __nv_bfloat162 h = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
-                    u[k] = *reinterpret_cast<const uint32_t*>(&h);
-                }
-                d[i] = make_uint4(u[0], u[1], u[2], u[3]);
+            for (int k = 0; k < 4; ++k) {
+                const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+                u[k] = *reinterpret_cast<const uint32_t*>(&h);
             }
+            *reinterpret_cast<uint4*>(dst) = make_uint4(u[0], u[1], u[2], u[3]);
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            if (i < nvalid) dst[i] = to_out<O>(v[i]);
+        for (int i = 0; i < 8; ++i) {
+            if (i < nvalid) {
+                if constexpr (sizeof(O) == 4) dst[i] = v[i];
+                else dst[i] = __float2bfloat16_rn(v[i]);
+            }
+        }
     }
 }
 
-// Grid: x = 256-chunk column tiles of a row (a chunk = 16 weights of one
-// group), y = row slices, z = matrices; each thread keeps its chunk column and
-// walks the rows of its slice (no integer division in the loop).
-template <typename O>
+// Grid: x = octet-column tiles, y = blocks of consecutive rows of the whole
+// batch (the output is dense, so a row's place does not depend on its
+// matrix).  A thread loads two rows' codes and scales before decoding either.
+template <int FMT, typename O>
 __global__ void __launch_bounds__(256)
-k_dequant(const uint8_t* __restrict__ packed, int fmt, const void* scales, const uint8_t* __restrict__ zeros,
-          const float* __restrict__ gs, int64_t Orows, int64_t I, int64_t rows_per_slice, O* __restrict__ out) {
-    const int lg = fmt == TQ_INT3_G64_SYM ? 2 : (fmt == TQ_INT4_G128_ASYM ? 3 : 0);   // log2(chunks per group)
-    const int64_t G = (I + (16 << lg) - 1) >> (4 + lg);
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
-    const int64_t C = (I + 15) >> 4;
-    if (c >= C) return;
-    const int64_t k = c >> lg;
-    const int part = static_cast<int>(c & ((1 << lg) - 1));
-    const int64_t e = blockIdx.z;
-    const int64_t j = c << 4;
-    const int nvalid = static_cast<int>(min(static_cast<int64_t>(16), I - j));
+k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t* __restrict__ zeros,
+          const float* __restrict__ gs, int64_t Orows, int64_t I, int64_t n_rows, int64_t rpb, O* __restrict__ out) {
+    using F = FmtTraits<FMT>;
+    const int64_t G = (I + F::group - 1) / F::group;
+    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= ((I + 7) >> 3)) return;
+    const int64_t k = c >> F::lg;
+    const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
+    const int64_t j = c << 3;
+    const int nvalid = static_cast<int>(min(static_cast<int64_t>(8), I - j));
     const bool vec_ok = ((I * static_cast<int64_t>(sizeof(O))) % 16) == 0;
-    const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rows_per_slice;
-    const int64_t o1 = min(Orows, o0 + rows_per_slice);
-    for (int64_t o = o0; o < o1; ++o) {
-        const int64_t row = e * Orows + o;
-        float v[16];
-        dq_unit(fmt, packed, scales, zeros, gs, Orows * G, row * G + k, part, v);
-        store16<O>(out + row * I + j, v, vec_ok, nvalid);
+    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rpb, r1 = min(n_rows, r0 + rpb);
+    int64_t e = 0, next_e = n_rows;   // NVFP4: matrix of row r and the first row of the next matrix
+    float g = 0.f;
+    if (FMT == TQ_NVFP4_G16) {
+        e = r0 / Orows;
+        next_e = (e + 1) * Orows;
+        g = __ldg(gs + e);
     }
+    int64_t gid = r0 * G + k;
+    O* dst = out + r0 * I + j;
+    for (int64_t r = r0; r < r1; r += 2, gid += 2 * G, dst += 2 * I) {
+        const bool two = r + 1 < r1;
+        const OctQ q0 = load_q<FMT>(packed, scales, zeros, gid, oct);
+        OctQ q1 = q0;
+        if (two) q1 = load_q<FMT>(packed, scales, zeros, gid + G, oct);
+        float v[8];
+        if (FMT == TQ_NVFP4_G16 && r == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
+        dec_oct<FMT>(q0, g, v);
+        store8<O>(dst, v, vec_ok, nvalid);
+        if (two) {
+            if (FMT == TQ_NVFP4_G16 && r + 1 == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
+            dec_oct<FMT>(q1, g, v);
+            store8<O>(dst + I, v, vec_ok, nvalid);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ host launchers
+// The grid holds at most as many blocks as the SMs keep resident (one wave),
+// rows split evenly over the row blocks.
+
+struct FlatGrid { int64_t width, cblocks, rblocks, rpb; };
+
+inline FlatGrid flat_grid(int64_t n_rows, int64_t cols, int64_t resident_per_sm) {
+    FlatGrid f;
+    const Walk w = walk_geometry(1, 1, cols, 1);
+    f.width = w.width;
+    f.cblocks = w.cblocks;
+    const int64_t cap = static_cast<int64_t>(num_sms()) * resident_per_sm;
+    int64_t rb = max(static_cast<int64_t>(1), cap / f.cblocks);
+    rb = min(rb, min(n_rows, static_cast<int64_t>(65535)));
+    f.rpb = (n_rows + rb - 1) / rb;
+    f.rblocks = (n_rows + f.rpb - 1) / f.rpb;
+    return f;
+}
+
+template <int FMT, typename T>
+void launch_pack(const tq_mat* W, int64_t ms, const void* scales, const uint8_t* zeros, const float* gs,
+                 uint8_t* packed, cudaStream_t st) {
+    const int64_t g = FmtTraits<FMT>::group;
+    const int64_t cols = (W->cols + g - 1) / g * (g / 8);
+    const int64_t n_rows = W->n_mat * W->rows;
+    const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
+    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_pack<FMT, T>, width));
+    const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
+    k_pack<FMT, T><<<grid, static_cast<unsigned>(f.width), 0, st>>>(static_cast<const T*>(W->ptr), W->rows, W->cols,
+                                                                    W->ld, ms, n_rows, f.rpb, scales, zeros, gs,
+                                                                    packed);
+}
+
+template <int FMT, typename O>
+void launch_dequant(const uint8_t* packed, const void* scales, const uint8_t* zeros, const float* gs, int64_t n_mat,
+                    int64_t Orows, int64_t I, void* out, cudaStream_t st) {
+    const int64_t cols = (I + 7) / 8;
+    const int64_t n_rows = n_mat * Orows;
+    const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
+    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_dequant<FMT, O>, width));
+    const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
+    k_dequant<FMT, O><<<grid, static_cast<unsigned>(f.width), 0, st>>>(packed, scales, zeros, gs, Orows, I, n_rows,
+                                                                      f.rpb, static_cast<O*>(out));
 }
 
 }  // namespace tq
@@ -237,23 +272,16 @@ TQ_API tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const
     TQ_REQUIRE(aligned16(packed), "tq_pack: packed not 16-byte aligned");
     TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_pack: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_pack: NVFP4 needs global_scale");
+    TQ_REQUIRE(W->n_mat <= 65535, "tq_pack: more than 65535 matrices in one call");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
-    const int64_t G = tq_num_groups(fmt, W->n_mat * W->rows, W->cols);
     const bool bf = W->dtype == TQ_BF16;
-    if (fmt == TQ_INT3_G64_SYM) {
-        const int grid = pk_grid(G, PK_WARPS);
-        if (bf) k_pack_int3<uint16_t><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const float*>(scales), packed);
-        else k_pack_int3<float><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const float*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const float*>(scales), packed);
-    } else if (fmt == TQ_INT4_G128_ASYM) {
-        const int grid = pk_grid(G, PK_WARPS);
-        if (bf) k_pack_int4<uint16_t><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const float*>(scales), zeros, packed);
-        else k_pack_int4<float><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const float*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const float*>(scales), zeros, packed);
-    } else {
-        const int grid = pk_grid(G, 2 * PK_WARPS);
-        if (bf) k_pack_nvfp4<uint16_t><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const uint8_t*>(scales), global_scale, packed);
-        else k_pack_nvfp4<float><<<grid, PK_WARPS * 32, 0, st>>>(static_cast<const float*>(W->ptr), W->n_mat, W->rows, W->cols, W->ld, ms, static_cast<const uint8_t*>(scales), global_scale, packed);
-    }
+    if (fmt == TQ_INT3_G64_SYM) bf ? launch_pack<TQ_INT3_G64_SYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
+                                   : launch_pack<TQ_INT3_G64_SYM, float>(W, ms, scales, zeros, global_scale, packed, st);
+    else if (fmt == TQ_INT4_G128_ASYM) bf ? launch_pack<TQ_INT4_G128_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
+                                          : launch_pack<TQ_INT4_G128_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
+    else bf ? launch_pack<TQ_NVFP4_G16, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
+            : launch_pack<TQ_NVFP4_G16, float>(W, ms, scales, zeros, global_scale, packed, st);
     return check_launch("tq_pack");
 }
 
@@ -296,19 +324,17 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_dequant: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant: NVFP4 needs global_scale");
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant: out dtype %d", out_dtype);
-    const int64_t C = (I + 15) / 16;
-    const int64_t cblocks = (C + 255) / 256;
-    int64_t slices = (16 * static_cast<int64_t>(num_sms()) + cblocks * n_mat - 1) / (cblocks * n_mat);
-    slices = max(static_cast<int64_t>(1), min(slices, O));
-    const int64_t rps = (O + slices - 1) / slices;
-    slices = (O + rps - 1) / rps;
-    const dim3 grid(static_cast<unsigned>(cblocks), static_cast<unsigned>(slices), static_cast<unsigned>(n_mat));
+    TQ_REQUIRE(n_mat <= 65535, "tq_dequant: more than 65535 matrices in one call");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (out_dtype == TQ_BF16)
-        k_dequant<__nv_bfloat16><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, O, I, rps,
-                                                       static_cast<__nv_bfloat16*>(out));
+    const bool bf = out_dtype == TQ_BF16;
+    if (fmt == TQ_INT3_G64_SYM)
+        bf ? launch_dequant<TQ_INT3_G64_SYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT3_G64_SYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G128_ASYM)
+        bf ? launch_dequant<TQ_INT4_G128_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G128_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
     else
-        k_dequant<float><<<grid, 256, 0, st>>>(packed, fmt, scales, zeros, global_scale, O, I, rps,
-                                               static_cast<float*>(out));
+        bf ? launch_dequant<TQ_NVFP4_G16, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
+           : launch_dequant<TQ_NVFP4_G16, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
     return check_launch("tq_dequant");
 }

@@ -19,8 +19,9 @@
 // saturating) and back, and packed FMA/multiply/FMA for the weighted square.  Candidates whose fp32 loss is within a relative 2^-15 of the
 // lane's best are queued; half-warps then re-rank each queued block in fp64
 // with codes from the IEEE quotient (one lane per element), which decides the
-// winner exactly as the definition does.  The winner's codes are rounded
-// from the IEEE quotient and packed into the block's 8 bytes by the lane.
+// winner exactly as the definition does.  The winner's codes (E2M1 rounding
+// of the IEEE quotient, nvfp4_rtn) are packed into the block's 8 bytes by
+// the lane.
 #include "group_pack.cuh"
 
 #include <cuda_fp16.h>
@@ -110,13 +111,12 @@ template <> struct Load16<float> {
 template <typename T>
 __global__ void __launch_bounds__(FP4_THREADS)
 k_search_nvfp4(const __grid_constant__ Fp4Args a) {
-    __shared__ float dec[128];
+    __shared__ float dec[128];                      // E4M3 values (a table beats building them per lane)
     __shared__ float2 qdat[FP4_WARPS][32][17];     // each lane's block (w, m), padded against bank conflicts
     __shared__ int qres_c[FP4_WARPS][32];
     __shared__ double qres_l[FP4_WARPS][32];
     for (int i = threadIdx.x; i < 128; i += blockDim.x) dec[i] = e4m3_value(i);
     __syncthreads();
-
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int half = lane >> 4, hl = lane & 15;
     const int64_t G = (a.I + 15) >> 4;
@@ -237,7 +237,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
                 int bc = 0;
                 while (__any_sync(FULL, todo != 0u)) {
                     const int c = todo ? __ffs(todo) - 1 : 0;
-                    const float Sc = __fmul_rn(og, dec[olo + c]);
+                    const float Sc = __fmul_rn(og, e4m3_value(olo + c));
                     const float y = e2m1_round(__fdiv_rn(d.x, Sc));
                     const double er = __dsub_rn(static_cast<double>(d.x),
                                                 __dmul_rn(static_cast<double>(Sc), static_cast<double>(y)));
@@ -261,18 +261,13 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             const int code = lo + cbest;
             uint32_t wd0 = 0u, wd1 = 0u;
             if (!degen) {
-                const float Sf = __fmul_rn(g, dec[code]);
+                float wv[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float wi = qdat[wid][lane][i].x;
-                    const float aw = fabsf(wi);
-                    unsigned c4 = 0u;
-                    if (aw != 0.f) {
-                        const int mag = e2m1_mag_code(e2m1_round(__fdiv_rn(aw, Sf)));
-                        c4 = static_cast<unsigned>(mag) | ((mag != 0 && wi < 0.f) ? 8u : 0u);
-                    }
-                    if (i < 8) wd0 |= c4 << (4 * i); else wd1 |= c4 << (4 * (i - 8));
-                }
+                for (int i = 0; i < 16; ++i) wv[i] = qdat[wid][lane][i].x;
+                uint32_t pk[2];
+                nvfp4_rtn<16>(wv, __fmul_rn(g, e4m3_value(code)), pk);
+                wd0 = pk[0];
+                wd1 = pk[1];
             } else {
                 lossd = 0.0;
 #pragma unroll

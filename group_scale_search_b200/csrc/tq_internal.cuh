@@ -4,9 +4,11 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 #include <stdio.h>
 #include <stdarg.h>
+#include <string.h>
 
 #include "../../include/tq.h"
 
@@ -188,6 +190,28 @@ __device__ __forceinline__ float e2m1_round(float y) {
     return fminf(r, 6.0f);
 }
 
+// Hardware E2M1 conversions of sm_100a.  e2m1x2_from_f32: a pair of fp32
+// values rounded to E2M1 (nearest, ties to even, saturating at +-6) and packed
+// into one byte, `lo` in the low nibble.  For non-negative finite inputs and
+// +inf this is the magnitude code e2m1_mag_code(e2m1_round(y)) of each value;
+// tq_selftest_e2m1 checks that on every such fp32 value.
+__device__ __forceinline__ unsigned e2m1x2_from_f32(float lo, float hi) {
+    unsigned short r;
+    asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %2, %1; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+// The two E2M1 values of an e2m1x2 byte (low nibble first) as fp32, exactly
+// (every E2M1 value is an f16 value; code 8 is -0).
+__device__ __forceinline__ float2 e2m1x2_to_f32(unsigned byte) {
+    unsigned h2;
+    asm("{ .reg .b8 t; cvt.u8.u32 t, %1; cvt.rn.f16x2.e2m1x2 %0, t; }" : "=r"(h2) : "r"(byte));
+    __half2_raw raw;
+    raw.x = static_cast<unsigned short>(h2 & 0xffffu);
+    raw.y = static_cast<unsigned short>(h2 >> 16);
+    return __half22float2(__half2(raw));
+}
+
 // E2M1 magnitude code (0..7) of a value produced by e2m1_round.
 __device__ __forceinline__ int e2m1_mag_code(float v) {
     return v < 2.0f ? static_cast<int>(v * 2.0f) : (v < 4.0f ? static_cast<int>(v) + 2 : (v < 5.0f ? 6 : 7));
@@ -198,11 +222,17 @@ __device__ __forceinline__ float e2m1_value(unsigned c) {
     return c < 4u ? 0.5f * static_cast<float>(c) : (c < 6u ? static_cast<float>(c - 2u) : (c == 6u ? 4.0f : 6.0f));
 }
 
-// E4M3 (e4m3fn) value of a positive code 1..126 (0 for code 0).
-__host__ __device__ __forceinline__ float e4m3_value(int c) {
-    int e = (c >> 3) & 15, m = c & 7;
-    float v = (e == 0) ? ldexpf(static_cast<float>(m), -9) : ldexpf(1.0f + m * 0.125f, e - 7);
-    return v;
+// E4M3 (e4m3fn) value of code bits c, sign bit ignored (codes 1..126 are the
+// positive finite values, 0 is zero), built from the bit fields without an
+// integer-to-float conversion: normal codes (exponent field e >= 1, mantissa
+// m) are 2^(e-7) (1 + m/8), i.e. the fp32 pattern (c << 20) + (120 << 23);
+// subnormal codes are m 2^-9, taken as ((2^23 + m) - 2^23) 2^-9.
+__host__ __device__ __forceinline__ float e4m3_value(unsigned c) {
+    c &= 0x7fu;
+    const uint32_t b = c < 8u ? (0x4b000000u | c) : (c << 20) + 0x3c000000u;
+    float v;
+    memcpy(&v, &b, sizeof v);
+    return c < 8u ? (v - 8388608.0f) * 0.001953125f : v;
 }
 
 }  // namespace tq

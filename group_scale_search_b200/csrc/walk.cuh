@@ -1,0 +1,268 @@
+// Building blocks of the stand-alone streaming kernels (RTN + pack with given
+// scales, dequantization, proxy error).  All three walk a matrix batch in
+// octets: 8 consecutive weights of one group (an int3-g64 group holds 8
+// octets, an int4-g128 group 16, an NVFP4-g16 block 2).  One thread per octet
+// column: a bf16 octet is one 16-byte load (and a bf16 dequantized octet one
+// 16-byte store), so the 32 lanes of a warp touch 512 contiguous bytes of a
+// row per instruction, every 32-byte sector whole.
+//
+// A thread keeps its octet column (and what depends only on the column: its
+// imatrix weights, its place in the record) and walks rows two at a time,
+// both rows' loads issued before either is used.  No integer division is
+// needed in the walk.
+#pragma once
+#include "group_pack.cuh"
+
+namespace tq {
+
+// lg = log2(octets per group), rec = record bytes per group.
+template <int FMT> struct FmtTraits;
+template <> struct FmtTraits<TQ_INT3_G64_SYM> { static constexpr int lg = 3, group = 64, rec = 24; };
+template <> struct FmtTraits<TQ_INT4_G128_ASYM> { static constexpr int lg = 4, group = 128, rec = 64; };
+template <> struct FmtTraits<TQ_NVFP4_G16> { static constexpr int lg = 1, group = 16, rec = 8; };
+
+// ------------------------------------------------------------------ host geometry
+
+struct Walk {
+    int64_t width;     // threads per block = octet columns per block (a multiple of 32, <= 256)
+    int64_t cblocks;   // column tiles per row
+    int64_t slices;    // row slices per matrix
+    int64_t rps;       // rows per slice
+};
+
+// `cols` octet columns per row, `rows` rows per matrix, about `target_blocks`
+// blocks in all (at least that many when round_up, at most that many
+// otherwise unless every matrix already needs more).  Column tiles are
+// balanced so a ragged row idles fewer than 32 threads per tile.
+inline Walk walk_geometry(int64_t n_mat, int64_t rows, int64_t cols, int64_t target_blocks, bool round_up = true) {
+    Walk w;
+    w.cblocks = (cols + 255) / 256;
+    const int64_t per = (cols + w.cblocks - 1) / w.cblocks;
+    w.width = (per + 31) / 32 * 32;
+    int64_t s = round_up ? (target_blocks + w.cblocks * n_mat - 1) / (w.cblocks * n_mat)
+                         : target_blocks / (w.cblocks * n_mat);
+    s = s < 1 ? 1 : (s > rows ? rows : s);
+    w.rps = (rows + s - 1) / s;
+    w.slices = (rows + w.rps - 1) / w.rps;
+    return w;
+}
+
+// ------------------------------------------------------------------ device: rows
+
+// Position of one thread's octet in row r of a matrix batch whose rows run
+// over all matrices in order: matrix e, row o, and the octet's address.
+template <typename T>
+struct RowCursor {
+    const T* base;
+    int64_t O, ld, ms, j, e, o;
+    const T* ptr;
+    __device__ __forceinline__ RowCursor(const T* W, int64_t O_, int64_t ld_, int64_t ms_, int64_t j_, int64_t r)
+        : base(W), O(O_), ld(ld_), ms(ms_), j(j_) {
+        e = r / O;
+        o = r - e * O;
+        ptr = base + e * ms + o * ld + j;
+    }
+    __device__ __forceinline__ void next() {
+        if (++o == O) {
+            o = 0;
+            ++e;
+            ptr = base + e * ms + j;
+        } else {
+            ptr += ld;
+        }
+    }
+};
+
+// ------------------------------------------------------------------ device: weights
+
+// The 8 weights of an octet as loaded (n of them valid, the rest 0): one
+// 16-byte load for bf16, two for fp32, when all 8 are valid (row strides are
+// multiples of 16 bytes and octets start at multiples of 8 elements).
+template <typename T> struct Oct;
+template <> struct Oct<uint16_t> {
+    uint4 v;
+    __device__ __forceinline__ void load(const uint16_t* p, int n) {
+        if (n == 8) {
+            v = __ldg(reinterpret_cast<const uint4*>(p));
+        } else {
+            uint32_t u[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const unsigned lo = 2 * i < n ? __ldg(p + 2 * i) : 0u;
+                const unsigned hi = 2 * i + 1 < n ? __ldg(p + 2 * i + 1) : 0u;
+                u[i] = lo | (hi << 16);
+            }
+            v = make_uint4(u[0], u[1], u[2], u[3]);
+        }
+    }
+    __device__ __forceinline__ void get(float w[8]) const {
+        const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            w[2 * i] = __uint_as_float(u[i] << 16);
+            w[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+        }
+    }
+};
+template <> struct Oct<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* p, int n) {
+        if (n == 8) {
+            a = __ldg(reinterpret_cast<const float4*>(p));
+            b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+        } else {
+            float f[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) f[i] = i < n ? __ldg(p + i) : 0.f;
+            a = make_float4(f[0], f[1], f[2], f[3]);
+            b = make_float4(f[4], f[5], f[6], f[7]);
+        }
+    }
+    __device__ __forceinline__ void get(float w[8]) const {
+        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
+        w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
+    }
+};
+
+// ------------------------------------------------------------------ device: codes of one octet
+
+// The packed bits, scale and zero-point of octet `oct` of group `gid`.
+// bits: int3 = its 2 low-plane bytes (bits 0..15) and its high-plane byte
+// (bits 16..23); int4 = its 4 record bytes; NVFP4 = its half of the 8-byte
+// record.  For NVFP4, s is the decoded E4M3 block scale (the caller
+// multiplies by the global scale).
+struct OctQ {
+    uint32_t bits;
+    float s;
+    int z;
+};
+
+template <int FMT>
+__device__ __forceinline__ OctQ load_q(const uint8_t* __restrict__ packed, const void* scales,
+                                       const uint8_t* __restrict__ zeros, int64_t gid, int oct) {
+    OctQ q;
+    if constexpr (FMT == TQ_INT3_G64_SYM) {
+        const uint8_t* rec = packed + gid * 24;
+        q.bits = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(rec) + oct)) |
+                 (static_cast<uint32_t>(__ldg(rec + 16 + oct)) << 16);
+        q.s = __ldg(static_cast<const float*>(scales) + gid);
+        q.z = 4;
+    } else if constexpr (FMT == TQ_INT4_G128_ASYM) {
+        q.bits = __ldg(reinterpret_cast<const uint32_t*>(packed + gid * 64) + oct);
+        q.s = __ldg(static_cast<const float*>(scales) + gid);
+        q.z = __ldg(zeros + gid);
+    } else {
+        q.bits = __ldg(reinterpret_cast<const uint32_t*>(packed + gid * 8) + (oct & 1));
+        q.s = e4m3_value(__ldg(static_cast<const uint8_t*>(scales) + gid));
+        q.z = 0;
+    }
+    return q;
+}
+
+// 2^23 + k for a small non-negative integer k, as a float; subtracting 2^23
+// (exactly) gives k without an integer-to-float conversion.
+__device__ __forceinline__ float f23(unsigned k) { return __uint_as_float(0x4b000000u | k); }
+
+// Dequantized values of an octet, rounded once to fp32 exactly as the pages'
+// formulas: int3 s v, int4 s (q - z), NVFP4 fl32(fl32(g dec(e)) dec(c)).
+// Integers become floats as 2^23 + k (exact) and the offset 2^23 + z comes
+// off in the same fp32 addition, pairs of elements per fp32x2 instruction;
+// NVFP4 bytes are decoded by the hardware E2M1 conversion (exact).
+template <int FMT>
+__device__ __forceinline__ void dec_oct(const OctQ& q, float g, float v[8]) {
+    if constexpr (FMT == TQ_INT3_G64_SYM) {
+        const float2 noff = make_float2(-8388612.0f, -8388612.0f);   // -(2^23 + 4): stored u = v + 4
+        const float2 s2 = make_float2(q.s, q.s);
+#pragma unroll
+        for (int i = 0; i < 8; i += 2) {
+            const unsigned u0 = ((q.bits >> (2 * i)) & 3u) | (((q.bits >> (16 + i)) & 1u) << 2);
+            const unsigned u1 = ((q.bits >> (2 * i + 2)) & 3u) | (((q.bits >> (17 + i)) & 1u) << 2);
+            const float2 r = __fmul2_rn(s2, __fadd2_rn(make_float2(f23(u0), f23(u1)), noff));
+            v[i] = r.x; v[i + 1] = r.y;
+        }
+    } else if constexpr (FMT == TQ_INT4_G128_ASYM) {
+        const float o = f23(static_cast<unsigned>(q.z) & 0xffu);   // 2^23 + z
+        const float2 noff = make_float2(-o, -o), s2 = make_float2(q.s, q.s);
+        const uint32_t ev = q.bits & 0x0f0f0f0fu, od = (q.bits >> 4) & 0x0f0f0f0fu;   // elements 2k, 2k+1 in byte k
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const unsigned sel = 0x5640u | static_cast<unsigned>(k);    // bytes: (byte k, 0, 0, 0x4b)
+            const float2 x = make_float2(__uint_as_float(__byte_perm(ev, 0x4b00u, sel)),
+                                         __uint_as_float(__byte_perm(od, 0x4b00u, sel)));
+            const float2 r = __fmul2_rn(s2, __fadd2_rn(x, noff));
+            v[2 * k] = r.x; v[2 * k + 1] = r.y;
+        }
+    } else {
+        const float S = __fmul_rn(g, q.s);
+        const float2 S2 = make_float2(S, S);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+            const float2 r = __fmul2_rn(S2, e2m1x2_to_f32((q.bits >> (8 * b)) & 0xffu));
+            v[2 * b] = r.x; v[2 * b + 1] = r.y;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ device: RTN codes of one octet
+
+// Integer codes q_i = clamp(rint(w_i / s) + z, 0, hi) of 8 weights, where
+// rint rounds the IEEE fp32 quotient half to even (int3: z = 4, hi = 7 gives
+// the stored u = clamp(rint(w/s), -4, 3) + 4; int4: hi = 15).  Elements at or
+// past n and a zero scale give z.  The quotient is first approximated as
+// w * rcp(s) (within 2^-21 relative when s and 1/s are normal); the rounded
+// codes agree with the IEEE quotient's unless it lies within 2^-20 relative of
+// a half-integer, and in that case (or for an extreme s) all 8 are redone
+// with IEEE divisions.  Codes come back in the low bits of code[i].
+__device__ __forceinline__ void rtn_int_oct(const float w[8], int n, float s, int z, float hi, unsigned code[8]) {
+    const float zf = static_cast<float>(z);
+    const unsigned se = (__float_as_uint(s) >> 23) & 255u;
+    bool exact = se < 3u || se > 251u;   // zero, subnormal or extreme scales
+    if (!exact) {
+        const float inv = rcp_approx(s);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float y = __fmul_rn(w[i], inv);
+            const float r = __fsub_rn(__fadd_rn(y, MAGIC), MAGIC);
+            exact |= fabsf(__fsub_rn(y, r)) >= __fmaf_rn(fabsf(y), -9.5367431640625e-07f, 0.5f);
+            const float qf = fminf(fmaxf(__fadd_rn(r, zf), 0.f), hi);
+            code[i] = __float_as_uint(__fadd_rn(qf, MAGIC));
+        }
+    }
+    if (exact) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float qf = zf;
+            if (s != 0.f) qf = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), zf), 0.f), hi);
+            code[i] = __float_as_uint(__fadd_rn(qf, MAGIC));
+        }
+    }
+    if (n < 8) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (i >= n) code[i] = static_cast<unsigned>(z);
+    }
+}
+
+// Stores an octet's integer codes into its share of the record: int3 = 2
+// low-plane bytes + 1 high-plane byte, int4 = 4 bytes.
+template <int FMT>
+__device__ __forceinline__ void store_oct(uint8_t* __restrict__ packed, int64_t gid, int oct, const unsigned code[8]) {
+    if constexpr (FMT == TQ_INT3_G64_SYM) {
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            lo |= (code[i] & 3u) << (2 * i);
+            hi |= ((code[i] >> 2) & 1u) << i;
+        }
+        uint8_t* rec = packed + gid * 24;
+        reinterpret_cast<uint16_t*>(rec)[oct] = static_cast<uint16_t>(lo);
+        rec[16 + oct] = static_cast<uint8_t>(hi);
+    } else {
+        uint32_t a = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a |= (code[i] & 15u) << (4 * i);
+        reinterpret_cast<uint32_t*>(packed + gid * 64)[oct] = a;
+    }
+}
+
+}  // namespace tq

@@ -251,6 +251,19 @@ tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, co
  * failed. */
 tq_status tq_sync(tq_stream_t stream);
 
+/* Self-test of the GPU's E2M1 conversion instructions, on which the NVFP4
+ * round-to-nearest (search, tq_pack) and decoding (tq_dequant,
+ * tq_proxy_error) rely.  The pages define the element format only (E2M1:
+ * values 0, .5, 1, 1.5, 2, 3, 4, 6 with a sign; [NVFP4] Quantization Recipe);
+ * this call has no counterpart there.  Checks every non-negative finite fp32
+ * value and +inf (rounded half to even, saturating at 6) in both nibbles of
+ * a byte, and all 256 bytes decoded bit for bit.  *mismatches (host) gets the
+ * number of failing cases, 0 on a conforming GPU; *first_bad (host, may be
+ * NULL) the first failing fp32 pattern (0x80000000 | byte for a decode
+ * failure, 0xffffffff when none).  Uses two words of static device memory
+ * (concurrent calls race on them) and synchronises `stream`. */
+tq_status tq_selftest_e2m1(uint64_t* mismatches, uint32_t* first_bad, tq_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -246,3 +246,99 @@ def test_p5_outlier_rows_property_on_gpu():
     rms3 = (Wo.double() - dq[0].double()).pow(2).mean().sqrt().item()
     rms4 = np.sqrt(np.mean((host32(Wo).astype(np.float64) - oracle.rowwise_int4(host32(Wo))) ** 2))
     assert rms3 < rms4
+
+
+# ------------------------------------------------------------------ RTN + pack with given scales
+
+def _edge_weights(rows, I, scales_per_group, g, seed, dtype):
+    """Weights that sit on, and one fp32 ulp either side of, the rounding
+    midpoints (k + 1/2) s of their group's scale, mixed with ordinary values."""
+    rng = np.random.default_rng(seed)
+    W = rng.standard_t(4, size=(rows, I)).astype(np.float32) * 0.02
+    for r in range(rows):
+        for j in range(I):
+            s = np.float32(scales_per_group[r, j // g])
+            if not np.isfinite(s) or s == 0 or abs(s) > 1e30 or abs(s) < 1e-30:
+                continue
+            mode = (r * 7 + j) % 4
+            if mode == 3:
+                continue
+            k = rng.integers(-5, 5)
+            x = np.float32((k + 0.5) * np.float64(s))
+            if mode == 1:
+                x = np.nextafter(x, np.float32(np.inf))
+            elif mode == 2:
+                x = np.nextafter(x, np.float32(-np.inf))
+            W[r, j] = x
+    W = torch.from_numpy(W)
+    return W.to(dtype) if dtype != torch.float32 else W
+
+
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("I", [300, 1024])
+def test_pack_given_scales_edge_cases(fmt, dtype, I):
+    """tq_pack with caller scales: zero, subnormal, extreme and negative (int3)
+    scales, weights on and next to the rounding midpoints; bit-exact."""
+    g = 64 if fmt == tq.INT3_G64_SYM else 128
+    rows, G = 24, (I + g - 1) // g
+    rng = np.random.default_rng(I + fmt)
+    special = np.array([0.0, 1e-40, 1.5 * 2.0 ** -124, 2.0 ** -126, 3e38, 0.25, 0.1, 0.013, 7e-3, 1.7e-5],
+                       np.float32)
+    sc = special[rng.integers(0, len(special), size=(rows, G))]
+    if fmt == tq.INT3_G64_SYM:
+        sc = sc * np.where(rng.random((rows, G)) < 0.3, -1, 1).astype(np.float32)
+    ld = (I + 7) // 8 * 8                           # 16-byte row stride for both dtypes
+    W = torch.zeros((rows, ld), dtype=dtype, device=DEV)
+    W[:, :I] = _edge_weights(rows, I, sc, g, I, dtype).to(DEV)
+    W = W[:, :I]
+    Wh = host32(W).reshape(1, rows, I)
+    zeros = rng.integers(0, 16, size=(rows, G)).astype(np.uint8)
+    st = torch.from_numpy(sc).to(DEV)
+    zt = torch.from_numpy(zeros).to(DEV) if fmt == tq.INT4_G128_ASYM else None
+    p = tq.tq_pack(W, fmt, st, zt, None)
+    torch.cuda.synchronize()
+    ref, _ = oracle_packed(fmt, Wh, sc.reshape(1, rows, G), None if zt is None else zeros.reshape(1, rows, G))
+    assert np.array_equal(p.cpu().numpy(), ref)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_pack_nvfp4_given_scales_edge_cases(dtype):
+    """NVFP4 tq_pack with every block-scale code, a zero global scale on one
+    matrix, and weights on and next to the E2M1 midpoints; bit-exact."""
+    E, O, I = 3, 16, 520
+    G = (I + 15) // 16
+    rng = np.random.default_rng(5)
+    codes = rng.integers(0, 127, size=(E, O, G)).astype(np.uint8)
+    codes.reshape(-1)[:127] = np.arange(127, dtype=np.uint8)
+    gsc = np.array([2.0 ** -9, 0.0, 3.1e-4], np.float32)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 7.0], np.float64)
+    W = (rng.standard_t(4, size=(E, O, I)) * 0.02).astype(np.float32)
+    for e in range(E):
+        for o in range(O):
+            for j in range(I):
+                S = np.float32(np.float64(gsc[e]) * oracle.e4m3_decode(int(codes[e, o, j // 16])))
+                if S == 0 or (e + o + j) % 3 == 0:
+                    continue
+                x = np.float32(mids[(o + j) % len(mids)] * np.float64(S)) * (1 if j % 2 else -1)
+                if (o + j) % 5 == 1:
+                    x = np.nextafter(x, np.float32(np.inf))
+                elif (o + j) % 5 == 2:
+                    x = np.nextafter(x, np.float32(-np.inf))
+                W[e, o, j] = x
+    Wt = torch.from_numpy(W)
+    Wt = (Wt.to(dtype) if dtype != torch.float32 else Wt).to(DEV)   # I = 520: 16-byte rows in both dtypes
+    Wh = host32(Wt)
+    p = tq.tq_pack(Wt, tq.NVFP4_G16, torch.from_numpy(codes).to(DEV), None, torch.from_numpy(gsc).to(DEV))
+    torch.cuda.synchronize()
+    ref, _ = oracle_packed(tq.NVFP4_G16, Wh, codes, None, gsc)
+    assert np.array_equal(p.cpu().numpy(), ref)
+
+
+def test_e2m1_conversion_selftest():
+    """The hardware E2M1 rounding (every non-negative finite fp32 value and
+    +inf, both nibbles) and decoding (all 256 bytes) that the NVFP4 RTN and
+    dequantization use agree with the E2M1 round-half-to-even definition."""
+    n, first = tq.tq_selftest_e2m1()
+    assert n == 0, f"{n} mismatches, first failing pattern {first:#010x}"
+    assert first == 0xFFFFFFFF
