@@ -53,34 +53,39 @@ __device__ __forceinline__ void pack_nvfp4_half(unsigned code, int hl, unsigned 
 // (every zero is +0); code 0 when S == 0.  Written as N/8 words of 8
 // nibbles, element i of a word in bits 4i..4i+3.
 //
-// Fast path (S positive, normal and not extreme, every |w| finite): with
-// inv = rcp(S), |w| inv approximates the IEEE quotient within 2^-21 relative,
-// so the products |w| inv (1 -+ 2^-20) bracket it; E2M1 rounding is monotone,
-// so when both ends round to the same code (hardware conversion, checked
-// against the definition by tq_selftest_e2m1) that is the quotient's code.
-// Otherwise -- a quotient within about 2^-20 of a rounding midpoint -- the
-// codes are redone with IEEE divisions.
+// Fast path (S positive, normal and not extreme): with inv = rcp(S), w inv
+// approximates the IEEE quotient w / S within 2^-21 relative, so the
+// products w inv (1 -+ 2^-20) bracket it.  The hardware conversion rounds
+// signed values (ties to even, saturating, sign kept, -0 for a negative value
+// that rounds to zero; tq_selftest_e2m1 checks it against the definition on
+// every non-NaN fp32 value); E2M1 rounding is monotone, so when both ends
+// give the same code that is the quotient's.  A -0 is then made +0 with a
+// word-wide test for zero magnitudes.  Otherwise -- a quotient within about
+// 2^-20 of a rounding midpoint -- the codes are redone with IEEE divisions.
+// For NaN weights the codes are unspecified.
 template <int N>
 __device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[N / 8]) {
-    unsigned mx = 0u;
-#pragma unroll
-    for (int i = 0; i < N; ++i) mx = max(mx, __float_as_uint(w[i]) & 0x7fffffffu);
     const unsigned se = __float_as_uint(S) >> 23;   // sign bit included: positive S gives se < 256
-    bool exact = !(S > 0.f) || se < 3u || se > 251u || mx >= 0x7f800000u;
-#pragma unroll
-    for (int h = 0; h < N / 8; ++h) m[h] = 0u;
+    bool exact = !(S > 0.f) || se < 3u || se > 251u;
     if (!exact) {
         const float inv = rcp_approx(S);
-        const float ilo = __fmul_rn(inv, 0.99999904632568359375f);   // 1 - 2^-20
-        const float ihi = __fmul_rn(inv, 1.00000095367431640625f);   // 1 + 2^-20
-        unsigned diff = 0u;
+        const float lo = __fmul_rn(inv, 0.99999904632568359375f), hi = __fmul_rn(inv, 1.00000095367431640625f);
+        const float2 lo2 = make_float2(lo, lo), hi2 = make_float2(hi, hi);
+        uint32_t diff = 0u, bytes[N / 2];
 #pragma unroll
         for (int p = 0; p < N / 2; ++p) {
-            const float a0 = fabsf(w[2 * p]), a1 = fabsf(w[2 * p + 1]);
-            const unsigned blo = e2m1x2_from_f32(__fmul_rn(a0, ilo), __fmul_rn(a1, ilo));
-            const unsigned bhi = e2m1x2_from_f32(__fmul_rn(a0, ihi), __fmul_rn(a1, ihi));
-            diff |= blo ^ bhi;
-            m[p >> 2] |= blo << (8 * (p & 3));
+            const float2 ww = make_float2(w[2 * p], w[2 * p + 1]);
+            const float2 yl = __fmul2_rn(ww, lo2), yh = __fmul2_rn(ww, hi2);
+            const unsigned bl = e2m1x2_from_f32(yl.x, yl.y), bh = e2m1x2_from_f32(yh.x, yh.y);
+            diff |= bl ^ bh;
+            bytes[p] = bl;
+        }
+#pragma unroll
+        for (int h = 0; h < N / 8; ++h) {
+            uint32_t x = __byte_perm(__byte_perm(bytes[4 * h], bytes[4 * h + 1], 0x0040u),
+                                     __byte_perm(bytes[4 * h + 2], bytes[4 * h + 3], 0x0040u), 0x5410u);
+            const uint32_t nz = (x | (x >> 1) | (x >> 2)) & 0x11111111u;   // magnitude != 0, per nibble
+            m[h] = x & (0x77777777u | (nz << 3));
         }
         exact = diff != 0u;
     }
@@ -92,16 +97,8 @@ __device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[
             const float aw = fabsf(w[i]);
             unsigned mag = 0u;
             if (S != 0.f && aw != 0.f) mag = static_cast<unsigned>(e2m1_mag_code(e2m1_round(__fdiv_rn(aw, S)))) & 7u;
-            m[i >> 3] |= mag << (4 * (i & 7));
+            m[i >> 3] |= (mag | ((mag != 0u && w[i] < 0.f) ? 8u : 0u)) << (4 * (i & 7));
         }
-    }
-#pragma unroll
-    for (int h = 0; h < N / 8; ++h) {
-        uint32_t sg = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) sg |= (w[8 * h + i] < 0.f ? 8u : 0u) << (4 * i);
-        const uint32_t nz = (m[h] | (m[h] >> 1) | (m[h] >> 2)) & 0x11111111u;
-        m[h] |= sg & (nz << 3);
     }
 }
 

@@ -30,12 +30,11 @@ __device__ __forceinline__ void pack_oct(const float w[8], int n, const void* sc
         uint32_t c;
         nvfp4_rtn<8>(w, S, &c);
         reinterpret_cast<uint32_t*>(packed + gid * 8)[oct & 1] = c;
+    } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+        store_oct<FMT>(packed, gid, oct, rtn_int_oct<7>(w, n, __ldg(static_cast<const float*>(scales) + gid), 4));
     } else {
-        unsigned code[8];
-        const float sc = __ldg(static_cast<const float*>(scales) + gid);
-        if constexpr (FMT == TQ_INT3_G64_SYM) rtn_int_oct(w, n, sc, 4, 7.f, code);
-        else rtn_int_oct(w, n, sc, __ldg(zeros + gid), 15.f, code);
-        store_oct<FMT>(packed, gid, oct, code);
+        store_oct<FMT>(packed, gid, oct,
+                       rtn_int_oct<15>(w, n, __ldg(static_cast<const float*>(scales) + gid), __ldg(zeros + gid)));
     }
 }
 

@@ -4,10 +4,11 @@
 // definition: round half to even on the E2M1 grid {0, .5, 1, 1.5, 2, 3, 4, 6},
 // saturating at 6 ("NVFP4" element format: E2M1 with an E4M3 block scale).
 //
-// Rounding: every non-negative finite fp32 value and +inf, once in the low
-// nibble (paired with 6.0) and once in the high nibble (paired with 0.0), so
-// both the values and the nibble order are checked.  Decoding: all 256 bytes,
-// bit for bit (code 8 is -0).
+// Rounding: every fp32 value but NaN (both signs, zeros and infinities
+// included; a negative value keeps its sign bit in bit 3 of the nibble, -0
+// too), once in the low nibble (paired with 6.0) and once in the high nibble
+// (paired with 0.0), so both the values and the nibble order are checked.
+// Decoding: all 256 bytes, bit for bit (code 8 is -0).
 #include "tq_internal.cuh"
 
 namespace tq {
@@ -16,18 +17,19 @@ static __device__ unsigned long long g_st_count;
 static __device__ unsigned g_st_first;
 
 __global__ void k_selftest_e2m1_round() {
-    const uint64_t n = 0x7f800001ull;   // fp32 bit patterns 0 .. +inf
+    const uint64_t half = 0x7f800001ull;   // fp32 bit patterns +0 .. +inf, then -0 .. -inf
     unsigned long long bad = 0;
     unsigned first = 0xffffffffu;
-    for (uint64_t u = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; u < n;
-         u += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
-        const float y = __uint_as_float(static_cast<unsigned>(u));
-        const unsigned r = static_cast<unsigned>(e2m1_mag_code(e2m1_round(y)));
+    for (uint64_t i = static_cast<uint64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < 2 * half;
+         i += static_cast<uint64_t>(gridDim.x) * blockDim.x) {
+        const unsigned u = i < half ? static_cast<unsigned>(i) : (static_cast<unsigned>(i - half) | 0x80000000u);
+        const float y = __uint_as_float(u);
+        const unsigned r = static_cast<unsigned>(e2m1_mag_code(e2m1_round(fabsf(y)))) | ((u >> 28) & 8u);
         const unsigned a = e2m1x2_from_f32(y, 6.0f);
         const unsigned b = e2m1x2_from_f32(0.0f, y);
         if (a != (r | 0x70u) || b != (r << 4)) {
             ++bad;
-            first = min(first, static_cast<unsigned>(u));
+            first = min(first, u);
         }
     }
     if (bad) {

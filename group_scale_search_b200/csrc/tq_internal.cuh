@@ -43,6 +43,10 @@ tq_status check_mat(const tq_mat* X, const char* name);
 
 int num_sms();
 
+// Reads and clears the flag the proxy kernels set when a bounded wait for a
+// bulk copy gives up (proxy.cu).
+bool take_proxy_fault();
+
 // ------------------------------------------------------------------ index arithmetic
 
 // Division of 32-bit unsigned integers by a fixed divisor d >= 1 with a
@@ -192,9 +196,10 @@ __device__ __forceinline__ float e2m1_round(float y) {
 
 // Hardware E2M1 conversions of sm_100a.  e2m1x2_from_f32: a pair of fp32
 // values rounded to E2M1 (nearest, ties to even, saturating at +-6) and packed
-// into one byte, `lo` in the low nibble.  For non-negative finite inputs and
-// +inf this is the magnitude code e2m1_mag_code(e2m1_round(y)) of each value;
-// tq_selftest_e2m1 checks that on every such fp32 value.
+// into one byte, `lo` in the low nibble.  For every non-NaN input y the
+// nibble is the magnitude code e2m1_mag_code(e2m1_round(|y|)), with bit 3 set
+// when y has its sign bit set (-0 included); tq_selftest_e2m1 checks that on
+// every such fp32 value.
 __device__ __forceinline__ unsigned e2m1x2_from_f32(float lo, float hi) {
     unsigned short r;
     asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %2, %1; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(lo), "f"(hi));

@@ -73,6 +73,49 @@ struct RowCursor {
     }
 };
 
+// ------------------------------------------------------------------ device: bulk copies (TMA)
+// One-dimensional bulk copies global -> shared (cp.async.bulk, no tensor map,
+// no multicast), completed on an mbarrier that counts the bytes.  Waits are
+// bounded: after TQ_WAIT_POLLS polls a wait gives up and returns false.
+
+constexpr uint32_t TQ_WAIT_POLLS = 1u << 22;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+// Makes barrier initialisation visible to the bulk-copy (async) proxy.
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+// Orders this thread's earlier shared-memory accesses before later bulk copies.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+    const uint32_t a = smem_u32(bar);
+    for (uint32_t it = 0; it < TQ_WAIT_POLLS; ++it) {
+        uint32_t done;
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}"
+                     : "=r"(done)
+                     : "r"(a), "r"(parity)
+                     : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
 // ------------------------------------------------------------------ device: weights
 
 // The 8 weights of an octet as loaded (n of them valid, the rest 0): one
@@ -205,63 +248,80 @@ __device__ __forceinline__ void dec_oct(const OctQ& q, float g, float v[8]) {
 
 // ------------------------------------------------------------------ device: RTN codes of one octet
 
-// Integer codes q_i = clamp(rint(w_i / s) + z, 0, hi) of 8 weights, where
-// rint rounds the IEEE fp32 quotient half to even (int3: z = 4, hi = 7 gives
-// the stored u = clamp(rint(w/s), -4, 3) + 4; int4: hi = 15).  Elements at or
-// past n and a zero scale give z.  The quotient is first approximated as
-// w * rcp(s) (within 2^-21 relative when s and 1/s are normal); the rounded
-// codes agree with the IEEE quotient's unless it lies within 2^-20 relative of
-// a half-integer, and in that case (or for an extreme s) all 8 are redone
-// with IEEE divisions.  Codes come back in the low bits of code[i].
-__device__ __forceinline__ void rtn_int_oct(const float w[8], int n, float s, int z, float hi, unsigned code[8]) {
-    const float zf = static_cast<float>(z);
+// Integer codes q_i = clamp(rint(w_i / s) + z, 0, HI) of an octet, as 8
+// nibbles (element i in bits 4i..4i+3), where rint rounds the IEEE fp32
+// quotient half to even (int3: z = 4, HI = 7 gives the stored
+// u = clamp(rint(w/s), -4, 3) + 4; int4: HI = 15).  Elements at or past n and
+// a zero scale give z.
+//
+// Fast path (s normal and not extreme): with inv = rcp(s) (within 2^-21
+// relative of 1/s), the exact products w inv (1 -+ 2^-20) bracket the IEEE
+// quotient; one FMA per end adds 1.5 2^23, which rounds the product to an
+// integer, half to even, in the low mantissa bits.  Rounding is monotone, so
+// when both ends give the same integer it is the quotient's.  Both ends are
+// finite or both are the same infinity (a quotient beyond +-2^127 clamps
+// either way); when they differ (a quotient within about 2^-20 of a
+// half-integer, or of magnitude 2^22 or more) the octet is redone with IEEE
+// divisions.  For NaN weights the codes are unspecified.
+template <int HI>
+__device__ __forceinline__ uint32_t rtn_int_oct(const float w[8], int n, float s, int z) {
     const unsigned se = (__float_as_uint(s) >> 23) & 255u;
     bool exact = se < 3u || se > 251u;   // zero, subnormal or extreme scales
+    uint32_t nib = 0u;
     if (!exact) {
         const float inv = rcp_approx(s);
+        const float lo = __fmul_rn(inv, 0.99999904632568359375f), hi = __fmul_rn(inv, 1.00000095367431640625f);
+        const float2 ilo = make_float2(lo, lo), ihi = make_float2(hi, hi), M2 = make_float2(MAGIC, MAGIC);
+        const int zo = z - static_cast<int>(0x4b400000u);   // code = bits(t) - bits(1.5 2^23) + z
+        uint32_t diff = 0u, bytes[4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const float y = __fmul_rn(w[i], inv);
-            const float r = __fsub_rn(__fadd_rn(y, MAGIC), MAGIC);
-            exact |= fabsf(__fsub_rn(y, r)) >= __fmaf_rn(fabsf(y), -9.5367431640625e-07f, 0.5f);
-            const float qf = fminf(fmaxf(__fadd_rn(r, zf), 0.f), hi);
-            code[i] = __float_as_uint(__fadd_rn(qf, MAGIC));
+        for (int p = 0; p < 4; ++p) {
+            const float2 ww = make_float2(w[2 * p], w[2 * p + 1]);
+            const float2 tl = __ffma2_rn(ww, ilo, M2), th = __ffma2_rn(ww, ihi, M2);
+            diff |= (__float_as_uint(tl.x) ^ __float_as_uint(th.x)) | (__float_as_uint(tl.y) ^ __float_as_uint(th.y));
+            const int c0 = __vimin_s32_relu(static_cast<int>(__float_as_uint(tl.x)) + zo, HI);
+            const int c1 = __vimin_s32_relu(static_cast<int>(__float_as_uint(tl.y)) + zo, HI);
+            bytes[p] = static_cast<uint32_t>(c0 + 16 * c1);
         }
+        nib = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040u), __byte_perm(bytes[2], bytes[3], 0x0040u), 0x5410u);
+        exact = diff != 0u;
     }
     if (exact) {
+        nib = 0u;
+        const float zf = static_cast<float>(z);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float qf = zf;
-            if (s != 0.f) qf = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), zf), 0.f), hi);
-            code[i] = __float_as_uint(__fadd_rn(qf, MAGIC));
+            if (s != 0.f) qf = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), zf), 0.f), static_cast<float>(HI));
+            nib |= (static_cast<uint32_t>(qf) & 15u) << (4 * i);
         }
     }
-    if (n < 8) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            if (i >= n) code[i] = static_cast<unsigned>(z);
+    if (n < 8) {   // padding: code z
+        const uint32_t keep = n <= 0 ? 0u : (0xffffffffu >> (32 - 4 * n));
+        nib = (nib & keep) | ((static_cast<uint32_t>(z) & 15u) * 0x11111111u & ~keep);
     }
+    return nib;
 }
 
-// Stores an octet's integer codes into its share of the record: int3 = 2
-// low-plane bytes + 1 high-plane byte, int4 = 4 bytes.
+// Stores an octet's integer codes (8 nibbles) into its share of the record:
+// int3 = 2 low-plane bytes (bits 0-1 of each code) + 1 high-plane byte (bit
+// 2), gathered with shift-and-mask compression; int4 = the 4 bytes as they are.
 template <int FMT>
-__device__ __forceinline__ void store_oct(uint8_t* __restrict__ packed, int64_t gid, int oct, const unsigned code[8]) {
+__device__ __forceinline__ void store_oct(uint8_t* __restrict__ packed, int64_t gid, int oct, uint32_t nib) {
     if constexpr (FMT == TQ_INT3_G64_SYM) {
-        uint32_t lo = 0u, hi = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            lo |= (code[i] & 3u) << (2 * i);
-            hi |= ((code[i] >> 2) & 1u) << i;
-        }
+        uint32_t x = nib & 0x33333333u;
+        x = (x | (x >> 2)) & 0x0f0f0f0fu;
+        x = (x | (x >> 4)) & 0x00ff00ffu;
+        x = (x | (x >> 8)) & 0x0000ffffu;
+        uint32_t y = (nib >> 2) & 0x11111111u;
+        y = (y | (y >> 3)) & 0x03030303u;
+        y = (y | (y >> 6)) & 0x000f000fu;
+        y = (y | (y >> 12)) & 0x000000ffu;
         uint8_t* rec = packed + gid * 24;
-        reinterpret_cast<uint16_t*>(rec)[oct] = static_cast<uint16_t>(lo);
-        rec[16 + oct] = static_cast<uint8_t>(hi);
+        reinterpret_cast<uint16_t*>(rec)[oct] = static_cast<uint16_t>(x);
+        rec[16 + oct] = static_cast<uint8_t>(y);
     } else {
-        uint32_t a = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) a |= (code[i] & 15u) << (4 * i);
-        reinterpret_cast<uint32_t*>(packed + gid * 64)[oct] = a;
+        reinterpret_cast<uint32_t*>(packed + gid * 64)[oct] = nib;
     }
 }
 

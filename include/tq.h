@@ -255,9 +255,9 @@ tq_status tq_sync(tq_stream_t stream);
  * round-to-nearest (search, tq_pack) and decoding (tq_dequant,
  * tq_proxy_error) rely.  The pages define the element format only (E2M1:
  * values 0, .5, 1, 1.5, 2, 3, 4, 6 with a sign; [NVFP4] Quantization Recipe);
- * this call has no counterpart there.  Checks every non-negative finite fp32
- * value and +inf (rounded half to even, saturating at 6) in both nibbles of
- * a byte, and all 256 bytes decoded bit for bit.  *mismatches (host) gets the
+ * this call has no counterpart there.  Checks every fp32 value but NaN
+ * (rounded half to even, saturating at 6, sign in bit 3 even for -0) in both
+ * nibbles of a byte, and all 256 bytes decoded bit for bit.  *mismatches (host) gets the
  * number of failing cases, 0 on a conforming GPU; *first_bad (host, may be
  * NULL) the first failing fp32 pattern (0x80000000 | byte for a decode
  * failure, 0xffffffff when none).  Uses two words of static device memory

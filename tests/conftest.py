@@ -18,3 +18,17 @@ def orc():
     import oracle
     oracle.build()
     return oracle
+
+
+@pytest.fixture(autouse=True)
+def _device_status_after_gpu_test(request):
+    """After every GPU test: synchronise and fail if a kernel reported a
+    device-side problem (a launch error, or a bounded wait that gave up)."""
+    yield
+    if request.node.get_closest_marker("gpu") is None:
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import group_scale_search_b200 as tq
+    tq.tq_sync()
