@@ -71,19 +71,18 @@ __device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[
         const float inv = rcp_approx(S);
         const float lo = __fmul_rn(inv, 0.99999904632568359375f), hi = __fmul_rn(inv, 1.00000095367431640625f);
         const float2 lo2 = make_float2(lo, lo), hi2 = make_float2(hi, hi);
-        uint32_t diff = 0u, bytes[N / 2];
-#pragma unroll
-        for (int p = 0; p < N / 2; ++p) {
-            const float2 ww = make_float2(w[2 * p], w[2 * p + 1]);
-            const float2 yl = __fmul2_rn(ww, lo2), yh = __fmul2_rn(ww, hi2);
-            const unsigned bl = e2m1x2_from_f32(yl.x, yl.y), bh = e2m1x2_from_f32(yh.x, yh.y);
-            diff |= bl ^ bh;
-            bytes[p] = bl;
-        }
+        uint32_t diff = 0u;
 #pragma unroll
         for (int h = 0; h < N / 8; ++h) {
-            uint32_t x = __byte_perm(__byte_perm(bytes[4 * h], bytes[4 * h + 1], 0x0040u),
-                                     __byte_perm(bytes[4 * h + 2], bytes[4 * h + 3], 0x0040u), 0x5410u);
+            float yl[8], yh[8];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const float2 ww = make_float2(w[8 * h + 2 * p], w[8 * h + 2 * p + 1]);
+                const float2 a = __fmul2_rn(ww, lo2), b = __fmul2_rn(ww, hi2);
+                yl[2 * p] = a.x; yl[2 * p + 1] = a.y; yh[2 * p] = b.x; yh[2 * p + 1] = b.y;
+            }
+            const uint32_t x = e2m1x8_from_f32(yl[0], yl[1], yl[2], yl[3], yl[4], yl[5], yl[6], yl[7]);
+            diff |= x ^ e2m1x8_from_f32(yh[0], yh[1], yh[2], yh[3], yh[4], yh[5], yh[6], yh[7]);
             const uint32_t nz = (x | (x >> 1) | (x >> 2)) & 0x11111111u;   // magnitude != 0, per nibble
             m[h] = x & (0x77777777u | (nz << 3));
         }

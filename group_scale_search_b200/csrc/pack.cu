@@ -22,40 +22,69 @@ int64_t resident_blocks(K kernel, int threads) {
 // padding included); it writes its share of the record: int3 = 2 low-plane
 // bytes + 1 high-plane byte, int4 = 4 bytes, NVFP4 = half the record.
 
-template <int FMT, typename T>
-__device__ __forceinline__ void pack_oct(const float w[8], int n, const void* scales, const uint8_t* __restrict__ zeros,
-                                         float g, int64_t gid, int oct, uint8_t* __restrict__ packed) {
+// Octets per thread of tq_pack (one or two consecutive octets of one group:
+// two halve the per-row loads of scales and the loop work per weight, which
+// pays for the integer formats; NVFP4, whose block is two octets, is faster
+// with one).
+template <int FMT> constexpr int pk_no() { return FMT == TQ_NVFP4_G16 ? 1 : 2; }
+
+// RTN codes of NO consecutive octets (starting at octet `oct` of the group
+// whose record is at rec) into their share of the record.  sc: the group's
+// scale (NVFP4: the block scale S = fl32(g dec(e))); z: int4 zero-point.
+template <int FMT, typename T, int NO>
+__device__ __forceinline__ void pack_unit(const Oct<T> o[NO], const int n[NO], float sc, int z, uint8_t* rec,
+                                          int oct) {
     if constexpr (FMT == TQ_NVFP4_G16) {   // padding has w = 0: code 0
-        const float S = __fmul_rn(g, e4m3_value(__ldg(static_cast<const uint8_t*>(scales) + gid)));
-        uint32_t c;
-        nvfp4_rtn<8>(w, S, &c);
-        reinterpret_cast<uint32_t*>(packed + gid * 8)[oct & 1] = c;
-    } else if constexpr (FMT == TQ_INT3_G64_SYM) {
-        store_oct<FMT>(packed, gid, oct, rtn_int_oct<7>(w, n, __ldg(static_cast<const float*>(scales) + gid), 4));
+        float w[8 * NO];
+#pragma unroll
+        for (int i = 0; i < NO; ++i) o[i].get(w + 8 * i);
+        uint32_t m[NO];
+        nvfp4_rtn<8 * NO>(w, sc, m);
+        if constexpr (NO == 1) reinterpret_cast<uint32_t*>(rec)[oct & 1] = m[0];
+        else *reinterpret_cast<uint2*>(rec) = make_uint2(m[0], m[1]);
     } else {
-        store_oct<FMT>(packed, gid, oct,
-                       rtn_int_oct<15>(w, n, __ldg(static_cast<const float*>(scales) + gid), __ldg(zeros + gid)));
+        uint32_t nib[NO];
+#pragma unroll
+        for (int i = 0; i < NO; ++i) {
+            float w[8];
+            o[i].get(w);
+            nib[i] = FMT == TQ_INT3_G64_SYM ? rtn_int_oct<7>(w, n[i], sc, 4) : rtn_int_oct<15>(w, n[i], sc, z);
+        }
+        store_unit<FMT, NO>(rec, oct, nib);
     }
 }
 
-// Grid: x = octet-column tiles, y = blocks of consecutive rows of the whole
-// batch (rows of all matrices in order, so every block gets the same number
-// of rows whatever the matrix count).
-template <int FMT, typename T>
+// Grid: x = unit-column tiles (a unit = NO octets), y = blocks of
+// consecutive rows of the whole batch (rows of all matrices in order, so
+// every block gets the same number of rows whatever the matrix count).
+// Pointers to the weights, records, scales and zero-points advance by their
+// row strides.
+template <int FMT, typename T, int NO>
 __global__ void __launch_bounds__(256)
 k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, int64_t n_rows, int64_t rpb,
        const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
        uint8_t* __restrict__ packed) {
     using F = FmtTraits<FMT>;
     const int64_t G = (I + F::group - 1) / F::group;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (c >= (G << F::lg)) return;
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (u >= (G << F::lg) / NO) return;
+    const int64_t c = u * NO;   // first octet of the unit
     const int64_t k = c >> F::lg;
     const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
     const int64_t j = c << 3;
-    const int n = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j)));
+    int n[NO];
+#pragma unroll
+    for (int i = 0; i < NO; ++i)
+        n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
     const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rpb, r1 = min(n_rows, r0 + rpb);
     RowCursor<T> cur(W, O, ld, ms, j, r0);
+    const int64_t rstride = G * F::rec;
+    uint8_t* rec = packed + (r0 * G + k) * F::rec;
+    const float* sp = static_cast<const float*>(scales) + (r0 * G + k);          // int3, int4
+    const uint8_t* bp = static_cast<const uint8_t*>(scales) + (r0 * G + k);      // NVFP4 block scales
+    const uint8_t* zp = zeros ? zeros + (r0 * G + k) : nullptr;
+    int64_t ecur = cur.e;
+    float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + ecur) : 0.f;
     for (int64_t r = r0; r < r1; r += 2) {
         const bool two = r + 1 < r1;
         const T* wa = cur.ptr;
@@ -64,17 +93,36 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
         const T* wb = cur.ptr;
         const int64_t eb = cur.e;
         cur.next();
-        Oct<T> ra, rb;
-        ra.load(wa, n);
-        if (two) rb.load(wb, n);
-        float w[8];
-        ra.get(w);
-        pack_oct<FMT, T>(w, n, scales, zeros, FMT == TQ_NVFP4_G16 ? __ldg(gs + ea) : 0.f, r * G + k, oct, packed);
-        if (two) {
-            rb.get(w);
-            pack_oct<FMT, T>(w, n, scales, zeros, FMT == TQ_NVFP4_G16 ? __ldg(gs + eb) : 0.f, (r + 1) * G + k, oct,
-                             packed);
+        Oct<T> ra[NO], rb[NO];
+#pragma unroll
+        for (int i = 0; i < NO; ++i) {
+            ra[i].load(wa + 8 * i, n[i]);
+            if (two) rb[i].load(wb + 8 * i, n[i]);
         }
+        float sa, sb = 0.f;
+        int za = 0, zb = 0;
+        if constexpr (FMT == TQ_NVFP4_G16) {
+            const unsigned ca = __ldg(bp), cb = two ? __ldg(bp + G) : 0u;
+            if (ea != ecur) { ecur = ea; g = __ldg(gs + ecur); }
+            sa = __fmul_rn(g, e4m3_value(ca));
+            if (two) {
+                if (eb != ecur) { ecur = eb; g = __ldg(gs + ecur); }
+                sb = __fmul_rn(g, e4m3_value(cb));
+            }
+        } else {
+            sa = __ldg(sp);
+            if (two) sb = __ldg(sp + G);
+            if constexpr (FMT == TQ_INT4_G128_ASYM) {
+                za = __ldg(zp);
+                if (two) zb = __ldg(zp + G);
+            }
+        }
+        pack_unit<FMT, T, NO>(ra, n, sa, za, rec, oct);
+        if (two) pack_unit<FMT, T, NO>(rb, n, sb, zb, rec + rstride, oct);
+        rec += 2 * rstride;
+        sp += 2 * G;
+        bp += 2 * G;
+        if (FMT == TQ_INT4_G128_ASYM) zp += 2 * G;
     }
 }
 
@@ -188,13 +236,15 @@ k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t*
         next_e = (e + 1) * Orows;
         g = __ldg(gs + e);
     }
-    int64_t gid = r0 * G + k;
+    QPtr<FMT> qp(packed, scales, zeros, r0 * G + k, G);
     O* dst = out + r0 * I + j;
-    for (int64_t r = r0; r < r1; r += 2, gid += 2 * G, dst += 2 * I) {
+    for (int64_t r = r0; r < r1; r += 2, dst += 2 * I) {
         const bool two = r + 1 < r1;
-        const OctQ q0 = load_q<FMT>(packed, scales, zeros, gid, oct);
+        const OctQ q0 = load_q<FMT>(qp, oct);
+        qp.next();
         OctQ q1 = q0;
-        if (two) q1 = load_q<FMT>(packed, scales, zeros, gid + G, oct);
+        if (two) q1 = load_q<FMT>(qp, oct);
+        qp.next();
         float v[8];
         if (FMT == TQ_NVFP4_G16 && r == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
         dec_oct<FMT>(q0, g, v);
@@ -230,14 +280,14 @@ template <int FMT, typename T>
 void launch_pack(const tq_mat* W, int64_t ms, const void* scales, const uint8_t* zeros, const float* gs,
                  uint8_t* packed, cudaStream_t st) {
     const int64_t g = FmtTraits<FMT>::group;
-    const int64_t cols = (W->cols + g - 1) / g * (g / 8);
+    constexpr int NO = pk_no<FMT>();
+    const int64_t cols = (W->cols + g - 1) / g * (g / 8) / NO;
     const int64_t n_rows = W->n_mat * W->rows;
     const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
-    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_pack<FMT, T>, width));
+    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_pack<FMT, T, NO>, width));
     const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
-    k_pack<FMT, T><<<grid, static_cast<unsigned>(f.width), 0, st>>>(static_cast<const T*>(W->ptr), W->rows, W->cols,
-                                                                    W->ld, ms, n_rows, f.rpb, scales, zeros, gs,
-                                                                    packed);
+    k_pack<FMT, T, NO><<<grid, static_cast<unsigned>(f.width), 0, st>>>(
+        static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, n_rows, f.rpb, scales, zeros, gs, packed);
 }
 
 template <int FMT, typename O>
@@ -248,8 +298,8 @@ void launch_dequant(const uint8_t* packed, const void* scales, const uint8_t* ze
     const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
     const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_dequant<FMT, O>, width));
     const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
-    k_dequant<FMT, O><<<grid, static_cast<unsigned>(f.width), 0, st>>>(packed, scales, zeros, gs, Orows, I, n_rows,
-                                                                      f.rpb, static_cast<O*>(out));
+    k_dequant<FMT, O><<<grid, static_cast<unsigned>(f.width), 0, st>>>(packed, scales, zeros, gs, Orows, I,
+                                                                             n_rows, f.rpb, static_cast<O*>(out));
 }
 
 }  // namespace tq

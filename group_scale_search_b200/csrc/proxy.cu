@@ -4,12 +4,10 @@
 //   num = sum_{o,j} m_j (W - What)^2,  den = sum_{o,j} m_j W^2.
 //
 // B200 mapping (HBM-bound): one thread per octet (8 consecutive weights of a
-// group) walking the rows of its slice.  The block's weight tile streams into
-// shared memory by bulk copies (TMA, issued by one thread, completed on
-// mbarriers) PX_STAGES tiles of PX_RB rows ahead, so about 48 KB per block
-// are in flight without costing registers; each thread keeps its 8 imatrix
-// weights in registers, dequantizes in registers (no What round trip through
-// memory), sums the 8 terms in fp32 and folds them into fp64 per row.  Each block writes an fp64 partial to
+// group, one 16-byte load of bf16) walking the rows of its slice two at a
+// time; it keeps its 8 imatrix weights in registers, dequantizes in
+// registers (no What round trip through memory), sums the 8 terms in fp32
+// and folds them into fp64 per row.  Each block writes an fp64 partial to
 // the workspace; the last block of a matrix (atomic ticket) adds the
 // partials in block order, so the result is deterministic for a given
 // device.
@@ -20,10 +18,6 @@ namespace tq {
 // Fixed block budget, so the workspace size (one fp64 pair per block) does
 // not depend on the device.
 constexpr int64_t PX_TARGET_BLOCKS = 148 * 8;
-
-inline Walk px_geometry(int64_t n_mat, int64_t O, int64_t I) {
-    return walk_geometry(n_mat, O, (I + 7) / 8, PX_TARGET_BLOCKS);
-}
 
 // Adds the 8 terms of one octet in fp32 (two interleaved partial sums of
 // fp32x2 pairs): m (W - What)^2 and m W^2.
@@ -42,134 +36,78 @@ __device__ __forceinline__ void px_terms(const float w[8], const float v[8], con
     sd = __fadd_rn(ad.x, ad.y);
 }
 
-// Row data in flight: PX_STAGES stages of PX_RB rows of the block's weight
-// tile (its full octets: `width` x 16 bytes of bf16 per row), filled by bulk
-// copies that one thread issues; the packed bits and scales (a quarter to an
-// eighth of the bytes) are loaded by each thread one tile ahead.
-constexpr int PX_RB = 4;
-constexpr int PX_STAGES = 3;
+// Octets per thread (one or two consecutive octets of one group).
+constexpr int PX_NO = 2;
 
-template <typename T>
-inline size_t px_smem_bytes(int width) {
-    return 64 + static_cast<size_t>(PX_STAGES) * PX_RB * width * sizeof(T) * 8;
+inline Walk px_geometry(int64_t n_mat, int64_t O, int64_t I) {
+    return walk_geometry(n_mat, O, ((I + 7) / 8 + PX_NO - 1) / PX_NO, PX_TARGET_BLOCKS);
 }
 
-// Set when a wait for a bulk copy gave up (the results are then invalid);
-// read and cleared by tq_sync.
-static __device__ unsigned g_px_fault;
-
-template <int FMT, typename T>
-__global__ void __launch_bounds__(256)
+template <int FMT, typename T, int NO>
+__global__ void __launch_bounds__(256, NO == 1 ? 4 : 3)
 k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, const uint8_t* __restrict__ packed,
         const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
         const float* __restrict__ m, int64_t m_stride, int64_t rps, double* __restrict__ part_out,
         unsigned* __restrict__ tickets, double* __restrict__ num, double* __restrict__ den) {
     using F = FmtTraits<FMT>;
-    constexpr int OB = static_cast<int>(sizeof(T)) * 8;   // bytes of one octet of W
-    extern __shared__ __align__(128) uint8_t px_smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(px_smem);
-    uint8_t* tiles = px_smem + 64;
-    const int width = static_cast<int>(blockDim.x), t = static_cast<int>(threadIdx.x);
-    const size_t row_bytes = static_cast<size_t>(width) * OB, stage_bytes = PX_RB * row_bytes;
-
     const int64_t G = (I + F::group - 1) / F::group;
+    const int64_t C = (I + 7) >> 3;
     const int64_t e = blockIdx.z;
-    const int64_t c0 = static_cast<int64_t>(blockIdx.x) * width;
-    const int64_t c = c0 + t;
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
     const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     const int nwarps = static_cast<int>(blockDim.x >> 5);
-    const int64_t C = (I + 7) >> 3, CF = I >> 3;   // octets per row, full octets per row
-    const uint32_t seg = static_cast<uint32_t>(max(static_cast<int64_t>(0), min(CF - c0, static_cast<int64_t>(width))) * OB);
-    const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rps, o1 = min(O, o0 + rps);
-    const int64_t ntiles = (o1 - o0 + PX_RB - 1) / PX_RB;
-    const T* wtile = W + e * ms + c0 * 8;   // row o of the tile at wtile + o * ld
-
-    if (t == 0) {
-#pragma unroll
-        for (int st = 0; st < PX_STAGES; ++st) mbar_init(&bars[st], 1);
-        mbar_init_fence();
-    }
-    __syncthreads();
-    auto issue = [&](int64_t tile) {
-        const int st = static_cast<int>(tile % PX_STAGES);
-        const int64_t r0 = o0 + tile * PX_RB;
-        const int rows = static_cast<int>(min(static_cast<int64_t>(PX_RB), o1 - r0));
-        mbar_expect_tx(&bars[st], static_cast<uint32_t>(rows) * seg);
-        if (seg)
-            for (int r = 0; r < rows; ++r)
-                bulk_g2s(tiles + st * stage_bytes + r * row_bytes, wtile + (r0 + r) * ld, seg, &bars[st]);
-    };
-    if (t == 0)
-        for (int64_t tile = 0; tile < min(static_cast<int64_t>(PX_STAGES), ntiles); ++tile) issue(tile);
-
-    const bool active = c < C;
-    const int64_t k = c >> F::lg;
-    const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
-    const int64_t j = c << 3;
-    const int n = active ? static_cast<int>(min(static_cast<int64_t>(8), I - j)) : 0;
-    float mm[8];
-    {
-        Oct<float> mo;
-        mo.load(m + e * m_stride + j, n);
-        mo.get(mm);
-    }
-    const float g = (FMT == TQ_NVFP4_G16 && active) ? __ldg(gs + e) : 0.f;
-    const int64_t gbase = e * O * G + k;
-    OctQ qn[PX_RB];
-#pragma unroll
-    for (int r = 0; r < PX_RB; ++r)
-        if (active && o0 + r < o1) qn[r] = load_q<FMT>(packed, scales, zeros, gbase + (o0 + r) * G, oct);
     double an = 0.0, ad = 0.0;
-    int64_t tile = 0;
-    for (; tile < ntiles; ++tile) {
-        const int st = static_cast<int>(tile % PX_STAGES);
-        const int64_t r0 = o0 + tile * PX_RB;
-        OctQ qc[PX_RB];
+    if (u < (C + NO - 1) / NO) {
+        const int64_t c = u * NO;
+        const int64_t k = c >> F::lg;
+        const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
+        const int64_t j = c << 3;
+        int n[NO];
+        float mm[NO][8];
 #pragma unroll
-        for (int r = 0; r < PX_RB; ++r) qc[r] = qn[r];
+        for (int i = 0; i < NO; ++i) {
+            n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
+            Oct<float> mo;
+            mo.load(m + e * m_stride + j + 8 * i, n[i]);
+            mo.get(mm[i]);
+        }
+        const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
+        const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rps, o1 = min(O, o0 + rps);
+        const T* wp = W + e * ms + o0 * ld + j;
+        QPtr<FMT> qp(packed, scales, zeros, (e * O + o0) * G + k, G);
+        for (int64_t o = o0; o < o1; o += 2, wp += 2 * ld) {
+            const bool two = o + 1 < o1;
+            Oct<T> ra[NO], rb[NO];
 #pragma unroll
-        for (int r = 0; r < PX_RB; ++r)   // next tile's codes and scales, while this one is worked on
-            if (active && r0 + PX_RB + r < o1) qn[r] = load_q<FMT>(packed, scales, zeros, gbase + (r0 + PX_RB + r) * G, oct);
-        const bool got = mbar_wait(&bars[st], static_cast<uint32_t>((tile / PX_STAGES) & 1));
-        if (active && got) {
+            for (int i = 0; i < NO; ++i) ra[i].load(wp + 8 * i, n[i]);
+            const UnitQ<NO> q0 = load_unit_q<FMT, NO>(qp, oct);
+            qp.next();
+            UnitQ<NO> q1 = q0;
+            if (two) {
 #pragma unroll
-            for (int r = 0; r < PX_RB; ++r) {
-                if (r0 + r >= o1) break;
-                Oct<T> ow;
-                if (n == 8) {
-                    const uint4* src = reinterpret_cast<const uint4*>(tiles + st * stage_bytes + r * row_bytes + t * OB);
-                    if constexpr (sizeof(T) == 2) {
-                        ow.v = src[0];
-                    } else {
-                        const uint4 a = src[0], b = src[1];
-                        ow.a = make_float4(__uint_as_float(a.x), __uint_as_float(a.y), __uint_as_float(a.z), __uint_as_float(a.w));
-                        ow.b = make_float4(__uint_as_float(b.x), __uint_as_float(b.y), __uint_as_float(b.z), __uint_as_float(b.w));
-                    }
-                } else {
-                    ow.load(W + e * ms + (r0 + r) * ld + j, n);   // the row's last, partial octet
+                for (int i = 0; i < NO; ++i) rb[i].load(wp + ld + 8 * i, n[i]);
+                q1 = load_unit_q<FMT, NO>(qp, oct);
+            }
+            qp.next();
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if (h == 1 && !two) break;
+                const UnitQ<NO>& q = h ? q1 : q0;
+                float sn = 0.f, sd = 0.f;
+#pragma unroll
+                for (int i = 0; i < NO; ++i) {
+                    float w[8], v[8], tn, td;
+                    (h ? rb : ra)[i].get(w);
+                    dec_oct<FMT>(OctQ{q.bits[i], q.s, q.z}, g, v);
+                    px_terms(w, v, mm[i], tn, td);
+                    sn = __fadd_rn(sn, tn);
+                    sd = __fadd_rn(sd, td);
                 }
-                float w[8], v[8], sn, sd;
-                ow.get(w);
-                dec_oct<FMT>(qc[r], g, v);
-                px_terms(w, v, mm, sn, sd);
                 an += static_cast<double>(sn);
                 ad += static_cast<double>(sd);
             }
         }
-        if (__syncthreads_or(!got)) break;   // every thread has read the stage (or a wait gave up)
-        if (t == 0 && tile + PX_STAGES < ntiles) {
-            fence_proxy_async_smem();
-            issue(tile + PX_STAGES);
-        }
-    }
-    if (tile < ntiles) {   // a wait gave up: flag it and let the copies in flight land before exiting
-        if (t == 0) {
-            atomicOr(&g_px_fault, 1u);
-            for (int64_t u = tile; u < min(ntiles, tile + PX_STAGES); ++u)
-                mbar_wait(&bars[u % PX_STAGES], static_cast<uint32_t>((u / PX_STAGES) & 1));
-        }
-        an = ad = 0.0;
     }
     // block reduction in fp64, fixed order
 #pragma unroll
@@ -222,29 +160,18 @@ template <int FMT, typename T>
 void launch_proxy(const tq_mat* W, int64_t ms, const uint8_t* packed, const void* scales, const uint8_t* zeros,
                   const float* gs, const float* m, int64_t mst, double* parts, unsigned* tickets, double* num,
                   double* den, cudaStream_t st) {
-    const int64_t cols = (W->cols + 7) / 8;
+    const int64_t cols = ((W->cols + 7) / 8 + PX_NO - 1) / PX_NO;
     Walk pg = walk_geometry(W->n_mat, W->rows, cols, 1);
-    const size_t smem = px_smem_bytes<T>(static_cast<int>(pg.width));
-    cudaFuncSetAttribute(k_proxy<FMT, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T>, static_cast<int>(pg.width), smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T, PX_NO>, static_cast<int>(pg.width), 0) !=
             cudaSuccess || per_sm < 1)
         per_sm = 1;
     pg = walk_geometry(W->n_mat, W->rows, cols, min(PX_TARGET_BLOCKS, static_cast<int64_t>(num_sms()) * per_sm),
                        false);
     const dim3 grid(static_cast<unsigned>(pg.cblocks), static_cast<unsigned>(pg.slices), static_cast<unsigned>(W->n_mat));
-    k_proxy<FMT, T><<<grid, static_cast<unsigned>(pg.width), smem, st>>>(static_cast<const T*>(W->ptr), W->rows,
-                                                                         W->cols, W->ld, ms, packed, scales, zeros, gs,
-                                                                         m, mst, pg.rps, parts, tickets, num, den);
-}
-
-// Reads and clears the bulk-copy wait flag of the proxy kernels (tq_sync).
-bool take_proxy_fault() {
-    unsigned f = 0;
-    const unsigned zero = 0;
-    if (cudaMemcpyFromSymbol(&f, g_px_fault, sizeof f) != cudaSuccess) return false;
-    if (f) cudaMemcpyToSymbol(g_px_fault, &zero, sizeof zero);
-    return f != 0;
+    k_proxy<FMT, T, PX_NO><<<grid, static_cast<unsigned>(pg.width), 0, st>>>(
+        static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, packed, scales, zeros, gs, m, mst, pg.rps, parts,
+        tickets, num, den);
 }
 
 }  // namespace tq

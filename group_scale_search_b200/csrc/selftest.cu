@@ -7,7 +7,8 @@
 // Rounding: every fp32 value but NaN (both signs, zeros and infinities
 // included; a negative value keeps its sign bit in bit 3 of the nibble, -0
 // too), once in the low nibble (paired with 6.0) and once in the high nibble
-// (paired with 0.0), so both the values and the nibble order are checked.
+// (paired with 0.0), so both the values and the nibble order are checked,
+// and once through the eight-value form used for whole octets.
 // Decoding: all 256 bytes, bit for bit (code 8 is -0).
 #include "tq_internal.cuh"
 
@@ -27,7 +28,10 @@ __global__ void k_selftest_e2m1_round() {
         const unsigned r = static_cast<unsigned>(e2m1_mag_code(e2m1_round(fabsf(y)))) | ((u >> 28) & 8u);
         const unsigned a = e2m1x2_from_f32(y, 6.0f);
         const unsigned b = e2m1x2_from_f32(0.0f, y);
-        if (a != (r | 0x70u) || b != (r << 4)) {
+        // eight at once: (y, 6, 0, y, -y, 1, y, .5) -> nibbles (r, 7, 0, r, r ^ 8, 2, r, 1)
+        const uint32_t w8 = e2m1x8_from_f32(y, 6.0f, 0.0f, y, -y, 1.0f, y, 0.5f);
+        const uint32_t e8 = r | (7u << 4) | (r << 12) | ((r ^ 8u) << 16) | (2u << 20) | (r << 24) | (1u << 28);
+        if (a != (r | 0x70u) || b != (r << 4) || w8 != e8) {
             ++bad;
             first = min(first, u);
         }

@@ -85,8 +85,5 @@ TQ_API tq_status tq_sync(tq_stream_t stream) {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return set_error(TQ_ERR_CUDA, "tq_sync: %s", cudaGetErrorString(e));
-    if (take_proxy_fault())
-        return set_error(TQ_ERR_CUDA, "tq_sync: a proxy-error kernel gave up waiting for a bulk copy; "
-                                      "its results are invalid");
     return TQ_OK;
 }

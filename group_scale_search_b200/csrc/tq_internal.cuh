@@ -43,10 +43,6 @@ tq_status check_mat(const tq_mat* X, const char* name);
 
 int num_sms();
 
-// Reads and clears the flag the proxy kernels set when a bounded wait for a
-// bulk copy gives up (proxy.cu).
-bool take_proxy_fault();
-
 // ------------------------------------------------------------------ index arithmetic
 
 // Division of 32-bit unsigned integers by a fixed divisor d >= 1 with a
@@ -204,6 +200,24 @@ __device__ __forceinline__ unsigned e2m1x2_from_f32(float lo, float hi) {
     unsigned short r;
     asm("{ .reg .b8 t; cvt.rn.satfinite.e2m1x2.f32 t, %2, %1; cvt.u16.u8 %0, t; }" : "=h"(r) : "f"(lo), "f"(hi));
     return r;
+}
+
+// Eight values at once: the four e2m1x2 bytes of (x0, x1) .. (x6, x7) packed
+// into one word, element i in bits 4i..4i+3.
+__device__ __forceinline__ uint32_t e2m1x8_from_f32(float x0, float x1, float x2, float x3, float x4, float x5,
+                                                    float x6, float x7) {
+    uint32_t w;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b16 h0, h1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b16 h0, {b0, b1};\n\t"
+        "mov.b16 h1, {b2, b3};\n\t"
+        "mov.b32 %0, {h0, h1};\n\t}"
+        : "=r"(w)
+        : "f"(x0), "f"(x1), "f"(x2), "f"(x3), "f"(x4), "f"(x5), "f"(x6), "f"(x7));
+    return w;
 }
 
 // The two E2M1 values of an e2m1x2 byte (low nibble first) as fp32, exactly

@@ -73,49 +73,6 @@ struct RowCursor {
     }
 };
 
-// ------------------------------------------------------------------ device: bulk copies (TMA)
-// One-dimensional bulk copies global -> shared (cp.async.bulk, no tensor map,
-// no multicast), completed on an mbarrier that counts the bytes.  Waits are
-// bounded: after TQ_WAIT_POLLS polls a wait gives up and returns false.
-
-constexpr uint32_t TQ_WAIT_POLLS = 1u << 22;
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
-}
-// Makes barrier initialisation visible to the bulk-copy (async) proxy.
-__device__ __forceinline__ void mbar_init_fence() {
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-// Orders this thread's earlier shared-memory accesses before later bulk copies.
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-    const uint32_t a = smem_u32(bar);
-    for (uint32_t it = 0; it < TQ_WAIT_POLLS; ++it) {
-        uint32_t done;
-        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t}"
-                     : "=r"(done)
-                     : "r"(a), "r"(parity)
-                     : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-
 // ------------------------------------------------------------------ device: weights
 
 // The 8 weights of an octet as loaded (n of them valid, the rest 0): one
@@ -169,37 +126,112 @@ template <> struct Oct<float> {
 
 // ------------------------------------------------------------------ device: codes of one octet
 
-// The packed bits, scale and zero-point of octet `oct` of group `gid`.
-// bits: int3 = its 2 low-plane bytes (bits 0..15) and its high-plane byte
-// (bits 16..23); int4 = its 4 record bytes; NVFP4 = its half of the 8-byte
-// record.  For NVFP4, s is the decoded E4M3 block scale (the caller
-// multiplies by the global scale).
+// Where one thread's octet sits in the per-group outputs of a row: its
+// group's record, scale and zero-point.  Advancing to the next row adds the
+// row strides (G records / scales / zero-points), no index arithmetic.
+template <int FMT>
+struct QPtr {
+    const uint8_t* rec;
+    const void* sc;
+    const uint8_t* zp;
+    int64_t G;
+    __device__ __forceinline__ QPtr(const uint8_t* packed, const void* scales, const uint8_t* zeros, int64_t gid,
+                                    int64_t G_)
+        : G(G_) {
+        rec = packed + gid * FmtTraits<FMT>::rec;
+        sc = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(scales) + gid)
+                                 : static_cast<const void*>(static_cast<const float*>(scales) + gid);
+        zp = zeros ? zeros + gid : nullptr;
+    }
+    __device__ __forceinline__ void next() {
+        rec += G * FmtTraits<FMT>::rec;
+        sc = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(sc) + G)
+                                 : static_cast<const void*>(static_cast<const float*>(sc) + G);
+        if (FMT == TQ_INT4_G128_ASYM) zp += G;
+    }
+};
+
+// The packed bits, scale and zero-point of octet `oct` of the group at q.
+// bits: int3 = its 8 codes u as nibbles (built from its 2 low-plane bytes and
+// its high-plane byte); int4 = its 4 record bytes (8 nibbles); NVFP4 = its
+// half of the 8-byte record.  For NVFP4, s is the decoded E4M3 block scale
+// (the caller multiplies by the global scale).
 struct OctQ {
     uint32_t bits;
     float s;
     int z;
 };
 
+// 8 int3 codes from their planes: lo = 8 x 2 bits (element k at bits 2k,
+// 2k+1), hi = 8 x 1 bit (element k at bit k) -> 8 nibbles, by shift-and-mask
+// spreading of both planes.
+__device__ __forceinline__ uint32_t int3_nibbles(uint32_t lo, uint32_t hi) {
+    uint32_t x = lo;
+    x = (x | (x << 8)) & 0x00ff00ffu;
+    x = (x | (x << 4)) & 0x0f0f0f0fu;
+    x = (x | (x << 2)) & 0x33333333u;
+    uint32_t y = hi;
+    y = (y | (y << 12)) & 0x000f000fu;
+    y = (y | (y << 6)) & 0x03030303u;
+    y = (y | (y << 3)) & 0x11111111u;
+    return x | (y << 2);
+}
+
 template <int FMT>
-__device__ __forceinline__ OctQ load_q(const uint8_t* __restrict__ packed, const void* scales,
-                                       const uint8_t* __restrict__ zeros, int64_t gid, int oct) {
-    OctQ q;
+__device__ __forceinline__ OctQ load_q(const QPtr<FMT>& q, int oct) {
+    OctQ o;
     if constexpr (FMT == TQ_INT3_G64_SYM) {
-        const uint8_t* rec = packed + gid * 24;
-        q.bits = static_cast<uint32_t>(__ldg(reinterpret_cast<const uint16_t*>(rec) + oct)) |
-                 (static_cast<uint32_t>(__ldg(rec + 16 + oct)) << 16);
-        q.s = __ldg(static_cast<const float*>(scales) + gid);
-        q.z = 4;
+        o.bits = int3_nibbles(__ldg(reinterpret_cast<const uint16_t*>(q.rec) + oct), __ldg(q.rec + 16 + oct));
+        o.s = __ldg(static_cast<const float*>(q.sc));
+        o.z = 4;
     } else if constexpr (FMT == TQ_INT4_G128_ASYM) {
-        q.bits = __ldg(reinterpret_cast<const uint32_t*>(packed + gid * 64) + oct);
-        q.s = __ldg(static_cast<const float*>(scales) + gid);
-        q.z = __ldg(zeros + gid);
+        o.bits = __ldg(reinterpret_cast<const uint32_t*>(q.rec) + oct);
+        o.s = __ldg(static_cast<const float*>(q.sc));
+        o.z = __ldg(q.zp);
     } else {
-        q.bits = __ldg(reinterpret_cast<const uint32_t*>(packed + gid * 8) + (oct & 1));
-        q.s = e4m3_value(__ldg(static_cast<const uint8_t*>(scales) + gid));
-        q.z = 0;
+        o.bits = __ldg(reinterpret_cast<const uint32_t*>(q.rec) + (oct & 1));
+        o.s = e4m3_value(__ldg(static_cast<const uint8_t*>(q.sc)));
+        o.z = 0;
     }
-    return q;
+    return o;
+}
+
+// The codes and scale of NO consecutive octets starting at octet `oct` (a
+// multiple of NO, so all of them lie in the group at q): bits[i] for octet
+// oct + i, in the form load_q gives.
+template <int NO>
+struct UnitQ {
+    uint32_t bits[NO];
+    float s;
+    int z;
+};
+
+template <int FMT, int NO>
+__device__ __forceinline__ UnitQ<NO> load_unit_q(const QPtr<FMT>& q, int oct) {
+    static_assert(NO == 1 || NO == 2, "units of one or two octets");
+    UnitQ<NO> u;
+    if constexpr (NO == 1) {
+        const OctQ o = load_q<FMT>(q, oct);
+        u.bits[0] = o.bits; u.s = o.s; u.z = o.z;
+    } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+        const uint32_t lo = __ldg(reinterpret_cast<const uint32_t*>(q.rec + 2 * oct));
+        const uint32_t hi = __ldg(reinterpret_cast<const uint16_t*>(q.rec + 16 + oct));
+        u.bits[0] = int3_nibbles(lo & 0xffffu, hi & 0xffu);
+        u.bits[1] = int3_nibbles(lo >> 16, hi >> 8);
+        u.s = __ldg(static_cast<const float*>(q.sc));
+        u.z = 4;
+    } else {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(q.rec + (FMT == TQ_NVFP4_G16 ? 0 : 4 * oct)));
+        u.bits[0] = v.x; u.bits[1] = v.y;
+        if constexpr (FMT == TQ_INT4_G128_ASYM) {
+            u.s = __ldg(static_cast<const float*>(q.sc));
+            u.z = __ldg(q.zp);
+        } else {
+            u.s = e4m3_value(__ldg(static_cast<const uint8_t*>(q.sc)));
+            u.z = 0;
+        }
+    }
+    return u;
 }
 
 // 2^23 + k for a small non-negative integer k, as a float; subtracting 2^23
@@ -213,17 +245,15 @@ __device__ __forceinline__ float f23(unsigned k) { return __uint_as_float(0x4b00
 // NVFP4 bytes are decoded by the hardware E2M1 conversion (exact).
 template <int FMT>
 __device__ __forceinline__ void dec_oct(const OctQ& q, float g, float v[8]) {
-    if constexpr (FMT == TQ_INT3_G64_SYM) {
-        const float2 noff = make_float2(-8388612.0f, -8388612.0f);   // -(2^23 + 4): stored u = v + 4
-        const float2 s2 = make_float2(q.s, q.s);
+    if constexpr (FMT == TQ_NVFP4_G16) {
+        const float S = __fmul_rn(g, q.s);
+        const float2 S2 = make_float2(S, S);
 #pragma unroll
-        for (int i = 0; i < 8; i += 2) {
-            const unsigned u0 = ((q.bits >> (2 * i)) & 3u) | (((q.bits >> (16 + i)) & 1u) << 2);
-            const unsigned u1 = ((q.bits >> (2 * i + 2)) & 3u) | (((q.bits >> (17 + i)) & 1u) << 2);
-            const float2 r = __fmul2_rn(s2, __fadd2_rn(make_float2(f23(u0), f23(u1)), noff));
-            v[i] = r.x; v[i + 1] = r.y;
+        for (int b = 0; b < 4; ++b) {
+            const float2 r = __fmul2_rn(S2, e2m1x2_to_f32((q.bits >> (8 * b)) & 0xffu));
+            v[2 * b] = r.x; v[2 * b + 1] = r.y;
         }
-    } else if constexpr (FMT == TQ_INT4_G128_ASYM) {
+    } else {   // int3 (u = v + 4, z = 4) and int4: s (q - z) from 8 nibbles
         const float o = f23(static_cast<unsigned>(q.z) & 0xffu);   // 2^23 + z
         const float2 noff = make_float2(-o, -o), s2 = make_float2(q.s, q.s);
         const uint32_t ev = q.bits & 0x0f0f0f0fu, od = (q.bits >> 4) & 0x0f0f0f0fu;   // elements 2k, 2k+1 in byte k
@@ -234,14 +264,6 @@ __device__ __forceinline__ void dec_oct(const OctQ& q, float g, float v[8]) {
                                          __uint_as_float(__byte_perm(od, 0x4b00u, sel)));
             const float2 r = __fmul2_rn(s2, __fadd2_rn(x, noff));
             v[2 * k] = r.x; v[2 * k + 1] = r.y;
-        }
-    } else {
-        const float S = __fmul_rn(g, q.s);
-        const float2 S2 = make_float2(S, S);
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const float2 r = __fmul2_rn(S2, e2m1x2_to_f32((q.bits >> (8 * b)) & 0xffu));
-            v[2 * b] = r.x; v[2 * b + 1] = r.y;
         }
     }
 }
@@ -303,11 +325,12 @@ __device__ __forceinline__ uint32_t rtn_int_oct(const float w[8], int n, float s
     return nib;
 }
 
-// Stores an octet's integer codes (8 nibbles) into its share of the record:
-// int3 = 2 low-plane bytes (bits 0-1 of each code) + 1 high-plane byte (bit
-// 2), gathered with shift-and-mask compression; int4 = the 4 bytes as they are.
+// Stores an octet's integer codes (8 nibbles) into its share of the record
+// at rec: int3 = 2 low-plane bytes (bits 0-1 of each code) + 1 high-plane
+// byte (bit 2), gathered with shift-and-mask compression; int4 = the 4 bytes
+// as they are.
 template <int FMT>
-__device__ __forceinline__ void store_oct(uint8_t* __restrict__ packed, int64_t gid, int oct, uint32_t nib) {
+__device__ __forceinline__ void store_oct(uint8_t* rec, int oct, uint32_t nib) {
     if constexpr (FMT == TQ_INT3_G64_SYM) {
         uint32_t x = nib & 0x33333333u;
         x = (x | (x >> 2)) & 0x0f0f0f0fu;
@@ -317,11 +340,38 @@ __device__ __forceinline__ void store_oct(uint8_t* __restrict__ packed, int64_t 
         y = (y | (y >> 3)) & 0x03030303u;
         y = (y | (y >> 6)) & 0x000f000fu;
         y = (y | (y >> 12)) & 0x000000ffu;
-        uint8_t* rec = packed + gid * 24;
         reinterpret_cast<uint16_t*>(rec)[oct] = static_cast<uint16_t>(x);
         rec[16 + oct] = static_cast<uint8_t>(y);
     } else {
-        reinterpret_cast<uint32_t*>(packed + gid * 64)[oct] = nib;
+        reinterpret_cast<uint32_t*>(rec)[oct] = nib;
+    }
+}
+
+// Stores NO octets' integer codes (nibble words) into the record at rec,
+// starting at octet `oct` (a multiple of NO).
+template <int FMT, int NO>
+__device__ __forceinline__ void store_unit(uint8_t* rec, int oct, const uint32_t nib[NO]) {
+    if constexpr (NO == 1) {
+        store_oct<FMT>(rec, oct, nib[0]);
+    } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+        uint32_t lo = 0u, hi = 0u;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+            uint32_t x = nib[i] & 0x33333333u;
+            x = (x | (x >> 2)) & 0x0f0f0f0fu;
+            x = (x | (x >> 4)) & 0x00ff00ffu;
+            x = (x | (x >> 8)) & 0x0000ffffu;
+            uint32_t y = (nib[i] >> 2) & 0x11111111u;
+            y = (y | (y >> 3)) & 0x03030303u;
+            y = (y | (y >> 6)) & 0x000f000fu;
+            y = (y | (y >> 12)) & 0x000000ffu;
+            lo |= x << (16 * i);
+            hi |= y << (8 * i);
+        }
+        *reinterpret_cast<uint32_t*>(rec + 2 * oct) = lo;
+        *reinterpret_cast<uint16_t*>(rec + 16 + oct) = static_cast<uint16_t>(hi);
+    } else {
+        *reinterpret_cast<uint2*>(rec + 4 * oct) = make_uint2(nib[0], nib[1]);
     }
 }
 
