@@ -246,6 +246,27 @@ def oracle_sample(wl, budget_s: float = 12.0):
     return n / dt, oracle.num_threads(), desc, dt
 
 
+def oracle_one_thread(config: str, frac: float = 0.01):
+    """The same oracle on one host thread (OMP_NUM_THREADS=1 in a child
+    process, so the parent's thread pool is untouched) over a fixed `frac` of
+    the first unit's rows: the scaling reference for the multi-core figure.
+    Returns (weights/s, description) or None if the child fails."""
+    import subprocess
+    code = (f"import json, time, synth, bench, oracle; oracle.build(); wl = synth.make({config!r}, 'cpu'); "
+            f"u = [x for x in wl.units if x.timed][0]; rows = max(8, int(u.W.shape[1] * {frac!r})); "
+            f"t0 = time.perf_counter(); bench._oracle_unit(oracle, wl, u, rows); dt = time.perf_counter() - t0; "
+            f"print(json.dumps([rows * u.W.shape[2] / dt, rows, u.W.shape[2], oracle.num_threads(), dt]))")
+    env = dict(os.environ, OMP_NUM_THREADS="1")
+    try:
+        r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, env=env,
+                           cwd=os.path.dirname(os.path.abspath(__file__)))
+        v, rows, cols, threads, dt = json.loads(r.stdout.strip().splitlines()[-1])
+    except Exception:   # noqa: BLE001 -- the figure is optional context
+        return None
+    return v, (f"{rows} rows x {cols} of the first unit ({frac:.0%}), {threads} thread, imatrix of the site "
+               f"+ search+pack + dequant + proxy, {dt:.1f} s")
+
+
 def _oracle_unit(oracle, wl, u, rows):
     X = wl.sites[u.site].X[0].float().cpu().numpy()
     m = oracle.imatrix(X).astype(np.float32)
@@ -430,6 +451,9 @@ def main():
         v, cores, desc, dt = oracle_sample(wl)
         line["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
                                 "sample": desc, "seconds": dt}
+        one = oracle_one_thread(args.config)
+        if one is not None:
+            line["cpu_baseline"]["one_thread"] = {"value": one[0], "unit": "weights/s", "sample": one[1]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

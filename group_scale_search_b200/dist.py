@@ -3,10 +3,12 @@ torch.distributed: NCCL on GPUs, gloo on CPU for tests).
 
 The search, RTN, packing, dequantization and proxy error act on independent
 groups, so GPUs split the work (whole matrices, or row ranges of one matrix)
-and exchange nothing.  The one exchange is token-sharded calibration: every
-rank sums x^2 over its own tokens (tq_imatrix with alpha = 1) and an
+and exchange nothing.  The exchanges are small and only arise when one
+matrix or one calibration set is split: token-sharded calibration (every
+rank sums x^2 over its own tokens with tq_imatrix(alpha = 1) and an
 all-reduce adds the partial sums before the division by the total token
-count.
+count), and a row-sharded matrix's proxy error (an all-reduce of the
+per-matrix fp64 (num, den) pairs before the ratio).
 """
 from __future__ import annotations
 
@@ -16,7 +18,7 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 import torch.distributed as dist
 
-__all__ = ["shard_range", "shard_units", "allreduce_imatrix", "max_over_ranks", "init_from_env"]
+__all__ = ["shard_range", "shard_units", "allreduce_imatrix", "allreduce_proxy", "max_over_ranks", "init_from_env"]
 
 
 def shard_range(n: int, rank: int, world: int) -> Tuple[int, int]:
@@ -53,6 +55,19 @@ def allreduce_imatrix(local_sums: torch.Tensor, total_tokens: int, group=None) -
     if dist.is_available() and dist.is_initialized():
         dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
     return (acc / float(total_tokens)).to(torch.float32)
+
+
+def allreduce_proxy(num: torch.Tensor, den: torch.Tensor, group=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Proxy error of matrices whose rows are split over ranks: every rank
+    passes tq_proxy_error's fp64 (num, den) of its own rows; the sums over
+    ranks are the whole matrices' tr(E H E^T) and tr(W H W^T) (the ratio is
+    taken after the sum, never averaged over ranks)."""
+    if num.dtype != torch.float64 or den.dtype != torch.float64:
+        raise ValueError("num and den must be float64")
+    both = torch.stack([num, den])
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(both, op=dist.ReduceOp.SUM, group=group)
+    return both[0], both[1]
 
 
 def max_over_ranks(value: float, device: Optional[torch.device] = None, group=None) -> float:

@@ -33,6 +33,30 @@ def imatrix_shards(rank, world, port, root, out_dir):
     dist.destroy_process_group()
 
 
+def proxy_row_shards(rank, world, port, root, out_dir):
+    """Each rank takes half of the rows of every matrix and reduces its
+    (num, den); the all-reduced sums are the whole matrices'."""
+    sys.path.insert(0, root)
+    import oracle
+    from group_scale_search_b200.dist import allreduce_proxy, shard_range
+    _init(rank, world, port)
+    rng = np.random.default_rng(4)                      # same data on every rank
+    E, O, I = 3, 37, 200
+    W = (rng.standard_t(4, size=(E, O, I)) * 0.02).astype(np.float32)
+    What = (W + rng.normal(0, 1e-3, size=W.shape)).astype(np.float32)
+    m = rng.lognormal(0, 1, size=(E, I)).astype(np.float32)
+    o0, o1 = shard_range(O, rank, world)
+    nums, dens = [], []
+    for e in range(E):
+        n, d = oracle.proxy_error(W[e, o0:o1], What[e, o0:o1], m[e])
+        nums.append(n)
+        dens.append(d)
+    num, den = allreduce_proxy(torch.tensor(nums, dtype=torch.float64), torch.tensor(dens, dtype=torch.float64))
+    np.save(os.path.join(out_dir, f"p{rank}.npy"), np.stack([num.numpy(), den.numpy()]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def peer_dies(rank, world, port, out_dir):
     """Rank 1 leaves before the collective; rank 0 must get an error, not hang."""
     _init(rank, world, port, timeout_s=8.0)

@@ -1,6 +1,7 @@
 """Multi-process (N > 1) host path on CPU with gloo ranks: work sharding,
-token-sharded imatrix all-reduce, max-over-ranks timing, and a rank that dies
-before a collective (the survivor must fail fast, not hang)."""
+token-sharded imatrix all-reduce, row-sharded proxy-error all-reduce,
+max-over-ranks timing, and a rank that dies before a collective (the
+survivor must fail fast, not hang)."""
 import multiprocessing as mp
 import os
 import socket
@@ -67,6 +68,21 @@ def test_token_sharded_imatrix_allreduce(tmp_path):
         m = np.load(tmp_path / f"m{r}.npy")
         assert np.max(np.abs(m - ref) / ref) <= 1e-6
         assert np.load(tmp_path / f"t{r}.npy")[0] == 2.0      # max over ranks of (rank + 1)
+
+
+def test_row_sharded_proxy_allreduce(tmp_path):
+    import oracle
+    codes = _run(dist_workers.proxy_row_shards, (_port(), ROOT, str(tmp_path)))
+    assert codes == [0, 0]
+    rng = np.random.default_rng(4)
+    E, O, I = 3, 37, 200
+    W = (rng.standard_t(4, size=(E, O, I)) * 0.02).astype(np.float32)
+    What = (W + rng.normal(0, 1e-3, size=W.shape)).astype(np.float32)
+    m = rng.lognormal(0, 1, size=(E, I)).astype(np.float32)
+    ref = np.array([oracle.proxy_error(W[e], What[e], m[e]) for e in range(E)]).T
+    for r in range(2):
+        got = np.load(tmp_path / f"p{r}.npy")
+        assert np.max(np.abs(got - ref) / ref) <= 1e-12      # fp64 sums of two halves
 
 
 def test_surviving_rank_fails_fast_when_a_peer_dies(tmp_path):
