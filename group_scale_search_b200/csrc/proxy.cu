@@ -3,11 +3,11 @@
 // Precision": proxy error tr(E H E^T) / tr(W H W^T)); with H = diag(m):
 //   num = sum_{o,j} m_j (W - What)^2,  den = sum_{o,j} m_j W^2.
 //
-// B200 mapping (HBM-bound): one thread per octet (8 consecutive weights of a
-// group, one 16-byte load of bf16) walking the rows of its slice two at a
-// time; it keeps its 8 imatrix weights in registers, dequantizes in
-// registers (no What round trip through memory), sums the 8 terms in fp32
-// and folds them into fp64 per row.  Each block writes an fp64 partial to
+// B200 mapping (HBM-bound): one thread per two octets (16 consecutive
+// weights of a group, two 16-byte loads of bf16) walking the rows of its
+// slice; its 16 imatrix weights sit in shared memory (read only by it), it
+// dequantizes in registers (no What round trip through memory), sums the
+// terms in fp32 and folds them into fp64 per row.  Each block writes an fp64 partial to
 // the workspace; the last block of a matrix (atomic ticket) adds the
 // partials in block order, so the result is deterministic for a given
 // device.
@@ -18,6 +18,20 @@ namespace tq {
 // Fixed block budget, so the workspace size (one fp64 pair per block) does
 // not depend on the device.
 constexpr int64_t PX_TARGET_BLOCKS = 148 * 8;
+
+// Octets per thread (one or two consecutive octets of one group), rows per
+// iteration (all their loads issued before any is used), and whether the
+// thread's imatrix weights sit in shared memory (fewer registers) or in
+// registers.  Measured on the MoE and dense workloads: two octets, one row,
+// weights in shared memory (60-64 registers, 4 blocks of up to 256 threads
+// per SM) beat two rows in flight per thread at 3 blocks per SM.
+constexpr int PX_NO = 2;
+constexpr int PX_ROWS = 1;
+constexpr bool PX_MSMEM = true;
+
+inline Walk px_geometry(int64_t n_mat, int64_t O, int64_t I) {
+    return walk_geometry(n_mat, O, ((I + 7) / 8 + PX_NO - 1) / PX_NO, PX_TARGET_BLOCKS);
+}
 
 // Adds the 8 terms of one octet in fp32 (two interleaved partial sums of
 // fp32x2 pairs): m (W - What)^2 and m W^2.
@@ -36,15 +50,8 @@ __device__ __forceinline__ void px_terms(const float w[8], const float v[8], con
     sd = __fadd_rn(ad.x, ad.y);
 }
 
-// Octets per thread (one or two consecutive octets of one group).
-constexpr int PX_NO = 2;
-
-inline Walk px_geometry(int64_t n_mat, int64_t O, int64_t I) {
-    return walk_geometry(n_mat, O, ((I + 7) / 8 + PX_NO - 1) / PX_NO, PX_TARGET_BLOCKS);
-}
-
 template <int FMT, typename T, int NO>
-__global__ void __launch_bounds__(256, NO == 1 ? 4 : 3)
+__global__ void __launch_bounds__(256, NO == 1 || PX_MSMEM ? 4 : 3)
 k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, const uint8_t* __restrict__ packed,
         const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
         const float* __restrict__ m, int64_t m_stride, int64_t rps, double* __restrict__ part_out,
@@ -57,6 +64,7 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
     const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
     const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
     const int nwarps = static_cast<int>(blockDim.x >> 5);
+    __shared__ float4 msm[PX_MSMEM ? 2 * NO : 1][PX_MSMEM ? 256 : 1];
     double an = 0.0, ad = 0.0;
     if (u < (C + NO - 1) / NO) {
         const int64_t c = u * NO;
@@ -64,43 +72,53 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
         const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
         const int64_t j = c << 3;
         int n[NO];
-        float mm[NO][8];
+        float mreg[PX_MSMEM ? 1 : NO][8];
 #pragma unroll
         for (int i = 0; i < NO; ++i) {
             n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
             Oct<float> mo;
             mo.load(m + e * m_stride + j + 8 * i, n[i]);
-            mo.get(mm[i]);
+            if constexpr (PX_MSMEM) {
+                msm[2 * i][threadIdx.x] = mo.a;
+                msm[2 * i + 1][threadIdx.x] = mo.b;
+            } else {
+                mo.get(mreg[i]);
+            }
         }
         const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
         const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rps, o1 = min(O, o0 + rps);
         const T* wp = W + e * ms + o0 * ld + j;
         QPtr<FMT> qp(packed, scales, zeros, (e * O + o0) * G + k, G);
-        for (int64_t o = o0; o < o1; o += 2, wp += 2 * ld) {
-            const bool two = o + 1 < o1;
-            Oct<T> ra[NO], rb[NO];
+        for (int64_t o = o0; o < o1; o += PX_ROWS, wp += PX_ROWS * ld) {
+            Oct<T> rw[PX_ROWS][NO];
+            UnitQ<NO> q[PX_ROWS];
 #pragma unroll
-            for (int i = 0; i < NO; ++i) ra[i].load(wp + 8 * i, n[i]);
-            const UnitQ<NO> q0 = load_unit_q<FMT, NO>(qp, oct);
-            qp.next();
-            UnitQ<NO> q1 = q0;
-            if (two) {
+            for (int h = 0; h < PX_ROWS; ++h) {
+                if (o + h < o1) {
 #pragma unroll
-                for (int i = 0; i < NO; ++i) rb[i].load(wp + ld + 8 * i, n[i]);
-                q1 = load_unit_q<FMT, NO>(qp, oct);
+                    for (int i = 0; i < NO; ++i) rw[h][i].load(wp + h * ld + 8 * i, n[i]);
+                    q[h] = load_unit_q<FMT, NO>(qp, oct);
+                }
+                qp.next();
             }
-            qp.next();
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                if (h == 1 && !two) break;
-                const UnitQ<NO>& q = h ? q1 : q0;
+            for (int h = 0; h < PX_ROWS; ++h) {
+                if (o + h >= o1) break;
                 float sn = 0.f, sd = 0.f;
 #pragma unroll
                 for (int i = 0; i < NO; ++i) {
-                    float w[8], v[8], tn, td;
-                    (h ? rb : ra)[i].get(w);
-                    dec_oct<FMT>(OctQ{q.bits[i], q.s, q.z}, g, v);
-                    px_terms(w, v, mm[i], tn, td);
+                    float w[8], v[8], mm[8], tn, td;
+                    rw[h][i].get(w);
+                    dec_oct<FMT>(OctQ{q[h].bits[i], q[h].s, q[h].z}, g, v);
+                    if constexpr (PX_MSMEM) {
+                        const float4 a = msm[2 * i][threadIdx.x], b = msm[2 * i + 1][threadIdx.x];
+                        mm[0] = a.x; mm[1] = a.y; mm[2] = a.z; mm[3] = a.w;
+                        mm[4] = b.x; mm[5] = b.y; mm[6] = b.z; mm[7] = b.w;
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < 8; ++t) mm[t] = mreg[i][t];
+                    }
+                    px_terms(w, v, mm, tn, td);
                     sn = __fadd_rn(sn, tn);
                     sd = __fadd_rn(sd, td);
                 }
