@@ -27,6 +27,8 @@ int64_t resident_blocks(K kernel, int threads) {
 // pays for the integer formats; NVFP4, whose block is two octets, is faster
 // with one).
 template <int FMT> constexpr int pk_no() { return FMT == TQ_NVFP4_G16 ? 1 : 2; }
+// Rows per iteration of tq_pack (all their loads issued before any is used).
+constexpr int PK_ROWS = 2;
 
 // RTN codes of NO consecutive octets (starting at octet `oct` of the group
 // whose record is at rec) into their share of the record.  sc: the group's
@@ -85,44 +87,36 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
     const uint8_t* zp = zeros ? zeros + (r0 * G + k) : nullptr;
     int64_t ecur = cur.e;
     float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + ecur) : 0.f;
-    for (int64_t r = r0; r < r1; r += 2) {
-        const bool two = r + 1 < r1;
-        const T* wa = cur.ptr;
-        const int64_t ea = cur.e;
-        cur.next();
-        const T* wb = cur.ptr;
-        const int64_t eb = cur.e;
-        cur.next();
-        Oct<T> ra[NO], rb[NO];
+    for (int64_t r = r0; r < r1; r += PK_ROWS) {
+        Oct<T> rw[PK_ROWS][NO];
+        float sc[PK_ROWS];
+        int zc[PK_ROWS];
 #pragma unroll
-        for (int i = 0; i < NO; ++i) {
-            ra[i].load(wa + 8 * i, n[i]);
-            if (two) rb[i].load(wb + 8 * i, n[i]);
-        }
-        float sa, sb = 0.f;
-        int za = 0, zb = 0;
-        if constexpr (FMT == TQ_NVFP4_G16) {
-            const unsigned ca = __ldg(bp), cb = two ? __ldg(bp + G) : 0u;
-            if (ea != ecur) { ecur = ea; g = __ldg(gs + ecur); }
-            sa = __fmul_rn(g, e4m3_value(ca));
-            if (two) {
-                if (eb != ecur) { ecur = eb; g = __ldg(gs + ecur); }
-                sb = __fmul_rn(g, e4m3_value(cb));
+        for (int h = 0; h < PK_ROWS; ++h) {
+            sc[h] = 0.f;
+            zc[h] = 0;
+            if (r + h < r1) {
+#pragma unroll
+                for (int i = 0; i < NO; ++i) rw[h][i].load(cur.ptr + 8 * i, n[i]);
+                if constexpr (FMT == TQ_NVFP4_G16) {
+                    if (cur.e != ecur) { ecur = cur.e; g = __ldg(gs + ecur); }
+                    sc[h] = __fmul_rn(g, e4m3_value(__ldg(bp + h * G)));
+                } else {
+                    sc[h] = __ldg(sp + h * G);
+                    if constexpr (FMT == TQ_INT4_G128_ASYM) zc[h] = __ldg(zp + h * G);
+                }
             }
-        } else {
-            sa = __ldg(sp);
-            if (two) sb = __ldg(sp + G);
-            if constexpr (FMT == TQ_INT4_G128_ASYM) {
-                za = __ldg(zp);
-                if (two) zb = __ldg(zp + G);
-            }
+            cur.next();
         }
-        pack_unit<FMT, T, NO>(ra, n, sa, za, rec, oct);
-        if (two) pack_unit<FMT, T, NO>(rb, n, sb, zb, rec + rstride, oct);
-        rec += 2 * rstride;
-        sp += 2 * G;
-        bp += 2 * G;
-        if (FMT == TQ_INT4_G128_ASYM) zp += 2 * G;
+#pragma unroll
+        for (int h = 0; h < PK_ROWS; ++h) {
+            if (r + h >= r1) break;
+            pack_unit<FMT, T, NO>(rw[h], n, sc[h], zc[h], rec + h * rstride, oct);
+        }
+        rec += PK_ROWS * rstride;
+        sp += PK_ROWS * G;
+        bp += PK_ROWS * G;
+        if (FMT == TQ_INT4_G128_ASYM) zp += PK_ROWS * G;
     }
 }
 
