@@ -61,43 +61,52 @@ __device__ __forceinline__ void pack_nvfp4_half(unsigned code, int hl, unsigned 
 // every non-NaN fp32 value); E2M1 rounding is monotone, so when both ends
 // give the same code that is the quotient's.  A -0 is then made +0 with a
 // word-wide test for zero magnitudes.  Otherwise -- a quotient within about
-// 2^-20 of a rounding midpoint -- the codes are redone with IEEE divisions.
-// For NaN weights the codes are unspecified.
+// 2^-20 of a rounding midpoint -- that element's code is redone with an IEEE
+// division.  For NaN weights the codes are unspecified.
+// The NVFP4 code of one weight from the IEEE quotient (the definition,
+// spelled out): magnitude by arithmetic E2M1 rounding, sign when w < 0 and
+// the magnitude is not 0.
+__device__ __forceinline__ uint32_t nvfp4_code_exact(float w, float S) {
+    const float aw = fabsf(w);
+    unsigned mag = 0u;
+    if (S != 0.f && aw != 0.f) mag = static_cast<unsigned>(e2m1_mag_code(e2m1_round(__fdiv_rn(aw, S)))) & 7u;
+    return mag | ((mag != 0u && w < 0.f) ? 8u : 0u);
+}
+
 template <int N>
 __device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[N / 8]) {
     const unsigned se = __float_as_uint(S) >> 23;   // sign bit included: positive S gives se < 256
-    bool exact = !(S > 0.f) || se < 3u || se > 251u;
-    if (!exact) {
-        const float inv = rcp_approx(S);
-        const float lo = __fmul_rn(inv, 0.99999904632568359375f), hi = __fmul_rn(inv, 1.00000095367431640625f);
-        const float2 lo2 = make_float2(lo, lo), hi2 = make_float2(hi, hi);
-        uint32_t diff = 0u;
+    if (!(S > 0.f) || se < 3u || se > 251u) {       // zero, negative, subnormal or extreme block scale
 #pragma unroll
         for (int h = 0; h < N / 8; ++h) {
-            float yl[8], yh[8];
+            m[h] = 0u;
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                const float2 ww = make_float2(w[8 * h + 2 * p], w[8 * h + 2 * p + 1]);
-                const float2 a = __fmul2_rn(ww, lo2), b = __fmul2_rn(ww, hi2);
-                yl[2 * p] = a.x; yl[2 * p + 1] = a.y; yh[2 * p] = b.x; yh[2 * p + 1] = b.y;
-            }
-            const uint32_t x = e2m1x8_from_f32(yl[0], yl[1], yl[2], yl[3], yl[4], yl[5], yl[6], yl[7]);
-            diff |= x ^ e2m1x8_from_f32(yh[0], yh[1], yh[2], yh[3], yh[4], yh[5], yh[6], yh[7]);
-            const uint32_t nz = (x | (x >> 1) | (x >> 2)) & 0x11111111u;   // magnitude != 0, per nibble
-            m[h] = x & (0x77777777u | (nz << 3));
+            for (int i = 0; i < 8; ++i) m[h] |= nvfp4_code_exact(w[8 * h + i], S) << (4 * i);
         }
-        exact = diff != 0u;
+        return;
     }
-    if (exact) {
+    const float inv = rcp_approx(S);
+    const float lo = __fmul_rn(inv, 0.99999904632568359375f), hi = __fmul_rn(inv, 1.00000095367431640625f);
+    const float2 lo2 = make_float2(lo, lo), hi2 = make_float2(hi, hi);
 #pragma unroll
-        for (int h = 0; h < N / 8; ++h) m[h] = 0u;
+    for (int h = 0; h < N / 8; ++h) {
+        float yl[8], yh[8];
 #pragma unroll
-        for (int i = 0; i < N; ++i) {
-            const float aw = fabsf(w[i]);
-            unsigned mag = 0u;
-            if (S != 0.f && aw != 0.f) mag = static_cast<unsigned>(e2m1_mag_code(e2m1_round(__fdiv_rn(aw, S)))) & 7u;
-            m[i >> 3] |= (mag | ((mag != 0u && w[i] < 0.f) ? 8u : 0u)) << (4 * (i & 7));
+        for (int p = 0; p < 4; ++p) {
+            const float2 ww = make_float2(w[8 * h + 2 * p], w[8 * h + 2 * p + 1]);
+            const float2 a = __fmul2_rn(ww, lo2), b = __fmul2_rn(ww, hi2);
+            yl[2 * p] = a.x; yl[2 * p + 1] = a.y; yh[2 * p] = b.x; yh[2 * p + 1] = b.y;
         }
+        uint32_t x = e2m1x8_from_f32(yl[0], yl[1], yl[2], yl[3], yl[4], yl[5], yl[6], yl[7]);
+        const uint32_t d = x ^ e2m1x8_from_f32(yh[0], yh[1], yh[2], yh[3], yh[4], yh[5], yh[6], yh[7]);
+        if (d) {   // rare: only the elements whose bracket ends disagree take an IEEE division
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if ((d >> (4 * i)) & 15u)
+                    x = (x & ~(15u << (4 * i))) | (nvfp4_code_exact(w[8 * h + i], S) << (4 * i));
+        }
+        const uint32_t nz = (x | (x >> 1) | (x >> 2)) & 0x11111111u;   // magnitude != 0, per nibble
+        m[h] = x & (0x77777777u | (nz << 3));
     }
 }
 
