@@ -2,7 +2,8 @@
 runs it (one call per unit over all matrices), checked against the oracle on
 outputs it can compute one by one -- whole sampled rows of every unit
 (search choice and loss, scales, packed records, dequantized weights),
-sampled imatrix columns, and the proxy error of one whole matrix per unit."""
+sampled imatrix columns, and the proxy error of one whole matrix per unit --
+and the stand-alone pack against the fused one on whole tensors."""
 import numpy as np
 import pytest
 import torch
@@ -112,6 +113,11 @@ def _run_workload(name, n_rows=24, seed=0):
         if fmt == tq.NVFP4_G16:   # per-tensor global scales, one expert at a time
             gso = np.concatenate([oracle.nvfp4_global(host32(u.W[e:e + 1])) for e in range(E)])
         rows, idx, codes, gs, gz, grow, match = _check_unit(u, m, res, n_rows, seed + k, gso)
+        # stand-alone RTN + pack with the searched scales: the whole tensor, bit for bit
+        p2 = tq.tq_pack(u.W, fmt, res.scales, res.zeros, res.global_scale)
+        torch.cuda.synchronize()
+        assert torch.equal(p2, res.packed), f"{name}/{u.name}: tq_pack differs from the fused pack"
+        del p2
         # dequantized weights of the sampled rows, bit-exact
         ref = oracle_dequant(fmt, codes, gs.reshape(len(rows), 1, -1),
                              None if gz is None else gz.reshape(len(rows), 1, -1), grow)
