@@ -39,6 +39,45 @@ __device__ __forceinline__ void load_vec<float>(const float* p, float* out) {
     out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
 }
 
+// A 16-byte load as VEC floats.
+template <typename T>
+__device__ __forceinline__ void unpack_vec(uint4 v, float* out);
+template <>
+__device__ __forceinline__ void unpack_vec<uint16_t>(uint4 v, float* out) {
+    const unsigned u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        out[2 * i] = __uint_as_float(u[i] << 16);
+        out[2 * i + 1] = __uint_as_float(u[i] & 0xffff0000u);
+    }
+}
+template <>
+__device__ __forceinline__ void unpack_vec<float>(uint4 v, float* out) {
+    out[0] = __uint_as_float(v.x); out[1] = __uint_as_float(v.y);
+    out[2] = __uint_as_float(v.z); out[3] = __uint_as_float(v.w);
+}
+
+// Token rows in flight per warp in the main loop (loads kept as loaded, 4
+// registers each, so many can be in flight).
+constexpr int IM_U = 16;
+
+// Adds the squares of U token rows (t, t + IM_WARPS, ...) of this lane's
+// VEC columns to acc, all U loads issued before any is used.
+template <typename T, int U>
+__device__ __forceinline__ void im_rows(const T* base, int64_t t, int64_t ld, float* acc) {
+    constexpr int VEC = 16 / sizeof(T);
+    uint4 raw[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) raw[u] = __ldg(reinterpret_cast<const uint4*>(base + (t + u * IM_WARPS) * ld));
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        float x[VEC];
+        unpack_vec<T>(raw[u], x);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(x[i], x[i], acc[i]);
+    }
+}
+
 struct ImGeom {
     int64_t col_tiles, slices, tokens_per_slice;
 };
@@ -91,15 +130,10 @@ k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, in
     int run = 0;
     int64_t t = t0 + wid;
     if (full) {
-        for (; t + 3 * IM_WARPS < t1; t += 4 * IM_WARPS) {
-            float x[4][VEC];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) load_vec<T>(base + (t + u * IM_WARPS) * ld, x[u]);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-#pragma unroll
-                for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(x[u][i], x[u][i], acc[i]);
-            run += 4;
+        // IM_U token rows in flight per warp, then one at a time.
+        for (; t + (IM_U - 1) * IM_WARPS < t1; t += IM_U * IM_WARPS) {
+            im_rows<T, IM_U>(base, t, ld, acc);
+            run += IM_U;
             if (run >= 32) {
 #pragma unroll
                 for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
