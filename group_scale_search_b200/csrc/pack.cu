@@ -27,8 +27,10 @@ int64_t resident_blocks(K kernel, int threads) {
 // pays for the integer formats; NVFP4, whose block is two octets, is faster
 // with one).
 template <int FMT> constexpr int pk_no() { return FMT == TQ_NVFP4_G16 ? 1 : 2; }
-// Rows per iteration of tq_pack (all their loads issued before any is used).
+// Rows per iteration of tq_pack and tq_dequant (all their loads issued
+// before any is used).
 constexpr int PK_ROWS = 2;
+constexpr int DQ_ROWS = 2;
 
 // RTN codes of NO consecutive octets (starting at octet `oct` of the group
 // whose record is at rec) into their share of the record.  sc: the group's
@@ -208,7 +210,8 @@ __device__ __forceinline__ void store8(O* dst, const float v[8], bool vec_ok, in
 
 // Grid: x = octet-column tiles, y = blocks of consecutive rows of the whole
 // batch (the output is dense, so a row's place does not depend on its
-// matrix).  A thread loads two rows' codes and scales before decoding either.
+// matrix).  A thread loads DQ_ROWS rows' codes and scales before decoding
+// any of them.
 template <int FMT, typename O>
 __global__ void __launch_bounds__(256)
 k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t* __restrict__ zeros,
@@ -232,21 +235,20 @@ k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t*
     }
     QPtr<FMT> qp(packed, scales, zeros, r0 * G + k, G);
     O* dst = out + r0 * I + j;
-    for (int64_t r = r0; r < r1; r += 2, dst += 2 * I) {
-        const bool two = r + 1 < r1;
-        const OctQ q0 = load_q<FMT>(qp, oct);
-        qp.next();
-        OctQ q1 = q0;
-        if (two) q1 = load_q<FMT>(qp, oct);
-        qp.next();
-        float v[8];
-        if (FMT == TQ_NVFP4_G16 && r == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
-        dec_oct<FMT>(q0, g, v);
-        store8<O>(dst, v, vec_ok, nvalid);
-        if (two) {
-            if (FMT == TQ_NVFP4_G16 && r + 1 == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
-            dec_oct<FMT>(q1, g, v);
-            store8<O>(dst + I, v, vec_ok, nvalid);
+    for (int64_t r = r0; r < r1; r += DQ_ROWS, dst += DQ_ROWS * I) {
+        OctQ q[DQ_ROWS];
+#pragma unroll
+        for (int h = 0; h < DQ_ROWS; ++h) {
+            if (r + h < r1) q[h] = load_q<FMT>(qp, oct);
+            qp.next();
+        }
+#pragma unroll
+        for (int h = 0; h < DQ_ROWS; ++h) {
+            if (r + h >= r1) break;
+            if (FMT == TQ_NVFP4_G16 && r + h == next_e) { ++e; next_e += Orows; g = __ldg(gs + e); }
+            float v[8];
+            dec_oct<FMT>(q[h], g, v);
+            store8<O>(dst + h * I, v, vec_ok, nvalid);
         }
     }
 }
