@@ -23,13 +23,13 @@ int64_t resident_blocks(K kernel, int threads) {
 // bytes + 1 high-plane byte, int4 = 4 bytes, NVFP4 = half the record.
 
 // Octets per thread of tq_pack (one or two consecutive octets of one group:
-// two halve the per-row loads of scales and the loop work per weight, which
-// pays for the integer formats; NVFP4, whose block is two octets, is faster
-// with one).
-template <int FMT> constexpr int pk_no() { return FMT == TQ_NVFP4_G16 ? 1 : 2; }
+// two halve the per-row loads of scales and the loop work per weight; for
+// NVFP4 two octets are one whole block).
+template <int FMT> __host__ __device__ constexpr int pk_no() { return 2; }
 // Rows per iteration of tq_pack and tq_dequant (all their loads issued
-// before any is used).
-constexpr int PK_ROWS = 2;
+// before any is used).  NVFP4 pack, with the more instructions per weight,
+// prefers one row (more resident warps); the integer formats two.
+template <int FMT> __host__ __device__ constexpr int pk_rows() { return FMT == TQ_NVFP4_G16 ? 1 : 2; }
 constexpr int DQ_ROWS = 2;
 
 // RTN codes of NO consecutive octets (starting at octet `oct` of the group
@@ -89,12 +89,13 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
     const uint8_t* zp = zeros ? zeros + (r0 * G + k) : nullptr;
     int64_t ecur = cur.e;
     float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + ecur) : 0.f;
-    for (int64_t r = r0; r < r1; r += PK_ROWS) {
-        Oct<T> rw[PK_ROWS][NO];
-        float sc[PK_ROWS];
-        int zc[PK_ROWS];
+    constexpr int ROWS = pk_rows<FMT>();
+    for (int64_t r = r0; r < r1; r += ROWS) {
+        Oct<T> rw[ROWS][NO];
+        float sc[ROWS];
+        int zc[ROWS];
 #pragma unroll
-        for (int h = 0; h < PK_ROWS; ++h) {
+        for (int h = 0; h < ROWS; ++h) {
             sc[h] = 0.f;
             zc[h] = 0;
             if (r + h < r1) {
@@ -111,14 +112,14 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
             cur.next();
         }
 #pragma unroll
-        for (int h = 0; h < PK_ROWS; ++h) {
+        for (int h = 0; h < ROWS; ++h) {
             if (r + h >= r1) break;
             pack_unit<FMT, T, NO>(rw[h], n, sc[h], zc[h], rec + h * rstride, oct);
         }
-        rec += PK_ROWS * rstride;
-        sp += PK_ROWS * G;
-        bp += PK_ROWS * G;
-        if (FMT == TQ_INT4_G128_ASYM) zp += PK_ROWS * G;
+        rec += ROWS * rstride;
+        sp += ROWS * G;
+        bp += ROWS * G;
+        if (FMT == TQ_INT4_G128_ASYM) zp += ROWS * G;
     }
 }
 
