@@ -36,17 +36,6 @@ __device__ __forceinline__ void pack_int4_lane(const unsigned q[4], int lane, ui
     reinterpret_cast<uint16_t*>(rec)[lane] = static_cast<uint16_t>(v);
 }
 
-// NVFP4-g16 record: 8 bytes, element 2k in the low nibble of byte k.  The 16
-// lanes of a half-warp hold one block's codes (lane hl = element hl); lanes
-// hl = 0 and 8 store the two 4-byte words.
-__device__ __forceinline__ void pack_nvfp4_half(unsigned code, int hl, unsigned mask, uint8_t* rec) {
-    unsigned v = (code & 15u) << (4u * static_cast<unsigned>(hl & 7));
-    v |= __shfl_xor_sync(mask, v, 1);
-    v |= __shfl_xor_sync(mask, v, 2);
-    v |= __shfl_xor_sync(mask, v, 4);
-    if ((hl & 7) == 0) reinterpret_cast<uint32_t*>(rec)[hl >> 3] = v;
-}
-
 // NVFP4 codes of N (8 or 16) weights under block scale S = fl32(g dec(e)):
 // magnitude = E2M1 round-half-to-even, saturating at 6, of the IEEE fp32
 // quotient |w| / S; sign in bit 3 when w < 0 and the magnitude is not 0

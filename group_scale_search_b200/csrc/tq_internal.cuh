@@ -109,16 +109,6 @@ __device__ __forceinline__ void warp_argmin(float& L, int& idx) {
     }
 }
 
-// Same over aligned groups of `width` lanes (width a power of two <= 32).
-__device__ __forceinline__ void group_argmin(float& L, int& idx, unsigned mask, int width) {
-    if (L != L) L = __int_as_float(0x7f800000);
-    for (int off = width >> 1; off; off >>= 1) {
-        float Lo = __shfl_xor_sync(mask, L, off);
-        int io = __shfl_xor_sync(mask, idx, off);
-        if (Lo < L || (Lo == L && io < idx)) { L = Lo; idx = io; }
-    }
-}
-
 // Butterfly sum: every lane of the group ends with the bit-identical total
 // (each step adds the same pair of operands on both partner lanes).
 __device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width) {
