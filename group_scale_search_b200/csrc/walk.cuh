@@ -282,9 +282,10 @@ __device__ __forceinline__ void dec_oct(const OctQ& q, float g, float v[8]) {
 // integer, half to even, in the low mantissa bits.  Rounding is monotone, so
 // when both ends give the same integer it is the quotient's.  Both ends are
 // finite or both are the same infinity (a quotient beyond +-2^127 clamps
-// either way); when they differ (a quotient within about 2^-20 of a
-// half-integer, or of magnitude 2^22 or more) the octet is redone with IEEE
-// divisions.  For NaN weights the codes are unspecified.
+// either way); where they differ (a quotient within about 2^-20 of a
+// half-integer, or of magnitude 2^22 or more) that element (int4) or the
+// whole octet (int3, measured faster there) is redone with IEEE divisions.
+// For NaN weights the codes are unspecified.
 template <int HI>
 __device__ __forceinline__ uint32_t rtn_int_oct(const float w[8], int n, float s, int z) {
     const unsigned se = (__float_as_uint(s) >> 23) & 255u;
@@ -306,9 +307,26 @@ __device__ __forceinline__ uint32_t rtn_int_oct(const float w[8], int n, float s
             bytes[p] = static_cast<uint32_t>(c0 + 16 * c1);
         }
         nib = __byte_perm(__byte_perm(bytes[0], bytes[1], 0x0040u), __byte_perm(bytes[2], bytes[3], 0x0040u), 0x5410u);
-        exact = diff != 0u;
+        if (HI == 7) {
+            exact = diff != 0u;   // int3: the whole octet with IEEE divisions (measured faster for int3)
+        } else if (diff) {   // int4: elements whose bracket ends disagree take an IEEE division, one at a time
+            const float zf = static_cast<float>(z);
+            uint32_t todo = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                todo |= (__float_as_uint(__fmaf_rn(w[i], lo, MAGIC)) != __float_as_uint(__fmaf_rn(w[i], hi, MAGIC)) ? 1u : 0u) << i;
+            while (todo) {
+                const int i = __ffs(todo) - 1;
+                todo &= todo - 1u;
+                float wi = w[0];
+#pragma unroll
+                for (int k = 1; k < 8; ++k) wi = i == k ? w[k] : wi;
+                const float qf = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(wi, s)), zf), 0.f), static_cast<float>(HI));
+                nib = (nib & ~(15u << (4 * i))) | ((static_cast<uint32_t>(qf) & 15u) << (4 * i));
+            }
+        }
     }
-    if (exact) {   // rare: the whole octet with IEEE divisions (smaller code than per element, measured faster)
+    if (exact) {   // zero, subnormal or extreme scale (or an int3 disagreement): IEEE divisions throughout
         nib = 0u;
         const float zf = static_cast<float>(z);
 #pragma unroll
