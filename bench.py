@@ -314,7 +314,22 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--traffic-table", default=os.path.join(ROOT, "profiles", "traffic.md"),
                     help="ncu DRAM bytes per launch of the dominant kernel, by workload")
+    ap.add_argument("--jsonl", default=None,
+                    help="also append the result line, with a UTC time stamp and the git revision, to this file")
     return ap.parse_args()
+
+
+def append_jsonl(path, line):
+    """Run log: the JSON result line plus when and from which revision."""
+    rec = dict(line)
+    rec["time_utc"] = datetime.datetime.now(datetime.timezone.utc).isoformat(timespec="seconds")
+    try:
+        rec["git"] = subprocess.run(["git", "rev-parse", "--short", "HEAD"], cwd=ROOT, capture_output=True,
+                                    text=True, timeout=10).stdout.strip() or None
+    except Exception:   # noqa: BLE001 -- a copy without git history still logs
+        rec["git"] = None
+    with open(path, "a") as f:
+        f.write(json.dumps(rec) + "\n")
 
 
 def reference_arm(args, world, rank):
@@ -339,6 +354,8 @@ def reference_arm(args, world, rank):
                              "sample": desc},
             "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+    if args.jsonl:
+        append_jsonl(args.jsonl, line)
     return 0
 
 
@@ -456,6 +473,8 @@ def main():
             line["cpu_baseline"]["one_thread"] = {"value": one[0], "unit": "weights/s", "sample": one[1]}
     if rank == 0:
         print(json.dumps(line), flush=True)
+        if args.jsonl:
+            append_jsonl(args.jsonl, line)
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
