@@ -442,6 +442,7 @@ def main():
         hbm_rows[name] = {"ms": t_ms / args.steps, "bytes": nbytes // args.steps, "GB/s": gbs,
                           "frac": gbs / pk["hbm_gbs"]}
     hbm_rows["pack"] = time_pack(tq, step, pk)
+    next_rows = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -462,7 +463,7 @@ def main():
                               f"{n_sets} input sets ({n_sets * nbytes / 2**20:.1f} MiB) fit in L2"),
                        "parallelism": f"weak x{world}: independent workload per GPU"},
             "groups_per_s": value / tq.tq_group_size(tq.FORMATS[fmt_main]),
-            "roofline": roofline, "hbm_rows": hbm_rows, "clocks": clocks, "e2e": e2e,
+            "roofline": roofline, "hbm_rows": hbm_rows, "next_rows": next_rows, "clocks": clocks, "e2e": e2e,
             "gpu_launches": step.kernels_per_step() * args.steps}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, cores, desc, dt = oracle_sample(wl)
@@ -504,6 +505,49 @@ def time_pack(tq, step, pk, reps=12):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
             "note": f"first unit, back-to-back launches over {len(Ws)} rotating weight copies"}
+
+
+def time_gemv(tq, step, pk, B, reps=20):
+    """tq_dequant_gemv (y = What x straight from the records, B token vectors)
+    on the first unit's search output, outside the step, over rotating copies
+    of the records larger than L2 (x is per matrix for a batch of matrices,
+    shared for one): bytes = records + scales (+ zeros) read + x read + y
+    written."""
+    u, r = step.units[0], step.res[0]
+    fmt = tq.FORMATS[u.fmt]
+    E, O, I = u.W.shape
+    dev = r.packed.device
+    q_bytes = (r.packed.numel() + r.scales.numel() * r.scales.element_size()
+               + (0 if r.zeros is None else r.zeros.numel()))
+    n = max(1, min(64, math.ceil(2 * L2_BYTES / q_bytes)))
+    copies = [(r.packed.clone(), r.scales.clone(), None if r.zeros is None else r.zeros.clone()) for _ in range(n)]
+    gen = torch.Generator(device=dev).manual_seed(B)
+    x = torch.randn((E, B, I) if E > 1 else (B, I), generator=gen, device=dev).bfloat16()
+    y = torch.empty((E, B, O), dtype=torch.float32, device=dev)
+    nbytes = q_bytes + x.numel() * 2 + y.numel() * 4
+    def run():
+        for k in range(reps):
+            p, sc, z = copies[k % n]
+            tq.tq_dequant_gemv(p, fmt, sc, z, r.global_scale, E, O, I, x, out=y)
+
+    run()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()     # decode-time launches are replayed from a graph, not issued one by one
+    with torch.cuda.graph(graph):
+        run()
+    graph.replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    graph.replay()
+    b.record()
+    torch.cuda.synchronize()
+    del graph, copies
+    ms = a.elapsed_time(b) / reps
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
+            "weights_per_s": E * O * I / (ms * 1e-3),
+            "note": f"first unit, bf16 x, {reps} launches replayed from a CUDA graph over {n} rotating copies "
+                    f"of the records ({n * q_bytes / 2**20:.0f} MiB)"}
 
 
 def _empty_like_result(tq, r):

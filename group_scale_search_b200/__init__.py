@@ -32,7 +32,7 @@ __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_dequant", "tq_dequant_gemv", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -52,6 +52,7 @@ EXPORTS = [
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
+    "tq_dequant_gemv",
 ]
 
 
@@ -138,6 +139,7 @@ def lib():
             "tq_imatrix_static_capacity": (sz, []),
             "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
             "tq_selftest_e2m1": (i32, [P, P, P]),
+            "tq_dequant_gemv": (i32, [P, i32, P, P, P, i64, i64, i64, P, i32, i64, i64, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -353,6 +355,33 @@ def tq_dequant(packed: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Opti
     odt = _BF16 if out.dtype == torch.bfloat16 else _F32
     _check(lib().tq_dequant(_ptr(packed), fmt, _ptr(scales), _ptr(zeros), _ptr(global_scale), n_mat, O, I,
                             _ptr(out), odt, _stream(stream)), "tq_dequant")
+    return out
+
+
+def tq_dequant_gemv(packed: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Optional[torch.Tensor],
+                    global_scale: Optional[torch.Tensor], n_mat: int, O: int, I: int, x: torch.Tensor,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """y[e, b, o] = sum_j What[e, o, j] x[e, b, j] (fp32) for x of shape [B, I] (shared by every matrix) or
+    [n_mat, B, I], B <= 8, What dequantized as tq_dequant defines it."""
+    _cuda(packed, "packed")
+    _cuda(x, "x")
+    if x.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("x must be float32 or bfloat16")
+    if not x.is_contiguous():
+        raise ValueError("x must be contiguous")
+    if x.dim() == 2:
+        B, xms = x.shape[0], 0
+    elif x.dim() == 3 and x.shape[0] == n_mat:
+        B, xms = x.shape[1], x.shape[1] * x.shape[2]
+    else:
+        raise ValueError("x must be [B, I] or [n_mat, B, I]")
+    if x.shape[-1] != I:
+        raise ValueError("x's last dimension must be I")
+    if out is None:
+        out = torch.empty((n_mat, B, O), dtype=torch.float32, device=packed.device)
+    _check(lib().tq_dequant_gemv(_ptr(packed), fmt, _ptr(scales), _ptr(zeros), _ptr(global_scale), n_mat, O, I,
+                                 _ptr(x), _BF16 if x.dtype == torch.bfloat16 else _F32, B, xms, _ptr(out),
+                                 _stream(stream)), "tq_dequant_gemv")
     return out
 
 

@@ -72,7 +72,7 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
         const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
         const int64_t j = c << 3;
         int n[NO];
-        float mreg[PX_MSMEM ? 1 : NO][8];
+        [[maybe_unused]] float mreg[PX_MSMEM ? 1 : NO][8];
 #pragma unroll
         for (int i = 0; i < NO; ++i) {
             n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));

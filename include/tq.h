@@ -233,6 +233,31 @@ tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scales, con
                      const float* global_scale, int64_t n_mat, int64_t O, int64_t I, void* out,
                      int32_t out_dtype, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ dequant-GEMV
+ * The decode-time consumer of the packed formats ([INT3] Design: Kernel
+ * bullet, exact-fp32 product with the scale applied per group; GPU bullet;
+ * the step after packing): for b < B,
+ *   y[e][b][o] = sum_j What[e][o][j] * x[e][b][j],
+ * What the dequantized weights as tq_dequant defines them.  Computed as
+ * sum over groups (NVFP4: blocks) of s * sum_j d_j x_j in fp32 (d = v,
+ * q - z or dec(c); s = the group scale or fl32(g dec(e))), in an order fixed
+ * by the shape alone: per lane over its 32-weight quads, a butterfly over
+ * 32 lanes, then (rows split over up to 8 warps) the warps' sums in order.
+ * Deterministic; |y - sum What x| <= (4 ceil(I/1024) + 30) u sum |What x|
+ * (u = 2^-24), plus underflow.
+ * packed / scales / zeros / global_scale: as tq_dequant; packed 16-byte
+ * aligned.  x: x_dtype (TQ_F32 / TQ_BF16) dense [n_mat][B][I] with
+ * x_mat_stride elements between matrices (0: one x shared by all
+ * matrices), 16-byte aligned.  y: fp32 dense [n_mat][B][O], written once
+ * per element.  B in [1, 8] (larger batches are a GEMM, not this call).
+ * Errors: TQ_ERR_INVALID for null pointers, empty shapes, B outside [1, 8],
+ * 0 < x_mat_stride < B*I, misaligned packed/x, int4 without zeros or NVFP4
+ * without global_scale; TQ_ERR_UNSUPPORTED for an unknown fmt or x_dtype;
+ * nothing is enqueued then. */
+tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void* scales, const uint8_t* zeros,
+                          const float* global_scale, int64_t n_mat, int64_t O, int64_t I, const void* x,
+                          int32_t x_dtype, int64_t B, int64_t x_mat_stride, float* y, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ proxy error
  * Per matrix e ([TT] "Risks to measure: Precision", H = diag(m)):
  *   num[e] = sum_{o,j} m_j (W - What)^2 = tr(E H E^T),

@@ -93,6 +93,21 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     need = L.tq_imatrix_workspace_bytes(ctypes.byref(x))
     assert need > 0
     assert L.tq_imatrix(ctypes.byref(x), fake, 512, ctypes.c_float(1.0), 0, fake, need - 8, None) == 1
+    # dequant-GEMV: (packed, fmt, scales, zeros, gs, n_mat, O, I, x, x_dtype, B, x_mat_stride, y, stream)
+    gemv = L.tq_dequant_gemv
+    assert gemv(None, tq.INT3_G64_SYM, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
+    assert gemv(fake, 99, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 2
+    assert gemv(fake, tq.INT3_G64_SYM, fake, None, None, 1, 8, 64, fake, 7, 1, 0, fake, None) == 2
+    for B in (0, 9):
+        assert gemv(fake, tq.INT3_G64_SYM, fake, None, None, 1, 8, 64, fake, 0, B, 0, fake, None) == 1
+        assert b"B must" in L.tq_last_error_string()
+    assert gemv(fake, tq.INT3_G64_SYM, fake, None, None, 2, 8, 64, fake, 0, 2, 100, fake, None) == 1
+    assert gemv(fake, tq.INT3_G64_SYM, fake, None, None, 1, 0, 64, fake, 0, 1, 0, fake, None) == 1
+    assert gemv(ctypes.c_void_p(0x1008), tq.INT3_G64_SYM, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake,
+                None) == 1
+    assert b"aligned" in L.tq_last_error_string()
+    assert gemv(fake, tq.INT4_G128_ASYM, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
+    assert gemv(fake, tq.NVFP4_G16, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
 
 
 def test_binding_refuses_cpu_tensors(tq):

@@ -342,3 +342,116 @@ def test_e2m1_conversion_selftest():
     n, first = tq.tq_selftest_e2m1()
     assert n == 0, f"{n} mismatches, first failing pattern {first:#010x}"
     assert first == 0xFFFFFFFF
+
+
+# ------------------------------------------------------------------ dequant-GEMV
+
+def _gemv_case(fmt, E, O, I, seed):
+    """Seeded weights and per-group scales, quantized and packed by the oracle
+    (its RTN and packing), and the oracle's dequantized What."""
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_t(4, size=(E, O, I)) * 0.02).astype(np.float32)
+    g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.NVFP4_G16: 16}[fmt]
+    G = (I + g - 1) // g
+    zeros = gsc = None
+    if fmt == tq.NVFP4_G16:
+        sc = rng.integers(1, 127, size=(E, O, G)).astype(np.uint8)
+        gsc = (np.abs(W).reshape(E, -1).max(axis=1) / 2688.0).astype(np.float32)
+    else:
+        sc = (0.004 + 0.01 * rng.random((E, O, G))).astype(np.float32)
+        if fmt == tq.INT3_G64_SYM:
+            sc *= np.where(rng.random((E, O, G)) < 0.3, -1, 1).astype(np.float32)
+        else:
+            zeros = rng.integers(0, 16, size=(E, O, G)).astype(np.uint8)
+    packed, codes = oracle_packed(fmt, W, sc, zeros, gsc)
+    What = oracle_dequant(fmt, codes.reshape(E, O, I), sc, zeros, gsc)
+    dev = lambda a: None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)  # noqa: E731
+    return dict(packed=dev(packed), scales=dev(sc), zeros=dev(zeros), gs=dev(gsc), What=What)
+
+
+def _gemv_check(fmt, case, E, O, I, x, label):
+    """x: [B, I] or [E, B, I] on the device; checks y against What x in fp64
+    within the fp32 bound of the per-group accumulation."""
+    y = tq.tq_dequant_gemv(case["packed"], fmt, case["scales"], case["zeros"], case["gs"], E, O, I, x)
+    torch.cuda.synchronize()
+    xh = x.float().cpu().numpy().astype(np.float64)
+    if xh.ndim == 2:
+        xh = np.broadcast_to(xh, (E,) + xh.shape)
+    Wd = case["What"].astype(np.float64)
+    ref = np.einsum("eoi,ebi->ebo", Wd, xh)
+    mag = np.einsum("eoi,ebi->ebo", np.abs(Wd), np.abs(xh))
+    depth = 4 * -(-I // 1024) + 30
+    tol = 1.01 * depth * 2.0 ** -24 * mag + 2.0 ** -126 * I
+    got = y.cpu().numpy().astype(np.float64)
+    assert got.shape == ref.shape, label
+    bad = np.abs(got - ref) > tol
+    assert not bad.any(), (label, int(bad.sum()), np.argwhere(bad)[:3], got[bad][:3], ref[bad][:3])
+    return got
+
+
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("B", [1, 3, 8])
+@pytest.mark.parametrize("I", [100, 1802, 4096, 7000])
+def test_dequant_gemv_matches_oracle(fmt, B, I):
+    """y = What x against the oracle's What in fp64: bf16 and fp32 x, one x
+    shared by all matrices and one per matrix, ragged I, row counts that leave
+    a partial chunk, column tiles of x (7000 columns: three tiles at B = 8)."""
+    E, O = 3, 37
+    case = _gemv_case(fmt, E, O, I, seed=I * 10 + B)
+    rng = np.random.default_rng(B + I)
+    xs = torch.from_numpy(rng.standard_normal((B, I)).astype(np.float32)).to(DEV)
+    xm = torch.from_numpy(rng.standard_normal((E, B, I)).astype(np.float32)).to(DEV)
+    dt = torch.bfloat16 if (B + I) % 2 else torch.float32
+    _gemv_check(fmt, case, E, O, I, xs.to(dt), "shared")
+    _gemv_check(fmt, case, E, O, I, xm.to(dt), "per-matrix")
+    _gemv_check(fmt, case, E, O, I, xm.to(torch.float32 if dt == torch.bfloat16 else torch.bfloat16), "other dtype")
+
+
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.NVFP4_G16])
+def test_dequant_gemv_shapes(fmt):
+    """Many row chunks per block (x staged once), many small matrices with
+    their own x (staged per matrix), a single weight, rows split over 2, 4
+    and 8 warps (few rows, long rows), x in many column tiles, NVFP4 rows with
+    an odd block count (8-byte aligned rows) and scales at an odd address."""
+    for (E, O, I, B, per) in [(1, 20000, 64, 1, False), (64, 16, 256, 2, True), (1, 1, 1, 1, False),
+                              (2, 5, 48, 4, True), (2, 9, 16, 8, False), (2, 10, 3000, 3, True),
+                              (1, 7, 9000, 2, False), (1, 3, 20000, 8, False), (1, 2, 30000, 1, True)]:
+        case = _gemv_case(fmt, E, O, I, seed=E * 7 + O + I)
+        rng = np.random.default_rng(O + I)
+        shape = (E, B, I) if per else (B, I)
+        x = torch.from_numpy(rng.standard_normal(shape).astype(np.float32)).to(DEV).bfloat16()
+        _gemv_check(fmt, case, E, O, I, x, f"E={E} O={O} I={I} B={B}")
+    if fmt == tq.NVFP4_G16:
+        E, O, I = 2, 11, 4096
+        case = _gemv_case(fmt, E, O, I, seed=3)
+        odd = torch.empty(case["scales"].numel() + 1, dtype=torch.uint8, device=DEV)[1:]
+        odd.copy_(case["scales"].reshape(-1))
+        case["scales"] = odd
+        x = torch.randn(2, I, device=DEV)
+        _gemv_check(fmt, case, E, O, I, x, "odd scales address")
+
+
+def test_dequant_gemv_deterministic_and_exact_cases():
+    """Bitwise-repeatable results; a matrix of zero scales gives exact zeros;
+    one nonzero weight per row gives that weight times x exactly."""
+    E, O, I = 2, 24, 1000
+    case = _gemv_case(tq.INT4_G128_ASYM, E, O, I, seed=11)
+    x = torch.randn(5, I, device=DEV)
+    y1 = tq.tq_dequant_gemv(case["packed"], tq.INT4_G128_ASYM, case["scales"], case["zeros"], None, E, O, I, x)
+    y2 = tq.tq_dequant_gemv(case["packed"], tq.INT4_G128_ASYM, case["scales"], case["zeros"], None, E, O, I, x)
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y2)
+    # int3 with every code 0 except v = -4 at column 7 of each row, scale 0.5 (0 for row 1)
+    G = (I + 63) // 64
+    v = np.zeros((O, I), np.int8)
+    v[:, 7] = -4
+    sc = np.full((O, G), 0.5, np.float32)
+    sc[1] = 0.0
+    packed = torch.from_numpy(oracle.pack_int3(v)).to(DEV)
+    xh = np.random.default_rng(2).standard_normal((3, I)).astype(np.float32)
+    y = tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.from_numpy(sc).to(DEV), None, None, 1, O, I,
+                           torch.from_numpy(xh).to(DEV))
+    torch.cuda.synchronize()
+    want = np.float32(-2.0) * xh[:, 7][:, None] * np.ones((1, O), np.float32)
+    want[:, 1] = 0.0
+    assert np.array_equal(y.cpu().numpy()[0], want)
