@@ -23,10 +23,21 @@
 // 8 + 4 bytes), so consecutive lanes read consecutive bytes of a row.  The R
 // rows share every x load.  Integers become floats as 2^23 + k (byte_perm)
 // and (2^23 + k) - (2^23 + z) is exact, paired in fp32x2 adds; products go
-// into fp32x2 FMAs.  Lane sums are added by a fixed butterfly, so the result
-// does not depend on scheduling.  Blocks take contiguous runs of row chunks,
-// so x is staged again only when the matrix (per-matrix x) or the column tile
-// (I beyond one tile) changes.
+// into fp32x2 FMAs.  int3 codes are decoded by position across the quad's 4
+// octets (the low-plane bytes gathered with one byte_perm, the high-plane bit
+// shifted into place), so x is staged in that order for int3.  E2M1 and E4M3
+// codes go through the hardware f16x2 conversions.  Lane sums are added by a
+// fixed butterfly, so the result does not depend on scheduling.  Blocks take
+// contiguous runs of row chunks, so x is staged again only when the matrix
+// (per-matrix x) or the column tile (I beyond one tile) changes; a chunk's
+// first code loads are issued before x is staged.  Rows of few quads are
+// split over 2, 4 or 8 warps so that small matrices still fill the GPU.
+//
+// What bounds it (ncu, one B200): the decode instructions.  At B = 1 the
+// kernel issues about 4.5 (NVFP4) to 5 (int3) instructions per weight, and
+// the ALU pipe, not DRAM, is the busiest unit; small matrices (a few MB of
+// records) are bound by latency (x staging, one HBM round trip, the launch).
+
 #include <atomic>
 #include <mutex>
 
@@ -36,9 +47,11 @@ namespace tq {
 
 constexpr int GV_WARPS = 8;
 constexpr int GV_THREADS = GV_WARPS * 32;
-constexpr int64_t GV_XS_BYTES = 96 * 1024;   // x tile budget: two blocks per SM (their register share)
+constexpr int64_t GV_XS_BYTES = 72 * 1024;   // x tile budget: three blocks per SM
 
 template <int B> __host__ __device__ constexpr int gv_rows() { return B <= 2 ? 4 : 2; }   // rows per warp
+template <int B> __host__ __device__ constexpr int gv_min_blocks() { return B == 1 ? 3 : 2; }   // per SM
+constexpr bool GV_DB = false;   // double-buffered code loads (measured slower)
 
 // Columns of x per staged tile: a multiple of 1024 (32 lanes x 32 weights),
 // no more than the row needs.
@@ -49,34 +62,51 @@ inline int64_t gv_tile(int64_t B, int64_t I) {
     return 1024 * (need < k ? need : k);
 }
 
-// x[b][j0 .. j0 + TI) of matrix e as fp32 into the swizzled tile (zeros past I).
+// x[b][j0 .. j0 + TI) of matrix e as fp32 into the swizzled tile (zeros past
+// I).  Slot i (0..7) of a lane's quad holds 4 of the quad's 32 columns:
+// 4i .. 4i + 3 (int4, NVFP4), or i, 8 + i, 16 + i, 24 + i (int3: the
+// columns at position i of the quad's 4 octets, in the order its decoding
+// produces them).
+template <bool OCT_MAJOR>
 __device__ __forceinline__ void gv_stage(float4* xs, const void* x, bool x_bf16, int64_t xoff, int64_t I,
                                          int64_t j0, int64_t TI, int B, bool vec) {
     const int64_t slots = TI >> 2;   // float4 slots per vector, a multiple of GV_THREADS
     for (int b = 0; b < B; ++b) {
         for (int64_t s = threadIdx.x; s < slots; s += GV_THREADS) {
             const int64_t l = s & 31, ti = s >> 5;
-            const int64_t j = j0 + (((ti >> 3) * 32 + l) * 32) + 4 * (ti & 7);
-            const int64_t base = xoff + b * I + j;
+            const int64_t jq = j0 + ((ti >> 3) * 32 + l) * 32;   // the quad's first column
+            const int i = static_cast<int>(ti & 7);
+            const int64_t base = xoff + b * I;
             float f[4];
-            if (x_bf16) {
-                const uint16_t* p = static_cast<const uint16_t*>(x) + base;
-                if (vec && j + 3 < I) {
-                    const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-                    f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
-                    f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
-                } else {
+            if (OCT_MAJOR) {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) f[c] = j + c < I ? bf16_bits_to_f32(__ldg(p + c)) : 0.f;
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t j = jq + 8 * c + i;
+                    f[c] = j < I ? (x_bf16 ? bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(x) + base + j))
+                                           : __ldg(static_cast<const float*>(x) + base + j))
+                                 : 0.f;
                 }
             } else {
-                const float* p = static_cast<const float*>(x) + base;
-                if (vec && j + 3 < I) {
-                    const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-                    f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-                } else {
+                const int64_t j = jq + 4 * i;
+                if (x_bf16) {
+                    const uint16_t* p = static_cast<const uint16_t*>(x) + base + j;
+                    if (vec && j + 3 < I) {
+                        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
+                        f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
+                        f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
+                    } else {
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) f[c] = j + c < I ? __ldg(p + c) : 0.f;
+                        for (int c = 0; c < 4; ++c) f[c] = j + c < I ? bf16_bits_to_f32(__ldg(p + c)) : 0.f;
+                    }
+                } else {
+                    const float* p = static_cast<const float*>(x) + base + j;
+                    if (vec && j + 3 < I) {
+                        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
+                        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+                    } else {
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) f[c] = j + c < I ? __ldg(p + c) : 0.f;
+                    }
                 }
             }
             xs[b * slots + s] = make_float4(f[0], f[1], f[2], f[3]);
@@ -84,56 +114,107 @@ __device__ __forceinline__ void gv_stage(float4* xs, const void* x, bool x_bf16,
     }
 }
 
-// One quad (32 weights) of one row: codes and per-group factors.
-struct Quad {
-    uint32_t w[4];   // int: 8 nibbles per word (word k = weights 8k..8k+7); NVFP4: 2 E2M1 codes per byte
-    float s0, s1;    // int: group scale (s1 unused); NVFP4: the two blocks' fl32(g dec(e))
-    int z;           // int: zero-point (int3: 4)
-};
-
-// A16: NVFP4 rows start on 16-byte boundaries (an even number of blocks per row).
-template <int FMT, bool A16>
-__device__ __forceinline__ Quad gv_load(const uint8_t* rec_row, const void* sc_row, const uint8_t* zp_row, float g,
-                                        int64_t q, int64_t G) {
-    Quad u;
-    if constexpr (FMT == TQ_INT4_G128_ASYM) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(rec_row) + q);
-        u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
-        u.s0 = __ldg(static_cast<const float*>(sc_row) + (q >> 2));
-        u.z = __ldg(zp_row + (q >> 2));
-    } else if constexpr (FMT == TQ_INT3_G64_SYM) {
-        const uint8_t* rec = rec_row + (q >> 1) * 24;
-        const int h = static_cast<int>(q & 1);
-        const uint2 lo = __ldg(reinterpret_cast<const uint2*>(rec + 8 * h));
-        const uint32_t hi = __ldg(reinterpret_cast<const uint32_t*>(rec + 16 + 4 * h));
-        u.w[0] = int3_nibbles(lo.x & 0xffffu, hi & 0xffu);
-        u.w[1] = int3_nibbles(lo.x >> 16, (hi >> 8) & 0xffu);
-        u.w[2] = int3_nibbles(lo.y & 0xffffu, (hi >> 16) & 0xffu);
-        u.w[3] = int3_nibbles(lo.y >> 16, hi >> 24);
-        u.s0 = __ldg(static_cast<const float*>(sc_row) + (q >> 1));
-        u.z = 4;
-    } else {
-        const uint8_t* sc = static_cast<const uint8_t*>(sc_row) + 2 * q;
-        if constexpr (A16) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(rec_row) + q);
-            u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
-            const unsigned e2 = __ldg(reinterpret_cast<const uint16_t*>(sc));
-            u.s0 = __fmul_rn(g, e4m3_value(e2 & 0xffu));
-            u.s1 = __fmul_rn(g, e4m3_value(e2 >> 8));
-        } else {   // the second block may lie past the row (odd block count): it then counts as zero
-            const uint2 a = __ldg(reinterpret_cast<const uint2*>(rec_row) + 2 * q);
-            const bool two = 2 * q + 1 < G;
-            const uint2 b = two ? __ldg(reinterpret_cast<const uint2*>(rec_row) + 2 * q + 1) : make_uint2(0u, 0u);
-            u.w[0] = a.x; u.w[1] = a.y; u.w[2] = b.x; u.w[3] = b.y;
-            u.s0 = __fmul_rn(g, e4m3_value(__ldg(sc)));
-            u.s1 = two ? __fmul_rn(g, e4m3_value(__ldg(sc + 1))) : 0.f;
-        }
-        u.z = 0;
-    }
-    return u;
+// The two E4M3 values of a 16-bit pair of codes (low byte first) as fp32,
+// exactly (every E4M3 value is an f16 value).
+__device__ __forceinline__ float2 e4m3x2_to_f32(unsigned two_codes) {
+    unsigned h2;
+    asm("{ .reg .b16 t; cvt.u16.u32 t, %1; cvt.rn.f16x2.e4m3x2 %0, t; }" : "=r"(h2) : "r"(two_codes));
+    __half2_raw raw;
+    raw.x = static_cast<unsigned short>(h2 & 0xffffu);
+    raw.y = static_cast<unsigned short>(h2 >> 16);
+    return __half22float2(__half2(raw));
 }
 
-// d values of word k of an integer quad, as 4 pairs (elements 2i, 2i+1):
+// One quad (32 weights) of one row: codes and per-group factors.
+struct Quad {
+    uint32_t w[4];   // int4: 8 nibbles per word (word k = weights 8k..8k+7); NVFP4: 2 E2M1 codes per byte;
+                     // int3: low-plane bytes gathered by position (w0: positions 0-3, w1: 4-7; byte o =
+                     // octet o), w2 = high plane (byte o = octet o)
+    float s0, s1;    // int: group scale (s1 unused); NVFP4: the two blocks' fl32(g dec(e))
+    int z;           // int4: zero-point
+};
+
+// Where the current quads of a warp's R rows sit in the records, scales and
+// zero-points: one base pointer per array for the first row and 32-bit row
+// offsets (the rows are consecutive; rows past the matrix repeat its last
+// row), moved on by dq quads (a multiple of 32) without multiplications.
+// A16: NVFP4 rows start on 16-byte boundaries (an even number of blocks per row).
+template <int FMT, bool A16, int R>
+struct GvRows {
+    const uint8_t* c;    // codes of the first row's quad (int3: its low-plane half)
+    const uint8_t* s;    // scales of the first row's group (bytes)
+    const uint8_t* z;    // int4: zero-points
+    int cof[R], gof[R];  // row offsets: record bytes, groups
+    int ho;              // int3: high-plane half minus low-plane half
+    int q, G;            // NVFP4 rows with an odd block count: the last quad may hold one block
+    __device__ __forceinline__ void init(const uint8_t* packed, const void* scales, const uint8_t* zeros, int G_,
+                                         int64_t row0, const int (&rr)[R], int q_) {
+        constexpr int rec = FmtTraits<FMT>::rec, group = FmtTraits<FMT>::group;
+        G = G_;
+        q = q_;
+        const int64_t g0 = row0 * G;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            cof[r] = rr[r] * G * rec;
+            gof[r] = rr[r] * G;
+        }
+        const int qg = q * 32 / group;   // the quad's group (NVFP4: its first block)
+        if constexpr (FMT == TQ_INT3_G64_SYM) {
+            const int h = q & 1;
+            c = packed + g0 * rec + static_cast<int64_t>(qg) * rec + 8 * h;
+            ho = 16 - 4 * h;
+        } else {
+            c = packed + g0 * rec + static_cast<int64_t>(q) * 16;
+        }
+        s = static_cast<const uint8_t*>(scales) + (g0 + qg) * (FMT == TQ_NVFP4_G16 ? 1 : 4);
+        z = FMT == TQ_INT4_G128_ASYM ? zeros + g0 + qg : nullptr;
+    }
+    __device__ __forceinline__ Quad load(int r, float g) const {
+        Quad u;
+        const uint8_t* cr = c + cof[r];
+        if constexpr (FMT == TQ_INT4_G128_ASYM) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(cr));
+            u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
+            u.s0 = __ldg(reinterpret_cast<const float*>(s) + gof[r]);
+            u.z = __ldg(z + gof[r]);
+        } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+            const uint2 lo = __ldg(reinterpret_cast<const uint2*>(cr));
+            u.w[0] = __byte_perm(lo.x, lo.y, 0x6420u);   // byte o: octet o's low-plane byte for positions 0-3
+            u.w[1] = __byte_perm(lo.x, lo.y, 0x7531u);   // ... for positions 4-7
+            u.w[2] = __ldg(reinterpret_cast<const uint32_t*>(cr + ho));
+            u.s0 = __ldg(reinterpret_cast<const float*>(s) + gof[r]);
+        } else {
+            unsigned e2;   // the two blocks' E4M3 codes, first in the low byte
+            const uint8_t* sr = s + gof[r];
+            if constexpr (A16) {
+                const uint4 v = __ldg(reinterpret_cast<const uint4*>(cr));
+                u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
+                e2 = __ldg(reinterpret_cast<const uint16_t*>(sr));
+            } else {   // the second block may lie past the row: it then counts as zero (code 0)
+                const uint2 a = __ldg(reinterpret_cast<const uint2*>(cr));
+                const bool two = 2 * q + 1 < G;
+                const uint2 b = two ? __ldg(reinterpret_cast<const uint2*>(cr) + 1) : make_uint2(0u, 0u);
+                u.w[0] = a.x; u.w[1] = a.y; u.w[2] = b.x; u.w[3] = b.y;
+                e2 = __ldg(sr) | (two ? static_cast<unsigned>(__ldg(sr + 1)) << 8 : 0u);
+            }
+            const float2 d = e4m3x2_to_f32(e2 & 0x7f7fu);   // magnitudes, as tq_dequant reads the codes
+            u.s0 = __fmul_rn(g, d.x);
+            u.s1 = __fmul_rn(g, d.y);
+        }
+        return u;
+    }
+    __device__ __forceinline__ void next(int dq) {
+        if constexpr (FMT == TQ_INT4_G128_ASYM) {
+            c += 16 * dq; s += dq; z += dq >> 2;
+        } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+            c += 12 * dq; s += 2 * dq;
+        } else {
+            c += 16 * dq; s += 2 * dq; q += dq;
+        }
+    }
+};
+
+// d values of word k of an int4 quad, as 4 pairs (elements 2i, 2i+1):
 // (2^23 + code) - (2^23 + z), exact.
 __device__ __forceinline__ void gv_int_pairs(uint32_t bits, float2 noff, float2 d[4]) {
     const uint32_t ev = bits & 0x0f0f0f0fu, od = (bits >> 4) & 0x0f0f0f0fu;
@@ -142,6 +223,41 @@ __device__ __forceinline__ void gv_int_pairs(uint32_t bits, float2 noff, float2 
         const unsigned sel = 0x5640u | static_cast<unsigned>(i);   // bytes: (byte i, 0, 0, 0x4b)
         d[i] = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(ev, 0x4b00u, sel)),
                                       __uint_as_float(__byte_perm(od, 0x4b00u, sel))), noff);
+    }
+}
+
+// v = u - 4 of position a (0..7) of the quad's 4 octets (octets 0, 1 in d0,
+// octets 2, 3 in d1): u = low-plane bits 2(a & 3).. of the gathered byte,
+// plus 4 x the high-plane bit a of the octet's byte; (2^23 + u) - (2^23 + 4).
+__device__ __forceinline__ void gv_int3_pos(const Quad& q, int a, float2& d0, float2& d1) {
+    const uint32_t lo = (q.w[a >> 2] >> (2 * (a & 3))) & 0x03030303u;
+    const uint32_t hs = a >= 2 ? (q.w[2] >> (a - 2)) : (q.w[2] << (2 - a));
+    const uint32_t u = (hs & 0x04040404u) | lo;
+    const float o = f23(4u);
+    const float2 noff = make_float2(-o, -o);
+    d0 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4b00u, 0x5640u)),
+                                __uint_as_float(__byte_perm(u, 0x4b00u, 0x5641u))), noff);
+    d1 = __fadd2_rn(make_float2(__uint_as_float(__byte_perm(u, 0x4b00u, 0x5642u)),
+                                __uint_as_float(__byte_perm(u, 0x4b00u, 0x5643u))), noff);
+}
+
+// The 8 E2M1 values of a word (low nibble of byte 0 first) as fp32 pairs.
+__device__ __forceinline__ void gv_e2m1x8(uint32_t w, float2 d[4]) {
+    uint32_t h[4];
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(w));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        __half2_raw raw;
+        raw.x = static_cast<unsigned short>(h[i] & 0xffffu);
+        raw.y = static_cast<unsigned short>(h[i] >> 16);
+        d[i] = __half22float2(__half2(raw));
     }
 }
 
@@ -164,10 +280,12 @@ __device__ __forceinline__ void gv_quad(const Quad (&u)[R], const float4* xq, in
         }
 #pragma unroll
         for (int r = 0; r < R; ++r) {
-            float2 d[4];                 // pairs (8k + 2i, 8k + 2i + 1)
+            float2 d[4];                 // d[0], d[1] pair with slot 2k; d[2], d[3] with slot 2k + 1
             if constexpr (FMT == TQ_NVFP4_G16) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) d[i] = e2m1x2_to_f32((u[r].w[k] >> (8 * i)) & 0xffu);
+                gv_e2m1x8(u[r].w[k], d);
+            } else if constexpr (FMT == TQ_INT3_G64_SYM) {
+                gv_int3_pos(u[r], 2 * k, d[0], d[1]);
+                gv_int3_pos(u[r], 2 * k + 1, d[2], d[3]);
             } else {
                 const float o = f23(static_cast<unsigned>(u[r].z) & 0xffu);
                 gv_int_pairs(u[r].w[k], make_float2(-o, -o), d);
@@ -209,7 +327,7 @@ __device__ __forceinline__ void gv_quad(const Quad (&u)[R], const float4* xq, in
 // per matrix.  Each lane's next quads are loaded before the current ones
 // are used.
 template <int FMT, int B, bool A16>
-__global__ void __launch_bounds__(GV_THREADS)
+__global__ void __launch_bounds__(GV_THREADS, gv_min_blocks<B>())
 k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scales,
                const uint8_t* __restrict__ zeros, const float* __restrict__ gs, int64_t n_mat, int64_t O,
                int64_t I, const void* __restrict__ x, int x_bf16, int64_t x_ms, int64_t TI, int64_t cpm, int wl,
@@ -225,8 +343,7 @@ k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scal
     const int64_t nq = (I + 31) >> 5;                 // quads per row
     const int64_t nT = (I + TI - 1) / TI;             // column tiles
     const int64_t slots = TI >> 2;
-    const int64_t rec_bytes = G * F::rec;             // record bytes per row
-    const int64_t qstep = static_cast<int64_t>(32) << wl;
+    const int qstep = 32 << wl;
     const bool vec = (I % 4) == 0 && (x_ms % 4) == 0;
     const int64_t nchunks = n_mat * cpm;
     const int64_t c0 = nchunks * blockIdx.x / gridDim.x, c1 = nchunks * (blockIdx.x + 1) / gridDim.x;
@@ -235,52 +352,55 @@ k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scal
         const int64_t e = c / cpm;
         const int64_t ob = (c - e * cpm) * rows_per_chunk + rgi * R;
         const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
-        const int64_t row0 = e * O;   // this matrix's first row
-        const uint8_t* rec_m = packed + row0 * rec_bytes;
-        const void* sc_m = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(scales) + row0 * G)
-                                               : static_cast<const void*>(static_cast<const float*>(scales) + row0 * G);
-        const uint8_t* zp_m = FMT == TQ_INT4_G128_ASYM ? zeros + row0 * G : nullptr;
-        int rr[R];   // rows within the matrix; rows past O repeat the last one and are not stored
+        const int64_t ofirst = min(ob, O - 1);
+        int rr[R];   // rows relative to the first; rows past O repeat the last one and are not stored
 #pragma unroll
-        for (int r = 0; r < R; ++r) rr[r] = static_cast<int>(min(ob + r, O - 1));
-        auto load = [&](Quad (&u)[R], int64_t q) {
-#pragma unroll
-            for (int r = 0; r < R; ++r) {
-                const int64_t ro = rr[r];
-                u[r] = gv_load<FMT, A16>(rec_m + ro * rec_bytes,
-                                         FMT == TQ_NVFP4_G16
-                                             ? static_cast<const void*>(static_cast<const uint8_t*>(sc_m) + ro * G)
-                                             : static_cast<const void*>(static_cast<const float*>(sc_m) + ro * G),
-                                         FMT == TQ_INT4_G128_ASYM ? zp_m + ro * G : nullptr, g, q, G);
-            }
-        };
+        for (int r = 0; r < R; ++r) rr[r] = static_cast<int>(min(ob + r, O - 1) - ofirst);
         float acc[R][B];
 #pragma unroll
         for (int r = 0; r < R; ++r)
 #pragma unroll
             for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
         for (int64_t t = 0; t < nT; ++t) {
+            const int64_t qb = t * (TI >> 5);
+            const int nqt = static_cast<int>(min(TI >> 5, nq - qb));
+            int qt = slice * 32 + lane;   // quad within the tile
+            bool have = qt < nqt;
+            GvRows<FMT, A16, R> rw;
+            rw.init(packed, scales, zeros, static_cast<int>(G), e * O + ofirst, rr, static_cast<int>(qb) + qt);
+            Quad cur[R];
+            if (have) {                   // the first loads are in flight while x is staged
+#pragma unroll
+                for (int r = 0; r < R; ++r) cur[r] = rw.load(r, g);
+            }
             if (staged_t != t || (staged_e != e && x_ms != 0)) {   // block-uniform
                 __syncthreads();
-                gv_stage(xs, x, x_bf16 != 0, e * x_ms, I, t * TI, TI, B, vec);
+                gv_stage<FMT == TQ_INT3_G64_SYM>(xs, x, x_bf16 != 0, e * x_ms, I, t * TI, TI, B, vec);
                 __syncthreads();
                 staged_t = t;
                 staged_e = e;
             }
-            const int64_t qb = t * (TI >> 5);
-            const int64_t nqt = min(TI >> 5, nq - qb);
-            int64_t qt = static_cast<int64_t>(slice) * 32 + lane;   // quad within the tile
-            bool have = qt < nqt;
-            Quad cur[R];
-            if (have) load(cur, qb + qt);
             while (have) {
-                const int64_t qn = qt + qstep;
+                const int qn = qt + qstep;
                 const bool hn = qn < nqt;
-                Quad nxt[R];
-                if (hn) load(nxt, qb + qn);
-                gv_quad<FMT, B, R>(cur, xs + (qt >> 5) * 256 + lane, slots, acc);
+                if constexpr (GV_DB) {    // the next quads' loads are issued before these are used
+                    Quad nxt[R];
+                    if (hn) {
+                        rw.next(qstep);
 #pragma unroll
-                for (int r = 0; r < R; ++r) cur[r] = nxt[r];
+                        for (int r = 0; r < R; ++r) nxt[r] = rw.load(r, g);
+                    }
+                    gv_quad<FMT, B, R>(cur, xs + (qt >> 5) * 256 + lane, slots, acc);
+#pragma unroll
+                    for (int r = 0; r < R; ++r) cur[r] = nxt[r];
+                } else {
+                    gv_quad<FMT, B, R>(cur, xs + (qt >> 5) * 256 + lane, slots, acc);
+                    if (hn) {
+                        rw.next(qstep);
+#pragma unroll
+                        for (int r = 0; r < R; ++r) cur[r] = rw.load(r, g);
+                    }
+                }
                 qt = qn;
                 have = hn;
             }
