@@ -443,6 +443,8 @@ def main():
                           "frac": gbs / pk["hbm_gbs"]}
     hbm_rows["pack"] = time_pack(tq, step, pk)
     next_rows = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
+    if step.units[0].fmt == "int4_g128_asym":
+        next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -505,6 +507,32 @@ def time_pack(tq, step, pk, reps=12):
     gbs = nbytes / (ms * 1e-3) / 1e9
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
             "note": f"first unit, back-to-back launches over {len(Ws)} rotating weight copies"}
+
+
+def time_ladder(tq, step, peak_tinst, reps=3):
+    """The int4 search on the "256/64" grid (256 scales x 64 zero-points: 16
+    distinct zero-points, 4096 candidate-element evaluations per weight, 4x
+    the default grid's) on the first unit, rotating weight copies; the same
+    per-evaluation instruction figure as the default grid's roofline."""
+    u = step.units[0]
+    m = step._m_for(u)
+    p = tq.SearchParams(asym_n_scale=256, asym_n_zero=64)
+    Ws = [s[1][0] for s in step.sets]
+    res = tq.tq_search_groups(Ws[0], m, tq.INT4_G128_ASYM, params=p)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(reps):
+        tq.tq_search_groups(Ws[k % len(Ws)], m, tq.INT4_G128_ASYM, params=p, out=res)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    nw = u.W.numel()
+    cee = 256 * 16
+    achieved = cee * 5 * nw / (ms * 1e-3) / 1e12
+    return {"ms": ms, "weights_per_s": nw / (ms * 1e-3), "cee_per_s": cee * nw / (ms * 1e-3),
+            "achieved_tinst": achieved, "frac": achieved / peak_tinst,
+            "note": f"first unit, {reps} launches, 4096 candidate-element evaluations x 5 instr per weight"}
 
 
 def time_gemv(tq, step, pk, B, reps=20):

@@ -9,7 +9,9 @@
 //   L = sum_j m_j (w_j - s (q_j - z))^2; ties keep the lowest index nz k + i.
 //
 // B200 mapping: one warp per 128-weight group; lane l owns scales l and l+32
-// and all 16 distinct zero-points.  The group's weights (and sqrt of their
+// (and 64 p + l, 64 p + 32 + l in pass p of a grid of more than 64 scales:
+// the "256/64" end of the page's quality ladder, results bullet 2) and all 16
+// distinct zero-points.  The group's weights (and sqrt of their
 // imatrix weights) are staged in shared memory and broadcast to all lanes, so
 // the 1024 candidates reuse one HBM read.  Zero-points repeated in the
 // 32-point list never win under the lowest-index rule, so only the first
@@ -51,7 +53,7 @@ struct AsymArgs {
     int ns, nz;
     int zfirst[16];      // lowest i with z_i = z
     int8_t zval[64];     // z_i for i < nz (nz <= 64)
-    float c[64];         // fl32(f_k / 15)
+    float c[256];        // fl32(f_k / 15), k < ns <= 256
 };
 
 // Lane l holds elements 4l..4l+3 of the group.
@@ -115,7 +117,7 @@ __device__ __forceinline__ void acc_scale(float w, float sm, float s, float inv,
     }
 }
 
-template <typename T>
+template <typename T, int NP>
 __global__ void __launch_bounds__(ASYM_WARPS * 32)
 k_search_int4(const __grid_constant__ AsymArgs a) {
     __shared__ __align__(16) float2 lists[ASYM_WARPS][132];   // two sign lists, each padded to even length
@@ -123,8 +125,6 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
     const int64_t G = (a.I + 127) >> 7;
     const int64_t OG = a.O * G;
     const int64_t total = a.n_mat * OG;
-    const bool actA = lane < a.ns, actB = lane + 32 < a.ns;
-    const float cA = a.c[actA ? lane : 0], cB = a.c[actB ? lane + 32 : 0];
     const T* W = static_cast<const T*>(a.W);
     float2* list = lists[wid];
     const float4* list4 = reinterpret_cast<const float4*>(list);
@@ -218,72 +218,96 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         }
         __syncwarp();
 
-        const float sA = __fmul_rn(cA, Rs), sB = __fmul_rn(cB, Rs);
-        const float sAo = __fmul_rn(cA, R), sBo = __fmul_rn(cB, R);
-        const float iA = rcp_approx(sA), iB = rcp_approx(sB);
-        float2 a2[8], b2[8];
-#pragma unroll
-        for (int p = 0; p < 8; ++p) { a2[p] = make_float2(0.f, 0.f); b2[p] = make_float2(0.f, 0.f); }
-        for (int j = 0; j < (nneg_pad >> 1); ++j) {
-            const float4 p = list4[j];
-            acc_scale<false>(p.x, p.y, sA, iA, a2);
-            acc_scale<false>(p.x, p.y, sB, iB, b2);
-            acc_scale<false>(p.z, p.w, sA, iA, a2);
-            acc_scale<false>(p.z, p.w, sB, iB, b2);
-        }
-        for (int j = nneg_pad >> 1; j < ((nneg_pad + npos_pad) >> 1); ++j) {
-            const float4 p = list4[j];
-            acc_scale<true>(p.x, p.y, sA, iA, a2);
-            acc_scale<true>(p.x, p.y, sB, iB, b2);
-            acc_scale<true>(p.z, p.w, sA, iA, a2);
-            acc_scale<true>(p.z, p.w, sB, iB, b2);
-        }
-        float accA[16], accB[16];
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-            accA[2 * p] = a2[p].x; accA[2 * p + 1] = a2[p].y;
-            accB[2 * p] = b2[p].x; accB[2 * p + 1] = b2[p].y;
-        }
-
-        // lane-local argmin in index order (all of scale A precede scale B)
+        // NP passes of 64 scales: lane l takes scales 64 p + l (A) and 64 p + 32 + l (B).
+        // A pass flags its candidates within the window of the running minimum; the
+        // minimum only falls, so the flags are a superset of the final window.
         float L = __int_as_float(0x7f800000);
         int bi = INT_MAX;
-        if (actA) {
+        unsigned wm[NP];
 #pragma unroll
-            for (int z = 0; z < 16; ++z)
-                if (accA[z] < L) { L = accA[z]; bi = a.nz * lane + a.zfirst[z]; }
-        }
-        if (actB) {
+        for (int ps = 0; ps < NP; ++ps) {
+            const int kA = 64 * ps + lane, kB = kA + 32;
+            const bool actA = kA < a.ns, actB = kB < a.ns;
+            if (NP > 1 && !__any_sync(FULL, actA)) {   // passes past ns
+                wm[ps] = 0u;
+                continue;
+            }
+            const float cA = a.c[actA ? kA : 0], cB = a.c[actB ? kB : 0];
+            const float sA = __fmul_rn(cA, Rs), sB = __fmul_rn(cB, Rs);
+            const float iA = rcp_approx(sA), iB = rcp_approx(sB);
+            float2 a2[8], b2[8];
 #pragma unroll
-            for (int z = 0; z < 16; ++z)
-                if (accB[z] < L) { L = accB[z]; bi = a.nz * (lane + 32) + a.zfirst[z]; }
-        }
-        warp_argmin(L, bi);
-        const float thr = __fmaf_rn(L, AWIN, L);
-        unsigned wm = 0u;
+            for (int p = 0; p < 8; ++p) { a2[p] = make_float2(0.f, 0.f); b2[p] = make_float2(0.f, 0.f); }
+            for (int j = 0; j < (nneg_pad >> 1); ++j) {
+                const float4 p = list4[j];
+                acc_scale<false>(p.x, p.y, sA, iA, a2);
+                acc_scale<false>(p.x, p.y, sB, iB, b2);
+                acc_scale<false>(p.z, p.w, sA, iA, a2);
+                acc_scale<false>(p.z, p.w, sB, iB, b2);
+            }
+            for (int j = nneg_pad >> 1; j < ((nneg_pad + npos_pad) >> 1); ++j) {
+                const float4 p = list4[j];
+                acc_scale<true>(p.x, p.y, sA, iA, a2);
+                acc_scale<true>(p.x, p.y, sB, iB, b2);
+                acc_scale<true>(p.z, p.w, sA, iA, a2);
+                acc_scale<true>(p.z, p.w, sB, iB, b2);
+            }
+            float accA[16], accB[16];
 #pragma unroll
-        for (int z = 0; z < 16; ++z) {
-            if (actA && accA[z] <= thr) wm |= 1u << z;
-            if (actB && accB[z] <= thr) wm |= 1u << (16 + z);
+            for (int p = 0; p < 8; ++p) {
+                accA[2 * p] = a2[p].x; accA[2 * p + 1] = a2[p].y;
+                accB[2 * p] = b2[p].x; accB[2 * p + 1] = b2[p].y;
+            }
+
+            // lane-local argmin in index order (all of scale A precede scale B)
+            float Lp = __int_as_float(0x7f800000);
+            int bp = INT_MAX;
+            if (actA) {
+#pragma unroll
+                for (int z = 0; z < 16; ++z)
+                    if (accA[z] < Lp) { Lp = accA[z]; bp = a.nz * kA + a.zfirst[z]; }
+            }
+            if (actB) {
+#pragma unroll
+                for (int z = 0; z < 16; ++z)
+                    if (accB[z] < Lp) { Lp = accB[z]; bp = a.nz * kB + a.zfirst[z]; }
+            }
+            warp_argmin(Lp, bp);
+            if (Lp < L) { L = Lp; bi = bp; }   // earlier passes hold lower indices: ties keep them
+            const float thr = __fmaf_rn(L, AWIN, L);
+            unsigned f = 0u;
+#pragma unroll
+            for (int z = 0; z < 16; ++z) {
+                if (actA && accA[z] <= thr) f |= 1u << z;
+                if (actB && accB[z] <= thr) f |= 1u << (16 + z);
+            }
+            wm[ps] = f;
         }
-        const int cnt = static_cast<int>(__reduce_add_sync(FULL, static_cast<unsigned>(__popc(wm))));
+        int cnt = 0;
+#pragma unroll
+        for (int ps = 0; ps < NP; ++ps) cnt += __popc(wm[ps]);
+        cnt = static_cast<int>(__reduce_add_sync(FULL, static_cast<unsigned>(cnt)));
         double lossd = static_cast<double>(L) * back;
         if (cnt > 1) {   // near tie: decide in fp64, candidates in index order
             double best = __longlong_as_double(0x7ff0000000000000ll);
             int bidx = bi;
-            for (int part = 0; part < 2; ++part) {
-                unsigned ls = __ballot_sync(FULL, part ? (wm >> 16) != 0u : (wm & 0xffffu) != 0u);
-                while (ls) {
-                    const int l2 = __ffs(ls) - 1;
-                    ls &= ls - 1;
-                    unsigned zm = __shfl_sync(FULL, wm, l2);
-                    zm = part ? (zm >> 16) : (zm & 0xffffu);
-                    const float sc = __shfl_sync(FULL, part ? sBo : sAo, l2);
-                    while (zm) {
-                        const int z = __ffs(zm) - 1;
-                        zm &= zm - 1;
-                        const double Ld = loss64_int4(w, mv, sc, z);
-                        if (Ld < best) { best = Ld; bidx = a.nz * (l2 + 32 * part) + a.zfirst[z]; }
+#pragma unroll
+            for (int ps = 0; ps < NP; ++ps) {
+                for (int part = 0; part < 2; ++part) {
+                    unsigned ls = __ballot_sync(FULL, part ? (wm[ps] >> 16) != 0u : (wm[ps] & 0xffffu) != 0u);
+                    while (ls) {
+                        const int l2 = __ffs(ls) - 1;
+                        ls &= ls - 1;
+                        unsigned zm = __shfl_sync(FULL, wm[ps], l2);
+                        zm = part ? (zm >> 16) : (zm & 0xffffu);
+                        const int k = 64 * ps + 32 * part + l2;
+                        const float sc = __fmul_rn(a.c[k], R);
+                        while (zm) {
+                            const int z = __ffs(zm) - 1;
+                            zm &= zm - 1;
+                            const double Ld = loss64_int4(w, mv, sc, z);
+                            if (Ld < best) { best = Ld; bidx = a.nz * k + a.zfirst[z]; }
+                        }
                     }
                 }
             }
@@ -314,11 +338,23 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
     }
 }
 
+template <int NP>
+void launch_int4(const AsymArgs& a, bool bf16, int64_t total, cudaStream_t st) {
+    int bpsm = 0;
+    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t, NP>, ASYM_WARPS * 32, 0);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<float, NP>, ASYM_WARPS * 32, 0);
+    if (bpsm < 1) bpsm = 1;
+    const int64_t need = (total + ASYM_WARPS - 1) / ASYM_WARPS;
+    const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
+    if (bf16) k_search_int4<uint16_t, NP><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    else k_search_int4<float, NP><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+}
+
 tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
                              const tq_search_params* p, float* scales, uint8_t* zeros, int32_t* idx,
                              double* loss, uint8_t* packed, cudaStream_t st) {
-    if (p->asym_n_scale < 2 || p->asym_n_scale > 64)
-        return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_scale must be in [2, 64]");
+    if (p->asym_n_scale < 2 || p->asym_n_scale > 256)
+        return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_scale must be in [2, 256]");
     if (p->asym_n_zero < 16 || p->asym_n_zero > 64)
         return set_error(TQ_ERR_UNSUPPORTED, "int4 search: asym_n_zero must be in [16, 64]");
     if (!(p->asym_lo > 0.0) || !(p->asym_hi >= p->asym_lo))
@@ -330,7 +366,7 @@ tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
     a.scales = scales; a.zeros = zeros; a.idx = idx; a.loss = loss; a.packed = packed;
     a.ns = p->asym_n_scale; a.nz = p->asym_n_zero;
     const double lo = p->asym_lo, hi = p->asym_hi;
-    for (int k = 0; k < 64; ++k) {
+    for (int k = 0; k < 256; ++k) {
         const double f = lo + ((hi - lo) * static_cast<double>(k)) / static_cast<double>(a.ns - 1);
         a.c[k] = k < a.ns ? static_cast<float>(f / 15.0) : 1.0f;
     }
@@ -350,15 +386,9 @@ tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
     const int64_t total = W->n_mat * W->rows * G;
     if (total >= (int64_t(1) << 32)) return set_error(TQ_ERR_UNSUPPORTED, "int4 search: more than 2^32 groups");
     a.gi = GroupIndex(W->rows, G);
-    int bpsm = 0;
     const bool bf16 = W->dtype == TQ_BF16;
-    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t>, ASYM_WARPS * 32, 0);
-    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<float>, ASYM_WARPS * 32, 0);
-    if (bpsm < 1) bpsm = 1;
-    const int64_t need = (total + ASYM_WARPS - 1) / ASYM_WARPS;
-    const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
-    if (bf16) k_search_int4<uint16_t><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
-    else k_search_int4<float><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    if (a.ns <= 64) launch_int4<1>(a, bf16, total, st);
+    else launch_int4<4>(a, bf16, total, st);
     return check_launch("int4 search");
 }
 

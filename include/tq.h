@@ -194,7 +194,9 @@ tq_status tq_amax(const tq_mat* W, float* amax, tq_stream_t stream);
  *          as tq_pack would (round-to-nearest and packing fused into the
  *          search).
  * Grid limits of this build: sym_n1, sym_n2 in [2, 32]; asym_n_scale in
- * [2, 64], asym_n_zero >= 16 (every integer zero-point 0..15 occurs);
+ * [2, 256] (more than 64 scales run in passes of 64: the "256/64" end of
+ * [NeUQI]'s ladder, results bullet 2), asym_n_zero in [16, 64] (every
+ * integer zero-point 0..15 occurs);
  * fp4_window in [1, 16].  Others return TQ_ERR_UNSUPPORTED. */
 tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_stride, int32_t fmt,
                            const tq_search_params* params, void* scales, uint8_t* zeros,

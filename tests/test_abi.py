@@ -85,6 +85,11 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, None, fake, fake, None,
                               None, None, None, None) == 1
     # unsupported grid sizes
+    p2 = tq._Params()
+    L.tq_default_params(ctypes.byref(p2))
+    p2.asym_n_scale = 257
+    assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT4_G128_ASYM, ctypes.byref(p2), fake, fake,
+                              None, None, None, None, None) == 2
     p.sym_n1 = 40
     assert L.tq_search_groups(ctypes.byref(m), fake, 0, tq.INT3_G64_SYM, ctypes.byref(p), fake, None,
                               None, None, None, None, None) == 2

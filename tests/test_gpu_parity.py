@@ -178,6 +178,32 @@ def test_grid_variants():
     assert (r.cand_idx.cpu().numpy() == i).mean() >= 0.999
 
 
+def test_asym_ladder_256_64():
+    """The "256/64" end of the asymmetric grid ladder (256 scales x 64
+    zero-points, four passes of 64 scales): same candidate as the oracle,
+    bit-identical parameters on matching groups, never more than 1e-5 above
+    the oracle's minimum, fused pack identical to the oracle's packing."""
+    g = torch.Generator(device=DEV).manual_seed(29)
+    W = (synth.student_t((2, 40, 704), 4, g, DEV) * 0.02).bfloat16()   # 5.5 groups per row
+    m = synth.random_imatrix(704, 4, DEV)
+    Wh, mh = host32(W), m.cpu().numpy()
+    for ns, nz in [(256, 64), (100, 32), (65, 16)]:
+        p = tq.SearchParams(asym_n_scale=ns, asym_n_zero=nz)
+        r = tq.tq_search_groups(W, m, tq.INT4_G128_ASYM, params=p)
+        torch.cuda.synchronize()
+        s, z, i, L, q = oracle.search_asym_int4(Wh, mh, ns=ns, nz=nz)
+        gi = r.cand_idx.cpu().numpy()
+        same = gi == i
+        assert same.mean() >= 0.999, (ns, nz, same.mean())
+        assert gi.max() < ns * nz
+        assert np.array_equal(r.scales.cpu().numpy()[same], s[same])
+        assert np.array_equal(r.zeros.cpu().numpy()[same], z[same])
+        Lg = oracle.loss_given_int4(Wh, mh, r.scales.cpu().numpy(), r.zeros.cpu().numpy())
+        assert np.all(Lg - L * (1 + LOSS_RTOL) <= 1e-30), (ns, nz)
+        ref, _ = oracle_packed(tq.INT4_G128_ASYM, Wh, r.scales.cpu().numpy(), r.zeros.cpu().numpy())
+        assert np.array_equal(r.packed.cpu().numpy(), ref)
+
+
 # ------------------------------------------------------------------ code packing
 
 @pytest.mark.parametrize("fmt,lo,hi", [(tq.INT3_G64_SYM, -4, 4), (tq.INT4_G128_ASYM, 0, 16),
