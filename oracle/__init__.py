@@ -46,6 +46,9 @@ def lib():
         i64, i32, f64, f32 = ctypes.c_int64, ctypes.c_int, ctypes.c_double, ctypes.c_float
         sig = {
             "orc_imatrix": (None, [P, i64, i64, i64, P]),
+            "orc_hessian": (None, [P, i64, i64, i64, P]),
+            "orc_hessian_entry": (f64, [P, i64, i64, i64, i64]),
+            "orc_proxy_error_full": (None, [P, P, i64, i64, P, P, P]),
             "orc_sym_stage1_ratio": (f32, [i32, f64, f64, i32]),
             "orc_sym_stage2_ratio": (f32, [i32, i32, f64, f64, i32, i32]),
             "orc_sym_loss": (f64, [P, P, i32, f32, P]),
@@ -130,6 +133,30 @@ def imatrix(X) -> np.ndarray:
     m = np.empty(I, dtype=np.float64)
     lib().orc_imatrix(_p(X), T, I, I, _p(m))
     return m
+
+
+def hessian(X) -> np.ndarray:
+    """[T, I] activations -> fp64 H = X^T X (both triangles)."""
+    X = _f32(X)
+    T, I = X.shape
+    H = np.empty((I, I), dtype=np.float64)
+    lib().orc_hessian(_p(X), T, I, I, _p(H))
+    return H
+
+
+def hessian_entry(X, i: int, j: int) -> float:
+    X = _f32(X)
+    T, I = X.shape
+    return lib().orc_hessian_entry(_p(X), T, I, int(i), int(j))
+
+
+def proxy_error_full(W, What, H) -> Tuple[float, float]:
+    """(num, den) for one O x I matrix with a full Hessian: tr(E H E^T), tr(W H W^T)."""
+    W = _f32(W); What = _f32(What); H = np.ascontiguousarray(H, np.float64)
+    O, I = W.shape
+    num = ctypes.c_double(); den = ctypes.c_double()
+    lib().orc_proxy_error_full(_p(W), _p(What), O, I, _p(H), ctypes.byref(num), ctypes.byref(den))
+    return num.value, den.value
 
 
 # ---------------------------------------------------------------- searches

@@ -60,6 +60,61 @@ ORC_API void orc_imatrix(const float* X, int64_t T, int64_t I, int64_t ld, doubl
 }
 
 /* ------------------------------------------------------------------ */
+/* Hessian H = sum_t x_t^T x_t                                         */
+/* ------------------------------------------------------------------ */
+
+/* H[i][j] = sum_t x_{t,i} x_{t,j} in fp64 for one [T, I] activation matrix
+ * with row stride ld ([TT] pipeline table, step 1: the per-linear-input
+ * Hessian accumulated over the calibration tokens).  Products of fp32 (and
+ * bf16) values are exact in fp64; the sum is taken in token order.  H is
+ * written in full (both triangles), row stride I. */
+ORC_API void orc_hessian(const float* X, int64_t T, int64_t I, int64_t ld, double* H)
+{
+    #pragma omp parallel for schedule(dynamic, 4)
+    for (int64_t i = 0; i < I; ++i) {
+        for (int64_t j = i; j < I; ++j) {
+            double s = 0.0;
+            for (int64_t t = 0; t < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];
+            H[i * I + j] = s;
+            H[j * I + i] = s;
+        }
+    }
+}
+
+/* One entry H[i][j] (for sampled checks of large H). */
+ORC_API double orc_hessian_entry(const float* X, int64_t T, int64_t ld, int64_t i, int64_t j)
+{
+    double s = 0.0;
+    for (int64_t t = 0; t < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];
+    return s;
+}
+
+/* Proxy error with a full Hessian ([TT] "Risks to measure: Precision"):
+ * num = tr(E H E^T) = sum_o sum_{i,j} e_{o,i} H_{i,j} e_{o,j}, E = W - What,
+ * den = tr(W H W^T), for one O x I matrix; fp64 throughout. */
+ORC_API void orc_proxy_error_full(const float* W, const float* What, int64_t O, int64_t I,
+                                  const double* H, double* num, double* den)
+{
+    double n = 0.0, d = 0.0;
+    #pragma omp parallel for reduction(+:n, d) schedule(static)
+    for (int64_t o = 0; o < O; ++o) {
+        const float* w = W + o * I;
+        const float* wh = What + o * I;
+        for (int64_t i = 0; i < I; ++i) {
+            double hn = 0.0, hd = 0.0;
+            for (int64_t j = 0; j < I; ++j) {
+                hn += H[i * I + j] * ((double)w[j] - (double)wh[j]);
+                hd += H[i * I + j] * (double)w[j];
+            }
+            n += ((double)w[i] - (double)wh[i]) * hn;
+            d += (double)w[i] * hd;
+        }
+    }
+    *num = n;
+    *den = d;
+}
+
+/* ------------------------------------------------------------------ */
 /* Round-to-nearest helpers                                            */
 /* ------------------------------------------------------------------ */
 

@@ -32,6 +32,12 @@ MUTANTS = {
     "proxy_den_error": ("b += (double)m[j] * (w * w);", "b += (double)m[j] * (e * e) + (double)m[j] * (w * w) * 0.0 + (double)m[j] * (w * w);"),
     "argmin_last_tie": ("if (L < bestL) { bestL = L; best = 2 * k + sg; bestS = s; }", "if (L <= bestL) { bestL = L; best = 2 * k + sg; bestS = s; }"),
     "nvfp4_global_448": ("return (float)((double)amax / 2688.0);", "return (float)((double)amax / 448.0);"),
+    "hessian_transposed_operand": ("for (int64_t t = 0; t < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];\n            H[i * I + j] = s;",
+                                   "for (int64_t t = 0; t < T; ++t) s += (double)X[t * ld + i] * (double)X[j * ld + (t % I)];\n            H[i * I + j] = s;"),
+    "hessian_last_token_dropped": ("for (int64_t t = 0; t < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];\n            H[i * I + j] = s;",
+                                   "for (int64_t t = 0; t + 1 < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];\n            H[i * I + j] = s;"),
+    "proxy_full_diagonal_only": ("hn += H[i * I + j] * ((double)w[j] - (double)wh[j]);",
+                                 "hn += (i == j) * H[i * I + j] * ((double)w[j] - (double)wh[j]);"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }

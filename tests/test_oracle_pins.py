@@ -556,3 +556,45 @@ def test_int3_g64_beats_rowwise_int4_on_outlier_rows(orc):
     rms4 = np.sqrt(np.mean((np.float64(Wo) - What4) ** 2))
     assert rms3 < rms4
     assert rms4 / rms3 > 1.5
+
+
+# ------------------------------------------------------------------ Hessian (TT step 1)
+
+def test_hessian_pins(orc):
+    """H = X^T X ([TT] pipeline step 1): brute force on a tiny case, symmetry,
+    diag(H) = T m against the imatrix, integer-valued X exactly, a rank-one X
+    in closed form, and the single-entry form agreeing with the full one."""
+    rng = np.random.default_rng(41)
+    X = rng.standard_normal((7, 5)).astype(np.float32)
+    H = orc.hessian(X)
+    bf = [[sum(float(X[t, i]) * float(X[t, j]) for t in range(7)) for j in range(5)] for i in range(5)]
+    assert np.allclose(H, np.array(bf), rtol=1e-15, atol=0)
+    X = rng.standard_normal((300, 70)).astype(np.float32)
+    H = orc.hessian(X)
+    assert np.array_equal(H, H.T)
+    assert np.allclose(np.diag(H) / 300.0, orc.imatrix(X), rtol=1e-14)
+    Xi = rng.integers(-3, 4, size=(500, 40)).astype(np.float32)
+    assert np.array_equal(orc.hessian(Xi), Xi.astype(np.int64).T @ Xi.astype(np.int64))
+    u = rng.standard_normal(40).astype(np.float32)
+    R1 = np.tile(u, (3, 1))                          # every token the same vector: H = 3 u u^T
+    assert np.allclose(orc.hessian(R1), 3.0 * np.outer(u.astype(np.float64), u), rtol=1e-15)
+    assert orc.hessian_entry(X, 3, 11) == H[3, 11]
+
+
+def test_proxy_error_full_reduces_to_diagonal(orc):
+    """tr(E H E^T) with a diagonal H is the diagonal-imatrix proxy error; with
+    H = X^T X it equals ||E X^T||_F^2 (a second closed form)."""
+    rng = np.random.default_rng(43)
+    O, I = 6, 50
+    W = rng.standard_normal((O, I)).astype(np.float32)
+    Wh = (W + 0.01 * rng.standard_normal((O, I))).astype(np.float32)
+    m = rng.random(I).astype(np.float32)
+    n1, d1 = orc.proxy_error_full(W, Wh, np.diag(m.astype(np.float64)))
+    n2, d2 = orc.proxy_error(W, Wh, m)
+    assert np.isclose(n1, n2, rtol=1e-12) and np.isclose(d1, d2, rtol=1e-12)
+    X = rng.standard_normal((80, I)).astype(np.float32)
+    H = orc.hessian(X)
+    n, d = orc.proxy_error_full(W, Wh, H)
+    E = W.astype(np.float64) - Wh.astype(np.float64)
+    assert np.isclose(n, np.sum((E @ X.astype(np.float64).T) ** 2), rtol=1e-12)
+    assert np.isclose(d, np.sum((W.astype(np.float64) @ X.astype(np.float64).T) ** 2), rtol=1e-12)
