@@ -32,7 +32,7 @@ __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_dequant_gemv", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -52,7 +52,7 @@ EXPORTS = [
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
-    "tq_dequant_gemv",
+    "tq_dequant_gemv", "tq_hessian",
 ]
 
 
@@ -127,6 +127,7 @@ def lib():
             "tq_packed_bytes": (sz, [i32, i64, i64]),
             "tq_imatrix_workspace_bytes": (sz, [Mp]),
             "tq_imatrix": (i32, [Mp, P, i64, ctypes.c_float, i32, P, sz, P]),
+            "tq_hessian": (i32, [Mp, P, i64, i64, ctypes.c_float, i32, P]),
             "tq_amax": (i32, [Mp, P, P]),
             "tq_search_groups": (i32, [Mp, P, i64, i32, ctypes.POINTER(_Params), P, P, P, P, P, P, P]),
             "tq_pack": (i32, [Mp, i32, P, P, P, P, P]),
@@ -252,6 +253,25 @@ def tq_imatrix(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optiona
                             ctypes.c_float(alpha), int(accumulate), _ptr(workspace),
                             workspace.numel(), _stream(stream)), "tq_imatrix")
     return m
+
+
+def tq_hessian(X: torch.Tensor, out: Optional[torch.Tensor] = None, alpha: float = 1.0,
+               accumulate: bool = False, stream=None) -> torch.Tensor:
+    """H[e] = alpha * X[e]^T X[e] (+ H[e] when accumulate), fp32, on the tensor
+    cores.  X: [T, I] or [n_mat, T, I] bf16 on the GPU; returns [I, I] or
+    [n_mat, I, I] (both triangles, exactly symmetric)."""
+    d = _mat(X, "X")
+    shape = (d.cols, d.cols) if X.dim() == 2 else (d.n_mat, d.cols, d.cols)
+    if out is None:
+        out = (torch.zeros if accumulate else torch.empty)(shape, dtype=torch.float32, device=X.device)
+    _cuda(out, "out")
+    if out.dtype != torch.float32 or tuple(out.shape) != shape or out.stride(-1) != 1:
+        raise ValueError(f"out must be float32 {shape} with unit column stride")
+    ldh = out.stride(-2)
+    hms = out.stride(0) if out.dim() == 3 else 0
+    _check(lib().tq_hessian(ctypes.byref(d), _ptr(out), ldh, hms, ctypes.c_float(alpha), int(accumulate),
+                            _stream(stream)), "tq_hessian")
+    return out
 
 
 def tq_imatrix_static(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optional[float] = None,

@@ -1,0 +1,353 @@
+// Hessian of a linear's inputs, H = sum_t x_t^T x_t (fp32), from bf16
+// activations X [T][I] on the 5th-generation tensor cores.
+//
+// Source: "Quantize on TT cards: CUDA-free GPTQ/LDLQ bfp4 pipeline" (tt-stack
+// issue #67), pipeline table step 1: the per-linear-input Hessian accumulated
+// in fp32 over the calibration tokens, a pure rank-k accumulation (its
+// diagonal is T times the activation imatrix).  The page measures the bf16
+// X^T X on its own accelerator at 5.9e-5 relative error (stage-1 precision
+// results); here the products of bf16 values are exact and only the fp32
+// accumulation rounds.
+//
+// As a GEMM: H[i][j] = sum_t X[t][i] X[t][j], M = N = I, K = T; both operands
+// are columns of row-major X, i.e. MN-major in memory, which the tensor core
+// reads directly (no transpose pass).  H is symmetric, so only tiles with
+// bi <= bj are computed and each value is written to both triangles (exactly
+// symmetric output).
+//
+// B200 mapping (one CTA per 128 x 128 tile of H, 4 warps, 2 CTAs per SM):
+//  * TMA (cp.async.bulk.tensor, 128-byte swizzle) brings 64-token slices of the
+//    two 128-column panels into a 3-stage shared-memory ring; a diagonal tile
+//    loads its single panel once.
+//  * One thread issues tcgen05.mma (kind::f16, bf16 in, fp32 accumulate,
+//    M = N = 128, K = 16, both operands MN-major from shared memory); the
+//    accumulator lives in 128 TMEM columns.  tcgen05.commit frees a stage when
+//    its MMAs have read it.
+//  * The 4 warps read the accumulator with tcgen05.ld (warp w: rows 32w..32w+31)
+//    and store it: each thread its row segment (contiguous) and, mirrored, a
+//    column segment (coalesced across the warp).
+//  * Tiles are grouped in 8 x 8 super-blocks so that the CTAs in flight share
+//    their panels in L2.
+// Every wait on an mbarrier has an iteration limit; on timeout the kernel
+// records it (tq_sync reports it), drains its in-flight copies, frees TMEM and
+// returns.
+#include <cuda.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "tq_internal.cuh"
+
+namespace tq {
+
+constexpr int HS_TILE = 128;      // tile of H (M = N)
+constexpr int HS_BK = 64;         // tokens per stage
+constexpr int HS_STAGES = 3;
+constexpr int HS_THREADS = 128;
+constexpr int HS_SUPER = 8;       // tiles per super-block side
+constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;           // one TMA box: 64 columns x 64 tokens, bf16
+constexpr int HS_OPERAND_BYTES = 2 * HS_BOX_BYTES;      // 128 columns
+constexpr int HS_STAGE_BYTES = 2 * HS_OPERAND_BYTES;    // A and B
+constexpr int HS_SMEM_BYTES = HS_STAGES * HS_STAGE_BYTES + 1024 /* alignment */ + 256 /* barriers */;
+constexpr unsigned HS_WAIT_LIMIT = 1u << 22;            // try_wait rounds before a wait is declared hung
+
+__device__ unsigned g_hs_timeouts = 0;
+
+// ------------------------------------------------------------------ PTX wrappers
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Waits for the phase of parity `parity` to complete; false after the limit.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity) {
+    for (unsigned it = 0; it < HS_WAIT_LIMIT; ++it) {
+        unsigned ok;
+        asm volatile(
+            "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    atomicAdd(&g_hs_timeouts, 1u);
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
+// Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle, 64
+// elements (128 B) per row along M/N, rows = tokens.  LBO = bytes between the
+// two 64-column halves, SBO = bytes between groups of 8 token rows.
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
+    constexpr uint64_t lbo = HS_BOX_BYTES >> 4, sbo = (8 * 128) >> 4;
+    return (static_cast<uint64_t>((addr >> 4) & 0x3fffu)) | (lbo << 16) | (sbo << 32) | (1ull << 46) |
+           (2ull << 61);
+}
+
+// Instruction descriptor: kind::f16, fp32 accumulator, bf16 A and B, both
+// MN-major, N = M = 128.
+constexpr uint32_t HS_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                              (static_cast<uint32_t>(HS_TILE >> 3) << 17) | (static_cast<uint32_t>(HS_TILE >> 4) << 24);
+
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(HS_IDESC), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// ------------------------------------------------------------------ kernel
+
+struct HsArgs {
+    int64_t T, I, ldh, hms;   // tokens, columns, H row stride, H matrix stride (elements)
+    float* H;
+    float alpha;
+    int accumulate;
+    int nb;                   // tiles per side
+    int nsb;                  // super-blocks per side
+};
+
+__global__ void __launch_bounds__(HS_THREADS, 1)
+k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsArgs a) {
+    // the tile: super-block pair (BI <= BJ), then a tile inside it
+    int p = static_cast<int>(blockIdx.x) / (HS_SUPER * HS_SUPER);
+    const int local = static_cast<int>(blockIdx.x) % (HS_SUPER * HS_SUPER);
+    int BI = 0;
+    while (p >= a.nsb - BI) { p -= a.nsb - BI; ++BI; }
+    const int BJ = BI + p;
+    const int bi = BI * HS_SUPER + local / HS_SUPER, bj = BJ * HS_SUPER + local % HS_SUPER;
+    if (bi > bj || bj >= a.nb) return;   // lower triangle or past the edge: nothing to do
+    const int e = static_cast<int>(blockIdx.y);
+    const bool diag = bi == bj;
+
+    extern __shared__ uint8_t hs_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hs_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + HS_STAGES * HS_STAGE_BYTES);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * HS_STAGES + 1);
+    int* progress = reinterpret_cast<int*>(tmem_slot + 1);   // [0] stages armed, [1] stages consumed, [2] ok
+    const uint32_t s_base = smem_u32(smem);
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + HS_STAGES), done = smem_u32(bars + 2 * HS_STAGES);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nk = static_cast<int>((a.T + HS_BK - 1) / HS_BK);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < HS_STAGES; ++s) {
+            mbar_init(full0 + 8 * s, 1);
+            mbar_init(empty0 + 8 * s, 1);
+        }
+        mbar_init(done, 1);
+        progress[0] = 0;
+        progress[1] = 0;
+        progress[2] = 1;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {   // the whole warp allocates 128 TMEM columns
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                     "r"(HS_TILE));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0 && lane == 0) {   // TMA producer
+        const uint32_t bytes = diag ? HS_OPERAND_BYTES : HS_STAGE_BYTES;
+        int k = 0;
+        for (; k < nk; ++k) {
+            const int s = k % HS_STAGES;
+            if (!mbar_wait(empty0 + 8 * s, ((k / HS_STAGES) & 1) ^ 1)) break;
+            const uint32_t st = s_base + s * HS_STAGE_BYTES, bar = full0 + 8 * s;
+            mbar_expect_tx(bar, bytes);
+            const int t0 = k * HS_BK;
+            tma_load_3d(st, &xmap, bar, bi * HS_TILE, t0, e);
+            tma_load_3d(st + HS_BOX_BYTES, &xmap, bar, bi * HS_TILE + 64, t0, e);
+            if (!diag) {
+                tma_load_3d(st + HS_OPERAND_BYTES, &xmap, bar, bj * HS_TILE, t0, e);
+                tma_load_3d(st + HS_OPERAND_BYTES + HS_BOX_BYTES, &xmap, bar, bj * HS_TILE + 64, t0, e);
+            }
+            progress[0] = k + 1;
+        }
+        if (k < nk) progress[2] = 0;
+    } else if (warp == 1 && lane == 0) {   // MMA issuer
+        int k = 0;
+        for (; k < nk; ++k) {
+            const int s = k % HS_STAGES;
+            if (!mbar_wait(full0 + 8 * s, (k / HS_STAGES) & 1)) break;
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t sa = s_base + s * HS_STAGE_BYTES;
+            const uint32_t sb = diag ? sa : sa + HS_OPERAND_BYTES;
+#pragma unroll
+            for (int kk = 0; kk < HS_BK / 16; ++kk)   // 16 tokens = 16 rows of 128 B per MMA
+                umma_bf16(tmem, umma_desc(sa + kk * 2048), umma_desc(sb + kk * 2048), (k | kk) != 0);
+            umma_commit(empty0 + 8 * s);   // the stage is free once these MMAs have read it
+            progress[1] = k + 1;
+        }
+        if (k < nk) progress[2] = 0;
+        umma_commit(done);                 // every MMA issued so far is complete
+    }
+
+    __syncwarp();   // lanes 1-31 of the producer and MMA warps wait here, not in a spin loop
+
+    // epilogue: warp w holds rows 32w .. 32w + 31 of the tile
+    const bool have = mbar_wait(done, 0);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    __syncwarp();
+    const bool ok = have && *reinterpret_cast<volatile int*>(&progress[2]) != 0;
+    const int m = warp * 32 + lane;
+    const int64_t gi = static_cast<int64_t>(bi) * HS_TILE + m;   // row of H this thread holds
+    float* He = a.H + static_cast<int64_t>(e) * a.hms;
+#pragma unroll 1
+    for (int c0 = 0; c0 < HS_TILE; c0 += 32) {
+        float v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
+        if (!ok) continue;
+        if (a.alpha != 1.0f) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(a.alpha, v[i]);
+        }
+        const int64_t gj0 = static_cast<int64_t>(bj) * HS_TILE + c0;
+        // mirrored: H[gj][gi] (for fixed column, the warp's 32 rows are consecutive)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const int64_t gj = gj0 + i;
+            if (gi < a.I && gj < a.I && (!diag || gj > gi)) {
+                float* q = He + gj * a.ldh + gi;
+                *q = a.accumulate ? __fadd_rn(*q, v[i]) : v[i];
+            }
+        }
+        // direct: H[gi][gj], this thread's row segment
+        if (gi < a.I) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int64_t gj = gj0 + i;
+                if (gj < a.I && (!diag || gj >= gi)) {
+                    float* q = He + gi * a.ldh + gj;
+                    *q = a.accumulate ? __fadd_rn(*q, v[i]) : v[i];
+                }
+            }
+        }
+    }
+
+    // teardown: drain copies armed but not consumed, then free TMEM
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int k = progress[1]; k < progress[0]; ++k)
+            if (!mbar_wait(full0 + 8 * (k % HS_STAGES), (k / HS_STAGES) & 1)) break;
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(HS_TILE));
+    }
+}
+
+// ------------------------------------------------------------------ host
+
+using EncodeTiled = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled encode_tiled() {
+    static std::once_flag once;
+    static EncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+bool hessian_take_timeouts() {
+    unsigned n = 0;
+    if (cudaMemcpyFromSymbol(&n, g_hs_timeouts, sizeof(n)) != cudaSuccess || n == 0) return false;
+    const unsigned zero = 0;
+    cudaMemcpyToSymbol(g_hs_timeouts, &zero, sizeof(zero));
+    return true;
+}
+
+}  // namespace tq
+
+using namespace tq;
+
+TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_mat_stride, float alpha,
+                            int32_t accumulate, tq_stream_t stream) {
+    clear_error();
+    TQ_REQUIRE(X && X->ptr && H, "tq_hessian: null pointer");
+    if (X->dtype != TQ_BF16) return set_error(TQ_ERR_UNSUPPORTED, "tq_hessian: activations must be bf16");
+    TQ_REQUIRE(X->n_mat >= 1 && X->rows >= 1 && X->cols >= 1, "tq_hessian: empty shape");
+    TQ_REQUIRE(X->ld >= X->cols && (X->ld * 2) % 16 == 0, "tq_hessian: X row stride must be >= I and a multiple of 16 bytes");
+    TQ_REQUIRE(X->n_mat == 1 || (X->mat_stride >= X->rows * X->ld && (X->mat_stride * 2) % 16 == 0),
+               "tq_hessian: X matrix stride must be >= T*ld and a multiple of 16 bytes");
+    TQ_REQUIRE(aligned16(X->ptr), "tq_hessian: X not 16-byte aligned");
+    TQ_REQUIRE(ldh >= X->cols, "tq_hessian: ldh < I");
+    TQ_REQUIRE(X->n_mat == 1 || h_mat_stride >= X->cols * ldh, "tq_hessian: H matrix stride < I*ldh");
+    TQ_REQUIRE(X->rows < (int64_t(1) << 31) && X->cols < (int64_t(1) << 31) && X->n_mat <= 65535,
+               "tq_hessian: T, I < 2^31 and n_mat <= 65535");
+    EncodeTiled enc = encode_tiled();
+    if (!enc) return set_error(TQ_ERR_CUDA, "tq_hessian: cuTensorMapEncodeTiled unavailable");
+
+    CUtensorMap map;
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(X->cols), static_cast<cuuint64_t>(X->rows),
+                                static_cast<cuuint64_t>(X->n_mat)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(X->ld * 2),
+                                   static_cast<cuuint64_t>((X->n_mat > 1 ? X->mat_stride : X->rows * X->ld) * 2)};
+    const cuuint32_t box[3] = {64, HS_BK, 1}, estr[3] = {1, 1, 1};
+    CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(X->ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return set_error(TQ_ERR_CUDA, "tq_hessian: tensor map encoding failed (%d)", static_cast<int>(r));
+
+    HsArgs a;
+    a.T = X->rows; a.I = X->cols; a.ldh = ldh; a.hms = X->n_mat > 1 ? h_mat_stride : 0;
+    a.H = H; a.alpha = alpha; a.accumulate = accumulate ? 1 : 0;
+    a.nb = static_cast<int>((X->cols + HS_TILE - 1) / HS_TILE);
+    a.nsb = (a.nb + HS_SUPER - 1) / HS_SUPER;
+    static std::once_flag attr;
+    std::call_once(attr, [] { cudaFuncSetAttribute(k_hessian, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM_BYTES); });
+    const int64_t pairs = static_cast<int64_t>(a.nsb) * (a.nsb + 1) / 2;
+    const int64_t gx = pairs * HS_SUPER * HS_SUPER;
+    TQ_REQUIRE(gx < (int64_t(1) << 31), "tq_hessian: I too large");
+    dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(X->n_mat));
+    k_hessian<<<grid, HS_THREADS, HS_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, a);
+    return check_launch("tq_hessian");
+}

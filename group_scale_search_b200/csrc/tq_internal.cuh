@@ -29,6 +29,10 @@ tq_status check_launch(const char* what);
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// True (and the count cleared) if a tq_hessian launch since the last call
+// gave up on a pipeline wait.
+bool hessian_take_timeouts();
+
 inline int elem_bytes(int32_t dt) { return dt == TQ_BF16 ? 2 : (dt == TQ_F32 ? 4 : 0); }
 
 inline int64_t group_of(int32_t fmt) {

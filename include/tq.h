@@ -260,6 +260,23 @@ tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void* scales
                           const float* global_scale, int64_t n_mat, int64_t O, int64_t I, const void* x,
                           int32_t x_dtype, int64_t B, int64_t x_mat_stride, float* y, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ Hessian
+ * H[e] = alpha * sum_t X[e][t]^T X[e][t] (+ H[e] when accumulate): the
+ * per-linear-input Hessian ([TT] pipeline table, step 1), fp32, from bf16
+ * activations X (tq_mat: n_mat sites of T tokens x I columns, ld and
+ * mat_stride multiples of 8 elements, 16-byte aligned), on the tensor cores
+ * (bf16 products exact, fp32 accumulation; alpha applied once, after).
+ * Its diagonal is T * the imatrix of tq_imatrix.  H: fp32 dense [n_mat][I]
+ * rows of ldh >= I elements, h_mat_stride >= I * ldh between sites; both
+ * triangles are written, exactly symmetric.  Error bound against the exact
+ * sum: |H - X^T X| <= (T/16 + 32) 2^-22 (|X|^T |X|) elementwise (every
+ * 16-token step of the accumulation rounds once).  Errors: TQ_ERR_INVALID_ARG
+ * for null/misaligned pointers, bad sizes or strides; TQ_ERR_UNSUPPORTED for
+ * fp32 X.  A pipeline wait that exceeds its limit makes the kernel give up
+ * (results undefined) and the next tq_sync return TQ_ERR_CUDA. */
+tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_mat_stride, float alpha,
+                     int32_t accumulate, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ proxy error
  * Per matrix e ([TT] "Risks to measure: Precision", H = diag(m)):
  *   num[e] = sum_{o,j} m_j (W - What)^2 = tr(E H E^T),
@@ -275,7 +292,7 @@ tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, co
 
 /* ------------------------------------------------------------------ testing aid
  * Synchronises `stream` and returns TQ_ERR_CUDA if it or an earlier kernel
- * failed. */
+ * failed (including a tq_hessian launch that gave up on a pipeline wait). */
 tq_status tq_sync(tq_stream_t stream);
 
 /* Self-test of the GPU's E2M1 conversion instructions, on which the NVFP4

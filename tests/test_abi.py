@@ -113,6 +113,18 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     assert b"aligned" in L.tq_last_error_string()
     assert gemv(fake, tq.INT4_G128_ASYM, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
     assert gemv(fake, tq.NVFP4_G16, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
+    # Hessian: (X, H, ldh, h_mat_stride, alpha, accumulate, stream)
+    hs = L.tq_hessian
+    x = tq._Mat(fake, 1, 0, 1, 256, 128, 128, 0)
+    x = tq._Mat(fake, 0, 0, 1, 256, 128, 128, 0)   # fp32 X
+    assert hs(ctypes.byref(x), fake, 128, 0, ctypes.c_float(1.0), 0, None) == 2
+    x = tq._Mat(fake, 1, 0, 1, 256, 128, 128, 0)
+    assert hs(ctypes.byref(x), fake, 100, 0, ctypes.c_float(1.0), 0, None) == 1   # ldh < I
+    assert hs(ctypes.byref(x), None, 128, 0, ctypes.c_float(1.0), 0, None) == 1
+    x = tq._Mat(fake, 1, 0, 1, 256, 100, 100, 0)   # row stride 200 B
+    assert hs(ctypes.byref(x), fake, 100, 0, ctypes.c_float(1.0), 0, None) == 1
+    x = tq._Mat(ctypes.c_void_p(0x1008), 1, 0, 1, 256, 128, 128, 0)
+    assert hs(ctypes.byref(x), fake, 128, 0, ctypes.c_float(1.0), 0, None) == 1
 
 
 def test_binding_refuses_cpu_tensors(tq):

@@ -481,3 +481,77 @@ def test_dequant_gemv_deterministic_and_exact_cases():
     want = np.float32(-2.0) * xh[:, 7][:, None] * np.ones((1, O), np.float32)
     want[:, 1] = 0.0
     assert np.array_equal(y.cpu().numpy()[0], want)
+
+
+# ------------------------------------------------------------------ Hessian (tensor cores)
+
+def _hessian_bound(Xh):
+    """Elementwise bound (T/16 + 32) 2^-22 (|X|^T |X|) of the fp32 accumulation."""
+    T = Xh.shape[0]
+    A = np.abs(Xh).astype(np.float64)
+    return (T / 16 + 32) * 2.0 ** -22 * (A.T @ A)
+
+
+@pytest.mark.parametrize("T,I,E", [(300, 200, 2), (64, 128, 1), (1, 129, 1), (777, 1000, 1), (100, 1, 1),
+                                   (2048, 520, 1)])
+def test_hessian_integer_exact(T, I, E):
+    """Integer-valued activations (every partial sum an exact fp32 integer):
+    H equals X^T X bit for bit, both triangles; ragged T and I, one token,
+    one column, several 128 x 128 tiles and super-blocks, several sites."""
+    rng = np.random.default_rng(T * 7 + I)
+    Xi = rng.integers(-3, 4, size=(E, T, I)).astype(np.float32)
+    ld = (I + 7) // 8 * 8
+    X = torch.zeros((E, T, ld), dtype=torch.bfloat16, device=DEV)
+    X[:, :, :I] = torch.from_numpy(Xi).to(DEV).bfloat16()
+    X = X[:, :, :I] if E > 1 else X[0, :, :I]
+    H = tq.tq_hessian(X)
+    tq.tq_sync()
+    Hh = H.cpu().numpy().reshape(E, I, I)
+    for e in range(E):
+        ref = Xi[e].astype(np.int64).T @ Xi[e].astype(np.int64)
+        assert np.array_equal(Hh[e], ref.astype(np.float32)), (e, np.argwhere(Hh[e] != ref)[:5])
+
+
+@pytest.mark.parametrize("T,I", [(1000, 300), (4096, 640), (130, 1030)])
+def test_hessian_matches_oracle(T, I):
+    """Random bf16 activations with per-column LogNormal scales: H within the
+    fp32 accumulation bound of the oracle's fp64 X^T X, exactly symmetric,
+    its diagonal T times the imatrix; alpha and accumulate."""
+    g = torch.Generator(device=DEV).manual_seed(T + I)
+    ld = (I + 7) // 8 * 8                            # 16-byte rows
+    X = torch.zeros((T, ld), dtype=torch.bfloat16, device=DEV)
+    X[:, :I] = (torch.randn((T, I), generator=g, device=DEV) *
+                torch.exp(torch.randn((I,), generator=g, device=DEV))).bfloat16()
+    X = X[:, :I]
+    H = tq.tq_hessian(X)
+    tq.tq_sync()
+    Xh = X.float().cpu().numpy()
+    ref = oracle.hessian(Xh)
+    Hh = H.cpu().numpy().astype(np.float64)
+    bad = np.abs(Hh - ref) > _hessian_bound(Xh)
+    assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[:5])
+    assert np.array_equal(H.cpu().numpy(), H.cpu().numpy().T)
+    m = oracle.imatrix(Xh)
+    assert np.allclose(np.diag(Hh) / T, m, rtol=(T / 16 + 32) * 2.0 ** -22, atol=0)
+    # alpha = 1/T applied once after the sum; accumulate adds into the given H
+    Ha = tq.tq_hessian(X, alpha=0.25)
+    tq.tq_sync()
+    assert torch.equal(Ha, H * 0.25)
+    H2 = tq.tq_hessian(X, out=H.clone(), alpha=0.25, accumulate=True)
+    tq.tq_sync()
+    assert torch.equal(H2, H + Ha)
+
+
+def test_hessian_strided_sites():
+    """Three sites with padded rows and a matrix stride; H into a padded output."""
+    E, T, I, ld = 3, 333, 250, 264
+    g = torch.Generator(device=DEV).manual_seed(5)
+    buf = torch.randn((E, T + 3, ld), generator=g, device=DEV).bfloat16()
+    X = buf[:, :T, :I]
+    out = torch.full((E, I, I + 8), float("nan"), device=DEV)[:, :, :I]
+    tq.tq_hessian(X, out=out)
+    tq.tq_sync()
+    for e in range(E):
+        Xh = X[e].float().cpu().numpy()
+        bad = np.abs(out[e].cpu().numpy().astype(np.float64) - oracle.hessian(Xh)) > _hessian_bound(Xh)
+        assert not bad.any(), e
