@@ -56,12 +56,12 @@ def log(*a):
 
 
 def peaks():
-    p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "source": "fallback"}
+    p = {"hbm_gbs": 6650.0, "sm_max_mhz": 1965.0, "bf16_tflops": 1590.0, "source": "fallback"}
     f = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(f):
         d = json.load(open(f))
         p = {"hbm_gbs": d.get("hbm_gbs", 6650.0), "sm_max_mhz": d.get("sm_max_mhz", 1965.0),
-             "source": "measured"}
+             "bf16_tflops": d.get("bf16_tflops", 1590.0), "source": "measured"}
     return p
 
 
@@ -445,6 +445,7 @@ def main():
     next_rows = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
     if step.units[0].fmt == "int4_g128_asym":
         next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
+    next_rows["hessian"] = time_hessian(tq, step, pk)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -533,6 +534,44 @@ def time_ladder(tq, step, peak_tinst, reps=3):
     return {"ms": ms, "weights_per_s": nw / (ms * 1e-3), "cee_per_s": cee * nw / (ms * 1e-3),
             "achieved_tinst": achieved, "frac": achieved / peak_tinst,
             "note": f"first unit, {reps} launches, 4096 candidate-element evaluations x 5 instr per weight"}
+
+
+def time_hessian(tq, step, pk):
+    """tq_hessian (H = X^T X on the tensor cores) on the first unit's
+    calibration activations (one matrix: the first expert of a MoE site),
+    rotating through the input sets.  Algorithmic work: the distinct entries
+    of the symmetric H, T I (I + 1) flops; peak: the measured dense bf16
+    figure."""
+    u = step.units[0]
+    Xs = [s[0][u.site][0] for s in step.sets]
+    T, I = Xs[0].shape
+    H = torch.empty((I, I), dtype=torch.float32, device=Xs[0].device)
+    flops = T * I * (I + 1)
+    tq.tq_hessian(Xs[0], out=H)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    tq.tq_hessian(Xs[0], out=H)
+    b.record()
+    torch.cuda.synchronize()
+    reps = max(3, min(50, int(0.03 / max(a.elapsed_time(b) * 1e-3, 1e-6))))
+    a.record()
+    for k in range(reps):
+        tq.tq_hessian(Xs[k % len(Xs)], out=H)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    # roofline: the slower of the tensor work and the HBM traffic (X read once, H written)
+    nbytes = T * I * 2 + I * I * 4
+    t_min = max(flops / (peak * 1e12), nbytes / (pk["hbm_gbs"] * 1e9))
+    return {"ms": ms, "T": T, "I": I, "flops": flops, "TFLOP/s": tf, "peak": peak, "frac_tensor": tf / peak,
+            "bytes": nbytes, "bound": "tensor" if flops / (peak * 1e12) >= nbytes / (pk["hbm_gbs"] * 1e9) else "hbm",
+            "frac": t_min / (ms * 1e-3),
+            "note": f"first unit's activations [{T}, {I}] bf16, {reps} launches over {len(Xs)} input sets; "
+                    "H fp32 both triangles; frac = roofline time (slower of flops / measured dense bf16 "
+                    "burst and bytes / measured HBM) / measured time"}
 
 
 def time_gemv(tq, step, pk, B, reps=20):

@@ -11,23 +11,28 @@
 //
 // As a GEMM: H[i][j] = sum_t X[t][i] X[t][j], M = N = I, K = T; both operands
 // are columns of row-major X, i.e. MN-major in memory, which the tensor core
-// reads directly (no transpose pass).  H is symmetric, so only tiles with
-// bi <= bj are computed and each value is written to both triangles (exactly
-// symmetric output).
+// reads directly (no transpose pass).  H is symmetric, so only tiles that
+// reach the upper triangle are computed, and each upper entry is written to
+// both triangles (exactly symmetric output).
 //
-// B200 mapping (one CTA per 128 x 128 tile of H, 4 warps, 2 CTAs per SM):
-//  * TMA (cp.async.bulk.tensor, 128-byte swizzle) brings 64-token slices of the
-//    two 128-column panels into a 3-stage shared-memory ring; a diagonal tile
-//    loads its single panel once.
+// B200 mapping (one CTA per 128 x 256 tile of H, 4 warps, 2 CTAs per SM, all
+// 512 TMEM columns in use):
+//  * TMA (cp.async.bulk.tensor, 128-byte swizzle) brings 32-token slices of the
+//    128-column A panel and the 256-column B panel into a 4-stage shared-memory
+//    ring (24 KB per stage); when the A panel is half of the B panel (tiles on
+//    the diagonal) only B is loaded and A is read from it.
 //  * One thread issues tcgen05.mma (kind::f16, bf16 in, fp32 accumulate,
-//    M = N = 128, K = 16, both operands MN-major from shared memory); the
-//    accumulator lives in 128 TMEM columns.  tcgen05.commit frees a stage when
-//    its MMAs have read it.
+//    M = 128, N = 256, K = 16, both operands MN-major from shared memory); the
+//    accumulator lives in 256 TMEM columns.  tcgen05.commit frees a stage when
+//    its MMAs have read it.  A 128 x 256 tile keeps the shared-memory traffic
+//    (TMA writes plus operand reads) under the bandwidth a 128 x 128 tile
+//    exceeds at the tensor cores' rate.
 //  * The 4 warps read the accumulator with tcgen05.ld (warp w: rows 32w..32w+31)
-//    and store it: each thread its row segment (contiguous) and, mirrored, a
-//    column segment (coalesced across the warp).
-//  * Tiles are grouped in 8 x 8 super-blocks so that the CTAs in flight share
-//    their panels in L2.
+//    into the (then free) ring, 128 columns at a time, padded so that row and
+//    column walks are conflict-free, and store the upper entries and their
+//    mirror images with coalesced rows.
+//  * Tiles are grouped in 1024 x 1024 super-blocks so that the CTAs in flight
+//    share their panels in L2.
 // Every wait on an mbarrier has an iteration limit; on timeout the kernel
 // records it (tq_sync reports it), drains its in-flight copies, frees TMEM and
 // returns.
@@ -40,14 +45,16 @@
 
 namespace tq {
 
-constexpr int HS_TILE = 128;      // tile of H (M = N)
-constexpr int HS_BK = 64;         // tokens per stage
-constexpr int HS_STAGES = 3;
+constexpr int HS_M = 128;         // tile rows (A panel: 128 columns of X)
+constexpr int HS_N = 256;         // tile columns (B panel: 256 columns of X)
+constexpr int HS_BK = 32;         // tokens per stage
+constexpr int HS_STAGES = 4;
 constexpr int HS_THREADS = 128;
-constexpr int HS_SUPER = 8;       // tiles per super-block side
-constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;           // one TMA box: 64 columns x 64 tokens, bf16
-constexpr int HS_OPERAND_BYTES = 2 * HS_BOX_BYTES;      // 128 columns
-constexpr int HS_STAGE_BYTES = 2 * HS_OPERAND_BYTES;    // A and B
+constexpr int HS_SUPER_M = 8, HS_SUPER_N = 4;         // a super-block: 1024 x 1024 of H
+constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;           // one TMA box: 64 columns x 32 tokens, bf16
+constexpr int HS_A_BYTES = (HS_M / 64) * HS_BOX_BYTES;
+constexpr int HS_B_BYTES = (HS_N / 64) * HS_BOX_BYTES;
+constexpr int HS_STAGE_BYTES = HS_A_BYTES + HS_B_BYTES;
 constexpr int HS_SMEM_BYTES = HS_STAGES * HS_STAGE_BYTES + 1024 /* alignment */ + 256 /* barriers */;
 constexpr unsigned HS_WAIT_LIMIT = 1u << 22;            // try_wait rounds before a wait is declared hung
 
@@ -92,8 +99,8 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 }
 
 // Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle, 64
-// elements (128 B) per row along M/N, rows = tokens.  LBO = bytes between the
-// two 64-column halves, SBO = bytes between groups of 8 token rows.
+// elements (128 B) per row along M/N, rows = tokens.  LBO = bytes between
+// consecutive 64-column boxes, SBO = bytes between groups of 8 token rows.
 __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
     constexpr uint64_t lbo = HS_BOX_BYTES >> 4, sbo = (8 * 128) >> 4;
     return (static_cast<uint64_t>((addr >> 4) & 0x3fffu)) | (lbo << 16) | (sbo << 32) | (1ull << 46) |
@@ -101,9 +108,9 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
 }
 
 // Instruction descriptor: kind::f16, fp32 accumulator, bf16 A and B, both
-// MN-major, N = M = 128.
+// MN-major, M = 128, N = 256.
 constexpr uint32_t HS_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                              (static_cast<uint32_t>(HS_TILE >> 3) << 17) | (static_cast<uint32_t>(HS_TILE >> 4) << 24);
+                              (static_cast<uint32_t>(HS_N >> 3) << 17) | (static_cast<uint32_t>(HS_M >> 4) << 24);
 
 __device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
     asm volatile(
@@ -140,28 +147,28 @@ struct HsArgs {
     float* H;
     float alpha;
     int accumulate;
-    int nb;                   // tiles per side
+    int nbm, nbn;             // 128-row and 256-column blocks
     int nsb;                  // super-blocks per side
 };
 
 __global__ void __launch_bounds__(HS_THREADS, 1)
 k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsArgs a) {
-    // the tile: super-block pair (BI <= BJ), then a tile inside it
-    int p = static_cast<int>(blockIdx.x) / (HS_SUPER * HS_SUPER);
-    const int local = static_cast<int>(blockIdx.x) % (HS_SUPER * HS_SUPER);
+    // the tile: super-block pair (BI <= BJ), then a 128 x 256 tile inside it
+    int p = static_cast<int>(blockIdx.x) / (HS_SUPER_M * HS_SUPER_N);
+    const int local = static_cast<int>(blockIdx.x) % (HS_SUPER_M * HS_SUPER_N);
     int BI = 0;
     while (p >= a.nsb - BI) { p -= a.nsb - BI; ++BI; }
     const int BJ = BI + p;
-    const int bi = BI * HS_SUPER + local / HS_SUPER, bj = BJ * HS_SUPER + local % HS_SUPER;
-    if (bi > bj || bj >= a.nb) return;   // lower triangle or past the edge: nothing to do
+    const int bi = BI * HS_SUPER_M + local / HS_SUPER_N, bj = BJ * HS_SUPER_N + local % HS_SUPER_N;
+    if (bi >= a.nbm || bj >= a.nbn || 2 * bj + 1 < bi) return;   // past the edge or below the diagonal
     const int e = static_cast<int>(blockIdx.y);
-    const bool diag = bi == bj;
+    const bool a_in_b = (bi >> 1) == bj;   // the A panel is half of the B panel: load B only
 
     extern __shared__ uint8_t hs_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hs_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + HS_STAGES * HS_STAGE_BYTES);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * HS_STAGES + 1);
-    int* progress = reinterpret_cast<int*>(tmem_slot + 1);   // [0] stages armed, [1] stages consumed, [2] ok
+    int* progress = reinterpret_cast<int*>(tmem_slot + 1);   // [0] armed, [1] consumed, [2] loops ok, [3] MMAs done
     const uint32_t s_base = smem_u32(smem);
     const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + HS_STAGES), done = smem_u32(bars + 2 * HS_STAGES);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,11 +183,12 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
         progress[0] = 0;
         progress[1] = 0;
         progress[2] = 1;
+        progress[3] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {   // the whole warp allocates 128 TMEM columns
+    if (warp == 0) {   // the whole warp allocates HS_N TMEM columns (128 lanes x 256 fp32)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
-                     "r"(HS_TILE));
+                     "r"(HS_N));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -189,7 +197,7 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
     const uint32_t tmem = *tmem_slot;
 
     if (warp == 0 && lane == 0) {   // TMA producer
-        const uint32_t bytes = diag ? HS_OPERAND_BYTES : HS_STAGE_BYTES;
+        const uint32_t bytes = a_in_b ? HS_B_BYTES : HS_STAGE_BYTES;
         int k = 0;
         for (; k < nk; ++k) {
             const int s = k % HS_STAGES;
@@ -197,12 +205,14 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
             const uint32_t st = s_base + s * HS_STAGE_BYTES, bar = full0 + 8 * s;
             mbar_expect_tx(bar, bytes);
             const int t0 = k * HS_BK;
-            tma_load_3d(st, &xmap, bar, bi * HS_TILE, t0, e);
-            tma_load_3d(st + HS_BOX_BYTES, &xmap, bar, bi * HS_TILE + 64, t0, e);
-            if (!diag) {
-                tma_load_3d(st + HS_OPERAND_BYTES, &xmap, bar, bj * HS_TILE, t0, e);
-                tma_load_3d(st + HS_OPERAND_BYTES + HS_BOX_BYTES, &xmap, bar, bj * HS_TILE + 64, t0, e);
+            if (!a_in_b) {
+#pragma unroll
+                for (int q = 0; q < HS_M / 64; ++q)
+                    tma_load_3d(st + q * HS_BOX_BYTES, &xmap, bar, bi * HS_M + 64 * q, t0, e);
             }
+#pragma unroll
+            for (int q = 0; q < HS_N / 64; ++q)
+                tma_load_3d(st + HS_A_BYTES + q * HS_BOX_BYTES, &xmap, bar, bj * HS_N + 64 * q, t0, e);
             progress[0] = k + 1;
         }
         if (k < nk) progress[2] = 0;
@@ -212,8 +222,8 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
             const int s = k % HS_STAGES;
             if (!mbar_wait(full0 + 8 * s, (k / HS_STAGES) & 1)) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t sa = s_base + s * HS_STAGE_BYTES;
-            const uint32_t sb = diag ? sa : sa + HS_OPERAND_BYTES;
+            const uint32_t sb = s_base + s * HS_STAGE_BYTES + HS_A_BYTES;
+            const uint32_t sa = a_in_b ? sb + (bi & 1) * (HS_M / 64) * HS_BOX_BYTES : s_base + s * HS_STAGE_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HS_BK / 16; ++kk)   // 16 tokens = 16 rows of 128 B per MMA
                 umma_bf16(tmem, umma_desc(sa + kk * 2048), umma_desc(sb + kk * 2048), (k | kk) != 0);
@@ -224,46 +234,54 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
         umma_commit(done);                 // every MMA issued so far is complete
     }
 
-    __syncwarp();   // lanes 1-31 of the producer and MMA warps wait here, not in a spin loop
-
-    // epilogue: warp w holds rows 32w .. 32w + 31 of the tile
-    const bool have = mbar_wait(done, 0);
+    // epilogue.  One thread waits for the MMAs; the others wait at the block
+    // barrier (no spinning).  The accumulator goes through shared memory (the
+    // ring is free once every MMA is complete), 128 columns at a time, so that
+    // the tile's upper-triangle entries and their mirror images are stored
+    // with coalesced rows; entries below the diagonal are left to their mirror.
+    if (warp == 1 && lane == 0) progress[3] = mbar_wait(done, 0) ? 1 : 0;
+    __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-    __syncwarp();
-    const bool ok = have && *reinterpret_cast<volatile int*>(&progress[2]) != 0;
-    const int m = warp * 32 + lane;
-    const int64_t gi = static_cast<int64_t>(bi) * HS_TILE + m;   // row of H this thread holds
+    const bool ok = progress[3] != 0 && progress[2] != 0;
+    constexpr int LDT = 128 + 1;   // padded rows: row and column walks are conflict-free
+    float* tile = reinterpret_cast<float*>(smem);
     float* He = a.H + static_cast<int64_t>(e) * a.hms;
+    const int64_t r0 = static_cast<int64_t>(bi) * HS_M;
 #pragma unroll 1
-    for (int c0 = 0; c0 < HS_TILE; c0 += 32) {
-        float v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
-        if (!ok) continue;
-        if (a.alpha != 1.0f) {
+    for (int h = 0; h < HS_N / 128; ++h) {
+        const int m = warp * 32 + lane;
+#pragma unroll 1
+        for (int cc = 0; cc < 128; cc += 32) {
+            float v[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(128 * h + cc), v);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(a.alpha, v[i]);
+            for (int i = 0; i < 32; ++i) tile[m * LDT + cc + i] = a.alpha != 1.0f ? __fmul_rn(a.alpha, v[i]) : v[i];
         }
-        const int64_t gj0 = static_cast<int64_t>(bj) * HS_TILE + c0;
-        // mirrored: H[gj][gi] (for fixed column, the warp's 32 rows are consecutive)
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const int64_t gj = gj0 + i;
-            if (gi < a.I && gj < a.I && (!diag || gj > gi)) {
-                float* q = He + gj * a.ldh + gi;
-                *q = a.accumulate ? __fadd_rn(*q, v[i]) : v[i];
+        __syncthreads();
+        const int64_t c0 = static_cast<int64_t>(bj) * HS_N + 128 * h;
+        if (ok && c0 + 127 >= r0) {
+#pragma unroll 4
+            for (int idx = threadIdx.x; idx < 128 * 128; idx += HS_THREADS) {   // H[r0 + r][c0 + c]
+                const int r = idx >> 7, c = idx & 127;
+                const int64_t gr = r0 + r, gc = c0 + c;
+                if (gr < a.I && gc < a.I && gc >= gr) {
+                    float* q = He + gr * a.ldh + gc;
+                    const float v = tile[r * LDT + c];
+                    *q = a.accumulate ? __fadd_rn(*q, v) : v;
+                }
             }
-        }
-        // direct: H[gi][gj], this thread's row segment
-        if (gi < a.I) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int64_t gj = gj0 + i;
-                if (gj < a.I && (!diag || gj >= gi)) {
-                    float* q = He + gi * a.ldh + gj;
-                    *q = a.accumulate ? __fadd_rn(*q, v[i]) : v[i];
+#pragma unroll 4
+            for (int idx = threadIdx.x; idx < 128 * 128; idx += HS_THREADS) {   // mirror: H[c0 + c][r0 + r]
+                const int c = idx >> 7, r = idx & 127;
+                const int64_t gr = r0 + r, gc = c0 + c;
+                if (gr < a.I && gc < a.I && gc > gr) {
+                    float* q = He + gc * a.ldh + gr;
+                    const float v = tile[r * LDT + c];
+                    *q = a.accumulate ? __fadd_rn(*q, v) : v;
                 }
             }
         }
+        __syncthreads();
     }
 
     // teardown: drain copies armed but not consumed, then free TMEM
@@ -274,7 +292,7 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
             if (!mbar_wait(full0 + 8 * (k % HS_STAGES), (k / HS_STAGES) & 1)) break;
     }
     if (warp == 0) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(HS_TILE));
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(HS_N));
     }
 }
 
@@ -340,12 +358,13 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
     HsArgs a;
     a.T = X->rows; a.I = X->cols; a.ldh = ldh; a.hms = X->n_mat > 1 ? h_mat_stride : 0;
     a.H = H; a.alpha = alpha; a.accumulate = accumulate ? 1 : 0;
-    a.nb = static_cast<int>((X->cols + HS_TILE - 1) / HS_TILE);
-    a.nsb = (a.nb + HS_SUPER - 1) / HS_SUPER;
+    a.nbm = static_cast<int>((X->cols + HS_M - 1) / HS_M);
+    a.nbn = static_cast<int>((X->cols + HS_N - 1) / HS_N);
+    a.nsb = static_cast<int>((X->cols + 1023) / 1024);
     static std::once_flag attr;
     std::call_once(attr, [] { cudaFuncSetAttribute(k_hessian, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM_BYTES); });
     const int64_t pairs = static_cast<int64_t>(a.nsb) * (a.nsb + 1) / 2;
-    const int64_t gx = pairs * HS_SUPER * HS_SUPER;
+    const int64_t gx = pairs * HS_SUPER_M * HS_SUPER_N;
     TQ_REQUIRE(gx < (int64_t(1) << 31), "tq_hessian: I too large");
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(X->n_mat));
     k_hessian<<<grid, HS_THREADS, HS_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, a);

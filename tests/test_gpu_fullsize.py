@@ -150,3 +150,34 @@ def _run_workload(name, n_rows=24, seed=0):
 def test_full_size_workload(name):
     results = _run_workload(name)
     assert results
+
+
+@pytest.mark.parametrize("name", ["c1", "c3"])
+def test_full_size_hessian(name):
+    """tq_hessian on the first unit's full calibration activations (c1: 2048 x
+    4096; c3: 65,536 tokens x 5120), launched as bench.py launches it: sampled
+    entries (the diagonal corners, tile edges, random) against the oracle one
+    by one within the fp32 accumulation bound, exact symmetry of the whole H,
+    and its diagonal against the imatrix of the same activations."""
+    wl = synth.make(name, DEV)
+    u = [x for x in wl.units if x.timed][0]
+    X = wl.sites[u.site].X[0]
+    T, I = X.shape
+    H = tq.tq_hessian(X)
+    tq.tq_sync()
+    assert torch.equal(H, H.T)
+    Xh = X.float().cpu().numpy()
+    Ah = np.abs(Xh)
+    rng = np.random.default_rng(7)
+    pairs = {(0, 0), (I - 1, I - 1), (0, I - 1), (127, 128), (128, 127), (I // 2, I // 3)}
+    while len(pairs) < 300:
+        pairs.add((int(rng.integers(I)), int(rng.integers(I))))
+    Hh = H.cpu().numpy()
+    for i, j in sorted(pairs):
+        ref = oracle.hessian_entry(Xh, i, j)
+        bound = (T / 16 + 32) * 2.0 ** -22 * oracle.hessian_entry(Ah, i, j)
+        assert abs(float(Hh[i, j]) - ref) <= bound, (i, j, float(Hh[i, j]), ref, bound)
+    m = tq.tq_imatrix(X)[0]
+    tq.tq_sync()
+    d = np.diag(Hh).astype(np.float64) / T
+    assert np.allclose(d, m.cpu().numpy().astype(np.float64), rtol=(T / 16 + 64) * 2.0 ** -22, atol=0)
