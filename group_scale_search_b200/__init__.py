@@ -29,17 +29,19 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = [
-    "INT3_G64_SYM", "INT4_G128_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
+    "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
+INT4_G64_ASYM = 6
 INT3_G64_SYM = 5
 NVFP4_G16 = 16
-FORMATS = {"int3_g64_sym": INT3_G64_SYM, "int4_g128_asym": INT4_G128_ASYM, "nvfp4_g16": NVFP4_G16}
-_GROUP = {INT3_G64_SYM: 64, INT4_G128_ASYM: 128, NVFP4_G16: 16}
+FORMATS = {"int3_g64_sym": INT3_G64_SYM, "int4_g128_asym": INT4_G128_ASYM, "int4_g64_asym": INT4_G64_ASYM,
+           "nvfp4_g16": NVFP4_G16}
+_GROUP = {INT3_G64_SYM: 64, INT4_G128_ASYM: 128, INT4_G64_ASYM: 64, NVFP4_G16: 16}
 _F32, _BF16 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -317,7 +319,8 @@ def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optiona
         out = SearchResult(
             fmt=fmt,
             scales=torch.empty((E, O, G), dtype=sdt, device=dev),
-            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt == INT4_G128_ASYM else None,
+            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt in (INT4_G128_ASYM, INT4_G64_ASYM)
+            else None,
             global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
             cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
             loss=torch.empty((E, O, G), dtype=torch.float64, device=dev) if want_loss else None,

@@ -167,12 +167,12 @@ struct GvRows {
             c = packed + g0 * rec + static_cast<int64_t>(q) * 16;
         }
         s = static_cast<const uint8_t*>(scales) + (g0 + qg) * (FMT == TQ_NVFP4_G16 ? 1 : 4);
-        z = FMT == TQ_INT4_G128_ASYM ? zeros + g0 + qg : nullptr;
+        z = is_int4(FMT) ? zeros + g0 + qg : nullptr;
     }
     __device__ __forceinline__ Quad load(int r, float g) const {
         Quad u;
         const uint8_t* cr = c + cof[r];
-        if constexpr (FMT == TQ_INT4_G128_ASYM) {
+        if constexpr (is_int4(FMT)) {
             const uint4 v = __ldg(reinterpret_cast<const uint4*>(cr));
             u.w[0] = v.x; u.w[1] = v.y; u.w[2] = v.z; u.w[3] = v.w;
             u.s0 = __ldg(reinterpret_cast<const float*>(s) + gof[r]);
@@ -204,8 +204,9 @@ struct GvRows {
         return u;
     }
     __device__ __forceinline__ void next(int dq) {
-        if constexpr (FMT == TQ_INT4_G128_ASYM) {
-            c += 16 * dq; s += dq; z += dq >> 2;
+        if constexpr (is_int4(FMT)) {   // dq quads = dq * 32 / group groups
+            constexpr int qpg = FmtTraits<FMT>::group / 32;
+            c += 16 * dq; s += 4 * (dq / qpg); z += dq / qpg;
         } else if constexpr (FMT == TQ_INT3_G64_SYM) {
             c += 12 * dq; s += 2 * dq;
         } else {
@@ -503,7 +504,7 @@ TQ_API tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void*
     TQ_REQUIRE(B >= 1 && B <= 8, "tq_dequant_gemv: B must be in [1, 8]");
     TQ_REQUIRE(x_mat_stride == 0 || x_mat_stride >= B * I, "tq_dequant_gemv: x_mat_stride must be 0 or >= B*I");
     TQ_REQUIRE(aligned16(packed) && aligned16(x), "tq_dequant_gemv: packed/x not 16-byte aligned");
-    TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_dequant_gemv: int4 needs zeros");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_dequant_gemv: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant_gemv: NVFP4 needs global_scale");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t xms = n_mat > 1 ? x_mat_stride : 0;
@@ -512,6 +513,8 @@ TQ_API tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void*
         launch_gemv_b<TQ_INT3_G64_SYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else if (fmt == TQ_INT4_G128_ASYM) {
         launch_gemv_b<TQ_INT4_G128_ASYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
+    } else if (fmt == TQ_INT4_G64_ASYM) {
+        launch_gemv_b<TQ_INT4_G64_ASYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else if (((I + 15) / 16) % 2 == 0 && (reinterpret_cast<uintptr_t>(scales) & 1u) == 0) {
         launch_gemv_b<TQ_NVFP4_G16, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else {

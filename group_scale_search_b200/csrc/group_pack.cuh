@@ -31,9 +31,14 @@ __device__ __forceinline__ void pack_int3_record(unsigned u0, unsigned u1, int l
 
 // int4-g128 record: 64 bytes, element 2k in the low nibble of byte k.  Lane l
 // holds elements 4l..4l+3 and stores bytes 2l, 2l+1.
-__device__ __forceinline__ void pack_int4_lane(const unsigned q[4], int lane, uint8_t* rec) {
-    const unsigned v = (q[0] & 15u) | ((q[1] & 15u) << 4) | ((q[2] & 15u) << 8) | ((q[3] & 15u) << 12);
-    reinterpret_cast<uint16_t*>(rec)[lane] = static_cast<uint16_t>(v);
+template <int EPL>
+__device__ __forceinline__ void pack_int4_lane(const unsigned q[EPL], int lane, uint8_t* rec) {
+    if constexpr (EPL == 4) {
+        const unsigned v = (q[0] & 15u) | ((q[1] & 15u) << 4) | ((q[2] & 15u) << 8) | ((q[3] & 15u) << 12);
+        reinterpret_cast<uint16_t*>(rec)[lane] = static_cast<uint16_t>(v);
+    } else {
+        rec[lane] = static_cast<uint8_t>((q[0] & 15u) | ((q[1] & 15u) << 4));
+    }
 }
 
 // NVFP4 codes of N (8 or 16) weights under block scale S = fl32(g dec(e)):

@@ -106,7 +106,7 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
                     sc[h] = __fmul_rn(g, e4m3_value(__ldg(bp + h * G)));
                 } else {
                     sc[h] = __ldg(sp + h * G);
-                    if constexpr (FMT == TQ_INT4_G128_ASYM) zc[h] = __ldg(zp + h * G);
+                    if constexpr (is_int4(FMT)) zc[h] = __ldg(zp + h * G);
                 }
             }
             cur.next();
@@ -119,7 +119,7 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
         rec += ROWS * rstride;
         sp += ROWS * G;
         bp += ROWS * G;
-        if (FMT == TQ_INT4_G128_ASYM) zp += ROWS * G;
+        if (is_int4(FMT)) zp += ROWS * G;
     }
 }
 
@@ -128,7 +128,7 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
 // One thread per group record; codes are dense [rows][cols] bytes.
 __global__ void k_pack_codes(const uint8_t* __restrict__ codes, int fmt, int64_t rows, int64_t cols,
                              const uint8_t* __restrict__ zeros, uint8_t* __restrict__ packed) {
-    const int g = fmt == TQ_INT3_G64_SYM ? 64 : (fmt == TQ_INT4_G128_ASYM ? 128 : 16);
+    const int g = fmt == TQ_INT3_G64_SYM ? 64 : (fmt == TQ_INT4_G128_ASYM ? 128 : (fmt == TQ_INT4_G64_ASYM ? 64 : 16));
     const int64_t G = (cols + g - 1) / g;
     const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gid >= rows * G) return;
@@ -146,7 +146,7 @@ __global__ void k_pack_codes(const uint8_t* __restrict__ codes, int fmt, int64_t
         uint32_t* rec = reinterpret_cast<uint32_t*>(packed + gid * 24);
         rec[0] = lo[0]; rec[1] = lo[1]; rec[2] = lo[2]; rec[3] = lo[3]; rec[4] = hi[0]; rec[5] = hi[1];
     } else {
-        const unsigned pad = (fmt == TQ_INT4_G128_ASYM && zeros) ? (zeros[gid] & 15u) : 0u;
+        const unsigned pad = (is_int4(fmt) && zeros) ? (zeros[gid] & 15u) : 0u;
         uint32_t* rec = reinterpret_cast<uint32_t*>(packed + gid * (g / 2));
         for (int wd = 0; wd < g / 8; ++wd) {
             uint32_t v = 0u;
@@ -172,7 +172,7 @@ __global__ void k_unpack_codes(const uint8_t* __restrict__ packed, int fmt, int6
         const unsigned u = ((rec[i >> 2] >> (2 * (i & 3))) & 3u) | (((rec[16 + (i >> 3)] >> (i & 7)) & 1u) << 2);
         codes[idx] = static_cast<uint8_t>(static_cast<int8_t>(static_cast<int>(u) - 4));
     } else {
-        const int g = fmt == TQ_INT4_G128_ASYM ? 128 : 16;
+        const int g = fmt == TQ_INT4_G128_ASYM ? 128 : (fmt == TQ_INT4_G64_ASYM ? 64 : 16);
         const int64_t G = (cols + g - 1) / g;
         const uint8_t b = packed[(r * G + j / g) * (g / 2) + (j % g) / 2];
         codes[idx] = (j & 1) ? static_cast<uint8_t>(b >> 4) : static_cast<uint8_t>(b & 15u);
@@ -316,7 +316,7 @@ TQ_API tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const
     if ((s = check_fmt(fmt, "tq_pack")) != TQ_OK) return s;
     TQ_REQUIRE(scales != nullptr && packed != nullptr, "tq_pack: null scales or packed");
     TQ_REQUIRE(aligned16(packed), "tq_pack: packed not 16-byte aligned");
-    TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_pack: int4 needs zeros");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_pack: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_pack: NVFP4 needs global_scale");
     TQ_REQUIRE(W->n_mat <= 65535, "tq_pack: more than 65535 matrices in one call");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -326,6 +326,8 @@ TQ_API tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const
                                    : launch_pack<TQ_INT3_G64_SYM, float>(W, ms, scales, zeros, global_scale, packed, st);
     else if (fmt == TQ_INT4_G128_ASYM) bf ? launch_pack<TQ_INT4_G128_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
                                           : launch_pack<TQ_INT4_G128_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
+    else if (fmt == TQ_INT4_G64_ASYM) bf ? launch_pack<TQ_INT4_G64_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
+                                         : launch_pack<TQ_INT4_G64_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
     else bf ? launch_pack<TQ_NVFP4_G16, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
             : launch_pack<TQ_NVFP4_G16, float>(W, ms, scales, zeros, global_scale, packed, st);
     return check_launch("tq_pack");
@@ -367,7 +369,7 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     TQ_REQUIRE(packed && scales && out, "tq_dequant: null pointer");
     TQ_REQUIRE(n_mat >= 1 && O >= 1 && I >= 1, "tq_dequant: empty shape");
     TQ_REQUIRE(aligned16(packed) && aligned16(out), "tq_dequant: packed/out not 16-byte aligned");
-    TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_dequant: int4 needs zeros");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_dequant: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant: NVFP4 needs global_scale");
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant: out dtype %d", out_dtype);
     TQ_REQUIRE(n_mat <= 65535, "tq_dequant: more than 65535 matrices in one call");
@@ -379,6 +381,9 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     else if (fmt == TQ_INT4_G128_ASYM)
         bf ? launch_dequant<TQ_INT4_G128_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
            : launch_dequant<TQ_INT4_G128_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G64_ASYM)
+        bf ? launch_dequant<TQ_INT4_G64_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G64_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
     else
         bf ? launch_dequant<TQ_NVFP4_G16, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
            : launch_dequant<TQ_NVFP4_G16, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);

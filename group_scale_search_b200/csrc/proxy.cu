@@ -217,7 +217,7 @@ TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t 
     TQ_REQUIRE(aligned16(packed) && aligned16(m), "tq_proxy_error: packed/m not 16-byte aligned");
     TQ_REQUIRE(W->n_mat == 1 || m_stride == 0 || (m_stride >= W->cols && m_stride % 4 == 0),
                "tq_proxy_error: m_stride must be 0 or a multiple of 4 >= cols");
-    TQ_REQUIRE(fmt != TQ_INT4_G128_ASYM || zeros != nullptr, "tq_proxy_error: int4 needs zeros");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_proxy_error: int4 needs zeros");
     TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_proxy_error: NVFP4 needs global_scale");
     TQ_REQUIRE(workspace && aligned16(workspace), "tq_proxy_error: workspace null or not 16-byte aligned");
     const size_t need = tq_proxy_workspace_bytes(W, fmt);
@@ -238,6 +238,9 @@ TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t 
     else if (fmt == TQ_INT4_G128_ASYM)
         bf ? launch_proxy<TQ_INT4_G128_ASYM, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
            : launch_proxy<TQ_INT4_G128_ASYM, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);
+    else if (fmt == TQ_INT4_G64_ASYM)
+        bf ? launch_proxy<TQ_INT4_G64_ASYM, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
+           : launch_proxy<TQ_INT4_G64_ASYM, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);
     else
         bf ? launch_proxy<TQ_NVFP4_G16, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
            : launch_proxy<TQ_NVFP4_G16, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);

@@ -5,7 +5,7 @@
 namespace tq {
 tq_status launch_search_int3(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
                              float* scales, int32_t* idx, double* loss, uint8_t* packed, cudaStream_t st);
-tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
+tq_status launch_search_int4(const tq_mat* W, int gsize, const float* m, int64_t m_stride, const tq_search_params* p,
                              float* scales, uint8_t* zeros, int32_t* idx, double* loss, uint8_t* packed,
                              cudaStream_t st);
 tq_status launch_search_nvfp4(const tq_mat* W, const float* m, int64_t m_stride, const tq_search_params* p,
@@ -28,7 +28,7 @@ TQ_API tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_str
                "tq_search_groups: m_stride must be 0 or a multiple of 4 >= cols");
     TQ_REQUIRE(scales != nullptr, "tq_search_groups: null scales");
     TQ_REQUIRE(packed == nullptr || aligned16(packed), "tq_search_groups: packed not 16-byte aligned");
-    TQ_REQUIRE((fmt == TQ_INT4_G128_ASYM) == (zeros != nullptr),
+    TQ_REQUIRE(is_int4(fmt) == (zeros != nullptr),
                "tq_search_groups: zeros required for int4 and only for int4");
     TQ_REQUIRE((fmt == TQ_NVFP4_G16) == (global_scale != nullptr),
                "tq_search_groups: global_scale required for NVFP4 and only for NVFP4");
@@ -38,8 +38,9 @@ TQ_API tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_str
     const int64_t mst = W->n_mat > 1 ? m_stride : 0;
     if (fmt == TQ_INT3_G64_SYM)
         return launch_search_int3(W, m, mst, params, static_cast<float*>(scales), cand_idx, loss, packed, st);
-    if (fmt == TQ_INT4_G128_ASYM)
-        return launch_search_int4(W, m, mst, params, static_cast<float*>(scales), zeros, cand_idx, loss, packed, st);
+    if (is_int4(fmt))
+        return launch_search_int4(W, static_cast<int>(group_of(fmt)), m, mst, params, static_cast<float*>(scales),
+                                  zeros, cand_idx, loss, packed, st);
     return launch_search_nvfp4(W, m, mst, params, static_cast<uint8_t*>(scales), global_scale, cand_idx, loss,
                                packed, st);
 }

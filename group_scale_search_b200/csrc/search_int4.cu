@@ -8,6 +8,10 @@
 //   z_i = rint(15 i / (nz - 1)); q = clamp(rint(w/s) + z, 0, 15);
 //   L = sum_j m_j (w_j - s (q_j - z))^2; ties keep the lowest index nz k + i.
 //
+// The same search runs on 64-weight groups (int4-g64: the page "int3-g64
+// (fmt=5)"'s per-projection ablation table lists an int4-g64 scheme, and its
+// thread the grouped int4 format fmt=4): lanes then hold 2 weights each.
+//
 // B200 mapping: one warp per 128-weight group; lane l owns scales l and l+32
 // (and 64 p + l, 64 p + 32 + l in pass p of a grid of more than 64 scales:
 // the "256/64" end of the page's quality ladder, results bullet 2) and all 16
@@ -72,6 +76,21 @@ template <> struct Load4<float> {
     }
 };
 
+// Lane l holds elements 2l, 2l+1 of a 64-weight group.
+template <typename T> struct Load2;
+template <> struct Load2<uint16_t> {
+    static __device__ __forceinline__ void go(const uint16_t* p, float w[2]) {
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(p));
+        w[0] = __uint_as_float(v << 16); w[1] = __uint_as_float(v & 0xffff0000u);
+    }
+};
+template <> struct Load2<float> {
+    static __device__ __forceinline__ void go(const float* p, float w[2]) {
+        const float2 v = __ldg(reinterpret_cast<const float2*>(p));
+        w[0] = v.x; w[1] = v.y;
+    }
+};
+
 __device__ __forceinline__ unsigned ord_key(float x) {   // order-preserving float -> uint
     const unsigned b = __float_as_uint(x);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -80,10 +99,11 @@ __device__ __forceinline__ float ord_val(unsigned k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-__device__ __forceinline__ double loss64_int4(const float w[4], const float m[4], float s, int z) {
+template <int EPL>
+__device__ __forceinline__ double loss64_int4(const float w[EPL], const float m[EPL], float s, int z) {
     double t = 0.0;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < EPL; ++i) {
         const float q = (s == 0.f) ? static_cast<float>(z)
                                    : fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], s)), static_cast<float>(z)), 0.f), 15.f);
         const double e = __dsub_rn(static_cast<double>(w[i]),
@@ -117,12 +137,13 @@ __device__ __forceinline__ void acc_scale(float w, float sm, float s, float inv,
     }
 }
 
-template <typename T, int NP>
+template <typename T, int NP, int GS>
 __global__ void __launch_bounds__(ASYM_WARPS * 32)
 k_search_int4(const __grid_constant__ AsymArgs a) {
-    __shared__ __align__(16) float2 lists[ASYM_WARPS][132];   // two sign lists, each padded to even length
+    constexpr int EPL = GS / 32;   // elements per lane: 4 (g128) or 2 (g64)
+    __shared__ __align__(16) float2 lists[ASYM_WARPS][GS + 4];   // two sign lists, each padded to even length
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int64_t G = (a.I + 127) >> 7;
+    const int64_t G = (a.I + GS - 1) / GS;
     const int64_t OG = a.O * G;
     const int64_t total = a.n_mat * OG;
     const T* W = static_cast<const T*>(a.W);
@@ -134,22 +155,28 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         uint32_t e32, o32, k32;
         a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
         const int64_t e = e32, o = o32, k = k32;
-        const int64_t j0 = k << 7;
-        const int n = static_cast<int>(min(static_cast<int64_t>(128), a.I - j0));
+        const int64_t j0 = k * GS;
+        const int n = static_cast<int>(min(static_cast<int64_t>(GS), a.I - j0));
         const T* wp = W + e * a.ms + o * a.ld + j0;
         const float* mp = a.m + e * a.m_stride + j0;
-        float w[4], mv[4];
-        bool val[4];
-        if (n == 128) {
-            Load4<T>::go(wp + 4 * lane, w);
-            const float4 mm = __ldg(reinterpret_cast<const float4*>(mp + 4 * lane));
-            mv[0] = mm.x; mv[1] = mm.y; mv[2] = mm.z; mv[3] = mm.w;
+        float w[EPL], mv[EPL];
+        bool val[EPL];
+        if (n == GS) {
+            if constexpr (EPL == 4) {
+                Load4<T>::go(wp + 4 * lane, w);
+                const float4 mm = __ldg(reinterpret_cast<const float4*>(mp + 4 * lane));
+                mv[0] = mm.x; mv[1] = mm.y; mv[2] = mm.z; mv[3] = mm.w;
+            } else {
+                Load2<T>::go(wp + 2 * lane, w);
+                const float2 mm = __ldg(reinterpret_cast<const float2*>(mp + 2 * lane));
+                mv[0] = mm.x; mv[1] = mm.y;
+            }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) val[i] = true;
+            for (int i = 0; i < EPL; ++i) val[i] = true;
         } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int j = 4 * lane + i;
+            for (int i = 0; i < EPL; ++i) {
+                const int j = EPL * lane + i;
                 val[i] = j < n;
                 w[i] = val[i] ? Elem<T>::load(wp + j) : 0.f;
                 mv[i] = val[i] ? __ldg(mp + j) : 0.f;
@@ -157,12 +184,12 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         }
         unsigned kmin = 0xffffffffu, kmax = 0u;
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < EPL; ++i)
             if (val[i]) { kmin = min(kmin, ord_key(w[i])); kmax = max(kmax, ord_key(w[i])); }
         const float wmin = ord_val(__reduce_min_sync(FULL, kmin));
         const float wmax = ord_val(__reduce_max_sync(FULL, kmax));
         float R = __fsub_rn(wmax, wmin);
-        uint8_t* rec = a.packed ? a.packed + gid * 64 : nullptr;
+        uint8_t* rec = a.packed ? a.packed + gid * (GS / 2) : nullptr;
         if (R == 0.f) {
             if (wmax == 0.f) {   // all-zero group: s = 0, z = 0, q = 0
                 if (lane == 0) {
@@ -170,7 +197,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                     if (a.idx) a.idx[gid] = -1;
                     if (a.loss) a.loss[gid] = 0.0;
                 }
-                if (rec) { const unsigned q0[4] = {0u, 0u, 0u, 0u}; pack_int4_lane(q0, lane, rec); }
+                if (rec) { const unsigned q0[EPL] = {}; pack_int4_lane<EPL>(q0, lane, rec); }
                 continue;
             }
             R = fabsf(wmax);
@@ -180,24 +207,24 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
         const float pw = pow2_inv_binade(fmaxf(fabsf(wmin), fabsf(wmax)));
         float mloc = 0.f;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) mloc = fmaxf(mloc, fabsf(mv[i]));
+        for (int i = 0; i < EPL; ++i) mloc = fmaxf(mloc, fabsf(mv[i]));
         const float mmax = __uint_as_float(__reduce_max_sync(FULL, __float_as_uint(mloc)));
         const float pm = mmax > 0.f ? pow2_inv_binade(mmax) : 1.f;
         const double back = inv_pow2_sq(pw, pm);
         const float Rs = __fmul_rn(R, pw);
         // split by sign: negative weights first, non-negative after (tail: (0, 0))
-        float x[4], sq[4];
-        bool neg[4];
+        float x[EPL], sq[EPL];
+        bool neg[EPL];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < EPL; ++i) {
             x[i] = __fmul_rn(w[i], pw);
             sq[i] = sqrtf(__fmul_rn(mv[i], pm));
             neg[i] = val[i] && x[i] < 0.f;
         }
-        unsigned bn[4];
+        unsigned bn[EPL];
         int nneg = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) { bn[i] = __ballot_sync(FULL, neg[i]); nneg += __popc(bn[i]); }
+        for (int i = 0; i < EPL; ++i) { bn[i] = __ballot_sync(FULL, neg[i]); nneg += __popc(bn[i]); }
         const int npos_real = n - nneg;
         const int nneg_pad = (nneg + 1) & ~1;
         const int npos_pad = (npos_real + 1) & ~1;
@@ -206,7 +233,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             int before_n = 0, before_p = 0;
             const unsigned lt = (1u << lane) - 1u;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < EPL; ++i) {
                 const unsigned bp = __ballot_sync(FULL, val[i] && !neg[i]);
                 if (neg[i]) list[before_n + __popc(bn[i] & lt)] = make_float2(x[i], sq[i]);
                 else if (val[i]) list[nneg_pad + before_p + __popc(bp & lt)] = make_float2(x[i], sq[i]);
@@ -305,7 +332,7 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                         while (zm) {
                             const int z = __ffs(zm) - 1;
                             zm &= zm - 1;
-                            const double Ld = loss64_int4(w, mv, sc, z);
+                            const double Ld = loss64_int4<EPL>(w, mv, sc, z);
                             if (Ld < best) { best = Ld; bidx = a.nz * k + a.zfirst[z]; }
                         }
                     }
@@ -326,31 +353,31 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
             if (a.loss) a.loss[gid] = lossd;
         }
         if (rec) {
-            unsigned q[4];
+            unsigned q[EPL];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
+            for (int i = 0; i < EPL; ++i) {
                 const float qq = (sfin == 0.f || !val[i]) ? static_cast<float>(zb)
                     : fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w[i], sfin)), static_cast<float>(zb)), 0.f), 15.f);
                 q[i] = static_cast<unsigned>(qq);
             }
-            pack_int4_lane(q, lane, rec);
+            pack_int4_lane<EPL>(q, lane, rec);
         }
     }
 }
 
-template <int NP>
+template <int NP, int GS>
 void launch_int4(const AsymArgs& a, bool bf16, int64_t total, cudaStream_t st) {
     int bpsm = 0;
-    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t, NP>, ASYM_WARPS * 32, 0);
-    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<float, NP>, ASYM_WARPS * 32, 0);
+    if (bf16) cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<uint16_t, NP, GS>, ASYM_WARPS * 32, 0);
+    else cudaOccupancyMaxActiveBlocksPerMultiprocessor(&bpsm, k_search_int4<float, NP, GS>, ASYM_WARPS * 32, 0);
     if (bpsm < 1) bpsm = 1;
     const int64_t need = (total + ASYM_WARPS - 1) / ASYM_WARPS;
     const int grid = static_cast<int>(min(need, static_cast<int64_t>(num_sms()) * bpsm));
-    if (bf16) k_search_int4<uint16_t, NP><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
-    else k_search_int4<float, NP><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    if (bf16) k_search_int4<uint16_t, NP, GS><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
+    else k_search_int4<float, NP, GS><<<grid, ASYM_WARPS * 32, 0, st>>>(a);
 }
 
-tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
+tq_status launch_search_int4(const tq_mat* W, int gsize, const float* m, int64_t m_stride,
                              const tq_search_params* p, float* scales, uint8_t* zeros, int32_t* idx,
                              double* loss, uint8_t* packed, cudaStream_t st) {
     if (p->asym_n_scale < 2 || p->asym_n_scale > 256)
@@ -382,13 +409,18 @@ tq_status launch_search_int4(const tq_mat* W, const float* m, int64_t m_stride,
     for (int z = 0; z < 16; ++z)
         if (a.zfirst[z] < 0) return set_error(TQ_ERR_UNSUPPORTED, "int4 search: zero-point %d not on the grid", z);
 
-    const int64_t G = (W->cols + 127) / 128;
+    const int64_t G = (W->cols + gsize - 1) / gsize;
     const int64_t total = W->n_mat * W->rows * G;
     if (total >= (int64_t(1) << 32)) return set_error(TQ_ERR_UNSUPPORTED, "int4 search: more than 2^32 groups");
     a.gi = GroupIndex(W->rows, G);
     const bool bf16 = W->dtype == TQ_BF16;
-    if (a.ns <= 64) launch_int4<1>(a, bf16, total, st);
-    else launch_int4<4>(a, bf16, total, st);
+    if (gsize == 128) {
+        if (a.ns <= 64) launch_int4<1, 128>(a, bf16, total, st);
+        else launch_int4<4, 128>(a, bf16, total, st);
+    } else {
+        if (a.ns <= 64) launch_int4<1, 64>(a, bf16, total, st);
+        else launch_int4<4, 64>(a, bf16, total, st);
+    }
     return check_launch("int4 search");
 }
 

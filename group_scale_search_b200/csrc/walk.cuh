@@ -19,6 +19,7 @@ namespace tq {
 template <int FMT> struct FmtTraits;
 template <> struct FmtTraits<TQ_INT3_G64_SYM> { static constexpr int lg = 3, group = 64, rec = 24; };
 template <> struct FmtTraits<TQ_INT4_G128_ASYM> { static constexpr int lg = 4, group = 128, rec = 64; };
+template <> struct FmtTraits<TQ_INT4_G64_ASYM> { static constexpr int lg = 3, group = 64, rec = 32; };
 template <> struct FmtTraits<TQ_NVFP4_G16> { static constexpr int lg = 1, group = 16, rec = 8; };
 
 // ------------------------------------------------------------------ host geometry
@@ -147,7 +148,7 @@ struct QPtr {
         rec += G * FmtTraits<FMT>::rec;
         sc = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(sc) + G)
                                  : static_cast<const void*>(static_cast<const float*>(sc) + G);
-        if (FMT == TQ_INT4_G128_ASYM) zp += G;
+        if (is_int4(FMT)) zp += G;
     }
 };
 
@@ -184,7 +185,7 @@ __device__ __forceinline__ OctQ load_q(const QPtr<FMT>& q, int oct) {
         o.bits = int3_nibbles(__ldg(reinterpret_cast<const uint16_t*>(q.rec) + oct), __ldg(q.rec + 16 + oct));
         o.s = __ldg(static_cast<const float*>(q.sc));
         o.z = 4;
-    } else if constexpr (FMT == TQ_INT4_G128_ASYM) {
+    } else if constexpr (is_int4(FMT)) {
         o.bits = __ldg(reinterpret_cast<const uint32_t*>(q.rec) + oct);
         o.s = __ldg(static_cast<const float*>(q.sc));
         o.z = __ldg(q.zp);
@@ -223,7 +224,7 @@ __device__ __forceinline__ UnitQ<NO> load_unit_q(const QPtr<FMT>& q, int oct) {
     } else {
         const uint2 v = __ldg(reinterpret_cast<const uint2*>(q.rec + (FMT == TQ_NVFP4_G16 ? 0 : 4 * oct)));
         u.bits[0] = v.x; u.bits[1] = v.y;
-        if constexpr (FMT == TQ_INT4_G128_ASYM) {
+        if constexpr (is_int4(FMT)) {
             u.s = __ldg(static_cast<const float*>(q.sc));
             u.z = __ldg(q.zp);
         } else {

@@ -63,6 +63,7 @@ typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 typedef enum {
     TQ_INT4_G128_ASYM = 4,   /* nibble codes q in [0,15], f32 scale, u8 zero per 128 weights */
     TQ_INT3_G64_SYM = 5,     /* two bit-planes, v in [-4,3] as v+4, f32 scale per 64 weights  */
+    TQ_INT4_G64_ASYM = 6,    /* as TQ_INT4_G128_ASYM with 64 weights per group (32-byte records) */
     TQ_NVFP4_G16 = 16        /* E2M1 codes, E4M3 scale byte per 16 weights, f32 global scale   */
 } tq_format;
 

@@ -66,23 +66,23 @@ def lib():
             "orc_search_sym_int3": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, i32, f64, f64,
                                            P, P, P, P]),
             "orc_search_asym_int4": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, i32, f64, f64,
-                                            P, P, P, P, P]),
+                                            P, P, P, P, P, i32]),
             "orc_search_nvfp4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, i32, P, P, P, P]),
             "orc_rtn_int3": (None, [P, i64, i64, P, P]),
-            "orc_rtn_int4": (None, [P, i64, i64, P, P, P]),
+            "orc_rtn_int4": (None, [P, i64, i64, P, P, P, i32]),
             "orc_rtn_nvfp4": (None, [P, i64, i64, i64, P, P, P]),
             "orc_pack_int3": (None, [P, i64, i64, P]),
             "orc_unpack_int3": (None, [P, i64, i64, P]),
             "orc_pack_nibbles": (None, [P, i64, i64, i32, P, P]),
             "orc_unpack_nibbles": (None, [P, i64, i64, i32, P]),
             "orc_dequant_int3": (None, [P, i64, i64, P, P]),
-            "orc_dequant_int4": (None, [P, i64, i64, P, P, P]),
+            "orc_dequant_int4": (None, [P, i64, i64, P, P, P, i32]),
             "orc_dequant_nvfp4": (None, [P, i64, i64, i64, P, P, P]),
             "orc_proxy_error": (None, [P, P, i64, i64, P, P, P]),
             "orc_rowwise_int4": (None, [P, i64, i64, P]),
             "orc_num_threads": (i32, []),
             "orc_loss_given_int3": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P]),
-            "orc_loss_given_int4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P, P]),
+            "orc_loss_given_int4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P, P, i32]),
             "orc_loss_given_nvfp4": (None, [P, i64, i64, i64, i64, i64, P, i64, P, P, P]),
         }
         for name, (res, args) in sig.items():
@@ -179,21 +179,21 @@ def search_sym_int3(W, m, n1=32, n2=32, lo=0.5, hi=1.2, codes=True):
     return scales, idx, loss, v
 
 
-def search_asym_int4(W, m, ns=64, nz=32, lo=0.5, hi=1.2, codes=True):
+def search_asym_int4(W, m, ns=64, nz=32, lo=0.5, hi=1.2, codes=True, g=128):
     W = _f32(W)
     if W.ndim == 2:
         W = W[None]
     E, O, I = W.shape
     m = _f32(m)
     ms = I if m.ndim == 2 else 0
-    G = (I + 127) // 128
+    G = (I + g - 1) // g
     scales = np.empty((E, O, G), np.float32)
     zeros = np.empty((E, O, G), np.uint8)
     idx = np.empty((E, O, G), np.int32)
     loss = np.empty((E, O, G), np.float64)
     q = np.empty((E, O, I), np.uint8) if codes else None
     lib().orc_search_asym_int4(_p(W), E, O, I, I, O * I, _p(m), ms, ns, nz, lo, hi,
-                               _p(scales), _p(zeros), _p(idx), _p(loss), _p(q))
+                               _p(scales), _p(zeros), _p(idx), _p(loss), _p(q), g)
     return scales, zeros, idx, loss, q
 
 
@@ -306,10 +306,10 @@ def rtn_int3(W, scales):
     return v
 
 
-def rtn_int4(W, scales, zeros):
+def rtn_int4(W, scales, zeros, g=128):
     W = _f32(W); I = W.shape[-1]; rows = W.size // I
     q = np.empty(W.shape, np.uint8)
-    lib().orc_rtn_int4(_p(W), rows, I, _p(_f32(scales)), _p(np.ascontiguousarray(zeros, np.uint8)), _p(q))
+    lib().orc_rtn_int4(_p(W), rows, I, _p(_f32(scales)), _p(np.ascontiguousarray(zeros, np.uint8)), _p(q), g)
     return q
 
 
@@ -362,10 +362,10 @@ def dequant_int3(v, scales) -> np.ndarray:
     return out
 
 
-def dequant_int4(q, scales, zeros) -> np.ndarray:
+def dequant_int4(q, scales, zeros, g=128) -> np.ndarray:
     q = np.ascontiguousarray(q, np.uint8); I = q.shape[-1]; rows = q.size // I
     out = np.empty(q.shape, np.float32)
-    lib().orc_dequant_int4(_p(q), rows, I, _p(_f32(scales)), _p(np.ascontiguousarray(zeros, np.uint8)), _p(out))
+    lib().orc_dequant_int4(_p(q), rows, I, _p(_f32(scales)), _p(np.ascontiguousarray(zeros, np.uint8)), _p(out), g)
     return out
 
 
@@ -413,11 +413,11 @@ def loss_given_int3(W, m, scales) -> np.ndarray:
     return out
 
 
-def loss_given_int4(W, m, scales, zeros) -> np.ndarray:
+def loss_given_int4(W, m, scales, zeros, g=128) -> np.ndarray:
     W, m, E, O, I, ms = _batch(W, m)
-    out = np.empty((E, O, (I + 127) // 128), np.float64)
+    out = np.empty((E, O, (I + g - 1) // g), np.float64)
     lib().orc_loss_given_int4(_p(W), E, O, I, I, O * I, _p(m), ms, _p(_f32(scales)),
-                              _p(np.ascontiguousarray(zeros, np.uint8)), _p(out))
+                              _p(np.ascontiguousarray(zeros, np.uint8)), _p(out), g)
     return out
 
 

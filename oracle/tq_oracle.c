@@ -428,16 +428,19 @@ ORC_API void orc_search_sym_int3(const float* W, int64_t n_mat, int64_t O, int64
     }
 }
 
+/* g: weights per group, 128 (int4-g128) or 64 (int4-g64: the per-projection
+ * ablation's int4-g64 scheme on the int3-g64 page, read as the same joint
+ * search on 64-weight groups). */
 ORC_API void orc_search_asym_int4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
                                   int64_t ms, const float* m, int64_t m_stride, int ns, int nz,
                                   double lo, double hi, float* scales, uint8_t* zeros, int32_t* idx,
-                                  double* loss, uint8_t* codes)
+                                  double* loss, uint8_t* codes, int g)
 {
-    const int64_t G = (I + 127) / 128;
+    const int64_t G = (I + g - 1) / g;
     #pragma omp parallel for schedule(dynamic, 16)
     for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
         int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
-        int64_t j0 = k * 128; int n = (int)((I - j0) < 128 ? (I - j0) : 128);
+        int64_t j0 = k * g; int n = (int)((I - j0) < g ? (I - j0) : g);
         const float* w = W + e * ms + o * ld + j0;
         const float* mm = m + e * m_stride + j0;
         float s; uint8_t z; double L;
@@ -491,13 +494,13 @@ ORC_API void orc_loss_given_int3(const float* W, int64_t n_mat, int64_t O, int64
 
 ORC_API void orc_loss_given_int4(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld,
                                  int64_t ms, const float* m, int64_t m_stride, const float* scales,
-                                 const uint8_t* zeros, double* loss)
+                                 const uint8_t* zeros, double* loss, int g)
 {
-    const int64_t G = (I + 127) / 128;
+    const int64_t G = (I + g - 1) / g;
     #pragma omp parallel for schedule(static)
     for (int64_t gi = 0; gi < n_mat * O * G; ++gi) {
         int64_t e = gi / (O * G), o = (gi / G) % O, k = gi % G;
-        int64_t j0 = k * 128; int n = (int)((I - j0) < 128 ? (I - j0) : 128);
+        int64_t j0 = k * g; int n = (int)((I - j0) < g ? (I - j0) : g);
         loss[gi] = orc_asym_loss(W + e * ms + o * ld + j0, m + e * m_stride + j0, n, scales[gi],
                                  zeros[gi], NULL);
     }
@@ -532,13 +535,13 @@ ORC_API void orc_rtn_int3(const float* W, int64_t rows, int64_t I, const float* 
 }
 
 ORC_API void orc_rtn_int4(const float* W, int64_t rows, int64_t I, const float* scales,
-                          const uint8_t* zeros, uint8_t* q)
+                          const uint8_t* zeros, uint8_t* q, int g)
 {
-    const int64_t G = (I + 127) / 128;
+    const int64_t G = (I + g - 1) / g;
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t j = 0; j < I; ++j) {
-            float s = scales[r * G + j / 128]; int z = zeros[r * G + j / 128];
+            float s = scales[r * G + j / g]; int z = zeros[r * G + j / g];
             double qq;
             if (s == 0.0f) qq = (double)z;
             else {
@@ -649,12 +652,12 @@ ORC_API void orc_dequant_int3(const int8_t* v, int64_t rows, int64_t I, const fl
 }
 
 ORC_API void orc_dequant_int4(const uint8_t* q, int64_t rows, int64_t I, const float* scales,
-                              const uint8_t* zeros, float* out)
+                              const uint8_t* zeros, float* out, int g)
 {
-    const int64_t G = (I + 127) / 128;
+    const int64_t G = (I + g - 1) / g;
     for (int64_t r = 0; r < rows; ++r)
         for (int64_t j = 0; j < I; ++j) {
-            int64_t gi = r * G + j / 128;
+            int64_t gi = r * G + j / g;
             out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));
         }
 }

@@ -17,7 +17,8 @@ MATCH_MIN = 0.999
 LOSS_RTOL = 1e-5
 SUM_RTOL = 1e-5
 
-ORC_FMT = {tq.INT3_G64_SYM: "int3", tq.INT4_G128_ASYM: "int4", tq.NVFP4_G16: "nvfp4"}
+ORC_FMT = {tq.INT3_G64_SYM: "int3", tq.INT4_G128_ASYM: "int4", tq.INT4_G64_ASYM: "int4", tq.NVFP4_G16: "nvfp4"}
+INT4 = {tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64}   # int4 formats -> group size
 
 
 def host32(t: torch.Tensor) -> np.ndarray:
@@ -29,8 +30,8 @@ def oracle_search(fmt, Wh, mh):
     if fmt == tq.INT3_G64_SYM:
         s, i, L, v = oracle.search_sym_int3(Wh, mh)
         return dict(scales=s, idx=i, loss=L, codes=v)
-    if fmt == tq.INT4_G128_ASYM:
-        s, z, i, L, q = oracle.search_asym_int4(Wh, mh)
+    if fmt in INT4:
+        s, z, i, L, q = oracle.search_asym_int4(Wh, mh, g=INT4[fmt])
         return dict(scales=s, zeros=z, idx=i, loss=L, codes=q)
     g, sc, i, L, c = oracle.search_nvfp4(Wh, mh)
     return dict(gscale=g, scales=sc, idx=i, loss=L, codes=c)
@@ -40,8 +41,8 @@ def loss_of_gpu_choice(fmt, Wh, mh, res):
     s = res.scales.cpu().numpy()
     if fmt == tq.INT3_G64_SYM:
         return oracle.loss_given_int3(Wh, mh, s)
-    if fmt == tq.INT4_G128_ASYM:
-        return oracle.loss_given_int4(Wh, mh, s, res.zeros.cpu().numpy())
+    if fmt in INT4:
+        return oracle.loss_given_int4(Wh, mh, s, res.zeros.cpu().numpy(), g=INT4[fmt])
     return oracle.loss_given_nvfp4(Wh, mh, s, res.global_scale.cpu().numpy())
 
 
@@ -68,7 +69,7 @@ def check_search(fmt, W: torch.Tensor, m: torch.Tensor, res, label=""):
     same = gi == o["idx"]
     gs = res.scales.cpu().numpy()
     assert np.array_equal(gs[same], o["scales"][same]), f"{label}: scale bits differ on matching groups"
-    if fmt == tq.INT4_G128_ASYM:
+    if fmt in INT4:
         assert np.array_equal(res.zeros.cpu().numpy()[same], o["zeros"][same])
     if fmt == tq.NVFP4_G16:
         assert np.array_equal(res.global_scale.cpu().numpy(), o["gscale"]), f"{label}: global scale"
@@ -81,9 +82,9 @@ def oracle_packed(fmt, Wh, scales, zeros=None, gscale=None):
     if fmt == tq.INT3_G64_SYM:
         v = oracle.rtn_int3(Wh, scales)
         return oracle.pack_int3(v.reshape(E * O, I)), v
-    if fmt == tq.INT4_G128_ASYM:
-        q = oracle.rtn_int4(Wh, scales, zeros)
-        return oracle.pack_nibbles(q.reshape(E * O, I), 128, zeros.reshape(E * O, -1)), q
+    if fmt in INT4:
+        q = oracle.rtn_int4(Wh, scales, zeros, g=INT4[fmt])
+        return oracle.pack_nibbles(q.reshape(E * O, I), INT4[fmt], zeros.reshape(E * O, -1)), q
     c = oracle.rtn_nvfp4(Wh, scales, gscale)
     return oracle.pack_nibbles(c.reshape(E * O, I), 16), c
 
@@ -92,9 +93,9 @@ def oracle_dequant(fmt, codes, scales, zeros=None, gscale=None):
     E, O, I = codes.shape
     if fmt == tq.INT3_G64_SYM:
         return oracle.dequant_int3(codes.reshape(E * O, I), scales.reshape(E * O, -1)).reshape(E, O, I)
-    if fmt == tq.INT4_G128_ASYM:
+    if fmt in INT4:
         return oracle.dequant_int4(codes.reshape(E * O, I), scales.reshape(E * O, -1),
-                                   zeros.reshape(E * O, -1)).reshape(E, O, I)
+                                   zeros.reshape(E * O, -1), g=INT4[fmt]).reshape(E, O, I)
     return oracle.dequant_nvfp4(codes, scales, gscale)
 
 
