@@ -445,6 +445,7 @@ def main():
     next_rows = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
     if step.units[0].fmt == "int4_g128_asym":
         next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
+        next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
     next_rows["hessian"] = time_hessian(tq, step, pk)
 
     # end to end through the public API from pinned host buffers
@@ -534,6 +535,39 @@ def time_ladder(tq, step, peak_tinst, reps=3):
     return {"ms": ms, "weights_per_s": nw / (ms * 1e-3), "cee_per_s": cee * nw / (ms * 1e-3),
             "achieved_tinst": achieved, "frac": achieved / peak_tinst,
             "note": f"first unit, {reps} launches, 4096 candidate-element evaluations x 5 instr per weight"}
+
+
+def time_int4_g64(tq, step, pk, peak_tinst, reps=5):
+    """The int4-g64 format on the first unit: the joint search with fused RTN
+    and pack (1024 candidate-element evaluations per weight, as for g128)
+    against the FP32 issue roofline, and the bf16 dequantization against HBM
+    (records 0.5 B + scale and zero 5/64 B read, 2 B written per weight)."""
+    u = step.units[0]
+    m = step._m_for(u)
+    fmt = tq.INT4_G64_ASYM
+    Ws = [s[1][0] for s in step.sets]
+    E, O, I = u.W.shape
+    res = tq.tq_search_groups(Ws[0], m, fmt)
+    dq = torch.empty((E, O, I), dtype=torch.bfloat16, device=u.W.device)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    ev[0].record()
+    for k in range(reps):
+        tq.tq_search_groups(Ws[k % len(Ws)], m, fmt, out=res)
+    ev[1].record()
+    for k in range(reps):
+        tq.tq_dequant(res.packed, fmt, res.scales, res.zeros, None, E, O, I, out=dq)
+    ev[2].record()
+    torch.cuda.synchronize()
+    ms_s = ev[0].elapsed_time(ev[1]) / reps
+    ms_d = ev[1].elapsed_time(ev[2]) / reps
+    nw = u.W.numel()
+    ach = 1024 * 5 * nw / (ms_s * 1e-3) / 1e12
+    dbytes = res.packed.numel() + res.scales.numel() * 4 + res.zeros.numel() + dq.numel() * 2
+    return {"search_ms": ms_s, "search_frac": ach / peak_tinst, "search_weights_per_s": nw / (ms_s * 1e-3),
+            "dequant_ms": ms_d, "dequant_frac": dbytes / (ms_d * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "note": f"first unit, {reps} launches each; search: 1024 evaluations x 5 instr per weight vs the "
+                    "FP32 issue peak; dequant: bytes vs measured HBM (the records are L2-resident when small)"}
 
 
 def time_hessian(tq, step, pk):
