@@ -47,6 +47,10 @@ def lib():
         sig = {
             "orc_imatrix": (None, [P, i64, i64, i64, P]),
             "orc_hessian": (None, [P, i64, i64, i64, P]),
+            "orc_e4m3_rne": (i32, [f32]),
+            "orc_fp8_scale": (f32, [i32, f64, f64, i32, f32]),
+            "orc_search_fp8": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, f64, f64, P, P, P, P, P]),
+            "orc_dequant_fp8": (None, [P, i64, i64, P, P]),
             "orc_hessian_entry": (f64, [P, i64, i64, i64, i64]),
             "orc_proxy_error_full": (None, [P, P, i64, i64, P, P, P]),
             "orc_sym_stage1_ratio": (f32, [i32, f64, f64, i32]),
@@ -157,6 +161,42 @@ def proxy_error_full(W, What, H) -> Tuple[float, float]:
     num = ctypes.c_double(); den = ctypes.c_double()
     lib().orc_proxy_error_full(_p(W), _p(What), O, I, _p(H), ctypes.byref(num), ctypes.byref(den))
     return num.value, den.value
+
+
+def e4m3_rne(y: float) -> int:
+    return lib().orc_e4m3_rne(float(np.float32(y)))
+
+
+def fp8_scale(n: int, lo: float, hi: float, k: int, amax: float) -> float:
+    return lib().orc_fp8_scale(n, lo, hi, k, float(np.float32(amax)))
+
+
+def search_fp8(W, m, n=64, lo=0.5, hi=1.2, codes=True):
+    """W [n_mat, O, I] (or [O, I]), m [n_mat, I] or [I] -> (scales[n_mat], idx, loss, losses[n_mat, n], codes)."""
+    W = _f32(W)
+    if W.ndim == 2:
+        W = W[None]
+    E, O, I = W.shape
+    m = _f32(m)
+    ms = I if m.ndim == 2 else 0
+    scales = np.empty(E, np.float32)
+    idx = np.empty(E, np.int32)
+    loss = np.empty(E, np.float64)
+    losses = np.empty((E, n), np.float64)
+    c = np.empty((E, O, I), np.uint8) if codes else None
+    lib().orc_search_fp8(_p(W), E, O, I, I, O * I, _p(m), ms, n, lo, hi, _p(scales), _p(idx), _p(loss),
+                         _p(losses), _p(c))
+    return scales, idx, loss, losses, c
+
+
+def dequant_fp8(c, scales) -> np.ndarray:
+    c = np.ascontiguousarray(c, np.uint8)
+    if c.ndim == 2:
+        c = c[None]
+    E = c.shape[0]
+    out = np.empty(c.shape, np.float32)
+    lib().orc_dequant_fp8(_p(c), E, c[0].size, _p(_f32(scales)), _p(out))
+    return out
 
 
 # ---------------------------------------------------------------- searches

@@ -521,6 +521,106 @@ ORC_API void orc_loss_given_nvfp4(const float* W, int64_t n_mat, int64_t O, int6
 }
 
 /* ------------------------------------------------------------------ */
+/* FP8 (E4M3) with one scale per tensor                                */
+/* ------------------------------------------------------------------ */
+
+/* Code of a non-negative E4M3 value v (exactly representable). */
+static int e4m3_code_of_value(double v)
+{
+    if (v == 0.0) return 0;
+    if (v < ldexp(1.0, -6)) return (int)(v * 512.0);          /* subnormal: m 2^-9 */
+    int e;
+    double f = frexp(v, &e);                                  /* v = f 2^e, f in [0.5, 1) */
+    return ((e - 1 + 7) << 3) | (int)((2.0 * f - 1.0) * 8.0);  /* (1 + m/8) 2^(E-7) */
+}
+
+/* E4M3 code of y: round to nearest, ties to the even code, saturating at
+ * +-448 (the largest finite e4m3fn value); a value that rounds to zero is
+ * code 0 (+0); NaN gives 0.  [NVFP4] recipe table: FP8 per-tensor for the
+ * shared experts and the Mamba linears.  The rounding step is 2^-9 below
+ * 2^-6 (subnormals) and 2^(floor(log2 y) - 3) above (3 mantissa bits). */
+ORC_API int orc_e4m3_rne(float y)
+{
+    double a = fabs((double)y);
+    if (!(a == a)) return 0;
+    double v;
+    if (a >= 448.0) v = 448.0;
+    else {
+        double step = a < ldexp(1.0, -6) ? ldexp(1.0, -9) : ldexp(1.0, ilogb(a) - 3);
+        v = nearbyint(a / step) * step;                       /* a / step is exact */
+        if (v > 448.0) v = 448.0;
+    }
+    int c = e4m3_code_of_value(v);
+    return (y < 0.0f && c != 0) ? (c | 0x80) : c;
+}
+
+/* Candidate k of the per-tensor grid: ratio r_k = fl32(lo + ((hi - lo) k) /
+ * (n - 1)) of amax / 448, scale s_k = fl32(r_k amax / 448) (one rounding).
+ * Reading: the NeUQI search window [0.5, 1.2], as the asymmetric grid's. */
+ORC_API float orc_fp8_scale(int n, double lo, double hi, int k, float amax)
+{
+    float r = (float)(lo + ((hi - lo) * (double)k) / (double)(n - 1));
+    return (float)((double)r * (double)amax / 448.0);
+}
+
+/* Per matrix: amax = max |w|; for each of the n candidate scales the loss
+ * L_k = sum_{o,j} m_j (w - fl32(s_k dec(c)))^2 with c = orc_e4m3_rne(fl32(w / s_k))
+ * (fp64); the chosen k is the lowest of the minimum loss.  amax = 0 gives
+ * scale 0, index -1, loss 0 and codes 0.  codes: [n_mat][O][I] u8 (optional);
+ * losses: [n_mat][n] (optional). */
+ORC_API void orc_search_fp8(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
+                            const float* m, int64_t m_stride, int n, double lo, double hi,
+                            float* scales, int32_t* idx, double* loss, double* losses, uint8_t* codes)
+{
+    for (int64_t e = 0; e < n_mat; ++e) {
+        const float* We = W + e * ms;
+        const float* me = m + e * m_stride;
+        double amax = 0.0;
+        for (int64_t o = 0; o < O; ++o)
+            for (int64_t j = 0; j < I; ++j) {
+                double a = fabs((double)We[o * ld + j]);
+                if (a > amax) amax = a;
+            }
+        int best = -1;
+        double bestL = INFINITY;
+        float bestS = 0.0f;
+        for (int k = 0; k < n; ++k) {
+            float sk = orc_fp8_scale(n, lo, hi, k, (float)amax);
+            double L = 0.0;
+            if (amax > 0.0) {
+                #pragma omp parallel for reduction(+:L) schedule(static)
+                for (int64_t o = 0; o < O; ++o)
+                    for (int64_t j = 0; j < I; ++j) {
+                        float w = We[o * ld + j];
+                        int c = orc_e4m3_rne(w / sk);
+                        double wh = (double)(float)((double)sk * orc_e4m3_decode(c));
+                        double d = (double)w - wh;
+                        L += (double)me[j] * (d * d);
+                    }
+            }
+            if (losses) losses[e * n + k] = L;
+            if (amax > 0.0 && L < bestL) { bestL = L; best = k; bestS = sk; }
+        }
+        if (amax == 0.0) { bestL = 0.0; bestS = 0.0f; best = -1; }
+        scales[e] = bestS;
+        if (idx) idx[e] = best;
+        if (loss) loss[e] = bestL;
+        if (codes)
+            for (int64_t o = 0; o < O; ++o)
+                for (int64_t j = 0; j < I; ++j)
+                    codes[(e * O + o) * I + j] = bestS == 0.0f ? 0 : (uint8_t)orc_e4m3_rne(We[o * ld + j] / bestS);
+    }
+}
+
+/* What = fl32(s dec(c)) for codes [n_mat][O][I] and one scale per matrix. */
+ORC_API void orc_dequant_fp8(const uint8_t* c, int64_t n_mat, int64_t OI, const float* scales, float* out)
+{
+    for (int64_t e = 0; e < n_mat; ++e)
+        for (int64_t i = 0; i < OI; ++i)
+            out[e * OI + i] = (float)((double)scales[e] * orc_e4m3_decode(c[e * OI + i]));
+}
+
+/* ------------------------------------------------------------------ */
 /* Round-to-nearest with given scales (pack path)                      */
 /* ------------------------------------------------------------------ */
 

@@ -38,6 +38,12 @@ MUTANTS = {
                                    "for (int64_t t = 0; t + 1 < T; ++t) s += (double)X[t * ld + i] * (double)X[t * ld + j];\n            H[i * I + j] = s;"),
     "proxy_full_diagonal_only": ("hn += H[i * I + j] * ((double)w[j] - (double)wh[j]);",
                                  "hn += (i == j) * H[i * I + j] * ((double)w[j] - (double)wh[j]);"),
+    "e4m3_ties_away": ("v = nearbyint(a / step) * step;                       /* a / step is exact */",
+                       "v = round(a / step) * step;                       /* a / step is exact */"),
+    "e4m3_subnormal_step": ("double step = a < ldexp(1.0, -6) ? ldexp(1.0, -9) : ldexp(1.0, ilogb(a) - 3);",
+                            "double step = a < ldexp(1.0, -7) ? ldexp(1.0, -9) : ldexp(1.0, ilogb(a) - 3);"),
+    "fp8_scale_240": ("return (float)((double)r * (double)amax / 448.0);", "return (float)((double)r * (double)amax / 240.0);"),
+    "fp8_loss_unweighted": ("L += (double)me[j] * (d * d);", "L += (d * d);"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }

@@ -621,3 +621,85 @@ def test_int4_g64_batching(orc):
     inside = (q > 0) & (q < 15)
     assert np.all(np.abs(What - W)[inside] <= 0.5 * step[inside] * (1 + 1e-6))
     assert np.array_equal(orc.loss_given_int4(W, m, s, z, g=64), L)
+
+
+# ------------------------------------------------------------------ FP8 per-tensor ([NVFP4] recipe table)
+
+def _e4m3_values(orc):
+    return np.array([orc.e4m3_decode(c) for c in range(0x7F)], np.float64)   # codes 0..126
+
+
+def test_e4m3_rne_brute_force_and_torch(orc):
+    """E4M3 round-to-nearest: the nearest of the 127 finite magnitudes, ties to
+    the even code, saturating at 448, sign in bit 7 except for a zero result;
+    equal to torch's float8_e4m3fn cast on every in-range value."""
+    vals = _e4m3_values(orc)
+    rng = np.random.default_rng(53)
+    mids = (vals[1:] + vals[:-1]) / 2
+    xs = np.concatenate([vals, mids, np.nextafter(mids.astype(np.float32), np.float32(np.inf)),
+                         np.nextafter(mids.astype(np.float32), np.float32(0)),
+                         rng.uniform(0, 460, 3000), np.exp(rng.uniform(-14, 6, 3000)),
+                         [449.0, 463.9, 464.0, 480.0, 1e6, 2.0 ** -10, 3 * 2.0 ** -11]]).astype(np.float32)
+    for x in xs:
+        for y in (x, -x):
+            c = orc.e4m3_rne(y)
+            a = abs(float(y))
+            d = np.abs(vals - a)
+            cand = np.flatnonzero(d == d.min())
+            want = cand[0] if len(cand) == 1 else [k for k in cand if k % 2 == 0][0]
+            want = int(want) if a < 448 else 0x7E
+            if y < 0 and want != 0:
+                want |= 0x80
+            assert c == want, (float(y), c, want)
+    import torch
+    inr = xs[np.abs(xs) <= 448]
+    t = torch.from_numpy(np.concatenate([inr, -inr])).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    mine = np.array([orc.e4m3_rne(y) for y in np.concatenate([inr, -inr])])
+    t = np.where((t & 0x7F) == 0, 0, t)          # torch keeps -0; the format here writes +0
+    assert np.array_equal(mine, t)
+
+
+def test_fp8_search_direct(orc):
+    """Per-tensor search against the definition evaluated directly (torch's
+    e4m3 cast for the codes): every candidate's loss, the lowest-index argmin,
+    the codes of the chosen scale; degenerate all-zero tensor; a tensor made
+    of one candidate's grid values has zero loss there."""
+    import torch
+    rng = np.random.default_rng(59)
+    W = (rng.standard_t(4, size=(2, 9, 70)) * 0.02).astype(np.float32)
+    m = rng.random((2, 70)).astype(np.float32)
+    s, i, L, Ls, c = orc.search_fp8(W, m, n=16)
+    for e in range(2):
+        amax = np.float32(np.abs(W[e]).max())
+        for k in range(16):
+            sk = np.float32(np.float32(0.5 + 0.7 * k / 15) * np.float64(amax) / 448.0)
+            assert orc.fp8_scale(16, 0.5, 1.2, k, amax) == sk
+            y = torch.from_numpy((W[e] / sk).astype(np.float32)).clamp(-448, 448)
+            q = y.to(torch.float8_e4m3fn).to(torch.float64).numpy()
+            wh = (np.float64(sk) * q).astype(np.float32).astype(np.float64)
+            Ld = float(np.sum(m[e][None, :].astype(np.float64) * (W[e].astype(np.float64) - wh) ** 2))
+            assert np.isclose(Ls[e, k], Ld, rtol=1e-12)
+        assert i[e] == int(np.argmin(Ls[e])) and s[e] == orc.fp8_scale(16, 0.5, 1.2, int(i[e]), amax)
+        assert np.array_equal(c[e], np.vectorize(lambda w: orc.e4m3_rne(w / s[e]))(W[e]).astype(np.uint8))
+    z, iz, Lz, _, cz = orc.search_fp8(np.zeros((1, 3, 5), np.float32), np.ones(5, np.float32), n=8)
+    assert z[0] == 0 and iz[0] == -1 and Lz[0] == 0 and not cz.any()
+    # W on candidate 5's grid (amax kept by an entry at +448 s_5 / r_5)
+    k = 5
+    amax = np.float32(1.0)
+    sk = orc.fp8_scale(8, 0.5, 1.2, k, amax)
+    vals = _e4m3_values(orc)
+    Wg = (np.float64(sk) * rng.choice(vals[:100], size=(1, 4, 30)) * rng.choice([-1, 1], size=(1, 4, 30)))
+    Wg = Wg.astype(np.float32)
+    Wg[0, 0, 0] = amax
+    s2, i2, L2, Ls2, _ = orc.search_fp8(Wg, np.ones(30, np.float32), n=8)
+    assert Ls2[0].min() <= Ls2[0, k] and Ls2[0, k] <= 1e-6 * Ls2[0].max()
+
+
+def test_fp8_dequant(orc):
+    rng = np.random.default_rng(61)
+    c = rng.integers(0, 256, size=(2, 3, 40)).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0
+    s = np.array([0.01, 3.5], np.float32)
+    out = orc.dequant_fp8(c, s)
+    vals = np.array([orc.e4m3_decode(int(x)) for x in range(256)])
+    assert np.array_equal(out, (s[:, None, None].astype(np.float64) * vals[c]).astype(np.float32))
