@@ -19,6 +19,7 @@ path).  --impl reference times the CPU oracle on a bounded sample instead.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import json
 import math
@@ -447,6 +448,7 @@ def main():
         next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
         next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
     next_rows["hessian"] = time_hessian(tq, step, pk)
+    next_rows["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -568,6 +570,38 @@ def time_int4_g64(tq, step, pk, peak_tinst, reps=5):
             "dequant_ms": ms_d, "dequant_frac": dbytes / (ms_d * 1e-3) / 1e9 / pk["hbm_gbs"],
             "note": f"first unit, {reps} launches each; search: 1024 evaluations x 5 instr per weight vs the "
                     "FP32 issue peak; dequant: bytes vs measured HBM (the records are L2-resident when small)"}
+
+
+# FP32-issue work of one FP8 candidate-element evaluation in k_fp8_loss
+# (ncu instruction count of the kernel per evaluation, rounded).
+FP8_INSTR_PER_CEE = 14
+
+
+def time_fp8(tq, step, pk, peak_tinst, reps=3):
+    """FP8 (E4M3) per-tensor scale search on the first unit (amax, 64
+    candidate losses per weight in fp64, the pick, the fused pack of the
+    codes), rotating weight copies; CEE/s and the fraction of the FP32 issue
+    peak at FP8_INSTR_PER_CEE instructions per evaluation."""
+    u = step.units[0]
+    m = step._m_for(u)
+    Ws = [s[1][0] for s in step.sets]
+    res = tq.tq_search_fp8(Ws[0], m)
+    ws = torch.empty(max(16, tq.lib().tq_fp8_workspace_bytes(ctypes.byref(tq._mat(Ws[0], "W")))),
+                     dtype=torch.uint8, device=u.W.device)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(reps):
+        tq.tq_search_fp8(Ws[k % len(Ws)], m, out=res, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    nw = u.W.numel()
+    cee = 64 * nw / (ms * 1e-3)
+    return {"ms": ms, "weights_per_s": nw / (ms * 1e-3), "cee_per_s": cee,
+            "frac": cee * FP8_INSTR_PER_CEE / 1e12 / peak_tinst,
+            "note": f"first unit, {reps} launches of the whole call (amax + losses + pick + pack); "
+                    f"{FP8_INSTR_PER_CEE} FP32-issue instructions per candidate-element evaluation"}
 
 
 def time_hessian(tq, step, pk):

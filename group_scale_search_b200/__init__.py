@@ -32,7 +32,7 @@ __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -54,7 +54,7 @@ EXPORTS = [
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
-    "tq_dequant_gemv", "tq_hessian",
+    "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
 ]
 
 
@@ -130,6 +130,10 @@ def lib():
             "tq_imatrix_workspace_bytes": (sz, [Mp]),
             "tq_imatrix": (i32, [Mp, P, i64, ctypes.c_float, i32, P, sz, P]),
             "tq_hessian": (i32, [Mp, P, i64, i64, ctypes.c_float, i32, P]),
+            "tq_fp8_workspace_bytes": (sz, [Mp]),
+            "tq_search_fp8": (i32, [Mp, P, i64, i32, ctypes.c_double, ctypes.c_double, P, P, P, P, P, P, sz, P]),
+            "tq_pack_fp8": (i32, [Mp, P, P, P]),
+            "tq_dequant_fp8": (i32, [P, P, i64, i64, i64, P, i32, P]),
             "tq_amax": (i32, [Mp, P, P]),
             "tq_search_groups": (i32, [Mp, P, i64, i32, ctypes.POINTER(_Params), P, P, P, P, P, P, P]),
             "tq_pack": (i32, [Mp, i32, P, P, P, P, P]),
@@ -273,6 +277,59 @@ def tq_hessian(X: torch.Tensor, out: Optional[torch.Tensor] = None, alpha: float
     hms = out.stride(0) if out.dim() == 3 else 0
     _check(lib().tq_hessian(ctypes.byref(d), _ptr(out), ldh, hms, ctypes.c_float(alpha), int(accumulate),
                             _stream(stream)), "tq_hessian")
+    return out
+
+
+@dataclasses.dataclass
+class Fp8Result:
+    scales: torch.Tensor               # f32 [n_mat]
+    cand_idx: Optional[torch.Tensor]   # i32 [n_mat]
+    loss: Optional[torch.Tensor]       # f64 [n_mat]
+    losses: Optional[torch.Tensor]     # f64 [n_mat, n_cand]
+    packed: Optional[torch.Tensor]     # u8 [n_mat, O, I] E4M3 codes
+
+
+def tq_search_fp8(W: torch.Tensor, m: torch.Tensor, n_cand: int = 64, lo: float = 0.5, hi: float = 1.2,
+                  pack: bool = True, out: Optional[Fp8Result] = None, workspace: Optional[torch.Tensor] = None,
+                  stream=None) -> Fp8Result:
+    """FP8 (E4M3) with one scale per matrix, the scale searched over n_cand
+    candidates fl32(r amax / 448) by the imatrix-weighted squared error; with
+    pack=True the E4M3 codes of the chosen scale are written too."""
+    d = _mat(W, "W")
+    _cuda(m, "m")
+    E, O, I = d.n_mat, d.rows, d.cols
+    dev = W.device
+    if out is None:
+        out = Fp8Result(scales=torch.empty(E, dtype=torch.float32, device=dev),
+                        cand_idx=torch.empty(E, dtype=torch.int32, device=dev),
+                        loss=torch.empty(E, dtype=torch.float64, device=dev),
+                        losses=torch.empty((E, n_cand), dtype=torch.float64, device=dev),
+                        packed=torch.empty((E, O, I), dtype=torch.uint8, device=dev) if pack else None)
+    ws = int(lib().tq_fp8_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+    _check(lib().tq_search_fp8(ctypes.byref(d), _ptr(m), _m_stride(m), n_cand, lo, hi, _ptr(out.scales),
+                               _ptr(out.cand_idx), _ptr(out.loss), _ptr(out.losses), _ptr(out.packed),
+                               _ptr(workspace), workspace.numel(), _stream(stream)), "tq_search_fp8")
+    return out
+
+
+def tq_pack_fp8(W: torch.Tensor, scales: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    d = _mat(W, "W")
+    _cuda(scales, "scales")
+    if out is None:
+        out = torch.empty((d.n_mat, d.rows, d.cols), dtype=torch.uint8, device=W.device)
+    _check(lib().tq_pack_fp8(ctypes.byref(d), _ptr(scales), _ptr(out), _stream(stream)), "tq_pack_fp8")
+    return out
+
+
+def tq_dequant_fp8(packed: torch.Tensor, scales: torch.Tensor, n_mat: int, O: int, I: int,
+                   out_dtype=torch.float32, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    _cuda(packed, "packed")
+    if out is None:
+        out = torch.empty((n_mat, O, I), dtype=out_dtype, device=packed.device)
+    _check(lib().tq_dequant_fp8(_ptr(packed), _ptr(scales), n_mat, O, I, _ptr(out),
+                                _BF16 if out.dtype == torch.bfloat16 else _F32, _stream(stream)), "tq_dequant_fp8")
     return out
 
 

@@ -261,6 +261,32 @@ tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void* scales
                           const float* global_scale, int64_t n_mat, int64_t O, int64_t I, const void* x,
                           int32_t x_dtype, int64_t B, int64_t x_mat_stride, float* y, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ FP8 per tensor
+ * E4M3 weights with one fp32 scale per matrix ([NVFP4] Quantization Recipe
+ * table: FP8 per-tensor for the shared experts and the Mamba linears).  The
+ * scale is searched like the other formats' (imatrix-weighted squared error):
+ * candidates s_k = fl32(r_k amax / 448), r_k = fl32(lo + (hi - lo) k /
+ * (n_cand - 1)), amax = max |w| of the matrix; loss L_k = sum_{o,j} m_j
+ * (w - fl32(s_k dec(c)))^2 in fp64 with c the E4M3 code of fl32(w / s_k)
+ * (round to nearest, ties to even, saturating at 448, +0 for a zero
+ * result); the lowest k of the minimum wins (deterministic: fixed partition,
+ * fixed reduction order).  amax = 0 gives scale 0, index -1, loss 0, codes 0.
+ * scales: f32 [n_mat] (required); cand_idx: i32 [n_mat], loss: f64 [n_mat],
+ * losses: f64 [n_mat][n_cand] (optional); packed: u8 [n_mat][O][I] E4M3 codes
+ * of the chosen scale (optional, 16-byte aligned).  n_cand in [2, 64]
+ * (TQ_ERR_UNSUPPORTED otherwise); 0 < lo <= hi.  workspace: >=
+ * tq_fp8_workspace_bytes(W), 16-byte aligned, no initialisation needed.
+ * tq_pack_fp8 writes the codes for given scales; tq_dequant_fp8 writes
+ * What = fl32(s dec(c)) (fp32, or its RNE to bf16) as dense [n_mat][O][I]
+ * (scale codes are read as e4m3fn; 0x7F/0xFF are outside the domain). */
+size_t tq_fp8_workspace_bytes(const tq_mat* W);
+tq_status tq_search_fp8(const tq_mat* W, const float* m, int64_t m_stride, int32_t n_cand, double lo, double hi,
+                        float* scales, int32_t* cand_idx, double* loss, double* losses, uint8_t* packed,
+                        void* workspace, size_t workspace_bytes, tq_stream_t stream);
+tq_status tq_pack_fp8(const tq_mat* W, const float* scales, uint8_t* packed, tq_stream_t stream);
+tq_status tq_dequant_fp8(const uint8_t* packed, const float* scales, int64_t n_mat, int64_t O, int64_t I,
+                         void* out, int32_t out_dtype, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ Hessian
  * H[e] = alpha * sum_t X[e][t]^T X[e][t] (+ H[e] when accumulate): the
  * per-linear-input Hessian ([TT] pipeline table, step 1), fp32, from bf16

@@ -115,6 +115,16 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     assert b"aligned" in L.tq_last_error_string()
     assert gemv(fake, tq.INT4_G128_ASYM, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
     assert gemv(fake, tq.NVFP4_G16, fake, None, None, 1, 8, 64, fake, 0, 1, 0, fake, None) == 1
+    # FP8 per tensor: (W, m, m_stride, n_cand, lo, hi, scales, idx, loss, losses, packed, ws, ws_bytes, stream)
+    w8 = tq._Mat(fake, 1, 0, 1, 16, 64, 64, 0)
+    need8 = L.tq_fp8_workspace_bytes(ctypes.byref(w8))
+    assert need8 > 0
+    f8 = L.tq_search_fp8
+    assert f8(ctypes.byref(w8), fake, 0, 65, 0.5, 1.2, fake, None, None, None, None, fake, need8, None) == 2
+    assert f8(ctypes.byref(w8), fake, 0, 64, 0.5, 1.2, fake, None, None, None, None, fake, need8 - 8, None) == 1
+    assert f8(ctypes.byref(w8), fake, 0, 64, 1.2, 0.5, fake, None, None, None, None, fake, need8, None) == 1
+    assert f8(ctypes.byref(w8), None, 0, 64, 0.5, 1.2, fake, None, None, None, None, fake, need8, None) == 1
+    assert L.tq_dequant_fp8(fake, fake, 1, 4, 64, fake, 7, None) == 2
     # Hessian: (X, H, ldh, h_mat_stride, alpha, accumulate, stream)
     hs = L.tq_hessian
     x = tq._Mat(fake, 1, 0, 1, 256, 128, 128, 0)

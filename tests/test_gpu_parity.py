@@ -555,3 +555,76 @@ def test_hessian_strided_sites():
         Xh = X[e].float().cpu().numpy()
         bad = np.abs(out[e].cpu().numpy().astype(np.float64) - oracle.hessian(Xh)) > _hessian_bound(Xh)
         assert not bad.any(), e
+
+
+# ------------------------------------------------------------------ FP8 per tensor
+
+def _fp8_oracle_check(W, m, n, lo=0.5, hi=1.2, label=""):
+    r = tq.tq_search_fp8(W, m, n_cand=n, lo=lo, hi=hi)
+    torch.cuda.synchronize()
+    W3 = W if W.dim() == 3 else W.unsqueeze(0)
+    Wh, mh = host32(W3), m.cpu().numpy()
+    s, i, L, Ls, c = oracle.search_fp8(Wh, mh, n=n, lo=lo, hi=hi)
+    gi = r.cand_idx.cpu().numpy()
+    assert np.allclose(r.losses.cpu().numpy(), Ls, rtol=1e-12, atol=1e-300), label
+    for e in range(Wh.shape[0]):
+        if gi[e] != i[e]:   # only an fp64 near tie may differ: the GPU's choice is then as good
+            assert abs(Ls[e, gi[e]] - Ls[e].min()) <= 1e-12 * Ls[e].min(), (label, e)
+    same = gi == i
+    assert np.array_equal(r.scales.cpu().numpy()[same], s[same]), label
+    codes = oracle.search_fp8(Wh, mh, n=n, lo=lo, hi=hi)[4] if same.all() else None
+    if codes is not None:
+        assert np.array_equal(r.packed.cpu().numpy(), codes), label
+    # given the GPU's scales: pack and dequant bit-exact against the oracle
+    sc = r.scales.cpu().numpy()
+    ref = np.stack([np.vectorize(lambda w: oracle.e4m3_rne(w / sc[e]) if sc[e] != 0 else 0)(Wh[e])
+                    for e in range(Wh.shape[0])]).astype(np.uint8)
+    assert np.array_equal(r.packed.cpu().numpy(), ref), label
+    E, O, I = Wh.shape
+    dq = tq.tq_dequant_fp8(r.packed, r.scales, E, O, I)
+    dqb = tq.tq_dequant_fp8(r.packed, r.scales, E, O, I, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref_dq = oracle.dequant_fp8(ref, sc)
+    assert np.array_equal(dq.cpu().numpy(), ref_dq), label
+    assert torch.equal(dqb.cpu(), torch.from_numpy(ref_dq).to(torch.bfloat16)), label
+    return r
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n", [64, 16, 2])
+def test_fp8_search_matches_oracle(dtype, n):
+    """Per-tensor E4M3 scale search against the oracle: every candidate's fp64
+    loss, the chosen index and scale, the codes of the chosen scale and the
+    dequantized weights bit-exact; ragged rows (I = 300 in a padded row),
+    several matrices with their own imatrix, one shared."""
+    g = torch.Generator(device=DEV).manual_seed(n)
+    big = (synth.student_t((3, 37, 304), 4, g, DEV) * 0.02).to(dtype)
+    W = big[:, :, :300]
+    m = torch.stack([synth.random_imatrix(300, 3 + e, DEV) for e in range(3)])
+    _fp8_oracle_check(W, m, n, label=f"{dtype} n={n} per-matrix m")
+    _fp8_oracle_check(W, m[0], n, lo=0.8, hi=1.0, label=f"{dtype} n={n} shared m")
+
+
+def test_fp8_degenerate_and_rounding_edges():
+    """An all-zero matrix (scale 0, index -1, codes 0); tq_pack_fp8 with a given
+    scale on every E4M3 value, the midpoints between neighbours and the fp32
+    values next to them, subnormals, values past 448 and signed zeros."""
+    W = torch.zeros((2, 8, 64), device=DEV)
+    W[1] = torch.randn((8, 64), device=DEV) * 0.01
+    m = torch.ones(64, device=DEV)
+    r = _fp8_oracle_check(W, m, 64, label="zero matrix")
+    assert r.cand_idx[0].item() == -1 and r.scales[0].item() == 0.0 and not r.packed[0].any()
+    vals = np.array([oracle.e4m3_decode(c) for c in range(0x7F)], np.float64)
+    mids = ((vals[1:] + vals[:-1]) / 2).astype(np.float32)
+    xs = np.concatenate([vals.astype(np.float32), mids, np.nextafter(mids, np.float32(np.inf)),
+                         np.nextafter(mids, np.float32(0)), [449.0, 463.99, 464.0, 480.0, 1e30, 2.0 ** -10,
+                                                           2.0 ** -12, 0.0]]).astype(np.float32)
+    xs = np.concatenate([xs, -xs])
+    pad = (-len(xs)) % 8
+    xs = np.concatenate([xs, np.zeros(pad, np.float32)])
+    for scale in (1.0, 0.0625, 3.0):
+        Wt = torch.from_numpy((xs * np.float32(scale)).reshape(1, 1, -1)).to(DEV)
+        p = tq.tq_pack_fp8(Wt, torch.tensor([scale], dtype=torch.float32, device=DEV))
+        torch.cuda.synchronize()
+        want = np.array([oracle.e4m3_rne(np.float32(w) / np.float32(scale)) for w in Wt.cpu().numpy().reshape(-1)])
+        assert np.array_equal(p.cpu().numpy().reshape(-1), want.astype(np.uint8)), scale
