@@ -48,6 +48,8 @@ def lib():
             "orc_imatrix": (None, [P, i64, i64, i64, P]),
             "orc_hessian": (None, [P, i64, i64, i64, P]),
             "orc_e4m3_rne": (i32, [f32]),
+            "orc_lloyd_max_g32": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, P, P, P, P, P]),
+            "orc_lloyd_max_assign": (None, [P, i64, i64, i64, i64, i64, P, P, P]),
             "orc_fp8_scale": (f32, [i32, f64, f64, i32, f32]),
             "orc_search_fp8": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, f64, f64, P, P, P, P, P]),
             "orc_dequant_fp8": (None, [P, i64, i64, P, P]),
@@ -187,6 +189,38 @@ def search_fp8(W, m, n=64, lo=0.5, hi=1.2, codes=True):
     lib().orc_search_fp8(_p(W), E, O, I, I, O * I, _p(m), ms, n, lo, hi, _p(scales), _p(idx), _p(loss),
                          _p(losses), _p(c))
     return scales, idx, loss, losses, c
+
+
+LM_START = (-0.75, -0.25, 0.25, 0.75)
+
+
+def lloyd_max_g32(W, m, n_iter=16, start=LM_START, codes=True):
+    """W [n_mat, O, I], m [n_mat, I] or [I] -> (codebook[4], scales[n_mat, O, G32], codes, loss, history)."""
+    W = _f32(W)
+    if W.ndim == 2:
+        W = W[None]
+    E, O, I = W.shape
+    m = _f32(m)
+    ms = I if m.ndim == 2 else 0
+    cb = np.array(start, np.float32)
+    sc = np.empty((E, O, (I + 31) // 32), np.float32)
+    c = np.empty((E, O, I), np.uint8) if codes else None
+    loss = ctypes.c_double()
+    hist = np.empty(n_iter + 1, np.float64)
+    lib().orc_lloyd_max_g32(_p(W), E, O, I, I, O * I, _p(m), ms, n_iter, _p(cb), _p(sc), _p(c),
+                            ctypes.byref(loss), _p(hist))
+    return cb, sc, c, loss.value, hist
+
+
+def lloyd_max_assign(W, codebook):
+    W = _f32(W)
+    if W.ndim == 2:
+        W = W[None]
+    E, O, I = W.shape
+    sc = np.empty((E, O, (I + 31) // 32), np.float32)
+    c = np.empty((E, O, I), np.uint8)
+    lib().orc_lloyd_max_assign(_p(W), E, O, I, I, O * I, _p(_f32(codebook)), _p(sc), _p(c))
+    return sc, c
 
 
 def dequant_fp8(c, scales) -> np.ndarray:

@@ -621,6 +621,98 @@ ORC_API void orc_dequant_fp8(const uint8_t* c, int64_t n_mat, int64_t OI, const 
 }
 
 /* ------------------------------------------------------------------ */
+/* Imatrix-weighted Lloyd-Max 2-bit codebook                           */
+/* ------------------------------------------------------------------ */
+/* "Phase 2: math-accuracy regression on tq3a-tq2e g32" (turboquant-mlx issue
+ * #2), Phase-2 candidate 1: a Lloyd-Max codebook for the 2-bit experts fit to
+ * calibration data instead of the data-free one, fixed and shared.  Reading:
+ * 32-weight groups with an absmax scale s = max |w|; normalised values
+ * u = fl32(w / s) (0 when s = 0); one 4-level codebook c_0 < ... < c_3 (fp32)
+ * shared by every matrix of the call, fit by Lloyd iterations that minimise
+ * sum m_j (w - s c_a)^2 = sum omega (u - c_a)^2, omega = m_j s^2: each
+ * element goes to the nearest level (ties to the lower one: u above the exact
+ * midpoint (c_i + c_{i+1}) / 2 moves up), each level becomes the
+ * omega-weighted mean of its elements (fp64, rounded once to fp32; an empty
+ * level keeps its value); start from the data-free Lloyd-Max levels of a
+ * uniform source on [-1, 1], {-3/4, -1/4, 1/4, 3/4}. */
+
+static double lm_u(float w, float s) { return s == 0.0f ? 0.0 : (double)(w / s); }
+
+static int lm_assign(double u, const float* c)
+{
+    int a = 0;
+    for (int i = 0; i < 3; ++i)
+        if (u > ((double)c[i] + (double)c[i + 1]) / 2.0) a = i + 1;
+    return a;
+}
+
+/* Group absmax scales [rows][G32] of W. */
+static void lm_scales(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms, float* scales)
+{
+    const int64_t G = (I + 31) / 32;
+    for (int64_t e = 0; e < n_mat; ++e)
+        for (int64_t o = 0; o < O; ++o)
+            for (int64_t k = 0; k < G; ++k) {
+                float a = 0.0f;
+                for (int64_t j = 32 * k; j < I && j < 32 * k + 32; ++j) {
+                    float v = fabsf(W[e * ms + o * ld + j]);
+                    if (v > a) a = v;
+                }
+                scales[(e * O + o) * G + k] = a;
+            }
+}
+
+/* n_iter Lloyd iterations.  codebook: in/out [4] (the start, then the fit);
+ * scales: out [n_mat][O][G32]; codes: out [n_mat][O][I] (0..3, optional);
+ * loss: out, sum m (w - s c_a)^2 over every matrix for the final codebook;
+ * history: optional [n_iter + 1] losses before each update and after the last. */
+ORC_API void orc_lloyd_max_g32(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
+                               const float* m, int64_t m_stride, int n_iter, float* codebook, float* scales,
+                               uint8_t* codes, double* loss, double* history)
+{
+    const int64_t G = (I + 31) / 32;
+    lm_scales(W, n_mat, O, I, ld, ms, scales);
+    for (int it = 0; it <= n_iter; ++it) {
+        double num[4] = {0, 0, 0, 0}, den[4] = {0, 0, 0, 0}, L = 0.0;
+        for (int64_t e = 0; e < n_mat; ++e)
+            for (int64_t o = 0; o < O; ++o)
+                for (int64_t j = 0; j < I; ++j) {
+                    float s = scales[(e * O + o) * G + j / 32];
+                    double u = lm_u(W[e * ms + o * ld + j], s);
+                    int a = lm_assign(u, codebook);
+                    double om = (double)m[e * m_stride + j] * (double)s * (double)s;
+                    num[a] += om * u;
+                    den[a] += om;
+                    double d = u - (double)codebook[a];
+                    L += om * d * d;
+                }
+        if (history) history[it] = L;
+        if (it == n_iter) { *loss = L; break; }
+        for (int i = 0; i < 4; ++i)
+            if (den[i] > 0.0) codebook[i] = (float)(num[i] / den[i]);
+    }
+    if (codes)
+        for (int64_t e = 0; e < n_mat; ++e)
+            for (int64_t o = 0; o < O; ++o)
+                for (int64_t j = 0; j < I; ++j)
+                    codes[(e * O + o) * I + j] = (uint8_t)lm_assign(
+                        lm_u(W[e * ms + o * ld + j], scales[(e * O + o) * G + j / 32]), codebook);
+}
+
+/* Codes for a given codebook and the group absmax scales. */
+ORC_API void orc_lloyd_max_assign(const float* W, int64_t n_mat, int64_t O, int64_t I, int64_t ld, int64_t ms,
+                                  const float* codebook, float* scales, uint8_t* codes)
+{
+    const int64_t G = (I + 31) / 32;
+    lm_scales(W, n_mat, O, I, ld, ms, scales);
+    for (int64_t e = 0; e < n_mat; ++e)
+        for (int64_t o = 0; o < O; ++o)
+            for (int64_t j = 0; j < I; ++j)
+                codes[(e * O + o) * I + j] = (uint8_t)lm_assign(
+                    lm_u(W[e * ms + o * ld + j], scales[(e * O + o) * G + j / 32]), codebook);
+}
+
+/* ------------------------------------------------------------------ */
 /* Round-to-nearest with given scales (pack path)                      */
 /* ------------------------------------------------------------------ */
 

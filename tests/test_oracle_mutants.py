@@ -44,6 +44,8 @@ MUTANTS = {
                             "double step = a < ldexp(1.0, -7) ? ldexp(1.0, -9) : ldexp(1.0, ilogb(a) - 3);"),
     "fp8_scale_240": ("return (float)((double)r * (double)amax / 448.0);", "return (float)((double)r * (double)amax / 240.0);"),
     "fp8_loss_unweighted": ("L += (double)me[j] * (d * d);", "L += (d * d);"),
+    "lloyd_ties_up": ("if (u > ((double)c[i] + (double)c[i + 1]) / 2.0) a = i + 1;", "if (u >= ((double)c[i] + (double)c[i + 1]) / 2.0) a = i + 1;"),
+    "lloyd_scale_not_squared": ("double om = (double)m[e * m_stride + j] * (double)s * (double)s;", "double om = (double)m[e * m_stride + j] * (double)s;"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }

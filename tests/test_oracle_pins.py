@@ -703,3 +703,48 @@ def test_fp8_dequant(orc):
     out = orc.dequant_fp8(c, s)
     vals = np.array([orc.e4m3_decode(int(x)) for x in range(256)])
     assert np.array_equal(out, (s[:, None, None].astype(np.float64) * vals[c]).astype(np.float32))
+
+
+# ------------------------------------------------------------------ Lloyd-Max 2-bit codebook (turboquant-mlx issue #2)
+
+def test_lloyd_max_pins(orc):
+    """Weighted Lloyd-Max on absmax-normalised 32-weight groups: the loss never
+    rises; one iteration equals a direct numpy evaluation (nearest level, ties
+    to the lower level, omega-weighted means); data made of four normalised
+    values is fit exactly; codes agree with the assignment for the final
+    codebook; an all-zero tensor keeps the start."""
+    rng = np.random.default_rng(67)
+    W = (rng.standard_t(4, size=(2, 12, 100)) * 0.02).astype(np.float32)
+    m = rng.random((2, 100)).astype(np.float32)
+    cb, sc, c, L, hist = orc.lloyd_max_g32(W, m, n_iter=12)
+    assert np.all(np.diff(hist) <= 1e-15 * hist[0])
+    assert np.isclose(L, hist[-1])
+    # one iteration, directly
+    cb1 = orc.lloyd_max_g32(W, m, n_iter=1)[0]
+    G = 4
+    s = np.abs(np.pad(W, ((0, 0), (0, 0), (0, 28)))).reshape(2, 12, G, 32).max(axis=3)
+    assert np.array_equal(s, sc)
+    u = np.where(np.repeat(s, 32, axis=2)[:, :, :100] == 0, 0.0,
+                 (W / np.where(np.repeat(s, 32, axis=2)[:, :, :100] == 0, 1, np.repeat(s, 32, axis=2)[:, :, :100])))
+    u = u.astype(np.float32).astype(np.float64)
+    c0 = np.array(orc.LM_START, np.float32).astype(np.float64)
+    mids = (c0[1:] + c0[:-1]) / 2
+    a = (u[..., None] > mids).sum(axis=-1)
+    om = m[:, None, :].astype(np.float64) * np.repeat(s, 32, axis=2)[:, :, :100].astype(np.float64) ** 2
+    want = np.array([np.float32(np.sum(om[a == i] * u[a == i]) / np.sum(om[a == i])) for i in range(4)])
+    assert np.array_equal(cb1, want)
+    # four normalised values per group: entries in {-1, -1/3, 1/3, 1} times the
+    # group's scale, the group's first entry +scale (so u takes exactly those values)
+    base = np.array([-1.0, -1 / 3, 1 / 3, 1.0], np.float32)
+    gs = rng.choice([0.01, 0.03], size=(1, 8, 2)).astype(np.float32)
+    Wq = base[rng.integers(0, 4, size=(1, 8, 64))] * np.repeat(gs, 32, axis=2)
+    Wq[:, :, 0] = gs[:, :, 0]
+    Wq[:, :, 32] = gs[:, :, 1]
+    Wq = Wq.astype(np.float32)
+    cbq, scq, cq, Lq, hq = orc.lloyd_max_g32(Wq, np.ones(64, np.float32), n_iter=10)
+    assert Lq <= 1e-12 * hq[0]
+    assert np.allclose(cbq, base, atol=2e-7)
+    sc2, c2 = orc.lloyd_max_assign(W, cb)
+    assert np.array_equal(sc2, sc) and np.array_equal(c2, c)
+    z = orc.lloyd_max_g32(np.zeros((1, 2, 40), np.float32), np.ones(40, np.float32), n_iter=3)
+    assert np.array_equal(z[0], np.array(orc.LM_START, np.float32)) and z[3] == 0.0
