@@ -744,6 +744,10 @@ def test_lloyd_max_pins(orc):
     cbq, scq, cq, Lq, hq = orc.lloyd_max_g32(Wq, np.ones(64, np.float32), n_iter=10)
     assert Lq <= 1e-12 * hq[0]
     assert np.allclose(cbq, base, atol=2e-7)
+    # exact ties: u on the start codebook's midpoints -1/2, 0, 1/2 goes to the lower level
+    Wt = np.array([[[1.0, 0.5, 0.0, -0.5, -1.0, 0.25, -0.25, 0.75]]], np.float32)
+    sct, ct = orc.lloyd_max_assign(Wt, np.array(orc.LM_START, np.float32))
+    assert sct[0, 0, 0] == 1.0 and list(ct[0, 0]) == [3, 2, 1, 0, 0, 2, 1, 3]
     sc2, c2 = orc.lloyd_max_assign(W, cb)
     assert np.array_equal(sc2, sc) and np.array_equal(c2, c)
     z = orc.lloyd_max_g32(np.zeros((1, 2, 40), np.float32), np.ones(40, np.float32), n_iter=3)
