@@ -449,6 +449,7 @@ def main():
         next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
     next_rows["hessian"] = time_hessian(tq, step, pk)
     next_rows["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
+    next_rows["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
 
     # end to end through the public API from pinned host buffers
     e2e = None
@@ -602,6 +603,30 @@ def time_fp8(tq, step, pk, peak_tinst, reps=3):
             "frac": cee * FP8_INSTR_PER_CEE / 1e12 / peak_tinst,
             "note": f"first unit, {reps} launches of the whole call (amax + losses + pick + pack); "
                     f"{FP8_INSTR_PER_CEE} FP32-issue instructions per candidate-element evaluation"}
+
+
+def time_lloyd(tq, step, pk, n_iter=16, reps=3):
+    """Lloyd-Max 2-bit codebook (16 iterations) and codes on the first unit:
+    one HBM pass over W (+ the imatrix, L2-resident) per iteration, one for
+    the scales and one for the codes; bytes = (n_iter + 3) x W + scales +
+    packed codes."""
+    u = step.units[0]
+    m = step._m_for(u)
+    Ws = [s[1][0] for s in step.sets]
+    r = tq.tq_lloyd_max_g32(Ws[0], m, n_iter=n_iter)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(reps):
+        tq.tq_lloyd_max_g32(Ws[k % len(Ws)], m, n_iter=n_iter)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    wb = u.W.numel() * u.W.element_size()
+    nbytes = (n_iter + 3) * wb + r.scales.numel() * 4 * (n_iter + 3) + r.packed.numel()
+    return {"ms": ms, "iterations": n_iter, "bytes": nbytes, "GB/s": nbytes / (ms * 1e-3) / 1e9,
+            "frac": nbytes / (ms * 1e-3) / 1e9 / pk["hbm_gbs"],
+            "note": f"first unit, {reps} calls (binding allocations included); {n_iter} iterations, one pass each"}
 
 
 def time_hessian(tq, step, pk):

@@ -32,7 +32,8 @@ __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
+    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -55,6 +56,7 @@ EXPORTS = [
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
+    "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2",
 ]
 
 
@@ -131,6 +133,9 @@ def lib():
             "tq_imatrix": (i32, [Mp, P, i64, ctypes.c_float, i32, P, sz, P]),
             "tq_hessian": (i32, [Mp, P, i64, i64, ctypes.c_float, i32, P]),
             "tq_fp8_workspace_bytes": (sz, [Mp]),
+            "tq_lloyd_workspace_bytes": (sz, [Mp]),
+            "tq_lloyd_max_g32": (i32, [Mp, P, i64, i32, P, P, P, P, P, P, sz, P]),
+            "tq_dequant_lm2": (i32, [P, P, P, i64, i64, i64, P, i32, P]),
             "tq_search_fp8": (i32, [Mp, P, i64, i32, ctypes.c_double, ctypes.c_double, P, P, P, P, P, P, sz, P]),
             "tq_pack_fp8": (i32, [Mp, P, P, P]),
             "tq_dequant_fp8": (i32, [P, P, i64, i64, i64, P, i32, P]),
@@ -330,6 +335,50 @@ def tq_dequant_fp8(packed: torch.Tensor, scales: torch.Tensor, n_mat: int, O: in
         out = torch.empty((n_mat, O, I), dtype=out_dtype, device=packed.device)
     _check(lib().tq_dequant_fp8(_ptr(packed), _ptr(scales), n_mat, O, I, _ptr(out),
                                 _BF16 if out.dtype == torch.bfloat16 else _F32, _stream(stream)), "tq_dequant_fp8")
+    return out
+
+
+@dataclasses.dataclass
+class LloydResult:
+    codebook: torch.Tensor            # f32 [4]
+    scales: torch.Tensor              # f32 [n_mat, O, ceil(I/32)]
+    packed: Optional[torch.Tensor]    # u8 2-bit codes, 8 bytes per 32-weight group
+    loss: torch.Tensor                # f64 [1]
+    history: torch.Tensor             # f64 [n_iter + 1]
+
+
+LM_START = (-0.75, -0.25, 0.25, 0.75)   # the data-free Lloyd-Max levels of a uniform source on [-1, 1]
+
+
+def tq_lloyd_max_g32(W: torch.Tensor, m: torch.Tensor, n_iter: int = 16, start=LM_START, pack: bool = True,
+                     workspace: Optional[torch.Tensor] = None, stream=None) -> LloydResult:
+    """imatrix-weighted Lloyd-Max 2-bit codebook on absmax-normalised 32-weight
+    groups, shared by every matrix of W, and the 2-bit codes."""
+    d = _mat(W, "W")
+    _cuda(m, "m")
+    E, O, I = d.n_mat, d.rows, d.cols
+    dev = W.device
+    G = (I + 31) // 32
+    res = LloydResult(codebook=torch.tensor(start, dtype=torch.float32, device=dev),
+                      scales=torch.empty((E, O, G), dtype=torch.float32, device=dev),
+                      packed=torch.empty(E * O * G * 8, dtype=torch.uint8, device=dev) if pack else None,
+                      loss=torch.empty(1, dtype=torch.float64, device=dev),
+                      history=torch.empty(n_iter + 1, dtype=torch.float64, device=dev))
+    ws = int(lib().tq_lloyd_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=dev)
+    _check(lib().tq_lloyd_max_g32(ctypes.byref(d), _ptr(m), _m_stride(m), n_iter, _ptr(res.codebook),
+                                  _ptr(res.scales), _ptr(res.packed), _ptr(res.loss), _ptr(res.history),
+                                  _ptr(workspace), workspace.numel(), _stream(stream)), "tq_lloyd_max_g32")
+    return res
+
+
+def tq_dequant_lm2(packed: torch.Tensor, codebook: torch.Tensor, scales: torch.Tensor, n_mat: int, O: int, I: int,
+                   out_dtype=torch.float32, stream=None) -> torch.Tensor:
+    _cuda(packed, "packed")
+    out = torch.empty((n_mat, O, I), dtype=out_dtype, device=packed.device)
+    _check(lib().tq_dequant_lm2(_ptr(packed), _ptr(codebook), _ptr(scales), n_mat, O, I, _ptr(out),
+                                _BF16 if out_dtype == torch.bfloat16 else _F32, _stream(stream)), "tq_dequant_lm2")
     return out
 
 

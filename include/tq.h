@@ -287,6 +287,31 @@ tq_status tq_pack_fp8(const tq_mat* W, const float* scales, uint8_t* packed, tq_
 tq_status tq_dequant_fp8(const uint8_t* packed, const float* scales, int64_t n_mat, int64_t O, int64_t I,
                          void* out, int32_t out_dtype, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ Lloyd-Max 2-bit codebook
+ * A 4-level codebook for 2-bit weights fit to the data ("Phase 2:
+ * math-accuracy regression on tq3a-tq2e g32", Phase-2 candidate 1), read as:
+ * 32-weight groups with the absmax scale s; u = fl32(w / s) (0 for s = 0);
+ * one fp32 codebook c_0 < ... < c_3 shared by every matrix of the call,
+ * fit by n_iter Lloyd iterations that minimise sum m_j (w - s c_a)^2: each
+ * element to the nearest level (ties to the lower: u above the exact fp64
+ * midpoint moves up), each level to the (m s^2)-weighted mean of its elements
+ * (fp64 sums, rounded once to fp32; an empty level keeps its value).
+ * codebook: device f32 [4], the start on entry (sorted), the fit on return;
+ * scales: f32 [n_mat][O][ceil(I/32)] (out); packed: optional 2-bit codes, 8
+ * bytes per group (element k at bits 2 (k % 4) of byte k / 4; padding 0);
+ * loss: optional f64 [1], the weighted error of the final codebook; history:
+ * optional f64 [n_iter + 1], the error before each update and after the last.
+ * Deterministic (fixed partition and reduction order).  m: f32 [I] or
+ * [n_mat][I] (m_stride), 16-byte aligned.  workspace: >=
+ * tq_lloyd_workspace_bytes(W), 16-byte aligned.  n_iter in [0, 1000].
+ * tq_dequant_lm2: What = fl32(s c_a), dense [n_mat][O][I] fp32 or bf16. */
+size_t tq_lloyd_workspace_bytes(const tq_mat* W);
+tq_status tq_lloyd_max_g32(const tq_mat* W, const float* m, int64_t m_stride, int32_t n_iter, float* codebook,
+                           float* scales, uint8_t* packed, double* loss, double* history, void* workspace,
+                           size_t workspace_bytes, tq_stream_t stream);
+tq_status tq_dequant_lm2(const uint8_t* packed, const float* codebook, const float* scales, int64_t n_mat,
+                         int64_t O, int64_t I, void* out, int32_t out_dtype, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ Hessian
  * H[e] = alpha * sum_t X[e][t]^T X[e][t] (+ H[e] when accumulate): the
  * per-linear-input Hessian ([TT] pipeline table, step 1), fp32, from bf16

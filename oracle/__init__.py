@@ -50,6 +50,8 @@ def lib():
             "orc_e4m3_rne": (i32, [f32]),
             "orc_lloyd_max_g32": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, P, P, P, P, P]),
             "orc_lloyd_max_assign": (None, [P, i64, i64, i64, i64, i64, P, P, P]),
+            "orc_pack_lm2": (None, [P, i64, i64, P]),
+            "orc_dequant_lm2": (None, [P, i64, i64, P, P, P]),
             "orc_fp8_scale": (f32, [i32, f64, f64, i32, f32]),
             "orc_search_fp8": (None, [P, i64, i64, i64, i64, i64, P, i64, i32, f64, f64, P, P, P, P, P]),
             "orc_dequant_fp8": (None, [P, i64, i64, P, P]),
@@ -221,6 +223,20 @@ def lloyd_max_assign(W, codebook):
     c = np.empty((E, O, I), np.uint8)
     lib().orc_lloyd_max_assign(_p(W), E, O, I, I, O * I, _p(_f32(codebook)), _p(sc), _p(c))
     return sc, c
+
+
+def pack_lm2(codes) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8); I = codes.shape[-1]; rows = codes.size // I
+    out = np.empty(rows * ((I + 31) // 32) * 8, np.uint8)
+    lib().orc_pack_lm2(_p(codes), rows, I, _p(out))
+    return out
+
+
+def dequant_lm2(codes, scales, codebook) -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8); I = codes.shape[-1]; rows = codes.size // I
+    out = np.empty(codes.shape, np.float32)
+    lib().orc_dequant_lm2(_p(codes), rows, I, _p(_f32(scales)), _p(_f32(codebook)), _p(out))
+    return out
 
 
 def dequant_fp8(c, scales) -> np.ndarray:

@@ -712,6 +712,29 @@ ORC_API void orc_lloyd_max_assign(const float* W, int64_t n_mat, int64_t O, int6
                     lm_u(W[e * ms + o * ld + j], scales[(e * O + o) * G + j / 32]), codebook);
 }
 
+/* 2-bit codes (0..3) [rows][I] -> 8-byte records per 32-weight group:
+ * element k of a group at bits 2 (k % 4) of byte k / 4; padding code 0. */
+ORC_API void orc_pack_lm2(const uint8_t* codes, int64_t rows, int64_t I, uint8_t* out)
+{
+    const int64_t G = (I + 31) / 32;
+    memset(out, 0, (size_t)(rows * G * 8));
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j) {
+            int64_t k = j % 32, gi = r * G + j / 32;
+            out[gi * 8 + k / 4] |= (uint8_t)((codes[r * I + j] & 3) << (2 * (k % 4)));
+        }
+}
+
+/* What = fl32(s c_a) for codes [rows][I], group scales [rows][G32]. */
+ORC_API void orc_dequant_lm2(const uint8_t* codes, int64_t rows, int64_t I, const float* scales,
+                             const float* codebook, float* out)
+{
+    const int64_t G = (I + 31) / 32;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t j = 0; j < I; ++j)
+            out[r * I + j] = (float)((double)scales[r * G + j / 32] * (double)codebook[codes[r * I + j] & 3]);
+}
+
 /* ------------------------------------------------------------------ */
 /* Round-to-nearest with given scales (pack path)                      */
 /* ------------------------------------------------------------------ */

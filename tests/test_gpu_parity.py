@@ -628,3 +628,55 @@ def test_fp8_degenerate_and_rounding_edges():
         torch.cuda.synchronize()
         want = np.array([oracle.e4m3_rne(np.float32(w) / np.float32(scale)) for w in Wt.cpu().numpy().reshape(-1)])
         assert np.array_equal(p.cpu().numpy().reshape(-1), want.astype(np.uint8)), scale
+
+
+# ------------------------------------------------------------------ Lloyd-Max 2-bit codebook
+
+def _lloyd_check(W, m, n_iter, label):
+    r = tq.tq_lloyd_max_g32(W, m, n_iter=n_iter)
+    torch.cuda.synchronize()
+    W3 = W if W.dim() == 3 else W.unsqueeze(0)
+    Wh, mh = host32(W3), m.cpu().numpy()
+    cb, sc, c, L, hist = oracle.lloyd_max_g32(Wh, mh, n_iter=n_iter)
+    gcb = r.codebook.cpu().numpy()
+    # fp64 sums in another order: the fp32 codebook may differ in its last bit
+    assert np.all(np.abs(gcb - cb) <= 2 * np.spacing(np.abs(cb).astype(np.float32))), (label, gcb, cb)
+    assert np.allclose(r.history.cpu().numpy(), hist, rtol=1e-9, atol=0), label
+    assert np.array_equal(r.scales.cpu().numpy(), sc), label
+    # codes and dequant bit-exact for the GPU's codebook
+    sc2, c2 = oracle.lloyd_max_assign(Wh, gcb)
+    assert np.array_equal(r.packed.cpu().numpy(), oracle.pack_lm2(c2.reshape(-1, Wh.shape[2]))), label
+    E, O, I = Wh.shape
+    dq = tq.tq_dequant_lm2(r.packed, r.codebook, r.scales, E, O, I)
+    dqb = tq.tq_dequant_lm2(r.packed, r.codebook, r.scales, E, O, I, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle.dequant_lm2(c2.reshape(-1, I), sc2.reshape(-1, sc2.shape[2]), gcb).reshape(E, O, I)
+    assert np.array_equal(dq.cpu().numpy(), ref), label
+    assert torch.equal(dqb.cpu(), torch.from_numpy(ref).to(torch.bfloat16)), label
+    return r
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("n_iter", [0, 1, 12])
+def test_lloyd_max_matches_oracle(dtype, n_iter):
+    """Codebook, loss history, group scales, 2-bit codes and dequantized
+    weights against the oracle; ragged groups (I = 300), per-matrix and shared
+    imatrix."""
+    g = torch.Generator(device=DEV).manual_seed(n_iter + 3)
+    big = (synth.student_t((3, 37, 304), 4, g, DEV) * 0.02).to(dtype)
+    W = big[:, :, :300]
+    m = torch.stack([synth.random_imatrix(300, 9 + e, DEV) for e in range(3)])
+    _lloyd_check(W, m, n_iter, f"{dtype} {n_iter} per-matrix")
+    _lloyd_check(W, m[0], n_iter, f"{dtype} {n_iter} shared")
+
+
+def test_lloyd_max_edges():
+    """An all-zero matrix with a non-zero one, one column, exact ties on the
+    start codebook's midpoints (they go to the lower level)."""
+    W = torch.zeros((2, 8, 64), device=DEV)
+    W[1] = torch.randn((8, 64), device=DEV) * 0.01
+    _lloyd_check(W, torch.ones(64, device=DEV), 5, "zero matrix")
+    _lloyd_check(torch.randn((1, 5, 8), device=DEV)[:, :, :1], torch.ones(1, device=DEV), 3, "one column")
+    Wt = torch.tensor([[[1.0, 0.5, 0.0, -0.5, -1.0, 0.25, -0.25, 0.75] * 4]], device=DEV)
+    r = _lloyd_check(Wt, torch.ones(32, device=DEV), 0, "ties")
+    assert list(r.packed.cpu().numpy()[:2]) == [0b00011011, 0b11011000]
