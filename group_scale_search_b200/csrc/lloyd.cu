@@ -18,17 +18,19 @@
 // 2 (k % 4) of byte k / 4; padding past I is code 0); What = fl32(s c_a).
 //
 // B200 mapping: one HBM pass per iteration (k_lm_pass: 8 weights per thread,
-// one 16-byte bf16 load; per-level fp64 sums of omega u and omega and the
-// weighted squared error in registers, added over the block in a fixed
-// tree), then one block (k_lm_update) adds the block partials in block order
-// (deterministic) and writes the new codebook and the loss.  The group scales
+// one 16-byte bf16 load; u from a per-group reciprocal with a Markstein
+// correction; per-level fp64 sums of omega u and omega by predicated adds and
+// the sum of omega u^2 in registers, added over the block in a fixed tree),
+// then one block (k_lm_update) adds the block partials in block order
+// (deterministic), takes the loss sum omega (u - c_a)^2 from the sums and
+// writes the new codebook.  The group scales
 // come from one pass before (k_lm_scales: 4 threads per group, shuffle max).
 #include "walk.cuh"
 
 namespace tq {
 
 constexpr int LM_THREADS = 256;
-constexpr int LM_SUMS = 9;   // num[4], den[4], loss
+constexpr int LM_SUMS = 9;   // num[4] = sum omega u, den[4] = sum omega per level; sum omega u^2
 
 // Flat thread index -> (row, octet) with each row's octets padded to whole
 // groups (4 octets per group), so a group is 4 consecutive threads.
@@ -61,9 +63,27 @@ __global__ void k_lm_scales(const T* __restrict__ W, int64_t O, int64_t ld, int6
     }
 }
 
-__device__ __forceinline__ double lm_u(float w, float s) {
-    return s == 0.f ? 0.0 : static_cast<double>(__fdiv_rn(w, s));
-}
+// fl32(w / s) for the elements of one group: with r = fl32(1/s), the
+// correction q1 = fma(fma(-s, q0, w), r, q0) of q0 = w r is the correctly
+// rounded quotient when s, w, r, q0, the residual and the quotient are all
+// normal (Markstein): with s in [2^-60, 2^60] and |w| >= 2^-60, |u| lies in
+// [2^-120, 1] (|w| <= s: s is the group's max |w|).  Elsewhere (tiny w,
+// extreme or zero s) the IEEE division.
+struct LmDiv {
+    float s, r;
+    bool fast;
+    __device__ __forceinline__ explicit LmDiv(float s_) : s(s_) {
+        fast = s >= 8.673617379884035e-19f && s <= 1.152921504606847e18f;   // [2^-60, 2^60]
+        r = fast ? __frcp_rn(s) : 0.f;
+    }
+    __device__ __forceinline__ float u(float w) const {
+        if (fast && fabsf(w) >= 8.673617379884035e-19f) {
+            const float q0 = __fmul_rn(w, r);
+            return __fmaf_rn(__fmaf_rn(-s, q0, w), r, q0);
+        }
+        return s == 0.f ? 0.f : __fdiv_rn(w, s);
+    }
+};
 
 template <typename T>
 __global__ void __launch_bounds__(LM_THREADS)
@@ -92,22 +112,19 @@ k_lm_pass(const T* __restrict__ W, int64_t O, int64_t ld, int64_t ms, const floa
         mo.get(mv);
         const float s = __ldg(scales + (t >> 2));
         const double s2 = static_cast<double>(s) * static_cast<double>(s);
+        const LmDiv dv(s);
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
-            const double u = lm_u(w[i], s);
+            const double u = static_cast<double>(dv.u(w[i]));
             const double om = static_cast<double>(mv[i]) * s2;   // padding: m = 0
-            const bool g1 = u > m01, g2 = u > m12, g3 = u > m23;
-            const double ca = g3 ? c3 : (g2 ? c2 : (g1 ? c1 : c0));
-            const double ou = om * u, d = u - ca;
-            acc[0] += (!g1) ? ou : 0.0;
-            acc[1] += (g1 && !g2) ? ou : 0.0;
-            acc[2] += (g2 && !g3) ? ou : 0.0;
-            acc[3] += g3 ? ou : 0.0;
-            acc[4] += (!g1) ? om : 0.0;
-            acc[5] += (g1 && !g2) ? om : 0.0;
-            acc[6] += (g2 && !g3) ? om : 0.0;
-            acc[7] += g3 ? om : 0.0;
-            acc[8] = __fma_rn(om * d, d, acc[8]);
+            const double ou = om * u;
+            acc[8] = __fma_rn(ou, u, acc[8]);
+            // one predicated add per sum: the level's accumulators only
+            if (u > m12) {
+                if (u > m23) { acc[3] += ou; acc[7] += om; } else { acc[2] += ou; acc[6] += om; }
+            } else {
+                if (u > m01) { acc[1] += ou; acc[5] += om; } else { acc[0] += ou; acc[4] += om; }
+            }
         }
     }
     // block sum in a fixed order: warp butterfly, then warps in order
@@ -141,9 +158,16 @@ __global__ void k_lm_update(const double* __restrict__ part, int blocks, float* 
     }
     __syncthreads();
     if (threadIdx.x == 0) {
-        if (history) history[it] = sum[8];
+        // sum omega (u - c_a)^2 = sum omega u^2 - 2 sum_a c_a N_a + sum_a c_a^2 D_a
+        double L = sum[8];
+        for (int i = 0; i < 4; ++i) {
+            const double c = codebook[i];
+            L = L - 2.0 * c * sum[i] + c * c * sum[4 + i];
+        }
+        L = L > 0.0 ? L : 0.0;
+        if (history) history[it] = L;
         if (last) {
-            if (loss) *loss = sum[8];
+            if (loss) *loss = L;
         } else {
             for (int i = 0; i < 4; ++i)
                 if (sum[4 + i] > 0.0) codebook[i] = __double2float_rn(sum[i] / sum[4 + i]);
@@ -170,10 +194,10 @@ __global__ void k_lm_pack(const T* __restrict__ W, int64_t O, int64_t ld, int64_
             oc.load(W + e * ms + o * ld + j, n);
             float w[8];
             oc.get(w);
-            const float s = __ldg(scales + (t >> 2));
+            const LmDiv dv(__ldg(scales + (t >> 2)));
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const double u = lm_u(w[i], s);
+                const double u = static_cast<double>(dv.u(w[i]));
                 const unsigned a = (u > m01 ? 1u : 0u) + (u > m12 ? 1u : 0u) + (u > m23 ? 1u : 0u);
                 bits |= (i < n ? a : 0u) << (2 * i);
             }
