@@ -448,6 +448,7 @@ def main():
         next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
         next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
     next_rows["hessian"] = time_hessian(tq, step, pk)
+    next_rows["proxy_full_hessian"] = time_proxy_full(tq, step, pk)
     next_rows["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
     next_rows["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
 
@@ -665,6 +666,53 @@ def time_hessian(tq, step, pk):
             "note": f"first unit's activations [{T}, {I}] bf16, {reps} launches over {len(Xs)} input sets; "
                     "H fp32 both triangles; frac = roofline time (slower of flops / measured dense bf16 "
                     "burst and bytes / measured HBM) / measured time"}
+
+
+def time_proxy_full(tq, step, pk):
+    """tq_proxy_error_full (tr(E H E^T), tr(W H W^T) with H = X^T X, never
+    formed) on the first unit's search output and calibration activations,
+    rotating through the input sets.  Algorithmic work: the two products
+    X E^T and X W^T, 4 T O I flops per matrix (the kernel issues 8 T O I:
+    E enters as three exact bf16 pieces); peak: the measured dense bf16
+    figure."""
+    u, r = step.units[0], step.res[0]
+    fmt = tq.FORMATS[u.fmt]
+    sets = [(s[0][u.site], s[1][0]) for s in step.sets]
+    X0, W0 = sets[0]
+    if W0.dtype != torch.bfloat16 or X0.dtype != torch.bfloat16:
+        return {"skipped": "the tensor-core path takes bf16 weights and activations"}
+    E, O, I = W0.shape
+    T = X0.shape[-2]
+    flops = 4 * E * T * O * I
+    ws = torch.empty(tq.proxy_full_workspace_bytes(X0, W0), dtype=torch.uint8, device=W0.device)
+    out = (torch.empty(E, dtype=torch.float64, device=W0.device), torch.empty(E, dtype=torch.float64, device=W0.device))
+
+    def call(k):
+        X, W = sets[k % len(sets)]
+        tq.tq_proxy_error_full(X, W, r.packed, fmt, r.scales, r.zeros, r.global_scale, out=out, workspace=ws)
+
+    call(0)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    call(0)
+    b.record()
+    torch.cuda.synchronize()
+    reps = max(3, min(50, int(0.03 / max(a.elapsed_time(b) * 1e-3, 1e-6))))
+    a.record()
+    for k in range(reps):
+        call(k)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    tf = flops / (ms * 1e-3) / 1e12
+    peak = pk["bf16_tflops"]
+    del ws
+    return {"ms": ms, "T": T, "O": O, "I": I, "n_mat": E, "flops": flops, "TFLOP/s": tf, "peak": peak,
+            "bound": "tensor", "frac": tf / peak, "num/den": (out[0].sum() / out[1].sum()).item(),
+            "note": f"first unit, activations [{T}, {I}] bf16, {reps} calls over {len(sets)} input sets "
+                    "(E pieces + two GEMMs + reduce per call); flops = 4 T O I per matrix, "
+                    "frac of measured dense bf16 burst"}
 
 
 def time_gemv(tq, step, pk, B, reps=20):

@@ -33,7 +33,7 @@ __all__ = [
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
-    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -56,7 +56,8 @@ EXPORTS = [
     "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
-    "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2",
+    "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2", "tq_proxy_full_workspace_bytes",
+    "tq_proxy_error_full",
 ]
 
 
@@ -147,6 +148,8 @@ def lib():
             "tq_dequant": (i32, [P, i32, P, P, P, i64, i64, i64, P, i32, P]),
             "tq_proxy_workspace_bytes": (sz, [Mp, i32]),
             "tq_proxy_error": (i32, [Mp, P, i32, P, P, P, P, i64, P, P, P, sz, P]),
+            "tq_proxy_full_workspace_bytes": (sz, [Mp, Mp]),
+            "tq_proxy_error_full": (i32, [Mp, Mp, P, i32, P, P, P, P, P, P, sz, P]),
             "tq_sync": (i32, [P]),
             "tq_imatrix_static_capacity": (sz, []),
             "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
@@ -530,6 +533,31 @@ def tq_proxy_error(W: torch.Tensor, packed: torch.Tensor, fmt: int, scales: torc
                                 _ptr(global_scale), _ptr(m), _m_stride(m), _ptr(out[0]), _ptr(out[1]),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "tq_proxy_error")
     return out
+
+
+def tq_proxy_error_full(X: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, fmt: int, scales: torch.Tensor,
+                        zeros: Optional[torch.Tensor], global_scale: Optional[torch.Tensor],
+                        out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+                        workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """(num, den) fp64 per matrix with the full Hessian H = X^T X, never
+    formed: ||X (W - What)^T||_F^2 and ||X W^T||_F^2 on the tensor cores.
+    X: [T, I] or [n_mat, T, I] bf16 activations of each matrix's input;
+    W: [O, I] or [n_mat, O, I] bf16."""
+    dx, dw = _mat(X, "X"), _mat(W, "W")
+    if out is None:
+        out = (torch.empty(dw.n_mat, dtype=torch.float64, device=W.device),
+               torch.empty(dw.n_mat, dtype=torch.float64, device=W.device))
+    ws = int(lib().tq_proxy_full_workspace_bytes(ctypes.byref(dx), ctypes.byref(dw)))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=W.device)
+    _check(lib().tq_proxy_error_full(ctypes.byref(dx), ctypes.byref(dw), _ptr(packed), fmt, _ptr(scales),
+                                     _ptr(zeros), _ptr(global_scale), _ptr(out[0]), _ptr(out[1]),
+                                     _ptr(workspace), workspace.numel(), _stream(stream)), "tq_proxy_error_full")
+    return out
+
+
+def proxy_full_workspace_bytes(X: torch.Tensor, W: torch.Tensor) -> int:
+    return int(lib().tq_proxy_full_workspace_bytes(ctypes.byref(_mat(X, "X")), ctypes.byref(_mat(W, "W"))))
 
 
 def imatrix_workspace_bytes(X: torch.Tensor) -> int:

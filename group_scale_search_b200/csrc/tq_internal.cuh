@@ -32,6 +32,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 // True (and the count cleared) if a tq_hessian launch since the last call
 // gave up on a pipeline wait.
 bool hessian_take_timeouts();
+// The same for tq_proxy_error_full's GEMM pipeline.
+bool proxy_full_take_timeouts();
 
 inline int elem_bytes(int32_t dt) { return dt == TQ_BF16 ? 2 : (dt == TQ_F32 ? 4 : 0); }
 

@@ -342,9 +342,37 @@ tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, co
                          int64_t m_stride, double* num, double* den, void* workspace,
                          size_t workspace_bytes, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ proxy error, full Hessian
+ * Per matrix e ([TT] "Risks to measure: Precision", H = X^T X of the
+ * calibration activations, never formed):
+ *   num[e] = tr(E H E^T) = ||X E^T||_F^2,  E = W - What,
+ *   den[e] = tr(W H W^T) = ||X W^T||_F^2,
+ * on the tensor cores.  X: bf16 tq_mat of n_mat sites of T tokens x I
+ * columns; W: bf16 tq_mat [n_mat][O][I] (same I and n_mat); What: the fp32
+ * dequantized weights of `packed` (fmt, scales, zeros, global_scale as in
+ * tq_dequant).  E is rounded once to fp32 and split exactly into three bf16
+ * pieces, so the products are exact; Y = X E^T accumulates in fp32 and its
+ * squares add in fp64 in a fixed order (deterministic).  Error bound:
+ * |Y - X E^T| <= Delta = ((K/16 + 32) 2^-22 + 2^-23) (|X| |E|^T) elementwise,
+ * K = 3 ceil(I/64) 64 for num (ceil(I/64) 64 and no 2^-23 term for den), and
+ * |num - ||X E^T||^2| <= sum_{t,o} (2 |Y| + Delta) Delta.
+ * workspace: >= tq_proxy_full_workspace_bytes(X, W) (E's pieces, 6 bytes per
+ * weight with I padded to a multiple of 64, plus one fp64 per 128 x 256 tile
+ * of Y), 16-byte aligned, needs no initialisation.  Errors:
+ * TQ_ERR_INVALID_ARG for null/misaligned pointers, bad sizes or strides, a
+ * small workspace; TQ_ERR_UNSUPPORTED for fp32 X or W or an unknown format.
+ * A pipeline wait that exceeds its limit makes the kernel give up (the
+ * matrix's num/den become NaN) and the next tq_sync return TQ_ERR_CUDA. */
+size_t tq_proxy_full_workspace_bytes(const tq_mat* X, const tq_mat* W);
+tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uint8_t* packed, int32_t fmt,
+                              const void* scales, const uint8_t* zeros, const float* global_scale,
+                              double* num, double* den, void* workspace, size_t workspace_bytes,
+                              tq_stream_t stream);
+
 /* ------------------------------------------------------------------ testing aid
  * Synchronises `stream` and returns TQ_ERR_CUDA if it or an earlier kernel
- * failed (including a tq_hessian launch that gave up on a pipeline wait). */
+ * failed (including a tq_hessian or tq_proxy_error_full launch that gave up
+ * on a pipeline wait). */
 tq_status tq_sync(tq_stream_t stream);
 
 /* Self-test of the GPU's E2M1 conversion instructions, on which the NVFP4

@@ -138,6 +138,24 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     x = tq._Mat(ctypes.c_void_p(0x1008), 1, 0, 1, 256, 128, 128, 0)
     assert hs(ctypes.byref(x), fake, 128, 0, ctypes.c_float(1.0), 0, None) == 1
 
+    # proxy error with the full Hessian: (X, W, packed, fmt, scales, zeros, gs, num, den, ws, ws_bytes, stream)
+    pf = L.tq_proxy_error_full
+    xa = tq._Mat(fake, 1, 0, 1, 300, 200, 200, 0)
+    wa = tq._Mat(fake, 1, 0, 1, 300, 200, 200, 0)
+    needf = L.tq_proxy_full_workspace_bytes(ctypes.byref(xa), ctypes.byref(wa))
+    assert needf >= 300 * 3 * 256 * 2 + 2 * 3 * 2 * 8     # three bf16 pieces of E, I padded to 256; tile partials
+    args = (tq.INT3_G64_SYM, fake, None, None, fake, fake, fake, needf, None)
+    assert pf(ctypes.byref(xa), ctypes.byref(wa), None, *args) == 1
+    assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, 99, *args[1:]) == 2
+    assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, *args[:-2], needf - 8, None) == 1
+    assert b"workspace" in L.tq_last_error_string()
+    x32 = tq._Mat(fake, 0, 0, 1, 300, 200, 200, 0)
+    assert pf(ctypes.byref(x32), ctypes.byref(wa), fake, *args) == 2
+    xb = tq._Mat(fake, 1, 0, 1, 300, 208, 208, 0)            # I differs
+    assert pf(ctypes.byref(xb), ctypes.byref(wa), fake, *args) == 1
+    assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, tq.INT4_G128_ASYM, *args[1:]) == 1   # int4 needs zeros
+    assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, tq.NVFP4_G16, *args[1:]) == 1        # needs global scale
+
 
 def test_binding_refuses_cpu_tensors(tq):
     import torch

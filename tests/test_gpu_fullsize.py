@@ -181,3 +181,48 @@ def test_full_size_hessian(name):
     tq.tq_sync()
     d = np.diag(Hh).astype(np.float64) / T
     assert np.allclose(d, m.cpu().numpy().astype(np.float64), rtol=(T / 16 + 64) * 2.0 ** -22, atol=0)
+
+
+def test_full_size_proxy_full():
+    """tq_proxy_error_full on the dense int4-g128 4096 x 4096 workload (2048
+    calibration tokens), launched as bench.py launches it: the whole-matrix
+    call equals the sum of the calls on its 128-token blocks (each output tile
+    of X E^T is computed the same way in both) to fp64 rounding, and two
+    sampled 128-token x 256-row tiles match the oracle's tr(E H E^T),
+    tr(W H W^T) within the fp32 accumulation bound."""
+    wl = synth.make("c1", DEV)
+    u = [x for x in wl.units if x.timed][0]
+    X = wl.sites[u.site].X[0]
+    W = u.W
+    fmt = tq.FORMATS[u.fmt]
+    m = tq.tq_imatrix(X)[0]
+    res = tq.tq_search_groups(W, m, fmt)
+    num, den = tq.tq_proxy_error_full(X, W, res.packed, fmt, res.scales, res.zeros, res.global_scale)
+    tq.tq_sync()
+    T, I = X.shape
+    O = W.shape[1]
+    sn = sd = 0.0
+    for t0 in range(0, T, 128):
+        a, b = tq.tq_proxy_error_full(X[t0:t0 + 128], W, res.packed, fmt, res.scales, res.zeros, res.global_scale)
+        sn += a.item()
+        sd += b.item()
+    tq.tq_sync()
+    assert abs(num.item() - sn) <= 1e-12 * sn and abs(den.item() - sd) <= 1e-12 * sd
+    assert 0.0 < num.item() < den.item()
+    G = I // 128
+    for t0, o0 in [(0, 0), (T - 128, O - 256)]:
+        Wt = W[:, o0:o0 + 256]
+        sc, z = res.scales.view(1, O, G)[:, o0:o0 + 256], res.zeros.view(1, O, G)[:, o0:o0 + 256]
+        pk = res.packed.view(O, -1)[o0:o0 + 256]
+        a, b = tq.tq_proxy_error_full(X[t0:t0 + 128], Wt, pk, fmt, sc.contiguous(), z.contiguous(), None)
+        tq.tq_sync()
+        Wh = host32(Wt)[0]
+        codes = oracle.rtn_int4(Wh[None], sc.cpu().numpy(), z.cpu().numpy(), g=128)
+        What = oracle_dequant(fmt, codes, sc.cpu().numpy(), z.cpu().numpy())[0]
+        Xh = host32(X[t0:t0 + 128])
+        rn, rd = oracle.proxy_error_full(Wh, What, oracle.hessian(Xh))
+        X64, E64, W64 = Xh.astype(np.float64), Wh.astype(np.float64) - What, Wh.astype(np.float64)
+        for got, ref, M, K, extra in [(a.item(), rn, E64, 3 * I, 2.0 ** -23), (b.item(), rd, W64, I, 0.0)]:
+            D = ((K / 16 + 32) * 2.0 ** -22 + extra) * (np.abs(X64) @ np.abs(M).T)
+            bound = float(np.sum((2 * np.abs(X64 @ M.T) + D) * D))
+            assert abs(got - ref) <= bound + 1e-12 * ref, (t0, o0, got, ref, bound)

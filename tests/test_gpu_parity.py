@@ -680,3 +680,114 @@ def test_lloyd_max_edges():
     Wt = torch.tensor([[[1.0, 0.5, 0.0, -0.5, -1.0, 0.25, -0.25, 0.75] * 4]], device=DEV)
     r = _lloyd_check(Wt, torch.ones(32, device=DEV), 0, "ties")
     assert list(r.packed.cpu().numpy()[:2]) == [0b00011011, 0b11011000]
+
+
+# ------------------------------------------------------------------ proxy error, full Hessian
+
+def _pf_bound(Xh, Eh, K, extra):
+    """Bound on |GPU - exact| for ||X E^T||_F^2 with Y = X E^T accumulated in
+    fp32 over K (padded) columns: elementwise |dY| <= D = ((K/16 + 32) 2^-22 +
+    extra) (|X| |E|^T), so the sum of squares moves by at most
+    sum (2 |Y| + D) D."""
+    X64, E64 = Xh.astype(np.float64), Eh.astype(np.float64)
+    D = ((K / 16 + 32) * 2.0 ** -22 + extra) * (np.abs(X64) @ np.abs(E64).T)
+    return float(np.sum((2 * np.abs(X64 @ E64.T) + D) * D))
+
+
+def _pf_oracle(fmt, W3, res):
+    """The oracle's What from the search's own parameters (its RTN + pack,
+    checked equal to the GPU's records, then its dequant)."""
+    Wh = host32(W3)
+    gs = res.scales.cpu().numpy()
+    z = res.zeros.cpu().numpy() if res.zeros is not None else None
+    g = res.global_scale.cpu().numpy() if res.global_scale is not None else None
+    packed_ref, codes = oracle_packed(fmt, Wh, gs, z, g)
+    assert np.array_equal(res.packed.cpu().numpy(), packed_ref)
+    return Wh, oracle_dequant(fmt, codes, gs, z, g)
+
+
+def _pf_inputs(E, T, O, I, seed, onehot):
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    ld = (I + 7) // 8 * 8
+    W = (synth.student_t((E, O, ld), 4, g, DEV) * 0.02).bfloat16()[:, :, :I]
+    if onehot:   # one 2^k-scaled unit per token: every entry of Y is one product, exact in fp32
+        rng = np.random.default_rng(seed)
+        Xh = np.zeros((E, T, ld), np.float32)
+        cols = rng.integers(0, I, size=(E, T))
+        Xh[np.arange(E)[:, None], np.arange(T)[None, :], cols] = 2.0 ** rng.integers(-3, 4, size=(E, T))
+        X = torch.from_numpy(Xh).to(DEV).bfloat16()[:, :, :I]
+    else:
+        c = torch.exp(torch.randn((ld,), generator=g, device=DEV))   # LogNormal(0, 1) column scales
+        X = (torch.randn((E, T, ld), generator=g, device=DEV) * c).bfloat16()[:, :, :I]
+    return X, W
+
+
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("E,T,O,I", [(2, 300, 300, 200), (1, 128, 256, 64), (1, 1, 7, 16), (1, 257, 513, 1030)])
+def test_proxy_full_onehot_exact(fmt, E, T, O, I):
+    """Tokens that are scaled unit vectors: every entry of X E^T is a single
+    product, so the three bf16 pieces of E must add back to E exactly (a lost
+    piece moves num by ~2^-16 relative).  num within the fp32 rounding of E
+    (2^-23 relative), den exact; ragged T, O and I; several tiles and K stages."""
+    X, W = _pf_inputs(E, T, O, I, 11 * T + I, onehot=True)
+    m = synth.random_imatrix(I, 5, DEV)
+    res = _run(fmt, W, m)
+    num, den = tq.tq_proxy_error_full(X, W, res.packed, fmt, res.scales, res.zeros, res.global_scale)
+    tq.tq_sync()
+    Wh, What = _pf_oracle(fmt, W, res)
+    Xh = host32(X)
+    for e in range(E):
+        rn, rd = oracle.proxy_error_full(Wh[e], What[e], oracle.hessian(Xh[e]))
+        assert abs(num[e].item() - rn) <= 2.0 ** -23 * rn + 1e-300, (e, num[e].item(), rn)
+        assert abs(den[e].item() - rd) <= 1e-13 * rd, (e, den[e].item(), rd)
+
+
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("E,T,O,I", [(2, 300, 300, 320), (1, 700, 600, 1000), (3, 129, 257, 100)])
+def test_proxy_full_matches_oracle(fmt, E, T, O, I):
+    """Random activations with LogNormal column scales: num and den within the
+    fp32 accumulation bound of the oracle's fp64 tr(E H E^T), tr(W H W^T)
+    (H = the oracle's X^T X); per-matrix sites; deterministic on a repeat;
+    0 < num < den."""
+    X, W = _pf_inputs(E, T, O, I, 7 * T + I, onehot=False)
+    m = tq.tq_imatrix(X)
+    res = _run(fmt, W, m)
+    num, den = tq.tq_proxy_error_full(X, W, res.packed, fmt, res.scales, res.zeros, res.global_scale)
+    num2, den2 = tq.tq_proxy_error_full(X, W, res.packed, fmt, res.scales, res.zeros, res.global_scale)
+    tq.tq_sync()
+    assert torch.equal(num, num2) and torch.equal(den, den2)
+    Wh, What = _pf_oracle(fmt, W, res)
+    Xh = host32(X)
+    Ip = (I + 63) // 64 * 64
+    for e in range(E):
+        rn, rd = oracle.proxy_error_full(Wh[e], What[e], oracle.hessian(Xh[e]))
+        Eh = Wh[e].astype(np.float64) - What[e].astype(np.float64)
+        assert abs(num[e].item() - rn) <= _pf_bound(Xh[e], Eh, 3 * Ip, 2.0 ** -23) + 1e-12 * rn, (e, num[e].item(), rn)
+        assert abs(den[e].item() - rd) <= _pf_bound(Xh[e], Wh[e], Ip, 0.0) + 1e-12 * rd, (e, den[e].item(), rd)
+        assert 0.0 < num[e].item() < den[e].item()
+
+
+def test_proxy_full_exact_weights_and_strides():
+    """What == W (every weight on the grid: int4 codes times a power-of-two
+    scale) gives num = 0 exactly; padded rows and a matrix stride for X and W."""
+    E, T, O, I = 2, 200, 96, 256
+    g = torch.Generator(device=DEV).manual_seed(3)
+    q = torch.randint(0, 16, (E, O, I), generator=g, device=DEV)
+    Wf = ((q - 8).float() * 2.0 ** -6)
+    Wb = torch.zeros((E, O + 1, I + 8), dtype=torch.bfloat16, device=DEV)
+    Wb[:, :O, :I] = Wf.bfloat16()
+    W = Wb[:, :O, :I]
+    Xb = torch.randn((E, T + 5, I + 16), generator=g, device=DEV).bfloat16()
+    X = Xb[:, :T, :I]
+    fmt = tq.INT4_G128_ASYM
+    G = I // 128
+    scales = torch.full((E, O, G), 2.0 ** -6, device=DEV)
+    zeros = torch.full((E, O, G), 8, dtype=torch.uint8, device=DEV)
+    packed = tq.tq_pack(W, fmt, scales, zeros, None)
+    num, den = tq.tq_proxy_error_full(X, W, packed, fmt, scales, zeros, None)
+    tq.tq_sync()
+    assert torch.all(num == 0)
+    Xh, Wh = host32(X), host32(W)
+    for e in range(E):
+        rd = oracle.proxy_error_full(Wh[e], Wh[e], oracle.hessian(Xh[e]))[1]
+        assert abs(den[e].item() - rd) <= _pf_bound(Xh[e], Wh[e], I, 0.0) + 1e-12 * rd
