@@ -672,9 +672,8 @@ def time_proxy_full(tq, step, pk):
     """tq_proxy_error_full (tr(E H E^T), tr(W H W^T) with H = X^T X, never
     formed) on the first unit's search output and calibration activations,
     rotating through the input sets.  Algorithmic work: the two products
-    X E^T and X W^T, 4 T O I flops per matrix (the kernel issues 8 T O I:
-    E enters as three exact bf16 pieces); peak: the measured dense bf16
-    figure."""
+    X E^T and X W^T, 4 T O I flops per matrix (the kernel issues 6 T O I:
+    E enters as two bf16 pieces); peak: the measured dense bf16 figure."""
     u, r = step.units[0], step.res[0]
     fmt = tq.FORMATS[u.fmt]
     sets = [(s[0][u.site], s[1][0]) for s in step.sets]
@@ -711,7 +710,7 @@ def time_proxy_full(tq, step, pk):
     return {"ms": ms, "T": T, "O": O, "I": I, "n_mat": E, "flops": flops, "TFLOP/s": tf, "peak": peak,
             "bound": "tensor", "frac": tf / peak, "num/den": (out[0].sum() / out[1].sum()).item(),
             "note": f"first unit, activations [{T}, {I}] bf16, {reps} calls over {len(sets)} input sets "
-                    "(E pieces + two GEMMs + reduce per call); flops = 4 T O I per matrix, "
+                    "(E pieces + one fused two-product GEMM + reduce per call); flops = 4 T O I per matrix, "
                     "frac of measured dense bf16 burst"}
 
 

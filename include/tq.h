@@ -347,17 +347,18 @@ tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, co
  * calibration activations, never formed):
  *   num[e] = tr(E H E^T) = ||X E^T||_F^2,  E = W - What,
  *   den[e] = tr(W H W^T) = ||X W^T||_F^2,
- * on the tensor cores.  X: bf16 tq_mat of n_mat sites of T tokens x I
- * columns; W: bf16 tq_mat [n_mat][O][I] (same I and n_mat); What: the fp32
- * dequantized weights of `packed` (fmt, scales, zeros, global_scale as in
- * tq_dequant).  E is rounded once to fp32 and split exactly into three bf16
- * pieces, so the products are exact; Y = X E^T accumulates in fp32 and its
+ * on the tensor cores, one pass over X for both products.  X: bf16 tq_mat of
+ * n_mat sites of T tokens x I columns; W: bf16 tq_mat [n_mat][O][I] (same I
+ * and n_mat); What: the fp32 dequantized weights of `packed` (fmt, scales,
+ * zeros, global_scale as in tq_dequant).  E is rounded once to fp32 and
+ * carried as two bf16 pieces E1 + E2 (16 significant bits, relative error at
+ * most 2^-16); the products are exact, Y = X E^T accumulates in fp32 and its
  * squares add in fp64 in a fixed order (deterministic).  Error bound:
- * |Y - X E^T| <= Delta = ((K/16 + 32) 2^-22 + 2^-23) (|X| |E|^T) elementwise,
- * K = 3 ceil(I/64) 64 for num (ceil(I/64) 64 and no 2^-23 term for den), and
+ * |Y - X E^T| <= Delta = ((K/16 + 32) 2^-22 + 2^-15) (|X| |E|^T) elementwise,
+ * K = 2 ceil(I/64) 64 for num (ceil(I/64) 64 and no 2^-15 term for den), and
  * |num - ||X E^T||^2| <= sum_{t,o} (2 |Y| + Delta) Delta.
- * workspace: >= tq_proxy_full_workspace_bytes(X, W) (E's pieces, 6 bytes per
- * weight with I padded to a multiple of 64, plus one fp64 per 128 x 256 tile
+ * workspace: >= tq_proxy_full_workspace_bytes(X, W) (E's pieces, 4 bytes per
+ * weight with I padded to a multiple of 64, plus two fp64 per 128 x 256 tile
  * of Y), 16-byte aligned, needs no initialisation.  Errors:
  * TQ_ERR_INVALID_ARG for null/misaligned pointers, bad sizes or strides, a
  * small workspace; TQ_ERR_UNSUPPORTED for fp32 X or W or an unknown format.

@@ -222,7 +222,7 @@ def test_full_size_proxy_full():
         Xh = host32(X[t0:t0 + 128])
         rn, rd = oracle.proxy_error_full(Wh, What, oracle.hessian(Xh))
         X64, E64, W64 = Xh.astype(np.float64), Wh.astype(np.float64) - What, Wh.astype(np.float64)
-        for got, ref, M, K, extra in [(a.item(), rn, E64, 3 * I, 2.0 ** -23), (b.item(), rd, W64, I, 0.0)]:
+        for got, ref, M, K, extra in [(a.item(), rn, E64, 2 * I, 2.0 ** -15), (b.item(), rd, W64, I, 0.0)]:
             D = ((K / 16 + 32) * 2.0 ** -22 + extra) * (np.abs(X64) @ np.abs(M).T)
             bound = float(np.sum((2 * np.abs(X64 @ M.T) + D) * D))
             assert abs(got - ref) <= bound + 1e-12 * ref, (t0, o0, got, ref, bound)

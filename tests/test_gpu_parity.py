@@ -726,9 +726,10 @@ def _pf_inputs(E, T, O, I, seed, onehot):
 @pytest.mark.parametrize("E,T,O,I", [(2, 300, 300, 200), (1, 128, 256, 64), (1, 1, 7, 16), (1, 257, 513, 1030)])
 def test_proxy_full_onehot_exact(fmt, E, T, O, I):
     """Tokens that are scaled unit vectors: every entry of X E^T is a single
-    product, so the three bf16 pieces of E must add back to E exactly (a lost
-    piece moves num by ~2^-16 relative).  num within the fp32 rounding of E
-    (2^-23 relative), den exact; ragged T, O and I; several tiles and K stages."""
+    product, exact in fp32, so num differs from the oracle only by E's two-piece
+    representation (at most 2^-16 relative per weight, 2^-15 on a square; a
+    lost piece moves it by ~2^-8) and den is exact; ragged T, O and I; several
+    tiles and passes around both rings."""
     X, W = _pf_inputs(E, T, O, I, 11 * T + I, onehot=True)
     m = synth.random_imatrix(I, 5, DEV)
     res = _run(fmt, W, m)
@@ -738,7 +739,7 @@ def test_proxy_full_onehot_exact(fmt, E, T, O, I):
     Xh = host32(X)
     for e in range(E):
         rn, rd = oracle.proxy_error_full(Wh[e], What[e], oracle.hessian(Xh[e]))
-        assert abs(num[e].item() - rn) <= 2.0 ** -23 * rn + 1e-300, (e, num[e].item(), rn)
+        assert abs(num[e].item() - rn) <= 2.0 ** -14 * rn + 1e-300, (e, num[e].item(), rn)
         assert abs(den[e].item() - rd) <= 1e-13 * rd, (e, den[e].item(), rd)
 
 
@@ -762,7 +763,7 @@ def test_proxy_full_matches_oracle(fmt, E, T, O, I):
     for e in range(E):
         rn, rd = oracle.proxy_error_full(Wh[e], What[e], oracle.hessian(Xh[e]))
         Eh = Wh[e].astype(np.float64) - What[e].astype(np.float64)
-        assert abs(num[e].item() - rn) <= _pf_bound(Xh[e], Eh, 3 * Ip, 2.0 ** -23) + 1e-12 * rn, (e, num[e].item(), rn)
+        assert abs(num[e].item() - rn) <= _pf_bound(Xh[e], Eh, 2 * Ip, 2.0 ** -15) + 1e-12 * rn, (e, num[e].item(), rn)
         assert abs(den[e].item() - rd) <= _pf_bound(Xh[e], Wh[e], Ip, 0.0) + 1e-12 * rd, (e, den[e].item(), rd)
         assert 0.0 < num[e].item() < den[e].item()
 
