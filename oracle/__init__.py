@@ -57,6 +57,7 @@ def lib():
             "orc_dequant_fp8": (None, [P, i64, i64, P, P]),
             "orc_hessian_entry": (f64, [P, i64, i64, i64, i64]),
             "orc_proxy_error_full": (None, [P, P, i64, i64, P, P, P]),
+            "orc_gptq_sweep": (None, [P, i64, i64, i32, i32, P, P, P, i64, P, P]),
             "orc_sym_stage1_ratio": (f32, [i32, f64, f64, i32]),
             "orc_sym_stage2_ratio": (f32, [i32, i32, f64, f64, i32, i32]),
             "orc_sym_loss": (f64, [P, P, i32, f32, P]),
@@ -165,6 +166,23 @@ def proxy_error_full(W, What, H) -> Tuple[float, float]:
     num = ctypes.c_double(); den = ctypes.c_double()
     lib().orc_proxy_error_full(_p(W), _p(What), O, I, _p(H), ctypes.byref(num), ctypes.byref(den))
     return num.value, den.value
+
+
+def gptq_sweep(W, fmt: int, scales, zeros, U, g=None):
+    """GPTQ/LDLQ column sweep of W [rows, I] (or [n, O, I], one U for all)
+    with fixed group scales (and zeros): fmt 3 = int3-g64, 4 = int4 (g = 128
+    by default, or 64).  U: fp32 [I, I] upper factor with H^-1 = U^T U.
+    Returns (codes int8 [.., I], loss fp64 [rows])."""
+    W = _f32(W)
+    I = W.shape[-1]; rows = W.size // I
+    g = g or (64 if fmt == 3 else 128)
+    U = _f32(U)
+    codes = np.empty(W.shape, np.int8)
+    loss = np.empty(rows, np.float64)
+    z = None if zeros is None else np.ascontiguousarray(zeros, np.uint8)
+    lib().orc_gptq_sweep(_p(W), rows, I, int(fmt), int(g), _p(_f32(scales)), _p(z), _p(U), U.shape[-1],
+                         _p(codes), _p(loss))
+    return codes, loss
 
 
 def e4m3_rne(y: float) -> int:

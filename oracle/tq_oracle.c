@@ -15,8 +15,9 @@
  *           both weighted by the activation imatrix; results bullet 2: the
  *           "64/32" grid.
  *  [TT]     "Quantize on TT cards: CUDA-free GPTQ/LDLQ bfp4 pipeline" (tt-stack
- *           issue #67), pipeline table step 1 (H = sum X^T X) and "Risks to
- *           measure: Precision" (proxy error tr(E H E^T)/tr(W H W^T)).
+ *           issue #67), pipeline table step 1 (H = sum X^T X), step 3 (the
+ *           GPTQ/LDLQ column sweep) and "Risks to measure: Precision" (proxy
+ *           error tr(E H E^T)/tr(W H W^T); fp32 host propagation).
  *  [NVFP4]  "Nemotron-Cascade-2-30B-A3B-NVFP4" model card, Quantization Recipe
  *           table (NVFP4 group 16, MSE-calibrated static block scales) and the
  *           Calibration line (weight-MSE calibration).
@@ -875,6 +876,61 @@ ORC_API void orc_dequant_int4(const uint8_t* q, int64_t rows, int64_t I, const f
             int64_t gi = r * G + j / g;
             out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));
         }
+}
+
+/* GPTQ/LDLQ column sweep ([TT] pipeline table, step 3: serial rounding,
+ * with the rounding error of each column propagated to the later columns
+ * through the inverse Hessian's triangular factor), with the group scales
+ * (and zero-points) fixed by the search.  U: upper triangular, H^-1 = U^T U
+ * (fp32, I x I rows of ldu; only the upper triangle is read; U_ii > 0).  Per
+ * row, for each column i in order:
+ *   code of the current w_i under its group's scale (the format's RTN:
+ *   rtn_code, or the int4 zero-point form of orc_rtn_int4), dequantized
+ *   value what_i = fl32(s v) / fl32(s (q - z)),
+ *   e_i = (w_i - what_i) / U_ii in fp32,
+ *   w_j <- w_j - e_i U_ij for every later column j, one fused multiply-add
+ *   (fmaf) each.
+ * Precision (reading): fp32, the page's host propagator ("cpu-float32").
+ * The page's 128-column blocks and its propagation matmul
+ * W[:, rest] -= E U[blk, rest] reorder nothing when every weight's updates
+ * are applied in column order, as here.  loss[r] = sum_i e_i^2 in fp64,
+ * which in exact arithmetic is (w - What) H (w - What)^T for the row.
+ * fmt: 3 = int3 (codes v in [-4, 3], g = 64), 4 = int4 (codes q in [0, 15],
+ * zeros per group, g = 128 or 64).  codes: int8 [rows][I]. */
+ORC_API void orc_gptq_sweep(const float* W, int64_t rows, int64_t I, int fmt, int g, const float* scales,
+                            const uint8_t* zeros, const float* U, int64_t ldu, int8_t* codes, double* loss)
+{
+    const int64_t G = (I + g - 1) / g;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        float* w = (float*)malloc((size_t)I * sizeof(float));
+        memcpy(w, W + r * I, (size_t)I * sizeof(float));
+        double L = 0.0;
+        for (int64_t i = 0; i < I; ++i) {
+            const float s = scales[r * G + i / g];
+            double code;
+            float what;
+            if (fmt == 3) {
+                code = rtn_code(w[i], s, -4.0, 3.0);
+                what = (float)((double)s * code);
+            } else {
+                const int z = zeros[r * G + i / g];
+                if (s == 0.0f) code = (double)z;
+                else {
+                    code = nearbyint((double)(w[i] / s)) + (double)z;
+                    if (code < 0.0) code = 0.0;
+                    if (code > 15.0) code = 15.0;
+                }
+                what = (float)((double)s * (code - (double)z));
+            }
+            codes[r * I + i] = (int8_t)code;
+            const float e = (w[i] - what) / U[i * ldu + i];
+            L += (double)e * (double)e;
+            for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);
+        }
+        loss[r] = L;
+        free(w);
+    }
 }
 
 ORC_API void orc_dequant_nvfp4(const uint8_t* c, int64_t rows, int64_t mat_rows, int64_t I,

@@ -46,6 +46,13 @@ MUTANTS = {
     "fp8_loss_unweighted": ("L += (double)me[j] * (d * d);", "L += (d * d);"),
     "lloyd_ties_up": ("if (u > ((double)c[i] + (double)c[i + 1]) / 2.0) a = i + 1;", "if (u >= ((double)c[i] + (double)c[i + 1]) / 2.0) a = i + 1;"),
     "lloyd_scale_not_squared": ("double om = (double)m[e * m_stride + j] * (double)s * (double)s;", "double om = (double)m[e * m_stride + j] * (double)s;"),
+    "gptq_update_sign": ("for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);",
+                         "for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(e, U[i * ldu + j], w[j]);"),
+    "gptq_transposed_factor": ("for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);",
+                               "for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[j * ldu + i], w[j]);"),
+    "gptq_no_diagonal_division": ("const float e = (w[i] - what) / U[i * ldu + i];", "const float e = (w[i] - what);"),
+    "gptq_skips_next_column": ("for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);",
+                               "for (int64_t j = i + 2; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }
