@@ -449,6 +449,7 @@ def main():
         next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
     next_rows["hessian"] = time_hessian(tq, step, pk)
     next_rows["proxy_full_hessian"] = time_proxy_full(tq, step, pk)
+    next_rows["gptq_sweep"] = time_gptq(tq, step, peak_tinst)
     next_rows["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
     next_rows["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
 
@@ -712,6 +713,46 @@ def time_proxy_full(tq, step, pk):
             "note": f"first unit, activations [{T}, {I}] bf16, {reps} calls over {len(sets)} input sets "
                     "(E pieces + one fused two-product GEMM + reduce per call); flops = 4 T O I per matrix, "
                     "frac of measured dense bf16 burst"}
+
+
+def time_gptq(tq, step, peak_tinst, reps=3):
+    """tq_gptq_sweep (GPTQ/LDLQ column sweep with the search's scales held
+    fixed) on the first unit, with the factor U (H^-1 = U^T U) of its first
+    matrix's calibration Hessian, damped by 1 % of the mean diagonal (fp64
+    Cholesky and inverse by the library, before the timed calls; one factor
+    for every matrix of a batch).  Algorithmic work: the propagation's fused
+    multiply-adds, I (I - 1) / 2 per row, against the FP32 issue peak."""
+    u, r = step.units[0], step.res[0]
+    fmt = tq.FORMATS[u.fmt]
+    if fmt == tq.NVFP4_G16:
+        return {"skipped": "the sweep is built for the integer formats"}
+    X = step.sets[0][0][u.site][0]
+    W = step.sets[0][1][0]
+    E, O, I = W.shape
+    H = X.double().T @ X.double()
+    H += 0.01 * H.diagonal().mean() * torch.eye(I, device=H.device, dtype=torch.float64)
+    U = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H)), upper=True).float().contiguous()
+    del H
+    ws = torch.empty(tq.gptq_workspace_bytes(W), dtype=torch.uint8, device=W.device)
+    out = (torch.empty((E, O, I), dtype=torch.int8, device=W.device),
+           torch.empty((E, O), dtype=torch.float64, device=W.device))
+    Ws = [s[1][0] for s in step.sets]
+    tq.tq_gptq_sweep(W, fmt, r.scales, r.zeros, U, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for k in range(reps):
+        tq.tq_gptq_sweep(Ws[k % len(Ws)], fmt, r.scales, r.zeros, U, out=out, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    fma = E * O * I * (I - 1) / 2
+    achieved = fma / (ms * 1e-3) / 1e12
+    del ws, out, U
+    return {"ms": ms, "n_mat": E, "O": O, "I": I, "fma": fma, "achieved_tinst": achieved,
+            "frac": achieved / peak_tinst, "weights_per_s": E * O * I / (ms * 1e-3),
+            "note": f"first unit, {reps} calls over rotating weight copies; fused multiply-adds of the "
+                    "propagation (I (I-1)/2 per row) vs the FP32 issue peak; the serial rounding is not counted"}
 
 
 def time_gemv(tq, step, pk, B, reps=20):

@@ -33,7 +33,7 @@ __all__ = [
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
-    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -57,7 +57,7 @@ EXPORTS = [
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
     "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2", "tq_proxy_full_workspace_bytes",
-    "tq_proxy_error_full",
+    "tq_proxy_error_full", "tq_gptq_workspace_bytes", "tq_gptq_sweep",
 ]
 
 
@@ -149,6 +149,8 @@ def lib():
             "tq_proxy_workspace_bytes": (sz, [Mp, i32]),
             "tq_proxy_error": (i32, [Mp, P, i32, P, P, P, P, i64, P, P, P, sz, P]),
             "tq_proxy_full_workspace_bytes": (sz, [Mp, Mp]),
+            "tq_gptq_workspace_bytes": (sz, [Mp]),
+            "tq_gptq_sweep": (i32, [Mp, i32, P, P, P, i64, i64, P, P, P, sz, P]),
             "tq_proxy_error_full": (i32, [Mp, Mp, P, i32, P, P, P, P, P, P, sz, P]),
             "tq_sync": (i32, [P]),
             "tq_imatrix_static_capacity": (sz, []),
@@ -554,6 +556,35 @@ def tq_proxy_error_full(X: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, 
                                      _ptr(zeros), _ptr(global_scale), _ptr(out[0]), _ptr(out[1]),
                                      _ptr(workspace), workspace.numel(), _stream(stream)), "tq_proxy_error_full")
     return out
+
+
+def tq_gptq_sweep(W: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Optional[torch.Tensor], U: torch.Tensor,
+                  out: Optional[Tuple[torch.Tensor, Optional[torch.Tensor]]] = None, want_loss: bool = True,
+                  workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """GPTQ/LDLQ column sweep of W ([O, I] or [n_mat, O, I]) with the given
+    group scales (and zeros) held fixed.  U: fp32 [I, I] (one factor for all
+    matrices) or [n_mat, I, I] upper triangular with H^-1 = U^T U (unit column
+    stride).  Returns (codes int8 [n_mat, O, I], per-row loss fp64 [n_mat, O])."""
+    d = _mat(W, "W")
+    _cuda(U, "U")
+    if U.dtype != torch.float32 or U.stride(-1) != 1 or U.dim() not in (2, 3):
+        raise ValueError("U must be float32 [I, I] or [n_mat, I, I] with unit column stride")
+    E, O, I = d.n_mat, d.rows, d.cols
+    ums = U.stride(0) if U.dim() == 3 and U.shape[0] > 1 else 0
+    if out is None:
+        out = (torch.empty((E, O, I), dtype=torch.int8, device=W.device),
+               torch.empty((E, O), dtype=torch.float64, device=W.device) if want_loss else None)
+    ws = int(lib().tq_gptq_workspace_bytes(ctypes.byref(d)))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=W.device)
+    _check(lib().tq_gptq_sweep(ctypes.byref(d), fmt, _ptr(scales), _ptr(zeros), _ptr(U), U.stride(-2), ums,
+                               _ptr(out[0]), _ptr(out[1]), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "tq_gptq_sweep")
+    return out
+
+
+def gptq_workspace_bytes(W: torch.Tensor) -> int:
+    return int(lib().tq_gptq_workspace_bytes(ctypes.byref(_mat(W, "W"))))
 
 
 def proxy_full_workspace_bytes(X: torch.Tensor, W: torch.Tensor) -> int:

@@ -370,6 +370,35 @@ tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uint8_t* p
                               double* num, double* den, void* workspace, size_t workspace_bytes,
                               tq_stream_t stream);
 
+/* ------------------------------------------------------------------ GPTQ/LDLQ column sweep
+ * [TT] pipeline table, step 3: serial rounding with the rounding error of each
+ * column propagated to the later columns through the inverse Hessian's
+ * triangular factor, with the group scales (and zero-points) of a search held
+ * fixed.  U: fp32 upper triangular factor with H^-1 = U^T U, rows of ldu >= I
+ * elements, u_mat_stride elements between matrices (0: one factor for every
+ * matrix); only its upper triangle is read; U_ii > 0 (the caller's Cholesky
+ * of the damped, inverted H).  Per row, for each column i in order:
+ *   code of the current w_i under its group's scale (round half to even of
+ *   the IEEE fp32 quotient, clamped; int3 v in [-4, 3], int4 q in [0, 15]
+ *   with the group's zero-point; a zero scale gives v = 0 / q = z),
+ *   What_i = fl32(s v) or fl32(s (q - z)),
+ *   e_i = (w_i - What_i) / U_ii (fp32),
+ *   w_j <- fma(-e_i, U_ij, w_j) for every j > i (fp32, in column order).
+ * Deterministic and independent of the tiling: results are bitwise those of
+ * the unblocked sweep.  W: bf16 or fp32 tq_mat [n_mat][O][I]; fmt:
+ * TQ_INT3_G64_SYM, TQ_INT4_G128_ASYM or TQ_INT4_G64_ASYM; scales f32 and
+ * zeros u8 [n_mat][O][ceil(I/g)] as tq_search_groups writes them.  codes:
+ * int8 [n_mat][O][I] (int3: v; int4: q), the input of tq_pack_codes.  loss:
+ * optional fp64 [n_mat][O], sum_i e_i^2 per row in column order (equal to
+ * (w - What) H (w - What)^T in exact arithmetic).  workspace: >=
+ * tq_gptq_workspace_bytes(W) (an fp32 working copy of W), 16-byte aligned.
+ * Errors: TQ_ERR_INVALID_ARG for null/misaligned pointers, ldu < I, a short
+ * u_mat_stride or workspace; TQ_ERR_UNSUPPORTED for NVFP4. */
+size_t tq_gptq_workspace_bytes(const tq_mat* W);
+tq_status tq_gptq_sweep(const tq_mat* W, int32_t fmt, const void* scales, const uint8_t* zeros, const float* U,
+                        int64_t ldu, int64_t u_mat_stride, int8_t* codes, double* loss, void* workspace,
+                        size_t workspace_bytes, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ testing aid
  * Synchronises `stream` and returns TQ_ERR_CUDA if it or an earlier kernel
  * failed (including a tq_hessian or tq_proxy_error_full launch that gave up

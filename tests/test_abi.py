@@ -156,6 +156,19 @@ def test_invalid_arguments_are_rejected_before_any_launch(tq):
     assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, tq.INT4_G128_ASYM, *args[1:]) == 1   # int4 needs zeros
     assert pf(ctypes.byref(xa), ctypes.byref(wa), fake, tq.NVFP4_G16, *args[1:]) == 1        # needs global scale
 
+    # GPTQ sweep: (W, fmt, scales, zeros, U, ldu, u_mat_stride, codes, loss, ws, ws_bytes, stream)
+    gq = L.tq_gptq_sweep
+    wg = tq._Mat(fake, 1, 0, 2, 40, 200, 200, 40 * 200)
+    needg = L.tq_gptq_workspace_bytes(ctypes.byref(wg))
+    assert needg == 2 * 40 * 200 * 4
+    assert gq(ctypes.byref(wg), tq.NVFP4_G16, fake, None, fake, 200, 0, fake, None, fake, needg, None) == 2
+    assert gq(ctypes.byref(wg), tq.INT4_G128_ASYM, fake, None, fake, 200, 0, fake, None, fake, needg, None) == 1
+    assert gq(ctypes.byref(wg), tq.INT3_G64_SYM, fake, None, fake, 199, 0, fake, None, fake, needg, None) == 1
+    assert gq(ctypes.byref(wg), tq.INT3_G64_SYM, fake, None, fake, 200, 100, fake, None, fake, needg, None) == 1
+    assert gq(ctypes.byref(wg), tq.INT3_G64_SYM, fake, None, None, 200, 0, fake, None, fake, needg, None) == 1
+    assert gq(ctypes.byref(wg), tq.INT3_G64_SYM, fake, None, fake, 200, 0, fake, None, fake, needg - 4, None) == 1
+    assert b"workspace" in L.tq_last_error_string()
+
 
 def test_binding_refuses_cpu_tensors(tq):
     import torch

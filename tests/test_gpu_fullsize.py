@@ -226,3 +226,43 @@ def test_full_size_proxy_full():
             D = ((K / 16 + 32) * 2.0 ** -22 + extra) * (np.abs(X64) @ np.abs(M).T)
             bound = float(np.sum((2 * np.abs(X64 @ M.T) + D) * D))
             assert abs(got - ref) <= bound + 1e-12 * ref, (t0, o0, got, ref, bound)
+
+
+def test_full_size_gptq_sweep():
+    """tq_gptq_sweep on the dense int4-g128 4096 x 4096 workload with the
+    search's scales and the factor of its calibration Hessian (damped by 1 %
+    of the mean diagonal; fp64 Cholesky and inverse by the library, outside
+    the method), launched as bench.py launches it: sampled whole rows (the
+    first, the last, a CTA's 16th and random ones) bit for bit against the
+    oracle's sweep of the same rows, and a lower proxy error tr(E H E^T) than
+    round-to-nearest with the same scales."""
+    wl = synth.make("c1", DEV)
+    u = [x for x in wl.units if x.timed][0]
+    X = wl.sites[u.site].X[0]
+    W = u.W
+    fmt = tq.FORMATS[u.fmt]
+    m = tq.tq_imatrix(X)[0]
+    res = tq.tq_search_groups(W, m, fmt)
+    H = X.double().T @ X.double()
+    H += 0.01 * H.diagonal().mean() * torch.eye(H.shape[0], device=DEV, dtype=torch.float64)
+    U = torch.linalg.cholesky(torch.cholesky_inverse(torch.linalg.cholesky(H)), upper=True).float().contiguous()
+    codes, loss = tq.tq_gptq_sweep(W, fmt, res.scales, res.zeros, U)
+    tq.tq_sync()
+    O, I = W.shape[1], W.shape[2]
+    rng = np.random.default_rng(5)
+    rows = sorted({0, 15, 16, O - 1, *rng.integers(0, O, 5).tolist()})
+    Uh, Wh = U.cpu().numpy(), host32(W[0])
+    sc = res.scales.reshape(O, -1).cpu().numpy()
+    zz = res.zeros.reshape(O, -1).cpu().numpy()
+    c_ref, l_ref = oracle.gptq_sweep(Wh[rows], 4, sc[rows], zz[rows], Uh, g=128)
+    assert np.array_equal(codes[0, rows].cpu().numpy(), c_ref)
+    assert np.array_equal(loss[0, rows].cpu().numpy(), l_ref)
+    # the sweep's purpose, on the whole matrix: a lower tr(E H E^T) than RTN with the same scales
+    Hf = H - 0.01 * H.diagonal().mean() * torch.eye(I, device=DEV, dtype=torch.float64)
+    wq = tq.tq_dequant(tq.tq_pack_codes(codes.view(torch.uint8), fmt, res.zeros.reshape(O, -1)), fmt, res.scales,
+                       res.zeros, None, 1, O, I)
+    wr = tq.tq_dequant(res.packed, fmt, res.scales, res.zeros, None, 1, O, I)
+    tq.tq_sync()
+    pe = lambda Wq: float(torch.einsum("oi,ij,oj->", W[0].double() - Wq[0].double(), Hf,  # noqa: E731
+                                       W[0].double() - Wq[0].double()))
+    assert pe(wq) < pe(wr)

@@ -792,3 +792,88 @@ def test_proxy_full_exact_weights_and_strides():
     for e in range(E):
         rd = oracle.proxy_error_full(Wh[e], Wh[e], oracle.hessian(Xh[e]))[1]
         assert abs(den[e].item() - rd) <= _pf_bound(Xh[e], Wh[e], I, 0.0) + 1e-12 * rd
+
+
+# ------------------------------------------------------------------ GPTQ/LDLQ column sweep
+
+def _gptq_U(rng, I, ldu=None, T=None):
+    """fp32 upper factor U (rows of ldu) with H^-1 = U^T U for a damped,
+    correlated H = X^T X / T + 0.01 mean(diag) I (numpy fp64 Cholesky and
+    inverse: input preparation, not the method)."""
+    T = T or 2 * I
+    X = rng.standard_normal((T, I)) @ (np.eye(I) + 0.3 * rng.standard_normal((I, I)) / np.sqrt(I))
+    H = X.T @ X / T
+    H += 0.01 * np.mean(np.diag(H)) * np.eye(I)
+    U = np.linalg.cholesky(np.linalg.inv(H)).T.astype(np.float32)
+    out = np.zeros((I, ldu or I), np.float32)
+    out[:, :I] = U
+    return out
+
+
+_GQ_FMT = {tq.INT3_G64_SYM: (3, 64), tq.INT4_G128_ASYM: (4, 128), tq.INT4_G64_ASYM: (4, 64)}
+
+
+def _gptq_check(fmt, W, res, Uh, shared):
+    """GPU sweep vs the oracle's on the same W, scales, zeros and U: codes and
+    per-row losses bit for bit."""
+    E = W.shape[0]
+    Ud = torch.from_numpy(Uh).to(DEV)
+    codes, loss = tq.tq_gptq_sweep(W, fmt, res.scales, res.zeros, Ud)
+    tq.tq_sync()
+    Wh = host32(W)
+    kind, g = _GQ_FMT[fmt]
+    sc = res.scales.cpu().numpy().reshape(E, W.shape[1], -1)
+    zz = None if res.zeros is None else res.zeros.cpu().numpy().reshape(E, W.shape[1], -1)
+    for e in range(E):
+        Ue = Uh if shared else Uh[e]
+        c_ref, l_ref = oracle.gptq_sweep(Wh[e], kind, sc[e], None if zz is None else zz[e], Ue, g=g)
+        assert np.array_equal(codes[e].cpu().numpy(), c_ref), (e, np.argwhere(codes[e].cpu().numpy() != c_ref)[:5])
+        assert np.array_equal(loss[e].cpu().numpy(), l_ref), e
+    return codes, loss
+
+
+@pytest.mark.parametrize("fmt", list(_GQ_FMT))
+@pytest.mark.parametrize("E,O,I,dtype,shared", [(1, 37, 300, torch.bfloat16, True), (2, 16, 128, torch.float32, False),
+                                                (1, 5, 77, torch.bfloat16, True), (1, 1, 1, torch.float32, True),
+                                                (2, 33, 520, torch.bfloat16, True), (1, 18, 257, torch.float32, True)])
+def test_gptq_sweep_bit_exact(fmt, E, O, I, dtype, shared):
+    """Codes and per-row losses equal the oracle's bit for bit: one and several
+    128-column blocks, ragged last block and rows (not a multiple of the 16
+    rows of a CTA), one column, bf16 and fp32 weights, one factor for every
+    matrix or one per matrix, a padded factor row (ldu > I)."""
+    rng = np.random.default_rng(E * 1000 + O * 10 + I)
+    ld = (I + 7) // 8 * 8
+    Wf = (rng.standard_t(4, size=(E, O, ld)) * 0.02).astype(np.float32)
+    W = torch.from_numpy(Wf).to(DEV).to(dtype)[:, :, :I]
+    m = torch.from_numpy(np.exp(rng.standard_normal(I)).astype(np.float32) ** 2).to(DEV)
+    res = _run(fmt, W, m)
+    ldu = I + 4
+    Uh = _gptq_U(rng, I, ldu) if shared else np.stack([_gptq_U(rng, I, ldu) for _ in range(E)])
+    codes, _ = _gptq_check(fmt, W, res, Uh, shared)
+    # the codes pack like any others: tq_pack_codes of them == the oracle's packing of the same codes
+    if fmt == tq.INT3_G64_SYM:
+        ref = oracle.pack_int3(codes.cpu().numpy().reshape(E * O, I))
+        got = tq.tq_pack_codes(codes, fmt)
+    else:
+        z = res.zeros.reshape(E * O, -1)
+        ref = oracle.pack_nibbles(codes.cpu().numpy().reshape(E * O, I).astype(np.uint8), _GQ_FMT[fmt][1],
+                                  z.cpu().numpy())
+        got = tq.tq_pack_codes(codes.view(torch.uint8), fmt, z)
+    tq.tq_sync()
+    assert np.array_equal(got.cpu().numpy(), ref)
+
+
+def test_gptq_identity_factor_is_rtn():
+    """U = I propagates nothing: the sweep's codes are the fused RTN codes of
+    the search (tq_unpack_codes of its records)."""
+    rng = np.random.default_rng(9)
+    O, I = 40, 384
+    W = torch.from_numpy((rng.standard_t(4, size=(1, O, I)) * 0.02).astype(np.float32)).to(DEV).bfloat16()
+    m = torch.ones(I, device=DEV)
+    for fmt in _GQ_FMT:
+        res = _run(fmt, W, m)
+        codes, _ = tq.tq_gptq_sweep(W, fmt, res.scales, res.zeros, torch.eye(I, device=DEV))
+        ref = tq.tq_unpack_codes(res.packed, fmt, 1, O, I)
+        tq.tq_sync()
+        assert np.array_equal(codes.reshape(-1).cpu().numpy().astype(np.int16),
+                              ref.reshape(-1).cpu().numpy().astype(np.int16)), fmt
