@@ -22,8 +22,8 @@
 //    columns; lane 0 records the code and e_i.
 //  * propagation (nearly all the flops): each thread owns later columns j
 //    and keeps the 16 rows' w_j in registers; for i = 0..127 in order it
-//    loads U_ij once (coalesced, from L2) and applies 16 FMAs, e_i read as
-//    float4 broadcasts from shared memory.
+//    loads U_ij once (coalesced, from L2; the next four in flight) and applies
+//    16 FMAs, e_i read as float4 broadcasts from shared memory.
 // The rows' fp32 working copy lives in the workspace: one read and one write
 // of the remaining columns per block.
 #include "walk.cuh"
@@ -36,6 +36,7 @@ constexpr int GQ_THREADS = 256;
 constexpr int GQ_RPW = GQ_R / (GQ_THREADS / 32);  // rows per warp in the serial part
 constexpr int GQ_SMEM_BYTES = (GQ_B * GQ_B + GQ_R * GQ_B) * 4;
 static_assert(GQ_RPW * (GQ_THREADS / 32) == GQ_R, "rows split evenly over the warps");
+static_assert(GQ_B % 8 == 0, "the propagation takes the block in steps of 8 columns");
 
 struct GqArgs {
     const void* W;           // [n_mat][O][I] rows of ld, matrices ms apart (bf16 or fp32)
@@ -68,6 +69,19 @@ __device__ __forceinline__ float gq_round(float w, float s, int z, int& code) {
         if (s != 0.f) q = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(w, s)), zf), 0.f), 15.f);
         code = static_cast<int>(q);
         return __fmul_rn(s, __fsub_rn(q, zf));
+    }
+}
+
+// Four consecutive columns i..i+3 of the block applied to the GQ_R rows'
+// accumulators in column order: acc_r <- fma(-e_{r,i}, U_ij, acc_r).
+__device__ __forceinline__ void gq_step(float (&acc)[GQ_R], const float* Eb_i, const float (&u)[4]) {
+#pragma unroll
+    for (int r = 0; r < GQ_R; ++r) {
+        const float4 ev = *reinterpret_cast<const float4*>(Eb_i + r * GQ_B);
+        acc[r] = __fmaf_rn(-ev.x, u[0], acc[r]);
+        acc[r] = __fmaf_rn(-ev.y, u[1], acc[r]);
+        acc[r] = __fmaf_rn(-ev.z, u[2], acc[r]);
+        acc[r] = __fmaf_rn(-ev.w, u[3], acc[r]);
     }
 }
 
@@ -152,21 +166,28 @@ __global__ void __launch_bounds__(GQ_THREADS, 2) k_gptq(const GqArgs a) {
 
         // ---- propagation to the later columns (a later column exists only when the block is full)
         for (int64_t j = b0 + GQ_B + tid; j < I; j += GQ_THREADS) {
+            // two sets of four U_ij: one set is in flight (L2 latency) while the other is used
+            const float* up = U + b0 * a.ldu + j;
+            float ua[4], ub[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                ua[q] = __ldg(up + q * a.ldu);
+                ub[q] = __ldg(up + (4 + q) * a.ldu);
+            }
             float acc[GQ_R];
 #pragma unroll
             for (int r = 0; r < GQ_R; ++r) acc[r] = r < nr ? wk[r * I + j] : 0.f;
-            const float* up = U + b0 * a.ldu + j;
-#pragma unroll 2
-            for (int i = 0; i < GQ_B; i += 4) {
-                const float u0 = __ldg(up + (i + 0) * a.ldu), u1 = __ldg(up + (i + 1) * a.ldu);
-                const float u2 = __ldg(up + (i + 2) * a.ldu), u3 = __ldg(up + (i + 3) * a.ldu);
+#pragma unroll 1
+            for (int i = 0; i < GQ_B; i += 8) {
+                gq_step(acc, Eb + i, ua);
+                if (i + 8 < GQ_B) {
 #pragma unroll
-                for (int r = 0; r < GQ_R; ++r) {
-                    const float4 ev = *reinterpret_cast<const float4*>(Eb + r * GQ_B + i);
-                    acc[r] = __fmaf_rn(-ev.x, u0, acc[r]);
-                    acc[r] = __fmaf_rn(-ev.y, u1, acc[r]);
-                    acc[r] = __fmaf_rn(-ev.z, u2, acc[r]);
-                    acc[r] = __fmaf_rn(-ev.w, u3, acc[r]);
+                    for (int q = 0; q < 4; ++q) ua[q] = __ldg(up + (i + 8 + q) * a.ldu);
+                }
+                gq_step(acc, Eb + i + 4, ub);
+                if (i + 12 < GQ_B) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) ub[q] = __ldg(up + (i + 12 + q) * a.ldu);
                 }
             }
 #pragma unroll
