@@ -1,7 +1,8 @@
 // GPTQ/LDLQ column sweep ("Quantize on TT cards: CUDA-free GPTQ/LDLQ bfp4
-// pipeline", tt-stack issue #67, pipeline table step 3: serial rounding
-// inside 128-column blocks, then the propagation W[:, rest] -= E U[blk, rest]
-// through the inverse Hessian's triangular factor), with the group scales and
+// pipeline", tt-stack issue #67, pipeline table step 3: columns are rounded
+// one at a time within 128-wide blocks, and each block's rounding errors E
+// reach the columns after it through W[:, rest] -= E U[blk, rest], U the
+// inverse Hessian's triangular factor), with the group scales and
 // zero-points the search chose.
 //
 // Per row, column i in order: the code of the current w_i under its group's

@@ -371,10 +371,10 @@ tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uint8_t* p
                               tq_stream_t stream);
 
 /* ------------------------------------------------------------------ GPTQ/LDLQ column sweep
- * [TT] pipeline table, step 3: serial rounding with the rounding error of each
- * column propagated to the later columns through the inverse Hessian's
- * triangular factor, with the group scales (and zero-points) of a search held
- * fixed.  U: fp32 upper triangular factor with H^-1 = U^T U, rows of ldu >= I
+ * [TT] pipeline table, step 3: the columns are rounded one after another and
+ * each one's rounding error is carried to the later columns through the
+ * inverse Hessian's triangular factor, with the group scales (and
+ * zero-points) of a search held fixed.  U: fp32 upper triangular factor with H^-1 = U^T U, rows of ldu >= I
  * elements, u_mat_stride elements between matrices (0: one factor for every
  * matrix); only its upper triangle is read; U_ii > 0 (the caller's Cholesky
  * of the damped, inverted H).  Per row, for each column i in order:

@@ -878,9 +878,9 @@ ORC_API void orc_dequant_int4(const uint8_t* q, int64_t rows, int64_t I, const f
         }
 }
 
-/* GPTQ/LDLQ column sweep ([TT] pipeline table, step 3: serial rounding,
- * with the rounding error of each column propagated to the later columns
- * through the inverse Hessian's triangular factor), with the group scales
+/* GPTQ/LDLQ column sweep ([TT] pipeline table, step 3: the columns are
+ * rounded one after another and each one's rounding error is carried to the
+ * later columns through the inverse Hessian's triangular factor), with the group scales
  * (and zero-points) fixed by the search.  U: upper triangular, H^-1 = U^T U
  * (fp32, I x I rows of ldu; only the upper triangle is read; U_ii > 0).  Per
  * row, for each column i in order:
