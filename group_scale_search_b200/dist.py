@@ -8,7 +8,13 @@ matrix or one calibration set is split: token-sharded calibration (every
 rank sums x^2 over its own tokens with tq_imatrix(alpha = 1) and an
 all-reduce adds the partial sums before the division by the total token
 count), and a row-sharded matrix's proxy error (an all-reduce of the
-per-matrix fp64 (num, den) pairs before the ratio).
+per-matrix fp64 (num, den) pairs before the ratio).  The same two hold for the
+full-Hessian path: H = sum_t x_t^T x_t adds over token shards (every rank
+runs tq_hessian on its tokens, an all-reduce adds the fp64 copies), after
+which the GPTQ/LDLQ sweep splits the rows of W with no exchange (rows are
+independent given the factor of H^-1); and tr(E H E^T) = ||X E^T||^2 adds
+over token shards and over row shards, so tq_proxy_error_full's (num, den)
+go through allreduce_proxy.
 """
 from __future__ import annotations
 
@@ -18,7 +24,8 @@ from typing import List, Optional, Sequence, Tuple
 import torch
 import torch.distributed as dist
 
-__all__ = ["shard_range", "shard_units", "allreduce_imatrix", "allreduce_proxy", "max_over_ranks", "init_from_env"]
+__all__ = ["shard_range", "shard_units", "allreduce_imatrix", "allreduce_hessian", "allreduce_proxy",
+           "max_over_ranks", "init_from_env"]
 
 
 def shard_range(n: int, rank: int, world: int) -> Tuple[int, int]:
@@ -57,11 +64,25 @@ def allreduce_imatrix(local_sums: torch.Tensor, total_tokens: int, group=None) -
     return (acc / float(total_tokens)).to(torch.float32)
 
 
+def allreduce_hessian(local_h: torch.Tensor, group=None) -> torch.Tensor:
+    """H = sum over ranks of X_r^T X_r for token-sharded calibration.
+
+    local_h: this rank's Hessian of its own tokens (fp32 from tq_hessian, or
+    fp64); the sum runs in fp64 so it does not depend on the rank count beyond
+    fp64 rounding, and the fp64 result is what the factorisation of H^-1 for
+    the GPTQ sweep wants.  Every rank gets the whole H."""
+    acc = local_h.to(torch.float64)
+    if dist.is_available() and dist.is_initialized():
+        dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
+    return acc
+
+
 def allreduce_proxy(num: torch.Tensor, den: torch.Tensor, group=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Proxy error of matrices whose rows are split over ranks: every rank
-    passes tq_proxy_error's fp64 (num, den) of its own rows; the sums over
-    ranks are the whole matrices' tr(E H E^T) and tr(W H W^T) (the ratio is
-    taken after the sum, never averaged over ranks)."""
+    """Proxy error of matrices whose rows (or, for tq_proxy_error_full, whose
+    calibration tokens) are split over ranks: every rank passes its fp64
+    (num, den); the sums over ranks are the whole matrices' tr(E H E^T) and
+    tr(W H W^T) (the ratio is taken after the sum, never averaged over
+    ranks)."""
     if num.dtype != torch.float64 or den.dtype != torch.float64:
         raise ValueError("num and den must be float64")
     both = torch.stack([num, den])

@@ -57,6 +57,45 @@ def proxy_row_shards(rank, world, port, root, out_dir):
     dist.destroy_process_group()
 
 
+def hessian_gptq_shards(rank, world, port, root, out_dir):
+    """Token-sharded calibration: each rank forms X_r^T X_r of its tokens,
+    the all-reduce gives every rank the whole H; each rank then sweeps its
+    own rows of W (GPTQ with the factor of the damped H^-1) with no exchange,
+    and the token-sharded full-Hessian proxy error of the result goes through
+    allreduce_proxy.  The oracle stands in for the GPU calls (host logic)."""
+    sys.path.insert(0, root)
+    import oracle
+    from group_scale_search_b200.dist import allreduce_hessian, allreduce_proxy, shard_range
+    _init(rank, world, port)
+    rng = np.random.default_rng(8)                      # same data on every rank
+    T, O, I = 96, 21, 160
+    X = rng.standard_normal((T, I)).astype(np.float32)
+    W = (rng.standard_t(4, size=(O, I)) * 0.02).astype(np.float32)
+    t0, t1 = shard_range(T, rank, world)
+    H = allreduce_hessian(torch.from_numpy(oracle.hessian(X[t0:t1]))).numpy()
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(I)
+    U = np.ascontiguousarray(np.linalg.cholesky(np.linalg.inv(Hd)).T.astype(np.float32))
+    s, z = [a[0] for a in oracle.search_asym_int4(W[None], np.diag(H).astype(np.float32) / T)[:2]]
+    o0, o1 = shard_range(O, rank, world)
+    codes, _ = oracle.gptq_sweep(W[o0:o1], 4, s[o0:o1], z[o0:o1], U)
+    # every rank needs every (row shard, token shard) pair: gather the row shards' codes first
+    rows = [shard_range(O, r, world) for r in range(world)]
+    pad = max(b - a for a, b in rows)                    # gloo gathers equal sizes: pad, then trim
+    mine = torch.zeros((pad, I), dtype=torch.int8)
+    mine[: o1 - o0] = torch.from_numpy(codes)
+    allc = [torch.zeros((pad, I), dtype=torch.int8) for _ in range(world)]
+    dist.all_gather(allc, mine)
+    allc = [c[: b - a] for c, (a, b) in zip(allc, rows)]
+    Wq = oracle.dequant_int4(torch.cat(allc).numpy().astype(np.uint8), s, z)
+    n, d = oracle.proxy_error_full(W, Wq, oracle.hessian(X[t0:t1]))            # all rows x this rank's tokens
+    num, den = allreduce_proxy(torch.tensor([n], dtype=torch.float64), torch.tensor([d], dtype=torch.float64))
+    np.save(os.path.join(out_dir, f"h{rank}.npy"), H)
+    np.save(os.path.join(out_dir, f"c{rank}.npy"), torch.cat(allc).numpy())
+    np.save(os.path.join(out_dir, f"q{rank}.npy"), np.array([num.item(), den.item()]))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
 def peer_dies(rank, world, port, out_dir):
     """Rank 1 leaves before the collective; rank 0 must get an error, not hang."""
     _init(rank, world, port, timeout_s=8.0)

@@ -1,5 +1,6 @@
 """Multi-process (N > 1) host path on CPU with gloo ranks: work sharding,
 token-sharded imatrix all-reduce, row-sharded proxy-error all-reduce,
+token-sharded Hessian then row-sharded GPTQ sweep and full-Hessian proxy error,
 max-over-ranks timing, and a rank that dies before a collective (the
 survivor must fail fast, not hang)."""
 import multiprocessing as mp
@@ -83,6 +84,29 @@ def test_row_sharded_proxy_allreduce(tmp_path):
     for r in range(2):
         got = np.load(tmp_path / f"p{r}.npy")
         assert np.max(np.abs(got - ref) / ref) <= 1e-12      # fp64 sums of two halves
+
+
+def test_token_sharded_hessian_then_row_sharded_gptq(tmp_path):
+    """The full-Hessian path on 2 ranks: the all-reduced H equals X^T X of all
+    tokens, the row-sharded sweeps gathered equal the one-process sweep bit
+    for bit, and the token-sharded tr(E H E^T), tr(W H W^T) equal the whole."""
+    import oracle
+    codes = _run(dist_workers.hessian_gptq_shards, (_port(), ROOT, str(tmp_path)))
+    assert codes == [0, 0]
+    rng = np.random.default_rng(8)
+    T, O, I = 96, 21, 160
+    X = rng.standard_normal((T, I)).astype(np.float32)
+    W = (rng.standard_t(4, size=(O, I)) * 0.02).astype(np.float32)
+    H = oracle.hessian(X)
+    Hd = H + 0.01 * np.mean(np.diag(H)) * np.eye(I)
+    U = np.ascontiguousarray(np.linalg.cholesky(np.linalg.inv(Hd)).T.astype(np.float32))
+    s, z = [a[0] for a in oracle.search_asym_int4(W[None], np.diag(H).astype(np.float32) / T)[:2]]
+    ref_codes, _ = oracle.gptq_sweep(W, 4, s, z, U)
+    ref = oracle.proxy_error_full(W, oracle.dequant_int4(ref_codes.astype(np.uint8), s, z), H)
+    for r in range(2):
+        assert np.allclose(np.load(tmp_path / f"h{r}.npy"), H, rtol=1e-13, atol=1e-10)
+        assert np.array_equal(np.load(tmp_path / f"c{r}.npy"), ref_codes)
+        assert np.allclose(np.load(tmp_path / f"q{r}.npy"), ref, rtol=1e-12)
 
 
 def test_surviving_rank_fails_fast_when_a_peer_dies(tmp_path):
