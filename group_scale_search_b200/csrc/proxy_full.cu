@@ -383,6 +383,14 @@ TQ_API tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uin
     const int64_t tiles = pf_tiles(X, W);
     double* pn = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + ep_bytes);
     double* pd = pn + E * tiles;
+    // tensor maps first (host only), so a failure launches nothing
+    CUtensorMap xm, em, wm;
+    const int64_t xms = E > 1 ? X->mat_stride : X->rows * X->ld;
+    const int64_t wms = E > 1 ? W->mat_stride : W->rows * W->ld;
+    if (!pf_map(&xm, X->ptr, X->cols, X->rows, E, X->ld, xms, PF_M) ||
+        !pf_map(&em, ep, PF_PIECES * Ip, O, E, PF_PIECES * Ip, O * PF_PIECES * Ip, PF_N) ||
+        !pf_map(&wm, W->ptr, W->cols, O, E, W->ld, wms, PF_N))
+        return set_error(TQ_ERR_CUDA, "tq_proxy_error_full: tensor map encoding failed");
     // E = W - What in bf16 pieces
     {
         const int64_t ms = E > 1 ? W->mat_stride : 0;
@@ -398,13 +406,6 @@ TQ_API tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uin
         else
             k_pf_prep<TQ_NVFP4_G16, uint16_t><<<grid, 256, 0, st>>>(Wp, O, W->cols, W->ld, ms, packed, scales, zeros, global_scale, E, Ip, ep);
     }
-    CUtensorMap xm, em, wm;
-    const int64_t xms = E > 1 ? X->mat_stride : X->rows * X->ld;
-    const int64_t wms = E > 1 ? W->mat_stride : W->rows * W->ld;
-    if (!pf_map(&xm, X->ptr, X->cols, X->rows, E, X->ld, xms, PF_M) ||
-        !pf_map(&em, ep, PF_PIECES * Ip, O, E, PF_PIECES * Ip, O * PF_PIECES * Ip, PF_N) ||
-        !pf_map(&wm, W->ptr, W->cols, O, E, W->ld, wms, PF_N))
-        return set_error(TQ_ERR_CUDA, "tq_proxy_error_full: tensor map encoding failed");
     static std::once_flag attr;
     std::call_once(attr, [] { cudaFuncSetAttribute(k_pf_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, PF_SMEM_BYTES); });
     PfArgs a;
