@@ -600,27 +600,33 @@ def test_proxy_error_full_reduces_to_diagonal(orc):
     assert np.isclose(d, np.sum((W.astype(np.float64) @ X.astype(np.float64).T) ** 2), rtol=1e-12)
 
 
-def test_int4_g64_batching(orc):
-    """The int4 batch functions at g = 64: every group is the group search on
-    its own 64 weights (the last one ragged), RTN with the chosen scales gives
-    the search's codes, and dequantizing them reproduces W to half a step."""
-    rng = np.random.default_rng(47)
+@pytest.mark.parametrize("g", [64, 32])
+def test_int4_group_batching(orc, g):
+    """The int4 batch functions at g = 64 (colibri's fmt=4) and g = 32 (the
+    turboquant page's group size): every group is the group search on its own
+    g weights (the last one ragged), RTN with the chosen scales gives the
+    search's codes, dequantizing them reproduces W to half a step, and the
+    nibble records are g / 2 bytes with element 2k in the low nibble."""
+    rng = np.random.default_rng(47 + g)
     W = (rng.standard_t(4, size=(2, 3, 200)) * 0.02).astype(np.float32)
     m = rng.random(200).astype(np.float32) + 0.1
-    s, z, i, L, q = orc.search_asym_int4(W, m, g=64)
-    assert s.shape == (2, 3, 4)
+    G = (200 + g - 1) // g
+    s, z, i, L, q = orc.search_asym_int4(W, m, g=g)
+    assert s.shape == (2, 3, G)
     for e in range(2):
         for o in range(3):
-            for k in range(4):
-                j0, j1 = 64 * k, min(200, 64 * k + 64)
-                s1, z1, i1, L1, q1 = orc.search_asym_int4(W[e, o, j0:j1][None, None], m[j0:j1], g=64)
+            for k in range(G):
+                j0, j1 = g * k, min(200, g * k + g)
+                s1, z1, i1, L1, q1 = orc.search_asym_int4(W[e, o, j0:j1][None, None], m[j0:j1], g=g)
                 assert i1[0, 0, 0] == i[e, o, k] and s1[0, 0, 0] == s[e, o, k] and L1[0, 0, 0] == L[e, o, k]
-    assert np.array_equal(orc.rtn_int4(W, s, z, g=64), q)
-    What = orc.dequant_int4(q, s.reshape(6, 4), z.reshape(6, 4), g=64).reshape(W.shape)
-    step = np.repeat(s, 64, axis=2)[:, :, :200]
+    assert np.array_equal(orc.rtn_int4(W, s, z, g=g), q)
+    What = orc.dequant_int4(q, s.reshape(6, G), z.reshape(6, G), g=g).reshape(W.shape)
+    step = np.repeat(s, g, axis=2)[:, :, :200]
     inside = (q > 0) & (q < 15)
     assert np.all(np.abs(What - W)[inside] <= 0.5 * step[inside] * (1 + 1e-6))
-    assert np.array_equal(orc.loss_given_int4(W, m, s, z, g=64), L)
+    assert np.array_equal(orc.loss_given_int4(W, m, s, z, g=g), L)
+    rec = orc.pack_nibbles(q.reshape(6, 200), g, z.reshape(6, G)).reshape(6, G, g // 2)
+    assert np.array_equal(rec[..., 0] & 0xF, q.reshape(6, 200)[:, 0::g]) and np.array_equal(rec[..., 0] >> 4, q.reshape(6, 200)[:, 1::g])
 
 
 # ------------------------------------------------------------------ FP8 per-tensor ([NVFP4] recipe table)
