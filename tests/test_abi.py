@@ -174,3 +174,11 @@ def test_binding_refuses_cpu_tensors(tq):
     import torch
     with pytest.raises(tq.TQError):
         tq.tq_imatrix(torch.zeros(8, 64))
+    W = torch.zeros(8, 64, dtype=torch.bfloat16)
+    with pytest.raises(tq.TQError):
+        tq.tq_proxy_error_full(torch.zeros(4, 64, dtype=torch.bfloat16), W, torch.zeros(256, dtype=torch.uint8),
+                               tq.INT3_G64_SYM, torch.zeros(8), None, None)
+    with pytest.raises(tq.TQError):
+        tq.tq_gptq_sweep(W, tq.INT3_G64_SYM, torch.zeros(8), None, torch.eye(64))
+    with pytest.raises(tq.TQError):
+        tq.tq_hessian(torch.zeros(4, 64, dtype=torch.bfloat16))
