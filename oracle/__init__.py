@@ -58,6 +58,8 @@ def lib():
             "orc_hessian_entry": (f64, [P, i64, i64, i64, i64]),
             "orc_proxy_error_full": (None, [P, P, i64, i64, P, P, P]),
             "orc_gptq_sweep": (None, [P, i64, i64, i32, i32, P, P, P, i64, P, P]),
+            "orc_nvfp4_quant_act": (None, [P, i64, i64, P, P, P]),
+            "orc_gemm_nvfp4": (None, [P, P, f32, i64, P, P, f32, i64, i64, P]),
             "orc_sym_stage1_ratio": (f32, [i32, f64, f64, i32]),
             "orc_sym_stage2_ratio": (f32, [i32, i32, f64, f64, i32, i32]),
             "orc_sym_loss": (f64, [P, P, i32, f32, P]),
@@ -183,6 +185,30 @@ def gptq_sweep(W, fmt: int, scales, zeros, U, g=None):
     lib().orc_gptq_sweep(_p(W), rows, I, int(fmt), int(g), _p(_f32(scales)), _p(z), _p(U), U.shape[-1],
                          _p(codes), _p(loss))
     return codes, loss
+
+
+def nvfp4_quant_act(X):
+    """NVFP4 activations X [rows, I] -> (global scale, E4M3 block-scale codes
+    [rows, ceil(I/16)], E2M1 codes [rows, I] with the sign in bit 3)."""
+    X = _f32(X)
+    rows, I = X.shape
+    g = ctypes.c_float()
+    sc = np.empty((rows, (I + 15) // 16), np.uint8)
+    c = np.empty((rows, I), np.uint8)
+    lib().orc_nvfp4_quant_act(_p(X), rows, I, ctypes.byref(g), _p(sc), _p(c))
+    return g.value, sc, c
+
+
+def gemm_nvfp4(cw, ew, gw, cx, ex, gx):
+    """W4A4 product y [B, O] (fp64) of NVFP4 weight codes cw [O, I] / block
+    scales ew [O, G] / global gw and activation codes cx [B, I] / ex [B, G] / gx."""
+    cw = np.ascontiguousarray(cw, np.uint8); cx = np.ascontiguousarray(cx, np.uint8)
+    ew = np.ascontiguousarray(ew, np.uint8); ex = np.ascontiguousarray(ex, np.uint8)
+    O, I = cw.shape
+    B = cx.shape[0]
+    y = np.empty((B, O), np.float64)
+    lib().orc_gemm_nvfp4(_p(cw), _p(ew), float(gw), O, _p(cx), _p(ex), float(gx), B, I, _p(y))
+    return y
 
 
 def e4m3_rne(y: float) -> int:

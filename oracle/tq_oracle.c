@@ -787,6 +787,62 @@ ORC_API void orc_rtn_nvfp4(const float* W, int64_t rows, int64_t mat_rows, int64
     }
 }
 
+/* NVFP4 activations for a W4A4 product ([NVFP4] recipe table: the routed
+ * experts run W4A4 with 16-element groups; the card gives no activation
+ * recipe, so the reading is the weights' one without the search): per
+ * tensor g = fl32(amax / 2688); per 16-element block of a row (amax b) the
+ * positive finite E4M3 code nearest b / (6 g), ties to the lower code (the
+ * first code of orc_nvfp4_window; 0 when b or g is 0); the elements' E2M1
+ * codes by orc_rtn_nvfp4's rule.  scale_codes: [rows][ceil(I/16)], codes:
+ * [rows][I] (sign in bit 3). */
+ORC_API void orc_nvfp4_quant_act(const float* X, int64_t rows, int64_t I, float* g_out, uint8_t* scale_codes,
+                                 uint8_t* codes)
+{
+    const int64_t G = (I + 15) / 16;
+    const float g = orc_nvfp4_global(X, rows * I);
+    *g_out = g;
+    for (int64_t r = 0; r < rows; ++r)
+        for (int64_t k = 0; k < G; ++k) {
+            float b = 0.0f;
+            for (int64_t j = 16 * k; j < I && j < 16 * k + 16; ++j) {
+                float a = fabsf(X[r * I + j]);
+                if (a > b) b = a;
+            }
+            int code = 0;
+            if (g > 0.0f && b > 0.0f) orc_nvfp4_window(b, g, 1, &code);
+            scale_codes[r * G + k] = (uint8_t)code;
+        }
+    orc_rtn_nvfp4(X, rows, rows, I, scale_codes, &g, codes);
+}
+
+/* W4A4 product of NVFP4 weights and NVFP4 activations (the consumer of the
+ * packed experts on a block-scaled tensor core):
+ *   y[b][o] = gw gx sum_k dec(ew[o][k]) dec(ex[b][k]) sum_{j in block k} dec(cw[o][j]) dec(cx[b][j]),
+ * the exact value of the block-scaled representation (reading: the global
+ * scales multiply once, the E4M3 block scales per block, no rounding of the
+ * dequantized elements); fp64, each block's sum of E2M1 products exact. */
+ORC_API void orc_gemm_nvfp4(const uint8_t* cw, const uint8_t* ew, float gw, int64_t O, const uint8_t* cx,
+                            const uint8_t* ex, float gx, int64_t B, int64_t I, double* y)
+{
+    const int64_t G = (I + 15) / 16;
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < B; ++b)
+        for (int64_t o = 0; o < O; ++o) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < G; ++k) {
+                double p = 0.0;
+                for (int64_t j = 16 * k; j < I && j < 16 * k + 16; ++j) {
+                    const int u = cw[o * I + j], v = cx[b * I + j];
+                    const double dw = (u & 8) ? -E2M1_MAG[u & 7] : E2M1_MAG[u & 7];
+                    const double dx = (v & 8) ? -E2M1_MAG[v & 7] : E2M1_MAG[v & 7];
+                    p += dw * dx;
+                }
+                acc += orc_e4m3_decode(ew[o * G + k]) * orc_e4m3_decode(ex[b * G + k]) * p;
+            }
+            y[b * O + o] = (double)gw * (double)gx * acc;
+        }
+}
+
 /* ------------------------------------------------------------------ */
 /* Packing ([INT3] Design: Layout; nibble order for int4 / NVFP4)      */
 /* ------------------------------------------------------------------ */

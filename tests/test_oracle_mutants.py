@@ -53,6 +53,11 @@ MUTANTS = {
     "gptq_no_diagonal_division": ("const float e = (w[i] - what) / U[i * ldu + i];", "const float e = (w[i] - what);"),
     "gptq_skips_next_column": ("for (int64_t j = i + 1; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);",
                                "for (int64_t j = i + 2; j < I; ++j) w[j] = fmaf(-e, U[i * ldu + j], w[j]);"),
+    "act_block_amax_first_element": ("float a = fabsf(X[r * I + j]);\n                if (a > b) b = a;",
+                                     "float a = fabsf(X[r * I + j]);\n                if (j == 16 * k) b = a;"),
+    "w4a4_drops_activation_global": ("y[b * O + o] = (double)gw * (double)gx * acc;", "y[b * O + o] = (double)gw * acc;"),
+    "w4a4_first_block_scale": ("acc += orc_e4m3_decode(ew[o * G + k]) * orc_e4m3_decode(ex[b * G + k]) * p;",
+                               "acc += orc_e4m3_decode(ew[o * G + k]) * orc_e4m3_decode(ex[b * G]) * p;"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }

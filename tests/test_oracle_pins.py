@@ -854,3 +854,93 @@ def test_gptq_beats_rtn_on_correlated_hessians(orc):
         Wr = orc.dequant_int4(orc.rtn_int4(W, s, z), s, z)
         pe = lambda Wh: float(np.einsum("oi,ij,oj->", W - Wh.astype(np.float64), H, W - Wh.astype(np.float64)))  # noqa: E731
         assert pe(Wg) < 0.9 * pe(Wr), (seed, pe(Wg), pe(Wr))
+
+
+# ----------------------------------------------------------------- NVFP4 activations and the W4A4 product
+
+_E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _e2m1_brute(y):
+    """Nearest E2M1 magnitude code of y >= 0 by brute force, ties to the even code, 7 above 6."""
+    if y > 6.0:
+        return 7
+    d = np.abs(float(y) - _E2M1)
+    best = np.flatnonzero(d == d.min())
+    return int(best[0] if len(best) == 1 else best[best % 2 == 0][0])
+
+
+def _e2m1_value(c):
+    v = _E2M1[c & 7]
+    return -v if c & 8 else v
+
+
+def test_nvfp4_act_scales_and_codes_brute_force(orc):
+    """Each block's E4M3 code is the argmin over all 126 positive finite codes
+    of |6 g dec(c) - b| (lowest code on ties), a zero block gets code 0, and
+    every element's code is the nearest E2M1 value of |x| / fl32(g dec(e))."""
+    rng = _rng(71)
+    X = (rng.standard_normal((4, 40)) * np.exp(rng.uniform(-6, 3, size=(4, 1)))).astype(np.float32)
+    X[2, 16:32] = 0.0                                        # a zero block
+    X[3, :16] *= np.float32(1e-30)                           # a block far below the global scale
+    g, sc, c = orc.nvfp4_quant_act(X)
+    dec = np.array([orc.e4m3_decode(k) for k in range(127)])
+    for r in range(4):
+        for k in range(3):
+            blk = X[r, 16 * k:16 * k + 16]
+            b = float(np.max(np.abs(blk)))
+            if b == 0.0:
+                assert sc[r, k] == 0 and not c[r, 16 * k:16 * k + 16].any()
+                continue
+            d = np.abs(6.0 * float(g) * dec[1:127] - b)
+            assert sc[r, k] == 1 + int(np.argmin(d)), (r, k)
+            S = np.float32(float(g) * dec[sc[r, k]])
+            for j, x in enumerate(blk):
+                mag = _e2m1_brute(np.float32(abs(x)) / S)
+                want = (mag | 8) if (mag and x < 0) else mag
+                assert c[r, 16 * k + j] == want, (r, k, j)
+
+
+def test_nvfp4_act_round_trip(orc):
+    """Activations built exactly from a global scale g = 2^-10, block codes
+    and E2M1 codes (each block holding a +-6 so its amax is 6 g dec(e), and
+    one block at the top code 448 so the tensor amax is 2688 g) quantize back
+    to the same g, block codes and element codes."""
+    rng = _rng(73)
+    rows, I = 3, 64
+    G = I // 16
+    g = 2.0 ** -10
+    e = rng.integers(40, 126, size=(rows, G))
+    e[1, 2] = 126
+    mags = rng.integers(0, 8, size=(rows, I))
+    mags[:, ::16] = 7                                      # a +-6 in every block
+    signs = np.where(rng.random((rows, I)) < 0.5, -1.0, 1.0)
+    dec = np.array([orc.e4m3_decode(k) for k in range(127)])
+    S = g * dec[np.repeat(e, 16, axis=1)]
+    X = (signs * _E2M1[mags] * S).astype(np.float32)
+    assert np.array_equal(X.astype(np.float64), signs * _E2M1[mags] * S)     # exact in fp32
+    g2, sc, c = orc.nvfp4_quant_act(X)
+    assert g2 == np.float32(g)
+    assert np.array_equal(sc, e)
+    want = np.where((mags > 0) & (signs < 0), mags | 8, mags)
+    assert np.array_equal(c, want)
+
+
+def test_gemm_nvfp4_closed_form(orc):
+    """The W4A4 product equals the fp64 matrix product (numpy) of the exactly
+    dequantized operands g dec(e) dec(c); all-zero activations give 0."""
+    rng = _rng(79)
+    O, B, I = 7, 5, 72
+    G = (I + 15) // 16
+    cw = rng.integers(0, 16, size=(O, I)).astype(np.uint8)
+    cx = rng.integers(0, 16, size=(B, I)).astype(np.uint8)
+    ew = rng.integers(1, 127, size=(O, G)).astype(np.uint8)
+    ex = rng.integers(1, 127, size=(B, G)).astype(np.uint8)
+    gw, gx = np.float32(3.1e-4), np.float32(7.7e-3)
+    dec = np.array([orc.e4m3_decode(k) for k in range(127)])
+    val = np.vectorize(_e2m1_value)
+    Wd = float(gw) * val(cw) * dec[np.repeat(ew, 16, axis=1)[:, :I]]
+    Xd = float(gx) * val(cx) * dec[np.repeat(ex, 16, axis=1)[:, :I]]
+    y = orc.gemm_nvfp4(cw, ew, gw, cx, ex, gx)
+    assert np.allclose(y, Xd @ Wd.T, rtol=1e-12, atol=1e-300)
+    assert not orc.gemm_nvfp4(cw, ew, gw, np.zeros_like(cx), ex, gx).any()
