@@ -58,6 +58,10 @@ MUTANTS = {
     "w4a4_drops_activation_global": ("y[b * O + o] = (double)gw * (double)gx * acc;", "y[b * O + o] = (double)gw * acc;"),
     "w4a4_first_block_scale": ("acc += orc_e4m3_decode(ew[o * G + k]) * orc_e4m3_decode(ex[b * G + k]) * p;",
                                "acc += orc_e4m3_decode(ew[o * G + k]) * orc_e4m3_decode(ex[b * G]) * p;"),
+    "proxy_full_den_uses_error": ("hd += H[i * I + j] * (double)w[j];",
+                                  "hd += H[i * I + j] * ((double)w[j] - (double)wh[j]);"),
+    "proxy_full_drops_last_column": ("for (int64_t j = 0; j < I; ++j) {\n                hn += H[i * I + j]",
+                                     "for (int64_t j = 0; j + 1 < I; ++j) {\n                hn += H[i * I + j]"),
     "dequant_int4_no_zero": ("out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j] - (double)zeros[gi]));",
                              "out[r * I + j] = (float)((double)scales[gi] * ((double)q[r * I + j]));"),
 }
