@@ -27,7 +27,6 @@
 // that runs out makes the CTA write NaN partials and count the timeout.
 #include <cuda.h>
 
-#include <atomic>
 #include <mutex>
 
 #include "walk.cuh"
