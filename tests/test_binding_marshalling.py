@@ -1,0 +1,93 @@
+"""The Python binding's marshalling on the CPU: a fake library records the
+arguments each call passes through the C ABI (descriptor shapes and strides,
+factor strides, output shapes, workspace sizing).  The binding's own GPU
+check is bypassed only here, so no kernel is involved."""
+import ctypes
+
+import pytest
+import torch
+
+import group_scale_search_b200 as tq
+
+
+class _FakeLib:
+    """Records calls; size queries return fixed byte counts, calls return TQ_OK."""
+
+    def __init__(self):
+        self.calls = []
+
+    def __getattr__(self, name):
+        def fn(*args):
+            self.calls.append((name, args))
+            return 4096 if name.endswith("_workspace_bytes") else 0
+        return fn
+
+
+def _desc(arg):
+    d = arg._obj if hasattr(arg, "_obj") else arg
+    return (d.dtype, d.n_mat, d.rows, d.cols, d.ld, d.mat_stride)
+
+
+@pytest.fixture
+def fake(monkeypatch):
+    lib = _FakeLib()
+    monkeypatch.setattr(tq, "lib", lambda: lib)
+    monkeypatch.setattr(tq, "_cuda", lambda t, name: t)
+    monkeypatch.setattr(tq, "_stream", lambda stream=None: None)
+    return lib
+
+
+def _last(lib, name):
+    return [a for n, a in lib.calls if n == name][-1]
+
+
+def test_matrix_descriptors(fake):
+    W = torch.zeros((3, 40, 264), dtype=torch.bfloat16)[:, 2:34, :256]      # padded rows and a matrix stride
+    assert _desc(tq._mat(W, "W")) == (1, 3, 32, 256, 264, 40 * 264)
+    W2 = torch.zeros((32, 136))[:, :128]                                    # one fp32 matrix, ld 136
+    assert _desc(tq._mat(W2, "W")) == (0, 1, 32, 128, 136, 0)
+    with pytest.raises(tq.TQError):
+        tq._mat(torch.zeros((4, 8), dtype=torch.float16), "W")
+    with pytest.raises(tq.TQError):
+        tq._mat(torch.zeros((8, 4)).t(), "W")                               # last dimension not contiguous
+
+
+def test_gptq_marshalling(fake):
+    W = torch.zeros((2, 16, 128), dtype=torch.bfloat16)
+    U1 = torch.zeros((128, 132))[:, :128]                                   # one factor, rows of 132
+    codes, loss = tq.tq_gptq_sweep(W, tq.INT4_G128_ASYM, torch.zeros(2 * 16), torch.zeros(2 * 16, dtype=torch.uint8),
+                                   U1)
+    args = _last(fake, "tq_gptq_sweep")
+    assert _desc(args[0]) == (1, 2, 16, 128, 128, 16 * 128)
+    assert args[1] == tq.INT4_G128_ASYM and args[5] == 132 and args[6] == 0
+    assert codes.shape == (2, 16, 128) and codes.dtype == torch.int8
+    assert loss.shape == (2, 16) and loss.dtype == torch.float64
+    assert args[10] == 4096                                                 # the size the library asked for
+    U3 = torch.zeros((2, 128, 128))                                         # one factor per matrix
+    tq.tq_gptq_sweep(W, tq.INT3_G64_SYM, torch.zeros(64), None, U3, want_loss=False)
+    args = _last(fake, "tq_gptq_sweep")
+    assert args[5] == 128 and args[6] == 128 * 128 and args[8] is None
+    with pytest.raises(ValueError):
+        tq.tq_gptq_sweep(W, tq.INT3_G64_SYM, torch.zeros(64), None, torch.zeros((128, 128), dtype=torch.float64))
+
+
+def test_proxy_full_marshalling(fake):
+    X = torch.zeros((2, 300, 200), dtype=torch.bfloat16)
+    W = torch.zeros((2, 48, 208), dtype=torch.bfloat16)[:, :, :200]
+    num, den = tq.tq_proxy_error_full(X, W, torch.zeros(16, dtype=torch.uint8), tq.INT3_G64_SYM, torch.zeros(8),
+                                      None, None)
+    args = _last(fake, "tq_proxy_error_full")
+    assert _desc(args[0]) == (1, 2, 300, 200, 200, 300 * 200)
+    assert _desc(args[1]) == (1, 2, 48, 200, 208, 48 * 208)
+    assert args[3] == tq.INT3_G64_SYM and args[10] == 4096
+    assert num.shape == (2,) and den.dtype == torch.float64
+
+
+def test_hessian_marshalling(fake):
+    X = torch.zeros((3, 100, 64), dtype=torch.bfloat16)
+    H = tq.tq_hessian(X, alpha=0.5, accumulate=True)
+    args = _last(fake, "tq_hessian")
+    assert H.shape == (3, 64, 64) and H.dtype == torch.float32 and not H.any()      # accumulate starts from zeros
+    assert args[2] == 64 and args[3] == 64 * 64 and abs(args[4].value - 0.5) < 1e-7 and args[5] == 1
+    with pytest.raises(ValueError):
+        tq.tq_hessian(X, out=torch.zeros((3, 64, 65)))
