@@ -19,6 +19,8 @@ class _FakeLib:
     def __getattr__(self, name):
         def fn(*args):
             self.calls.append((name, args))
+            if name == "tq_packed_bytes":
+                return 1234
             return 4096 if name.endswith("_workspace_bytes") else 0
         return fn
 
@@ -91,3 +93,46 @@ def test_hessian_marshalling(fake):
     assert args[2] == 64 and args[3] == 64 * 64 and abs(args[4].value - 0.5) < 1e-7 and args[5] == 1
     with pytest.raises(ValueError):
         tq.tq_hessian(X, out=torch.zeros((3, 64, 65)))
+
+
+def test_search_marshalling(fake):
+    """Output shapes and dtypes per format (from the group sizes), the packed
+    buffer sized by the library's answer, the imatrix stride (per matrix or
+    shared) and the grid parameters."""
+    W = torch.zeros((2, 8, 300), dtype=torch.bfloat16)
+    m2 = torch.zeros((2, 304))[:, :300]
+    for fmt, g in [(tq.INT3_G64_SYM, 64), (tq.INT4_G128_ASYM, 128), (tq.INT4_G64_ASYM, 64), (tq.NVFP4_G16, 16)]:
+        r = tq.tq_search_groups(W, m2, fmt)
+        args = _last(fake, "tq_search_groups")
+        G = -(-300 // g)
+        assert r.scales.shape == (2, 8, G)
+        assert r.scales.dtype == (torch.uint8 if fmt == tq.NVFP4_G16 else torch.float32)
+        assert (r.zeros is not None) == (fmt in (tq.INT4_G128_ASYM, tq.INT4_G64_ASYM))
+        assert (r.global_scale is not None) == (fmt == tq.NVFP4_G16)
+        assert r.cand_idx.shape == (2, 8, G) and r.loss.dtype == torch.float64
+        assert r.packed.numel() == 1234
+        assert args[2] == 304 and args[3] == fmt
+        p = args[4]._obj
+        assert (p.sym_n1, p.sym_n2, p.asym_n_scale, p.asym_n_zero, p.fp4_window) == (32, 32, 64, 32, 16)
+    tq.tq_search_groups(W, torch.zeros(300), tq.INT3_G64_SYM, params=tq.SearchParams(sym_n1=16), pack=False)
+    args = _last(fake, "tq_search_groups")
+    assert args[2] == 0 and args[4]._obj.sym_n1 == 16 and args[10] is None
+
+
+def test_gemv_marshalling(fake):
+    """x shared by every matrix ([B, I], matrix stride 0) or one per matrix
+    ([n_mat, B, I]); the output [n_mat, B, O]; shapes that do not fit are refused."""
+    packed = torch.zeros(64, dtype=torch.uint8)
+    x = torch.zeros((3, 256), dtype=torch.bfloat16)
+    y = tq.tq_dequant_gemv(packed, tq.INT4_G128_ASYM, torch.zeros(4), torch.zeros(4, dtype=torch.uint8), None,
+                           2, 10, 256, x)
+    args = _last(fake, "tq_dequant_gemv")
+    assert y.shape == (2, 3, 10) and args[9] == 1 and args[10] == 3 and args[11] == 0
+    x3 = torch.zeros((2, 5, 256))
+    tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.zeros(4), None, None, 2, 10, 256, x3)
+    args = _last(fake, "tq_dequant_gemv")
+    assert args[9] == 0 and args[10] == 5 and args[11] == 5 * 256
+    with pytest.raises(ValueError):
+        tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.zeros(4), None, None, 2, 10, 255, x)
+    with pytest.raises(ValueError):
+        tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.zeros(4), None, None, 3, 10, 256, x3)
