@@ -33,7 +33,7 @@ from __future__ import annotations
 
 import dataclasses
 import zlib
-from typing import Dict, List, Optional
+from typing import Dict, List
 
 import torch
 

@@ -2,7 +2,6 @@
 arguments each call passes through the C ABI (descriptor shapes and strides,
 factor strides, output shapes, workspace sizing).  The binding's own GPU
 check is bypassed only here, so no kernel is involved."""
-import ctypes
 
 import pytest
 import torch

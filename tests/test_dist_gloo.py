@@ -9,7 +9,6 @@ import socket
 import time
 
 import numpy as np
-import pytest
 
 import dist_workers
 from group_scale_search_b200.dist import shard_range, shard_units
