@@ -3,27 +3,40 @@
 path on B200 -- imatrix -> group-scale search with fused RTN + pack ->
 dequant -> imatrix-weighted proxy error -- one JSON line on rank 0.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c1] [--impl tq|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config c2] [--impl tq|reference]
+                  [--workloads all|none|c0,c1,...] [--scaling strong|weak]
 
-A step is one pass of every row of the path over one batch of synthetic input
-(the workload named by --config; default: the dense int4-g128 4096 x 4096
-workload).  `value` is device-timed with inputs resident in HBM (CUDA events,
-barrier + synchronize on both sides, max over ranks); `e2e` repeats the step
-through the public API starting from pinned host buffers, with the host->device
-copies of the inputs and the device->host read of the results inside the
-timed region.  `roofline` reports the dominant kernel (the search) against the
-FP32 CUDA-core issue peak.  Under torchrun every rank quantizes its own
-independent copy of the workload (weak scaling; no collective on the data
-path).  --impl reference times the CPU oracle on a bounded sample instead.
+A step is one pass of every row of the path over one batch of synthetic input.
+The headline workload (--config, default c2: the int3-g64 MoE stack of 64
+experts of 2048 x 7168, the largest workload that is one job on one GPU)
+carries the line's `value`, `roofline`, `e2e` and `cpu_baseline`; every other
+workload gets a row of the same figures under `per_workload`.  `value` is
+device-timed with inputs resident in HBM (CUDA events, barrier + synchronize
+on both sides, max over ranks); `e2e` repeats the step through the public API
+from pinned host buffers, with the host->device copies of the inputs and the
+device->host read of the results inside the timed region.  `roofline` reports
+the dominant kernel (the search) against the FP32 CUDA-core issue peak;
+`hbm_rows` the streaming kernels against the HBM peak.
+
+--gpus N > 1 without a launcher re-executes this script under
+torch.distributed.run with N ranks (one per GPU, NCCL).  With --scaling strong
+(the default) the ranks split one workload the way the method partitions: the
+experts of a MoE stack (no exchange), or the rows of every dense matrix with
+the calibration tokens split too (an all-reduce of the per-column sums of x^2
+and of the per-matrix (num, den) pairs).  --scaling weak gives every rank its
+own independent copy of the workload.  --impl reference times the CPU oracle
+on bounded samples of the same workload instead (rank 0 alone).
 """
 from __future__ import annotations
 
 import argparse
 import ctypes
+import dataclasses
 import datetime
 import json
 import math
 import os
+import socket
 import statistics
 import subprocess
 import sys
@@ -41,9 +54,11 @@ import synth  # noqa: E402
 
 METRIC = "weights quantized/sec (search+pack) on 1 B200; % of FP32 / HBM roofline"
 L2_BYTES = 126 * 2 ** 20
+WORKLOAD_ORDER = ["c0", "c1", "c2", "c3", "c4"]
 # FP32 lane-instructions per weight of the search (the dominant kernel):
 # candidate-element evaluations per weight x instructions per evaluation
-# (sym int3: 96 x 7; asym int4: 1024 x 5; NVFP4: 16 x 10).
+# (sym int3: 96 x 7; asym int4: 1024 x 5; NVFP4: 16 x 10).  An algorithmic
+# model of the work, not a count of what the kernels issue.
 SEARCH_INSTR_PER_W = {"int3_g64_sym": 96 * 7, "int4_g128_asym": 1024 * 5, "nvfp4_g16": 16 * 10}
 SEARCH_CEE_PER_W = {"int3_g64_sym": 96, "int4_g128_asym": 1024, "nvfp4_g16": 16}
 # our kernels per call: imatrix 2 (partial + final), search 1 (NVFP4: amax +
@@ -66,6 +81,16 @@ def peaks():
     return p
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # ------------------------------------------------------------------ clocks
 
 class ClockSampler:
@@ -84,7 +109,7 @@ class ClockSampler:
             self.uuid = None
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.uuid:
             cmd[1:1] = ["-i", self.uuid]
         try:
@@ -117,19 +142,90 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(sm)}
 
 
+# ------------------------------------------------------------------ sharding over ranks
+
+@dataclasses.dataclass
+class Shard:
+    """This rank's part of a workload split over `world` ranks.
+
+    pieces[k] = (axis, start, end, extent) for timed unit k of the whole
+    workload: "experts" (a range of the matrices of a MoE stack) or "rows" (a
+    range of the rows of a dense matrix).  site_tokens maps a calibration
+    site whose tokens are split to its total token count (its imatrix is the
+    all-reduced sum of x^2 over every rank's tokens divided by that count)."""
+    world: int
+    rank: int
+    pieces: list
+    site_tokens: dict
+    row_units: list      # indices (into this rank's units) of row-split matrices: their (num, den) are all-reduced
+
+
+def shard_plan(layout, world: int, rank: int):
+    """The partition of the method's independent units over ranks: experts of
+    a MoE stack split in contiguous ranges (no exchange); a dense matrix
+    split by rows, its calibration site by tokens (sizes differ by at most
+    one).  Returns [(axis, start, end, extent)] per timed unit and the token
+    ranges {site: (t0, t1, T)}."""
+    from group_scale_search_b200.dist import shard_range
+    pieces, tokens = [], {}
+    for name, fmt, (E, O, I), site, timed in layout["units"]:
+        if not timed:
+            continue
+        if E > 1:
+            e0, e1 = shard_range(E, rank, world)
+            pieces.append(("experts", e0, e1, E))
+        else:
+            o0, o1 = shard_range(O, rank, world)
+            pieces.append(("rows", o0, o1, O))
+            if site not in tokens:
+                T = layout["sites"][site][1]
+                tokens[site] = shard_range(T, rank, world) + (T,)
+    return pieces, tokens
+
+
+def shard_workload(wl, world: int, rank: int):
+    """This rank's own copy of its part of `wl` (units and sites cloned, so
+    the whole workload can be freed) and its Shard description."""
+    units_all = [u for u in wl.units if u.timed]
+    lay = {"units": [(u.name, u.fmt, tuple(u.W.shape), u.site, True) for u in units_all],
+           "sites": {k: tuple(s.X.shape) + (str(s.X.dtype),) for k, s in wl.sites.items()}}
+    pieces, tokens = shard_plan(lay, world, rank)
+    units, sites, row_units = [], {}, []
+    for u, (axis, a, b, n) in zip(units_all, pieces):
+        if b <= a:
+            continue
+        X = wl.sites[u.site].X
+        if axis == "experts":
+            W = u.W[a:b].clone()
+            sites[u.site] = synth.Site(u.site, X[a:b].clone())
+        else:
+            W = u.W[:, a:b].clone()
+            if u.site not in sites:
+                t0, t1, T = tokens[u.site]
+                sites[u.site] = synth.Site(u.site, X[:, t0:t1].clone())
+            row_units.append(len(units))
+        units.append(synth.Unit(u.name, u.fmt, W, u.site))
+    site_tokens = {k: v[2] for k, v in tokens.items() if k in sites}
+    return synth.Workload(wl.name, units, sites), Shard(world, rank, pieces, site_tokens, row_units)
+
+
 # ------------------------------------------------------------------ the step
 
 class Step:
     """One pass of the whole path over one input set, on the current stream."""
 
-    def __init__(self, tq, wl, sets):
+    def __init__(self, tq, wl, sets, shard=None):
         self.tq = tq
         self.wl = wl
         self.sets = sets            # list of (sites dict name->X, units list of W)
+        self.shard = shard
         self.fmts = [tq.FORMATS[u.fmt] for u in wl.units if u.timed]
         self.units = [u for u in wl.units if u.timed]
         dev = self.units[0].W.device
-        # preallocated outputs and workspaces (the timed region allocates nothing)
+        # preallocated outputs and workspaces (the timed region allocates
+        # nothing); the search writes what the metric needs -- scales,
+        # zeros, global scales and the packed records -- and no per-group
+        # candidate index or loss
         self.m = {}
         self.ws_im = {}
         for name, site in wl.sites.items():
@@ -142,7 +238,7 @@ class Step:
         for u, fmt in zip(self.units, self.fmts):
             E, O, I = u.W.shape
             m = self._m_for(u)
-            self.res.append(tq.tq_search_groups(u.W, m, fmt))
+            self.res.append(tq.tq_search_groups(u.W, m, fmt, want_idx=False, want_loss=False))
             self.dq.append(torch.empty((E, O, I), dtype=torch.bfloat16, device=dev))
             self.px.append((torch.empty(E, dtype=torch.float64, device=dev),
                             torch.empty(E, dtype=torch.float64, device=dev)))
@@ -164,6 +260,7 @@ class Step:
     def __call__(self, k: int, time_search: bool = False):
         tq = self.tq
         sites, Ws = self.sets[k % len(self.sets)]
+        split_tokens = self.shard.site_tokens if self.shard is not None else {}
 
         def mark():
             if not time_search:
@@ -175,9 +272,16 @@ class Step:
         for name in self.m:
             X = sites[name]
             a = mark()
-            tq.tq_imatrix(X, m=self.m[name], alpha=1.0 / X.shape[1], workspace=self.ws_im[name])
+            if name in split_tokens:      # this rank's tokens: sums of x^2, then the sum over ranks / T
+                from group_scale_search_b200.dist import allreduce_imatrix
+                tq.tq_imatrix(X, m=self.m[name], alpha=1.0, workspace=self.ws_im[name])
+                b = mark()
+                self.m[name].copy_(allreduce_imatrix(self.m[name], split_tokens[name]))
+            else:
+                tq.tq_imatrix(X, m=self.m[name], alpha=1.0 / X.shape[1], workspace=self.ws_im[name])
+                b = mark()
             if time_search:
-                self.row_events.append(("imatrix", X.numel() * X.element_size(), a, mark()))
+                self.row_events.append(("imatrix", X.numel() * X.element_size(), a, b))
         for i, (u, fmt) in enumerate(zip(self.units, self.fmts)):
             W = Ws[i]
             m = self._m_for(u)
@@ -199,6 +303,11 @@ class Step:
                 self.row_events.append(("proxy", W.numel() * W.element_size() + r.packed.numel()
                                         + r.scales.numel() * r.scales.element_size()
                                         + (0 if r.zeros is None else r.zeros.numel()), c, mark()))
+            if self.shard is not None and i in self.shard.row_units:   # whole-matrix (num, den)
+                from group_scale_search_b200.dist import allreduce_proxy
+                num, den = allreduce_proxy(*self.px[i])
+                self.px[i][0].copy_(num)
+                self.px[i][1].copy_(den)
 
 
 def make_sets(wl, n_sets):
@@ -217,24 +326,68 @@ def input_bytes(wl):
     return b
 
 
+# ------------------------------------------------------------------ configuration (shared by both arms)
+
+_GROUP = {"int3_g64_sym": 64, "int4_g128_asym": 128, "nvfp4_g16": 16}
+
+
+def workload_weights(name: str, scale: float = 1.0) -> int:
+    lay = synth.layout(name, scale)
+    return sum(E * O * I for _, _, (E, O, I), _, timed in lay["units"] if timed)
+
+
+def config_dict(name: str, scale: float, world: int, scaling: str) -> dict:
+    """The workload and how the job runs it, from shapes alone (both arms
+    print the same dictionary)."""
+    lay = synth.layout(name, scale)
+    units = [u for u in lay["units"] if u[4]]
+    nw = sum(E * O * I for _, _, (E, O, I), _, _ in units)
+    groups = sum(E * O * (-(-I // _GROUP[fmt])) for _, fmt, (E, O, I), _, _ in units)
+    nbytes = sum(E * O * I * (4 if name == "c0" else 2) for _, _, (E, O, I), _, _ in units)
+    nbytes += sum(E * T * I * (4 if dt == "f32" else 2) for s, (E, T, I, dt) in lay["sites"].items()
+                  if any(u[3] == s for u in units))
+    per_rank = nbytes / world if scaling == "strong" else nbytes
+    n_sets = max(1, min(64, math.ceil(2 * L2_BYTES / per_rank)))
+    job = nw * (world if scaling == "weak" else 1)
+    if world == 1:
+        par = "one GPU"
+    elif scaling == "strong":
+        par = (f"strong x{world}: " + ("experts split over ranks, no exchange" if units[0][2][0] > 1 else
+                                       "rows of every matrix and calibration tokens split over ranks; "
+                                       "all-reduce of sum x^2 per column and of (num, den) per matrix"))
+    else:
+        par = f"weak x{world}: an independent copy of the workload per GPU"
+    return {"workload": f"{name}: {synth.DESCRIPTIONS[name]}" + ("" if scale == 1.0 else f" (scaled x{scale})"),
+            "weights": job, "groups": groups * (world if scaling == "weak" else 1),
+            "step": "imatrix + search with fused RTN/pack + dequant(bf16) + proxy error",
+            "l2": (f"{n_sets} rotating input sets per GPU, {n_sets * per_rank / 2**20:.0f} MiB > 126 MiB L2"
+                   if n_sets * per_rank > L2_BYTES else
+                   f"{n_sets} input sets per GPU ({n_sets * per_rank / 2**20:.1f} MiB) fit in L2"),
+            "parallelism": par}
+
+
 # ------------------------------------------------------------------ CPU oracle baseline
 
-def oracle_sample(wl, budget_s: float = 12.0):
-    """Times the oracle (as it stands) on a bounded sample of the workload:
-    for each unit, the imatrix of its site (first matrix) and search + pack +
-    dequant + proxy error over the first rows of its first matrix, the row
-    count sized to about `budget_s` seconds.  Returns (weights/s, cores,
-    description, seconds)."""
+def oracle_rows(wl, budget_s: float):
+    """Rows per unit for an oracle sample of about `budget_s` seconds."""
     import oracle
     oracle.build()
     units = [u for u in wl.units if u.timed]
-    # size the sample: rows per unit so that the search takes ~budget_s in total
     probe_rows = 8
     t0 = time.perf_counter()
-    for u in units[:1]:
-        _oracle_unit(oracle, wl, u, probe_rows)
+    _oracle_unit(oracle, wl, units[0], probe_rows)
     per_row = (time.perf_counter() - t0) / probe_rows
-    rows = max(8, min(units[0].W.shape[1], int(budget_s / max(per_row, 1e-6))))
+    return max(8, min(units[0].W.shape[1], int(budget_s / max(per_row, 1e-6) / len(units))))
+
+
+def oracle_sample(wl, rows: int):
+    """Times the oracle (as it stands) on a bounded sample of the workload:
+    for each unit, the imatrix of its site (first matrix) and search + pack +
+    dequant + proxy error over the first `rows` rows of its first matrix.
+    Returns (weights/s, cores, description, seconds, weights)."""
+    import oracle
+    oracle.build()
+    units = [u for u in wl.units if u.timed]
     t0 = time.perf_counter()
     n = 0
     for u in units:
@@ -243,8 +396,9 @@ def oracle_sample(wl, budget_s: float = 12.0):
         n += r * u.W.shape[2]
     dt = time.perf_counter() - t0
     desc = (f"oracle (C, fp64, OpenMP) on {rows} rows of the first matrix of each of {len(units)} unit(s) "
-            f"= {n} weights: imatrix of the site's columns over all tokens, search+pack, dequant, proxy")
-    return n / dt, oracle.num_threads(), desc, dt
+            f"= {n} weights: imatrix of the site's first matrix over all its tokens, search+pack, dequant, "
+            f"proxy; host CPU {cpu_model()}")
+    return n / dt, oracle.num_threads(), desc, dt, n
 
 
 def oracle_one_thread(config: str, frac: float = 0.01):
@@ -252,15 +406,14 @@ def oracle_one_thread(config: str, frac: float = 0.01):
     process, so the parent's thread pool is untouched) over a fixed `frac` of
     the first unit's rows: the scaling reference for the multi-core figure.
     Returns (weights/s, description) or None if the child fails."""
-    import subprocess
-    code = (f"import json, time, synth, bench, oracle; oracle.build(); wl = synth.make({config!r}, 'cpu'); "
+    code = (f"import json, time, synth, bench, oracle; oracle.build(); wl = synth.make({config!r}, 'cpu', max_mats=1); "
             f"u = [x for x in wl.units if x.timed][0]; rows = max(8, int(u.W.shape[1] * {frac!r})); "
             f"t0 = time.perf_counter(); bench._oracle_unit(oracle, wl, u, rows); dt = time.perf_counter() - t0; "
             f"print(json.dumps([rows * u.W.shape[2] / dt, rows, u.W.shape[2], oracle.num_threads(), dt]))")
     env = dict(os.environ, OMP_NUM_THREADS="1")
     try:
         r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True, timeout=300, env=env,
-                           cwd=os.path.dirname(os.path.abspath(__file__)))
+                           cwd=ROOT)
         v, rows, cols, threads, dt = json.loads(r.stdout.strip().splitlines()[-1])
     except Exception:   # noqa: BLE001 -- the figure is optional context
         return None
@@ -288,36 +441,67 @@ def _oracle_unit(oracle, wl, u, rows):
     oracle.proxy_error(W[0], What, m)
 
 
-def read_traffic(path, workload):
-    """DRAM bytes per launch of the dominant kernel from the profiles table."""
+def read_profile(path, workload, kernel):
+    """The ncu figures of `kernel` on `workload` from the profiles table:
+    DRAM bytes per launch (read + write) and the FP32-pipe share of issue,
+    or None where the table has no entry."""
+    out = {"traffic": None, "fp32_pipe_frac": None, "source": None}
     try:
         for line in open(path):
             cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 3 and cells[0] == workload and cells[2].isdigit():
-                return int(cells[2])
+            if len(cells) >= 6 and cells[0] == workload and cells[1] == kernel:
+                out["traffic"] = int(cells[2]) if cells[2].isdigit() else None
+                try:
+                    out["fp32_pipe_frac"] = float(cells[4])
+                except ValueError:
+                    pass
+                out["source"] = cells[5]
     except OSError:
         pass
-    return None
+    return out
 
 
-# ------------------------------------------------------------------ main
+# ------------------------------------------------------------------ arguments and launch
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=100)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--config", default="c1", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="c2", choices=WORKLOAD_ORDER,
+                    help="the headline workload (default c2, the largest one-GPU workload)")
+    ap.add_argument("--workloads", default="all",
+                    help="workloads timed beside the headline, each as a per_workload row: "
+                         "'all', 'none' or a comma list")
+    ap.add_argument("--scaling", default="strong", choices=["strong", "weak"],
+                    help="N > 1: split one workload over the ranks (strong) or give each its own (weak)")
     ap.add_argument("--impl", default="tq", choices=["tq", "reference"])
     ap.add_argument("--scale", type=float, default=1.0,
                     help="shrink the workload (profiling and tests only; the reported line is for scale 1)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--traffic-table", default=os.path.join(ROOT, "profiles", "traffic.md"),
-                    help="ncu DRAM bytes per launch of the dominant kernel, by workload")
+    ap.add_argument("--no-next-rows", action="store_true", help="skip the rows beyond the step")
+    ap.add_argument("--plan-only", action="store_true",
+                    help="print how the ranks split the workload (CPU and gloo without a GPU) and exit")
+    ap.add_argument("--profile-table", default=os.path.join(ROOT, "profiles", "traffic.md"),
+                    help="ncu DRAM bytes per launch and FP32-pipe share by workload and kernel")
     ap.add_argument("--jsonl", default=None,
                     help="also append the result line, with a UTC time stamp and the git revision, to this file")
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+def _free_port() -> int:
+    with socket.socket(socket.AF_INET, socket.SOCK_STREAM) as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def spawn_ranks(args) -> int:
+    """--gpus N with no launcher: run this script under torch.distributed.run
+    with N local ranks (rank 0 prints the line) and return its exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", f"--master-port={_free_port()}", os.path.abspath(__file__)] + sys.argv[1:]
+    return subprocess.call(cmd, cwd=ROOT)
 
 
 def append_jsonl(path, line):
@@ -333,26 +517,33 @@ def append_jsonl(path, line):
         f.write(json.dumps(rec) + "\n")
 
 
+# ------------------------------------------------------------------ the reference arm (the oracle)
+
 def reference_arm(args, world, rank):
+    """The oracle as it stands on the host cores: every step is the same
+    bounded sample of the headline workload (the first rows of the first
+    matrix of every unit, sized once to about 2 s), timed on its own."""
     if rank != 0:
         return 0
-    wl = synth.make(args.config, "cpu", seed=0)
-    nw = wl.n_weights
-    vals = []
+    wl = synth.make(args.config, "cpu", seed=0, scale=args.scale, max_mats=1)
+    rows = oracle_rows(wl, budget_s=2.0)
     for _ in range(args.warmup):
-        oracle_sample(wl, budget_s=2.0)
-    desc = cores = None
+        oracle_sample(wl, max(8, rows // 4))
+    vals, secs = [], []
+    desc = cores = n = None
     for _ in range(args.steps):
-        v, cores, desc, dt = oracle_sample(wl, budget_s=4.0)
+        v, cores, desc, dt, n = oracle_sample(wl, rows)
         vals.append(v)
-    v = statistics.median(vals)
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": nw / v * 1e3,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic",
-            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}", "weights": nw},
+        secs.append(dt)
+    dt = statistics.median(secs)
+    v = n / dt
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": 0,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+            "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_dict(args.config, args.scale, args.gpus, args.scaling),
+            "step_definition": f"one bounded sample of the workload per step ({n} weights), host cores only",
             "cpu_baseline": {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
-                             "sample": desc},
+                             "sample": desc, "cpu": cpu_model(), "seconds_per_step": dt},
             "e2e": {"value": v, "unit": "weights/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     if args.jsonl:
@@ -360,31 +551,142 @@ def reference_arm(args, world, rank):
     return 0
 
 
-def main():
-    args = parse()
+# ------------------------------------------------------------------ the tq arm
+
+def plan_only(args, world, rank):
+    """How the ranks split each workload: every rank builds the (scaled)
+    workload's shapes, takes its part, and rank 0 gathers and checks that
+    every expert / row / token is covered exactly once."""
+    import torch.distributed as dist
+    names = [args.config] + [w for w in _other_workloads(args) if w != args.config]
+    out = {}
+    for name in names:
+        lay = synth.layout(name, args.scale)
+        pieces, tokens = shard_plan(lay, world, rank)
+        mine = {"rank": rank, "pieces": pieces, "tokens": {k: list(v) for k, v in tokens.items()}}
+        got = [None] * world
+        if world > 1:
+            dist.all_gather_object(got, mine)
+        else:
+            got = [mine]
+        units = [u for u in lay["units"] if u[4]]
+        ok = True
+        for k, u in enumerate(units):
+            axis = got[0]["pieces"][k][0]
+            extent = got[0]["pieces"][k][3]
+            cover = np.zeros(extent, np.int64)
+            for g in got:
+                _, a, b, _ = g["pieces"][k]
+                cover[a:b] += 1
+            ok &= bool((cover == 1).all())
+        for site in got[0]["tokens"]:
+            T = got[0]["tokens"][site][2]
+            cover = np.zeros(T, np.int64)
+            for g in got:
+                a, b, _ = g["tokens"][site]
+                cover[a:b] += 1
+            ok &= bool((cover == 1).all())
+        out[name] = {"ranks": got, "covered_once": ok}
+    if rank == 0:
+        print(json.dumps({"plan": out, "world": world}), flush=True)
+    return 0
+
+
+def _other_workloads(args):
+    if args.workloads == "none":
+        return []
+    if args.workloads == "all":
+        return [w for w in WORKLOAD_ORDER if w != args.config]
+    return [w.strip() for w in args.workloads.split(",") if w.strip() and w.strip() != args.config]
+
+
+def main(argv=None):
+    args = parse(argv)
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+    env_world = os.environ.get("WORLD_SIZE")
+    if env_world is None and args.gpus > 1:
+        return spawn_ranks(args)
+    if env_world is not None and int(env_world) != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but the launcher started {env_world} ranks")
     if args.impl == "reference":   # rank 0 alone times the oracle; no process group
-        return reference_arm(args, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return reference_arm(args, int(env_world or "1"), int(os.environ.get("RANK", "0")))
+
+    from group_scale_search_b200.dist import init_from_env
+    backend = "nccl" if torch.cuda.is_available() and not args.plan_only else "gloo"
+    world, rank, local = init_from_env(backend, timeout_s=120.0)
+    if args.plan_only:
+        rc = plan_only(args, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+            dist.destroy_process_group()
+        return rc
 
     import group_scale_search_b200 as tq
-    from group_scale_search_b200.dist import init_from_env, max_over_ranks
-    world, rank, local = init_from_env("nccl", timeout_s=120.0)
     if world == 1:
         torch.cuda.set_device(0)
     tq.lib()
     dev = torch.device("cuda", torch.cuda.current_device())
-    wl = synth.make(args.config, dev, seed=rank, scale=args.scale)
-    nbytes = input_bytes(wl)
-    n_sets = max(1, min(64, math.ceil(2 * L2_BYTES / nbytes)))
-    sets = make_sets(wl, n_sets)
-    step = Step(tq, wl, sets)
-    nw = sum(u.W.numel() for u in step.units)
-    stream = torch.cuda.current_stream()
 
     def barrier():
         if world > 1:
             import torch.distributed as dist
             dist.barrier()
+
+    pk = peaks()
+    headline, wl_head = run_workload(tq, args.config, args, world, rank, dev, barrier, pk, keep_wl=True)
+    per = {}
+    for name in _other_workloads(args):
+        row, _ = run_workload(tq, name, args, world, rank, dev, barrier, pk)
+        per[name] = row
+
+    line = {"metric": METRIC, "value": headline["value"], "unit": "weights/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": headline["ms_per_step"],
+            "higher_is_better": True, "scaling": args.scaling if world > 1 else "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": config_dict(args.config, args.scale, world, args.scaling),
+            "groups_per_s": headline["groups_per_s"],
+            "roofline": headline["roofline"], "hbm_rows": headline["hbm_rows"],
+            "next_rows": headline.get("next_rows"), "clocks": headline["clocks"], "e2e": headline.get("e2e"),
+            "gpu_launches": headline["gpu_launches"],
+            "per_workload": per}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rows = oracle_rows(wl_head, budget_s=12.0)
+        v, cores, desc, dt, _ = oracle_sample(wl_head, rows)
+        line["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": dt, "cpu": cpu_model()}
+        one = oracle_one_thread(args.config)
+        if one is not None:
+            line["cpu_baseline"]["one_thread"] = {"value": one[0], "unit": "weights/s", "sample": one[1]}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+        if args.jsonl:
+            append_jsonl(args.jsonl, line)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def run_workload(tq, name, args, world, rank, dev, barrier, pk, keep_wl=False):
+    """Times `steps` steps of workload `name` (this rank's part of it) and
+    the rows around the step; returns the row's figures (and the workload
+    when `keep_wl`, for the CPU baseline)."""
+    from group_scale_search_b200.dist import max_over_ranks
+    strong = world > 1 and args.scaling == "strong"
+    wl = synth.make(name, dev, seed=0 if strong else rank, scale=args.scale)
+    shard = None
+    if strong:
+        wl, shard = shard_workload(wl, world, rank)
+        torch.cuda.empty_cache()
+    nbytes = input_bytes(wl)
+    n_sets = max(1, min(64, math.ceil(2 * L2_BYTES / nbytes)))
+    sets = make_sets(wl, n_sets)
+    step = Step(tq, wl, sets, shard)
+    nw_rank = sum(u.W.numel() for u in step.units)
+    nw_job = workload_weights(name, args.scale) * (1 if strong else world)
+    stream = torch.cuda.current_stream()
 
     for k in range(args.warmup):
         step(k)
@@ -403,7 +705,7 @@ def main():
     torch.cuda.synchronize()
     ms = max_over_ranks(ev0.elapsed_time(ev1), dev)
     ms_step = ms / args.steps
-    value = world * nw / (ms_step * 1e-3)
+    value = nw_job / (ms_step * 1e-3)
 
     # dominant kernel: the search (CUDA events on the launching stream)
     by_fmt = {}
@@ -413,83 +715,72 @@ def main():
         d[1] += n
     fmt_main = max(by_fmt, key=lambda f: by_fmt[f][0])
     search_ms = by_fmt[fmt_main][0] / args.steps
-    w_per_launch = by_fmt[fmt_main][1] / args.steps
-    pk = peaks()
+    w_per_launch = by_fmt[fmt_main][1] / args.steps / max(1, sum(1 for u in step.units if u.fmt == fmt_main))
+    n_launch = sum(1 for u in step.units if u.fmt == fmt_main)
     props = torch.cuda.get_device_properties(dev)
     sms = props.multi_processor_count
     peak_tinst = sms * 128 * pk["sm_max_mhz"] * 1e6 / 1e12
-    achieved = SEARCH_INSTR_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3) / 1e12
-    traffic = read_traffic(args.traffic_table, args.config)
+    achieved = SEARCH_INSTR_PER_W[fmt_main] * by_fmt[fmt_main][1] / args.steps / (search_ms * 1e-3) / 1e12
     clocks = clk.summary()
+    prof = read_profile(args.profile_table, name, f"search {fmt_main}")
     roofline = {"bound": "alu", "achieved": achieved, "peak": peak_tinst, "unit": "Tinst/s",
-                "frac": achieved / peak_tinst, "traffic": traffic,
-                "kernel": f"search {fmt_main}", "kernel_ms": search_ms,
+                "frac": achieved / peak_tinst, "traffic": prof["traffic"] if args.scale == 1.0 else None,
+                "kernel": f"search {fmt_main}", "kernel_ms": search_ms / n_launch, "launches_per_step": n_launch,
+                "weights_per_launch": w_per_launch,
                 "per_unit": f"{SEARCH_INSTR_PER_W[fmt_main]} FP32 lane-instr/weight "
-                            f"({SEARCH_CEE_PER_W[fmt_main]} candidate-element evaluations)",
+                            f"({SEARCH_CEE_PER_W[fmt_main]} candidate-element evaluations): an algorithmic "
+                            f"model of the work",
                 "peak_basis": f"{sms} SMs x 128 FP32 lanes x {pk['sm_max_mhz']:.0f} MHz ({pk['source']} max clock)",
                 "frac_at_observed_clock": (achieved / (sms * 128 * clocks["sm_mhz"] * 1e6 / 1e12))
                 if clocks.get("sm_mhz") else None,
-                "cee_per_s": SEARCH_CEE_PER_W[fmt_main] * w_per_launch / (search_ms * 1e-3)}
+                "cee_per_s": SEARCH_CEE_PER_W[fmt_main] * by_fmt[fmt_main][1] / args.steps / (search_ms * 1e-3),
+                "ncu_fp32_pipe_frac": prof["fp32_pipe_frac"], "ncu_source": prof["source"]}
 
     # every HBM-bound row of the step: algorithmic bytes / CUDA-event time vs the HBM peak
     rows = {}
-    for name, nbytes, a, b in step.row_events:
-        d = rows.setdefault(name, [0.0, 0])
+    for rname, nbytes_row, a, b in step.row_events:
+        d = rows.setdefault(rname, [0.0, 0, 0])
         d[0] += a.elapsed_time(b)
-        d[1] += nbytes
+        d[1] += nbytes_row
+        d[2] += 1
     hbm_rows = {}
-    for name, (t_ms, nbytes) in rows.items():
-        gbs = nbytes / (t_ms * 1e-3) / 1e9
-        hbm_rows[name] = {"ms": t_ms / args.steps, "bytes": nbytes // args.steps, "GB/s": gbs,
-                          "frac": gbs / pk["hbm_gbs"]}
+    kname = {"imatrix": "k_imatrix_partial", "dequant": "k_dequant", "proxy": "k_proxy"}
+    for rname, (t_ms, nb, cnt) in rows.items():
+        gbs = nb / (t_ms * 1e-3) / 1e9
+        p = read_profile(args.profile_table, name, kname[rname])
+        hbm_rows[rname] = {"ms": t_ms / args.steps, "bytes": nb // args.steps, "launches_per_step": cnt // args.steps,
+                           "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
+                           "ncu_traffic": p["traffic"] if args.scale == 1.0 else None}
     hbm_rows["pack"] = time_pack(tq, step, pk)
-    next_rows = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
-    if step.units[0].fmt == "int4_g128_asym":
-        next_rows["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
-        next_rows["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
-    next_rows["hessian"] = time_hessian(tq, step, pk)
-    next_rows["proxy_full_hessian"] = time_proxy_full(tq, step, pk)
-    next_rows["gptq_sweep"] = time_gptq(tq, step, peak_tinst)
-    next_rows["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
-    next_rows["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
-
-    # end to end through the public API from pinned host buffers
-    e2e = None
+    row = {"value": value, "ms_per_step": ms_step, "weights": nw_job, "weights_this_rank": nw_rank,
+           "groups_per_s": value / _GROUP[fmt_main], "roofline": roofline, "hbm_rows": hbm_rows,
+           "clocks": clocks, "gpu_launches": step.kernels_per_step() * args.steps,
+           "config": config_dict(name, args.scale, world, args.scaling)}
+    if not args.no_next_rows:
+        row["next_rows"] = next_rows(tq, step, pk, peak_tinst)
     if not args.no_e2e:
-        e2e = run_e2e(tq, wl, step, args, world, barrier, dev)
+        row["e2e"] = run_e2e(tq, wl, step, args, nw_job, barrier, dev)
+    del step, sets
+    if not keep_wl:
+        del wl
+        wl = None
+    torch.cuda.empty_cache()
+    return row, wl
 
-    line = {"metric": METRIC, "value": value, "unit": "weights/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": f"{args.config}: {synth.DESCRIPTIONS[args.config]}"
-                                   + ("" if args.scale == 1.0 else f" (scaled x{args.scale})"),
-                       "weights_per_gpu": nw,
-                       "groups_per_gpu": sum(tq.tq_num_groups(tq.FORMATS[u.fmt], u.W.shape[0] * u.W.shape[1],
-                                                              u.W.shape[2]) for u in step.units),
-                       "step": "imatrix + search with fused RTN/pack + dequant(bf16) + proxy error",
-                       "l2": (f"{n_sets} rotating input sets, {n_sets * nbytes / 2**20:.0f} MiB > 126 MiB L2"
-                              if n_sets * nbytes > L2_BYTES else
-                              f"{n_sets} input sets ({n_sets * nbytes / 2**20:.1f} MiB) fit in L2"),
-                       "parallelism": f"weak x{world}: independent workload per GPU"},
-            "groups_per_s": value / tq.tq_group_size(tq.FORMATS[fmt_main]),
-            "roofline": roofline, "hbm_rows": hbm_rows, "next_rows": next_rows, "clocks": clocks, "e2e": e2e,
-            "gpu_launches": step.kernels_per_step() * args.steps}
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc, dt = oracle_sample(wl)
-        line["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": dt}
-        one = oracle_one_thread(args.config)
-        if one is not None:
-            line["cpu_baseline"]["one_thread"] = {"value": one[0], "unit": "weights/s", "sample": one[1]}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
-        if args.jsonl:
-            append_jsonl(args.jsonl, line)
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-        dist.destroy_process_group()
-    return 0
+
+def next_rows(tq, step, pk, peak_tinst):
+    """The rows beyond the step, each on the first unit of the workload,
+    outside the step's timed region."""
+    out = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
+    if step.units[0].fmt == "int4_g128_asym":
+        out["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
+        out["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
+    out["hessian"] = time_hessian(tq, step, pk)
+    out["proxy_full_hessian"] = time_proxy_full(tq, step, pk)
+    out["gptq_sweep"] = time_gptq(tq, step, peak_tinst)
+    out["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
+    out["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
+    return out
 
 
 def time_pack(tq, step, pk, reps=12):
@@ -804,7 +1095,7 @@ def _empty_like_result(tq, r):
                            cand_idx=e(r.cand_idx), loss=e(r.loss), packed=e(r.packed))
 
 
-def run_e2e(tq, wl, step, args, world, barrier, dev):
+def run_e2e(tq, wl, step, args, nw_job, barrier, dev):
     """Same step from pinned host inputs: every step copies its inputs host ->
     device, runs the path and copies the quantized weights (packed codes +
     scales + zeros/global scales) and the proxy-error sums device -> host,
@@ -885,8 +1176,7 @@ def run_e2e(tq, wl, step, args, world, barrier, dev):
     barrier()
     from group_scale_search_b200.dist import max_over_ranks
     ms = max_over_ranks(a.elapsed_time(b), dev)
-    nw = sum(u.W.numel() for u in step.units)
-    return {"value": world * nw / (ms / steps * 1e-3), "unit": "weights/s", "h2d_bytes_per_step": h2d,
+    return {"value": nw_job / (ms / steps * 1e-3), "unit": "weights/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms / steps,
             "pipeline": "3 streams (copy-in, compute, copy-out), double-buffered inputs and outputs"}
 

@@ -213,6 +213,32 @@ def _m_stride(m: torch.Tensor) -> int:
     return m.stride(0) if m.dim() == 2 and m.shape[0] > 1 else 0
 
 
+def _check_m(m: torch.Tensor, n_mat: int, cols: int, name: str = "m", shared_ok: bool = True) -> torch.Tensor:
+    """An imatrix the kernels may read or write in place: fp32 on the GPU,
+    [cols] (one vector for every matrix, where allowed) or [n_mat, cols]
+    ([1, cols] for one matrix), unit column stride and rows at least cols
+    apart -- anything else would make a kernel touch memory outside the
+    tensor, so it is refused here."""
+    _cuda(m, name)
+    if m.dtype != torch.float32:
+        raise TQError(f"{name} must be float32, not {m.dtype}")
+    if m.dim() == 1:
+        if not shared_ok and n_mat > 1:
+            raise TQError(f"{name} must be [n_mat={n_mat}, {cols}]")
+        if m.shape[0] != cols:
+            raise TQError(f"{name} has {m.shape[0]} columns, expected {cols}")
+    elif m.dim() == 2:
+        if m.shape[1] != cols or m.shape[0] not in ((n_mat, 1) if shared_ok else (n_mat,)):
+            raise TQError(f"{name} is {tuple(m.shape)}, expected ({n_mat}, {cols})")
+        if m.shape[0] > 1 and m.stride(0) < cols:
+            raise TQError(f"{name}: rows overlap (stride {m.stride(0)} < {cols})")
+    else:
+        raise TQError(f"{name} must be [cols] or [n_mat, cols]")
+    if m.stride(-1) != 1:
+        raise TQError(f"{name} must have unit column stride")
+    return m
+
+
 def _groups(W: torch.Tensor, fmt: int):
     E, O, I = (W.unsqueeze(0) if W.dim() == 2 else W).shape
     g = _GROUP[fmt]
@@ -261,7 +287,7 @@ def tq_imatrix(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: Optiona
         alpha = 1.0 / d.rows
     if m is None:
         m = torch.zeros((d.n_mat, d.cols), dtype=torch.float32, device=X.device)
-    _cuda(m, "m")
+    _check_m(m, d.n_mat, d.cols, shared_ok=False)
     ws_bytes = int(lib().tq_imatrix_workspace_bytes(ctypes.byref(d)))
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=X.device)
@@ -306,7 +332,7 @@ def tq_search_fp8(W: torch.Tensor, m: torch.Tensor, n_cand: int = 64, lo: float 
     candidates fl32(r amax / 448) by the imatrix-weighted squared error; with
     pack=True the E4M3 codes of the chosen scale are written too."""
     d = _mat(W, "W")
-    _cuda(m, "m")
+    _check_m(m, d.n_mat, d.cols)
     E, O, I = d.n_mat, d.rows, d.cols
     dev = W.device
     if out is None:
@@ -360,7 +386,7 @@ def tq_lloyd_max_g32(W: torch.Tensor, m: torch.Tensor, n_iter: int = 16, start=L
     """imatrix-weighted Lloyd-Max 2-bit codebook on absmax-normalised 32-weight
     groups, shared by every matrix of W, and the 2-bit codes."""
     d = _mat(W, "W")
-    _cuda(m, "m")
+    _check_m(m, d.n_mat, d.cols)
     E, O, I = d.n_mat, d.rows, d.cols
     dev = W.device
     G = (I + 31) // 32
@@ -397,7 +423,7 @@ def tq_imatrix_static(X: torch.Tensor, m: Optional[torch.Tensor] = None, alpha: 
         alpha = 1.0 / d.rows
     if m is None:
         m = torch.zeros((d.n_mat, d.cols), dtype=torch.float32, device=X.device)
-    _cuda(m, "m")
+    _check_m(m, d.n_mat, d.cols, shared_ok=False)
     _check(lib().tq_imatrix_static(ctypes.byref(d), _ptr(m), _m_stride(m) if m.dim() == 2 else 0,
                                    ctypes.c_float(alpha), int(accumulate), _stream(stream)), "tq_imatrix_static")
     return m
@@ -422,7 +448,7 @@ def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optiona
     pack=True the chosen codes are rounded and packed in the same kernel.
     m: [I] (shared) or [n_mat, I] fp32 imatrix."""
     d = _mat(W, "W")
-    _cuda(m, "m")
+    _check_m(m, d.n_mat, d.cols)
     E, O, I, G = _groups(W, fmt)
     dev = W.device
     if out is None:
@@ -525,6 +551,7 @@ def tq_proxy_error(W: torch.Tensor, packed: torch.Tensor, fmt: int, scales: torc
                    workspace: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """(num, den) fp64 per matrix: tr(E H E^T), tr(W H W^T) with H = diag(m)."""
     d = _mat(W, "W")
+    _check_m(m, d.n_mat, d.cols)
     if out is None:
         out = (torch.empty(d.n_mat, dtype=torch.float64, device=W.device),
                torch.empty(d.n_mat, dtype=torch.float64, device=W.device))

@@ -103,24 +103,41 @@ def _activations(n_mat, T, I, dtype, gen, device) -> torch.Tensor:
     return X
 
 
-def _c0(device, seed, scale):
+def _dims(name: str, scale: float):
+    """Shapes of a workload at ``scale``: (matrices E, rows O, columns I,
+    tokens T); c3's per-linear shapes are scaled the same way from
+    C3_LINEARS / C3_SITES."""
+    if name == "c0":
+        return 1, 256, 512, 128
+    if name == "c1":
+        return 1, _scaled(4096, scale, 8), _scaled(4096, scale, 128), _scaled(2048, scale, 8)
+    if name == "c2":
+        return (_scaled(64, scale, 1), _scaled(2048, scale, 8),
+                7168 if scale >= 1 else _scaled(7168, scale, 64, 128), _scaled(512, scale, 8))
+    if name == "c3":
+        return 1, None, None, _scaled(8 * 8192, scale, 8)
+    if name == "c4":
+        return (_scaled(128, scale, 1), _scaled(1856, scale, 8),
+                2688 if scale >= 1 else _scaled(2688, scale, 16, 32), _scaled(512, scale, 8))
+    raise KeyError(name)
+
+
+def _c0(device, seed, scale, max_mats=None):
     g = _gen(device, seed, "c0", "W")
-    O, I = 256, 512
+    _, O, I, T = _dims("c0", scale)
     W = student_t((O, I), 4, g, device) * 0.02
     rows = torch.randperm(O, generator=g, device=device)[:2]
     n_out = max(1, round(0.01 * I))
     for r in rows.tolist():
         cols = torch.randperm(I, generator=g, device=device)[:n_out]
         W[r, cols] *= 25.0
-    X = _activations(1, 128, I, torch.float32, _gen(device, seed, "c0", "X"), device)
+    X = _activations(1, T, I, torch.float32, _gen(device, seed, "c0", "X"), device)
     return Workload("c0", [Unit("w", "int3_g64_sym", W.unsqueeze(0), "x")], {"x": Site("x", X)})
 
 
-def _c1(device, seed, scale):
+def _c1(device, seed, scale, max_mats=None):
     g = _gen(device, seed, "c1", "W")
-    O = _scaled(4096, scale, 8)
-    I = _scaled(4096, scale, 128)
-    T = _scaled(2048, scale, 8)
+    _, O, I, T = _dims("c1", scale)
     W = torch.randn((O, I), generator=g, device=device) * 0.02
     cols = torch.randperm(I, generator=g, device=device)[: max(1, round(0.001 * I))]
     W[:, cols] *= 10.0
@@ -129,11 +146,9 @@ def _c1(device, seed, scale):
                     {"x": Site("x", X)})
 
 
-def _c2(device, seed, scale):
-    E = _scaled(64, scale, 1)
-    O = _scaled(2048, scale, 8)
-    I = 7168 if scale >= 1 else _scaled(7168, scale, 64, 128)
-    T = _scaled(512, scale, 8)
+def _c2(device, seed, scale, max_mats=None):
+    E, O, I, T = _dims("c2", scale)
+    E = E if max_mats is None else min(E, max_mats)
     g = _gen(device, seed, "c2", "W")
     W = torch.empty((E, O, I), dtype=torch.bfloat16, device=device)
     n_rows = max(1, round(0.005 * O))
@@ -163,8 +178,8 @@ C3_LINEARS = [  # name, O, I, input site
 C3_SITES = [("qkv_in", 5120), ("o_in", 5120), ("gateup_in", 5120), ("down_in", 17408)]
 
 
-def _c3(device, seed, scale):
-    T = _scaled(8 * 8192, scale, 8)
+def _c3(device, seed, scale, max_mats=None):
+    T = _dims("c3", scale)[3]
     units = []
     for name, O, I, site in C3_LINEARS:
         g = _gen(device, seed, "c3", "W", name)
@@ -181,11 +196,9 @@ def _c3(device, seed, scale):
     return Workload("c3", units, sites)
 
 
-def _c4(device, seed, scale):
-    E = _scaled(128, scale, 1)
-    O = _scaled(1856, scale, 8)
-    I = 2688 if scale >= 1 else _scaled(2688, scale, 16, 32)
-    T = _scaled(512, scale, 8)
+def _c4(device, seed, scale, max_mats=None):
+    E, O, I, T = _dims("c4", scale)
+    E = E if max_mats is None else min(E, max_mats)
     g = _gen(device, seed, "c4", "W")
     W = torch.empty((E, O, I), dtype=torch.bfloat16, device=device)
     for e in range(E):
@@ -205,9 +218,32 @@ DESCRIPTIONS = {
 }
 
 
-def make(name: str, device="cpu", seed: int = 0, scale: float = 1.0) -> Workload:
-    """Build workload ``name`` on ``device``; ``scale`` < 1 shrinks it for tests."""
-    return WORKLOADS[name](device, seed, scale)
+def make(name: str, device="cpu", seed: int = 0, scale: float = 1.0, max_mats=None) -> Workload:
+    """Build workload ``name`` on ``device``; ``scale`` < 1 shrinks it for
+    tests; ``max_mats`` draws only the first experts of a MoE workload (the
+    same values as the first experts of the whole draw on that device)."""
+    return WORKLOADS[name](device, seed, scale, max_mats)
+
+
+def layout(name: str, scale: float = 1.0):
+    """The workload's shapes without drawing anything: ``units`` as
+    (name, fmt, (E, O, I), site, timed) and ``sites`` as name -> (E, T, I, dtype)."""
+    E, O, I, T = _dims(name, scale)
+    if name == "c0":
+        return {"units": [("w", "int3_g64_sym", (1, O, I), "x", True)], "sites": {"x": (1, T, I, "f32")}}
+    if name == "c1":
+        return {"units": [("w", "int4_g128_asym", (1, O, I), "x", True)], "sites": {"x": (1, T, I, "bf16")}}
+    if name == "c2":
+        return {"units": [("experts", "int3_g64_sym", (E, O, I), "x", True),
+                          ("tail", "int3_g64_sym", (1, O, I + 40), "xtail", False)],
+                "sites": {"x": (E, T, I, "bf16"), "xtail": (1, T, I + 40, "bf16")}}
+    if name == "c3":
+        units = [(n, "int4_g128_asym", (1, _scaled(o, scale, 8), _scaled(i, scale, 128)), s, True)
+                 for n, o, i, s in C3_LINEARS]
+        return {"units": units, "sites": {n: (1, T, _scaled(i, scale, 128), "bf16") for n, i in C3_SITES}}
+    if name == "c4":
+        return {"units": [("experts", "nvfp4_g16", (E, O, I), "x", True)], "sites": {"x": (E, T, I, "bf16")}}
+    raise KeyError(name)
 
 
 def random_groups(n_groups: int, group: int, dist: str, seed: int, device="cpu",

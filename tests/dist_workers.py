@@ -110,3 +110,71 @@ def peer_dies(rank, world, port, out_dir):
     with open(os.path.join(out_dir, "status.txt"), "w") as f:
         f.write(status)
     os._exit(0)
+
+
+class _HostStandIn:
+    """A host stand-in for the library's four step calls, used only to check
+    bench.py's sharding and exchanges on CPU: deterministic per-group and
+    per-column arithmetic in torch (not the method), so that a sharded run
+    can be compared with a one-process run of the same inputs."""
+    FORMATS = {"int3_g64_sym": 5, "int4_g128_asym": 4, "nvfp4_g16": 16}
+    GROUP = {5: 64, 4: 128, 16: 16}
+
+    class Result:
+        def __init__(self, scales):
+            self.scales, self.zeros, self.global_scale, self.packed = scales, None, None, scales
+            self.cand_idx = self.loss = None
+
+    def imatrix_workspace_bytes(self, X):
+        return 16
+
+    def proxy_workspace_bytes(self, W, fmt):
+        return 16
+
+    def tq_imatrix(self, X, m, alpha, workspace=None):
+        m.copy_((X.double().square().sum(dim=1) * alpha).float())
+        return m
+
+    def tq_search_groups(self, W, m, fmt, want_idx=True, want_loss=True, out=None):
+        E, O, I = W.shape
+        g = self.GROUP[fmt]
+        G = -(-I // g)
+        pad = torch.nn.functional.pad(W.float().abs(), (0, G * g - I))
+        s = pad.reshape(E, O, G, g).amax(dim=3)
+        if out is None:
+            return self.Result(s)
+        out.scales.copy_(s)
+        return out
+
+    def tq_dequant(self, packed, fmt, scales, zeros, gs, E, O, I, out):
+        g = self.GROUP[fmt]
+        out.copy_(scales.repeat_interleave(g, dim=2)[:, :, :I].to(out.dtype))
+        return out
+
+    def tq_proxy_error(self, W, packed, fmt, scales, zeros, gs, m, out, workspace=None):
+        mm = m if m.dim() == 2 else m.unsqueeze(0)
+        w = W.double()
+        out[0].copy_((w.square() * mm.double().unsqueeze(1)).sum(dim=(1, 2)))
+        out[1].copy_((w.abs() * mm.double().unsqueeze(1)).sum(dim=(1, 2)))
+        return out
+
+
+def bench_sharded_step(rank, world, port, root, out_dir, config):
+    """bench.py's strong-scaling split of `config` (scale 0.05) over gloo ranks:
+    this rank's part, one step with the host stand-in, results saved for the
+    parent to compare with a one-process run."""
+    sys.path.insert(0, root)
+    import bench
+    import synth
+    _init(rank, world, port)
+    wl = synth.make(config, "cpu", seed=0, scale=0.05)
+    part, shard = bench.shard_workload(wl, world, rank)
+    step = bench.Step(_HostStandIn(), part, bench.make_sets(part, 1), shard)
+    step(0)
+    out = {"m": {k: v.numpy() for k, v in step.m.items()},
+           "scales": [r.scales.numpy() for r in step.res],
+           "px": [np.stack([a.numpy(), b.numpy()]) for a, b in step.px],
+           "pieces": shard.pieces}
+    np.save(os.path.join(out_dir, f"s{rank}.npy"), np.array([out], dtype=object), allow_pickle=True)
+    dist.barrier()
+    dist.destroy_process_group()

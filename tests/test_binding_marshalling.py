@@ -135,3 +135,48 @@ def test_gemv_marshalling(fake):
         tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.zeros(4), None, None, 2, 10, 255, x)
     with pytest.raises(ValueError):
         tq.tq_dequant_gemv(packed, tq.INT3_G64_SYM, torch.zeros(4), None, None, 3, 10, 256, x3)
+
+
+@pytest.mark.parametrize("bad", [
+    torch.zeros((2, 64), dtype=torch.float64),               # not fp32
+    torch.zeros((2, 63)),                                    # too few columns
+    torch.zeros((3, 64)),                                    # wrong matrix count
+    torch.zeros(10),                                         # a short vector
+    torch.zeros((64, 2)).t(),                                # non-unit column stride
+    torch.zeros((2, 64, 1)),                                 # wrong rank
+])
+def test_imatrix_outputs_refused_before_any_call(fake, bad):
+    """tq_imatrix / tq_imatrix_static write m in place: a tensor of the wrong
+    dtype, shape or strides is refused on the host, and nothing is called."""
+    X = torch.zeros((2, 16, 64), dtype=torch.bfloat16)
+    for fn in (tq.tq_imatrix, tq.tq_imatrix_static):
+        with pytest.raises(tq.TQError):
+            fn(X, m=bad)
+    assert not [n for n, _ in fake.calls if n in ("tq_imatrix", "tq_imatrix_static")]
+
+
+def test_imatrix_output_rows_must_not_overlap(fake):
+    X = torch.zeros((2, 16, 64), dtype=torch.bfloat16)
+    m = torch.zeros(128).as_strided((2, 64), (32, 1))        # rows 32 floats apart: overlapping
+    with pytest.raises(tq.TQError):
+        tq.tq_imatrix(X, m=m)
+    m_ok = torch.zeros((2, 80))[:, :64]                      # padded rows are fine
+    tq.tq_imatrix(X, m=m_ok)
+    assert _last(fake, "tq_imatrix")[2] == 80
+
+
+@pytest.mark.parametrize("bad", [torch.zeros(63), torch.zeros((3, 64)), torch.zeros(64, dtype=torch.bfloat16)])
+def test_imatrix_inputs_refused(fake, bad):
+    """The search, proxy error, FP8 search and Lloyd-Max read m: the same
+    checks, with one shared [I] vector (or [1, I]) also allowed."""
+    W = torch.zeros((2, 8, 64), dtype=torch.bfloat16)
+    with pytest.raises(tq.TQError):
+        tq.tq_search_groups(W, bad, tq.INT3_G64_SYM)
+    with pytest.raises(tq.TQError):
+        tq.tq_proxy_error(W, torch.zeros(16, dtype=torch.uint8), tq.INT3_G64_SYM, torch.zeros(16), None, None, bad)
+    with pytest.raises(tq.TQError):
+        tq.tq_search_fp8(W, bad)
+    with pytest.raises(tq.TQError):
+        tq.tq_lloyd_max_g32(W, bad)
+    for ok in (torch.zeros(64), torch.zeros((1, 64)), torch.zeros((2, 64))):
+        tq.tq_search_groups(W, ok, tq.INT3_G64_SYM)

@@ -57,3 +57,19 @@ def test_seeded_and_deterministic():
     assert torch.equal(a.units[0].W, b.units[0].W) and torch.equal(a.sites["x"].X, b.sites["x"].X)
     assert not torch.equal(a.units[0].W, c.units[0].W)
     assert np.isfinite(a.units[0].W.float().numpy()).all()
+
+
+def test_layout_matches_the_drawn_shapes():
+    """synth.layout (shapes only, used for the bench's configuration and the
+    ranks' split) agrees with what synth.make draws, and max_mats draws the
+    first experts of the whole stack."""
+    for name in ("c0", "c1", "c2", "c3", "c4"):
+        lay = synth.layout(name, 0.05)
+        wl = synth.make(name, "cpu", scale=0.05)
+        assert [(u.name, u.fmt, tuple(u.W.shape), u.site, u.timed) for u in wl.units] == lay["units"]
+        assert {k: tuple(s.X.shape) for k, s in wl.sites.items()} == {k: v[:3] for k, v in lay["sites"].items()}
+    full = synth.make("c4", "cpu", scale=0.05)
+    first = synth.make("c4", "cpu", scale=0.05, max_mats=1)
+    assert torch.equal(first.units[0].W[0], full.units[0].W[0]) and first.units[0].W.shape[0] == 1
+    assert torch.equal(first.sites["x"].X[0], full.sites["x"].X[0])
+    assert synth.layout("c2")["units"][0][2] == (64, 2048, 7168)
