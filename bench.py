@@ -774,7 +774,8 @@ def next_rows(tq, step, pk, peak_tinst):
     out = {"dequant_gemv": {f"B={B}": time_gemv(tq, step, pk, B) for B in (1, 8)}}
     if step.units[0].fmt == "int4_g128_asym":
         out["asym_ladder_256_64"] = time_ladder(tq, step, peak_tinst)
-        out["int4_g64"] = time_int4_g64(tq, step, pk, peak_tinst)
+        out["int4_g64"] = time_int4_group(tq, step, pk, peak_tinst, tq.INT4_G64_ASYM)
+        out["int4_g32"] = time_int4_group(tq, step, pk, peak_tinst, tq.INT4_G32_ASYM)
     out["hessian"] = time_hessian(tq, step, pk)
     out["proxy_full_hessian"] = time_proxy_full(tq, step, pk)
     out["gptq_sweep"] = time_gptq(tq, step, peak_tinst)
@@ -833,17 +834,17 @@ def time_ladder(tq, step, peak_tinst, reps=3):
             "note": f"first unit, {reps} launches, 4096 candidate-element evaluations x 5 instr per weight"}
 
 
-def time_int4_g64(tq, step, pk, peak_tinst, reps=5):
-    """The int4-g64 format on the first unit: the joint search with fused RTN
-    and pack (1024 candidate-element evaluations per weight, as for g128)
-    against the FP32 issue roofline, and the bf16 dequantization against HBM
-    (records 0.5 B + scale and zero 5/64 B read, 2 B written per weight)."""
+def time_int4_group(tq, step, pk, peak_tinst, fmt, reps=5):
+    """An int4 format with smaller groups (int4-g64, int4-g32) on the first
+    unit: the joint search with fused RTN and pack (1024 candidate-element
+    evaluations per weight, as for g128) against the FP32 issue roofline, and
+    the bf16 dequantization against HBM (records 0.5 B + scale and zero 5/g B
+    read, 2 B written per weight)."""
     u = step.units[0]
     m = step._m_for(u)
-    fmt = tq.INT4_G64_ASYM
     Ws = [s[1][0] for s in step.sets]
     E, O, I = u.W.shape
-    res = tq.tq_search_groups(Ws[0], m, fmt)
+    res = tq.tq_search_groups(Ws[0], m, fmt, want_idx=False, want_loss=False)
     dq = torch.empty((E, O, I), dtype=torch.bfloat16, device=u.W.device)
     torch.cuda.synchronize()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]

@@ -29,20 +29,22 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = [
-    "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
+    "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "INT4_G32_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
-    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_debug_set_wait_limit", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
 INT4_G64_ASYM = 6
+INT4_G32_ASYM = 7
 INT3_G64_SYM = 5
 NVFP4_G16 = 16
 FORMATS = {"int3_g64_sym": INT3_G64_SYM, "int4_g128_asym": INT4_G128_ASYM, "int4_g64_asym": INT4_G64_ASYM,
-           "nvfp4_g16": NVFP4_G16}
-_GROUP = {INT3_G64_SYM: 64, INT4_G128_ASYM: 128, INT4_G64_ASYM: 64, NVFP4_G16: 16}
+           "int4_g32_asym": INT4_G32_ASYM, "nvfp4_g16": NVFP4_G16}
+_GROUP = {INT3_G64_SYM: 64, INT4_G128_ASYM: 128, INT4_G64_ASYM: 64, INT4_G32_ASYM: 32, NVFP4_G16: 16}
+_INT4 = (INT4_G128_ASYM, INT4_G64_ASYM, INT4_G32_ASYM)
 _F32, _BF16 = 0, 1
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -57,7 +59,7 @@ EXPORTS = [
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
     "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2", "tq_proxy_full_workspace_bytes",
-    "tq_proxy_error_full", "tq_gptq_workspace_bytes", "tq_gptq_sweep",
+    "tq_proxy_error_full", "tq_gptq_workspace_bytes", "tq_gptq_sweep", "tq_debug_set_wait_limit",
 ]
 
 
@@ -153,6 +155,7 @@ def lib():
             "tq_gptq_sweep": (i32, [Mp, i32, P, P, P, i64, i64, P, P, P, sz, P]),
             "tq_proxy_error_full": (i32, [Mp, Mp, P, i32, P, P, P, P, P, P, sz, P]),
             "tq_sync": (i32, [P]),
+            "tq_debug_set_wait_limit": (i32, [i64]),
             "tq_imatrix_static_capacity": (sz, []),
             "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
             "tq_selftest_e2m1": (i32, [P, P, P]),
@@ -265,6 +268,12 @@ def tq_packed_bytes(fmt: int, rows: int, cols: int) -> int:
 
 def tq_sync(stream=None) -> None:
     _check(lib().tq_sync(_stream(stream)), "tq_sync")
+
+
+def tq_debug_set_wait_limit(rounds: int) -> None:
+    """Testing aid: try-wait rounds after which the copy/MMA ring waits of
+    later tq_hessian / tq_proxy_error_full launches give up (< 0: default)."""
+    _check(lib().tq_debug_set_wait_limit(int(rounds)), "tq_debug_set_wait_limit")
 
 
 def tq_selftest_e2m1(stream=None) -> Tuple[int, int]:
@@ -456,8 +465,7 @@ def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optiona
         out = SearchResult(
             fmt=fmt,
             scales=torch.empty((E, O, G), dtype=sdt, device=dev),
-            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt in (INT4_G128_ASYM, INT4_G64_ASYM)
-            else None,
+            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt in _INT4 else None,
             global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
             cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
             loss=torch.empty((E, O, G), dtype=torch.float64, device=dev) if want_loss else None,

@@ -515,6 +515,8 @@ TQ_API tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void*
         launch_gemv_b<TQ_INT4_G128_ASYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else if (fmt == TQ_INT4_G64_ASYM) {
         launch_gemv_b<TQ_INT4_G64_ASYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
+    } else if (fmt == TQ_INT4_G32_ASYM) {
+        launch_gemv_b<TQ_INT4_G32_ASYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else if (((I + 15) / 16) % 2 == 0 && (reinterpret_cast<uintptr_t>(scales) & 1u) == 0) {
         launch_gemv_b<TQ_NVFP4_G16, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else {

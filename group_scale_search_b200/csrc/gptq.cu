@@ -263,7 +263,9 @@ TQ_API tq_status tq_gptq_sweep(const tq_mat* W, int32_t fmt, const void* scales,
         bf ? launch_gptq<TQ_INT3_G64_SYM, uint16_t>(a, W->n_mat, st) : launch_gptq<TQ_INT3_G64_SYM, float>(a, W->n_mat, st);
     else if (fmt == TQ_INT4_G128_ASYM)
         bf ? launch_gptq<TQ_INT4_G128_ASYM, uint16_t>(a, W->n_mat, st) : launch_gptq<TQ_INT4_G128_ASYM, float>(a, W->n_mat, st);
-    else
+    else if (fmt == TQ_INT4_G64_ASYM)
         bf ? launch_gptq<TQ_INT4_G64_ASYM, uint16_t>(a, W->n_mat, st) : launch_gptq<TQ_INT4_G64_ASYM, float>(a, W->n_mat, st);
+    else
+        bf ? launch_gptq<TQ_INT4_G32_ASYM, uint16_t>(a, W->n_mat, st) : launch_gptq<TQ_INT4_G32_ASYM, float>(a, W->n_mat, st);
     return check_launch("tq_gptq_sweep");
 }

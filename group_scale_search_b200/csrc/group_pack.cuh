@@ -29,15 +29,21 @@ __device__ __forceinline__ void pack_int3_record(unsigned u0, unsigned u1, int l
     }
 }
 
-// int4-g128 record: 64 bytes, element 2k in the low nibble of byte k.  Lane l
-// holds elements 4l..4l+3 and stores bytes 2l, 2l+1.
+// int4 records: g/2 bytes, element 2k in the low nibble of byte k.  Lane l
+// holds elements EPL l .. EPL l + EPL - 1: with 4 (g128) it stores bytes 2l,
+// 2l+1, with 2 (g64) byte l; with 1 (g32) the even lane stores byte l/2 with
+// its odd neighbour's code (from a shuffle) in the high nibble.  Every lane
+// of the warp must call it.
 template <int EPL>
 __device__ __forceinline__ void pack_int4_lane(const unsigned q[EPL], int lane, uint8_t* rec) {
     if constexpr (EPL == 4) {
         const unsigned v = (q[0] & 15u) | ((q[1] & 15u) << 4) | ((q[2] & 15u) << 8) | ((q[3] & 15u) << 12);
         reinterpret_cast<uint16_t*>(rec)[lane] = static_cast<uint16_t>(v);
-    } else {
+    } else if constexpr (EPL == 2) {
         rec[lane] = static_cast<uint8_t>((q[0] & 15u) | ((q[1] & 15u) << 4));
+    } else {
+        const unsigned hi = __shfl_down_sync(FULL, q[0] & 15u, 1);
+        if ((lane & 1) == 0) rec[lane >> 1] = static_cast<uint8_t>((q[0] & 15u) | (hi << 4));
     }
 }
 

@@ -33,9 +33,10 @@
 //    mirror images with coalesced rows.
 //  * Tiles are grouped in 1024 x 1024 super-blocks so that the CTAs in flight
 //    share their panels in L2.
-// Every wait on an mbarrier has an iteration limit; on timeout the kernel
-// records it (tq_sync reports it), drains its in-flight copies, frees TMEM and
-// returns.
+// Every wait on an mbarrier has an iteration limit; when a wait of the
+// copy/MMA ring runs out the kernel records it (tq_sync reports it), skips
+// the stores, waits (with the default limit) for the MMAs it committed and
+// the copies it issued, frees TMEM and returns.
 #include <cuda.h>
 
 #include <atomic>
@@ -56,7 +57,7 @@ constexpr int HS_A_BYTES = (HS_M / 64) * HS_BOX_BYTES;
 constexpr int HS_B_BYTES = (HS_N / 64) * HS_BOX_BYTES;
 constexpr int HS_STAGE_BYTES = HS_A_BYTES + HS_B_BYTES;
 constexpr int HS_SMEM_BYTES = HS_STAGES * HS_STAGE_BYTES + 1024 /* alignment */ + 256 /* barriers */;
-constexpr unsigned HS_WAIT_LIMIT = 1u << 22;            // try_wait rounds before a wait is declared hung
+constexpr unsigned HS_WAIT_LIMIT = DEFAULT_WAIT_LIMIT;  // try_wait rounds before a wait is declared hung
 
 __device__ unsigned g_hs_timeouts = 0;
 
@@ -74,9 +75,9 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, unsigned bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
 }
 
-// Waits for the phase of parity `parity` to complete; false after the limit.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity) {
-    for (unsigned it = 0; it < HS_WAIT_LIMIT; ++it) {
+// Waits for the phase of parity `parity` to complete; false after `limit` rounds.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, unsigned parity, unsigned limit = HS_WAIT_LIMIT) {
+    for (unsigned it = 0; it < limit; ++it) {
         unsigned ok;
         asm volatile(
             "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
@@ -149,6 +150,7 @@ struct HsArgs {
     int accumulate;
     int nbm, nbn;             // 128-row and 256-column blocks
     int nsb;                  // super-blocks per side
+    unsigned wait_limit;      // try_wait rounds of the ring waits
 };
 
 __global__ void __launch_bounds__(HS_THREADS, 1)
@@ -201,7 +203,7 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
         int k = 0;
         for (; k < nk; ++k) {
             const int s = k % HS_STAGES;
-            if (!mbar_wait(empty0 + 8 * s, ((k / HS_STAGES) & 1) ^ 1)) break;
+            if (!mbar_wait(empty0 + 8 * s, ((k / HS_STAGES) & 1) ^ 1, a.wait_limit)) break;
             const uint32_t st = s_base + s * HS_STAGE_BYTES, bar = full0 + 8 * s;
             mbar_expect_tx(bar, bytes);
             const int t0 = k * HS_BK;
@@ -220,7 +222,7 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
         int k = 0;
         for (; k < nk; ++k) {
             const int s = k % HS_STAGES;
-            if (!mbar_wait(full0 + 8 * s, (k / HS_STAGES) & 1)) break;
+            if (!mbar_wait(full0 + 8 * s, (k / HS_STAGES) & 1, a.wait_limit)) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sb = s_base + s * HS_STAGE_BYTES + HS_A_BYTES;
             const uint32_t sa = a_in_b ? sb + (bi & 1) * (HS_M / 64) * HS_BOX_BYTES : s_base + s * HS_STAGE_BYTES;
@@ -284,13 +286,16 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
         __syncthreads();
     }
 
-    // teardown: drain copies armed but not consumed, then free TMEM
+    // teardown: drain copies armed but not consumed and (if the epilogue's
+    // wait gave up) the committed MMAs, then free TMEM
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if (threadIdx.x == 0) {
         for (int k = progress[1]; k < progress[0]; ++k)
             if (!mbar_wait(full0 + 8 * (k % HS_STAGES), (k / HS_STAGES) & 1)) break;
+        if (progress[3] == 0) mbar_wait(done, 0);
     }
+    __syncthreads();
     if (warp == 0) {
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(HS_N));
     }
@@ -361,6 +366,7 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
     a.nbm = static_cast<int>((X->cols + HS_M - 1) / HS_M);
     a.nbn = static_cast<int>((X->cols + HS_N - 1) / HS_N);
     a.nsb = static_cast<int>((X->cols + 1023) / 1024);
+    a.wait_limit = pipeline_wait_limit();
     static std::once_flag attr;
     std::call_once(attr, [] { cudaFuncSetAttribute(k_hessian, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM_BYTES); });
     const int64_t pairs = static_cast<int64_t>(a.nsb) * (a.nsb + 1) / 2;

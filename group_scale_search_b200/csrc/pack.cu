@@ -128,7 +128,7 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
 // One thread per group record; codes are dense [rows][cols] bytes.
 __global__ void k_pack_codes(const uint8_t* __restrict__ codes, int fmt, int64_t rows, int64_t cols,
                              const uint8_t* __restrict__ zeros, uint8_t* __restrict__ packed) {
-    const int g = fmt == TQ_INT3_G64_SYM ? 64 : (fmt == TQ_INT4_G128_ASYM ? 128 : (fmt == TQ_INT4_G64_ASYM ? 64 : 16));
+    const int g = static_cast<int>(group_of(fmt));
     const int64_t G = (cols + g - 1) / g;
     const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (gid >= rows * G) return;
@@ -172,7 +172,7 @@ __global__ void k_unpack_codes(const uint8_t* __restrict__ packed, int fmt, int6
         const unsigned u = ((rec[i >> 2] >> (2 * (i & 3))) & 3u) | (((rec[16 + (i >> 3)] >> (i & 7)) & 1u) << 2);
         codes[idx] = static_cast<uint8_t>(static_cast<int8_t>(static_cast<int>(u) - 4));
     } else {
-        const int g = fmt == TQ_INT4_G128_ASYM ? 128 : (fmt == TQ_INT4_G64_ASYM ? 64 : 16);
+        const int g = static_cast<int>(group_of(fmt));
         const int64_t G = (cols + g - 1) / g;
         const uint8_t b = packed[(r * G + j / g) * (g / 2) + (j % g) / 2];
         codes[idx] = (j & 1) ? static_cast<uint8_t>(b >> 4) : static_cast<uint8_t>(b & 15u);
@@ -328,6 +328,8 @@ TQ_API tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const
                                           : launch_pack<TQ_INT4_G128_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
     else if (fmt == TQ_INT4_G64_ASYM) bf ? launch_pack<TQ_INT4_G64_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
                                          : launch_pack<TQ_INT4_G64_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
+    else if (fmt == TQ_INT4_G32_ASYM) bf ? launch_pack<TQ_INT4_G32_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
+                                         : launch_pack<TQ_INT4_G32_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
     else bf ? launch_pack<TQ_NVFP4_G16, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
             : launch_pack<TQ_NVFP4_G16, float>(W, ms, scales, zeros, global_scale, packed, st);
     return check_launch("tq_pack");
@@ -384,6 +386,9 @@ TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scal
     else if (fmt == TQ_INT4_G64_ASYM)
         bf ? launch_dequant<TQ_INT4_G64_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
            : launch_dequant<TQ_INT4_G64_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G32_ASYM)
+        bf ? launch_dequant<TQ_INT4_G32_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G32_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
     else
         bf ? launch_dequant<TQ_NVFP4_G16, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
            : launch_dequant<TQ_NVFP4_G16, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);

@@ -241,6 +241,9 @@ TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t 
     else if (fmt == TQ_INT4_G64_ASYM)
         bf ? launch_proxy<TQ_INT4_G64_ASYM, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
            : launch_proxy<TQ_INT4_G64_ASYM, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);
+    else if (fmt == TQ_INT4_G32_ASYM)
+        bf ? launch_proxy<TQ_INT4_G32_ASYM, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
+           : launch_proxy<TQ_INT4_G32_ASYM, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);
     else
         bf ? launch_proxy<TQ_NVFP4_G16, uint16_t>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st)
            : launch_proxy<TQ_NVFP4_G16, float>(W, ms, packed, scales, zeros, global_scale, m, mst, parts, tickets, num, den, st);

@@ -42,7 +42,7 @@ constexpr int PF_B_BYTES = PF_N * PF_BK * 2;               // 32 KB
 constexpr int PF_RING_BYTES = PF_XS * PF_X_BYTES + PF_BS * PF_B_BYTES;
 constexpr int PF_NBAR = 2 * PF_XS + 2 * PF_BS + 1;
 constexpr int PF_SMEM_BYTES = PF_RING_BYTES + 1024 + 256;
-constexpr unsigned PF_WAIT_LIMIT = 1u << 22;
+constexpr unsigned PF_WAIT_LIMIT = DEFAULT_WAIT_LIMIT;
 static_assert(PF_NBAR * 8 + 4 + 6 * 4 <= 192 && PF_RING_BYTES + 1023 + 256 <= PF_SMEM_BYTES, "shared layout");
 
 __device__ unsigned g_pf_timeouts = 0;
@@ -51,8 +51,8 @@ __device__ __forceinline__ uint32_t pf_smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ bool pf_wait(uint32_t bar, unsigned parity) {
-    for (unsigned it = 0; it < PF_WAIT_LIMIT; ++it) {
+__device__ __forceinline__ bool pf_wait(uint32_t bar, unsigned parity, unsigned limit = PF_WAIT_LIMIT) {
+    for (unsigned it = 0; it < limit; ++it) {
         unsigned ok;
         asm volatile(
             "{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
@@ -96,6 +96,7 @@ struct PfArgs {
     int tiles_m, tiles_n;
     double* pn;          // [n_mat][tiles_m * tiles_n] partials of ||X E^T||^2
     double* pd;          // the same for ||X W^T||^2
+    unsigned wait_limit; // try_wait rounds of the ring waits
 };
 
 __device__ __forceinline__ double pf_tile_sq(uint32_t taddr) {
@@ -163,13 +164,13 @@ k_pf_gemm(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
             const int c = j / PF_OPS, p = j - c * PF_OPS;
             if (p == 0) {
                 const int xs = c % PF_XS;
-                if (!(ok = pf_wait(xempty + 8 * xs, ((c / PF_XS) & 1) ^ 1))) break;
+                if (!(ok = pf_wait(xempty + 8 * xs, ((c / PF_XS) & 1) ^ 1, a.wait_limit))) break;
                 pf_arm(xfull + 8 * xs, PF_X_BYTES);
                 pf_tma_3d(xs0 + xs * PF_X_BYTES, &xmap, xfull + 8 * xs, c * PF_BK, tm * PF_M, e);
                 progress[0] = c + 1;
             }
             const int bs = j % PF_BS;
-            if (!(ok = pf_wait(bempty + 8 * bs, ((j / PF_BS) & 1) ^ 1))) break;
+            if (!(ok = pf_wait(bempty + 8 * bs, ((j / PF_BS) & 1) ^ 1, a.wait_limit))) break;
             pf_arm(bfull + 8 * bs, PF_B_BYTES);
             if (p < PF_PIECES)
                 pf_tma_3d(bs0 + bs * PF_B_BYTES, &emap, bfull + 8 * bs, (p * nc + c) * PF_BK, tn * PF_N, e);
@@ -182,8 +183,8 @@ k_pf_gemm(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
         bool ok = true;
         for (int j = 0; j < nb && ok; ++j) {
             const int c = j / PF_OPS, p = j - c * PF_OPS, xs = c % PF_XS, bs = j % PF_BS;
-            if (p == 0 && !(ok = pf_wait(xfull + 8 * xs, (c / PF_XS) & 1))) break;
-            if (!(ok = pf_wait(bfull + 8 * bs, (j / PF_BS) & 1))) break;
+            if (p == 0 && !(ok = pf_wait(xfull + 8 * xs, (c / PF_XS) & 1, a.wait_limit))) break;
+            if (!(ok = pf_wait(bfull + 8 * bs, (j / PF_BS) & 1, a.wait_limit))) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sa = xs0 + xs * PF_X_BYTES, sb = bs0 + bs * PF_B_BYTES;
             const uint32_t d = tmem + (p < PF_PIECES ? 0u : static_cast<uint32_t>(PF_N));
@@ -234,7 +235,9 @@ k_pf_gemm(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
             if (!pf_wait(xfull + 8 * (c % PF_XS), (c / PF_XS) & 1)) break;
         for (int j = progress[3]; j < progress[2]; ++j)
             if (!pf_wait(bfull + 8 * (j % PF_BS), (j / PF_BS) & 1)) break;
+        if (progress[5] == 0) pf_wait(done, 0);   // the committed MMAs, before TMEM is freed
     }
+    __syncthreads();
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(2 * PF_N));
 }
 
@@ -402,6 +405,8 @@ TQ_API tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uin
             k_pf_prep<TQ_INT4_G128_ASYM, uint16_t><<<grid, 256, 0, st>>>(Wp, O, W->cols, W->ld, ms, packed, scales, zeros, global_scale, E, Ip, ep);
         else if (fmt == TQ_INT4_G64_ASYM)
             k_pf_prep<TQ_INT4_G64_ASYM, uint16_t><<<grid, 256, 0, st>>>(Wp, O, W->cols, W->ld, ms, packed, scales, zeros, global_scale, E, Ip, ep);
+        else if (fmt == TQ_INT4_G32_ASYM)
+            k_pf_prep<TQ_INT4_G32_ASYM, uint16_t><<<grid, 256, 0, st>>>(Wp, O, W->cols, W->ld, ms, packed, scales, zeros, global_scale, E, Ip, ep);
         else
             k_pf_prep<TQ_NVFP4_G16, uint16_t><<<grid, 256, 0, st>>>(Wp, O, W->cols, W->ld, ms, packed, scales, zeros, global_scale, E, Ip, ep);
     }
@@ -413,6 +418,7 @@ TQ_API tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uin
     a.kx = static_cast<int>(Ip / 64);
     a.pn = pn;
     a.pd = pd;
+    a.wait_limit = pipeline_wait_limit();
     k_pf_gemm<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(E)), PF_THREADS, PF_SMEM_BYTES, st>>>(xm, em, wm, a);
     k_pf_reduce<<<static_cast<unsigned>(E), 32, 0, st>>>(pn, pd, tiles, num, den);
     return check_launch("tq_proxy_error_full");

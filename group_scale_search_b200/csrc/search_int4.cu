@@ -10,7 +10,9 @@
 //
 // The same search runs on 64-weight groups (int4-g64: the page "int3-g64
 // (fmt=5)"'s per-projection ablation table lists an int4-g64 scheme, and its
-// thread the grouped int4 format fmt=4): lanes then hold 2 weights each.
+// thread the grouped int4 format fmt=4): lanes then hold 2 weights each; and
+// on 32-weight groups ("Phase 2: math-accuracy regression on tq3a-tq2e g32",
+// Summary: group_size=32), one weight per lane.
 //
 // B200 mapping: one warp per 128-weight group; lane l owns scales l and l+32
 // (and 64 p + l, 64 p + 32 + l in pass p of a grid of more than 64 scales:
@@ -91,6 +93,15 @@ template <> struct Load2<float> {
     }
 };
 
+// Lane l holds element l of a 32-weight group.
+template <typename T> struct Load1;
+template <> struct Load1<uint16_t> {
+    static __device__ __forceinline__ void go(const uint16_t* p, float w[1]) { w[0] = bf16_bits_to_f32(__ldg(p)); }
+};
+template <> struct Load1<float> {
+    static __device__ __forceinline__ void go(const float* p, float w[1]) { w[0] = __ldg(p); }
+};
+
 __device__ __forceinline__ unsigned ord_key(float x) {   // order-preserving float -> uint
     const unsigned b = __float_as_uint(x);
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
@@ -140,7 +151,7 @@ __device__ __forceinline__ void acc_scale(float w, float sm, float s, float inv,
 template <typename T, int NP, int GS>
 __global__ void __launch_bounds__(ASYM_WARPS * 32)
 k_search_int4(const __grid_constant__ AsymArgs a) {
-    constexpr int EPL = GS / 32;   // elements per lane: 4 (g128) or 2 (g64)
+    constexpr int EPL = GS / 32;   // elements per lane: 4 (g128), 2 (g64) or 1 (g32)
     __shared__ __align__(16) float2 lists[ASYM_WARPS][GS + 4];   // two sign lists, each padded to even length
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int64_t G = (a.I + GS - 1) / GS;
@@ -166,10 +177,13 @@ k_search_int4(const __grid_constant__ AsymArgs a) {
                 Load4<T>::go(wp + 4 * lane, w);
                 const float4 mm = __ldg(reinterpret_cast<const float4*>(mp + 4 * lane));
                 mv[0] = mm.x; mv[1] = mm.y; mv[2] = mm.z; mv[3] = mm.w;
-            } else {
+            } else if constexpr (EPL == 2) {
                 Load2<T>::go(wp + 2 * lane, w);
                 const float2 mm = __ldg(reinterpret_cast<const float2*>(mp + 2 * lane));
                 mv[0] = mm.x; mv[1] = mm.y;
+            } else {
+                Load1<T>::go(wp + lane, w);
+                mv[0] = __ldg(mp + lane);
             }
 #pragma unroll
             for (int i = 0; i < EPL; ++i) val[i] = true;
@@ -417,9 +431,12 @@ tq_status launch_search_int4(const tq_mat* W, int gsize, const float* m, int64_t
     if (gsize == 128) {
         if (a.ns <= 64) launch_int4<1, 128>(a, bf16, total, st);
         else launch_int4<4, 128>(a, bf16, total, st);
-    } else {
+    } else if (gsize == 64) {
         if (a.ns <= 64) launch_int4<1, 64>(a, bf16, total, st);
         else launch_int4<4, 64>(a, bf16, total, st);
+    } else {
+        if (a.ns <= 64) launch_int4<1, 32>(a, bf16, total, st);
+        else launch_int4<4, 32>(a, bf16, total, st);
     }
     return check_launch("int4 search");
 }

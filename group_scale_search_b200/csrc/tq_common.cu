@@ -3,7 +3,16 @@
 
 #include <string.h>
 
+#include <atomic>
+
 namespace tq {
+
+static std::atomic<int64_t> g_wait_limit{-1};
+
+unsigned pipeline_wait_limit() {
+    const int64_t v = g_wait_limit.load(std::memory_order_relaxed);
+    return v < 0 ? DEFAULT_WAIT_LIMIT : static_cast<unsigned>(v > 0xffffffffll ? 0xffffffffll : v);
+}
 
 static thread_local char g_err[512];
 
@@ -78,6 +87,12 @@ TQ_API int64_t tq_num_groups(int32_t fmt, int64_t rows, int64_t cols) {
 
 TQ_API size_t tq_packed_bytes(int32_t fmt, int64_t rows, int64_t cols) {
     return static_cast<size_t>(tq_num_groups(fmt, rows, cols) * record_bytes(fmt));
+}
+
+TQ_API tq_status tq_debug_set_wait_limit(int64_t rounds) {
+    clear_error();
+    g_wait_limit.store(rounds < 0 ? -1 : rounds, std::memory_order_relaxed);
+    return TQ_OK;
 }
 
 TQ_API tq_status tq_sync(tq_stream_t stream) {

@@ -37,16 +37,23 @@ bool proxy_full_take_timeouts();
 
 inline int elem_bytes(int32_t dt) { return dt == TQ_BF16 ? 2 : (dt == TQ_F32 ? 4 : 0); }
 
-inline int64_t group_of(int32_t fmt) {
+__host__ __device__ inline int64_t group_of(int32_t fmt) {
     return fmt == TQ_INT3_G64_SYM ? 64 : fmt == TQ_INT4_G128_ASYM ? 128 : fmt == TQ_INT4_G64_ASYM ? 64
-         : fmt == TQ_NVFP4_G16 ? 16 : 0;
+         : fmt == TQ_INT4_G32_ASYM ? 32 : fmt == TQ_NVFP4_G16 ? 16 : 0;
 }
-inline int64_t record_bytes(int32_t fmt) {
+__host__ __device__ inline int64_t record_bytes(int32_t fmt) {
     return fmt == TQ_INT3_G64_SYM ? 24 : fmt == TQ_INT4_G128_ASYM ? 64 : fmt == TQ_INT4_G64_ASYM ? 32
-         : fmt == TQ_NVFP4_G16 ? 8 : 0;
+         : fmt == TQ_INT4_G32_ASYM ? 16 : fmt == TQ_NVFP4_G16 ? 8 : 0;
 }
 // The asymmetric int4 formats (nibble codes with a zero-point), any group size.
-__host__ __device__ constexpr bool is_int4(int fmt) { return fmt == TQ_INT4_G128_ASYM || fmt == TQ_INT4_G64_ASYM; }
+__host__ __device__ constexpr bool is_int4(int fmt) {
+    return fmt == TQ_INT4_G128_ASYM || fmt == TQ_INT4_G64_ASYM || fmt == TQ_INT4_G32_ASYM;
+}
+
+// Try-wait rounds of the tensor-core pipelines' ring waits for the next
+// launch (tq_debug_set_wait_limit; default 2^22).
+unsigned pipeline_wait_limit();
+constexpr unsigned DEFAULT_WAIT_LIMIT = 1u << 22;
 
 // Validates a matrix batch descriptor; returns TQ_OK or an error (set).
 tq_status check_mat(const tq_mat* X, const char* name);

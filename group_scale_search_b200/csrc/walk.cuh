@@ -20,6 +20,7 @@ template <int FMT> struct FmtTraits;
 template <> struct FmtTraits<TQ_INT3_G64_SYM> { static constexpr int lg = 3, group = 64, rec = 24; };
 template <> struct FmtTraits<TQ_INT4_G128_ASYM> { static constexpr int lg = 4, group = 128, rec = 64; };
 template <> struct FmtTraits<TQ_INT4_G64_ASYM> { static constexpr int lg = 3, group = 64, rec = 32; };
+template <> struct FmtTraits<TQ_INT4_G32_ASYM> { static constexpr int lg = 2, group = 32, rec = 16; };
 template <> struct FmtTraits<TQ_NVFP4_G16> { static constexpr int lg = 1, group = 16, rec = 8; };
 
 // ------------------------------------------------------------------ host geometry

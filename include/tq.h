@@ -17,6 +17,8 @@
  *  [NVFP4]  "Nemotron-Cascade-2-30B-A3B-NVFP4" model card: Quantization Recipe
  *           table (NVFP4, group size 16, MSE-calibrated static block scales).
  *  [INT3]   "int3-g64 (fmt=5)" (colibri PR #168): Design, Layout bullet.
+ *  [G32]    "Phase 2: math-accuracy regression on tq3a-tq2e g32"
+ *           (turboquant-mlx issue #2): Summary (group_size=32).
  *
  * Conventions shared by every call
  *  - Memory: every tensor pointer is a DEVICE pointer owned by the caller.
@@ -64,6 +66,7 @@ typedef enum {
     TQ_INT4_G128_ASYM = 4,   /* nibble codes q in [0,15], f32 scale, u8 zero per 128 weights */
     TQ_INT3_G64_SYM = 5,     /* two bit-planes, v in [-4,3] as v+4, f32 scale per 64 weights  */
     TQ_INT4_G64_ASYM = 6,    /* as TQ_INT4_G128_ASYM with 64 weights per group (32-byte records) */
+    TQ_INT4_G32_ASYM = 7,    /* as TQ_INT4_G128_ASYM with 32 weights per group (16-byte records) [G32] */
     TQ_NVFP4_G16 = 16        /* E2M1 codes, E4M3 scale byte per 16 weights, f32 global scale   */
 } tq_format;
 
@@ -386,7 +389,7 @@ tq_status tq_proxy_error_full(const tq_mat* X, const tq_mat* W, const uint8_t* p
  *   w_j <- fma(-e_i, U_ij, w_j) for every j > i (fp32, in column order).
  * Deterministic and independent of the tiling: results are bitwise those of
  * the unblocked sweep.  W: bf16 or fp32 tq_mat [n_mat][O][I]; fmt:
- * TQ_INT3_G64_SYM, TQ_INT4_G128_ASYM or TQ_INT4_G64_ASYM; scales f32 and
+ * TQ_INT3_G64_SYM or an int4 format (g128, g64, g32); scales f32 and
  * zeros u8 [n_mat][O][ceil(I/g)] as tq_search_groups writes them.  codes:
  * int8 [n_mat][O][I] (int3: v; int4: q), the input of tq_pack_codes.  loss:
  * optional fp64 [n_mat][O], sum_i e_i^2 per row in column order (equal to
@@ -404,6 +407,17 @@ tq_status tq_gptq_sweep(const tq_mat* W, int32_t fmt, const void* scales, const 
  * failed (including a tq_hessian or tq_proxy_error_full launch that gave up
  * on a pipeline wait). */
 tq_status tq_sync(tq_stream_t stream);
+
+/* Testing aid for the give-up path of the tensor-core pipelines: the number
+ * of try-wait rounds after which a pipeline wait of a later tq_hessian or
+ * tq_proxy_error_full launch (in this process) gives up; rounds < 0 restores
+ * the default (2^22 rounds, seconds of waiting).  Only the waits of the
+ * copy/MMA ring use it: a launch that gives up still waits, with the default
+ * limit, for every copy it issued and every MMA it committed before it frees
+ * its shared memory and tensor memory, so a small limit (0 gives up at the
+ * first wait, before any copy is issued) leaves nothing in flight.  Not for
+ * production use; returns TQ_OK. */
+tq_status tq_debug_set_wait_limit(int64_t rounds);
 
 /* Self-test of the GPU's E2M1 conversion instructions, on which the NVFP4
  * round-to-nearest (search, tq_pack) and decoding (tq_dequant,

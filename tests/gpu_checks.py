@@ -17,8 +17,9 @@ MATCH_MIN = 0.999
 LOSS_RTOL = 1e-5
 SUM_RTOL = 1e-5
 
-ORC_FMT = {tq.INT3_G64_SYM: "int3", tq.INT4_G128_ASYM: "int4", tq.INT4_G64_ASYM: "int4", tq.NVFP4_G16: "nvfp4"}
-INT4 = {tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64}   # int4 formats -> group size
+ORC_FMT = {tq.INT3_G64_SYM: "int3", tq.INT4_G128_ASYM: "int4", tq.INT4_G64_ASYM: "int4", tq.INT4_G32_ASYM: "int4",
+           tq.NVFP4_G16: "nvfp4"}
+INT4 = {tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.INT4_G32_ASYM: 32}   # int4 formats -> group size
 
 
 def host32(t: torch.Tensor) -> np.ndarray:

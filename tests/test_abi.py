@@ -43,6 +43,9 @@ def test_sizes(tq):
     assert tq.tq_group_size(tq.NVFP4_G16) == 16
     assert tq.tq_group_size(tq.INT4_G64_ASYM) == 64
     assert tq.tq_packed_bytes(tq.INT4_G64_ASYM, 5, 200) == 5 * 4 * 32   # 32-byte records, ragged last group
+    assert tq.tq_group_size(tq.INT4_G32_ASYM) == 32
+    assert tq.tq_packed_bytes(tq.INT4_G32_ASYM, 5, 200) == 5 * 7 * 16   # 16-byte records, ragged last group
+    assert tq.tq_num_groups(tq.INT4_G32_ASYM, 5, 200) == 35
     assert tq.tq_group_size(99) == 0
     # int3-g64: 24 bytes per 64 weights + f32 scale = 3.5 bits/weight
     assert tq.tq_packed_bytes(tq.INT3_G64_SYM, 2048, 7168) == 2048 * 112 * 24

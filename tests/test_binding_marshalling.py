@@ -100,13 +100,14 @@ def test_search_marshalling(fake):
     shared) and the grid parameters."""
     W = torch.zeros((2, 8, 300), dtype=torch.bfloat16)
     m2 = torch.zeros((2, 304))[:, :300]
-    for fmt, g in [(tq.INT3_G64_SYM, 64), (tq.INT4_G128_ASYM, 128), (tq.INT4_G64_ASYM, 64), (tq.NVFP4_G16, 16)]:
+    for fmt, g in [(tq.INT3_G64_SYM, 64), (tq.INT4_G128_ASYM, 128), (tq.INT4_G64_ASYM, 64), (tq.INT4_G32_ASYM, 32),
+                   (tq.NVFP4_G16, 16)]:
         r = tq.tq_search_groups(W, m2, fmt)
         args = _last(fake, "tq_search_groups")
         G = -(-300 // g)
         assert r.scales.shape == (2, 8, G)
         assert r.scales.dtype == (torch.uint8 if fmt == tq.NVFP4_G16 else torch.float32)
-        assert (r.zeros is not None) == (fmt in (tq.INT4_G128_ASYM, tq.INT4_G64_ASYM))
+        assert (r.zeros is not None) == (fmt in (tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM))
         assert (r.global_scale is not None) == (fmt == tq.NVFP4_G16)
         assert r.cand_idx.shape == (2, 8, G) and r.loss.dtype == torch.float64
         assert r.packed.numel() == 1234

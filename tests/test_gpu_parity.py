@@ -119,7 +119,7 @@ def test_search_pack_dequant_proxy(name, scale):
         _search_and_check(fmt, u.W, m, f"{name}/{u.name}")
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("I", [100, 200, 1802, 48, 7])
 def test_ragged_tails_and_dtypes(fmt, dtype, I):
@@ -131,7 +131,7 @@ def test_ragged_tails_and_dtypes(fmt, dtype, I):
     _search_and_check(fmt, W, m, f"tail I={I} {dtype}")
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 def test_degenerate_groups(fmt):
     g = torch.Generator(device=DEV).manual_seed(11)
     W = (torch.randn((2, 16, 256), generator=g, device=DEV) * 0.02)
@@ -146,7 +146,7 @@ def test_degenerate_groups(fmt):
         _search_and_check(fmt, W.to(dt), m, f"degenerate {dt}")
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 def test_strided_weights_and_per_matrix_imatrix(fmt):
     g = torch.Generator(device=DEV).manual_seed(12)
     big = (synth.student_t((4, 40, 512), 4, g, DEV) * 0.02).to(torch.bfloat16)
@@ -207,13 +207,13 @@ def test_asym_ladder_256_64():
 # ------------------------------------------------------------------ code packing
 
 @pytest.mark.parametrize("fmt,lo,hi", [(tq.INT3_G64_SYM, -4, 4), (tq.INT4_G128_ASYM, 0, 16), (tq.INT4_G64_ASYM, 0, 16),
-                                       (tq.NVFP4_G16, 0, 16)])
+                                       (tq.INT4_G32_ASYM, 0, 16), (tq.NVFP4_G16, 0, 16)])
 @pytest.mark.parametrize("cols", [64, 7208, 300, 2688])
 def test_pack_codes_bit_exact_and_roundtrip(fmt, lo, hi, cols):
     rng = np.random.default_rng(cols + fmt)
     rows = 19
     codes = rng.integers(lo, hi, size=(rows, cols)).astype(np.int8 if lo < 0 else np.uint8)
-    g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.NVFP4_G16: 16}[fmt]
+    g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.INT4_G32_ASYM: 32, tq.NVFP4_G16: 16}[fmt]
     G = (cols + g - 1) // g
     zeros = rng.integers(0, 16, size=(rows, G)).astype(np.uint8)
     ct = torch.from_numpy(codes).to(DEV)
@@ -300,7 +300,7 @@ def _edge_weights(rows, I, scales_per_group, g, seed, dtype):
     return W.to(dtype) if dtype != torch.float32 else W
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("I", [300, 1024])
 def test_pack_given_scales_edge_cases(fmt, dtype, I):
@@ -377,7 +377,7 @@ def _gemv_case(fmt, E, O, I, seed):
     (its RTN and packing), and the oracle's dequantized What."""
     rng = np.random.default_rng(seed)
     W = (rng.standard_t(4, size=(E, O, I)) * 0.02).astype(np.float32)
-    g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.NVFP4_G16: 16}[fmt]
+    g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.INT4_G32_ASYM: 32, tq.NVFP4_G16: 16}[fmt]
     G = (I + g - 1) // g
     zeros = gsc = None
     if fmt == tq.NVFP4_G16:
@@ -415,7 +415,7 @@ def _gemv_check(fmt, case, E, O, I, x, label):
     return got
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 @pytest.mark.parametrize("B", [1, 3, 8])
 @pytest.mark.parametrize("I", [100, 1802, 4096, 7000])
 def test_dequant_gemv_matches_oracle(fmt, B, I):
@@ -433,7 +433,7 @@ def test_dequant_gemv_matches_oracle(fmt, B, I):
     _gemv_check(fmt, case, E, O, I, xm.to(torch.float32 if dt == torch.bfloat16 else torch.bfloat16), "other dtype")
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 def test_dequant_gemv_shapes(fmt):
     """Many row chunks per block (x staged once), many small matrices with
     their own x (staged per matrix), a single weight, rows split over 2, 4
@@ -730,7 +730,7 @@ def _pf_inputs(E, T, O, I, seed, onehot):
     return X, W
 
 
-@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.NVFP4_G16])
+@pytest.mark.parametrize("fmt", [tq.INT3_G64_SYM, tq.INT4_G128_ASYM, tq.INT4_G64_ASYM, tq.INT4_G32_ASYM, tq.NVFP4_G16])
 @pytest.mark.parametrize("E,T,O,I", [(2, 300, 300, 200), (1, 128, 256, 64), (1, 1, 7, 16), (1, 257, 513, 1030)])
 def test_proxy_full_onehot_exact(fmt, E, T, O, I):
     """Tokens that are scaled unit vectors: every entry of X E^T is a single
@@ -818,7 +818,8 @@ def _gptq_U(rng, I, ldu=None, T=None):
     return out
 
 
-_GQ_FMT = {tq.INT3_G64_SYM: (3, 64), tq.INT4_G128_ASYM: (4, 128), tq.INT4_G64_ASYM: (4, 64)}
+_GQ_FMT = {tq.INT3_G64_SYM: (3, 64), tq.INT4_G128_ASYM: (4, 128), tq.INT4_G64_ASYM: (4, 64),
+           tq.INT4_G32_ASYM: (4, 32)}
 
 
 def _gptq_check(fmt, W, res, Uh, shared):
