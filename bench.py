@@ -781,7 +781,58 @@ def next_rows(tq, step, pk, peak_tinst):
     out["gptq_sweep"] = time_gptq(tq, step, peak_tinst)
     out["fp8_tensor"] = time_fp8(tq, step, pk, peak_tinst)
     out["lloyd_max_2bit"] = time_lloyd(tq, step, pk)
+    if step.units[0].fmt == "nvfp4_g16":
+        out["nvfp4_w4a4_gemm"] = time_w4a4(tq, step, pk)
     return out
+
+
+def time_w4a4(tq, step, pk, reps=5):
+    """NVFP4 W4A4 product on the first unit: every expert's calibration tokens
+    quantized to NVFP4 (tq_quant_nvfp4_act), their scales re-laid out as the
+    tensor core's scale tiles, and the block-scaled tcgen05 GEMM against the
+    expert's searched records (the weights' scale tiles made once, outside
+    the timed calls).  Roofline of the GEMM: the slower of its flops against
+    the dense FP4 peak (the measured bf16 figure x 4, the nominal FP4:bf16
+    ratio) and its bytes (records, scales, fp32 outputs) against HBM."""
+    u, r = step.units[0], step.res[0]
+    sets = [(s[0][u.site], s[1][0]) for s in step.sets]
+    X0 = sets[0][0]
+    E, O, I = u.W.shape
+    T = X0.shape[1]
+    if I % 32:
+        return {"skipped": "I must be a multiple of 32"}
+    G = I // 16
+    ws = tq.tq_nvfp4_scales_to_mma(r.scales.reshape(E, O, G).contiguous(), E, O, I)
+    act = tq.tq_quant_nvfp4_act(X0)
+    xs = tq.tq_nvfp4_scales_to_mma(act.scales, E, T, I)
+    y = torch.empty((E, T, O), dtype=torch.float32, device=X0.device)
+    tq.tq_gemm_nvfp4(act.packed, xs, act.global_scale, r.packed, ws, r.global_scale, E, T, O, I, out=y)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps + 1)]
+    ev[0].record()
+    for k in range(reps):
+        X = sets[k % len(sets)][0]
+        tq.tq_quant_nvfp4_act(X, out=act)
+        tq.tq_nvfp4_scales_to_mma(act.scales, E, T, I, out=xs)
+        ev[2 * k + 1].record()
+        tq.tq_gemm_nvfp4(act.packed, xs, act.global_scale, r.packed, ws, r.global_scale, E, T, O, I, out=y)
+        ev[2 * k + 2].record()
+    torch.cuda.synchronize()
+    call_ms = ev[0].elapsed_time(ev[-1]) / reps
+    gemm_ms = sum(ev[2 * k + 1].elapsed_time(ev[2 * k + 2]) for k in range(reps)) / reps
+    flops = 2 * E * T * O * I
+    nbytes = (E * O * G * 8 + E * O * G + E * T * G * 8 + E * T * G + E * T * O * 4)
+    fp4_peak = pk["bf16_tflops"] * 4
+    t_min = max(flops / (fp4_peak * 1e12), nbytes / (pk["hbm_gbs"] * 1e9))
+    return {"gemm_ms": gemm_ms, "call_ms": call_ms, "E": E, "T": T, "O": O, "I": I, "flops": flops,
+            "TFLOP/s": flops / (gemm_ms * 1e-3) / 1e12, "fp4_peak_tflops": fp4_peak,
+            "frac_tensor": flops / (gemm_ms * 1e-3) / 1e12 / fp4_peak, "bytes": nbytes,
+            "GB/s": nbytes / (gemm_ms * 1e-3) / 1e9,
+            "bound": "tensor" if flops / (fp4_peak * 1e12) >= nbytes / (pk["hbm_gbs"] * 1e9) else "hbm",
+            "frac": t_min / (gemm_ms * 1e-3),
+            "note": f"first unit: {E} experts x {T} tokens x {O} x {I}; {reps} calls (activation quantizer + "
+                    "scale tiles + GEMM), GEMM timed alone with CUDA events; fp4 peak = measured bf16 x 4 "
+                    "(nominal ratio); y fp32"}
 
 
 def time_pack(tq, step, pk, reps=12):

@@ -33,7 +33,8 @@ __all__ = [
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
-    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_debug_set_wait_limit", "tq_selftest_e2m1", "FORMATS", "EXPORTS",
+    "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_debug_set_wait_limit", "tq_selftest_e2m1",
+    "tq_quant_nvfp4_act", "Nvfp4Act", "tq_nvfp4_scales_to_mma", "tq_gemm_nvfp4", "FORMATS", "EXPORTS",
 ]
 
 INT4_G128_ASYM = 4
@@ -60,6 +61,7 @@ EXPORTS = [
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
     "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2", "tq_proxy_full_workspace_bytes",
     "tq_proxy_error_full", "tq_gptq_workspace_bytes", "tq_gptq_sweep", "tq_debug_set_wait_limit",
+    "tq_quant_nvfp4_act", "tq_nvfp4_scales_mma_bytes", "tq_nvfp4_scales_to_mma", "tq_gemm_nvfp4",
 ]
 
 
@@ -156,6 +158,10 @@ def lib():
             "tq_proxy_error_full": (i32, [Mp, Mp, P, i32, P, P, P, P, P, P, sz, P]),
             "tq_sync": (i32, [P]),
             "tq_debug_set_wait_limit": (i32, [i64]),
+            "tq_quant_nvfp4_act": (i32, [Mp, P, P, P, P]),
+            "tq_nvfp4_scales_mma_bytes": (sz, [i64, i64, i64]),
+            "tq_nvfp4_scales_to_mma": (i32, [P, i64, i64, i64, P, P]),
+            "tq_gemm_nvfp4": (i32, [P, P, P, P, P, P, i64, i64, i64, i64, P, P]),
             "tq_imatrix_static_capacity": (sz, []),
             "tq_imatrix_static": (i32, [Mp, P, i64, ctypes.c_float, i32, P]),
             "tq_selftest_e2m1": (i32, [P, P, P]),
@@ -615,6 +621,83 @@ def tq_gptq_sweep(W: torch.Tensor, fmt: int, scales: torch.Tensor, zeros: Option
     _check(lib().tq_gptq_sweep(ctypes.byref(d), fmt, _ptr(scales), _ptr(zeros), _ptr(U), U.stride(-2), ums,
                                _ptr(out[0]), _ptr(out[1]), _ptr(workspace), workspace.numel(), _stream(stream)),
            "tq_gptq_sweep")
+    return out
+
+
+@dataclasses.dataclass
+class Nvfp4Act:
+    packed: torch.Tensor        # u8 [n_mat, T, ceil(I/16) * 8] NVFP4 records
+    scales: torch.Tensor        # u8 [n_mat, T, ceil(I/16)] E4M3 block-scale codes
+    global_scale: torch.Tensor  # f32 [n_mat]
+
+
+def tq_quant_nvfp4_act(X: torch.Tensor, out: Optional[Nvfp4Act] = None, stream=None) -> Nvfp4Act:
+    """NVFP4 activations (the weights' recipe without the search): per matrix
+    g = amax / 2688, per 16-block the nearest E4M3 scale, E2M1 codes.
+    X: [T, I] or [n_mat, T, I] bf16/fp32 on the GPU."""
+    d = _mat(X, "X")
+    E, T, I = d.n_mat, d.rows, d.cols
+    G = (I + 15) // 16
+    if out is None:
+        out = Nvfp4Act(packed=torch.empty((E, T, G * 8), dtype=torch.uint8, device=X.device),
+                       scales=torch.empty((E, T, G), dtype=torch.uint8, device=X.device),
+                       global_scale=torch.empty(E, dtype=torch.float32, device=X.device))
+    for t, n, shape in ((out.packed, "packed", (E, T, G * 8)), (out.scales, "scales", (E, T, G))):
+        _cuda(t, n)
+        if t.dtype != torch.uint8 or not t.is_contiguous() or t.numel() != E * T * shape[2]:
+            raise TQError(f"{n} must be a contiguous uint8 tensor of {E * T * shape[2]} bytes")
+    _check(lib().tq_quant_nvfp4_act(ctypes.byref(d), _ptr(out.packed), _ptr(out.scales), _ptr(out.global_scale),
+                                    _stream(stream)), "tq_quant_nvfp4_act")
+    return out
+
+
+def tq_nvfp4_scales_mma_bytes(n_mat: int, rows: int, cols: int) -> int:
+    return int(lib().tq_nvfp4_scales_mma_bytes(n_mat, rows, cols))
+
+
+def tq_nvfp4_scales_to_mma(scales: torch.Tensor, n_mat: int, rows: int, cols: int,
+                           out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """E4M3 block-scale codes [n_mat, rows, ceil(cols/16)] in the tensor core's
+    scale tiles (include/tq.h)."""
+    _cuda(scales, "scales")
+    G = (cols + 15) // 16
+    if scales.dtype != torch.uint8 or not scales.is_contiguous() or scales.numel() != n_mat * rows * G:
+        raise TQError(f"scales must be contiguous uint8 [{n_mat}, {rows}, {G}]")
+    nb = tq_nvfp4_scales_mma_bytes(n_mat, rows, cols)
+    if out is None:
+        out = torch.empty(nb, dtype=torch.uint8, device=scales.device)
+    _cuda(out, "out")
+    if out.numel() < nb:
+        raise TQError(f"out needs {nb} bytes")
+    _check(lib().tq_nvfp4_scales_to_mma(_ptr(scales), n_mat, rows, cols, _ptr(out), _stream(stream)),
+           "tq_nvfp4_scales_to_mma")
+    return out
+
+
+def tq_gemm_nvfp4(x_packed: torch.Tensor, x_scales_mma: torch.Tensor, x_global: torch.Tensor,
+                  w_packed: torch.Tensor, w_scales_mma: torch.Tensor, w_global: torch.Tensor,
+                  n_mat: int, T: int, O: int, I: int, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """W4A4 product y [n_mat, T, O] (fp32) of NVFP4 activations and weights on
+    the block-scaled tensor cores; scales in the tiles of tq_nvfp4_scales_to_mma."""
+    G = (I + 15) // 16
+    for t, n, need in ((x_packed, "x_packed", n_mat * T * G * 8), (w_packed, "w_packed", n_mat * O * G * 8),
+                       (x_scales_mma, "x_scales_mma", tq_nvfp4_scales_mma_bytes(n_mat, T, I)),
+                       (w_scales_mma, "w_scales_mma", tq_nvfp4_scales_mma_bytes(n_mat, O, I))):
+        _cuda(t, n)
+        if t.dtype != torch.uint8 or not t.is_contiguous() or t.numel() < need:
+            raise TQError(f"{n} must be contiguous uint8 with at least {need} bytes")
+    for t, n in ((x_global, "x_global"), (w_global, "w_global")):
+        _cuda(t, n)
+        if t.dtype != torch.float32 or t.numel() < n_mat:
+            raise TQError(f"{n} must be float32 [{n_mat}]")
+    if out is None:
+        out = torch.empty((n_mat, T, O), dtype=torch.float32, device=x_packed.device)
+    _cuda(out, "out")
+    if out.dtype != torch.float32 or not out.is_contiguous() or out.numel() != n_mat * T * O:
+        raise TQError(f"out must be contiguous float32 [{n_mat}, {T}, {O}]")
+    _check(lib().tq_gemm_nvfp4(_ptr(x_packed), _ptr(x_scales_mma), _ptr(x_global), _ptr(w_packed),
+                               _ptr(w_scales_mma), _ptr(w_global), n_mat, T, O, I, _ptr(out), _stream(stream)),
+           "tq_gemm_nvfp4")
     return out
 
 

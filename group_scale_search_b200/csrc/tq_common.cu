@@ -103,5 +103,7 @@ TQ_API tq_status tq_sync(tq_stream_t stream) {
     if (hessian_take_timeouts()) return set_error(TQ_ERR_CUDA, "tq_sync: a tq_hessian pipeline wait timed out");
     if (proxy_full_take_timeouts())
         return set_error(TQ_ERR_CUDA, "tq_sync: a tq_proxy_error_full pipeline wait timed out");
+    if (nvfp4_gemm_take_timeouts())
+        return set_error(TQ_ERR_CUDA, "tq_sync: a tq_gemm_nvfp4 pipeline wait timed out");
     return TQ_OK;
 }

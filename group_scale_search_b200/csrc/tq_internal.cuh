@@ -34,6 +34,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 bool hessian_take_timeouts();
 // The same for tq_proxy_error_full's GEMM pipeline.
 bool proxy_full_take_timeouts();
+// The same for tq_gemm_nvfp4.
+bool nvfp4_gemm_take_timeouts();
 
 inline int elem_bytes(int32_t dt) { return dt == TQ_BF16 ? 2 : (dt == TQ_F32 ? 4 : 0); }
 

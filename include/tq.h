@@ -264,6 +264,51 @@ tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void* scales
                           const float* global_scale, int64_t n_mat, int64_t O, int64_t I, const void* x,
                           int32_t x_dtype, int64_t B, int64_t x_mat_stride, float* y, tq_stream_t stream);
 
+/* ------------------------------------------------------------------ NVFP4 W4A4 product
+ * [NVFP4] Quantization Recipe table (routed experts W4A4, group size 16) and
+ * Serving Instructions (FP4 MoE GEMM on Blackwell): y = x W^T with both
+ * operands NVFP4, on the block-scaled tensor cores.
+ *
+ * tq_quant_nvfp4_act: activations X (bf16 or fp32 tq_mat, n_mat matrices of
+ * T tokens x I) to NVFP4 with the weights' recipe minus the search: per
+ * matrix g = fl32(amax / 2688) (global_scale[n_mat], fp32); per 16-element
+ * block the positive finite E4M3 code nearest b / (6 g), b the block amax,
+ * by the exact distance |6 g dec(c) - b| with ties to the lower code (0 for
+ * an all-zero block or g = 0); elements E2M1 round-to-nearest-even of the
+ * IEEE quotient x / fl32(g dec(code)), saturating, sign in bit 3, zero +0.
+ * packed: NVFP4 records as tq_pack writes them (8 bytes per block, element
+ * 2k in the low nibble of byte k), dense [n_mat][T][ceil(I/16)]; scales:
+ * E4M3 codes [n_mat][T][ceil(I/16)].  Errors as tq_pack.
+ *
+ * tq_nvfp4_scales_to_mma: E4M3 block-scale codes [n_mat][rows][ceil(cols/16)]
+ * re-laid out as the tensor core's scale tiles (out: tq_nvfp4_scales_mma_bytes
+ * bytes, 16-byte aligned): per matrix, row tiles of 128 rows (their count
+ * rounded up to an even number) by chunks of 4 blocks (rounded up to a
+ * multiple of 4), each chunk 512 bytes with the scale of row r, block k at
+ * byte (r % 32) * 16 + ((r % 128) / 32) * 4 + k % 4; order [matrix][row
+ * tile][chunk]; padding is zero.  Weights need it once; activations per call.
+ *
+ * tq_gemm_nvfp4: y[e][t][o] = x_global[e] w_global[e] sum_k dec(ex[e][t][k])
+ * dec(ew[e][o][k]) sum_{j in block k} dec(cx[e][t][j]) dec(cw[e][o][j]),
+ * fp32 [n_mat][T][O] (row stride O), for records x_packed [n_mat][T][I/16]
+ * and w_packed [n_mat][O][I/16] (8 bytes per block, as tq_search_groups /
+ * tq_pack / tq_quant_nvfp4_act write them) and scales in the tiles of
+ * tq_nvfp4_scales_to_mma (T and O rows).  I must be a multiple of 32 and
+ * every pointer 16-byte aligned.  Accumulation is fp32 on the tensor cores:
+ * |y - y_exact| <= (I/16 + 32) 2^-22 sum_j |x_j w_j| (dequantized values),
+ * plus one rounding of the global-scale product.  Errors: TQ_ERR_INVALID_ARG
+ * for null/misaligned pointers or bad sizes.  A pipeline wait that exceeds
+ * its limit makes the CTA store nothing and the next tq_sync return
+ * TQ_ERR_CUDA. */
+tq_status tq_quant_nvfp4_act(const tq_mat* X, uint8_t* packed, uint8_t* scales, float* global_scale,
+                             tq_stream_t stream);
+size_t tq_nvfp4_scales_mma_bytes(int64_t n_mat, int64_t rows, int64_t cols);
+tq_status tq_nvfp4_scales_to_mma(const uint8_t* scales, int64_t n_mat, int64_t rows, int64_t cols, uint8_t* out,
+                                 tq_stream_t stream);
+tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_mma, const float* x_global,
+                        const uint8_t* w_packed, const uint8_t* w_scales_mma, const float* w_global,
+                        int64_t n_mat, int64_t T, int64_t O, int64_t I, float* y, tq_stream_t stream);
+
 /* ------------------------------------------------------------------ FP8 per tensor
  * E4M3 weights with one fp32 scale per matrix ([NVFP4] Quantization Recipe
  * table: FP8 per-tensor for the shared experts and the Mamba linears).  The
@@ -404,13 +449,13 @@ tq_status tq_gptq_sweep(const tq_mat* W, int32_t fmt, const void* scales, const 
 
 /* ------------------------------------------------------------------ testing aid
  * Synchronises `stream` and returns TQ_ERR_CUDA if it or an earlier kernel
- * failed (including a tq_hessian or tq_proxy_error_full launch that gave up
- * on a pipeline wait). */
+ * failed (including a tq_hessian, tq_proxy_error_full or tq_gemm_nvfp4 launch
+ * that gave up on a pipeline wait). */
 tq_status tq_sync(tq_stream_t stream);
 
 /* Testing aid for the give-up path of the tensor-core pipelines: the number
- * of try-wait rounds after which a pipeline wait of a later tq_hessian or
- * tq_proxy_error_full launch (in this process) gives up; rounds < 0 restores
+ * of try-wait rounds after which a pipeline wait of a later tq_hessian,
+ * tq_proxy_error_full or tq_gemm_nvfp4 launch (in this process) gives up; rounds < 0 restores
  * the default (2^22 rounds, seconds of waiting).  Only the waits of the
  * copy/MMA ring use it: a launch that gives up still waits, with the default
  * limit, for every copy it issued and every MMA it committed before it frees
