@@ -111,7 +111,7 @@ inline ImGeom im_geometry(const tq_mat* X) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(IM_THREADS)
+__global__ void __launch_bounds__(IM_THREADS, IM_RESIDENT)
 k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, int64_t ms,
                   int64_t tps, double* __restrict__ partial, int64_t n_mat) {
     constexpr int VEC = VecOf<T>::n;
@@ -130,11 +130,28 @@ k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, in
     int run = 0;
     int64_t t = t0 + wid;
     if (full) {
-        // IM_U token rows in flight per warp, then one at a time.
+        // IM_U token rows in flight per warp, then 8 and 4 (short slices keep
+        // their loads in flight too), then one at a time.
         for (; t + (IM_U - 1) * IM_WARPS < t1; t += IM_U * IM_WARPS) {
             im_rows<T, IM_U>(base, t, ld, acc);
             run += IM_U;
             if (run >= 32) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
+                run = 0;
+            }
+        }
+        for (; t + 7 * IM_WARPS < t1; t += 8 * IM_WARPS) {
+            im_rows<T, 8>(base, t, ld, acc);
+            if ((run += 8) >= 32) {
+#pragma unroll
+                for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
+                run = 0;
+            }
+        }
+        for (; t + 3 * IM_WARPS < t1; t += 4 * IM_WARPS) {
+            im_rows<T, 4>(base, t, ld, acc);
+            if ((run += 4) >= 32) {
 #pragma unroll
                 for (int i = 0; i < VEC; ++i) { accd[i] += static_cast<double>(acc[i]); acc[i] = 0.f; }
                 run = 0;

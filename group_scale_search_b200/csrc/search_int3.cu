@@ -81,14 +81,29 @@ __device__ __forceinline__ float2 err_clamped2(float2 w2, float2 m2, float2 ns2,
 }
 
 // fp64 loss of signed scale s over the warp's 64 elements (lane: l, l + 32),
-// codes from the IEEE quotient.  Identical in every lane.
+// codes those of the IEEE quotient (rtn_fast: the reciprocal's rounding is
+// redone with the IEEE division wherever it could differ).  Identical in
+// every lane.
 __device__ __forceinline__ double loss64_int3(float w0, float m0, float w1, float m1, float s) {
-    const double v0 = rtn_exact(w0, s, -4.f, 3.f), v1 = rtn_exact(w1, s, -4.f, 3.f);
+    const float inv = rcp_approx(s);
+    const double v0 = rtn_fast(w0, s, inv, -4.f, 3.f), v1 = rtn_fast(w1, s, inv, -4.f, 3.f);
     const double e0 = __dsub_rn(static_cast<double>(w0), __dmul_rn(static_cast<double>(s), v0));
     const double e1 = __dsub_rn(static_cast<double>(w1), __dmul_rn(static_cast<double>(s), v1));
     const double t = __dadd_rn(__dmul_rn(static_cast<double>(m0), __dmul_rn(e0, e0)),
                                __dmul_rn(static_cast<double>(m1), __dmul_rn(e1, e1)));
     return group_sum_d(t, FULL, 32);
+}
+
+// Warp argmin of non-negative losses (NaN ranks as +inf) whose candidate
+// indices grow with the lane: one min-reduction of the loss bits (non-negative
+// floats order like their bit patterns) and a ballot for the lowest lane that
+// holds it -- the lowest index on ties, as warp_argmin gives.
+__device__ __forceinline__ void warp_argmin_by_lane(float& L, int& idx) {
+    const unsigned key = L >= 0.f ? (__float_as_uint(L) & 0x7fffffffu) : 0x7f800000u;
+    const unsigned kmin = __reduce_min_sync(FULL, key);
+    const int src = __ffs(__ballot_sync(FULL, key == kmin)) - 1;
+    L = __uint_as_float(kmin);
+    idx = __shfl_sync(FULL, idx, src);
 }
 
 template <typename T>
@@ -114,27 +129,18 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const unsigned lt = (1u << lane) - 1u;
 
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * SYM_WARPS;
-    auto fetch = [&](int64_t g, float& a0, float& a1, float& b0, float& b1) {
-        uint32_t e32, o32, k32;
-        a.gi.split(static_cast<uint32_t>(g), e32, o32, k32);
-        const int64_t j0 = static_cast<int64_t>(k32) << 6;
-        const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
-        const T* wp = W + static_cast<int64_t>(e32) * a.ms + static_cast<int64_t>(o32) * a.ld + j0;
-        const float* mp = a.m + static_cast<int64_t>(e32) * a.m_stride + j0;
-        a0 = lane < n ? Elem<T>::load(wp + lane) : 0.f;
-        a1 = lane + 32 < n ? Elem<T>::load(wp + lane + 32) : 0.f;
-        b0 = lane < n ? __ldg(mp + lane) : 0.f;
-        b1 = lane + 32 < n ? __ldg(mp + lane + 32) : 0.f;
-    };
     for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total; gid += gstride) {
-        float w0, w1, m0, m1;
-        fetch(gid, w0, w1, m0, m1);
         uint32_t e32, o32, k32;
         a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
-        const int64_t k = k32;
-        const int64_t j0 = k << 6;
+        const int64_t j0 = static_cast<int64_t>(k32) << 6;
         const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
         const bool v0 = lane < n, v1 = lane + 32 < n;
+        const T* wp = W + static_cast<int64_t>(e32) * a.ms + static_cast<int64_t>(o32) * a.ld + j0;
+        const float* mp = a.m + static_cast<int64_t>(e32) * a.m_stride + j0;
+        const float w0 = v0 ? Elem<T>::load(wp + lane) : 0.f;
+        const float w1 = v1 ? Elem<T>::load(wp + lane + 32) : 0.f;
+        const float m0 = v0 ? __ldg(mp + lane) : 0.f;
+        const float m1 = v1 ? __ldg(mp + lane + 32) : 0.f;
         const float M = warp_max_abs(w0, w1);
         uint8_t* rec = a.packed ? a.packed + gid * 24 : nullptr;
 
@@ -182,12 +188,15 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float s1o = __fmul_rn(__fmul_rn(r1v, M), 0.25f);    // the candidate itself
         const float i1 = rcp_approx(s1);
         const float2 ns1 = make_float2(-s1, -s1), inv1 = make_float2(i1, i1);
-        float2 accC = make_float2(0.f, 0.f), accP = make_float2(0.f, 0.f), accN = make_float2(0.f, 0.f);
-        for (int j = 0; j < (ns_pad >> 2); ++j) {
+        float2 accC = make_float2(0.f, 0.f), accD = make_float2(0.f, 0.f);
+        float2 accP = make_float2(0.f, 0.f), accN = make_float2(0.f, 0.f);
+#pragma unroll 2
+        for (int j = 0; j < (ns_pad >> 2); ++j) {   // two independent accumulator chains
             const float4 w4 = spw[j], m4 = spm[j];
             accC = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns1, inv1, accC);
-            accC = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns1, inv1, accC);
+            accD = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns1, inv1, accD);
         }
+        accC = __fadd2_rn(accC, accD);
         for (int j = 0; j < (nl_pad >> 1); ++j) {
             const float2 w2 = reinterpret_cast<const float2*>(lgw)[j], m2 = reinterpret_cast<const float2*>(lgm)[j];
             err_both2(w2, m2, ns1, inv1, accP, accN);
@@ -200,7 +209,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         if (act1) {
             if (LN < LP) { L = LN; bi = 2 * lane + 1; } else { L = LP; bi = 2 * lane; }
         }
-        warp_argmin(L, bi);
+        warp_argmin_by_lane(L, bi);
         if (bi < 0 || bi >= 2 * a.n1) bi = 0;   // every loss non-finite: keep index 0
         int b1 = bi;
         bool have64 = false;
@@ -232,12 +241,14 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float i2 = rcp_approx(s2);
         const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
         const float2 ns2 = make_float2(-s2, -s2), inv2 = make_float2(i2, i2);
-        float2 a2 = make_float2(0.f, 0.f);
+        float2 a2 = make_float2(0.f, 0.f), a2b = make_float2(0.f, 0.f);
+#pragma unroll 2
         for (int j = 0; j < (ns_pad >> 2); ++j) {
             const float4 w4 = spw[j], m4 = spm[j];
             a2 = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns2, inv2, a2);
-            a2 = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns2, inv2, a2);
+            a2b = err_free2(make_float2(w4.z, w4.w), make_float2(m4.z, m4.w), ns2, inv2, a2b);
         }
+        a2 = __fadd2_rn(a2, a2b);
         for (int j = 0; j < (nl_pad >> 1); ++j) {
             const float2 w2 = reinterpret_cast<const float2*>(lgw)[j], m2 = reinterpret_cast<const float2*>(lgm)[j];
             a2 = err_clamped2(w2, m2, ns2, inv2, clo, chi, a2);
@@ -247,7 +258,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float L2 = act2 ? acc2 : __int_as_float(0x7f800000);
         float L2m = L2;
         int b2 = act2 ? 2 * a.n1 + lane : INT_MAX;
-        warp_argmin(L2m, b2);
+        warp_argmin_by_lane(L2m, b2);
 
         const float Lmin = fminf(L1f, L2m);
         const float thr2 = __fmaf_rn(Lmin, WIN, Lmin);

@@ -79,3 +79,28 @@ def test_sharded_step_equals_one_process(tmp_path, config):
                     np.testing.assert_allclose(got, m.numpy(), rtol=1e-6)
                 else:                     # expert-split site: this rank's experts
                     assert got.shape[1] == m.shape[1]
+
+
+def test_profile_table_rows_are_read_by_workload_and_kernel(tmp_path):
+    sys.path.insert(0, ROOT)
+    import bench
+    got = bench.read_profile(os.path.join(ROOT, "profiles", "traffic.md"), "c1", "search int4_g128_asym")
+    assert got["traffic"] == 33601792 and got["fp32_pipe_frac"] == 0.728
+    assert bench.read_profile(os.path.join(ROOT, "profiles", "traffic.md"), "c9", "k_proxy")["traffic"] is None
+    t = tmp_path / "t.md"
+    t.write_text("| c2 | k_proxy | 123 | 0.1 | - | x.md |\n")
+    assert bench.read_profile(str(t), "c2", "k_proxy") == {"traffic": 123, "fp32_pipe_frac": None, "source": "x.md"}
+
+
+def test_config_dictionary_is_shared_by_both_arms():
+    """The reference arm and the tq arm print the same config for the same
+    workload, GPU count and scaling; weights and groups follow the shapes."""
+    sys.path.insert(0, ROOT)
+    import bench
+    c = bench.config_dict("c2", 1.0, 1, "strong")
+    assert c["weights"] == 64 * 2048 * 7168 and c["groups"] == 64 * 2048 * 112
+    assert c["workload"].startswith("c2:") and "> 126 MiB L2" in c["l2"]
+    assert bench.config_dict("c2", 1.0, 8, "strong")["weights"] == 64 * 2048 * 7168
+    assert bench.config_dict("c2", 1.0, 8, "weak")["weights"] == 8 * 64 * 2048 * 7168
+    assert bench.config_dict("c4", 1.0, 1, "strong")["groups"] == 128 * 1856 * 168
+    assert bench.workload_weights("c3") == sum(o * i for _, o, i, _ in __import__("synth").C3_LINEARS)
