@@ -982,6 +982,8 @@ def time_hessian(tq, step, pk):
     figure."""
     u = step.units[0]
     Xs = [s[0][u.site][0] for s in step.sets]
+    if Xs[0].dtype != torch.bfloat16:
+        return {"skipped": "the tensor-core path takes bf16 activations"}
     T, I = Xs[0].shape
     H = torch.empty((I, I), dtype=torch.float32, device=Xs[0].device)
     flops = T * I * (I + 1)

@@ -197,8 +197,18 @@ __global__ void k_imatrix_final(const double* __restrict__ partial, int64_t slic
     const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     if (idx >= n_mat * I) return;
     const int64_t e = idx / I, j = idx - e * I;
+    const double* p = partial + e * I + j;
+    const int64_t step = n_mat * I;
     double s = 0.0;
-    for (int64_t k = 0; k < slices; ++k) s += partial[(k * n_mat + e) * I + j];
+    int64_t k = 0;
+    for (; k + 8 <= slices; k += 8) {   // 8 loads in flight, added in slice order
+        double v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldg(p + (k + u) * step);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) s += v[u];
+    }
+    for (; k < slices; ++k) s += __ldg(p + k * step);
     float v = static_cast<float>(alpha * s);
     float* dst = m + e * m_stride + j;
     if (accumulate) v = __fadd_rn(*dst, v);

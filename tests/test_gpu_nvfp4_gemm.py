@@ -28,8 +28,11 @@ def _setup():
 
 
 def _acts(E, T, I, seed, dtype=torch.bfloat16):
+    """Tokens with LogNormal channel scales; rows padded to a 16-byte stride
+    (the library's alignment rule) when I alone would not give one."""
     g = torch.Generator(device=DEV).manual_seed(seed)
-    X = torch.empty((E, T, I), dtype=dtype, device=DEV)
+    ld = -(-I * torch.tensor([], dtype=dtype).element_size() // 16) * 16 // torch.tensor([], dtype=dtype).element_size()
+    X = torch.zeros((E, T, ld), dtype=dtype, device=DEV)[:, :, :I]
     for e in range(E):
         c = synth.lognormal_channels(I, g, DEV)
         X[e] = (torch.randn((T, I), generator=g, device=DEV) * c).to(dtype)
