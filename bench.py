@@ -369,35 +369,40 @@ def config_dict(name: str, scale: float, world: int, scaling: str) -> dict:
 # ------------------------------------------------------------------ CPU oracle baseline
 
 def oracle_rows(wl, budget_s: float):
-    """Rows per unit for an oracle sample of about `budget_s` seconds."""
+    """(rows per unit, passes) for an oracle sample of about `budget_s`
+    seconds: the first rows of every unit's first matrix, repeated in whole
+    passes when that matrix is too small to fill the budget."""
     import oracle
     oracle.build()
     units = [u for u in wl.units if u.timed]
     probe_rows = 8
     t0 = time.perf_counter()
     _oracle_unit(oracle, wl, units[0], probe_rows)
-    per_row = (time.perf_counter() - t0) / probe_rows
-    return max(8, min(units[0].W.shape[1], int(budget_s / max(per_row, 1e-6) / len(units))))
+    per_row = max((time.perf_counter() - t0) / probe_rows, 1e-6)
+    rows = max(8, min(units[0].W.shape[1], int(budget_s / per_row / len(units))))
+    passes = max(1, int(round(budget_s / (per_row * rows * len(units)))))
+    return rows, passes
 
 
-def oracle_sample(wl, rows: int):
+def oracle_sample(wl, rows: int, passes: int = 1):
     """Times the oracle (as it stands) on a bounded sample of the workload:
     for each unit, the imatrix of its site (first matrix) and search + pack +
-    dequant + proxy error over the first `rows` rows of its first matrix.
-    Returns (weights/s, cores, description, seconds, weights)."""
+    dequant + proxy error over the first `rows` rows of its first matrix,
+    `passes` times.  Returns (weights/s, cores, description, seconds, weights)."""
     import oracle
     oracle.build()
     units = [u for u in wl.units if u.timed]
     t0 = time.perf_counter()
     n = 0
-    for u in units:
-        r = min(rows, u.W.shape[1])
-        _oracle_unit(oracle, wl, u, r)
-        n += r * u.W.shape[2]
+    for _ in range(passes):
+        for u in units:
+            r = min(rows, u.W.shape[1])
+            _oracle_unit(oracle, wl, u, r)
+            n += r * u.W.shape[2]
     dt = time.perf_counter() - t0
-    desc = (f"oracle (C, fp64, OpenMP) on {rows} rows of the first matrix of each of {len(units)} unit(s) "
-            f"= {n} weights: imatrix of the site's first matrix over all its tokens, search+pack, dequant, "
-            f"proxy; host CPU {cpu_model()}")
+    desc = (f"oracle (C, fp64, OpenMP) on {rows} rows of the first matrix of each of {len(units)} unit(s), "
+            f"{passes} pass(es) = {n} weights: imatrix of the site's first matrix over all its tokens, "
+            f"search+pack, dequant, proxy; host CPU {cpu_model()}")
     return n / dt, oracle.num_threads(), desc, dt, n
 
 
@@ -526,20 +531,21 @@ def reference_arm(args, world, rank):
     if rank != 0:
         return 0
     wl = synth.make(args.config, "cpu", seed=0, scale=args.scale, max_mats=1)
-    rows = oracle_rows(wl, budget_s=2.0)
+    rows, passes = oracle_rows(wl, budget_s=2.0)
     for _ in range(args.warmup):
         oracle_sample(wl, max(8, rows // 4))
     vals, secs = [], []
     desc = cores = n = None
     for _ in range(args.steps):
-        v, cores, desc, dt, n = oracle_sample(wl, rows)
+        v, cores, desc, dt, n = oracle_sample(wl, rows, passes)
         vals.append(v)
         secs.append(dt)
     dt = statistics.median(secs)
     v = n / dt
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "weights/s", "n_gpus": 0,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
-            "higher_is_better": True, "scaling": args.scaling, "vs_baseline": None, "dtype": "f64",
+            "higher_is_better": True, "scaling": args.scaling if args.gpus > 1 else "weak", "vs_baseline": None,
+            "dtype": "f64",
             "data": "synthetic", "config": config_dict(args.config, args.scale, args.gpus, args.scaling),
             "step_definition": f"one bounded sample of the workload per step ({n} weights), host cores only",
             "cpu_baseline": {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
@@ -651,8 +657,8 @@ def main(argv=None):
             "gpu_launches": headline["gpu_launches"],
             "per_workload": per}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rows = oracle_rows(wl_head, budget_s=12.0)
-        v, cores, desc, dt, _ = oracle_sample(wl_head, rows)
+        rows, passes = oracle_rows(wl_head, budget_s=12.0)
+        v, cores, desc, dt, _ = oracle_sample(wl_head, rows, passes)
         line["cpu_baseline"] = {"value": v, "unit": "weights/s", "cores": cores, "kind": "oracle",
                                 "sample": desc, "seconds": dt, "cpu": cpu_model()}
         one = oracle_one_thread(args.config)
