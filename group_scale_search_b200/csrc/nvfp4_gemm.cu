@@ -141,25 +141,37 @@ __global__ void k_sf_to_mma(const uint8_t* __restrict__ sc, int64_t rows, int64_
 
 // ------------------------------------------------------------------ GEMM
 
-constexpr int NG_M = 128, NG_N = 256;
+constexpr int NG_M = 128;
 constexpr int NG_BKB = 128;                                 // K bytes per stage (256 E2M1 codes)
-constexpr int NG_STAGES = 4;
 constexpr int NG_THREADS = 128;
 constexpr int NG_A_BYTES = NG_M * NG_BKB;                   // 16 KB
-constexpr int NG_B_BYTES = NG_N * NG_BKB;                   // 32 KB
 constexpr int NG_SFA_BYTES = 4 * 512;                       // 4 MMAs x one 128-row chunk
-constexpr int NG_SFB_BYTES = 8 * 512;                       // 4 MMAs x two 128-row chunks
-constexpr int NG_STAGE_BYTES = NG_A_BYTES + NG_B_BYTES + NG_SFA_BYTES + NG_SFB_BYTES;
-constexpr int NG_SMEM_BYTES = NG_STAGES * NG_STAGE_BYTES + 1024 + 256;
-constexpr uint32_t NG_TMEM_COLS = 512;                      // accumulator 256 + 2 x 48 scale columns
-constexpr uint32_t NG_SF_COL = 256;                         // first scale column
-static_assert(NG_STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
-static_assert(NG_SMEM_BYTES <= 232448, "shared memory");
 
-// kind::mxf4nvf4 block-scaled descriptor: E2M1 A and B (format 1), both
-// K-major, UE4M3 scales, dense K = 64, N = 256, M = 128.
-constexpr uint32_t NG_IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(NG_N >> 3) << 17) |
-                              (static_cast<uint32_t>(NG_M >> 4) << 24);
+// Tile shapes: 128 tokens x BN weight rows.  BN = 256: 4 stages, 216 KB of
+// shared memory and all 512 TMEM columns, one CTA per SM.  BN = 128: 3
+// stages, 2 CTAs per SM (each 256 TMEM columns), so one CTA's epilogue runs
+// while the other's MMAs do.
+template <int BN>
+struct NgCfg {
+    static constexpr int N = BN;
+    static constexpr int HALVES = BN / 128;                          // 128-row scale tiles per B tile
+    static constexpr int STAGES = BN == 256 ? 4 : 3;
+    static constexpr int B_BYTES = BN * NG_BKB;
+    static constexpr int SFB_BYTES = 4 * 512 * HALVES;               // 4 MMAs x HALVES chunks
+    static constexpr int STAGE_BYTES = NG_A_BYTES + B_BYTES + NG_SFA_BYTES + SFB_BYTES;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + 256;
+    static constexpr uint32_t SF_COL = BN;                           // first scale column
+    static constexpr uint32_t SF_COLS = 16 + 16 * HALVES;             // per stage parity: A 4 x 4, B 4 x 4 x HALVES
+    static constexpr uint32_t TMEM_COLS = BN == 256 ? 512 : 256;      // accumulator + 2 x SF_COLS, a power of 2
+    static constexpr int MIN_BLOCKS = BN == 256 ? 1 : 2;
+    // kind::mxf4nvf4 block-scaled descriptor: E2M1 A and B (format 1), both
+    // K-major, UE4M3 scales, dense K = 64, N = BN, M = 128.
+    static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
+                                      (static_cast<uint32_t>(NG_M >> 4) << 24);
+    static_assert(STAGE_BYTES % 1024 == 0, "stage bases stay 1024-byte aligned");
+    static_assert(SF_COL + 2 * SF_COLS <= TMEM_COLS, "TMEM columns");
+    static_assert(SMEM_BYTES * MIN_BLOCKS <= 232448, "shared memory");
+};
 
 __device__ unsigned g_ng_timeouts = 0;
 
@@ -211,12 +223,12 @@ __device__ __forceinline__ void ng_cp_sf(uint32_t taddr, uint64_t sdesc) {
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
-__device__ __forceinline__ void ng_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t tsfa, uint32_t tsfb,
-                                       uint32_t accumulate) {
+__device__ __forceinline__ void ng_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t tsfa,
+                                       uint32_t tsfb, uint32_t accumulate) {
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
         "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p; }" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(NG_IDESC), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
         : "memory");
 }
 
@@ -252,9 +264,13 @@ struct NgArgs {
     unsigned wait_limit;
 };
 
-__global__ void __launch_bounds__(NG_THREADS, 1)
+template <int BN>
+__global__ void __launch_bounds__(NG_THREADS, NgCfg<BN>::MIN_BLOCKS)
 k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
              const __grid_constant__ NgArgs a) {
+    using C = NgCfg<BN>;
+    constexpr int NG_N = C::N, NG_STAGES = C::STAGES, NG_STAGE_BYTES = C::STAGE_BYTES, NG_B_BYTES = C::B_BYTES;
+    constexpr int NG_SFB_BYTES = C::SFB_BYTES;
     const int tm = static_cast<int>(blockIdx.x) % a.tiles_m, tn = static_cast<int>(blockIdx.x) / a.tiles_m;
     const int e = static_cast<int>(blockIdx.y);
     extern __shared__ uint8_t ng_raw[];
@@ -278,7 +294,7 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(ng_smem_u32(tmem_slot)),
-                     "r"(NG_TMEM_COLS));
+                     "r"(C::TMEM_COLS));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -288,7 +304,7 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
 
     if (warp == 0 && lane == 0) {   // producer: TMA for the codes, bulk copies for the scale chunks
         const uint8_t* sfa = a.sfa + (static_cast<int64_t>(e) * a.rt_a + tm) * a.kc * 512;
-        const uint8_t* sfb0 = a.sfb + (static_cast<int64_t>(e) * a.rt_b + 2 * tn) * a.kc * 512;
+        const uint8_t* sfb0 = a.sfb + (static_cast<int64_t>(e) * a.rt_b + C::HALVES * tn) * a.kc * 512;
         const uint8_t* sfb1 = sfb0 + a.kc * 512;
         int kt = 0;
         for (; kt < nk; ++kt) {
@@ -301,8 +317,8 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
             ng_tma_3d(st + NG_A_BYTES, &bmap, bar, kt * NG_BKB, tn * NG_N, e);
             const int64_t off = static_cast<int64_t>(4 * kt) * 512;
             ng_bulk(st + NG_A_BYTES + NG_B_BYTES, sfa + off, NG_SFA_BYTES, bar);
-            ng_bulk(st + NG_A_BYTES + NG_B_BYTES + NG_SFA_BYTES, sfb0 + off, NG_SFB_BYTES / 2, bar);
-            ng_bulk(st + NG_A_BYTES + NG_B_BYTES + NG_SFA_BYTES + NG_SFB_BYTES / 2, sfb1 + off, NG_SFB_BYTES / 2, bar);
+            ng_bulk(st + NG_A_BYTES + NG_B_BYTES + NG_SFA_BYTES, sfb0 + off, 2048, bar);
+            if (C::HALVES == 2) ng_bulk(st + NG_A_BYTES + NG_B_BYTES + NG_SFA_BYTES + 2048, sfb1 + off, 2048, bar);
             progress[0] = kt + 1;
         }
         if (kt < nk) progress[2] = 0;
@@ -314,17 +330,18 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sa = s_base + s * NG_STAGE_BYTES, sb = sa + NG_A_BYTES;
             const uint32_t ssfa = sb + NG_B_BYTES, ssfb = ssfa + NG_SFA_BYTES;
-            const uint32_t tsf = tmem + NG_SF_COL + 48u * static_cast<uint32_t>(kt & 1);
+            const uint32_t tsf = tmem + C::SF_COL + C::SF_COLS * static_cast<uint32_t>(kt & 1);
+            constexpr uint32_t BC = 4 * C::HALVES;   // TMEM columns of B's scales per MMA
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 ng_cp_sf(tsf + 4 * j, ng_desc_sf(ssfa + 512 * j));
-                ng_cp_sf(tsf + 16 + 8 * j, ng_desc_sf(ssfb + 512 * j));
-                ng_cp_sf(tsf + 16 + 8 * j + 4, ng_desc_sf(ssfb + NG_SFB_BYTES / 2 + 512 * j));
+                ng_cp_sf(tsf + 16 + BC * j, ng_desc_sf(ssfb + 512 * j));
+                if (C::HALVES == 2) ng_cp_sf(tsf + 16 + BC * j + 4, ng_desc_sf(ssfb + 2048 + 512 * j));
             }
 #pragma unroll
             for (int j = 0; j < 4; ++j)   // K = 64 codes = 32 bytes of each row per MMA
-                ng_mma(tmem, ng_desc_sw128(sa + 32 * j), ng_desc_sw128(sb + 32 * j), tsf + 4 * j, tsf + 16 + 8 * j,
-                       (kt | j) != 0);
+                ng_mma(tmem, ng_desc_sw128(sa + 32 * j), ng_desc_sw128(sb + 32 * j), C::IDESC, tsf + 4 * j,
+                       tsf + 16 + BC * j, (kt | j) != 0);
             ng_commit(empty0 + 8 * s);   // the stage is free once these have read it
             progress[1] = kt + 1;
         }
@@ -369,7 +386,7 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
         if (progress[3] == 0) ng_wait(done, 0);
     }
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(NG_TMEM_COLS));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
 }
 
 // ------------------------------------------------------------------ host
@@ -464,6 +481,11 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     EncodeTiledFn enc = ng_encode();
     if (!enc) return set_error(TQ_ERR_CUDA, "tq_gemm_nvfp4: cuTensorMapEncodeTiled unavailable");
     const int64_t rowb = I / 2;
+#ifndef TQ_NG_N
+#define TQ_NG_N 256
+#endif
+    constexpr int BN = TQ_NG_N;
+    using C = NgCfg<BN>;
     CUtensorMap amap, bmap;
     const cuuint32_t estr[3] = {1, 1, 1};
     {
@@ -478,7 +500,7 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(rowb), static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(n_mat)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rowb), static_cast<cuuint64_t>(O * rowb)};
-        const cuuint32_t box[3] = {NG_BKB, NG_N, 1};
+        const cuuint32_t box[3] = {NG_BKB, static_cast<cuuint32_t>(BN), 1};
         CUresult r = enc(&bmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(w_packed), dims, strides, box,
                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -488,7 +510,7 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     a.T = T;
     a.O = O;
     a.tiles_m = static_cast<int>((T + NG_M - 1) / NG_M);
-    const int64_t tiles_n = (O + NG_N - 1) / NG_N;
+    const int64_t tiles_n = (O + BN - 1) / BN;
     a.nk = static_cast<int>((rowb + NG_BKB - 1) / NG_BKB);
     a.kc = sf_k_chunks((I + 15) / 16);
     a.rt_a = sf_row_tiles(T);
@@ -503,8 +525,10 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     const int64_t tiles = static_cast<int64_t>(a.tiles_m) * tiles_n;
     TQ_REQUIRE(tiles < (int64_t(1) << 31), "tq_gemm_nvfp4: too many tiles");
     static std::once_flag attr;
-    std::call_once(attr, [] { cudaFuncSetAttribute(k_gemm_nvfp4, cudaFuncAttributeMaxDynamicSharedMemorySize, NG_SMEM_BYTES); });
-    k_gemm_nvfp4<<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(n_mat)), NG_THREADS, NG_SMEM_BYTES,
+    std::call_once(attr, [] {
+        cudaFuncSetAttribute(k_gemm_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    });
+    k_gemm_nvfp4<BN><<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(n_mat)), NG_THREADS, C::SMEM_BYTES,
                    reinterpret_cast<cudaStream_t>(stream)>>>(amap, bmap, a);
     return check_launch("tq_gemm_nvfp4");
 }

@@ -27,6 +27,9 @@
 namespace tq {
 
 constexpr int SYM_WARPS = 8;
+// The next group's weights and imatrix are loaded while the current group is
+// searched (their HBM latency hidden inside the warp, not only across warps).
+constexpr bool SYM_PREFETCH = true;
 constexpr float WIN = 3.0517578125e-05f;   // 2^-15: bound on fp32 ranking error x 2 (with margin)
 
 struct SymArgs {
@@ -106,8 +109,28 @@ __device__ __forceinline__ void warp_argmin_by_lane(float& L, int& idx) {
     idx = __shfl_sync(FULL, idx, src);
 }
 
+// The group's 64 weights (and imatrix weights) as lane l holds them:
+// elements l and l + 32, zero past the group's n real elements.
 template <typename T>
-__global__ void __launch_bounds__(SYM_WARPS * 32)
+struct SymLoad {
+    float w0, w1, m0, m1;
+    int n;
+    __device__ __forceinline__ void load(const SymArgs& a, const T* W, int64_t gid, int lane) {
+        uint32_t e32, o32, k32;
+        a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
+        const int64_t j0 = static_cast<int64_t>(k32) << 6;
+        n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
+        const T* wp = W + static_cast<int64_t>(e32) * a.ms + static_cast<int64_t>(o32) * a.ld + j0;
+        const float* mp = a.m + static_cast<int64_t>(e32) * a.m_stride + j0;
+        w0 = lane < n ? Elem<T>::load(wp + lane) : 0.f;
+        w1 = lane + 32 < n ? Elem<T>::load(wp + lane + 32) : 0.f;
+        m0 = lane < n ? __ldg(mp + lane) : 0.f;
+        m1 = lane + 32 < n ? __ldg(mp + lane + 32) : 0.f;
+    }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(SYM_WARPS * 32, 32 / SYM_WARPS)
 k_search_int3(const __grid_constant__ SymArgs a) {
     __shared__ float r2s[32 * 32];
     __shared__ __align__(16) float lists[SYM_WARPS][2][2][64];   // [warp][small|large][w|m][element]
@@ -129,18 +152,20 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const unsigned lt = (1u << lane) - 1u;
 
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * SYM_WARPS;
-    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total; gid += gstride) {
-        uint32_t e32, o32, k32;
-        a.gi.split(static_cast<uint32_t>(gid), e32, o32, k32);
-        const int64_t j0 = static_cast<int64_t>(k32) << 6;
-        const int n = static_cast<int>(min(static_cast<int64_t>(64), a.I - j0));
+    SymLoad<T> nxt;
+    int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid;
+    if (SYM_PREFETCH && gid < total) nxt.load(a, W, gid, lane);
+    for (; gid < total; gid += gstride) {
+        SymLoad<T> cur;
+        if (SYM_PREFETCH) {
+            cur = nxt;
+            if (gid + gstride < total) nxt.load(a, W, gid + gstride, lane);
+        } else {
+            cur.load(a, W, gid, lane);
+        }
+        const int n = cur.n;
         const bool v0 = lane < n, v1 = lane + 32 < n;
-        const T* wp = W + static_cast<int64_t>(e32) * a.ms + static_cast<int64_t>(o32) * a.ld + j0;
-        const float* mp = a.m + static_cast<int64_t>(e32) * a.m_stride + j0;
-        const float w0 = v0 ? Elem<T>::load(wp + lane) : 0.f;
-        const float w1 = v1 ? Elem<T>::load(wp + lane + 32) : 0.f;
-        const float m0 = v0 ? __ldg(mp + lane) : 0.f;
-        const float m1 = v1 ? __ldg(mp + lane + 32) : 0.f;
+        const float w0 = cur.w0, w1 = cur.w1, m0 = cur.m0, m1 = cur.m1;
         const float M = warp_max_abs(w0, w1);
         uint8_t* rec = a.packed ? a.packed + gid * 24 : nullptr;
 
