@@ -261,13 +261,21 @@ struct NgArgs {
     const float* gx;
     const float* gw;
     float* y;                   // [n_mat][T][O]
+    int y_tma;                  // O % 4 == 0: the tile leaves through shared memory by TMA stores
     unsigned wait_limit;
 };
+
+__device__ __forceinline__ void ng_tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
 
 template <int BN>
 __global__ void __launch_bounds__(NG_THREADS, NgCfg<BN>::MIN_BLOCKS)
 k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
-             const __grid_constant__ NgArgs a) {
+             const __grid_constant__ CUtensorMap ymap, const __grid_constant__ NgArgs a) {
     using C = NgCfg<BN>;
     constexpr int NG_N = C::N, NG_STAGES = C::STAGES, NG_STAGE_BYTES = C::STAGE_BYTES, NG_B_BYTES = C::B_BYTES;
     constexpr int NG_SFB_BYTES = C::SFB_BYTES;
@@ -356,23 +364,50 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
     const int64_t m = static_cast<int64_t>(tm) * NG_M + warp * 32 + lane;
     const float gg = __fmul_rn(__ldg(a.gx + e), __ldg(a.gw + e));
     float* yr = a.y + (static_cast<int64_t>(e) * a.T + m) * a.O;
-    const bool vec = (a.O & 3) == 0;
+    if (ok && a.y_tma) {
+        // The tile goes through the (now idle) ring as 32-column chunks of
+        // 128 rows x 128 B in the 128-byte swizzled layout, and leaves by TMA
+        // stores (rows and columns past the matrix are clipped).  Thread r
+        // writes its row's 16-byte unit u at u ^ (r % 8): conflict-free.
+        const int r = warp * 32 + lane;
 #pragma unroll 1
-    for (int c0 = 0; c0 < NG_N; c0 += 32) {
-        float v[32];
-        ng_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
-        const int64_t o0 = static_cast<int64_t>(tn) * NG_N + c0;
-        if (!ok || m >= a.T || o0 >= a.O) continue;
-        if (vec && o0 + 32 <= a.O) {
-            float4* d = reinterpret_cast<float4*>(yr + o0);
+        for (int c0 = 0; c0 < NG_N; c0 += 32) {
+            float v[32];
+            ng_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
+            float4* row = reinterpret_cast<float4*>(smem + (c0 / 32) * (NG_M * 128) + r * 128);
 #pragma unroll
-            for (int i = 0; i < 8; ++i)
-                d[i] = make_float4(__fmul_rn(v[4 * i], gg), __fmul_rn(v[4 * i + 1], gg), __fmul_rn(v[4 * i + 2], gg),
-                                   __fmul_rn(v[4 * i + 3], gg));
-        } else {
+            for (int u = 0; u < 8; ++u)
+                row[u ^ (r & 7)] = make_float4(__fmul_rn(v[4 * u], gg), __fmul_rn(v[4 * u + 1], gg),
+                                               __fmul_rn(v[4 * u + 2], gg), __fmul_rn(v[4 * u + 3], gg));
+        }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            for (int q = 0; q < NG_N / 32; ++q)
+                if (static_cast<int64_t>(tn) * NG_N + 32 * q < a.O)
+                    ng_tma_store_3d(&ymap, s_base + q * (NG_M * 128), tn * NG_N + 32 * q, tm * NG_M, e);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        }
+    } else {
+        const bool vec = (a.O & 3) == 0;
+#pragma unroll 1
+        for (int c0 = 0; c0 < NG_N; c0 += 32) {
+            float v[32];
+            ng_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(c0), v);
+            const int64_t o0 = static_cast<int64_t>(tn) * NG_N + c0;
+            if (!ok || m >= a.T || o0 >= a.O) continue;
+            if (vec && o0 + 32 <= a.O) {
+                float4* d = reinterpret_cast<float4*>(yr + o0);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                if (o0 + i < a.O) yr[o0 + i] = __fmul_rn(v[i], gg);
+                for (int i = 0; i < 8; ++i)
+                    d[i] = make_float4(__fmul_rn(v[4 * i], gg), __fmul_rn(v[4 * i + 1], gg),
+                                       __fmul_rn(v[4 * i + 2], gg), __fmul_rn(v[4 * i + 3], gg));
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (o0 + i < a.O) yr[o0 + i] = __fmul_rn(v[i], gg);
+            }
         }
     }
 
@@ -486,8 +521,19 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
 #endif
     constexpr int BN = TQ_NG_N;
     using C = NgCfg<BN>;
-    CUtensorMap amap, bmap;
+    CUtensorMap amap, bmap, ymap;
     const cuuint32_t estr[3] = {1, 1, 1};
+    memset(&ymap, 0, sizeof ymap);
+    const int y_tma = (O % 4) == 0;
+    if (y_tma) {
+        const cuuint64_t dims[3] = {static_cast<cuuint64_t>(O), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(n_mat)};
+        const cuuint64_t strides[2] = {static_cast<cuuint64_t>(O * 4), static_cast<cuuint64_t>(T * O * 4)};
+        const cuuint32_t box[3] = {32, NG_M, 1};
+        CUresult r = enc(&ymap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, y, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return set_error(TQ_ERR_CUDA, "tq_gemm_nvfp4: y tensor map (%d)", static_cast<int>(r));
+    }
     {
         const cuuint64_t dims[3] = {static_cast<cuuint64_t>(rowb), static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(n_mat)};
         const cuuint64_t strides[2] = {static_cast<cuuint64_t>(rowb), static_cast<cuuint64_t>(T * rowb)};
@@ -520,6 +566,7 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     a.gx = x_global;
     a.gw = w_global;
     a.y = y;
+    a.y_tma = y_tma;
     a.wait_limit = pipeline_wait_limit();
     TQ_REQUIRE(a.kc == 4 * a.nk, "tq_gemm_nvfp4: internal tiling mismatch");
     const int64_t tiles = static_cast<int64_t>(a.tiles_m) * tiles_n;
@@ -529,6 +576,6 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
         cudaFuncSetAttribute(k_gemm_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     k_gemm_nvfp4<BN><<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(n_mat)), NG_THREADS, C::SMEM_BYTES,
-                   reinterpret_cast<cudaStream_t>(stream)>>>(amap, bmap, a);
+                   reinterpret_cast<cudaStream_t>(stream)>>>(amap, bmap, ymap, a);
     return check_launch("tq_gemm_nvfp4");
 }
