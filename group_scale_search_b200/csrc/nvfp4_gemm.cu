@@ -60,20 +60,34 @@ namespace tq {
 
 // ------------------------------------------------------------------ activation quantizer
 
-// The positive finite E4M3 code (1..126) nearest t = b / (6 g): the first c
-// with d(c) <= d(c + 1), d(c) = |6 g dec(c) - b| (exact in fp64: 6 g dec(c)
-// has at most 31 significant bits), which is the lowest code of the minimum
-// because d falls and then rises along the codes.
+// Largest E4M3 code (1..126) whose value does not exceed the fp32 value t
+// (1 below the smallest subnormal); exact for t itself, so within one code
+// of the floor code of the exact quotient b / (6 g) that t rounds.
+__device__ __forceinline__ int e4m3_floor(float t) {
+    if (!(t > 0.f)) return 1;
+    if (t < 0.015625f) return max(1, static_cast<int>(t * 512.f));
+    const unsigned u = __float_as_uint(t);
+    const int E = static_cast<int>((u >> 23) & 255u) - 127;
+    return min(max(((E + 7) << 3) | static_cast<int>((u >> 20) & 7u), 1), 126);
+}
+
+// The positive finite E4M3 code (1..126) nearest t = b / (6 g) by the exact
+// distance d(c) = |6 g dec(c) - b| (fp64: 6 g dec(c) has at most 31
+// significant bits), ties to the lower code.  The nearest code is the floor
+// code of the exact t or the next one; the fp32 estimate of t is within one
+// code of that floor, so the four codes around it hold the answer, compared
+// in ascending order with strict improvement.
 __device__ __forceinline__ int nearest_e4m3_code(float b, float g) {
     const double g6 = 6.0 * static_cast<double>(g), bd = static_cast<double>(b);
-    int lo = 1, hi = 126;
-    while (lo < hi) {
-        const int mid = (lo + hi) >> 1;
-        const bool falls = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(e4m3_value(mid))), bd)) >
-                           fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(e4m3_value(mid + 1))), bd));
-        if (falls) lo = mid + 1; else hi = mid;
+    const int c0 = max(1, min(123, e4m3_floor(__fdiv_rn(b, __fmul_rn(6.f, g))) - 1));
+    int best = c0;
+    double bdist = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(e4m3_value(c0))), bd));
+#pragma unroll
+    for (int i = 1; i < 4; ++i) {
+        const double d = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(e4m3_value(c0 + i))), bd));
+        if (d < bdist) { bdist = d; best = c0 + i; }
     }
-    return lo;
+    return best;
 }
 
 // amax -> g = fl32(amax / 2688), in place.
@@ -517,7 +531,7 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     if (!enc) return set_error(TQ_ERR_CUDA, "tq_gemm_nvfp4: cuTensorMapEncodeTiled unavailable");
     const int64_t rowb = I / 2;
 #ifndef TQ_NG_N
-#define TQ_NG_N 256
+#define TQ_NG_N 128
 #endif
     constexpr int BN = TQ_NG_N;
     using C = NgCfg<BN>;

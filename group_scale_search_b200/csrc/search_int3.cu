@@ -27,9 +27,6 @@
 namespace tq {
 
 constexpr int SYM_WARPS = 8;
-// The next group's weights and imatrix are loaded while the current group is
-// searched (their HBM latency hidden inside the warp, not only across warps).
-constexpr bool SYM_PREFETCH = true;
 constexpr float WIN = 3.0517578125e-05f;   // 2^-15: bound on fp32 ranking error x 2 (with margin)
 
 struct SymArgs {
@@ -130,7 +127,7 @@ struct SymLoad {
 };
 
 template <typename T>
-__global__ void __launch_bounds__(SYM_WARPS * 32, 32 / SYM_WARPS)
+__global__ void __launch_bounds__(SYM_WARPS * 32)
 k_search_int3(const __grid_constant__ SymArgs a) {
     __shared__ float r2s[32 * 32];
     __shared__ __align__(16) float lists[SYM_WARPS][2][2][64];   // [warp][small|large][w|m][element]
@@ -152,17 +149,9 @@ k_search_int3(const __grid_constant__ SymArgs a) {
     const unsigned lt = (1u << lane) - 1u;
 
     const int64_t gstride = static_cast<int64_t>(gridDim.x) * SYM_WARPS;
-    SymLoad<T> nxt;
-    int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid;
-    if (SYM_PREFETCH && gid < total) nxt.load(a, W, gid, lane);
-    for (; gid < total; gid += gstride) {
+    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * SYM_WARPS + wid; gid < total; gid += gstride) {
         SymLoad<T> cur;
-        if (SYM_PREFETCH) {
-            cur = nxt;
-            if (gid + gstride < total) nxt.load(a, W, gid + gstride, lane);
-        } else {
-            cur.load(a, W, gid, lane);
-        }
+        cur.load(a, W, gid, lane);
         const int n = cur.n;
         const bool v0 = lane < n, v1 = lane + 32 < n;
         const float w0 = cur.w0, w1 = cur.w1, m0 = cur.m0, m1 = cur.m1;

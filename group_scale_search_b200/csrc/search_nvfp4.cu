@@ -33,6 +33,9 @@ namespace tq {
 constexpr int FP4_THREADS = 128;
 constexpr int FP4_WARPS = FP4_THREADS / 32;
 constexpr float FWIN = 3.0517578125e-05f;   // 2^-15
+// E4M3 values from a shared-memory table (true) or built from the code's
+// bit fields in registers (false).
+constexpr bool FP4_DEC_SMEM = true;
 
 struct Fp4Args {
     const void* W;
@@ -117,6 +120,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
     __shared__ double qres_l[FP4_WARPS][32];
     for (int i = threadIdx.x; i < 128; i += blockDim.x) dec[i] = e4m3_value(i);
     __syncthreads();
+    auto decv = [&](int c) { return FP4_DEC_SMEM ? dec[c] : e4m3_value(static_cast<unsigned>(c)); };
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     const int half = lane >> 4, hl = lane & 15;
     const int64_t G = (a.I + 15) >> 4;
@@ -174,8 +178,8 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
             int lo_a = max(1, cdn - 17), hi_a = min(lo_max, cdn + 2);
             while (lo_a < hi_a) {
                 const int mid = (lo_a + hi_a) >> 1;
-                const bool p = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(dec[mid])), ad)) >
-                               fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(dec[mid + Wn])), ad));
+                const bool p = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(decv(mid))), ad)) >
+                               fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(decv(mid + Wn))), ad));
                 if (p) lo_a = mid + 1; else hi_a = mid;
             }
             lo = lo_a;
@@ -193,7 +197,7 @@ k_search_nvfp4(const __grid_constant__ Fp4Args a) {
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
                 const int code = lo + (c < Wn ? c : 0);
-                const float S = __fmul_rn(__fmul_rn(g, dec[code]), pw);
+                const float S = __fmul_rn(__fmul_rn(g, decv(code)), pw);
                 const float inv = rcp_approx(S);
                 const float2 S2 = make_float2(-S, -S), inv2 = make_float2(inv, inv);
                 float2 acc = make_float2(0.f, 0.f);
