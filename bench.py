@@ -448,19 +448,22 @@ def _oracle_unit(oracle, wl, u, rows):
 
 def read_profile(path, workload, kernel):
     """The ncu figures of `kernel` on `workload` from the profiles table:
-    DRAM bytes per launch (read + write) and the FP32-pipe share of issue,
-    or None where the table has no entry."""
-    out = {"traffic": None, "fp32_pipe_frac": None, "source": None}
+    launches per step, DRAM bytes (read + write) and duration summed over
+    them, and the FP32-pipe share of its peak; None where the table has no
+    entry."""
+    out = {"launches": None, "traffic": None, "ms": None, "fp32_pipe_frac": None, "source": None}
     try:
         for line in open(path):
             cells = [c.strip() for c in line.strip().strip("|").split("|")]
-            if len(cells) >= 6 and cells[0] == workload and cells[1] == kernel:
-                out["traffic"] = int(cells[2]) if cells[2].isdigit() else None
-                try:
-                    out["fp32_pipe_frac"] = float(cells[4])
-                except ValueError:
-                    pass
-                out["source"] = cells[5]
+            if len(cells) >= 7 and cells[0] == workload and cells[1] == kernel and cells[2].isdigit():
+                out["launches"] = int(cells[2])
+                out["traffic"] = int(cells[3]) if cells[3].isdigit() else None
+                for key, cell in (("ms", cells[4]), ("fp32_pipe_frac", cells[5])):
+                    try:
+                        out[key] = float(cell)
+                    except ValueError:
+                        pass
+                out["source"] = cells[6]
     except OSError:
         pass
     return out
@@ -729,8 +732,9 @@ def run_workload(tq, name, args, world, rank, dev, barrier, pk, keep_wl=False):
     achieved = SEARCH_INSTR_PER_W[fmt_main] * by_fmt[fmt_main][1] / args.steps / (search_ms * 1e-3) / 1e12
     clocks = clk.summary()
     prof = read_profile(args.profile_table, name, f"search {fmt_main}")
+    per_launch_traffic = (prof["traffic"] // prof["launches"]) if prof["traffic"] and prof["launches"] else None
     roofline = {"bound": "alu", "achieved": achieved, "peak": peak_tinst, "unit": "Tinst/s",
-                "frac": achieved / peak_tinst, "traffic": prof["traffic"] if args.scale == 1.0 else None,
+                "frac": achieved / peak_tinst, "traffic": per_launch_traffic if args.scale == 1.0 else None,
                 "kernel": f"search {fmt_main}", "kernel_ms": search_ms / n_launch, "launches_per_step": n_launch,
                 "weights_per_launch": w_per_launch,
                 "per_unit": f"{SEARCH_INSTR_PER_W[fmt_main]} FP32 lane-instr/weight "
@@ -754,9 +758,12 @@ def run_workload(tq, name, args, world, rank, dev, barrier, pk, keep_wl=False):
     for rname, (t_ms, nb, cnt) in rows.items():
         gbs = nb / (t_ms * 1e-3) / 1e9
         p = read_profile(args.profile_table, name, kname[rname])
+        ok = args.scale == 1.0 and p["traffic"] is not None
         hbm_rows[rname] = {"ms": t_ms / args.steps, "bytes": nb // args.steps, "launches_per_step": cnt // args.steps,
                            "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
-                           "ncu_traffic": p["traffic"] if args.scale == 1.0 else None}
+                           "ncu_traffic": p["traffic"] if ok else None, "ncu_ms": p["ms"] if ok else None,
+                           "ncu_frac": (nb / args.steps / (p["ms"] * 1e-3) / 1e9 / pk["hbm_gbs"])
+                           if ok and p["ms"] else None}
     hbm_rows["pack"] = time_pack(tq, step, pk)
     row = {"value": value, "ms_per_step": ms_step, "weights": nw_job, "weights_this_rank": nw_rank,
            "groups_per_s": value / _GROUP[fmt_main], "roofline": roofline, "hbm_rows": hbm_rows,

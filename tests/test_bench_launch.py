@@ -85,11 +85,12 @@ def test_profile_table_rows_are_read_by_workload_and_kernel(tmp_path):
     sys.path.insert(0, ROOT)
     import bench
     got = bench.read_profile(os.path.join(ROOT, "profiles", "traffic.md"), "c1", "search int4_g128_asym")
-    assert got["traffic"] == 33601792 and got["fp32_pipe_frac"] == 0.728
+    assert got["traffic"] == 33601792 and got["fp32_pipe_frac"] == 0.728 and got["launches"] == 1
     assert bench.read_profile(os.path.join(ROOT, "profiles", "traffic.md"), "c9", "k_proxy")["traffic"] is None
     t = tmp_path / "t.md"
-    t.write_text("| c2 | k_proxy | 123 | 0.1 | - | x.md |\n")
-    assert bench.read_profile(str(t), "c2", "k_proxy") == {"traffic": 123, "fp32_pipe_frac": None, "source": "x.md"}
+    t.write_text("| c2 | k_proxy | 2 | 123 | 0.1 | - | x.md |\n")
+    assert bench.read_profile(str(t), "c2", "k_proxy") == {"launches": 2, "traffic": 123, "ms": 0.1,
+                                                          "fp32_pipe_frac": None, "source": "x.md"}
 
 
 def test_config_dictionary_is_shared_by_both_arms():
