@@ -292,7 +292,6 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
              const __grid_constant__ CUtensorMap ymap, const __grid_constant__ NgArgs a) {
     using C = NgCfg<BN>;
     constexpr int NG_N = C::N, NG_STAGES = C::STAGES, NG_STAGE_BYTES = C::STAGE_BYTES, NG_B_BYTES = C::B_BYTES;
-    constexpr int NG_SFB_BYTES = C::SFB_BYTES;
     const int tm = static_cast<int>(blockIdx.x) % a.tiles_m, tn = static_cast<int>(blockIdx.x) / a.tiles_m;
     const int e = static_cast<int>(blockIdx.y);
     extern __shared__ uint8_t ng_raw[];
@@ -436,6 +435,203 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
     }
     __syncthreads();
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(C::TMEM_COLS));
+}
+
+// ------------------------------------------------------------------ persistent GEMM
+
+// Persistent form: one CTA per SM walks the output tiles (128 tokens x 128
+// weight rows) in order, with warp roles: warp 0 lane 0 feeds a 4-stage ring
+// (TMA + bulk copies, as above) across tile boundaries; warp 1 lane 0 issues
+// the scale copies and MMAs into one of two TMEM accumulators (columns 0-127
+// and 128-255); warps 2-5 drain the other accumulator -- tcgen05.ld, scale,
+// swizzled shared-memory tile, TMA store -- while the next tile's MMAs run.
+// mbarriers: full/empty per stage (copies / MMA reads), acc_full per
+// accumulator (MMAs complete, tcgen05.commit) and acc_empty per accumulator
+// (the 128 epilogue threads have read it).
+// The persistent form (true) or one CTA per tile (false).
+constexpr bool NG_PERSISTENT = true;
+constexpr int NP_STAGES = 4;
+constexpr int NP_THREADS = 192;
+constexpr int NP_B_BYTES = 128 * NG_BKB;
+constexpr int NP_STAGE_BYTES = NG_A_BYTES + NP_B_BYTES + NG_SFA_BYTES + 2048;
+constexpr int NP_OUT_BYTES = 128 * 128 * 4;                      // one fp32 output tile
+constexpr int NP_SMEM_BYTES = NP_STAGES * NP_STAGE_BYTES + NP_OUT_BYTES + 1024 + 256;
+constexpr uint32_t NP_SF_COL = 256, NP_SF_COLS = 32;           // per k-step parity: A 4 x 4, B 4 x 4
+constexpr uint32_t NP_IDESC = NgCfg<128>::IDESC;
+static_assert(NP_STAGE_BYTES % 1024 == 0 && NP_SMEM_BYTES <= 232448, "persistent GEMM shared memory");
+
+__device__ __forceinline__ void ng_named_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
+__global__ void __launch_bounds__(NP_THREADS, 1)
+k_gemm_nvfp4_persistent(const __grid_constant__ CUtensorMap amap, const __grid_constant__ CUtensorMap bmap,
+                        const __grid_constant__ CUtensorMap ymap, const __grid_constant__ NgArgs a,
+                        int tiles_n, int64_t n_tiles) {
+    extern __shared__ uint8_t np_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(np_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* outbuf = smem + NP_STAGES * NP_STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(outbuf + NP_OUT_BYTES);
+    // bars: full[S], empty[S], acc_full[2], acc_empty[2], done
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * NP_STAGES + 5);
+    volatile int* st = reinterpret_cast<volatile int*>(tmem_slot + 1);   // [0] armed, [1] consumed, [2] abort
+    const uint32_t s_base = ng_smem_u32(smem), o_base = ng_smem_u32(outbuf);
+    const uint32_t full0 = ng_smem_u32(bars), empty0 = full0 + 8 * NP_STAGES;
+    const uint32_t accf0 = empty0 + 8 * NP_STAGES, acce0 = accf0 + 16, done = acce0 + 16;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nk = a.nk;
+    const int tiles_per_mat = a.tiles_m * tiles_n;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2 * NP_STAGES + 2; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(full0 + 8 * i) : "memory");
+        for (int i = 0; i < 2; ++i)
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], 128;" ::"r"(acce0 + 8 * i) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(done) : "memory");
+        st[0] = 0;
+        st[1] = 0;
+        st[2] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(ng_smem_u32(tmem_slot)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_slot;
+
+    auto tile_of = [&](int64_t t, int& e, int& tm, int& tn) {
+        e = static_cast<int>(t / tiles_per_mat);
+        const int r = static_cast<int>(t - static_cast<int64_t>(e) * tiles_per_mat);
+        tn = r / a.tiles_m;
+        tm = r - tn * a.tiles_m;
+    };
+
+    if (warp == 0 && lane == 0) {   // producer, across tile boundaries
+        int q = 0;   // stage uses so far
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
+            int e, tm, tn;
+            tile_of(t, e, tm, tn);
+            const uint8_t* sfa = a.sfa + (static_cast<int64_t>(e) * a.rt_a + tm) * a.kc * 512;
+            const uint8_t* sfb = a.sfb + (static_cast<int64_t>(e) * a.rt_b + tn) * a.kc * 512;
+            for (int kt = 0; kt < nk; ++kt, ++q) {
+                const int s = q % NP_STAGES;
+                if (st[2] || !ng_wait(empty0 + 8 * s, ((q / NP_STAGES) & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+                const uint32_t sb = s_base + s * NP_STAGE_BYTES, bar = full0 + 8 * s;
+                asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(NP_STAGE_BYTES)
+                             : "memory");
+                ng_tma_3d(sb, &amap, bar, kt * NG_BKB, tm * NG_M, e);
+                ng_tma_3d(sb + NG_A_BYTES, &bmap, bar, kt * NG_BKB, tn * 128, e);
+                const int64_t off = static_cast<int64_t>(4 * kt) * 512;
+                ng_bulk(sb + NG_A_BYTES + NP_B_BYTES, sfa + off, NG_SFA_BYTES, bar);
+                ng_bulk(sb + NG_A_BYTES + NP_B_BYTES + NG_SFA_BYTES, sfb + off, 2048, bar);
+                st[0] = q + 1;
+            }
+        }
+        if (!ok) st[2] = 1;
+    } else if (warp == 1 && lane == 0) {   // scale copies and MMAs
+        int q = 0, i = 0;
+        bool ok = true;
+        for (int64_t t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++i) {
+            const int b = i & 1, u = i >> 1;
+            if (st[2] || !ng_wait(acce0 + 8 * b, (u & 1) ^ 1, a.wait_limit)) { ok = false; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t acc = tmem + 128u * static_cast<uint32_t>(b);
+            for (int kt = 0; kt < nk; ++kt, ++q) {
+                const int s = q % NP_STAGES;
+                if (st[2] || !ng_wait(full0 + 8 * s, (q / NP_STAGES) & 1, a.wait_limit)) { ok = false; break; }
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t sa = s_base + s * NP_STAGE_BYTES, sb = sa + NG_A_BYTES;
+                const uint32_t ssfa = sb + NP_B_BYTES, ssfb = ssfa + NG_SFA_BYTES;
+                const uint32_t tsf = tmem + NP_SF_COL + NP_SF_COLS * static_cast<uint32_t>(q & 1);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    ng_cp_sf(tsf + 4 * j, ng_desc_sf(ssfa + 512 * j));
+                    ng_cp_sf(tsf + 16 + 4 * j, ng_desc_sf(ssfb + 512 * j));
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    ng_mma(acc, ng_desc_sw128(sa + 32 * j), ng_desc_sw128(sb + 32 * j), NP_IDESC, tsf + 4 * j,
+                           tsf + 16 + 4 * j, (kt | j) != 0);
+                ng_commit(empty0 + 8 * s);
+                st[1] = q + 1;
+            }
+            if (!ok) break;
+            ng_commit(accf0 + 8 * b);   // this tile's accumulator is complete once its MMAs are
+        }
+        if (!ok) st[2] = 1;
+        ng_commit(done);
+    } else if (warp >= 2) {   // epilogue: 4 warps, warp w reads TMEM lanes 32 (w % 4) ..
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;   // row of the tile
+        int i = 0;
+        for (int64_t t = blockIdx.x; t < n_tiles; t += gridDim.x, ++i) {
+            const int b = i & 1, u = i >> 1;
+            if (!ng_wait(accf0 + 8 * b, u & 1, a.wait_limit) || st[2]) { st[2] = 1; break; }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            int e, tm, tn;
+            tile_of(t, e, tm, tn);
+            const float gg = __fmul_rn(__ldg(a.gx + e), __ldg(a.gw + e));
+            const uint32_t acc = tmem + 128u * static_cast<uint32_t>(b) + (static_cast<uint32_t>(quarter * 32) << 16);
+            if (a.y_tma) {
+                if (threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                ng_named_sync(1, 128);   // the previous tile's stores have read the staging tile
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float v[32];
+                    ng_ld32(acc + static_cast<uint32_t>(c0), v);
+                    float4* row = reinterpret_cast<float4*>(outbuf + (c0 / 32) * (NG_M * 128) + r * 128);
+#pragma unroll
+                    for (int w = 0; w < 8; ++w)
+                        row[w ^ (r & 7)] = make_float4(__fmul_rn(v[4 * w], gg), __fmul_rn(v[4 * w + 1], gg),
+                                                       __fmul_rn(v[4 * w + 2], gg), __fmul_rn(v[4 * w + 3], gg));
+                }
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                ng_named_sync(1, 128);
+                if (threadIdx.x == 64) {
+                    for (int qq = 0; qq < 4; ++qq)
+                        if (static_cast<int64_t>(tn) * 128 + 32 * qq < a.O)
+                            ng_tma_store_3d(&ymap, o_base + qq * (NG_M * 128), tn * 128 + 32 * qq, tm * NG_M, e);
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                }
+            } else {
+                const int64_t m = static_cast<int64_t>(tm) * NG_M + r;
+                float* yr = a.y + (static_cast<int64_t>(e) * a.T + m) * a.O;
+#pragma unroll 1
+                for (int c0 = 0; c0 < 128; c0 += 32) {
+                    float v[32];
+                    ng_ld32(acc + static_cast<uint32_t>(c0), v);
+                    const int64_t o0 = static_cast<int64_t>(tn) * 128 + c0;
+                    if (m < a.T && o0 < a.O) {
+#pragma unroll
+                        for (int k = 0; k < 32; ++k)
+                            if (o0 + k < a.O) yr[o0 + k] = __fmul_rn(v[k], gg);
+                    }
+                }
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(acce0 + 8 * b) : "memory");
+            }
+        }
+        if (threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+    }
+
+    // teardown: the copies armed but not consumed and the MMAs committed,
+    // with the default limit; then free TMEM
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        for (int k = st[1]; k < st[0]; ++k)
+            if (!ng_wait(full0 + 8 * (k % NP_STAGES), (k / NP_STAGES) & 1)) break;
+        ng_wait(done, 0);
+    }
+    __syncthreads();
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(512));
 }
 
 // ------------------------------------------------------------------ host
@@ -585,11 +781,23 @@ TQ_API tq_status tq_gemm_nvfp4(const uint8_t* x_packed, const uint8_t* x_scales_
     TQ_REQUIRE(a.kc == 4 * a.nk, "tq_gemm_nvfp4: internal tiling mismatch");
     const int64_t tiles = static_cast<int64_t>(a.tiles_m) * tiles_n;
     TQ_REQUIRE(tiles < (int64_t(1) << 31), "tq_gemm_nvfp4: too many tiles");
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (NG_PERSISTENT && BN == 128) {
+        static std::once_flag pattr;
+        std::call_once(pattr, [] {
+            cudaFuncSetAttribute(k_gemm_nvfp4_persistent, cudaFuncAttributeMaxDynamicSharedMemorySize, NP_SMEM_BYTES);
+        });
+        const int64_t n_tiles = tiles * n_mat;
+        const unsigned grid = static_cast<unsigned>(min(n_tiles, static_cast<int64_t>(num_sms())));
+        k_gemm_nvfp4_persistent<<<grid, NP_THREADS, NP_SMEM_BYTES, st>>>(amap, bmap, ymap, a,
+                                                                         static_cast<int>(tiles_n), n_tiles);
+        return check_launch("tq_gemm_nvfp4");
+    }
     static std::once_flag attr;
     std::call_once(attr, [] {
         cudaFuncSetAttribute(k_gemm_nvfp4<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
     });
     k_gemm_nvfp4<BN><<<dim3(static_cast<unsigned>(tiles), static_cast<unsigned>(n_mat)), NG_THREADS, C::SMEM_BYTES,
-                   reinterpret_cast<cudaStream_t>(stream)>>>(amap, bmap, ymap, a);
+                   st>>>(amap, bmap, ymap, a);
     return check_launch("tq_gemm_nvfp4");
 }
