@@ -449,7 +449,7 @@ k_gemm_nvfp4(const __grid_constant__ CUtensorMap amap, const __grid_constant__ C
 // accumulator (MMAs complete, tcgen05.commit) and acc_empty per accumulator
 // (the 128 epilogue threads have read it).
 // The persistent form (true) or one CTA per tile (false).
-constexpr bool NG_PERSISTENT = true;
+constexpr bool NG_PERSISTENT = false;
 constexpr int NP_STAGES = 4;
 constexpr int NP_THREADS = 192;
 constexpr int NP_B_BYTES = 128 * NG_BKB;

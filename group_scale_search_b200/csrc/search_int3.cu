@@ -204,7 +204,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float2 ns1 = make_float2(-s1, -s1), inv1 = make_float2(i1, i1);
         float2 accC = make_float2(0.f, 0.f), accD = make_float2(0.f, 0.f);
         float2 accP = make_float2(0.f, 0.f), accN = make_float2(0.f, 0.f);
-#pragma unroll 2
+#pragma unroll 4
         for (int j = 0; j < (ns_pad >> 2); ++j) {   // two independent accumulator chains
             const float4 w4 = spw[j], m4 = spm[j];
             accC = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns1, inv1, accC);
@@ -256,7 +256,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
         const float2 ns2 = make_float2(-s2, -s2), inv2 = make_float2(i2, i2);
         float2 a2 = make_float2(0.f, 0.f), a2b = make_float2(0.f, 0.f);
-#pragma unroll 2
+#pragma unroll 4
         for (int j = 0; j < (ns_pad >> 2); ++j) {
             const float4 w4 = spw[j], m4 = spm[j];
             a2 = err_free2(make_float2(w4.x, w4.y), make_float2(m4.x, m4.y), ns2, inv2, a2);
