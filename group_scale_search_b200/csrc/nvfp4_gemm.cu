@@ -454,7 +454,10 @@ constexpr int NP_STAGES = 4;
 constexpr int NP_THREADS = 192;
 constexpr int NP_B_BYTES = 128 * NG_BKB;
 constexpr int NP_STAGE_BYTES = NG_A_BYTES + NP_B_BYTES + NG_SFA_BYTES + 2048;
-constexpr int NP_OUT_BYTES = 128 * 128 * 4;                      // one fp32 output tile
+// The output tile leaves through a shared-memory staging tile by TMA stores
+// (true) or straight from registers (false: more ring stages fit).
+constexpr bool NP_STAGED = true;
+constexpr int NP_OUT_BYTES = NP_STAGED ? 128 * 128 * 4 : 0;      // one fp32 output tile
 constexpr int NP_SMEM_BYTES = NP_STAGES * NP_STAGE_BYTES + NP_OUT_BYTES + 1024 + 256;
 constexpr uint32_t NP_SF_COL = 256, NP_SF_COLS = 32;           // per k-step parity: A 4 x 4, B 4 x 4
 constexpr uint32_t NP_IDESC = NgCfg<128>::IDESC;
@@ -577,7 +580,7 @@ k_gemm_nvfp4_persistent(const __grid_constant__ CUtensorMap amap, const __grid_c
             tile_of(t, e, tm, tn);
             const float gg = __fmul_rn(__ldg(a.gx + e), __ldg(a.gw + e));
             const uint32_t acc = tmem + 128u * static_cast<uint32_t>(b) + (static_cast<uint32_t>(quarter * 32) << 16);
-            if (a.y_tma) {
+            if (NP_STAGED && a.y_tma) {
                 if (threadIdx.x == 64) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
                 ng_named_sync(1, 128);   // the previous tile's stores have read the staging tile
 #pragma unroll 1
