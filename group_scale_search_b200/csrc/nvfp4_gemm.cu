@@ -74,12 +74,16 @@ __device__ __forceinline__ int e4m3_floor(float t) {
 // The positive finite E4M3 code (1..126) nearest t = b / (6 g) by the exact
 // distance d(c) = |6 g dec(c) - b| (fp64: 6 g dec(c) has at most 31
 // significant bits), ties to the lower code.  The nearest code is the floor
-// code of the exact t or the next one; the fp32 estimate of t is within one
-// code of that floor, so the four codes around it hold the answer, compared
-// in ascending order with strict improvement.
-__device__ __forceinline__ int nearest_e4m3_code(float b, float g) {
+// code of the exact t or the next one; an fp32 estimate of t within a few
+// ulps (b times the approximate reciprocal inv6g of 6 g) is within one code
+// of that floor (E4M3 codes are at least 2^-3 apart relatively), so the four
+// codes around it hold the answer, compared in ascending order with strict
+// improvement.  inv6g = 0 (6 g outside the range where the approximate
+// reciprocal is accurate) takes the IEEE quotient instead.
+__device__ __forceinline__ int nearest_e4m3_code(float b, float g, float inv6g) {
     const double g6 = 6.0 * static_cast<double>(g), bd = static_cast<double>(b);
-    const int c0 = max(1, min(123, e4m3_floor(__fdiv_rn(b, __fmul_rn(6.f, g))) - 1));
+    const float t = inv6g != 0.f ? __fmul_rn(b, inv6g) : __fdiv_rn(b, __fmul_rn(6.f, g));
+    const int c0 = max(1, min(123, e4m3_floor(t) - 1));
     int best = c0;
     double bdist = fabs(__dsub_rn(__dmul_rn(g6, static_cast<double>(e4m3_value(c0))), bd));
 #pragma unroll
@@ -117,7 +121,9 @@ k_quant_act_nvfp4(const T* __restrict__ X, int64_t I, int64_t ld, int64_t ms, co
 #pragma unroll
         for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(w[i]));
         const float g = __ldg(gs + e);
-        const int code = (g > 0.f && b > 0.f) ? nearest_e4m3_code(b, g) : 0;
+        const float g6f = __fmul_rn(6.f, g);
+        const float inv6g = (g6f > 1e-30f && g6f < 1e30f) ? rcp_approx(g6f) : 0.f;
+        const int code = (g > 0.f && b > 0.f) ? nearest_e4m3_code(b, g, inv6g) : 0;
         const float S = code ? __fmul_rn(g, e4m3_value(static_cast<unsigned>(code))) : 0.f;
         uint32_t pk[2];
         nvfp4_rtn<16>(w, S, pk);
