@@ -182,3 +182,17 @@ def test_gemm_deterministic_and_refusals():
     assert np.all(np.abs(yy - yy.T) <= 2 * bound + 2.0 ** -22 * np.abs(yy))
     with pytest.raises(tq.TQError):
         tq.tq_gemm_nvfp4(act.packed, xs, act.global_scale, act.packed, xs, act.global_scale, E, T, T, 48)
+
+
+@pytest.mark.parametrize("mag", [1e-36, 1e-20, 1e20])
+def test_quant_act_extreme_magnitudes(mag):
+    """Tiny (a subnormal global scale), small and huge activations: the
+    nearest-code estimate switches to the IEEE quotient where the
+    approximate reciprocal is not accurate; the result stays bit-exact."""
+    X = (_acts(2, 33, 256, seed=9, dtype=torch.float32) * mag).contiguous()
+    r = tq.tq_quant_nvfp4_act(X)
+    tq.tq_sync()
+    g, sc, c, rec = _oracle_quant(host32(X))
+    assert np.array_equal(r.global_scale.cpu().numpy(), g)
+    assert np.array_equal(r.scales.cpu().numpy(), sc)
+    assert np.array_equal(r.packed.cpu().numpy().reshape(2, -1), rec.reshape(2, -1))
