@@ -217,49 +217,76 @@ __global__ void k_imatrix_final(const double* __restrict__ partial, int64_t slic
 
 // ------------------------------------------------------------------ amax
 
+// One warp per row at a time (warps of all blocks interleaved over the
+// matrix's rows), each lane with 4 16-byte loads in flight; the blocks of
+// one matrix are sized to fill one wave of resident blocks.
+constexpr int AM_THREADS = 256;
+
 template <typename T>
-__global__ void k_amax(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms,
-                       unsigned* __restrict__ amax) {
+__global__ void __launch_bounds__(AM_THREADS)
+k_amax(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, unsigned* __restrict__ amax) {
     constexpr int VEC = VecOf<T>::n;
     const int64_t e = blockIdx.y;
     const T* base = W + e * ms;
+    const int lane = threadIdx.x & 31;
+    const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (AM_THREADS / 32);
+    const int64_t nvec = I / VEC;   // whole 16-byte vectors per row (rows start 16-byte aligned)
     float mx = 0.f;
-    for (int64_t r = blockIdx.x; r < O; r += gridDim.x) {
+    for (int64_t r = static_cast<int64_t>(blockIdx.x) * (AM_THREADS / 32) + (threadIdx.x >> 5); r < O; r += nwarps) {
         const T* row = base + r * ld;
-        for (int64_t c = static_cast<int64_t>(threadIdx.x) * VEC; c < I; c += static_cast<int64_t>(blockDim.x) * VEC) {
-            if (c + VEC <= I) {
+        int64_t c = lane;
+        for (; c + 96 < nvec; c += 128) {
+            uint4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = __ldg(reinterpret_cast<const uint4*>(row + (c + 32 * q) * VEC));
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
                 float x[VEC];
-                load_vec<T>(row + c, x);
+                unpack_vec<T>(v[q], x);
 #pragma unroll
                 for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(x[i]));
-            } else {
-                for (int64_t i = c; i < I; ++i) mx = fmaxf(mx, fabsf(Elem<T>::load(row + i)));
             }
         }
+        for (; c < nvec; c += 32) {
+            float x[VEC];
+            load_vec<T>(row + c * VEC, x);
+#pragma unroll
+            for (int i = 0; i < VEC; ++i) mx = fmaxf(mx, fabsf(x[i]));
+        }
+        for (int64_t i = nvec * VEC + lane; i < I; i += 32) mx = fmaxf(mx, fabsf(Elem<T>::load(row + i)));
     }
     unsigned u = __reduce_max_sync(FULL, __float_as_uint(mx));
-    __shared__ unsigned wmax[32];
-    if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = u;
+    __shared__ unsigned wmax[AM_THREADS / 32];
+    if (lane == 0) wmax[threadIdx.x >> 5] = u;
     __syncthreads();
     if (threadIdx.x < 32) {
-        unsigned v = threadIdx.x < (blockDim.x >> 5) ? wmax[threadIdx.x] : 0u;
+        unsigned v = threadIdx.x < AM_THREADS / 32 ? wmax[threadIdx.x] : 0u;
         v = __reduce_max_sync(FULL, v);
         if (threadIdx.x == 0) atomicMax(amax + e, v);   // non-negative floats order like their bits
     }
 }
 
 tq_status launch_amax(const tq_mat* W, float* amax, cudaStream_t st) {
+    TQ_REQUIRE(W->n_mat <= 65535, "amax: more than 65535 matrices in one call");
     cudaError_t ce = cudaMemsetAsync(amax, 0, static_cast<size_t>(W->n_mat) * sizeof(float), st);
     if (ce != cudaSuccess) return set_error(TQ_ERR_CUDA, "amax: %s", cudaGetErrorString(ce));
-    const int64_t per = max(static_cast<int64_t>(1), static_cast<int64_t>(num_sms()) * 4 / W->n_mat);
-    const dim3 grid(static_cast<unsigned>(min(per, W->rows)), static_cast<unsigned>(W->n_mat));
+    int per_sm = 0;
+    const bool bf = W->dtype == TQ_BF16;
+    if ((bf ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_amax<uint16_t>, AM_THREADS, 0)
+            : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_amax<float>, AM_THREADS, 0)) != cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
+    const int64_t per = max(static_cast<int64_t>(1), slots / W->n_mat);   // blocks per matrix
+    const int64_t need = (W->rows + AM_THREADS / 32 - 1) / (AM_THREADS / 32);   // one row per warp at most
+    const dim3 grid(static_cast<unsigned>(min(per, need)), static_cast<unsigned>(W->n_mat));
     const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
-    if (W->dtype == TQ_BF16)
-        k_amax<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->rows, W->cols, W->ld, ms,
-                                              reinterpret_cast<unsigned*>(amax));
+    if (bf)
+        k_amax<uint16_t><<<grid, AM_THREADS, 0, st>>>(static_cast<const uint16_t*>(W->ptr), W->rows, W->cols, W->ld,
+                                                      ms, reinterpret_cast<unsigned*>(amax));
     else
-        k_amax<float><<<grid, 256, 0, st>>>(static_cast<const float*>(W->ptr), W->rows, W->cols, W->ld, ms,
-                                           reinterpret_cast<unsigned*>(amax));
+        k_amax<float><<<grid, AM_THREADS, 0, st>>>(static_cast<const float*>(W->ptr), W->rows, W->cols, W->ld, ms,
+                                                   reinterpret_cast<unsigned*>(amax));
     return check_launch("amax");
 }
 

@@ -691,7 +691,17 @@ TQ_API tq_status tq_quant_nvfp4_act(const tq_mat* X, uint8_t* packed, uint8_t* s
     k_act_global<<<static_cast<unsigned>((X->n_mat + 255) / 256), 256, 0, st>>>(global_scale, X->n_mat);
     const GroupIndex gi(X->rows, G);
     const int64_t ms = X->n_mat > 1 ? X->mat_stride : 0;
-    const unsigned grid = static_cast<unsigned>(min((total + 255) / 256, static_cast<int64_t>(num_sms()) * 8));
+    // one wave of resident blocks (a second, partial wave would leave most
+    // SMs idle for its duration)
+    int per_sm = 0;
+    if ((X->dtype == TQ_BF16
+             ? cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_act_nvfp4<uint16_t>, 256, 0)
+             : cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_quant_act_nvfp4<float>, 256, 0)) !=
+            cudaSuccess ||
+        per_sm < 1)
+        per_sm = 1;
+    const unsigned grid =
+        static_cast<unsigned>(min((total + 255) / 256, static_cast<int64_t>(num_sms()) * per_sm));
     if (X->dtype == TQ_BF16)
         k_quant_act_nvfp4<uint16_t><<<grid, 256, 0, st>>>(static_cast<const uint16_t*>(X->ptr), X->cols, X->ld, ms,
                                                           global_scale, gi, total, scales, packed);

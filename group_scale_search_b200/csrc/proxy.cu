@@ -5,33 +5,57 @@
 //
 // B200 mapping (HBM-bound): one thread per two octets (16 consecutive
 // weights of a group, two 16-byte loads of bf16) walking the rows of its
-// slice; its 16 imatrix weights sit in shared memory (read only by it), it
+// block; its 16 imatrix weights sit in shared memory (read only by it), it
 // dequantizes in registers (no What round trip through memory), sums the
-// terms in fp32 and folds them into fp64 per row.  Each block writes an fp64 partial to
-// the workspace; the last block of a matrix (atomic ticket) adds the
-// partials in block order, so the result is deterministic for a given
-// device.
+// terms in fp32 and folds them into fp64 per row.  The blocks split the rows
+// of the whole batch (all matrices' rows in order) evenly, one wave of
+// resident blocks, so every SM is kept busy whatever the matrix count; where
+// a block's rows cross from one matrix to the next it writes the fp64
+// partial of the finished matrix to the workspace, and the last block to
+// finish a matrix (atomic ticket) adds that matrix's partials in block
+// order, so the result is deterministic for a given device.
 #include "walk.cuh"
 
 namespace tq {
 
-// Fixed block budget, so the workspace size (one fp64 pair per block) does
-// not depend on the device.
-constexpr int64_t PX_TARGET_BLOCKS = 148 * 8;
+// Bound on the blocks of one launch (one wave of resident blocks at most),
+// so the workspace size does not depend on the device.
+constexpr int64_t PX_MAX_BLOCKS = 148 * 8;
 
-// Octets per thread (one or two consecutive octets of one group), rows per
-// iteration (all their loads issued before any is used), and whether the
-// thread's imatrix weights sit in shared memory (fewer registers) or in
-// registers.  Measured on the MoE and dense workloads: two octets, one row,
-// weights in shared memory (60-64 registers, 4 blocks of up to 256 threads
-// per SM) beat two rows in flight per thread at 3 blocks per SM.
+// Octets per thread: two consecutive octets of one group (one 16-weight
+// NVFP4 block; half the per-row code and scale loads of one octet).
+// Measured on the MoE and dense workloads: two octets, one row per
+// iteration, imatrix weights in shared memory (60-64 registers, 4 blocks of
+// up to 256 threads per SM) beat two rows in flight per thread at 3 blocks
+// per SM, and beat a private ring of 2-4 rows per thread filled by
+// asynchronous 16-byte copies (0.65 against 0.57 ms on the int3 MoE stack).
 constexpr int PX_NO = 2;
-constexpr int PX_ROWS = 1;
-constexpr bool PX_MSMEM = true;
 
-inline Walk px_geometry(int64_t n_mat, int64_t O, int64_t I) {
-    return walk_geometry(n_mat, O, ((I + 7) / 8 + PX_NO - 1) / PX_NO, PX_TARGET_BLOCKS);
+// Launch geometry: x = unit-column tiles, y = blocks of rpb consecutive rows
+// of the batch.
+struct PxGrid {
+    int64_t width, cblocks, rblocks, rpb;
+};
+
+inline PxGrid px_grid(int64_t n_mat, int64_t O, int64_t I, int64_t max_blocks) {
+    PxGrid f;
+    const Walk w = walk_geometry(1, 1, ((I + 7) / 8 + PX_NO - 1) / PX_NO, 1);
+    f.width = w.width;
+    f.cblocks = w.cblocks;
+    const int64_t n_rows = n_mat * O;
+    int64_t rb = max(static_cast<int64_t>(1), min(max_blocks, PX_MAX_BLOCKS) / f.cblocks);
+    rb = min(rb, min(n_rows, static_cast<int64_t>(65535)));
+    f.rpb = (n_rows + rb - 1) / rb;
+    f.rblocks = (n_rows + f.rpb - 1) / f.rpb;
+    return f;
 }
+
+// Workspace: a ticket per matrix, then an fp64 (num, den) pair per (block
+// row y + matrix e, column tile): the blocks whose rows reach into matrix e
+// are a contiguous run of y, and a later y never reaches an earlier matrix,
+// so (e + y) never repeats between two (block, matrix) pairs of one column
+// tile.
+inline int64_t px_ticket_bytes(int64_t n_mat) { return ((n_mat * 4 + 15) / 16) * 16; }
 
 // Adds the 8 terms of one octet in fp32 (two interleaved partial sums of
 // fp32x2 pairs): m (W - What)^2 and m W^2.
@@ -51,73 +75,65 @@ __device__ __forceinline__ void px_terms(const float w[8], const float v[8], con
 }
 
 template <int FMT, typename T, int NO>
-__global__ void __launch_bounds__(256, NO == 1 || PX_MSMEM ? 4 : 3)
+__global__ void __launch_bounds__(256, 4)
 k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, const uint8_t* __restrict__ packed,
         const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
-        const float* __restrict__ m, int64_t m_stride, int64_t rps, double* __restrict__ part_out,
+        const float* __restrict__ m, int64_t m_stride, int64_t n_rows, int64_t rpb, double* __restrict__ part,
         unsigned* __restrict__ tickets, double* __restrict__ num, double* __restrict__ den) {
     using F = FmtTraits<FMT>;
     const int64_t G = (I + F::group - 1) / F::group;
     const int64_t C = (I + 7) >> 3;
-    const int64_t e = blockIdx.z;
+    const int64_t cb = gridDim.x, y = blockIdx.y;
     const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    const int64_t nblk = static_cast<int64_t>(gridDim.x) * gridDim.y;
-    const int64_t bid = static_cast<int64_t>(blockIdx.y) * gridDim.x + blockIdx.x;
+    const bool active = u < (C + NO - 1) / NO;
     const int nwarps = static_cast<int>(blockDim.x >> 5);
-    __shared__ float4 msm[PX_MSMEM ? 2 * NO : 1][PX_MSMEM ? 256 : 1];
-    double an = 0.0, ad = 0.0;
-    if (u < (C + NO - 1) / NO) {
-        const int64_t c = u * NO;
-        const int64_t k = c >> F::lg;
-        const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
-        const int64_t j = c << 3;
-        int n[NO];
-        [[maybe_unused]] float mreg[PX_MSMEM ? 1 : NO][8];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    __shared__ float4 msm[2 * NO][256];
+    __shared__ double sw[2][8];
+    __shared__ bool last;
+    const int64_t c = u * NO;
+    const int64_t k = c >> F::lg;
+    const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
+    const int64_t j = c << 3;
+    int n[NO];
 #pragma unroll
-        for (int i = 0; i < NO; ++i) {
-            n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
-            Oct<float> mo;
-            mo.load(m + e * m_stride + j + 8 * i, n[i]);
-            if constexpr (PX_MSMEM) {
-                msm[2 * i][threadIdx.x] = mo.a;
-                msm[2 * i + 1][threadIdx.x] = mo.b;
-            } else {
-                mo.get(mreg[i]);
-            }
-        }
-        const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
-        const int64_t o0 = static_cast<int64_t>(blockIdx.y) * rps, o1 = min(O, o0 + rps);
-        const T* wp = W + e * ms + o0 * ld + j;
-        QPtr<FMT> qp(packed, scales, zeros, (e * O + o0) * G + k, G);
-        for (int64_t o = o0; o < o1; o += PX_ROWS, wp += PX_ROWS * ld) {
-            Oct<T> rw[PX_ROWS][NO];
-            UnitQ<NO> q[PX_ROWS];
+    for (int i = 0; i < NO; ++i)
+        n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
+    int64_t r = y * rpb;
+    const int64_t r1 = min(n_rows, r + rpb);
+    int64_t e = r / O;
+    const T* wp = W + e * ms + (r - e * O) * ld + j;
+    QPtr<FMT> qp(packed, scales, zeros, r * G + k, G);
+    bool first = true;
+    while (r < r1) {   // the block's rows of matrix e: [r, seg_end); the same for every thread
+        const int64_t seg_end = min(r1, (e + 1) * O);
+        double an = 0.0, ad = 0.0;
+        if (active) {
+            if (first || m_stride != 0) {
 #pragma unroll
-            for (int h = 0; h < PX_ROWS; ++h) {
-                if (o + h < o1) {
-#pragma unroll
-                    for (int i = 0; i < NO; ++i) rw[h][i].load(wp + h * ld + 8 * i, n[i]);
-                    q[h] = load_unit_q<FMT, NO>(qp, oct);
+                for (int i = 0; i < NO; ++i) {
+                    Oct<float> mo;
+                    mo.load(m + e * m_stride + j + 8 * i, n[i]);
+                    msm[2 * i][threadIdx.x] = mo.a;   // read back by this thread only
+                    msm[2 * i + 1][threadIdx.x] = mo.b;
                 }
-                qp.next();
             }
+            const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
+            for (int64_t o = r; o < seg_end; ++o, wp += ld) {
+                Oct<T> rw[NO];
 #pragma unroll
-            for (int h = 0; h < PX_ROWS; ++h) {
-                if (o + h >= o1) break;
+                for (int i = 0; i < NO; ++i) rw[i].load(wp + 8 * i, n[i]);
+                const UnitQ<NO> q = load_unit_q<FMT, NO>(qp, oct);
+                qp.next();
                 float sn = 0.f, sd = 0.f;
 #pragma unroll
                 for (int i = 0; i < NO; ++i) {
                     float w[8], v[8], mm[8], tn, td;
-                    rw[h][i].get(w);
-                    dec_oct<FMT>(OctQ{q[h].bits[i], q[h].s, q[h].z}, g, v);
-                    if constexpr (PX_MSMEM) {
-                        const float4 a = msm[2 * i][threadIdx.x], b = msm[2 * i + 1][threadIdx.x];
-                        mm[0] = a.x; mm[1] = a.y; mm[2] = a.z; mm[3] = a.w;
-                        mm[4] = b.x; mm[5] = b.y; mm[6] = b.z; mm[7] = b.w;
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < 8; ++t) mm[t] = mreg[i][t];
-                    }
+                    rw[i].get(w);
+                    dec_oct<FMT>(OctQ{q.bits[i], q.s, q.z}, g, v);
+                    const float4 a = msm[2 * i][threadIdx.x], b = msm[2 * i + 1][threadIdx.x];
+                    mm[0] = a.x; mm[1] = a.y; mm[2] = a.z; mm[3] = a.w;
+                    mm[4] = b.x; mm[5] = b.y; mm[6] = b.z; mm[7] = b.w;
                     px_terms(w, v, mm, tn, td);
                     sn = __fadd_rn(sn, tn);
                     sd = __fadd_rn(sd, td);
@@ -126,70 +142,73 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
                 ad += static_cast<double>(sd);
             }
         }
-    }
-    // block reduction in fp64, fixed order
-#pragma unroll
-    for (int off = 16; off; off >>= 1) {
-        an += __shfl_xor_sync(FULL, an, off);
-        ad += __shfl_xor_sync(FULL, ad, off);
-    }
-    __shared__ double sw[2][8];
-    __shared__ bool last;
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    if (lane == 0) { sw[0][wid] = an; sw[1][wid] = ad; }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double bn = 0.0, bd = 0.0;
-        for (int i = 0; i < nwarps; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
-        part_out[(e * nblk + bid) * 2] = bn;
-        part_out[(e * nblk + bid) * 2 + 1] = bd;
-        __threadfence();
-        last = atomicAdd(tickets + e, 1u) == static_cast<unsigned>(nblk - 1);
-    }
-    __syncthreads();
-    if (last) {   // the matrix's last block adds the partials: fixed strides, fixed tree
-        __threadfence();
-        double tn = 0.0, td = 0.0;
-        for (int64_t b = threadIdx.x; b < nblk; b += blockDim.x) {
-            tn += __ldcg(part_out + (e * nblk + b) * 2);
-            td += __ldcg(part_out + (e * nblk + b) * 2 + 1);
-        }
+        // the block's partial of matrix e, in fp64, fixed order
 #pragma unroll
         for (int off = 16; off; off >>= 1) {
-            tn += __shfl_xor_sync(FULL, tn, off);
-            td += __shfl_xor_sync(FULL, td, off);
+            an += __shfl_xor_sync(FULL, an, off);
+            ad += __shfl_xor_sync(FULL, ad, off);
         }
+        if (lane == 0) { sw[0][wid] = an; sw[1][wid] = ad; }
         __syncthreads();
-        if (lane == 0) { sw[0][wid] = tn; sw[1][wid] = td; }
-        __syncthreads();
+        // blocks (all column tiles) whose rows reach into matrix e
+        const int64_t ylo = (e * O) / rpb, yhi = ((e + 1) * O - 1) / rpb;
         if (threadIdx.x == 0) {
             double bn = 0.0, bd = 0.0;
             for (int i = 0; i < nwarps; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
-            num[e] = bn;
-            den[e] = bd;
+            part[((e + y) * cb + blockIdx.x) * 2] = bn;
+            part[((e + y) * cb + blockIdx.x) * 2 + 1] = bd;
+            __threadfence();
+            last = atomicAdd(tickets + e, 1u) == static_cast<unsigned>((yhi - ylo + 1) * cb - 1);
         }
+        __syncthreads();
+        if (last) {   // the matrix's last block adds its partials: y ascending, then column tiles
+            __threadfence();
+            const int64_t np = (yhi - ylo + 1) * cb;
+            double tn = 0.0, td = 0.0;
+            for (int64_t t = threadIdx.x; t < np; t += blockDim.x) {
+                const int64_t idx = (e + ylo) * cb + t;   // (e + yy) * cb + x with yy = ylo + t / cb, x = t % cb
+                tn += __ldcg(part + idx * 2);
+                td += __ldcg(part + idx * 2 + 1);
+            }
+#pragma unroll
+            for (int off = 16; off; off >>= 1) {
+                tn += __shfl_xor_sync(FULL, tn, off);
+                td += __shfl_xor_sync(FULL, td, off);
+            }
+            __syncthreads();
+            if (lane == 0) { sw[0][wid] = tn; sw[1][wid] = td; }
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                double bn = 0.0, bd = 0.0;
+                for (int i = 0; i < nwarps; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
+                num[e] = bn;
+                den[e] = bd;
+            }
+        }
+        __syncthreads();   // sw and `last` are reused by the next matrix
+        r = seg_end;
+        ++e;
+        wp = W + e * ms + j;
+        first = false;
     }
 }
 
-// At most one wave of resident blocks (slices per matrix rounded down, so no
-// second partial wave) and at most the block count the workspace is sized
-// for (PX_TARGET_BLOCKS, rounded up: never fewer slots than blocks).
+// One wave of resident blocks at most (and at most PX_MAX_BLOCKS, the count
+// the workspace is sized for).
 template <int FMT, typename T>
 void launch_proxy(const tq_mat* W, int64_t ms, const uint8_t* packed, const void* scales, const uint8_t* zeros,
                   const float* gs, const float* m, int64_t mst, double* parts, unsigned* tickets, double* num,
                   double* den, cudaStream_t st) {
-    const int64_t cols = ((W->cols + 7) / 8 + PX_NO - 1) / PX_NO;
-    Walk pg = walk_geometry(W->n_mat, W->rows, cols, 1);
+    const int width = static_cast<int>(px_grid(1, 1, W->cols, 1).width);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T, PX_NO>, static_cast<int>(pg.width), 0) !=
-            cudaSuccess || per_sm < 1)
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T, PX_NO>, width, 0) != cudaSuccess ||
+        per_sm < 1)
         per_sm = 1;
-    pg = walk_geometry(W->n_mat, W->rows, cols, min(PX_TARGET_BLOCKS, static_cast<int64_t>(num_sms()) * per_sm),
-                       false);
-    const dim3 grid(static_cast<unsigned>(pg.cblocks), static_cast<unsigned>(pg.slices), static_cast<unsigned>(W->n_mat));
-    k_proxy<FMT, T, PX_NO><<<grid, static_cast<unsigned>(pg.width), 0, st>>>(
-        static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, packed, scales, zeros, gs, m, mst, pg.rps, parts,
-        tickets, num, den);
+    const PxGrid f = px_grid(W->n_mat, W->rows, W->cols, static_cast<int64_t>(num_sms()) * per_sm);
+    const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
+    k_proxy<FMT, T, PX_NO><<<grid, static_cast<unsigned>(f.width), 0, st>>>(
+        static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, packed, scales, zeros, gs, m, mst,
+        W->n_mat * W->rows, f.rpb, parts, tickets, num, den);
 }
 
 }  // namespace tq
@@ -199,9 +218,8 @@ using namespace tq;
 TQ_API size_t tq_proxy_workspace_bytes(const tq_mat* W, int32_t fmt) {
     const int64_t g = group_of(fmt);
     if (!W || g == 0 || W->n_mat < 1 || W->rows < 1 || W->cols < 1) return 0;
-    const Walk pg = px_geometry(W->n_mat, W->rows, W->cols);
-    const int64_t tick = ((W->n_mat * 4 + 15) / 16) * 16;
-    return static_cast<size_t>(tick + W->n_mat * pg.cblocks * pg.slices * 16);
+    const PxGrid f = px_grid(W->n_mat, W->rows, W->cols, PX_MAX_BLOCKS);   // the most block rows of any launch
+    return static_cast<size_t>(px_ticket_bytes(W->n_mat) + (W->n_mat + f.rblocks) * f.cblocks * 16);
 }
 
 TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, const void* scales,
@@ -223,8 +241,7 @@ TQ_API tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t 
     const size_t need = tq_proxy_workspace_bytes(W, fmt);
     TQ_REQUIRE(workspace_bytes >= need, "tq_proxy_error: workspace too small (%zu < %zu)", workspace_bytes, need);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    TQ_REQUIRE(W->n_mat <= 65535, "tq_proxy_error: more than 65535 matrices in one call");
-    const int64_t tick = ((W->n_mat * 4 + 15) / 16) * 16;
+    const int64_t tick = px_ticket_bytes(W->n_mat);
     unsigned* tickets = static_cast<unsigned*>(workspace);
     double* parts = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + tick);
     cudaError_t ce = cudaMemsetAsync(tickets, 0, static_cast<size_t>(W->n_mat) * 4, st);
