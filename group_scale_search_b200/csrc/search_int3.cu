@@ -18,7 +18,7 @@
 // half to even is odd-symmetric), so stage 1 evaluates them once per
 // magnitude and only the few large elements per sign.  Candidates are ranked
 // in fp32 with the multiply-by-reciprocal rounding; all candidates within a
-// relative 2^-15 of the best are re-evaluated in fp64 with codes from the IEEE
+// relative 2^-16 of the best are re-evaluated in fp64 with codes from the IEEE
 // quotient, which decides the winner exactly as the definition does.
 #include "group_pack.cuh"
 
@@ -26,8 +26,22 @@
 
 namespace tq {
 
-constexpr int SYM_WARPS = 8;
-constexpr float WIN = 3.0517578125e-05f;   // 2^-15: bound on fp32 ranking error x 2 (with margin)
+constexpr int SYM_WARPS = 32;
+// Ranking window.  A candidate's fp32 loss is within eps of its exact loss,
+// relative: the reciprocal (one Newton step on rcp.approx) is within 2^-24 of
+// 1/s, so a code differs from the IEEE quotient's only where y = w/s lies
+// within |y| 2^-23 <= 4.5 2^-23 of a half-integer, which moves that element's
+// term by at most 8 x 4.5 2^-23 = 2^-17.8 of itself; the fp32 sums (chains of
+// at most 35 additions, 3 roundings per term) add at most 38 2^-24 = 2^-18.75.
+// eps <= 2^-17.2, and a candidate the fp32 order could misplace is within
+// (1 + eps) / (1 - eps) - 1 <= 2^-16.2 of the fp32 best: WIN = 2^-16 covers it.
+constexpr float WIN = 1.52587890625e-05f;   // 2^-16
+
+// 1/s to within 2^-24 (relative): rcp.approx refined by one Newton step.
+__device__ __forceinline__ float rcp_refined(float s) {
+    const float r = rcp_approx(s);
+    return __fmaf_rn(r, __fmaf_rn(-s, r, 1.f), r);
+}
 
 struct SymArgs {
     const void* W;
@@ -200,7 +214,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         // ---- stage 1: lane = magnitude, both signs
         const float s1 = __fmul_rn(__fmul_rn(r1v, Ms), 0.25f);    // scaled candidate
         const float s1o = __fmul_rn(__fmul_rn(r1v, M), 0.25f);    // the candidate itself
-        const float i1 = rcp_approx(s1);
+        const float i1 = rcp_refined(s1);
         const float2 ns1 = make_float2(-s1, -s1), inv1 = make_float2(i1, i1);
         float2 accC = make_float2(0.f, 0.f), accD = make_float2(0.f, 0.f);
         float2 accP = make_float2(0.f, 0.f), accN = make_float2(0.f, 0.f);
@@ -252,7 +266,7 @@ k_search_int3(const __grid_constant__ SymArgs a) {
         const float r2v = r2s[ks * 32 + (act2 ? lane : 0)];
         const float s2 = __fmul_rn(__fmul_rn(r2v, Ms), 0.25f);
         const float s2o = __fmul_rn(__fmul_rn(r2v, M), 0.25f);
-        const float i2 = rcp_approx(s2);
+        const float i2 = rcp_refined(s2);
         const float clo = sg ? MAGIC - 3.f : MAGIC - 4.f, chi = sg ? MAGIC + 4.f : MAGIC + 3.f;
         const float2 ns2 = make_float2(-s2, -s2), inv2 = make_float2(i2, i2);
         float2 a2 = make_float2(0.f, 0.f), a2b = make_float2(0.f, 0.f);
