@@ -238,7 +238,7 @@ class Step:
         for u, fmt in zip(self.units, self.fmts):
             E, O, I = u.W.shape
             m = self._m_for(u)
-            self.res.append(tq.tq_search_groups(u.W, m, fmt, want_idx=False, want_loss=False))
+            self.res.append(tq.search_result_empty(u.W, fmt, want_idx=False, want_loss=False))
             self.dq.append(torch.empty((E, O, I), dtype=torch.bfloat16, device=dev))
             self.px.append((torch.empty(E, dtype=torch.float64, device=dev),
                             torch.empty(E, dtype=torch.float64, device=dev)))

@@ -30,7 +30,7 @@ import torch
 
 __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "INT4_G32_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
-    "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes",
+    "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes", "search_result_empty",
     "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
     "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
     "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_debug_set_wait_limit", "tq_selftest_e2m1",
@@ -456,6 +456,24 @@ def tq_amax(W: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) ->
     return out
 
 
+def search_result_empty(W: torch.Tensor, fmt: int, pack: bool = True, want_idx: bool = True,
+                        want_loss: bool = True) -> SearchResult:
+    """Uninitialised outputs of tq_search_groups for W and fmt (for callers
+    that preallocate: pass the result as `out`)."""
+    E, O, I, G = _groups(W, fmt)
+    dev = W.device
+    sdt = torch.uint8 if fmt == NVFP4_G16 else torch.float32
+    return SearchResult(
+        fmt=fmt,
+        scales=torch.empty((E, O, G), dtype=sdt, device=dev),
+        zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt in _INT4 else None,
+        global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
+        cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
+        loss=torch.empty((E, O, G), dtype=torch.float64, device=dev) if want_loss else None,
+        packed=torch.empty(tq_packed_bytes(fmt, E * O, I), dtype=torch.uint8, device=dev) if pack else None,
+    )
+
+
 def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optional[SearchParams] = None,
                      pack: bool = True, want_idx: bool = True, want_loss: bool = True,
                      out: Optional[SearchResult] = None, stream=None) -> SearchResult:
@@ -464,19 +482,8 @@ def tq_search_groups(W: torch.Tensor, m: torch.Tensor, fmt: int, params: Optiona
     m: [I] (shared) or [n_mat, I] fp32 imatrix."""
     d = _mat(W, "W")
     _check_m(m, d.n_mat, d.cols)
-    E, O, I, G = _groups(W, fmt)
-    dev = W.device
     if out is None:
-        sdt = torch.uint8 if fmt == NVFP4_G16 else torch.float32
-        out = SearchResult(
-            fmt=fmt,
-            scales=torch.empty((E, O, G), dtype=sdt, device=dev),
-            zeros=torch.empty((E, O, G), dtype=torch.uint8, device=dev) if fmt in _INT4 else None,
-            global_scale=torch.empty(E, dtype=torch.float32, device=dev) if fmt == NVFP4_G16 else None,
-            cand_idx=torch.empty((E, O, G), dtype=torch.int32, device=dev) if want_idx else None,
-            loss=torch.empty((E, O, G), dtype=torch.float64, device=dev) if want_loss else None,
-            packed=torch.empty(tq_packed_bytes(fmt, E * O, I), dtype=torch.uint8, device=dev) if pack else None,
-        )
+        out = search_result_empty(W, fmt, pack, want_idx, want_loss)
     p = (params or SearchParams())._c()
     _check(lib().tq_search_groups(ctypes.byref(d), _ptr(m), _m_stride(m), fmt, ctypes.byref(p),
                                   _ptr(out.scales), _ptr(out.zeros), _ptr(out.global_scale),

@@ -135,6 +135,11 @@ class _HostStandIn:
         m.copy_((X.double().square().sum(dim=1) * alpha).float())
         return m
 
+    def search_result_empty(self, W, fmt, want_idx=True, want_loss=True):
+        E, O, I = W.shape
+        G = -(-I // self.GROUP[fmt])
+        return self.Result(torch.empty((E, O, G), dtype=torch.float32))
+
     def tq_search_groups(self, W, m, fmt, want_idx=True, want_loss=True, out=None):
         E, O, I = W.shape
         g = self.GROUP[fmt]
