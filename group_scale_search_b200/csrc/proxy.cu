@@ -30,6 +30,12 @@ constexpr int64_t PX_MAX_BLOCKS = 148 * 8;
 // per SM, and beat a private ring of 2-4 rows per thread filled by
 // asynchronous 16-byte copies (0.65 against 0.57 ms on the int3 MoE stack).
 constexpr int PX_NO = 2;
+// Row walkers per block (blockDim.y): they share the block's columns (and
+// its imatrix weights in shared memory) and take interleaved rows.
+// Measured on the full-size workloads: one block of four walkers per SM
+// beat four one-walker blocks (0.550 -> 0.486 ms on the int3 MoE stack,
+// 0.027 -> 0.026 ms on the dense q projection, even on the NVFP4 stack).
+constexpr int PX_PY = 4;
 
 // Launch geometry: x = unit-column tiles, y = blocks of rpb consecutive rows
 // of the batch.
@@ -75,7 +81,7 @@ __device__ __forceinline__ void px_terms(const float w[8], const float v[8], con
 }
 
 template <int FMT, typename T, int NO>
-__global__ void __launch_bounds__(256, 4)
+__global__ void __launch_bounds__(256 * PX_PY, 4 / PX_PY)
 k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, const uint8_t* __restrict__ packed,
         const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
         const float* __restrict__ m, int64_t m_stride, int64_t n_rows, int64_t rpb, double* __restrict__ part,
@@ -86,10 +92,13 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
     const int64_t cb = gridDim.x, y = blockIdx.y;
     const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
     const bool active = u < (C + NO - 1) / NO;
-    const int nwarps = static_cast<int>(blockDim.x >> 5);
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int nthreads = static_cast<int>(blockDim.x * blockDim.y);
+    const int tid = static_cast<int>(threadIdx.y * blockDim.x + threadIdx.x);
+    const int nwarps = nthreads >> 5;   // blockDim.x is a multiple of 32
+    const int lane = tid & 31, wid = tid >> 5;
+    const int64_t py = blockDim.y, ty = threadIdx.y;
     __shared__ float4 msm[2 * NO][256];
-    __shared__ double sw[2][8];
+    __shared__ double sw[2][32];
     __shared__ bool last;
     const int64_t c = u * NO;
     const int64_t k = c >> F::lg;
@@ -102,29 +111,31 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
     int64_t r = y * rpb;
     const int64_t r1 = min(n_rows, r + rpb);
     int64_t e = r / O;
-    const T* wp = W + e * ms + (r - e * O) * ld + j;
-    QPtr<FMT> qp(packed, scales, zeros, r * G + k, G);
     bool first = true;
     while (r < r1) {   // the block's rows of matrix e: [r, seg_end); the same for every thread
         const int64_t seg_end = min(r1, (e + 1) * O);
+        if (active && ty == 0 && (first || m_stride != 0)) {
+#pragma unroll
+            for (int i = 0; i < NO; ++i) {
+                Oct<float> mo;
+                mo.load(m + e * m_stride + j + 8 * i, n[i]);
+                msm[2 * i][threadIdx.x] = mo.a;   // read by the column's walkers
+                msm[2 * i + 1][threadIdx.x] = mo.b;
+            }
+        }
+        __syncthreads();
         double an = 0.0, ad = 0.0;
         if (active) {
-            if (first || m_stride != 0) {
-#pragma unroll
-                for (int i = 0; i < NO; ++i) {
-                    Oct<float> mo;
-                    mo.load(m + e * m_stride + j + 8 * i, n[i]);
-                    msm[2 * i][threadIdx.x] = mo.a;   // read back by this thread only
-                    msm[2 * i + 1][threadIdx.x] = mo.b;
-                }
-            }
             const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
-            for (int64_t o = r; o < seg_end; ++o, wp += ld) {
+            // this walker's rows: r + ty, r + ty + py, ...
+            const T* wp = W + e * ms + (r + ty - e * O) * ld + j;
+            QPtr<FMT> qp(packed, scales, zeros, (r + ty) * G + k, G);
+            for (int64_t o = r + ty; o < seg_end; o += py, wp += py * ld) {
                 Oct<T> rw[NO];
 #pragma unroll
                 for (int i = 0; i < NO; ++i) rw[i].load(wp + 8 * i, n[i]);
                 const UnitQ<NO> q = load_unit_q<FMT, NO>(qp, oct);
-                qp.next();
+                qp.skip(py);
                 float sn = 0.f, sd = 0.f;
 #pragma unroll
                 for (int i = 0; i < NO; ++i) {
@@ -152,7 +163,7 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
         __syncthreads();
         // blocks (all column tiles) whose rows reach into matrix e
         const int64_t ylo = (e * O) / rpb, yhi = ((e + 1) * O - 1) / rpb;
-        if (threadIdx.x == 0) {
+        if (tid == 0) {
             double bn = 0.0, bd = 0.0;
             for (int i = 0; i < nwarps; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
             part[((e + y) * cb + blockIdx.x) * 2] = bn;
@@ -165,7 +176,7 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
             __threadfence();
             const int64_t np = (yhi - ylo + 1) * cb;
             double tn = 0.0, td = 0.0;
-            for (int64_t t = threadIdx.x; t < np; t += blockDim.x) {
+            for (int64_t t = tid; t < np; t += nthreads) {
                 const int64_t idx = (e + ylo) * cb + t;   // (e + yy) * cb + x with yy = ylo + t / cb, x = t % cb
                 tn += __ldcg(part + idx * 2);
                 td += __ldcg(part + idx * 2 + 1);
@@ -178,17 +189,16 @@ k_proxy(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, c
             __syncthreads();
             if (lane == 0) { sw[0][wid] = tn; sw[1][wid] = td; }
             __syncthreads();
-            if (threadIdx.x == 0) {
+            if (tid == 0) {
                 double bn = 0.0, bd = 0.0;
                 for (int i = 0; i < nwarps; ++i) { bn += sw[0][i]; bd += sw[1][i]; }
                 num[e] = bn;
                 den[e] = bd;
             }
         }
-        __syncthreads();   // sw and `last` are reused by the next matrix
+        __syncthreads();   // sw, msm and `last` are reused by the next matrix
         r = seg_end;
         ++e;
-        wp = W + e * ms + j;
         first = false;
     }
 }
@@ -201,12 +211,14 @@ void launch_proxy(const tq_mat* W, int64_t ms, const uint8_t* packed, const void
                   double* den, cudaStream_t st) {
     const int width = static_cast<int>(px_grid(1, 1, W->cols, 1).width);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T, PX_NO>, width, 0) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k_proxy<FMT, T, PX_NO>, width * PX_PY, 0) !=
+            cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     const PxGrid f = px_grid(W->n_mat, W->rows, W->cols, static_cast<int64_t>(num_sms()) * per_sm);
     const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
-    k_proxy<FMT, T, PX_NO><<<grid, static_cast<unsigned>(f.width), 0, st>>>(
+    const dim3 block(static_cast<unsigned>(f.width), static_cast<unsigned>(PX_PY));
+    k_proxy<FMT, T, PX_NO><<<grid, block, 0, st>>>(
         static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, packed, scales, zeros, gs, m, mst,
         W->n_mat * W->rows, f.rpb, parts, tickets, num, den);
 }

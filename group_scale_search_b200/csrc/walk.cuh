@@ -73,6 +73,17 @@ struct RowCursor {
             ptr += ld;
         }
     }
+    // n rows on (a division only where the step crosses into another matrix)
+    __device__ __forceinline__ void advance(int64_t n) {
+        o += n;
+        if (o >= O) {
+            e += o / O;
+            o %= O;
+            ptr = base + e * ms + o * ld + j;
+        } else {
+            ptr += n * ld;
+        }
+    }
 };
 
 // ------------------------------------------------------------------ device: weights
@@ -144,6 +155,12 @@ struct QPtr {
         sc = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(scales) + gid)
                                  : static_cast<const void*>(static_cast<const float*>(scales) + gid);
         zp = zeros ? zeros + gid : nullptr;
+    }
+    __device__ __forceinline__ void skip(int64_t rows) {   // `rows` rows on
+        rec += rows * G * FmtTraits<FMT>::rec;
+        sc = FMT == TQ_NVFP4_G16 ? static_cast<const void*>(static_cast<const uint8_t*>(sc) + rows * G)
+                                 : static_cast<const void*>(static_cast<const float*>(sc) + rows * G);
+        if (is_int4(FMT)) zp += rows * G;
     }
     __device__ __forceinline__ void next() {
         rec += G * FmtTraits<FMT>::rec;
