@@ -244,6 +244,13 @@ class Step:
                             torch.empty(E, dtype=torch.float64, device=dev)))
             self.ws_px.append(torch.empty(max(16, tq.proxy_workspace_bytes(u.W, fmt)), dtype=torch.uint8,
                                           device=dev))
+        # several units of one format (a dense model's projections): their
+        # dequant and proxy run as one grouped launch each
+        self.grouped = len(self.units) > 1 and len(set(self.fmts)) == 1 and hasattr(tq, "tq_dequant_batch")
+        if self.grouped:
+            self.ws_px_batch = torch.empty(max(16, tq.proxy_batch_workspace_bytes([u.W for u in self.units],
+                                                                                  self.fmts[0])),
+                                           dtype=torch.uint8, device=dev)
         self.search_events = []
         self.row_events = []
 
@@ -254,7 +261,11 @@ class Step:
     def kernels_per_step(self):
         n = KERNELS["imatrix"] * len(self.m)
         for u in self.units:
-            n += KERNELS["search"][u.fmt] + KERNELS["dequant"] + KERNELS["proxy"]
+            n += KERNELS["search"][u.fmt]
+            if not self.grouped:
+                n += KERNELS["dequant"] + KERNELS["proxy"]
+        if self.grouped:
+            n += KERNELS["dequant"] + KERNELS["proxy"]
         return n
 
     def __call__(self, k: int, time_search: bool = False):
@@ -282,6 +293,9 @@ class Step:
                 b = mark()
             if time_search:
                 self.row_events.append(("imatrix", X.numel() * X.element_size(), a, b))
+        if self.grouped:
+            self._grouped(Ws, mark, time_search)
+            return
         for i, (u, fmt) in enumerate(zip(self.units, self.fmts)):
             W = Ws[i]
             m = self._m_for(u)
@@ -294,21 +308,56 @@ class Step:
             tq.tq_dequant(r.packed, fmt, r.scales, r.zeros, r.global_scale, E, O, I, out=self.dq[i])
             if time_search:
                 c = mark()
-                self.row_events.append(("dequant", r.packed.numel() + self.dq[i].numel() * 2
-                                        + r.scales.numel() * r.scales.element_size()
-                                        + (0 if r.zeros is None else r.zeros.numel()), b, c))
+                self.row_events.append(("dequant", self._dq_bytes(i), b, c))
             tq.tq_proxy_error(W, r.packed, fmt, r.scales, r.zeros, r.global_scale, m, out=self.px[i],
                               workspace=self.ws_px[i])
             if time_search:
-                self.row_events.append(("proxy", W.numel() * W.element_size() + r.packed.numel()
-                                        + r.scales.numel() * r.scales.element_size()
-                                        + (0 if r.zeros is None else r.zeros.numel()), c, mark()))
-            if self.shard is not None and i in self.shard.row_units:   # whole-matrix (num, den)
-                from group_scale_search_b200.dist import allreduce_proxy
-                num, den = allreduce_proxy(*self.px[i])
-                self.px[i][0].copy_(num)
-                self.px[i][1].copy_(den)
+                self.row_events.append(("proxy", self._px_bytes(W, i), c, mark()))
+            self._exchange_proxy(i)
 
+    def _dq_bytes(self, i):
+        r = self.res[i]
+        return (r.packed.numel() + self.dq[i].numel() * 2 + r.scales.numel() * r.scales.element_size()
+                + (0 if r.zeros is None else r.zeros.numel()))
+
+    def _px_bytes(self, W, i):
+        r = self.res[i]
+        return (W.numel() * W.element_size() + r.packed.numel() + r.scales.numel() * r.scales.element_size()
+                + (0 if r.zeros is None else r.zeros.numel()))
+
+    def _exchange_proxy(self, i):
+        if self.shard is not None and i in self.shard.row_units:   # whole-matrix (num, den)
+            from group_scale_search_b200.dist import allreduce_proxy
+            num, den = allreduce_proxy(*self.px[i])
+            self.px[i][0].copy_(num)
+            self.px[i][1].copy_(den)
+
+    def _grouped(self, Ws, mark, time_search):
+        """Every unit's search, then one grouped dequant and one grouped proxy
+        launch over all units."""
+        tq = self.tq
+        fmt = self.fmts[0]
+        for i, u in enumerate(self.units):
+            a = mark()
+            tq.tq_search_groups(Ws[i], self._m_for(u), fmt, out=self.res[i])
+            if time_search:
+                self.search_events.append((u.fmt, Ws[i].numel(), a, mark()))
+        res = self.res
+        zeros = [r.zeros for r in res] if res[0].zeros is not None else None
+        gsc = [r.global_scale for r in res] if res[0].global_scale is not None else None
+        scales = [r.scales for r in res]
+        packed = [r.packed for r in res]
+        b = mark()
+        tq.tq_dequant_batch(packed, fmt, scales, zeros, gsc, [tuple(W.shape) for W in Ws], out=self.dq)
+        c = mark()
+        tq.tq_proxy_error_batch(Ws, packed, fmt, scales, zeros, gsc, [self._m_for(u) for u in self.units],
+                                out=self.px, workspace=self.ws_px_batch)
+        d = mark()
+        if time_search:
+            self.row_events.append(("dequant", sum(self._dq_bytes(i) for i in range(len(Ws))), b, c))
+            self.row_events.append(("proxy", sum(self._px_bytes(W, i) for i, W in enumerate(Ws)), c, d))
+        for i in range(len(Ws)):
+            self._exchange_proxy(i)
 
 def make_sets(wl, n_sets):
     """Input sets rotated through HBM so that no step finds its inputs in L2
@@ -850,26 +899,42 @@ def time_w4a4(tq, step, pk, reps=5):
 
 def time_pack(tq, step, pk, reps=12):
     """tq_pack (RTN + pack with given scales, the stand-alone form of the fused
-    pack) on the first unit, outside the step, rotating through the input
-    sets: bytes = weights read + packed records written + scales (+ zeros) read."""
-    u, r = step.units[0], step.res[0]
-    fmt = tq.FORMATS[u.fmt]
-    out = torch.empty_like(r.packed)
-    Ws = [s[1][0] for s in step.sets]
-    nbytes = (u.W.numel() * u.W.element_size() + out.numel() + r.scales.numel() * r.scales.element_size()
-              + (0 if r.zeros is None else r.zeros.numel()))
+    pack) outside the step, rotating through the input sets: on the first
+    unit, or on all units in one grouped launch (tq_pack_batch) where the step
+    groups them; bytes = weights read + packed records written + scales
+    (+ zeros) read."""
+    n = len(step.units) if step.grouped else 1
+    res = step.res[:n]
+    fmt = tq.FORMATS[step.units[0].fmt]
+    outs = [torch.empty_like(r.packed) for r in res]
+    Wsets = [s[1][:n] for s in step.sets]
+    nbytes = sum(W.numel() * W.element_size() + o.numel() + r.scales.numel() * r.scales.element_size()
+                 + (0 if r.zeros is None else r.zeros.numel()) for W, o, r in zip(Wsets[0], outs, res))
+    scales = [r.scales for r in res]
+    zeros = [r.zeros for r in res] if res[0].zeros is not None else None
+    gsc = [r.global_scale for r in res] if res[0].global_scale is not None else None
+
+    def call(k):
+        Ws = Wsets[k % len(Wsets)]
+        if step.grouped:
+            tq.tq_pack_batch(Ws, fmt, scales, zeros, gsc, out=outs)
+        else:
+            r = res[0]
+            tq.tq_pack(Ws[0], fmt, r.scales, r.zeros, r.global_scale, out=outs[0])
+
     for k in range(3):
-        tq.tq_pack(Ws[k % len(Ws)], fmt, r.scales, r.zeros, r.global_scale, out=out)
+        call(k)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for k in range(reps):
-        tq.tq_pack(Ws[k % len(Ws)], fmt, r.scales, r.zeros, r.global_scale, out=out)
+        call(k)
     b.record()
     torch.cuda.synchronize()
     ms = a.elapsed_time(b) / reps
     gbs = nbytes / (ms * 1e-3) / 1e9
+    what = f"all {n} units in one grouped launch" if step.grouped else "first unit"
     return {"ms": ms, "bytes": nbytes, "GB/s": gbs, "frac": gbs / pk["hbm_gbs"],
-            "note": f"first unit, back-to-back launches over {len(Ws)} rotating weight copies"}
+            "note": f"{what}, back-to-back launches over {len(Wsets)} rotating weight copies"}
 
 
 def time_ladder(tq, step, peak_tinst, reps=3):

@@ -31,8 +31,8 @@ import torch
 __all__ = [
     "INT3_G64_SYM", "INT4_G128_ASYM", "INT4_G64_ASYM", "INT4_G32_ASYM", "NVFP4_G16", "SearchParams", "SearchResult", "TQError",
     "lib", "lib_path", "tq_version", "tq_group_size", "tq_num_groups", "tq_packed_bytes", "search_result_empty",
-    "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_codes", "tq_unpack_codes",
-    "tq_dequant", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
+    "tq_imatrix", "tq_amax", "tq_search_groups", "tq_pack", "tq_pack_batch", "tq_pack_codes", "tq_unpack_codes",
+    "tq_dequant", "tq_dequant_batch", "tq_proxy_error_batch", "proxy_batch_workspace_bytes", "MAX_BATCH", "tq_dequant_gemv", "tq_hessian", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8", "Fp8Result",
     "tq_lloyd_max_g32", "tq_dequant_lm2", "LloydResult", "tq_proxy_error", "tq_proxy_error_full", "tq_gptq_sweep", "tq_sync", "tq_debug_set_wait_limit", "tq_selftest_e2m1",
     "tq_quant_nvfp4_act", "Nvfp4Act", "tq_nvfp4_scales_to_mma", "tq_gemm_nvfp4", "FORMATS", "EXPORTS",
 ]
@@ -56,7 +56,8 @@ _lib = None
 EXPORTS = [
     "tq_default_params", "tq_last_error_string", "tq_version", "tq_group_size", "tq_num_groups",
     "tq_packed_bytes", "tq_imatrix_workspace_bytes", "tq_imatrix", "tq_amax", "tq_search_groups",
-    "tq_pack", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_proxy_workspace_bytes",
+    "tq_pack", "tq_pack_batch", "tq_pack_codes", "tq_unpack_codes", "tq_dequant", "tq_dequant_batch",
+    "tq_proxy_workspace_bytes", "tq_proxy_batch_workspace_bytes", "tq_proxy_error_batch",
     "tq_proxy_error", "tq_sync", "tq_imatrix_static_capacity", "tq_imatrix_static", "tq_selftest_e2m1",
     "tq_dequant_gemv", "tq_hessian", "tq_fp8_workspace_bytes", "tq_search_fp8", "tq_pack_fp8", "tq_dequant_fp8",
     "tq_lloyd_workspace_bytes", "tq_lloyd_max_g32", "tq_dequant_lm2", "tq_proxy_full_workspace_bytes",
@@ -147,6 +148,10 @@ def lib():
             "tq_amax": (i32, [Mp, P, P]),
             "tq_search_groups": (i32, [Mp, P, i64, i32, ctypes.POINTER(_Params), P, P, P, P, P, P, P]),
             "tq_pack": (i32, [Mp, i32, P, P, P, P, P]),
+            "tq_pack_batch": (i32, [i32, Mp, i32, P, P, P, P, P]),
+            "tq_dequant_batch": (i32, [i32, P, i32, P, P, P, P, P, P, P, i32, P]),
+            "tq_proxy_batch_workspace_bytes": (sz, [i32, Mp, i32]),
+            "tq_proxy_error_batch": (i32, [i32, Mp, P, i32, P, P, P, P, P, P, P, P, sz, P]),
             "tq_pack_codes": (i32, [P, i32, i64, i64, P, P, P]),
             "tq_unpack_codes": (i32, [P, i32, i64, i64, P, P]),
             "tq_dequant": (i32, [P, i32, P, P, P, i64, i64, i64, P, i32, P]),
@@ -582,6 +587,86 @@ def tq_proxy_error(W: torch.Tensor, packed: torch.Tensor, fmt: int, scales: torc
     _check(lib().tq_proxy_error(ctypes.byref(d), _ptr(packed), fmt, _ptr(scales), _ptr(zeros),
                                 _ptr(global_scale), _ptr(m), _m_stride(m), _ptr(out[0]), _ptr(out[1]),
                                 _ptr(workspace), workspace.numel(), _stream(stream)), "tq_proxy_error")
+    return out
+
+
+# ---------------------------------------------------------------- grouped launches
+
+MAX_BATCH = 16   # TQ_MAX_BATCH
+
+
+def _ptrs(ts) -> ctypes.Array:
+    """A host array of device pointers (NULL for None entries)."""
+    return (ctypes.c_void_p * len(ts))(*[None if t is None else t.data_ptr() for t in ts])
+
+
+def _opt_ptrs(ts):
+    return None if ts is None or all(t is None for t in ts) else _ptrs(ts)
+
+
+def _mats(Ws, name: str):
+    ds = [_mat(W, f"{name}[{i}]") for i, W in enumerate(Ws)]
+    if not 1 <= len(ds) <= MAX_BATCH:
+        raise TQError(f"{name}: {len(ds)} units, expected 1..{MAX_BATCH}")
+    return (_Mat * len(ds))(*ds)
+
+
+def tq_pack_batch(Ws, fmt: int, scales, zeros=None, global_scale=None, out=None, stream=None):
+    """tq_pack of several units (matrix batches of any shapes, one format and
+    weight dtype) in one launch; lists of tensors per unit."""
+    arr = _mats(Ws, "Ws")
+    if out is None:
+        out = [torch.empty(tq_packed_bytes(fmt, d.n_mat * d.rows, d.cols), dtype=torch.uint8, device=W.device)
+               for W, d in zip(Ws, arr)]
+    _check(lib().tq_pack_batch(len(Ws), arr, fmt, _ptrs(scales), _opt_ptrs(zeros), _opt_ptrs(global_scale),
+                               _ptrs(out), _stream(stream)), "tq_pack_batch")
+    return out
+
+
+def tq_dequant_batch(packed, fmt: int, scales, zeros, global_scale, shapes, out_dtype=torch.float32, out=None,
+                     stream=None):
+    """tq_dequant of several units in one launch; shapes = [(n_mat, O, I), ...]."""
+    n = len(packed)
+    if not 1 <= n <= MAX_BATCH:
+        raise TQError(f"tq_dequant_batch: {n} units, expected 1..{MAX_BATCH}")
+    for i, t in enumerate(packed):
+        _cuda(t, f"packed[{i}]")
+    if out is None:
+        out = [torch.empty(tuple(sh), dtype=out_dtype, device=packed[0].device) for sh in shapes]
+    odt = _BF16 if out[0].dtype == torch.bfloat16 else _F32
+    if any(o.dtype != out[0].dtype for o in out):
+        raise TQError("tq_dequant_batch: outputs of different dtypes")
+    i64 = ctypes.c_int64 * n
+    _check(lib().tq_dequant_batch(n, _ptrs(packed), fmt, _ptrs(scales), _opt_ptrs(zeros), _opt_ptrs(global_scale),
+                                  i64(*[s[0] for s in shapes]), i64(*[s[1] for s in shapes]),
+                                  i64(*[s[2] for s in shapes]), _ptrs(out), odt, _stream(stream)),
+           "tq_dequant_batch")
+    return out
+
+
+def proxy_batch_workspace_bytes(Ws, fmt: int) -> int:
+    arr = _mats(Ws, "Ws")
+    return int(lib().tq_proxy_batch_workspace_bytes(len(Ws), arr, fmt))
+
+
+def tq_proxy_error_batch(Ws, packed, fmt: int, scales, zeros, global_scale, ms, out=None, workspace=None,
+                         stream=None):
+    """tq_proxy_error of several units in one launch: [(num, den), ...]."""
+    arr = _mats(Ws, "Ws")
+    for d, m in zip(arr, ms):
+        _check_m(m, d.n_mat, d.cols)
+    n = len(Ws)
+    if out is None:
+        out = [(torch.empty(d.n_mat, dtype=torch.float64, device=W.device),
+                torch.empty(d.n_mat, dtype=torch.float64, device=W.device)) for W, d in zip(Ws, arr)]
+    ws = int(lib().tq_proxy_batch_workspace_bytes(n, arr, fmt))
+    if workspace is None:
+        workspace = torch.empty(max(ws, 16), dtype=torch.uint8, device=Ws[0].device)
+    _check(lib().tq_proxy_error_batch(n, arr, _ptrs(packed), fmt, _ptrs(scales), _opt_ptrs(zeros),
+                                      _opt_ptrs(global_scale), _ptrs(ms),
+                                      (ctypes.c_int64 * n)(*[_m_stride(m) for m in ms]),
+                                      _ptrs([o[0] for o in out]), _ptrs([o[1] for o in out]), _ptr(workspace),
+                                      workspace.numel(), _stream(stream)), "tq_proxy_error_batch")
     return out
 
 

@@ -5,7 +5,7 @@
 // records of a 2-bit low plane and a 1-bit high plane, v + 4); int4 and NVFP4
 // records hold one code per nibble, element 2k in the low nibble of byte k.
 // Dequantization rounds once to fp32: s v, s (q - z), fl32(fl32(g dec(e)) dec(c)).
-#include "walk.cuh"
+#include "batch.cuh"
 
 namespace tq {
 
@@ -58,11 +58,26 @@ __device__ __forceinline__ void pack_unit(const Oct<T> o[NO], const int n[NO], f
     }
 }
 
-// Grid: x = unit-column tiles (a unit = NO octets), y = blocks of
-// consecutive rows of the whole batch (rows of all matrices in order, so
-// every block gets the same number of rows whatever the matrix count).
-// Pointers to the weights, records, scales and zero-points advance by their
-// row strides.
+// One unit of a grouped tq_pack launch.
+struct PkUnit {
+    const void* W;
+    int64_t O, I, ld, ms, n_rows;
+    const void* scales;
+    const uint8_t* zeros;
+    const float* gs;
+    uint8_t* packed;
+    BatchSlot s;
+};
+struct PkArgs {
+    int n;
+    PkUnit u[BATCH_MAX];
+};
+
+// Blocks: the units' ranges of the 1-D grid; within a unit, column tiles
+// (a unit column = NO octets) times blocks of consecutive rows of its whole
+// batch (rows of all matrices in order, so every block gets the same
+// number of rows whatever the matrix count).  Pointers to the weights,
+// records, scales and zero-points advance by their row strides.
 // Row walkers per block (blockDim.y): they share the block's unit columns
 // and take interleaved rows of its range.  Measured on the full-size
 // workloads: four walkers per block for int3 (0.523 -> 0.479 ms on the MoE
@@ -71,15 +86,17 @@ __device__ __forceinline__ void pack_unit(const Oct<T> o[NO], const int n[NO], f
 // instead of six of 6).
 template <int FMT> __host__ __device__ constexpr int pk_py() { return FMT == TQ_INT3_G64_SYM ? 4 : 1; }
 
+// The body of both kernels below: column tile cx (cw unit columns wide) and
+// row block ry of one unit.
 template <int FMT, typename T, int NO>
-__global__ void __launch_bounds__(256 * pk_py<FMT>())
-k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, int64_t n_rows, int64_t rpb,
-       const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
-       uint8_t* __restrict__ packed) {
+__device__ __forceinline__ void pack_rows(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms,
+                                          int64_t n_rows, int64_t rpb, const void* scales,
+                                          const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
+                                          uint8_t* __restrict__ packed, int64_t cx, int64_t ry, int64_t cw) {
     using F = FmtTraits<FMT>;
     const int64_t G = (I + F::group - 1) / F::group;
-    const int64_t u = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (u >= (G << F::lg) / NO) return;
+    const int64_t u = cx * cw + threadIdx.x;
+    if (threadIdx.x >= cw || u >= (G << F::lg) / NO) return;   // no barrier in these kernels
     const int64_t c = u * NO;   // first octet of the unit
     const int64_t k = c >> F::lg;
     const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
@@ -89,7 +106,7 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
     for (int i = 0; i < NO; ++i)
         n[i] = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(8), I - j - 8 * i)));
     const int64_t py = blockDim.y;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rpb + threadIdx.y, r1 = min(n_rows, r0 - threadIdx.y + rpb);
+    const int64_t r0 = ry * rpb + threadIdx.y, r1 = min(n_rows, r0 - threadIdx.y + rpb);
     RowCursor<T> cur(W, O, ld, ms, j, r0);
     const int64_t rstride = py * G * F::rec;   // this walker's rows: r0, r0 + py, ...
     uint8_t* rec = packed + (r0 * G + k) * F::rec;
@@ -130,6 +147,26 @@ k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, in
         bp += ROWS * py * G;
         if (is_int4(FMT)) zp += ROWS * py * G;
     }
+}
+
+// One unit: grid x = column tiles, y = row blocks.
+template <int FMT, typename T, int NO>
+__global__ void __launch_bounds__(256 * pk_py<FMT>())
+k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, int64_t n_rows, int64_t rpb,
+       const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
+       uint8_t* __restrict__ packed) {
+    pack_rows<FMT, T, NO>(W, O, I, ld, ms, n_rows, rpb, scales, zeros, gs, packed, blockIdx.x, blockIdx.y,
+                          blockDim.x);
+}
+
+// Several units: each block looks up its unit's range of the 1-D grid.
+template <int FMT, typename T, int NO>
+__global__ void __launch_bounds__(256 * pk_py<FMT>())
+k_pack_batch(const __grid_constant__ PkArgs a) {
+    const PkUnit& p = a.u[batch_unit(a.u, a.n, blockIdx.x)];
+    const int64_t lb = static_cast<int64_t>(blockIdx.x) - p.s.block0;
+    pack_rows<FMT, T, NO>(static_cast<const T*>(p.W), p.O, p.I, p.ld, p.ms, p.n_rows, p.s.rpb, p.scales, p.zeros,
+                          p.gs, p.packed, lb % p.s.cblocks, lb / p.s.cblocks, p.s.cw);
 }
 
 // ------------------------------------------------------------------ pack / unpack integer codes
@@ -218,24 +255,41 @@ __device__ __forceinline__ void store8(O* dst, const float v[8], bool vec_ok, in
     }
 }
 
-// Grid: x = octet-column tiles, y = blocks of consecutive rows of the whole
-// batch (the output is dense, so a row's place does not depend on its
+// One unit of a grouped tq_dequant launch.
+struct DqUnit {
+    const uint8_t* packed;
+    const void* scales;
+    const uint8_t* zeros;
+    const float* gs;
+    int64_t Orows, I, n_rows;
+    void* out;
+    BatchSlot s;
+};
+struct DqArgs {
+    int n;
+    DqUnit u[BATCH_MAX];
+};
+
+// Within a unit: octet-column tiles times blocks of consecutive rows of its
+// whole batch (the output is dense, so a row's place does not depend on its
 // matrix).  A thread loads DQ_ROWS rows' codes and scales before decoding
-// any of them.
+// any of them.  The body of both kernels below: column tile cx (cw octet
+// columns wide) and row block ry of one unit.
 template <int FMT, typename O>
-__global__ void __launch_bounds__(256)
-k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t* __restrict__ zeros,
-          const float* __restrict__ gs, int64_t Orows, int64_t I, int64_t n_rows, int64_t rpb, O* __restrict__ out) {
+__device__ __forceinline__ void dequant_rows(const uint8_t* __restrict__ packed, const void* scales,
+                                             const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
+                                             int64_t Orows, int64_t I, int64_t n_rows, int64_t rpb,
+                                             O* __restrict__ out, int64_t cx, int64_t ry, int64_t cw) {
     using F = FmtTraits<FMT>;
     const int64_t G = (I + F::group - 1) / F::group;
-    const int64_t c = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (c >= ((I + 7) >> 3)) return;
+    const int64_t c = cx * cw + threadIdx.x;
+    if (threadIdx.x >= cw || c >= ((I + 7) >> 3)) return;
     const int64_t k = c >> F::lg;
     const int oct = static_cast<int>(c & ((1 << F::lg) - 1));
     const int64_t j = c << 3;
     const int nvalid = static_cast<int>(min(static_cast<int64_t>(8), I - j));
     const bool vec_ok = ((I * static_cast<int64_t>(sizeof(O))) % 16) == 0;
-    const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rpb, r1 = min(n_rows, r0 + rpb);
+    const int64_t r0 = ry * rpb, r1 = min(n_rows, r0 + rpb);
     int64_t e = 0, next_e = n_rows;   // NVFP4: matrix of row r and the first row of the next matrix
     float g = 0.f;
     if (FMT == TQ_NVFP4_G16) {
@@ -263,51 +317,104 @@ k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t*
     }
 }
 
-// ------------------------------------------------------------------ host launchers
-// The grid holds at most as many blocks as the SMs keep resident (one wave),
-// rows split evenly over the row blocks.
-
-struct FlatGrid { int64_t width, cblocks, rblocks, rpb; };
-
-inline FlatGrid flat_grid(int64_t n_rows, int64_t cols, int64_t resident_per_sm) {
-    FlatGrid f;
-    const Walk w = walk_geometry(1, 1, cols, 1);
-    f.width = w.width;
-    f.cblocks = w.cblocks;
-    const int64_t cap = static_cast<int64_t>(num_sms()) * resident_per_sm;
-    int64_t rb = max(static_cast<int64_t>(1), cap / f.cblocks);
-    rb = min(rb, min(n_rows, static_cast<int64_t>(65535)));
-    f.rpb = (n_rows + rb - 1) / rb;
-    f.rblocks = (n_rows + f.rpb - 1) / f.rpb;
-    return f;
+// One unit: grid x = octet-column tiles, y = row blocks.  At most 32
+// registers (8 blocks of 256 threads per SM): the loads in flight come from
+// resident warps.
+template <int FMT, typename O>
+__global__ void __launch_bounds__(256, 8)
+k_dequant(const uint8_t* __restrict__ packed, const void* scales, const uint8_t* __restrict__ zeros,
+          const float* __restrict__ gs, int64_t Orows, int64_t I, int64_t n_rows, int64_t rpb, O* __restrict__ out) {
+    dequant_rows<FMT, O>(packed, scales, zeros, gs, Orows, I, n_rows, rpb, out, blockIdx.x, blockIdx.y, blockDim.x);
 }
 
+// Several units: each block looks up its unit's range of the 1-D grid.
+template <int FMT, typename O>
+__global__ void __launch_bounds__(256, 8)
+k_dequant_batch(const __grid_constant__ DqArgs a) {
+    const DqUnit& p = a.u[batch_unit(a.u, a.n, blockIdx.x)];
+    const int64_t lb = static_cast<int64_t>(blockIdx.x) - p.s.block0;
+    dequant_rows<FMT, O>(p.packed, p.scales, p.zeros, p.gs, p.Orows, p.I, p.n_rows, p.s.rpb, static_cast<O*>(p.out),
+                         lb % p.s.cblocks, lb / p.s.cblocks, p.s.cw);
+}
+
+// ------------------------------------------------------------------ host launchers
+// The grid holds at most as many blocks as the SMs keep resident (one wave),
+// split over the units by size; within a unit, rows split evenly over its
+// row blocks.
+
 template <int FMT, typename T>
-void launch_pack(const tq_mat* W, int64_t ms, const void* scales, const uint8_t* zeros, const float* gs,
-                 uint8_t* packed, cudaStream_t st) {
+void launch_pack(int n, const tq_mat* W, const void* const* scales, const uint8_t* const* zeros,
+                 const float* const* gs, uint8_t* const* packed, cudaStream_t st) {
     const int64_t g = FmtTraits<FMT>::group;
     constexpr int NO = pk_no<FMT>();
-    const int64_t cols = (W->cols + g - 1) / g * (g / 8) / NO;
-    const int64_t n_rows = W->n_mat * W->rows;
-    const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
     constexpr int PY = pk_py<FMT>();
-    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_pack<FMT, T, NO>, width * PY));
-    const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
-    const dim3 block(static_cast<unsigned>(f.width), static_cast<unsigned>(PY));
-    k_pack<FMT, T, NO><<<grid, block, 0, st>>>(
-        static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms, n_rows, f.rpb, scales, zeros, gs, packed);
+    int64_t cols[BATCH_MAX], rows[BATCH_MAX];
+    for (int i = 0; i < n; ++i) {
+        cols[i] = (W[i].cols + g - 1) / g * (g / 8) / NO;
+        rows[i] = W[i].n_mat * W[i].rows;
+    }
+    int64_t width = 32;
+    BatchSlot sl[BATCH_MAX];
+    batch_split(n, cols, rows, 1, sl, &width);   // the widest tile sets the block shape
+    const dim3 block(static_cast<unsigned>(width), static_cast<unsigned>(PY));
+    if (n == 1) {
+        const int64_t slots = static_cast<int64_t>(num_sms()) * resident_blocks(k_pack<FMT, T, NO>, static_cast<int>(width) * PY);
+        batch_split(1, cols, rows, slots, sl, &width);
+        const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
+        const dim3 grid(static_cast<unsigned>(sl[0].cblocks), static_cast<unsigned>(sl[0].rblocks));
+        k_pack<FMT, T, NO><<<grid, block, 0, st>>>(static_cast<const T*>(W->ptr), W->rows, W->cols, W->ld, ms,
+                                                   rows[0], sl[0].rpb, scales[0], zeros ? zeros[0] : nullptr,
+                                                   gs ? gs[0] : nullptr, packed[0]);
+        return;
+    }
+    static thread_local PkArgs a;
+    const int64_t slots = static_cast<int64_t>(num_sms()) * resident_blocks(k_pack_batch<FMT, T, NO>, static_cast<int>(width) * PY);
+    const int64_t blocks = batch_split(n, cols, rows, slots, sl, &width);
+    a.n = n;
+    for (int i = 0; i < n; ++i) {
+        PkUnit& u = a.u[i];
+        u.W = W[i].ptr; u.O = W[i].rows; u.I = W[i].cols; u.ld = W[i].ld;
+        u.ms = W[i].n_mat > 1 ? W[i].mat_stride : 0;
+        u.n_rows = rows[i];
+        u.scales = scales[i]; u.zeros = zeros ? zeros[i] : nullptr; u.gs = gs ? gs[i] : nullptr;
+        u.packed = packed[i];
+        u.s = sl[i];
+    }
+    k_pack_batch<FMT, T, NO><<<static_cast<unsigned>(blocks), block, 0, st>>>(a);
 }
 
 template <int FMT, typename O>
-void launch_dequant(const uint8_t* packed, const void* scales, const uint8_t* zeros, const float* gs, int64_t n_mat,
-                    int64_t Orows, int64_t I, void* out, cudaStream_t st) {
-    const int64_t cols = (I + 7) / 8;
-    const int64_t n_rows = n_mat * Orows;
-    const int width = static_cast<int>(walk_geometry(1, 1, cols, 1).width);
-    const FlatGrid f = flat_grid(n_rows, cols, resident_blocks(k_dequant<FMT, O>, width));
-    const dim3 grid(static_cast<unsigned>(f.cblocks), static_cast<unsigned>(f.rblocks));
-    k_dequant<FMT, O><<<grid, static_cast<unsigned>(f.width), 0, st>>>(packed, scales, zeros, gs, Orows, I,
-                                                                             n_rows, f.rpb, static_cast<O*>(out));
+void launch_dequant(int n, const uint8_t* const* packed, const void* const* scales, const uint8_t* const* zeros,
+                    const float* const* gs, const int64_t* n_mat, const int64_t* Orows, const int64_t* I,
+                    void* const* out, cudaStream_t st) {
+    int64_t cols[BATCH_MAX], rows[BATCH_MAX];
+    for (int i = 0; i < n; ++i) {
+        cols[i] = (I[i] + 7) / 8;
+        rows[i] = n_mat[i] * Orows[i];
+    }
+    int64_t width = 32;
+    BatchSlot sl[BATCH_MAX];
+    batch_split(n, cols, rows, 1, sl, &width);
+    if (n == 1) {
+        const int64_t slots = static_cast<int64_t>(num_sms()) * resident_blocks(k_dequant<FMT, O>, static_cast<int>(width));
+        batch_split(1, cols, rows, slots, sl, &width);
+        const dim3 grid(static_cast<unsigned>(sl[0].cblocks), static_cast<unsigned>(sl[0].rblocks));
+        k_dequant<FMT, O><<<grid, static_cast<unsigned>(width), 0, st>>>(
+            packed[0], scales[0], zeros ? zeros[0] : nullptr, gs ? gs[0] : nullptr, Orows[0], I[0], rows[0],
+            sl[0].rpb, static_cast<O*>(out[0]));
+        return;
+    }
+    static thread_local DqArgs a;
+    const int64_t slots = static_cast<int64_t>(num_sms()) * resident_blocks(k_dequant_batch<FMT, O>, static_cast<int>(width));
+    const int64_t blocks = batch_split(n, cols, rows, slots, sl, &width);
+    a.n = n;
+    for (int i = 0; i < n; ++i) {
+        DqUnit& u = a.u[i];
+        u.packed = packed[i]; u.scales = scales[i]; u.zeros = zeros ? zeros[i] : nullptr; u.gs = gs ? gs[i] : nullptr;
+        u.Orows = Orows[i]; u.I = I[i]; u.n_rows = rows[i]; u.out = out[i];
+        u.s = sl[i];
+    }
+    k_dequant_batch<FMT, O><<<static_cast<unsigned>(blocks), static_cast<unsigned>(width), 0, st>>>(a);
 }
 
 }  // namespace tq
@@ -319,31 +426,62 @@ static tq_status check_fmt(int32_t fmt, const char* who) {
     return TQ_OK;
 }
 
+// Checks of one unit of tq_pack / tq_pack_batch.
+static tq_status check_pack_unit(const tq_mat* W, int32_t fmt, const void* scales, const uint8_t* zeros,
+                                 const float* global_scale, const uint8_t* packed, const char* who) {
+    tq_status s = check_mat(W, who);
+    if (s != TQ_OK) return s;
+    TQ_REQUIRE(scales != nullptr && packed != nullptr, "%s: null scales or packed", who);
+    TQ_REQUIRE(aligned16(packed), "%s: packed not 16-byte aligned", who);
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "%s: int4 needs zeros", who);
+    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "%s: NVFP4 needs global_scale", who);
+    return TQ_OK;
+}
+
+static void dispatch_pack(int n, const tq_mat* W, int32_t fmt, const void* const* scales,
+                          const uint8_t* const* zeros, const float* const* gs, uint8_t* const* packed,
+                          cudaStream_t st) {
+    const bool bf = W[0].dtype == TQ_BF16;
+    if (fmt == TQ_INT3_G64_SYM) bf ? launch_pack<TQ_INT3_G64_SYM, uint16_t>(n, W, scales, zeros, gs, packed, st)
+                                   : launch_pack<TQ_INT3_G64_SYM, float>(n, W, scales, zeros, gs, packed, st);
+    else if (fmt == TQ_INT4_G128_ASYM) bf ? launch_pack<TQ_INT4_G128_ASYM, uint16_t>(n, W, scales, zeros, gs, packed, st)
+                                          : launch_pack<TQ_INT4_G128_ASYM, float>(n, W, scales, zeros, gs, packed, st);
+    else if (fmt == TQ_INT4_G64_ASYM) bf ? launch_pack<TQ_INT4_G64_ASYM, uint16_t>(n, W, scales, zeros, gs, packed, st)
+                                         : launch_pack<TQ_INT4_G64_ASYM, float>(n, W, scales, zeros, gs, packed, st);
+    else if (fmt == TQ_INT4_G32_ASYM) bf ? launch_pack<TQ_INT4_G32_ASYM, uint16_t>(n, W, scales, zeros, gs, packed, st)
+                                         : launch_pack<TQ_INT4_G32_ASYM, float>(n, W, scales, zeros, gs, packed, st);
+    else bf ? launch_pack<TQ_NVFP4_G16, uint16_t>(n, W, scales, zeros, gs, packed, st)
+            : launch_pack<TQ_NVFP4_G16, float>(n, W, scales, zeros, gs, packed, st);
+}
+
 TQ_API tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const uint8_t* zeros,
                          const float* global_scale, uint8_t* packed, tq_stream_t stream) {
     clear_error();
-    tq_status s = check_mat(W, "tq_pack W");
+    tq_status s = check_fmt(fmt, "tq_pack");
     if (s != TQ_OK) return s;
-    if ((s = check_fmt(fmt, "tq_pack")) != TQ_OK) return s;
-    TQ_REQUIRE(scales != nullptr && packed != nullptr, "tq_pack: null scales or packed");
-    TQ_REQUIRE(aligned16(packed), "tq_pack: packed not 16-byte aligned");
-    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_pack: int4 needs zeros");
-    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_pack: NVFP4 needs global_scale");
-    TQ_REQUIRE(W->n_mat <= 65535, "tq_pack: more than 65535 matrices in one call");
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0;
-    const bool bf = W->dtype == TQ_BF16;
-    if (fmt == TQ_INT3_G64_SYM) bf ? launch_pack<TQ_INT3_G64_SYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
-                                   : launch_pack<TQ_INT3_G64_SYM, float>(W, ms, scales, zeros, global_scale, packed, st);
-    else if (fmt == TQ_INT4_G128_ASYM) bf ? launch_pack<TQ_INT4_G128_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
-                                          : launch_pack<TQ_INT4_G128_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
-    else if (fmt == TQ_INT4_G64_ASYM) bf ? launch_pack<TQ_INT4_G64_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
-                                         : launch_pack<TQ_INT4_G64_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
-    else if (fmt == TQ_INT4_G32_ASYM) bf ? launch_pack<TQ_INT4_G32_ASYM, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
-                                         : launch_pack<TQ_INT4_G32_ASYM, float>(W, ms, scales, zeros, global_scale, packed, st);
-    else bf ? launch_pack<TQ_NVFP4_G16, uint16_t>(W, ms, scales, zeros, global_scale, packed, st)
-            : launch_pack<TQ_NVFP4_G16, float>(W, ms, scales, zeros, global_scale, packed, st);
+    if ((s = check_pack_unit(W, fmt, scales, zeros, global_scale, packed, "tq_pack")) != TQ_OK) return s;
+    dispatch_pack(1, W, fmt, &scales, &zeros, &global_scale, &packed, reinterpret_cast<cudaStream_t>(stream));
     return check_launch("tq_pack");
+}
+
+TQ_API tq_status tq_pack_batch(int32_t n, const tq_mat* W, int32_t fmt, const void* const* scales,
+                               const uint8_t* const* zeros, const float* const* global_scale,
+                               uint8_t* const* packed, tq_stream_t stream) {
+    clear_error();
+    tq_status s = check_fmt(fmt, "tq_pack_batch");
+    if (s != TQ_OK) return s;
+    TQ_REQUIRE(n >= 1 && n <= TQ_MAX_BATCH, "tq_pack_batch: n = %d outside [1, %d]", n, TQ_MAX_BATCH);
+    TQ_REQUIRE(W && scales && packed, "tq_pack_batch: null array");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_pack_batch: int4 needs zeros");
+    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_pack_batch: NVFP4 needs global_scale");
+    for (int i = 0; i < n; ++i) {
+        if ((s = check_pack_unit(&W[i], fmt, scales[i], zeros ? zeros[i] : nullptr,
+                                 global_scale ? global_scale[i] : nullptr, packed[i], "tq_pack_batch")) != TQ_OK)
+            return s;
+        TQ_REQUIRE(W[i].dtype == W[0].dtype, "tq_pack_batch: units of different dtypes");
+    }
+    dispatch_pack(n, W, fmt, scales, zeros, global_scale, packed, reinterpret_cast<cudaStream_t>(stream));
+    return check_launch("tq_pack_batch");
 }
 
 TQ_API tq_status tq_pack_codes(const uint8_t* codes, int32_t fmt, int64_t rows, int64_t cols,
@@ -373,35 +511,69 @@ TQ_API tq_status tq_unpack_codes(const uint8_t* packed, int32_t fmt, int64_t row
     return check_launch("tq_unpack_codes");
 }
 
+static tq_status check_dequant_unit(const uint8_t* packed, int32_t fmt, const void* scales, const uint8_t* zeros,
+                                    const float* global_scale, int64_t n_mat, int64_t O, int64_t I, const void* out,
+                                    const char* who) {
+    TQ_REQUIRE(packed && scales && out, "%s: null pointer", who);
+    TQ_REQUIRE(n_mat >= 1 && O >= 1 && I >= 1, "%s: empty shape", who);
+    TQ_REQUIRE(aligned16(packed) && aligned16(out), "%s: packed/out not 16-byte aligned", who);
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "%s: int4 needs zeros", who);
+    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "%s: NVFP4 needs global_scale", who);
+    return TQ_OK;
+}
+
+static void dispatch_dequant(int n, const uint8_t* const* packed, int32_t fmt, const void* const* scales,
+                             const uint8_t* const* zeros, const float* const* gs, const int64_t* n_mat,
+                             const int64_t* O, const int64_t* I, void* const* out, bool bf, cudaStream_t st) {
+    if (fmt == TQ_INT3_G64_SYM)
+        bf ? launch_dequant<TQ_INT3_G64_SYM, __nv_bfloat16>(n, packed, scales, zeros, gs, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT3_G64_SYM, float>(n, packed, scales, zeros, gs, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G128_ASYM)
+        bf ? launch_dequant<TQ_INT4_G128_ASYM, __nv_bfloat16>(n, packed, scales, zeros, gs, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G128_ASYM, float>(n, packed, scales, zeros, gs, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G64_ASYM)
+        bf ? launch_dequant<TQ_INT4_G64_ASYM, __nv_bfloat16>(n, packed, scales, zeros, gs, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G64_ASYM, float>(n, packed, scales, zeros, gs, n_mat, O, I, out, st);
+    else if (fmt == TQ_INT4_G32_ASYM)
+        bf ? launch_dequant<TQ_INT4_G32_ASYM, __nv_bfloat16>(n, packed, scales, zeros, gs, n_mat, O, I, out, st)
+           : launch_dequant<TQ_INT4_G32_ASYM, float>(n, packed, scales, zeros, gs, n_mat, O, I, out, st);
+    else
+        bf ? launch_dequant<TQ_NVFP4_G16, __nv_bfloat16>(n, packed, scales, zeros, gs, n_mat, O, I, out, st)
+           : launch_dequant<TQ_NVFP4_G16, float>(n, packed, scales, zeros, gs, n_mat, O, I, out, st);
+}
+
 TQ_API tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scales, const uint8_t* zeros,
                             const float* global_scale, int64_t n_mat, int64_t O, int64_t I, void* out,
                             int32_t out_dtype, tq_stream_t stream) {
     clear_error();
     tq_status s = check_fmt(fmt, "tq_dequant");
     if (s != TQ_OK) return s;
-    TQ_REQUIRE(packed && scales && out, "tq_dequant: null pointer");
-    TQ_REQUIRE(n_mat >= 1 && O >= 1 && I >= 1, "tq_dequant: empty shape");
-    TQ_REQUIRE(aligned16(packed) && aligned16(out), "tq_dequant: packed/out not 16-byte aligned");
-    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_dequant: int4 needs zeros");
-    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant: NVFP4 needs global_scale");
+    if ((s = check_dequant_unit(packed, fmt, scales, zeros, global_scale, n_mat, O, I, out, "tq_dequant")) != TQ_OK)
+        return s;
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant: out dtype %d", out_dtype);
-    TQ_REQUIRE(n_mat <= 65535, "tq_dequant: more than 65535 matrices in one call");
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const bool bf = out_dtype == TQ_BF16;
-    if (fmt == TQ_INT3_G64_SYM)
-        bf ? launch_dequant<TQ_INT3_G64_SYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
-           : launch_dequant<TQ_INT3_G64_SYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
-    else if (fmt == TQ_INT4_G128_ASYM)
-        bf ? launch_dequant<TQ_INT4_G128_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
-           : launch_dequant<TQ_INT4_G128_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
-    else if (fmt == TQ_INT4_G64_ASYM)
-        bf ? launch_dequant<TQ_INT4_G64_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
-           : launch_dequant<TQ_INT4_G64_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
-    else if (fmt == TQ_INT4_G32_ASYM)
-        bf ? launch_dequant<TQ_INT4_G32_ASYM, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
-           : launch_dequant<TQ_INT4_G32_ASYM, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
-    else
-        bf ? launch_dequant<TQ_NVFP4_G16, __nv_bfloat16>(packed, scales, zeros, global_scale, n_mat, O, I, out, st)
-           : launch_dequant<TQ_NVFP4_G16, float>(packed, scales, zeros, global_scale, n_mat, O, I, out, st);
+    dispatch_dequant(1, &packed, fmt, &scales, &zeros, &global_scale, &n_mat, &O, &I, &out, out_dtype == TQ_BF16,
+                     reinterpret_cast<cudaStream_t>(stream));
     return check_launch("tq_dequant");
+}
+
+TQ_API tq_status tq_dequant_batch(int32_t n, const uint8_t* const* packed, int32_t fmt, const void* const* scales,
+                                  const uint8_t* const* zeros, const float* const* global_scale,
+                                  const int64_t* n_mat, const int64_t* O, const int64_t* I, void* const* out,
+                                  int32_t out_dtype, tq_stream_t stream) {
+    clear_error();
+    tq_status s = check_fmt(fmt, "tq_dequant_batch");
+    if (s != TQ_OK) return s;
+    TQ_REQUIRE(n >= 1 && n <= TQ_MAX_BATCH, "tq_dequant_batch: n = %d outside [1, %d]", n, TQ_MAX_BATCH);
+    TQ_REQUIRE(packed && scales && n_mat && O && I && out, "tq_dequant_batch: null array");
+    TQ_REQUIRE(!is_int4(fmt) || zeros != nullptr, "tq_dequant_batch: int4 needs zeros");
+    TQ_REQUIRE(fmt != TQ_NVFP4_G16 || global_scale != nullptr, "tq_dequant_batch: NVFP4 needs global_scale");
+    if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant_batch: out dtype %d", out_dtype);
+    for (int i = 0; i < n; ++i)
+        if ((s = check_dequant_unit(packed[i], fmt, scales[i], zeros ? zeros[i] : nullptr,
+                                    global_scale ? global_scale[i] : nullptr, n_mat[i], O[i], I[i], out[i],
+                                    "tq_dequant_batch")) != TQ_OK)
+            return s;
+    dispatch_dequant(n, packed, fmt, scales, zeros, global_scale, n_mat, O, I, out, out_dtype == TQ_BF16,
+                     reinterpret_cast<cudaStream_t>(stream));
+    return check_launch("tq_dequant_batch");
 }

@@ -62,6 +62,10 @@ typedef enum {
 
 typedef enum { TQ_F32 = 0, TQ_BF16 = 1 } tq_dtype;
 
+/* Most units one grouped call (tq_pack_batch, tq_dequant_batch,
+ * tq_proxy_error_batch) takes. */
+#define TQ_MAX_BATCH 16
+
 typedef enum {
     TQ_INT4_G128_ASYM = 4,   /* nibble codes q in [0,15], f32 scale, u8 zero per 128 weights */
     TQ_INT3_G64_SYM = 5,     /* two bit-planes, v in [-4,3] as v+4, f32 scale per 64 weights  */
@@ -215,6 +219,18 @@ tq_status tq_search_groups(const tq_mat* W, const float* m, int64_t m_stride, in
 tq_status tq_pack(const tq_mat* W, int32_t fmt, const void* scales, const uint8_t* zeros,
                   const float* global_scale, uint8_t* packed, tq_stream_t stream);
 
+/* tq_pack of n units in one launch (1 <= n <= TQ_MAX_BATCH; one format and
+ * one weight dtype; shapes free): unit i is W[i] with scales[i], zeros[i],
+ * global_scale[i], packed[i] as tq_pack takes them.  W and the pointer arrays
+ * are host arrays of n entries (zeros may be NULL when fmt is not int4,
+ * global_scale when it is not NVFP4).  The units share one wave of resident
+ * blocks, split by their sizes, so small matrices do not each pay a launch's
+ * ramp-up and tail.  Results are those of n tq_pack calls.  Errors as tq_pack,
+ * TQ_ERR_INVALID_ARG for n out of range or mixed dtypes. */
+tq_status tq_pack_batch(int32_t n, const tq_mat* W, int32_t fmt, const void* const* scales,
+                        const uint8_t* const* zeros, const float* const* global_scale,
+                        uint8_t* const* packed, tq_stream_t stream);
+
 /* Pack integer codes: `codes` is dense [rows][cols] bytes (int3: int8 v in
  * [-4,3]; int4: q in [0,15]; NVFP4: 4-bit E2M1 code, sign in bit 3).
  * Records ([INT3] Layout): int3 = 24 bytes per 64 weights, u = v + 4, low
@@ -238,6 +254,17 @@ tq_status tq_unpack_codes(const uint8_t* packed, int32_t fmt, int64_t rows, int6
 tq_status tq_dequant(const uint8_t* packed, int32_t fmt, const void* scales, const uint8_t* zeros,
                      const float* global_scale, int64_t n_mat, int64_t O, int64_t I, void* out,
                      int32_t out_dtype, tq_stream_t stream);
+
+/* tq_dequant of n units in one launch (1 <= n <= TQ_MAX_BATCH; one format
+ * and one out_dtype): unit i is packed[i], scales[i], zeros[i],
+ * global_scale[i], n_mat[i] x O[i] x I[i], out[i].  All arguments but fmt,
+ * out_dtype and stream are host arrays of n entries (zeros / global_scale
+ * may be NULL as in tq_pack_batch).  Results are those of n tq_dequant calls;
+ * errors as tq_dequant. */
+tq_status tq_dequant_batch(int32_t n, const uint8_t* const* packed, int32_t fmt, const void* const* scales,
+                           const uint8_t* const* zeros, const float* const* global_scale,
+                           const int64_t* n_mat, const int64_t* O, const int64_t* I, void* const* out,
+                           int32_t out_dtype, tq_stream_t stream);
 
 /* ------------------------------------------------------------------ dequant-GEMV
  * The decode-time consumer of the packed formats ([INT3] Design: Kernel
@@ -389,6 +416,20 @@ tq_status tq_proxy_error(const tq_mat* W, const uint8_t* packed, int32_t fmt, co
                          const uint8_t* zeros, const float* global_scale, const float* m,
                          int64_t m_stride, double* num, double* den, void* workspace,
                          size_t workspace_bytes, tq_stream_t stream);
+
+/* tq_proxy_error of n units in one launch (1 <= n <= TQ_MAX_BATCH; one
+ * format, one weight dtype): unit i is W[i], packed[i], scales[i], zeros[i],
+ * global_scale[i], m[i] (m_stride[i]) -> num[i][e], den[i][e].  W, m_stride
+ * and the pointer arrays are host arrays of n entries.  workspace: >=
+ * tq_proxy_batch_workspace_bytes(n, W, fmt), no initialisation needed.  The
+ * values are those of n tq_proxy_error calls up to the order of their fp64
+ * additions (fixed for a given device and batch); errors as tq_proxy_error. */
+size_t tq_proxy_batch_workspace_bytes(int32_t n, const tq_mat* W, int32_t fmt);
+tq_status tq_proxy_error_batch(int32_t n, const tq_mat* W, const uint8_t* const* packed, int32_t fmt,
+                               const void* const* scales, const uint8_t* const* zeros,
+                               const float* const* global_scale, const float* const* m,
+                               const int64_t* m_stride, double* const* num, double* const* den,
+                               void* workspace, size_t workspace_bytes, tq_stream_t stream);
 
 /* ------------------------------------------------------------------ proxy error, full Hessian
  * Per matrix e ([TT] "Risks to measure: Precision", H = X^T X of the

@@ -156,6 +156,19 @@ class _HostStandIn:
         out.copy_(scales.repeat_interleave(g, dim=2)[:, :, :I].to(out.dtype))
         return out
 
+    def proxy_batch_workspace_bytes(self, Ws, fmt):
+        return 16
+
+    def tq_dequant_batch(self, packed, fmt, scales, zeros, gs, shapes, out):
+        for i, (E, O, I) in enumerate(shapes):
+            self.tq_dequant(packed[i], fmt, scales[i], None, None, E, O, I, out=out[i])
+        return out
+
+    def tq_proxy_error_batch(self, Ws, packed, fmt, scales, zeros, gs, ms, out, workspace=None):
+        for i, W in enumerate(Ws):
+            self.tq_proxy_error(W, packed[i], fmt, scales[i], None, None, ms[i], out=out[i])
+        return out
+
     def tq_proxy_error(self, W, packed, fmt, scales, zeros, gs, m, out, workspace=None):
         mm = m if m.dim() == 2 else m.unsqueeze(0)
         w = W.double()
