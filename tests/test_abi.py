@@ -185,3 +185,34 @@ def test_binding_refuses_cpu_tensors(tq):
         tq.tq_gptq_sweep(W, tq.INT3_G64_SYM, torch.zeros(8), None, torch.eye(64))
     with pytest.raises(tq.TQError):
         tq.tq_hessian(torch.zeros(4, 64, dtype=torch.bfloat16))
+
+
+def test_grouped_calls_validate_before_any_launch(tq):
+    """tq_pack_batch / tq_dequant_batch / tq_proxy_error_batch: unit counts,
+    mixed dtypes, missing zero-points and bad shapes are refused on the host;
+    the workspace query follows the units' shapes."""
+    L = tq.lib()
+    fake = ctypes.c_void_p(0x1000)   # never dereferenced: validation fails first
+    V = ctypes.c_void_p
+    mats = (tq._Mat * 2)(tq._Mat(fake, 1, 0, 1, 8, 64, 64, 0), tq._Mat(fake, 0, 0, 1, 8, 64, 64, 0))
+    ptrs = (V * 2)(0x1000, 0x2000)
+    for n in (0, tq.MAX_BATCH + 1):
+        assert L.tq_pack_batch(n, mats, tq.INT3_G64_SYM, ptrs, None, None, ptrs, None) == 1
+        assert b"outside" in L.tq_last_error_string()
+    assert L.tq_pack_batch(2, mats, tq.INT3_G64_SYM, ptrs, None, None, ptrs, None) == 1   # bf16 + fp32
+    assert b"dtypes" in L.tq_last_error_string()
+    assert L.tq_pack_batch(1, mats, tq.INT4_G128_ASYM, ptrs, None, None, ptrs, None) == 1  # no zeros
+    assert L.tq_pack_batch(1, mats, 99, ptrs, None, None, ptrs, None) == 2
+    i64 = ctypes.c_int64 * 2
+    assert L.tq_dequant_batch(2, ptrs, tq.INT3_G64_SYM, ptrs, None, None, i64(1, 1), i64(8, 0), i64(64, 64),
+                              ptrs, 1, None) == 1   # empty shape in unit 1
+    assert b"empty" in L.tq_last_error_string()
+    assert L.tq_dequant_batch(1, ptrs, tq.NVFP4_G16, ptrs, None, None, i64(1, 1), i64(8, 8), i64(64, 64),
+                              ptrs, 1, None) == 1   # NVFP4 without global scales
+    one = L.tq_proxy_batch_workspace_bytes(1, mats, tq.INT3_G64_SYM)
+    assert one == L.tq_proxy_workspace_bytes(mats, tq.INT3_G64_SYM) and one > 0
+    assert L.tq_proxy_batch_workspace_bytes(2, mats, tq.INT3_G64_SYM) > one
+    assert L.tq_proxy_batch_workspace_bytes(tq.MAX_BATCH + 1, mats, tq.INT3_G64_SYM) == 0
+    assert L.tq_proxy_error_batch(1, mats, ptrs, tq.INT3_G64_SYM, ptrs, None, None, ptrs, i64(0, 0), ptrs, ptrs,
+                                  fake, 8, None) == 1   # workspace too small
+    assert b"workspace" in L.tq_last_error_string()
