@@ -63,7 +63,7 @@ SEARCH_INSTR_PER_W = {"int3_g64_sym": 96 * 7, "int4_g128_asym": 1024 * 5, "nvfp4
 SEARCH_CEE_PER_W = {"int3_g64_sym": 96, "int4_g128_asym": 1024, "nvfp4_g16": 16}
 # our kernels per call: imatrix 2 (partial + final), search 1 (NVFP4: amax +
 # global + search = 3), dequant 1, proxy 1
-KERNELS = {"imatrix": 2, "search": {"int3_g64_sym": 1, "int4_g128_asym": 1, "nvfp4_g16": 3},
+KERNELS = {"imatrix": 1, "search": {"int3_g64_sym": 1, "int4_g128_asym": 1, "nvfp4_g16": 3},
            "dequant": 1, "proxy": 1}
 
 
@@ -804,6 +804,8 @@ def run_workload(tq, name, args, world, rank, dev, barrier, pk, keep_wl=False):
         d[2] += 1
     hbm_rows = {}
     kname = {"imatrix": "k_imatrix_partial", "dequant": "k_dequant", "proxy": "k_proxy"}
+    if step.grouped:   # one grouped launch per row for all units
+        kname.update(dequant="k_dequant_batch", proxy="k_proxy_batch")
     for rname, (t_ms, nb, cnt) in rows.items():
         gbs = nb / (t_ms * 1e-3) / 1e9
         p = read_profile(args.profile_table, name, kname[rname])

@@ -7,9 +7,11 @@
 // consecutive columns (16-byte loads, VEC = 8 bf16 / 4 fp32 per lane) and a
 // slice of tokens; its 8 warps walk interleaved tokens with 4 loads in
 // flight each.  Squares are summed in fp32 over runs of 32 tokens and folded
-// into fp64; the 8 warps are combined in shared memory and each (slice,
-// column) partial is written to the caller's workspace.  A second kernel adds
-// the slices in a fixed order, so results do not depend on scheduling.
+// into fp64; the 8 warps are combined in shared memory.  With one token
+// slice per column tile the block writes m itself; with several, each
+// (slice, column) partial goes to the caller's workspace and the last slice
+// block of the tile to finish (atomic ticket) adds the slices in slice order,
+// so results do not depend on scheduling.
 #include "tq_internal.cuh"
 
 #include <mutex>
@@ -110,10 +112,26 @@ inline ImGeom im_geometry(const tq_mat* X) {
     return g;
 }
 
+inline int64_t im_ticket_bytes(const ImGeom& g, int64_t n_mat) { return ((g.col_tiles * n_mat * 4 + 15) / 16) * 16; }
+
+// Writes one (matrix, column) result: alpha * s rounded once to fp32, added
+// to the existing m when accumulating.
+__device__ __forceinline__ void im_store(float* __restrict__ m, int64_t idx, double s, double alpha, int accumulate) {
+    float v = static_cast<float>(alpha * s);
+    if (accumulate) v = __fadd_rn(m[idx], v);
+    m[idx] = v;
+}
+
+// Each block sums its token slice of one column tile; with one slice it
+// writes m itself, otherwise it writes its fp64 partial and the last slice
+// block of the (tile, matrix) to finish (atomic ticket) adds the slices'
+// partials in slice order and writes m.
 template <typename T>
 __global__ void __launch_bounds__(IM_THREADS, IM_RESIDENT)
 k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, int64_t ms,
-                  int64_t tps, double* __restrict__ partial, int64_t n_mat) {
+                  int64_t tps, double* __restrict__ partial, int64_t n_mat, int64_t slices,
+                  unsigned* __restrict__ tickets, float* __restrict__ m, int64_t m_stride, double alpha,
+                  int accumulate) {
     constexpr int VEC = VecOf<T>::n;
     __shared__ double red[IM_WARPS][32 * VEC];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -187,33 +205,31 @@ k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, in
 #pragma unroll
         for (int w = 0; w < IM_WARPS; ++w) s += red[w][c];
         const int64_t j = tile * 32 * VEC + c;
-        if (j < I) partial[(slice * n_mat + e) * I + j] = s;
+        if (j < I) {
+            if (slices == 1) im_store(m, e * m_stride + j, 0.0 + s, alpha, accumulate);
+            else partial[(slice * n_mat + e) * I + j] = s;
+        }
+    }
+    if (slices == 1) return;   // block-uniform
+    __shared__ bool last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+        last = atomicAdd(tickets + e * gridDim.x + tile, 1u) == static_cast<unsigned>(slices - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
+    for (int c = threadIdx.x; c < 32 * VEC; c += IM_THREADS) {   // slices added in order, as one pass would
+        const int64_t j = tile * 32 * VEC + c;
+        if (j >= I) continue;
+        const double* p = partial + e * I + j;
+        const int64_t step = n_mat * I;
+        double s = 0.0;
+        for (int64_t k = 0; k < slices; ++k) s += __ldcg(p + k * step);
+        im_store(m, e * m_stride + j, s, alpha, accumulate);
     }
 }
 
-__global__ void k_imatrix_final(const double* __restrict__ partial, int64_t slices, int64_t n_mat,
-                                int64_t I, float* __restrict__ m, int64_t m_stride, double alpha,
-                                int accumulate) {
-    const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-    if (idx >= n_mat * I) return;
-    const int64_t e = idx / I, j = idx - e * I;
-    const double* p = partial + e * I + j;
-    const int64_t step = n_mat * I;
-    double s = 0.0;
-    int64_t k = 0;
-    for (; k + 8 <= slices; k += 8) {   // 8 loads in flight, added in slice order
-        double v[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = __ldg(p + (k + u) * step);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) s += v[u];
-    }
-    for (; k < slices; ++k) s += __ldg(p + k * step);
-    float v = static_cast<float>(alpha * s);
-    float* dst = m + e * m_stride + j;
-    if (accumulate) v = __fadd_rn(*dst, v);
-    *dst = v;
-}
 
 // ------------------------------------------------------------------ amax
 
@@ -297,7 +313,8 @@ using namespace tq;
 TQ_API size_t tq_imatrix_workspace_bytes(const tq_mat* X) {
     if (!X || X->n_mat < 1 || X->rows < 1 || X->cols < 1 || elem_bytes(X->dtype) == 0) return 0;
     const ImGeom g = im_geometry(X);
-    return static_cast<size_t>(g.slices * X->n_mat * X->cols) * sizeof(double);
+    if (g.slices == 1) return 16;   // one slice: m is written directly, nothing is kept between blocks
+    return static_cast<size_t>(im_ticket_bytes(g, X->n_mat) + g.slices * X->n_mat * X->cols * sizeof(double));
 }
 
 TQ_API tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float alpha, int32_t accumulate,
@@ -312,20 +329,26 @@ TQ_API tq_status tq_imatrix(const tq_mat* X, float* m, int64_t m_stride, float a
     TQ_REQUIRE(workspace_bytes >= need, "tq_imatrix: workspace too small (%zu < %zu bytes)", workspace_bytes, need);
     const ImGeom g = im_geometry(X);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    double* partial = static_cast<double*>(workspace);
+    // workspace: the tickets (one per column tile and matrix), then the partials
+    const int64_t tick = im_ticket_bytes(g, X->n_mat);
+    unsigned* tickets = static_cast<unsigned*>(workspace);
+    double* partial = reinterpret_cast<double*>(static_cast<uint8_t*>(workspace) + tick);
+    if (g.slices > 1) {
+        const cudaError_t ce = cudaMemsetAsync(tickets, 0, static_cast<size_t>(g.col_tiles * X->n_mat) * 4, st);
+        if (ce != cudaSuccess) return set_error(TQ_ERR_CUDA, "tq_imatrix: %s", cudaGetErrorString(ce));
+    }
     const dim3 grid(static_cast<unsigned>(g.col_tiles), static_cast<unsigned>(g.slices), static_cast<unsigned>(X->n_mat));
     const int64_t ms = X->n_mat > 1 ? X->mat_stride : 0;
+    const int64_t mst = X->n_mat > 1 ? m_stride : 0;
     if (X->dtype == TQ_BF16)
-        k_imatrix_partial<uint16_t><<<grid, IM_THREADS, 0, st>>>(static_cast<const uint16_t*>(X->ptr), X->rows, X->cols,
-                                                                 X->ld, ms, g.tokens_per_slice, partial, X->n_mat);
+        k_imatrix_partial<uint16_t><<<grid, IM_THREADS, 0, st>>>(
+            static_cast<const uint16_t*>(X->ptr), X->rows, X->cols, X->ld, ms, g.tokens_per_slice, partial, X->n_mat,
+            g.slices, tickets, m, mst, static_cast<double>(alpha), accumulate);
     else
-        k_imatrix_partial<float><<<grid, IM_THREADS, 0, st>>>(static_cast<const float*>(X->ptr), X->rows, X->cols,
-                                                              X->ld, ms, g.tokens_per_slice, partial, X->n_mat);
-    if ((s = check_launch("imatrix partial")) != TQ_OK) return s;
-    const int64_t n = X->n_mat * X->cols;
-    k_imatrix_final<<<static_cast<unsigned>((n + 255) / 256), 256, 0, st>>>(
-        partial, g.slices, X->n_mat, X->cols, m, X->n_mat > 1 ? m_stride : 0, static_cast<double>(alpha), accumulate);
-    return check_launch("imatrix final");
+        k_imatrix_partial<float><<<grid, IM_THREADS, 0, st>>>(
+            static_cast<const float*>(X->ptr), X->rows, X->cols, X->ld, ms, g.tokens_per_slice, partial, X->n_mat,
+            g.slices, tickets, m, mst, static_cast<double>(alpha), accumulate);
+    return check_launch("imatrix");
 }
 
 // ------------------------------------------------------------------ allocation-free variant

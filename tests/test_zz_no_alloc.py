@@ -3,6 +3,8 @@ device memory where they call it (an engine hook handed only its buffers, or
 memory fully planned by an arena): through the C ABI it must give the same
 imatrix as tq_imatrix with a caller workspace, call after call, while its
 scratch lives in the library.  Collected last on purpose."""
+import ctypes
+
 import pytest
 import torch
 
@@ -46,8 +48,16 @@ def test_static_scratch_accumulates_and_rejects_oversize():
     torch.cuda.synchronize()
     assert _rel(m, ref) <= 1e-5
     cap = tq.tq_imatrix_static_capacity()
-    # one slice of one 2^20-column matrix already needs 8 MiB of partials
-    big = torch.empty((64, 1 << 20), dtype=torch.bfloat16, device="cuda")
-    assert cap < 8 << 20
-    with pytest.raises(tq.TQError, match="scratch"):
-        tq.tq_imatrix_static(big)
+    # A shape whose fp64 token-slice partials exceed the fixed scratch: one
+    # column tile more than a wave of blocks, over 2^24 tokens, splits into
+    # many slices.  The call is refused on the host, before any launch, so
+    # the descriptor's pointer is never read.
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cols = (4 * sms + 1) * 256
+    L = tq.lib()
+    fake = ctypes.c_void_p(0x1000)
+    d = tq._Mat(fake, 1, 0, 1, 1 << 24, cols, cols, 0)   # bf16 [1, 2^24, cols], never dereferenced
+    assert L.tq_imatrix_workspace_bytes(ctypes.byref(d)) > cap
+    m_dev = torch.empty(cols, dtype=torch.float32, device="cuda")
+    st = L.tq_imatrix_static(ctypes.byref(d), ctypes.c_void_p(m_dev.data_ptr()), cols, ctypes.c_float(1.0), 0, None)
+    assert st == 1 and b"scratch" in L.tq_last_error_string()
