@@ -45,18 +45,23 @@
 
 namespace tq {
 
-constexpr int GV_WARPS = 8;
-constexpr int GV_THREADS = GV_WARPS * 32;
-constexpr int64_t GV_XS_BYTES = 72 * 1024;   // x tile budget: three blocks per SM
+// Warps per block and x tile budget (bytes of shared memory per block):
+// B = 1 runs GV_WARPS1 warps per block, more vectors 8 warps at up to 128
+// registers (two blocks per SM).
+constexpr int GV_WARPS1 = 8;
+template <int B> __host__ __device__ constexpr int gv_warps() { return B == 1 ? GV_WARPS1 : 8; }
+template <int B> __host__ __device__ constexpr int gv_threads() { return gv_warps<B>() * 32; }
+template <int B> __host__ __device__ constexpr int64_t gv_xs_bytes() { return B == 1 ? 216 * 1024 * GV_WARPS1 / 24 : 72 * 1024; }
 
 template <int B> __host__ __device__ constexpr int gv_rows() { return B <= 2 ? 4 : 2; }   // rows per warp
-template <int B> __host__ __device__ constexpr int gv_min_blocks() { return B == 1 ? 3 : 2; }   // per SM
+template <int B> __host__ __device__ constexpr int gv_min_blocks() { return B == 1 ? 24 / GV_WARPS1 : 2; }   // per SM
 constexpr bool GV_DB = false;   // double-buffered code loads (measured slower)
 
 // Columns of x per staged tile: a multiple of 1024 (32 lanes x 32 weights),
 // no more than the row needs.
-inline int64_t gv_tile(int64_t B, int64_t I) {
-    int64_t k = GV_XS_BYTES / (B * 4 * 1024);
+template <int B>
+inline int64_t gv_tile(int64_t I) {
+    int64_t k = gv_xs_bytes<B>() / (B * 4 * 1024);
     k = k < 1 ? 1 : k;
     const int64_t need = (I + 1023) / 1024;
     return 1024 * (need < k ? need : k);
@@ -66,50 +71,49 @@ inline int64_t gv_tile(int64_t B, int64_t I) {
 // I).  Slot i (0..7) of a lane's quad holds 4 of the quad's 32 columns:
 // 4i .. 4i + 3 (int4, NVFP4), or i, 8 + i, 16 + i, 24 + i (int3: the
 // columns at position i of the quad's 4 octets, in the order its decoding
-// produces them).
+// produces them).  A thread stages one quad (32 columns) at a time: four
+// 16-byte loads of bf16 x (eight of fp32) where the quad lies inside the row
+// and vec (16-byte aligned rows) holds, then its 8 slots.
 template <bool OCT_MAJOR>
 __device__ __forceinline__ void gv_stage(float4* xs, const void* x, bool x_bf16, int64_t xoff, int64_t I,
                                          int64_t j0, int64_t TI, int B, bool vec) {
-    const int64_t slots = TI >> 2;   // float4 slots per vector, a multiple of GV_THREADS
+    const int64_t slots = TI >> 2;   // float4 slots per vector
+    const int64_t nqt = TI >> 5;     // quads of the tile
     for (int b = 0; b < B; ++b) {
-        for (int64_t s = threadIdx.x; s < slots; s += GV_THREADS) {
-            const int64_t l = s & 31, ti = s >> 5;
-            const int64_t jq = j0 + ((ti >> 3) * 32 + l) * 32;   // the quad's first column
-            const int i = static_cast<int>(ti & 7);
-            const int64_t base = xoff + b * I;
-            float f[4];
-            if (OCT_MAJOR) {
+        const int64_t base = xoff + b * I;
+        for (int64_t qd = threadIdx.x; qd < nqt; qd += blockDim.x) {
+            const int64_t jq = j0 + qd * 32;   // the quad's first column
+            float4* dst = xs + b * slots + (qd >> 5) * 256 + (qd & 31);   // slot i of the quad at dst[32 i]
+            if (vec && x_bf16 && jq + 31 < I) {   // raw bf16 words, widened as the slots are written
+                const uint4* p = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + base + jq);
+                uint32_t w[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 u = __ldg(p + v);
+                    w[4 * v] = u.x; w[4 * v + 1] = u.y; w[4 * v + 2] = u.z; w[4 * v + 3] = u.w;
+                }
+                auto col = [&](int c) {   // column c of the quad: word c / 2, low half for even c
+                    return __uint_as_float((c & 1) ? (w[c >> 1] & 0xffff0000u) : (w[c >> 1] << 16));
+                };
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dst[32 * i] = OCT_MAJOR ? make_float4(col(i), col(8 + i), col(16 + i), col(24 + i))
+                                            : make_float4(col(4 * i), col(4 * i + 1), col(4 * i + 2), col(4 * i + 3));
+                continue;
+            }
+            // fp32 x, or a quad at the row's end / rows not 16-byte aligned: slot by slot
+#pragma unroll 1
+            for (int i = 0; i < 8; ++i) {
+                float f[4];
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    const int64_t j = jq + 8 * c + i;
+                    const int64_t j = jq + (OCT_MAJOR ? 8 * c + i : 4 * i + c);
                     f[c] = j < I ? (x_bf16 ? bf16_bits_to_f32(__ldg(static_cast<const uint16_t*>(x) + base + j))
                                            : __ldg(static_cast<const float*>(x) + base + j))
                                  : 0.f;
                 }
-            } else {
-                const int64_t j = jq + 4 * i;
-                if (x_bf16) {
-                    const uint16_t* p = static_cast<const uint16_t*>(x) + base + j;
-                    if (vec && j + 3 < I) {
-                        const uint2 u = __ldg(reinterpret_cast<const uint2*>(p));
-                        f[0] = __uint_as_float(u.x << 16); f[1] = __uint_as_float(u.x & 0xffff0000u);
-                        f[2] = __uint_as_float(u.y << 16); f[3] = __uint_as_float(u.y & 0xffff0000u);
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) f[c] = j + c < I ? bf16_bits_to_f32(__ldg(p + c)) : 0.f;
-                    }
-                } else {
-                    const float* p = static_cast<const float*>(x) + base + j;
-                    if (vec && j + 3 < I) {
-                        const float4 v = __ldg(reinterpret_cast<const float4*>(p));
-                        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
-                    } else {
-#pragma unroll
-                        for (int c = 0; c < 4; ++c) f[c] = j + c < I ? __ldg(p + c) : 0.f;
-                    }
-                }
+                dst[32 * i] = make_float4(f[0], f[1], f[2], f[3]);
             }
-            xs[b * slots + s] = make_float4(f[0], f[1], f[2], f[3]);
         }
     }
 }
@@ -328,7 +332,7 @@ __device__ __forceinline__ void gv_quad(const Quad (&u)[R], const float4* xq, in
 // per matrix.  Each lane's next quads are loaded before the current ones
 // are used.
 template <int FMT, int B, bool A16>
-__global__ void __launch_bounds__(GV_THREADS, gv_min_blocks<B>())
+__global__ void __launch_bounds__(gv_threads<B>(), gv_min_blocks<B>())
 k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scales,
                const uint8_t* __restrict__ zeros, const float* __restrict__ gs, int64_t n_mat, int64_t O,
                int64_t I, const void* __restrict__ x, int x_bf16, int64_t x_ms, int64_t TI, int64_t cpm, int wl,
@@ -336,6 +340,7 @@ k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scal
     constexpr int R = gv_rows<B>();
     using F = FmtTraits<FMT>;
     extern __shared__ float4 xs[];
+    constexpr int GV_WARPS = gv_warps<B>();
     __shared__ float red[GV_WARPS][R * B];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int slice = warp & ((1 << wl) - 1), rgi = warp >> wl;
@@ -345,26 +350,31 @@ k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scal
     const int64_t nT = (I + TI - 1) / TI;             // column tiles
     const int64_t slots = TI >> 2;
     const int qstep = 32 << wl;
-    const bool vec = (I % 4) == 0 && (x_ms % 4) == 0;
+    // 16-byte x loads: rows (and matrices) of x start on 16-byte boundaries
+    const int64_t xa = x_bf16 ? 8 : 4;
+    const bool vec = (I % xa) == 0 && (x_ms % xa) == 0;
     const int64_t nchunks = n_mat * cpm;
     const int64_t c0 = nchunks * blockIdx.x / gridDim.x, c1 = nchunks * (blockIdx.x + 1) / gridDim.x;
     int64_t staged_e = -1, staged_t = -1;
-    for (int64_t c = c0; c < c1; ++c) {
-        const int64_t e = c / cpm;
-        const int64_t ob = (c - e * cpm) * rows_per_chunk + rgi * R;
-        const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
-        const int64_t ofirst = min(ob, O - 1);
-        int rr[R];   // rows relative to the first; rows past O repeat the last one and are not stored
+    // Column tiles outermost: x is staged once per tile (and matrix, where x
+    // is per matrix) for all of the block's chunks, and each row's y adds the
+    // tiles' partial sums in tile order (the block owns its rows).
+    for (int64_t t = 0; t < nT; ++t) {
+        const int64_t qb = t * (TI >> 5);
+        const int nqt = static_cast<int>(min(TI >> 5, nq - qb));
+        for (int64_t c = c0; c < c1; ++c) {
+            const int64_t e = c / cpm;
+            const int64_t ob = (c - e * cpm) * rows_per_chunk + rgi * R;
+            const float g = FMT == TQ_NVFP4_G16 ? __ldg(gs + e) : 0.f;
+            const int64_t ofirst = min(ob, O - 1);
+            int rr[R];   // rows relative to the first; rows past O repeat the last one and are not stored
 #pragma unroll
-        for (int r = 0; r < R; ++r) rr[r] = static_cast<int>(min(ob + r, O - 1) - ofirst);
-        float acc[R][B];
+            for (int r = 0; r < R; ++r) rr[r] = static_cast<int>(min(ob + r, O - 1) - ofirst);
+            float acc[R][B];
 #pragma unroll
-        for (int r = 0; r < R; ++r)
+            for (int r = 0; r < R; ++r)
 #pragma unroll
-            for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
-        for (int64_t t = 0; t < nT; ++t) {
-            const int64_t qb = t * (TI >> 5);
-            const int nqt = static_cast<int>(min(TI >> 5, nq - qb));
+                for (int b = 0; b < B; ++b) acc[r][b] = 0.f;
             int qt = slice * 32 + lane;   // quad within the tile
             bool have = qt < nqt;
             GvRows<FMT, A16, R> rw;
@@ -405,30 +415,36 @@ k_dequant_gemv(const uint8_t* __restrict__ packed, const void* __restrict__ scal
                 qt = qn;
                 have = hn;
             }
-        }
 #pragma unroll
-        for (int r = 0; r < R; ++r) {
+            for (int r = 0; r < R; ++r) {
 #pragma unroll
-            for (int b = 0; b < B; ++b) {
-                float s = acc[r][b];
+                for (int b = 0; b < B; ++b) {
+                    float s = acc[r][b];
 #pragma unroll
-                for (int off = 16; off; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(FULL, s, off));
-                if (wl == 0) {
-                    if (lane == 0 && ob + r < O) y[(e * B + b) * O + ob + r] = s;
-                } else if (lane == 0) {
-                    red[warp][r * B + b] = s;
+                    for (int off = 16; off; off >>= 1) s = __fadd_rn(s, __shfl_xor_sync(FULL, s, off));
+                    if (wl == 0) {
+                        if (lane == 0 && ob + r < O) {
+                            float* yp = y + (e * B + b) * O + ob + r;
+                            *yp = t == 0 ? s : __fadd_rn(*yp, s);
+                        }
+                    } else if (lane == 0) {
+                        red[warp][r * B + b] = s;
+                    }
                 }
             }
-        }
-        if (wl != 0) {   // block-uniform: add the slices' sums in slice order
-            __syncthreads();
-            if (slice == 0 && lane < R * B) {
-                float s = red[warp][lane];
-                for (int k = 1; k < (1 << wl); ++k) s = __fadd_rn(s, red[warp + k][lane]);
-                const int r = lane / B, b = lane - (lane / B) * B;
-                if (ob + r < O) y[(e * B + b) * O + ob + r] = s;
+            if (wl != 0) {   // block-uniform: add the slices' sums in slice order
+                __syncthreads();
+                if (slice == 0 && lane < R * B) {
+                    float s = red[warp][lane];
+                    for (int k = 1; k < (1 << wl); ++k) s = __fadd_rn(s, red[warp + k][lane]);
+                    const int r = lane / B, b = lane - (lane / B) * B;
+                    if (ob + r < O) {
+                        float* yp = y + (e * B + b) * O + ob + r;
+                        *yp = t == 0 ? s : __fadd_rn(*yp, s);
+                    }
+                }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
 }
@@ -442,12 +458,13 @@ int gv_blocks_per_sm(int64_t TI, size_t smem) {
     static std::once_flag raised;
     auto kern = k_dequant_gemv<FMT, B, A16>;
     std::call_once(raised, [&] {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(GV_XS_BYTES));
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(gv_xs_bytes<B>()));
     });
     const int64_t i = TI / 1024;
     int n = i < 25 ? cache[i].load(std::memory_order_relaxed) : 0;
     if (n == 0) {
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, GV_THREADS, smem) != cudaSuccess || n < 1) n = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, gv_threads<B>(), smem) != cudaSuccess || n < 1)
+            n = 1;
         if (i < 25) cache[i].store(n, std::memory_order_relaxed);
     }
     return n;
@@ -457,7 +474,8 @@ template <int FMT, int B, bool A16>
 void launch_gemv(const uint8_t* packed, const void* scales, const uint8_t* zeros, const float* gs, int64_t n_mat,
                  int64_t O, int64_t I, const void* x, bool x_bf16, int64_t x_ms, float* y, cudaStream_t st) {
     constexpr int R = gv_rows<B>();
-    const int64_t TI = gv_tile(B, I);
+    constexpr int GV_WARPS = gv_warps<B>();
+    const int64_t TI = gv_tile<B>(I);
     const size_t smem = static_cast<size_t>(B * TI * 4);
     const int per_sm = gv_blocks_per_sm<FMT, B, A16>(TI, smem);
     const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
@@ -469,7 +487,7 @@ void launch_gemv(const uint8_t* packed, const void* scales, const uint8_t* zeros
     while (wl < 3 && chunks(wl) < slots && nq >= (static_cast<int64_t>(32) << (wl + 1))) ++wl;
     const int64_t cpm = (O + (GV_WARPS >> wl) * R - 1) / ((GV_WARPS >> wl) * R);
     const int64_t grid = min(n_mat * cpm, slots);
-    k_dequant_gemv<FMT, B, A16><<<static_cast<unsigned>(grid), GV_THREADS, smem, st>>>(
+    k_dequant_gemv<FMT, B, A16><<<static_cast<unsigned>(grid), gv_threads<B>(), smem, st>>>(
         packed, scales, zeros, gs, n_mat, O, I, x, x_bf16 ? 1 : 0, x_ms, TI, cpm, wl, y);
 }
 
