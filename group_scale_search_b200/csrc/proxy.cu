@@ -35,7 +35,11 @@ constexpr int PX_NO = 2;
 // Measured on the full-size workloads: one block of four walkers per SM
 // beat four one-walker blocks (0.550 -> 0.486 ms on the int3 MoE stack,
 // 0.027 -> 0.026 ms on the dense q projection, even on the NVFP4 stack).
+// At launch the walkers fill a block of up to 1024 threads (tiles narrower
+// than 256 columns get more walkers: 5 for the NVFP4 stack's 192-wide tiles,
+// 0.378 -> 0.343 ms); PX_PY sets the register bound.
 constexpr int PX_PY = 4;
+constexpr bool PX_FILL = true;
 
 inline int64_t px_cols(int64_t I) { return ((I + 7) / 8 + PX_NO - 1) / PX_NO; }
 
@@ -285,13 +289,15 @@ void launch_proxy(int n, const tq_mat* W, const uint8_t* const* packed, const vo
     auto kern = direct ? reinterpret_cast<const void*>(k_proxy<FMT, T, PX_NO>)
                        : reinterpret_cast<const void*>(k_proxy_batch<FMT, T, PX_NO>);
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, static_cast<int>(width) * PX_PY, 0) !=
+    // as many walkers as fill a block of up to 1024 threads (narrow tiles: more walkers)
+    const int py = PX_FILL ? static_cast<int>(min(static_cast<int64_t>(8), 1024 / width)) : PX_PY;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, static_cast<int>(width) * py, 0) !=
             cudaSuccess ||
         per_sm < 1)
         per_sm = 1;
     const int64_t slots = min(static_cast<int64_t>(num_sms()) * per_sm, PX_MAX_BLOCKS);
     const int64_t blocks = batch_split(n, cols, rows, slots, sl, &width);
-    const dim3 block(static_cast<unsigned>(width), static_cast<unsigned>(PX_PY));
+    const dim3 block(static_cast<unsigned>(width), static_cast<unsigned>(py));
     if (direct) {
         const dim3 grid(static_cast<unsigned>(sl[0].cblocks), static_cast<unsigned>(sl[0].rblocks));
         k_proxy<FMT, T, PX_NO><<<grid, block, 0, st>>>(
