@@ -806,6 +806,8 @@ def run_workload(tq, name, args, world, rank, dev, barrier, pk, keep_wl=False):
     kname = {"imatrix": "k_imatrix_partial", "dequant": "k_dequant", "proxy": "k_proxy"}
     if step.grouped:   # one grouped launch per row for all units
         kname.update(dequant="k_dequant_batch", proxy="k_proxy_batch")
+    elif fmt_main == "int3_g64_sym":   # the int3 proxy runs the grouped kernel for one unit too
+        kname.update(proxy="k_proxy_batch")
     for rname, (t_ms, nb, cnt) in rows.items():
         gbs = nb / (t_ms * 1e-3) / 1e9
         p = read_profile(args.profile_table, name, kname[rname])
