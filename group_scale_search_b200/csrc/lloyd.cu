@@ -36,6 +36,8 @@ constexpr int LM_SUMS = 9;   // num[4] = sum omega u, den[4] = sum omega per lev
 // groups (4 octets per group), so a group is 4 consecutive threads.
 struct LmGeom {
     int64_t rows, I, G, per_row;   // per_row = 4 G octets
+    GroupIndex gi;                 // octet t -> (matrix, row, octet of the row), 32-bit (< 2^32 octets)
+    FastDiv pr;                    // octet t -> row of the flattened batch
 };
 
 template <typename T>
@@ -46,11 +48,13 @@ __global__ void k_lm_scales(const T* __restrict__ W, int64_t O, int64_t ld, int6
         const int64_t t = t0 + threadIdx.x;
         float a = 0.f;
         if (t < total) {
-            const int64_t row = t / g.per_row, c = t - row * g.per_row, e = row / O, o = row - e * O;
-            const int64_t j = c << 3;
+            uint32_t e, o, c;
+            g.gi.split(static_cast<uint32_t>(t), e, o, c);
+            const int64_t j = static_cast<int64_t>(c) << 3;
             if (j < g.I) {
                 Oct<T> oc;
-                oc.load(W + e * ms + o * ld + j, static_cast<int>(min(static_cast<int64_t>(8), g.I - j)));
+                oc.load(W + static_cast<int64_t>(e) * ms + static_cast<int64_t>(o) * ld + j,
+                        static_cast<int>(min(static_cast<int64_t>(8), g.I - j)));
                 float w[8];
                 oc.get(w);
 #pragma unroll
@@ -98,16 +102,17 @@ k_lm_pass(const T* __restrict__ W, int64_t O, int64_t ld, int64_t ms, const floa
     const int64_t total = g.rows * g.per_row;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t row = t / g.per_row, c = t - row * g.per_row, e = row / O, o = row - e * O;
-        const int64_t j = c << 3;
+        uint32_t e, o, c;
+        g.gi.split(static_cast<uint32_t>(t), e, o, c);
+        const int64_t j = static_cast<int64_t>(c) << 3;
         if (j >= g.I) continue;
         const int n = static_cast<int>(min(static_cast<int64_t>(8), g.I - j));
         Oct<T> oc;
-        oc.load(W + e * ms + o * ld + j, n);
+        oc.load(W + static_cast<int64_t>(e) * ms + static_cast<int64_t>(o) * ld + j, n);
         float w[8];
         oc.get(w);
         Oct<float> mo;
-        mo.load(m + e * m_stride + j, n);
+        mo.load(m + static_cast<int64_t>(e) * m_stride + j, n);
         float mv[8];
         mo.get(mv);
         const float s = __ldg(scales + (t >> 2));
@@ -185,13 +190,14 @@ __global__ void k_lm_pack(const T* __restrict__ W, int64_t O, int64_t ld, int64_
     const int64_t total = g.rows * g.per_row;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t row = t / g.per_row, c = t - row * g.per_row, e = row / O, o = row - e * O;
-        const int64_t j = c << 3;
+        uint32_t e, o, c;
+        g.gi.split(static_cast<uint32_t>(t), e, o, c);
+        const int64_t j = static_cast<int64_t>(c) << 3;
         unsigned bits = 0u;
         if (j < g.I) {
             const int n = static_cast<int>(min(static_cast<int64_t>(8), g.I - j));
             Oct<T> oc;
-            oc.load(W + e * ms + o * ld + j, n);
+            oc.load(W + static_cast<int64_t>(e) * ms + static_cast<int64_t>(o) * ld + j, n);
             float w[8];
             oc.get(w);
             const LmDiv dv(__ldg(scales + (t >> 2)));
@@ -213,7 +219,7 @@ __global__ void k_lm_dequant(const uint8_t* __restrict__ packed, const float* __
     const int64_t total = g.rows * g.per_row;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
          t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t row = t / g.per_row, c = t - row * g.per_row;
+        const int64_t row = g.pr.div(static_cast<uint32_t>(t)), c = t - row * g.per_row;
         const int64_t j = c << 3;
         if (j >= g.I) continue;
         const int n = static_cast<int>(min(static_cast<int64_t>(8), g.I - j));
@@ -233,9 +239,12 @@ __global__ void k_lm_dequant(const uint8_t* __restrict__ packed, const float* __
     }
 }
 
-static LmGeom lm_geom(int64_t rows, int64_t I) {
+// O: rows per matrix (the flattened rows are n_mat * O).
+static LmGeom lm_geom(int64_t rows, int64_t O, int64_t I) {
     LmGeom g;
     g.rows = rows; g.I = I; g.G = (I + 31) / 32; g.per_row = 4 * g.G;
+    g.gi = GroupIndex(O, g.per_row);
+    g.pr = FastDiv(static_cast<uint32_t>(g.per_row));
     return g;
 }
 
@@ -251,7 +260,7 @@ using namespace tq;
 
 TQ_API size_t tq_lloyd_workspace_bytes(const tq_mat* W) {
     if (!W || W->n_mat < 1 || W->rows < 1 || W->cols < 1) return 0;
-    const LmGeom g = lm_geom(W->n_mat * W->rows, W->cols);
+    const LmGeom g = lm_geom(W->n_mat * W->rows, W->rows, W->cols);
     return static_cast<size_t>(lm_blocks(g.rows * g.per_row) * LM_SUMS * 8);
 }
 
@@ -268,8 +277,10 @@ TQ_API tq_status tq_lloyd_max_g32(const tq_mat* W, const float* m, int64_t m_str
     TQ_REQUIRE(packed == nullptr || aligned16(packed), "tq_lloyd_max_g32: packed not 16-byte aligned");
     TQ_REQUIRE(n_iter >= 0 && n_iter <= 1000, "tq_lloyd_max_g32: n_iter in [0, 1000]");
     TQ_REQUIRE(workspace_bytes >= tq_lloyd_workspace_bytes(W), "tq_lloyd_max_g32: workspace too small");
+    TQ_REQUIRE(W->n_mat * W->rows * 4 * ((W->cols + 31) / 32) < (int64_t(1) << 32),
+               "tq_lloyd_max_g32: more than 2^32 octets of weights in one call");
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const LmGeom g = lm_geom(W->n_mat * W->rows, W->cols);
+    const LmGeom g = lm_geom(W->n_mat * W->rows, W->rows, W->cols);
     const int64_t ms = W->n_mat > 1 ? W->mat_stride : 0, mst = W->n_mat > 1 ? m_stride : 0;
     const int64_t threads = g.rows * g.per_row;
     const unsigned blocks = static_cast<unsigned>(lm_blocks(threads));
@@ -299,9 +310,10 @@ TQ_API tq_status tq_dequant_lm2(const uint8_t* packed, const float* codebook, co
     TQ_REQUIRE(packed && codebook && scales && out, "tq_dequant_lm2: null pointer");
     TQ_REQUIRE(n_mat >= 1 && O >= 1 && I >= 1, "tq_dequant_lm2: empty shape");
     TQ_REQUIRE(aligned16(packed), "tq_dequant_lm2: packed not 16-byte aligned");
+    TQ_REQUIRE(n_mat * O * 4 * ((I + 31) / 32) < (int64_t(1) << 32), "tq_dequant_lm2: more than 2^32 octets");
     if (elem_bytes(out_dtype) == 0) return set_error(TQ_ERR_UNSUPPORTED, "tq_dequant_lm2: out dtype %d", out_dtype);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const LmGeom g = lm_geom(n_mat * O, I);
+    const LmGeom g = lm_geom(n_mat * O, O, I);
     const unsigned blocks = static_cast<unsigned>(lm_blocks(g.rows * g.per_row));
     if (out_dtype == TQ_BF16)
         k_lm_dequant<__nv_bfloat16><<<blocks, LM_THREADS, 0, st>>>(packed, scales, codebook, g, static_cast<__nv_bfloat16*>(out));
