@@ -17,8 +17,9 @@
 //    broadcast; 4 consecutive elements per shared-memory load).  The code
 //    comes from the hardware E4M3 conversion of the two products
 //    w inv (1 -+ 2^-20), which bracket the IEEE quotient (E4M3 rounding is
-//    monotone), and from an IEEE division where the two disagree; codes are
-//    decoded in pairs; w - What is exact in fp32 for ratios >= 0.5 and the
+//    monotone), and from an IEEE division where the two disagree; elements
+//    go in pairs through packed fp32x2 products, one conversion per bracket
+//    end and one decode; w - What is exact in fp32 for ratios >= 0.5 and the
 //    weighted square is accumulated in fp64.  Blocks write per-candidate
 //    partial sums; k_fp8_pick adds them in block order (deterministic) and
 //    takes the lowest candidate of the minimum.
@@ -97,14 +98,21 @@ struct F8Args {
     int64_t bpm;         // blocks per matrix
 };
 
-// E4M3 code of fl32(w / s) in the loss loop: the sign of a zero result is
-// kept (it does not change the error), the IEEE division only where the
-// bracket ends disagree.
-__device__ __forceinline__ unsigned fp8_code_raw(float w, const Fp8Scale& sc) {
-    const unsigned two = e4m3x2_from_f32(__fmul_rn(w, sc.ilo), __fmul_rn(w, sc.ihi));
-    if (sc.fast && (two & 0xffu) == (two >> 8)) return two & 0xffu;
+// E4M3 codes of fl32(w0 / s), fl32(w1 / s) as a pair (w0's in the low
+// byte), for the loss loop: one packed multiply per bracket end, one
+// conversion per end for both elements; an IEEE division only for an element
+// whose two ends disagree.  The sign of a zero result is kept (it does not
+// change the error).
+__device__ __forceinline__ unsigned fp8_code_pair(float w0, float w1, const Fp8Scale& sc) {
+    const float2 ww = make_float2(w0, w1);
+    const float2 lo = __fmul2_rn(ww, make_float2(sc.ilo, sc.ilo)), hi = __fmul2_rn(ww, make_float2(sc.ihi, sc.ihi));
+    const unsigned clo = e4m3x2_from_f32(lo.x, lo.y), chi = e4m3x2_from_f32(hi.x, hi.y);
+    if (sc.fast && clo == chi) return clo;
     if (sc.s == 0.f) return 0u;
-    return e4m3x2_from_f32(__fdiv_rn(w, sc.s), 0.f) & 0xffu;
+    unsigned c = clo;
+    if (!sc.fast || ((clo ^ chi) & 0xffu)) c = (c & 0xff00u) | (e4m3x2_from_f32(__fdiv_rn(w0, sc.s), 0.f) & 0xffu);
+    if (!sc.fast || ((clo ^ chi) & 0xff00u)) c = (c & 0xffu) | ((e4m3x2_from_f32(__fdiv_rn(w1, sc.s), 0.f) & 0xffu) << 8);
+    return c;
 }
 
 // EXACT_F32: every candidate ratio is >= 0.5, so |w / s| <= 896 and w - What
@@ -130,15 +138,20 @@ k_fp8_loss(const __grid_constant__ F8Args a) {
         for (int64_t c0 = 0; c0 < n_el; c0 += F8_CHUNK) {
             const int nc = static_cast<int>(min(static_cast<int64_t>(F8_CHUNK), n_el - c0));
             __syncthreads();
+            // element c0 + i of the block's rows: one division per chunk, then
+            // the column steps on by the thread stride (wrapping into the next row)
+            int64_t rq = (c0 + threadIdx.x) / a.I;
+            int64_t jq = c0 + threadIdx.x - rq * a.I;
             for (int i = threadIdx.x; i < F8_CHUNK; i += F8_THREADS) {   // zeros past the chunk's end
                 float w = 0.f, mm = 0.f;
                 if (i < nc) {
-                    const int64_t q = c0 + i, r = r0 + q / a.I, j = q - (q / a.I) * a.I;
-                    w = Elem<T>::load(W + r * a.ld + j);
-                    mm = __ldg(m + j);
+                    w = Elem<T>::load(W + (r0 + rq) * a.ld + jq);
+                    mm = __ldg(m + jq);
                 }
                 sw[i] = w;
                 smv[i] = static_cast<double>(mm);
+                jq += F8_THREADS;
+                while (jq >= a.I) { jq -= a.I; ++rq; }
             }
             __syncthreads();
             if (active) {
@@ -149,18 +162,22 @@ k_fp8_loss(const __grid_constant__ F8Args a) {
                     const double2 ma = sm2[2 * i4], mb = sm2[2 * i4 + 1];
                     const float w[4] = {w4.x, w4.y, w4.z, w4.w};
                     const double mv[4] = {ma.x, ma.y, mb.x, mb.y};
-                    unsigned c[4];
+                    const float2 s2 = make_float2(sc.s, sc.s);
 #pragma unroll
-                    for (int t = 0; t < 4; ++t) c[t] = fp8_code_raw(w[t], sc);
-                    const float2 v01 = f8x2_to_f32(c[0] | (c[1] << 8)), v23 = f8x2_to_f32(c[2] | (c[3] << 8));
-                    const float v[4] = {v01.x, v01.y, v23.x, v23.y};
-#pragma unroll
-                    for (int t = 0; t < 4; ++t) {
-                        const float wh = __fmul_rn(sc.s, v[t]);
-                        double d;
-                        if constexpr (EXACT_F32) d = static_cast<double>(__fsub_rn(w[t], wh));
-                        else d = __dsub_rn(static_cast<double>(w[t]), static_cast<double>(wh));
-                        acc = __fma_rn(mv[t], __dmul_rn(d, d), acc);   // padding: m = 0
+                    for (int h = 0; h < 2; ++h) {   // elements 2h, 2h + 1 as a pair
+                        const float2 ww = make_float2(w[2 * h], w[2 * h + 1]);
+                        const float2 wh = __fmul2_rn(s2, f8x2_to_f32(fp8_code_pair(ww.x, ww.y, sc)));
+                        double d0, d1;
+                        if constexpr (EXACT_F32) {
+                            const float2 d = __fadd2_rn(ww, make_float2(-wh.x, -wh.y));
+                            d0 = static_cast<double>(d.x);
+                            d1 = static_cast<double>(d.y);
+                        } else {
+                            d0 = __dsub_rn(static_cast<double>(ww.x), static_cast<double>(wh.x));
+                            d1 = __dsub_rn(static_cast<double>(ww.y), static_cast<double>(wh.y));
+                        }
+                        acc = __fma_rn(mv[2 * h], __dmul_rn(d0, d0), acc);   // padding: m = 0
+                        acc = __fma_rn(mv[2 * h + 1], __dmul_rn(d1, d1), acc);
                     }
                 }
             }
