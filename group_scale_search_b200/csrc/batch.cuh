@@ -6,7 +6,7 @@
 // Every unit gets a range of the launch's 1-D block index: its column tiles
 // (cblocks, each `cw` unit columns wide, cw <= blockDim.x) times its row
 // blocks (rblocks of rpb rows).  The resident blocks of one wave are split
-// over the units in proportion to their rows x column tiles.
+// over the units so that the longest block, in rows, is as short as it can be.
 #pragma once
 #include "walk.cuh"
 
@@ -24,7 +24,9 @@ struct BatchSlot {
 
 // `cols[i]` unit columns and `rows[i]` rows (all matrices' rows, flattened)
 // of unit i; `slots` = blocks of one wave.  Returns the block count and the
-// widest tile (the launch's blockDim.x, a multiple of 32).
+// widest tile (the launch's blockDim.x, a multiple of 32).  Every unit gets at
+// least one row block per column tile; the count is at most `slots` when
+// that leaves room for it.
 inline int64_t batch_split(int n, const int64_t* cols, const int64_t* rows, int64_t slots, BatchSlot* out,
                            int64_t* width) {
     // Tiles of at most `best` columns, balanced within each unit; the block
@@ -56,19 +58,31 @@ inline int64_t batch_split(int n, const int64_t* cols, const int64_t* rows, int6
         for (int t = 0; t < 8; ++t)
             if (frac[t] <= lo + 0.03) { best = 256 - 32 * t; break; }
     }
-    int64_t total = 0;
     *width = 32;
     for (int i = 0; i < n; ++i) {
         tile(best, i, &out[i].cblocks, &out[i].cw);
         *width = out[i].cw > *width ? out[i].cw : *width;
-        total += rows[i] * out[i].cblocks;
+    }
+    // Rows per block: the fewest R such that every unit's blocks, cblocks x
+    // ceil(rows / R), fit in the wave (all units' blocks run at once, so the
+    // longest block sets the launch's time); without room for one row block
+    // per column tile, one row block per unit.
+    int64_t rmax = 1;
+    for (int i = 0; i < n; ++i) rmax = rows[i] > rmax ? rows[i] : rmax;
+    auto blocks_at = [&](int64_t R) {
+        int64_t t = 0;
+        for (int i = 0; i < n; ++i) t += out[i].cblocks * ((rows[i] + R - 1) / R);
+        return t;
+    };
+    int64_t R = 1, rhi = rmax;   // blocks_at(rmax) is the fewest possible
+    while (R < rhi) {
+        const int64_t mid = R + (rhi - R) / 2;
+        if (blocks_at(mid) <= slots) rhi = mid;
+        else R = mid + 1;
     }
     int64_t b = 0;
     for (int i = 0; i < n; ++i) {
-        // the unit's share of the wave, in row blocks (at least one)
-        const double share = static_cast<double>(slots) * static_cast<double>(rows[i]) / static_cast<double>(total);
-        int64_t rb = static_cast<int64_t>(share);
-        rb = rb < 1 ? 1 : (rb > rows[i] ? rows[i] : rb);
+        const int64_t rb = (rows[i] + R - 1) / R;   // the unit's row blocks, balanced within it
         out[i].rpb = (rows[i] + rb - 1) / rb;
         out[i].rblocks = (rows[i] + out[i].rpb - 1) / out[i].rpb;
         out[i].block0 = b;

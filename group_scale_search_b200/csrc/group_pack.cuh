@@ -99,20 +99,24 @@ __device__ __forceinline__ void nvfp4_rtn(const float w[N], float S, uint32_t m[
         }
         uint32_t x = e2m1x8_from_f32(yl[0], yl[1], yl[2], yl[3], yl[4], yl[5], yl[6], yl[7]);
         const uint32_t d = x ^ e2m1x8_from_f32(yh[0], yh[1], yh[2], yh[3], yh[4], yh[5], yh[6], yh[7]);
-        // Elements whose bracket ends disagree take an IEEE division, one at a
-        // time: the element is picked with a chain of selects (no per-element
-        // branch, no indexed registers).
-        uint32_t todo = ((d | (d >> 1) | (d >> 2) | (d >> 3)) & 0x11111111u);
-        while (todo) {
-            const int b = __ffs(todo) - 1;   // bit 4i of element i
-            todo &= todo - 1u;
-            float wi = w[8 * h];
+        if (d) {
+            // Elements whose bracket ends disagree take an IEEE division, one
+            // at a time: the element is picked with a chain of selects (no
+            // per-element branch, no indexed registers).
+            uint32_t todo = ((d | (d >> 1) | (d >> 2) | (d >> 3)) & 0x11111111u);
+            while (todo) {
+                const int b = __ffs(todo) - 1;   // bit 4i of element i
+                todo &= todo - 1u;
+                float wi = w[8 * h];
 #pragma unroll
-            for (int i = 1; i < 8; ++i) wi = b == 4 * i ? w[8 * h + i] : wi;
-            x = (x & ~(15u << b)) | (nvfp4_code_exact(wi, S) << b);
+                for (int i = 1; i < 8; ++i) wi = b == 4 * i ? w[8 * h + i] : wi;
+                x = (x & ~(15u << b)) | (nvfp4_code_exact(wi, S) << b);
+            }
         }
-        const uint32_t nz = (x | (x >> 1) | (x >> 2)) & 0x11111111u;   // magnitude != 0, per nibble
-        m[h] = x & (0x77777777u | (nz << 3));
+        // a -0 (sign with magnitude 0) becomes +0: magnitude + 7 carries into
+        // bit 3 of its nibble exactly when the magnitude is not 0
+        const uint32_t mag = x & 0x77777777u;
+        m[h] = mag | (x & (mag + 0x77777777u) & 0x88888888u);
     }
 }
 

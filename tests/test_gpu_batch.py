@@ -106,3 +106,40 @@ def test_batch_argument_errors():
         tq.tq_pack_batch([W, W.float()], tq.INT3_G64_SYM, [s, s])
     with pytest.raises(tq.TQError):   # int4 without zero-points
         tq.tq_pack_batch([W], tq.INT4_G128_ASYM, [s])
+
+
+def _strided_units(seed):
+    """bf16 units with padded row and matrix strides: a ragged last column
+    tile, a last group shorter than the group, and a matrix batch with many
+    rows per block whose row ranges cross matrices."""
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    shapes = [(8, 1000, 512), (1, 37, 200), (2, 300, 4160), (1, 64, 2688), (3, 5, 1032)]
+    Ws, ms = [], []
+    for k, (E, O, I) in enumerate(shapes):
+        ld = I + (8 if k % 2 == 0 else 0)
+        mstride = O * ld + (64 if k % 2 == 0 else 0)
+        buf = (synth.student_t((E * mstride,), 4, g, DEV) * 0.02).to(torch.bfloat16)
+        Ws.append(buf.as_strided((E, O, I), (mstride, ld, 1)))
+        ms.append(synth.random_imatrix(I, 50 + k, DEV))
+    return Ws, ms
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_strided_pack_matches_oracle(fmt):
+    """tq_pack and tq_pack_batch on strided units, bit-exact against the
+    oracle's RTN and record layout, and equal to the search's fused pack."""
+    Ws, ms = _strided_units(211 + fmt)
+    res = [tq.tq_search_groups(W, m, fmt, want_idx=False, want_loss=False) for W, m in zip(Ws, ms)]
+    zeros = [r.zeros for r in res] if res[0].zeros is not None else None
+    gsc = [r.global_scale for r in res] if res[0].global_scale is not None else None
+    packed = tq.tq_pack_batch(Ws, fmt, [r.scales for r in res], zeros, gsc)
+    single = [tq.tq_pack(W, fmt, r.scales, r.zeros, r.global_scale) for W, r in zip(Ws, res)]
+    torch.cuda.synchronize()
+    for i, (W, r) in enumerate(zip(Ws, res)):
+        z = r.zeros.cpu().numpy() if r.zeros is not None else None
+        gl = r.global_scale.cpu().numpy() if r.global_scale is not None else None
+        packed_ref, _ = oracle_packed(fmt, host32(W), r.scales.cpu().numpy(), z, gl)
+        label = f"unit {i} {tuple(W.shape)} strides {W.stride()}"
+        assert np.array_equal(packed[i].cpu().numpy(), packed_ref), f"{label}: batched pack differs"
+        assert np.array_equal(single[i].cpu().numpy(), packed_ref), f"{label}: pack differs"
+        assert torch.equal(r.packed, single[i]), f"{label}: fused pack differs from tq_pack"
