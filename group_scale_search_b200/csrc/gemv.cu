@@ -527,6 +527,10 @@ TQ_API tq_status tq_dequant_gemv(const uint8_t* packed, int32_t fmt, const void*
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     const int64_t xms = n_mat > 1 ? x_mat_stride : 0;
     const bool xb = x_dtype == TQ_BF16;
+    if (gemv_mma_ok(fmt, I, B, xms, xb)) {   // several bf16 vectors: the tensor-core form (gemv_mma.cu)
+        launch_gemv_mma(fmt, packed, scales, zeros, global_scale, n_mat, O, I, x, B, xms, y, st);
+        return check_launch("tq_dequant_gemv");
+    }
     if (fmt == TQ_INT3_G64_SYM) {
         launch_gemv_b<TQ_INT3_G64_SYM, true>(B, packed, scales, zeros, global_scale, n_mat, O, I, x, xb, xms, y, st);
     } else if (fmt == TQ_INT4_G128_ASYM) {

@@ -52,6 +52,13 @@ __host__ __device__ constexpr bool is_int4(int fmt) {
     return fmt == TQ_INT4_G128_ASYM || fmt == TQ_INT4_G64_ASYM || fmt == TQ_INT4_G32_ASYM;
 }
 
+// The tensor-core form of tq_dequant_gemv (bf16 x, 2 <= B <= 8, I and the
+// x matrix stride multiples of 8) and its launch.
+bool gemv_mma_ok(int32_t fmt, int64_t I, int64_t B, int64_t x_ms, bool x_bf16);
+void launch_gemv_mma(int32_t fmt, const uint8_t* packed, const void* scales, const uint8_t* zeros, const float* gs,
+                     int64_t n_mat, int64_t O, int64_t I, const void* x, int64_t B, int64_t x_ms, float* y,
+                     cudaStream_t st);
+
 // Try-wait rounds of the tensor-core pipelines' ring waits for the next
 // launch (tq_debug_set_wait_limit; default 2^22).
 unsigned pipeline_wait_limit();

@@ -274,11 +274,17 @@ tq_status tq_dequant_batch(int32_t n, const uint8_t* const* packed, int32_t fmt,
  * What the dequantized weights as tq_dequant defines them.  Computed as
  * sum over groups (NVFP4: blocks) of s * sum_j d_j x_j in fp32 (d = v,
  * q - z or dec(c); s = the group scale or fl32(g dec(e))), in an order fixed
- * by the shape alone: for each column tile (the columns whose x fits the
- * kernel's shared memory at once), per lane over its 32-weight quads, a butterfly over 32 lanes, then (rows
+ * by the shape alone.  bf16 x with B >= 2, I and x_mat_stride multiples of 8:
+ * each group's sum on the tensor cores (bf16 MMA, every product d_j x_j
+ * exact, fp32 accumulation per group), scaled once per group in group order
+ * by each of 4 warps (groups w, w + 4, ...), the warps' sums added in order;
+ * |y - sum What x| <= (g/4 + ceil(G/4) + 4) u sum |What x| (g = group size,
+ * G = groups per row, u = 2^-24).  Otherwise on the CUDA cores: for each
+ * column tile (the columns whose x fits the kernel's shared memory at once),
+ * per lane over its 32-weight quads, a butterfly over 32 lanes, then (rows
  * split over up to 8 warps) the warps' sums in order; the tiles' sums are
- * added in tile order.  Deterministic; |y - sum What x| <=
- * (4 ceil(I/1024) + 30) u sum |What x| (u = 2^-24), plus underflow.
+ * added in tile order; |y - sum What x| <= (4 ceil(I/1024) + 30) u
+ * sum |What x|.  Both deterministic, plus underflow.
  * packed / scales / zeros / global_scale: as tq_dequant; packed 16-byte
  * aligned.  x: x_dtype (TQ_F32 / TQ_BF16) dense [n_mat][B][I] with
  * x_mat_stride elements between matrices (0: one x shared by all

@@ -406,7 +406,14 @@ def _gemv_check(fmt, case, E, O, I, x, label):
     Wd = case["What"].astype(np.float64)
     ref = np.einsum("eoi,ebi->ebo", Wd, xh)
     mag = np.einsum("eoi,ebi->ebo", np.abs(Wd), np.abs(xh))
-    depth = 4 * -(-I // 1024) + 30
+    B = xh.shape[1]
+    xms = (B * I) if x.dim() == 3 and E > 1 else 0
+    if x.dtype == torch.bfloat16 and B >= 2 and I % 8 == 0 and xms % 8 == 0:   # tensor-core form
+        g = {tq.INT3_G64_SYM: 64, tq.INT4_G128_ASYM: 128, tq.INT4_G64_ASYM: 64, tq.INT4_G32_ASYM: 32,
+             tq.NVFP4_G16: 16}[fmt]
+        depth = g / 4 + -(-(-(-I // g)) // 4) + 4
+    else:
+        depth = 4 * -(-I // 1024) + 30
     tol = 1.01 * depth * 2.0 ** -24 * mag + 2.0 ** -126 * I
     got = y.cpu().numpy().astype(np.float64)
     assert got.shape == ref.shape, label
