@@ -102,6 +102,14 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
 // Shared-memory matrix descriptor: MN-major operand, 128-byte swizzle, 64
 // elements (128 B) per row along M/N, rows = tokens.  LBO = bytes between
 // consecutive 64-column boxes, SBO = bytes between groups of 8 token rows.
+// A box of the 3-D map from shared memory to global memory (bulk group).
+__device__ __forceinline__ void hs_tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
     constexpr uint64_t lbo = HS_BOX_BYTES >> 4, sbo = (8 * 128) >> 4;
     return (static_cast<uint64_t>((addr >> 4) & 0x3fffu)) | (lbo << 16) | (sbo << 32) | (1ull << 46) |
@@ -148,13 +156,15 @@ struct HsArgs {
     float* H;
     float alpha;
     int accumulate;
+    int h_tma;                // H leaves by TMA stores where a quarter is wholly above the diagonal
     int nbm, nbn;             // 128-row and 256-column blocks
     int nsb;                  // super-blocks per side
     unsigned wait_limit;      // try_wait rounds of the ring waits
 };
 
 __global__ void __launch_bounds__(HS_THREADS, 1)
-k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsArgs a) {
+k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap hmap,
+          const __grid_constant__ HsArgs a) {
     // the tile: super-block pair (BI <= BJ), then a 128 x 256 tile inside it
     int p = static_cast<int>(blockIdx.x) / (HS_SUPER_M * HS_SUPER_N);
     const int local = static_cast<int>(blockIdx.x) % (HS_SUPER_M * HS_SUPER_N);
@@ -237,54 +247,99 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ HsAr
     }
 
     // epilogue.  One thread waits for the MMAs; the others wait at the block
-    // barrier (no spinning).  The accumulator goes through shared memory (the
-    // ring is free once every MMA is complete), 128 columns at a time, so that
-    // the tile's upper-triangle entries and their mirror images are stored
-    // with coalesced rows; entries below the diagonal are left to their mirror.
+    // barrier (no spinning).  The accumulator leaves through shared memory
+    // (the ring is free once every MMA is complete), 64 columns at a time.
+    // A quarter wholly above the diagonal is written, with its mirror image,
+    // by TMA stores: the rows as 32-column chunks of 128 rows x 128 B in the
+    // 128-byte swizzled layout (thread r writes 16-byte unit u of its row at
+    // u ^ (r % 8)), the mirror as 32-row chunks of the transposed quarter
+    // (64 rows of 128 B; a warp writes one 128-byte row per column).  A
+    // quarter that crosses the diagonal stores its upper-triangle entries and
+    // their mirror images from a padded tile with coalesced rows; entries
+    // below the diagonal are left to their mirror, so H is exactly symmetric.
     if (warp == 1 && lane == 0) progress[3] = mbar_wait(done, 0) ? 1 : 0;
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
     const bool ok = progress[3] != 0 && progress[2] != 0;
-    constexpr int LDT = 128 + 1;   // padded rows: row and column walks are conflict-free
-    float* tile = reinterpret_cast<float*>(smem);
     float* He = a.H + static_cast<int64_t>(e) * a.hms;
     const int64_t r0 = static_cast<int64_t>(bi) * HS_M;
+    const int rr = warp * 32 + lane;   // this thread's accumulator row
+    bool stored = false;               // TMA stores issued (thread 0)
 #pragma unroll 1
-    for (int h = 0; h < HS_N / 128; ++h) {
-        const int m = warp * 32 + lane;
-#pragma unroll 1
-        for (int cc = 0; cc < 128; cc += 32) {
-            float v[32];
-            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(128 * h + cc), v);
+    for (int qh = 0; qh < HS_N / 64; ++qh) {
+        const int64_t ca = static_cast<int64_t>(bj) * HS_N + 64 * qh;   // the quarter's first column
+        if (!ok || ca >= a.I || ca + 63 < r0) continue;                  // past the edge or below the diagonal
+        float v[2][32];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) tile[m * LDT + cc + i] = a.alpha != 1.0f ? __fmul_rn(a.alpha, v[i]) : v[i];
+        for (int h = 0; h < 2; ++h) {
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(64 * qh + 32 * h), v[h]);
+            if (a.alpha != 1.0f) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[h][i] = __fmul_rn(a.alpha, v[h][i]);
+            }
         }
-        __syncthreads();
-        const int64_t c0 = static_cast<int64_t>(bj) * HS_N + 128 * h;
-        if (ok && c0 + 127 >= r0) {
+        if (a.h_tma && ca >= r0 + HS_M) {   // wholly above the diagonal
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                float4* row = reinterpret_cast<float4*>(smem + h * (HS_M * 128) + rr * 128);
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    row[u ^ (rr & 7)] = make_float4(v[h][4 * u], v[h][4 * u + 1], v[h][4 * u + 2], v[h][4 * u + 3]);
+            }
+            uint8_t* mch = smem + 2 * (HS_M * 128) + warp * (64 * 128);   // mirror chunk of rows 32 warp ..
+#pragma unroll
+            for (int c = 0; c < 64; ++c)
+                *reinterpret_cast<float*>(mch + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + ((lane & 3) << 2)) =
+                    v[c >> 5][c & 31];
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            if (threadIdx.x == 0) {
+#pragma unroll 1
+                for (int h = 0; h < 2; ++h)
+                    for (int half = 0; half < 2; ++half)
+                        if (ca + 32 * h < a.I && r0 + 64 * half < a.I)
+                            hs_tma_store_3d(&hmap, s_base + h * (HS_M * 128) + half * (64 * 128),
+                                            static_cast<int>(ca + 32 * h), static_cast<int>(r0 + 64 * half), e);
+#pragma unroll 1
+                for (int k = 0; k < HS_M / 32; ++k)
+                    if (r0 + 32 * k < a.I)
+                        hs_tma_store_3d(&hmap, s_base + 2 * (HS_M * 128) + k * (64 * 128), static_cast<int>(r0 + 32 * k),
+                                        static_cast<int>(ca), e);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the chunks may be rewritten
+                stored = true;
+            }
+            __syncthreads();
+        } else {
+            constexpr int LDT = 64 + 1;   // padded rows: row and column walks are conflict-free
+            float* tile = reinterpret_cast<float*>(smem);
+#pragma unroll
+            for (int i = 0; i < 64; ++i) tile[rr * LDT + i] = v[i >> 5][i & 31];
+            __syncthreads();
 #pragma unroll 4
-            for (int idx = threadIdx.x; idx < 128 * 128; idx += HS_THREADS) {   // H[r0 + r][c0 + c]
-                const int r = idx >> 7, c = idx & 127;
-                const int64_t gr = r0 + r, gc = c0 + c;
+            for (int idx = threadIdx.x; idx < HS_M * 64; idx += HS_THREADS) {   // H[r0 + r][ca + c]
+                const int r = idx >> 6, c = idx & 63;
+                const int64_t gr = r0 + r, gc = ca + c;
                 if (gr < a.I && gc < a.I && gc >= gr) {
                     float* q = He + gr * a.ldh + gc;
-                    const float v = tile[r * LDT + c];
-                    *q = a.accumulate ? __fadd_rn(*q, v) : v;
+                    const float x = tile[r * LDT + c];
+                    *q = a.accumulate ? __fadd_rn(*q, x) : x;
                 }
             }
 #pragma unroll 4
-            for (int idx = threadIdx.x; idx < 128 * 128; idx += HS_THREADS) {   // mirror: H[c0 + c][r0 + r]
+            for (int idx = threadIdx.x; idx < HS_M * 64; idx += HS_THREADS) {   // mirror: H[ca + c][r0 + r]
                 const int c = idx >> 7, r = idx & 127;
-                const int64_t gr = r0 + r, gc = c0 + c;
+                const int64_t gr = r0 + r, gc = ca + c;
                 if (gr < a.I && gc < a.I && gc > gr) {
                     float* q = He + gc * a.ldh + gr;
-                    const float v = tile[r * LDT + c];
-                    *q = a.accumulate ? __fadd_rn(*q, v) : v;
+                    const float x = tile[r * LDT + c];
+                    *q = a.accumulate ? __fadd_rn(*q, x) : x;
                 }
             }
+            __syncthreads();
         }
-        __syncthreads();
     }
+    if (stored) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");   // the stores are complete
 
     // teardown: drain copies armed but not consumed and (if the epilogue's
     // wait gave up) the committed MMAs, then free TMEM
@@ -363,6 +418,22 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
     HsArgs a;
     a.T = X->rows; a.I = X->cols; a.ldh = ldh; a.hms = X->n_mat > 1 ? h_mat_stride : 0;
     a.H = H; a.alpha = alpha; a.accumulate = accumulate ? 1 : 0;
+    // H by TMA stores: written (not accumulated), 16-byte aligned rows and matrices
+    CUtensorMap hmap;
+    memset(&hmap, 0, sizeof hmap);
+    a.h_tma = !accumulate && aligned16(H) && ldh % 4 == 0 && (X->n_mat == 1 || h_mat_stride % 4 == 0) &&
+              X->cols >= 64;
+    if (a.h_tma) {
+        const cuuint64_t hd[3] = {static_cast<cuuint64_t>(X->cols), static_cast<cuuint64_t>(X->cols),
+                                  static_cast<cuuint64_t>(X->n_mat)};
+        const cuuint64_t hs[2] = {static_cast<cuuint64_t>(ldh * 4),
+                                  static_cast<cuuint64_t>((X->n_mat > 1 ? h_mat_stride : X->cols * ldh) * 4)};
+        const cuuint32_t hbox[3] = {32, 64, 1};
+        CUresult hr = enc(&hmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, H, hd, hs, hbox, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (hr != CUDA_SUCCESS) a.h_tma = 0;
+    }
     a.nbm = static_cast<int>((X->cols + HS_M - 1) / HS_M);
     a.nbn = static_cast<int>((X->cols + HS_N - 1) / HS_N);
     a.nsb = static_cast<int>((X->cols + 1023) / 1024);
@@ -373,6 +444,6 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
     const int64_t gx = pairs * HS_SUPER_M * HS_SUPER_N;
     TQ_REQUIRE(gx < (int64_t(1) << 31), "tq_hessian: I too large");
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(X->n_mat));
-    k_hessian<<<grid, HS_THREADS, HS_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, a);
+    k_hessian<<<grid, HS_THREADS, HS_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, hmap, a);
     return check_launch("tq_hessian");
 }
