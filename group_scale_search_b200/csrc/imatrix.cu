@@ -181,7 +181,7 @@ k_imatrix_partial(const T* __restrict__ X, int64_t Tn, int64_t I, int64_t ld, in
 #pragma unroll
             for (int i = 0; i < VEC; ++i) acc[i] = __fmaf_rn(x[i], x[i], acc[i]);
         }
-    } else {
+    } else if (col < I) {   // the row's last columns (lanes past its end have nothing to add)
         for (; t < t1; t += IM_WARPS) {
 #pragma unroll
             for (int i = 0; i < VEC; ++i) {
