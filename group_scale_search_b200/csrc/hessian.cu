@@ -47,16 +47,28 @@
 namespace tq {
 
 constexpr int HS_M = 128;         // tile rows (A panel: 128 columns of X)
-constexpr int HS_N = 256;         // tile columns (B panel: 256 columns of X)
 constexpr int HS_BK = 32;         // tokens per stage
 constexpr int HS_STAGES = 4;
 constexpr int HS_THREADS = 128;
-constexpr int HS_SUPER_M = 8, HS_SUPER_N = 4;         // a super-block: 1024 x 1024 of H
+constexpr int HS_SUPER_M = 8;                          // a super-block: 1024 x 1024 of H
 constexpr int HS_BOX_BYTES = 64 * HS_BK * 2;           // one TMA box: 64 columns x 32 tokens, bf16
 constexpr int HS_A_BYTES = (HS_M / 64) * HS_BOX_BYTES;
-constexpr int HS_B_BYTES = (HS_N / 64) * HS_BOX_BYTES;
-constexpr int HS_STAGE_BYTES = HS_A_BYTES + HS_B_BYTES;
-constexpr int HS_SMEM_BYTES = HS_STAGES * HS_STAGE_BYTES + 1024 /* alignment */ + 256 /* barriers */;
+
+// Tile columns N (B panel: N columns of X): 256, or 128 where the tiles of
+// the upper triangle fill whole waves better (chosen per shape at launch).
+template <int N>
+struct HsCfg {
+    static_assert(N == 256 || N == 128, "tile width");
+    static constexpr int SUPER_N = 1024 / N;
+    static constexpr int B_BYTES = (N / 64) * HS_BOX_BYTES;
+    static constexpr int STAGE_BYTES = HS_A_BYTES + B_BYTES;
+    static constexpr int SMEM_BYTES = HS_STAGES * STAGE_BYTES + 1024 /* alignment */ + 256 /* barriers */;
+    // Instruction descriptor: kind::f16, fp32 accumulator, bf16 A and B, both
+    // MN-major, M = 128, N.
+    static constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
+                                      (static_cast<uint32_t>(N >> 3) << 17) |
+                                      (static_cast<uint32_t>(HS_M >> 4) << 24);
+};
 constexpr unsigned HS_WAIT_LIMIT = DEFAULT_WAIT_LIMIT;  // try_wait rounds before a wait is declared hung
 
 __device__ unsigned g_hs_timeouts = 0;
@@ -116,16 +128,12 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
            (2ull << 61);
 }
 
-// Instruction descriptor: kind::f16, fp32 accumulator, bf16 A and B, both
-// MN-major, M = 128, N = 256.
-constexpr uint32_t HS_IDESC = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (1u << 16) |
-                              (static_cast<uint32_t>(HS_N >> 3) << 17) | (static_cast<uint32_t>(HS_M >> 4) << 24);
-
-__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                          uint32_t accumulate) {
     asm volatile(
         "{ .reg .pred p; setp.ne.b32 p, %4, 0; "
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(HS_IDESC), "r"(accumulate)
+        "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
         : "memory");
 }
 
@@ -157,24 +165,28 @@ struct HsArgs {
     float alpha;
     int accumulate;
     int h_tma;                // H leaves by TMA stores where a quarter is wholly above the diagonal
-    int nbm, nbn;             // 128-row and 256-column blocks
+    int nbm, nbn;             // 128-row and N-column blocks
     int nsb;                  // super-blocks per side
     unsigned wait_limit;      // try_wait rounds of the ring waits
 };
 
+template <int N>
 __global__ void __launch_bounds__(HS_THREADS, 1)
 k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUtensorMap hmap,
           const __grid_constant__ HsArgs a) {
-    // the tile: super-block pair (BI <= BJ), then a 128 x 256 tile inside it
+    using C = HsCfg<N>;
+    constexpr int HS_N = N, HS_SUPER_N = C::SUPER_N, HS_B_BYTES = C::B_BYTES, HS_STAGE_BYTES = C::STAGE_BYTES;
+    constexpr int R = N / HS_M;   // row tiles per column tile (2 or 1)
+    // the tile: super-block pair (BI <= BJ), then a 128 x N tile inside it
     int p = static_cast<int>(blockIdx.x) / (HS_SUPER_M * HS_SUPER_N);
     const int local = static_cast<int>(blockIdx.x) % (HS_SUPER_M * HS_SUPER_N);
     int BI = 0;
     while (p >= a.nsb - BI) { p -= a.nsb - BI; ++BI; }
     const int BJ = BI + p;
     const int bi = BI * HS_SUPER_M + local / HS_SUPER_N, bj = BJ * HS_SUPER_N + local % HS_SUPER_N;
-    if (bi >= a.nbm || bj >= a.nbn || 2 * bj + 1 < bi) return;   // past the edge or below the diagonal
+    if (bi >= a.nbm || bj >= a.nbn || R * bj + R - 1 < bi) return;   // past the edge or below the diagonal
     const int e = static_cast<int>(blockIdx.y);
-    const bool a_in_b = (bi >> 1) == bj;   // the A panel is half of the B panel: load B only
+    const bool a_in_b = bi / R == bj;   // the A panel is part of the B panel: load B only
 
     extern __shared__ uint8_t hs_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hs_raw) + 1023) & ~uintptr_t(1023));
@@ -198,7 +210,7 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
         progress[3] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 0) {   // the whole warp allocates HS_N TMEM columns (128 lanes x 256 fp32)
+    if (warp == 0) {   // the whole warp allocates N TMEM columns (128 lanes x N fp32)
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"(HS_N));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
@@ -235,10 +247,10 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
             if (!mbar_wait(full0 + 8 * s, (k / HS_STAGES) & 1, a.wait_limit)) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
             const uint32_t sb = s_base + s * HS_STAGE_BYTES + HS_A_BYTES;
-            const uint32_t sa = a_in_b ? sb + (bi & 1) * (HS_M / 64) * HS_BOX_BYTES : s_base + s * HS_STAGE_BYTES;
+            const uint32_t sa = a_in_b ? sb + (bi % R) * (HS_M / 64) * HS_BOX_BYTES : s_base + s * HS_STAGE_BYTES;
 #pragma unroll
             for (int kk = 0; kk < HS_BK / 16; ++kk)   // 16 tokens = 16 rows of 128 B per MMA
-                umma_bf16(tmem, umma_desc(sa + kk * 2048), umma_desc(sb + kk * 2048), (k | kk) != 0);
+                umma_bf16(tmem, umma_desc(sa + kk * 2048), umma_desc(sb + kk * 2048), C::IDESC, (k | kk) != 0);
             umma_commit(empty0 + 8 * s);   // the stage is free once these MMAs have read it
             progress[1] = k + 1;
         }
@@ -269,28 +281,36 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
     for (int qh = 0; qh < HS_N / 64; ++qh) {
         const int64_t ca = static_cast<int64_t>(bj) * HS_N + 64 * qh;   // the quarter's first column
         if (!ok || ca >= a.I || ca + 63 < r0) continue;                  // past the edge or below the diagonal
-        float v[2][32];
-#pragma unroll
+        const bool tma = a.h_tma && ca >= r0 + HS_M;   // wholly above the diagonal
+        constexpr int LDT = 64 + 1;                     // padded tile: row and column walks are conflict-free
+        float* tile = reinterpret_cast<float*>(smem);
+        // the quarter's two 32-column halves, one at a time (32 registers of values)
+#pragma unroll 1
         for (int h = 0; h < 2; ++h) {
-            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(64 * qh + 32 * h), v[h]);
+            float v[32];
+            tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + static_cast<uint32_t>(64 * qh + 32 * h), v);
             if (a.alpha != 1.0f) {
 #pragma unroll
-                for (int i = 0; i < 32; ++i) v[h][i] = __fmul_rn(a.alpha, v[h][i]);
+                for (int i = 0; i < 32; ++i) v[i] = __fmul_rn(a.alpha, v[i]);
             }
-        }
-        if (a.h_tma && ca >= r0 + HS_M) {   // wholly above the diagonal
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
+            if (tma) {
                 float4* row = reinterpret_cast<float4*>(smem + h * (HS_M * 128) + rr * 128);
 #pragma unroll
                 for (int u = 0; u < 8; ++u)
-                    row[u ^ (rr & 7)] = make_float4(v[h][4 * u], v[h][4 * u + 1], v[h][4 * u + 2], v[h][4 * u + 3]);
-            }
-            uint8_t* mch = smem + 2 * (HS_M * 128) + warp * (64 * 128);   // mirror chunk of rows 32 warp ..
+                    row[u ^ (rr & 7)] = make_float4(v[4 * u], v[4 * u + 1], v[4 * u + 2], v[4 * u + 3]);
+                uint8_t* mch = smem + 2 * (HS_M * 128) + warp * (64 * 128);   // mirror chunk of rows 32 warp ..
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-                *reinterpret_cast<float*>(mch + c * 128 + (((lane >> 2) ^ (c & 7)) << 4) + ((lane & 3) << 2)) =
-                    v[c >> 5][c & 31];
+                for (int c = 0; c < 32; ++c) {
+                    const int cc = 32 * h + c;
+                    *reinterpret_cast<float*>(mch + cc * 128 + (((lane >> 2) ^ (cc & 7)) << 4) + ((lane & 3) << 2)) =
+                        v[c];
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) tile[rr * LDT + 32 * h + i] = v[i];
+            }
+        }
+        if (tma) {
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncthreads();
             if (threadIdx.x == 0) {
@@ -311,10 +331,6 @@ k_hessian(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ CUte
             }
             __syncthreads();
         } else {
-            constexpr int LDT = 64 + 1;   // padded rows: row and column walks are conflict-free
-            float* tile = reinterpret_cast<float*>(smem);
-#pragma unroll
-            for (int i = 0; i < 64; ++i) tile[rr * LDT + i] = v[i >> 5][i & 31];
             __syncthreads();
 #pragma unroll 4
             for (int idx = threadIdx.x; idx < HS_M * 64; idx += HS_THREADS) {   // H[r0 + r][ca + c]
@@ -435,15 +451,38 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
         if (hr != CUDA_SUCCESS) a.h_tma = 0;
     }
     a.nbm = static_cast<int>((X->cols + HS_M - 1) / HS_M);
-    a.nbn = static_cast<int>((X->cols + HS_N - 1) / HS_N);
     a.nsb = static_cast<int>((X->cols + 1023) / 1024);
     a.wait_limit = pipeline_wait_limit();
     static std::once_flag attr;
-    std::call_once(attr, [] { cudaFuncSetAttribute(k_hessian, cudaFuncAttributeMaxDynamicSharedMemorySize, HS_SMEM_BYTES); });
+    std::call_once(attr, [] {
+        cudaFuncSetAttribute(k_hessian<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, HsCfg<256>::SMEM_BYTES);
+        cudaFuncSetAttribute(k_hessian<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, HsCfg<128>::SMEM_BYTES);
+    });
+    // The tile width: the SMs' time is about waves x resident tiles per SM x
+    // columns per tile; 128-column tiles where that is less (more, narrower
+    // tiles that fill the last wave better), else 256.
+    auto cost = [&](int n, const void* kern, int smem) {
+        const int64_t nbn = (X->cols + n - 1) / n, r = n / HS_M;
+        int64_t tiles = 0;
+        for (int64_t bi = 0; bi < a.nbm; ++bi) tiles += nbn - min(nbn, bi / r);   // tiles with r bj + r - 1 >= bi
+        int per_sm = 1;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, HS_THREADS, smem) != cudaSuccess ||
+            per_sm < 1)
+            per_sm = 1;
+        const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
+        return ((tiles * X->n_mat + slots - 1) / slots) * per_sm * n;
+    };
+    const bool narrow = cost(128, reinterpret_cast<const void*>(k_hessian<128>), HsCfg<128>::SMEM_BYTES) <
+                        cost(256, reinterpret_cast<const void*>(k_hessian<256>), HsCfg<256>::SMEM_BYTES);
+    const int n = narrow ? 128 : 256;
+    a.nbn = static_cast<int>((X->cols + n - 1) / n);
     const int64_t pairs = static_cast<int64_t>(a.nsb) * (a.nsb + 1) / 2;
-    const int64_t gx = pairs * HS_SUPER_M * HS_SUPER_N;
+    const int64_t gx = pairs * HS_SUPER_M * (1024 / n);
     TQ_REQUIRE(gx < (int64_t(1) << 31), "tq_hessian: I too large");
     dim3 grid(static_cast<unsigned>(gx), static_cast<unsigned>(X->n_mat));
-    k_hessian<<<grid, HS_THREADS, HS_SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, hmap, a);
+    if (narrow)
+        k_hessian<128><<<grid, HS_THREADS, HsCfg<128>::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, hmap, a);
+    else
+        k_hessian<256><<<grid, HS_THREADS, HsCfg<256>::SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(map, hmap, a);
     return check_launch("tq_hessian");
 }
