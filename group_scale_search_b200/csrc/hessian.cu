@@ -461,14 +461,28 @@ TQ_API tq_status tq_hessian(const tq_mat* X, float* H, int64_t ldh, int64_t h_ma
     // The tile width: the SMs' time is about waves x resident tiles per SM x
     // columns per tile; 128-column tiles where that is less (more, narrower
     // tiles that fill the last wave better), else 256.
+    // Resident CTAs per SM, counted from the three limits: shared memory
+    // (with the per-block reserve), registers and TMEM columns (512 per SM).
+    auto resident = [&](int n, const void* kern, int smem) {
+        int dev = 0, smem_sm = 0, reserve = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&reserve, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+        cudaFuncAttributes fa;
+        int by_regs = 1;
+        if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess && fa.numRegs > 0) {
+            const int per_warp = (fa.numRegs * 32 + 255) / 256 * 256;   // allocated per warp in units of 256
+            by_regs = 65536 / (per_warp * (HS_THREADS / 32));
+        }
+        const int by_smem = smem_sm > 0 ? smem_sm / (smem + reserve) : 1;
+        const int by_tmem = 512 / n;
+        return max(1, min(by_smem, min(by_regs, by_tmem)));
+    };
     auto cost = [&](int n, const void* kern, int smem) {
         const int64_t nbn = (X->cols + n - 1) / n, r = n / HS_M;
         int64_t tiles = 0;
         for (int64_t bi = 0; bi < a.nbm; ++bi) tiles += nbn - min(nbn, bi / r);   // tiles with r bj + r - 1 >= bi
-        int per_sm = 1;
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, HS_THREADS, smem) != cudaSuccess ||
-            per_sm < 1)
-            per_sm = 1;
+        const int per_sm = resident(n, kern, smem);
         const int64_t slots = static_cast<int64_t>(num_sms()) * per_sm;
         return ((tiles * X->n_mat + slots - 1) / slots) * per_sm * n;
     };
