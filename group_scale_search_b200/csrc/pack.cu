@@ -191,9 +191,15 @@ __device__ __forceinline__ void pack_rows(const T* __restrict__ W, int64_t O, in
     }
 }
 
+// Resident blocks the one-unit int4 pack is compiled for: 64 registers, so
+// a dense matrix's 256-wide tiles fit four blocks per SM (0.43 -> 0.47 of the
+// HBM peak on 4096 x 4096; the grouped kernel measured slower so bounded and
+// keeps the compiler's choice).  0 leaves the other formats to the compiler.
+template <int FMT> __host__ __device__ constexpr int pk_min_blocks() { return is_int4(FMT) ? 4 : 0; }
+
 // One unit: grid x = column tiles, y = row blocks.
 template <int FMT, typename T, int NO>
-__global__ void __launch_bounds__(256 * pk_py<FMT>())
+__global__ void __launch_bounds__(256 * pk_py<FMT>(), pk_min_blocks<FMT>())
 k_pack(const T* __restrict__ W, int64_t O, int64_t I, int64_t ld, int64_t ms, int64_t n_rows, int64_t rpb,
        const void* scales, const uint8_t* __restrict__ zeros, const float* __restrict__ gs,
        uint8_t* __restrict__ packed) {
